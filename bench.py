@@ -1,0 +1,354 @@
+#!/usr/bin/env python
+"""Benchmark of the Flash-LoRA-Attention hot path on B200.
+
+One step = one decode step of the LLaMA-3.1-8B-shaped layer with three agents
+over an 8192-token shared context (hidden 4096, 32 query / 8 KV heads,
+head_dim 128, LoRA rank 16, alpha 32, bf16 caches, fp32 accumulation):
+  1. lr_cache_append of the new token's row X_t [A_k | A_v];
+  2. lora_attn_decode of every agent's query over the shared base and LR caches.
+value = agent-tokens per second over all ranks (3 per step per rank).
+
+The working set of one step is 34 MB, which fits in the 126 MB L2, so the
+steps rotate over enough independent cache sets (each a full synthetic
+problem) that consecutive steps never find their inputs in L2.
+
+--impl reference times the fp64 CPU oracle on the same workload (rank 0 only).
+Multi-GPU: one process per GPU, each serving its own independent requests
+(weak scaling); the only collective is the timing barrier / max.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Flash-LoRA-Attn decode agent-tokens/s & % HBM peak; prefill TFLOP/s & % TC peak"
+UNIT = "agent-tokens/s"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.2)
+        self.proc.terminate()
+        self.proc.wait(timeout=10)
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]),
+                "reasons": reasons, "samples": len(rows)}
+
+
+def decode_bytes(s) -> int:
+    """Algorithmic HBM bytes of one decode launch: base K and V read once, LR
+    cache read once, every agent's B_k and B_v, the queries and the fp32 outputs."""
+    e = 2  # bf16
+    base = 2 * s.n_seqs * s.n_kv_heads * s.kv_len * s.head_dim * e
+    lr = s.n_seqs * s.kv_len * 2 * s.r * e
+    Bw = 2 * s.n_agents * s.r * s.n_kv_heads * s.head_dim * e
+    q = s.n_seqs * s.n_agents * s.n_q_heads * s.head_dim * e
+    out = s.n_seqs * s.n_agents * s.n_q_heads * s.head_dim * 4
+    return base + lr + Bw + q + out
+
+
+def append_bytes(s, n_tok: int) -> int:
+    return s.n_seqs * (n_tok * s.hidden * 2 + n_tok * 2 * s.r * 2) + s.hidden * 2 * s.r * 2
+
+
+def oracle_step(inp, new, s):
+    """One decode step on the fp64 oracle: append the new LR row, then attend."""
+    from oracle import impl as oracle
+    lr = oracle.lr_cache_append(inp["lr"], new["X"], new["A_kv"], s.kv_len - 1)
+    return oracle.lora_attention(inp["k_base"], inp["v_base"], lr, inp["B_k"], inp["B_v"],
+                                 inp["q"], inp["kv_len"], lora_scale=s.lora_scale,
+                                 softmax_scale=s.softmax_scale, rope_base=s.rope_base,
+                                 mode="decode")
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def time_oracle(s, steps: int, budget_s: float):
+    """Time the oracle's decode step; at most `steps` steps or `budget_s` seconds."""
+    from rank_attention_b200 import workloads as W
+    inp = W.direct_cache_inputs(s)
+    new = W.append_inputs(1, s.hidden, s.r, s.dtype, seed=s.seed + 100, n_seqs=s.n_seqs)
+    times = []
+    t_all = time.perf_counter()
+    for _ in range(max(1, steps)):
+        t0 = time.perf_counter()
+        oracle_step(inp, new, s)
+        times.append(time.perf_counter() - t0)
+        if time.perf_counter() - t_all > budget_s:
+            break
+    per = sum(times) / len(times)
+    return s.n_seqs * s.n_agents / per, len(times), per
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from rank_attention_b200 import workloads as W
+    s = W.LLAMA8B_DECODE_8K
+    # warm-up steps, then the timed steps (a bounded sample: the oracle is slow)
+    time_oracle(s, max(1, min(args.warmup, 1)), 5.0)
+    value, n, per = time_oracle(s, args.steps, 60.0)
+    cores = blas_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": n, "warmup": args.warmup,
+            "ms_per_step": per * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": s.name, "sample": f"{n} full decode steps"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"{n} full decode steps of {s.name} (append + attention)"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from rank_attention_b200 import lora_attn as la
+    from rank_attention_b200 import workloads as W
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    s = W.LLAMA8B_DECODE_8K
+    step_bytes = decode_bytes(s) + append_bytes(s, 1)
+    n_sets = max(2, math.ceil(2 * L2_BYTES / step_bytes))
+    sets, steps_fn = [], []
+    A_kv = W.append_inputs(1, s.hidden, s.r, s.dtype, seed=s.seed + 100)["A_kv"].to(dev)
+    for i in range(n_sets):
+        si = s.replace(seed=s.seed + 1000 * (rank + 1) + i)
+        inp = {k: v.to(dev) for k, v in W.direct_cache_inputs(si, device=dev).items()}
+        x_new = W.append_inputs(1, s.hidden, s.r, s.dtype, seed=si.seed + 7, device=dev)["X"]
+        out = torch.empty(inp["q"].shape, dtype=torch.float32, device=dev)
+        st = la.DecodeStep(inp["k_base"], inp["v_base"], inp["lr"], inp["B_k"], inp["B_v"],
+                           inp["q"], out, inp["kv_len"], lora_scale=s.lora_scale,
+                           rope_base=s.rope_base, max_kv_len=s.kv_len, A_kv=A_kv, x_new=x_new,
+                           pos_new=s.kv_len - 1)
+        sets.append((inp, x_new, out))
+        steps_fn.append(st)
+
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.synchronize()
+    # warm-up (eager), then capture CUDA graphs of whole rotations over the sets
+    with torch.cuda.stream(stream):
+        for k in range(args.warmup):
+            steps_fn[k % n_sets]()
+    torch.cuda.synchronize()
+
+    def capture(fns):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for f in fns:
+                f()
+        return g
+
+    full, rem = divmod(args.steps, n_sets)
+    g_rot = capture(steps_fn) if full else None
+    g_rem = capture(steps_fn[:rem]) if rem else None
+    # decode kernel alone, for the roofline of the dominant kernel
+    reps = max(1, 64 // n_sets)
+    dec_fns = [(lambda st=st: la.lora_attn_decode(st.args, st.workspace)) for st in steps_fn]
+    g_dec = capture(dec_fns * reps)
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        for _ in range(full):
+            g_rot.replay()
+        if g_rem is not None:
+            g_rem.replay()
+        ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(ev0.elapsed_time(ev1))
+    # decode kernel alone
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        d0.record(stream)
+        g_dec.replay()
+        d1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    dec_ms = d0.elapsed_time(d1) / (n_sets * reps)
+
+    agent_tokens = s.n_seqs * s.n_agents * args.steps * world
+    value = agent_tokens / (ms / 1e3)
+
+    # end to end through the public API with host buffers: H2D of the step's
+    # inputs (new hidden row, queries, lengths), the two calls, D2H of outputs
+    h_x = [x.cpu().pin_memory() for (_, x, _) in sets]
+    h_q = [i["q"].cpu().pin_memory() for (i, _, _) in sets]
+    h_len = [i["kv_len"].cpu().pin_memory() for (i, _, _) in sets]
+    h_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for (_, _, o) in sets]
+    h2d = h_x[0].numel() * 2 + h_q[0].numel() * 2 + h_len[0].numel() * 4
+    d2h = h_out[0].numel() * 4
+    e_steps = min(args.steps, 100)
+
+    def e2e_step(k):
+        i = k % n_sets
+        inp, x, out = sets[i]
+        x.copy_(h_x[i], non_blocking=True)
+        inp["q"].copy_(h_q[i], non_blocking=True)
+        inp["kv_len"].copy_(h_len[i], non_blocking=True)
+        steps_fn[i]()
+        h_out[i].copy_(out, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for k in range(3):
+            e2e_step(k)
+    torch.cuda.synchronize()
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for k in range(e_steps):
+            e2e_step(k)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e_ms = max_over_ranks(e0.elapsed_time(e1))
+    e2e_value = s.n_seqs * s.n_agents * e_steps * world / (e_ms / 1e3)
+
+    hbm, peak_kind = peaks()
+    dbytes = decode_bytes(s)
+    achieved = dbytes / (dec_ms / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": s.name, "kv_len": s.kv_len, "agents": s.n_agents, "r": s.r,
+                   "step": "lr_cache_append(1 token) + lora_attn_decode",
+                   "l2": f"inputs larger than L2: {n_sets} rotating cache sets of "
+                         f"{step_bytes / 1e6:.1f} MB ({n_sets * step_bytes / 1e6:.0f} MB > 126 MB)",
+                   "timing": "CUDA graphs of the steps, CUDA events on the launch stream",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"kernel": "lora_attn_decode", "bound": "hbm", "achieved": achieved,
+                     "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                     "peak_kind": f"{peak_kind} copy bandwidth",
+                     "algorithmic_bytes_per_launch": dbytes, "launch_us": dec_ms * 1e3,
+                     "traffic": None},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e_steps},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, n, per = time_oracle(s, 20, 15.0)
+        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": blas_threads(),
+                                "kind": "oracle",
+                                "sample": f"{n} full decode steps of {s.name} on the host"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        del g_rot, g_rem, g_dec
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

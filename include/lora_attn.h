@@ -1,0 +1,174 @@
+/*
+ * lora_attn.h -- C ABI of the Flash-LoRA-Attention library (liblora_attn.so).
+ *
+ * Multi-LoRA agents that share one trajectory keep ONE base KV cache
+ * (K_base = RoPE(X W_k), V_base = X W_v, computed with the pretrained
+ * weights) and ONE low-rank (LR) cache LR = X [A_k | A_v] of width 2r,
+ * because the LoRA down-projection A is shared by every agent (shared-A
+ * multi-LoRA).  Agent a owns only its up-projections B_k^a and B_v^a.
+ *   - Cache decomposition Y = X W_0 + (X A) B: LRAgent summary
+ *     (paperlayer.ai/abs/2602.01053v2), App. A.3; LRAgent explainer
+ *     (gist.science/pt/paper/2602.01053), Metodologia 1.
+ *   - One shared LR cache (BaseLRShared): LRAgent summary §3; explainer,
+ *     Metodologia 2.
+ *   - LR rows computed once when a chunk is first processed (PreLRShared):
+ *     PReCache abstract (ai.info, PReCache paper page) and PReCache blog
+ *     (rit.work).
+ *   - Flash-LoRA-Attention, which streams K/V blocks, keeps the value-side
+ *     LoRA at rank r inside an online softmax and applies B once per query
+ *     block: LRAgent summary App. B; explainer, Metodologia 3.
+ *   - Key-side LoRA rebuilt in head dimension and rotated, since RoPE blocks
+ *     the reordering on the key side: LRAgent summary App. D.1.
+ *
+ * What the attention entry points compute, per sequence, agent a, query head
+ * h and its KV head j = floor(h / g), g = n_q_heads / n_kv_heads:
+ *   K^a_t = K_base[j]_t + RoPE_t( s * LRk_t * B_k^a[:, j*d:(j+1)*d] )
+ *   V^a_t = V_base[j]_t +         s * LRv_t * B_v^a[:, j*d:(j+1)*d]
+ *   out   = softmax( q K^a^T * softmax_scale, causal ) V^a
+ * with s = lora_scale = alpha / r, LRk_t = LR[t, 0:r], LRv_t = LR[t, r:2r].
+ * RoPE pairs element i with i + d/2 and turns the pair by angle
+ * t * rope_base^(-2i/d) at 0-based position t.  Queries arrive already
+ * rotated.  Per-agent K^a / V^a are never written to memory.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  Nothing
+ *     is retained after return.  The library never allocates device memory;
+ *     decode scratch comes from the caller's workspace.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and runs asynchronously; the library does not synchronise.
+ *   - Argument errors are reported synchronously, BEFORE anything is
+ *     launched, and nothing is written.  Launch failures return LA_ERR_CUDA.
+ *   - Strides are in ELEMENTS.  Every base pointer must be 16-byte aligned
+ *     and every stride a multiple of 16 bytes.
+ *   - No C++ exception crosses this interface.
+ */
+#ifndef LORA_ATTN_H_
+#define LORA_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void* la_stream_t; /* a cudaStream_t */
+
+typedef enum {
+  LA_OK = 0,
+  LA_ERR_INVALID_ARG = 1,  /* null pointer, bad shape, stride or alignment */
+  LA_ERR_UNSUPPORTED = 2,  /* valid but not built: head_dim, rank, dtype mix */
+  LA_ERR_CAPACITY = 3,     /* rows would land at or beyond L_max */
+  LA_ERR_WORKSPACE = 4,    /* decode workspace missing or too small */
+  LA_ERR_CUDA = 5,         /* a CUDA call or launch failed */
+  LA_ERR_DEVICE_CHECK = 6  /* a kernel's own bounds check fired (see la_device_check) */
+} la_status;
+
+typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* la_status_string(la_status s);
+
+/*
+ * lr_cache_append -- PreLRShared precompute of the shared LR cache.
+ *
+ * For every sequence q in [0, n_seqs) and chunk row i in [0, n_tokens):
+ *   lr_cache[q][pos0 + i][c] = sum_k X[q][i][k] * A_kv[k][c],  c in [0, 2r)
+ * i.e. the row [X A_k | X A_v]: unscaled (s is applied when rows are read)
+ * and unrotated.  Accumulation is fp32; bf16 outputs are rounded to nearest
+ * even.  Rows outside [pos0, pos0 + n_tokens) are not touched.
+ *
+ *   X        [n_seqs][n_tokens][hidden], row stride ldx, sequence stride
+ *            seq_stride_x (elements).
+ *   A_kv     [hidden][2r] row-major (A_k in columns 0..r-1, A_v in r..2r-1),
+ *            shared by all sequences.
+ *   lr_cache [n_seqs][L_max][2r], row stride 2r, sequence stride
+ *            seq_stride_lr (elements).
+ *   dt       dtype of X, A_kv and lr_cache (all the same).
+ * Errors: LA_ERR_INVALID_ARG (null pointer, non-positive size, misaligned
+ * pointer or stride), LA_ERR_UNSUPPORTED (r not in {8,16,32,64}),
+ * LA_ERR_CAPACITY (pos0 < 0 or pos0 + n_tokens > L_max).
+ */
+la_status lr_cache_append(const void* X, int64_t ldx, int64_t n_tokens, int64_t hidden,
+                          const void* A_kv, int32_t r, void* lr_cache, int64_t L_max,
+                          int64_t pos0, int32_t n_seqs, int64_t seq_stride_x,
+                          int64_t seq_stride_lr, la_dtype dt, la_stream_t stream);
+
+/* Arguments shared by lora_attn_prefill and lora_attn_decode. */
+typedef struct {
+  int32_t n_seqs;       /* independent sequences, each with its own caches */
+  int32_t n_agents;     /* agents sharing each sequence's caches */
+  int32_t n_q_heads;    /* query heads; a multiple of n_kv_heads */
+  int32_t n_kv_heads;
+  int32_t head_dim;     /* d: 64 or 128 */
+  int32_t r;            /* LoRA rank: 8, 16, 32 or 64 */
+  float lora_scale;     /* s = alpha / r */
+  float softmax_scale;  /* usually 1 / sqrt(d) */
+  double rope_base;     /* theta_i = rope_base^(-2i/d) */
+  int64_t L_max;        /* rows allocated per (sequence, KV head) and per sequence in lr_cache */
+  /* Base cache, already rotated: element (q, j, t, c) at
+   * q*kv_seq_stride + j*kv_head_stride + t*kv_tok_stride + c; kv_tok_stride >= d. */
+  const void* k_base;
+  const void* v_base;
+  int64_t kv_seq_stride, kv_head_stride, kv_tok_stride;
+  /* LR cache [n_seqs][L_max][2r]: element (q, t, c) at q*lr_seq_stride + t*2r + c. */
+  const void* lr_cache;
+  int64_t lr_seq_stride;
+  /* Per-agent up-projections [n_agents][r][n_kv_heads*d], contiguous. */
+  const void* B_k;
+  const void* B_v;
+  /* Queries (already rotated) and outputs, contiguous
+   * [n_seqs][n_agents][n_q_tokens][n_q_heads][d]. */
+  const void* q;
+  void* out;
+  /* Decode: device int32 [n_seqs]; sequence q's query sits at position
+   * kv_len[q]-1 and sees keys [0, kv_len[q]).  Ignored by prefill. */
+  const int32_t* kv_len;
+  int64_t max_kv_len;   /* decode: host upper bound on every kv_len[q], <= L_max */
+  /* Prefill: query token j sits at position q_pos0 + j and sees keys
+   * [0, q_pos0 + j]; the chunk's own base and LR rows must already be cached. */
+  int64_t q_pos0;
+  int32_t n_q_tokens;   /* decode: must be 1 */
+  la_dtype io_dtype;    /* dtype of k_base, v_base, lr_cache, B_k, B_v and q */
+  la_dtype out_dtype;   /* dtype of out */
+} la_attn_args;
+
+/*
+ * lora_attn_prefill -- causal Flash-LoRA-Attention for a chunk of n_q_tokens
+ * query tokens per (sequence, agent) over prefix + chunk.
+ * Errors: LA_ERR_INVALID_ARG, LA_ERR_UNSUPPORTED, LA_ERR_CAPACITY
+ * (q_pos0 + n_q_tokens > L_max), LA_ERR_CUDA.
+ */
+la_status lora_attn_prefill(const la_attn_args* args, la_stream_t stream);
+
+/*
+ * lora_attn_decode -- one query token per (sequence, agent), split over the
+ * sequence (split-K) with the partial results merged inside the same launch.
+ *
+ * workspace: device memory of at least lora_attn_decode_workspace_bytes(args)
+ * bytes, 256-byte aligned, ZERO-FILLED BEFORE ITS FIRST USE.  Each call
+ * leaves the arrival counters it used back at zero, so a workspace can be
+ * reused by later calls on the same stream; calls that run concurrently
+ * need separate workspaces.
+ * Errors: as prefill, plus LA_ERR_WORKSPACE.  A kv_len[q] outside
+ * [1, max_kv_len] is caught on the device: that sequence's outputs are left
+ * unwritten and la_device_check() reports LA_ERR_DEVICE_CHECK.
+ */
+la_status lora_attn_decode(const la_attn_args* args, void* workspace, size_t workspace_bytes,
+                           la_stream_t stream);
+
+/* Workspace bytes lora_attn_decode needs for these arguments (0 if invalid). */
+size_t lora_attn_decode_workspace_bytes(const la_attn_args* args);
+
+/*
+ * la_device_check -- synchronises the current device, then reads and clears
+ * the library's device error word.  Returns LA_OK, LA_ERR_DEVICE_CHECK if a
+ * kernel's bounds check fired since the last call, or LA_ERR_CUDA.
+ */
+la_status la_device_check(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LORA_ATTN_H_ */

@@ -1,0 +1,241 @@
+// The C ABI: argument checks, launch planning and dispatch to the kernels.
+// Every check runs before anything is enqueued; on error nothing is written.
+#include <math.h>
+#include <string.h>
+
+#include "la_internal.cuh"
+
+namespace la {
+
+__device__ int g_error_word;
+
+int* error_word_ptr() {
+  static int* cached[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return nullptr;
+  if (dev < 64 && cached[dev]) return cached[dev];
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_error_word) != cudaSuccess) return nullptr;
+  if (dev < 64) cached[dev] = static_cast<int*>(ptr);
+  return static_cast<int*>(ptr);
+}
+
+size_t simt_rows_cap(const AttnParams& p);
+int simt_key_tile();
+bool bf16_decode_supported(const AttnParams& p);
+void bf16_decode_plan(const AttnParams& p, int* n_splits, int64_t* split_len, int* rows);
+cudaError_t launch_decode_bf16(const AttnParams& p, la_dtype out, cudaStream_t st);
+bool bf16_prefill_supported(const AttnParams& p);
+cudaError_t launch_prefill_bf16(const AttnParams& p, la_dtype out, cudaStream_t st);
+bool bf16_append_supported(int64_t H, int r);
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t esize(la_dtype t) { return t == LA_F32 ? 4 : 2; }
+bool dtype_ok(int t) { return t == LA_F32 || t == LA_BF16; }
+bool rank_ok(int r) { return r == 8 || r == 16 || r == 32 || r == 64; }
+bool stride_ok(int64_t s, la_dtype t) { return s > 0 && ((s * (int64_t)esize(t)) % 16) == 0; }
+
+// Checks common to prefill and decode; fills p on success.
+la_status check_attn(const la_attn_args* a, int decode, AttnParams* p) {
+  if (!a) return LA_ERR_INVALID_ARG;
+  if (!dtype_ok(a->io_dtype) || !dtype_ok(a->out_dtype)) return LA_ERR_INVALID_ARG;
+  if (a->n_seqs < 0 || a->n_agents < 1 || a->n_q_heads < 1 || a->n_kv_heads < 1)
+    return LA_ERR_INVALID_ARG;
+  if (a->n_q_heads % a->n_kv_heads != 0) return LA_ERR_INVALID_ARG;
+  if (a->head_dim != 64 && a->head_dim != 128) return LA_ERR_UNSUPPORTED;
+  if (!rank_ok(a->r)) return LA_ERR_UNSUPPORTED;
+  if (!isfinite(a->lora_scale) || !isfinite(a->softmax_scale) || !(a->softmax_scale > 0.f))
+    return LA_ERR_INVALID_ARG;
+  if (!isfinite(a->rope_base) || !(a->rope_base > 1.0)) return LA_ERR_INVALID_ARG;
+  if (a->L_max < 1) return LA_ERR_INVALID_ARG;
+  if (!a->k_base || !a->v_base || !a->lr_cache || !a->B_k || !a->B_v || !a->q || !a->out)
+    return LA_ERR_INVALID_ARG;
+  if (!aligned16(a->k_base) || !aligned16(a->v_base) || !aligned16(a->lr_cache) ||
+      !aligned16(a->B_k) || !aligned16(a->B_v) || !aligned16(a->q) || !aligned16(a->out))
+    return LA_ERR_INVALID_ARG;
+  const la_dtype io = a->io_dtype;
+  if (a->kv_tok_stride < a->head_dim || !stride_ok(a->kv_tok_stride, io) ||
+      !stride_ok(a->kv_head_stride, io) || !stride_ok(a->kv_seq_stride, io))
+    return LA_ERR_INVALID_ARG;
+  if (a->lr_seq_stride < a->L_max * 2 * a->r || !stride_ok(a->lr_seq_stride, io))
+    return LA_ERR_INVALID_ARG;
+  const int g = a->n_q_heads / a->n_kv_heads;
+  if ((int64_t)a->n_agents * g > kMaxRowsSimt) return LA_ERR_UNSUPPORTED;
+  if (decode) {
+    if (a->n_q_tokens != 1) return LA_ERR_INVALID_ARG;
+    if (!a->kv_len) return LA_ERR_INVALID_ARG;
+    if (a->max_kv_len < 1) return LA_ERR_INVALID_ARG;
+    if (a->max_kv_len > a->L_max) return LA_ERR_CAPACITY;
+  } else {
+    if (a->n_q_tokens < 0 || a->q_pos0 < 0) return LA_ERR_INVALID_ARG;
+    if (a->q_pos0 + a->n_q_tokens > a->L_max) return LA_ERR_CAPACITY;
+  }
+  memset(p, 0, sizeof(*p));
+  p->n_seqs = a->n_seqs;
+  p->n_agents = a->n_agents;
+  p->n_q = a->n_q_heads;
+  p->n_kv = a->n_kv_heads;
+  p->d = a->head_dim;
+  p->r = a->r;
+  p->g = g;
+  p->rows_per_tok = a->n_agents * g;
+  p->s = a->lora_scale;
+  p->scale = a->softmax_scale;
+  p->rope_base = a->rope_base;
+  p->L_max = a->L_max;
+  p->k_base = a->k_base;
+  p->v_base = a->v_base;
+  p->kv_seq = a->kv_seq_stride;
+  p->kv_head = a->kv_head_stride;
+  p->kv_tok = a->kv_tok_stride;
+  p->lr = a->lr_cache;
+  p->lr_seq = a->lr_seq_stride;
+  p->B_k = a->B_k;
+  p->B_v = a->B_v;
+  p->q = a->q;
+  p->out = a->out;
+  p->kv_len = a->kv_len;
+  p->max_kv_len = a->max_kv_len;
+  p->q_pos0 = a->q_pos0;
+  p->n_q_tokens = decode ? 1 : a->n_q_tokens;
+  p->decode = decode;
+  return LA_OK;
+}
+
+constexpr int kNumSMs = 148;
+
+DecodePlan plan_decode(const AttnParams& p, la_dtype io) {
+  DecodePlan d;
+  memset(&d, 0, sizeof(d));
+  const int units = p.n_seqs * p.n_kv;
+  if (io == LA_BF16 && bf16_decode_supported(p)) {
+    d.kind = 1;
+    bf16_decode_plan(p, &d.n_splits, &d.split_len, &d.rows);
+  } else {
+    d.kind = 0;
+    const int tk = simt_key_tile();
+    const int64_t max_tiles = (p.max_kv_len + tk - 1) / tk;
+    int64_t want = (2 * kNumSMs + units - 1) / (units > 0 ? units : 1);
+    if (want > max_tiles) want = max_tiles;
+    if (want < 1) want = 1;
+    int64_t tiles_per = (max_tiles + want - 1) / want;
+    d.split_len = tiles_per * tk;
+    d.n_splits = (int)((p.max_kv_len + d.split_len - 1) / d.split_len);
+    d.rows = (int)simt_rows_cap(p);
+  }
+  const size_t W = (size_t)p.d + p.r + 2;
+  d.partial_bytes = d.n_splits > 1 ? (size_t)units * d.n_splits * d.rows * W * sizeof(float) : 0;
+  d.partial_bytes = (d.partial_bytes + 255) / 256 * 256;
+  d.counter_bytes = ((size_t)units * sizeof(int) + 255) / 256 * 256;
+  return d;
+}
+
+}  // namespace
+}  // namespace la
+
+using namespace la;
+
+extern "C" const char* la_status_string(la_status s) {
+  switch (s) {
+    case LA_OK: return "LA_OK";
+    case LA_ERR_INVALID_ARG: return "LA_ERR_INVALID_ARG: invalid argument";
+    case LA_ERR_UNSUPPORTED: return "LA_ERR_UNSUPPORTED: configuration not supported";
+    case LA_ERR_CAPACITY: return "LA_ERR_CAPACITY: rows beyond L_max";
+    case LA_ERR_WORKSPACE: return "LA_ERR_WORKSPACE: workspace missing or too small";
+    case LA_ERR_CUDA: return "LA_ERR_CUDA: CUDA call or launch failed";
+    case LA_ERR_DEVICE_CHECK: return "LA_ERR_DEVICE_CHECK: a kernel bounds check fired";
+  }
+  return "unknown la_status";
+}
+
+extern "C" la_status lr_cache_append(const void* X, int64_t ldx, int64_t n_tokens, int64_t hidden,
+                                     const void* A_kv, int32_t r, void* lr_cache, int64_t L_max,
+                                     int64_t pos0, int32_t n_seqs, int64_t seq_stride_x,
+                                     int64_t seq_stride_lr, la_dtype dt, la_stream_t stream) {
+  if (!dtype_ok(dt)) return LA_ERR_INVALID_ARG;
+  if (n_tokens < 0 || n_seqs < 0 || hidden < 1 || L_max < 1) return LA_ERR_INVALID_ARG;
+  if (!rank_ok(r)) return LA_ERR_UNSUPPORTED;
+  if (pos0 < 0 || pos0 + n_tokens > L_max) return LA_ERR_CAPACITY;
+  if (n_tokens == 0 || n_seqs == 0) return LA_OK;  // nothing is read or written
+  if (!X || !A_kv || !lr_cache) return LA_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(A_kv) || !aligned16(lr_cache)) return LA_ERR_INVALID_ARG;
+  if (ldx < hidden || !stride_ok(ldx, dt)) return LA_ERR_INVALID_ARG;
+  if (n_seqs > 1 && (!stride_ok(seq_stride_x, dt) || !stride_ok(seq_stride_lr, dt)))
+    return LA_ERR_INVALID_ARG;
+  if (n_seqs > 1 && seq_stride_lr < L_max * 2 * r) return LA_ERR_INVALID_ARG;
+  if ((hidden * (int64_t)esize(dt)) % 16 != 0) return LA_ERR_INVALID_ARG;
+  if (n_seqs > 65535) return LA_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (dt == LA_BF16 && bf16_append_supported(hidden, r))
+    e = launch_append_bf16_mma(X, ldx, n_tokens, hidden, A_kv, r, lr_cache, pos0, n_seqs,
+                               seq_stride_x, seq_stride_lr, st);
+  else
+    e = launch_append_simt(X, ldx, n_tokens, hidden, A_kv, r, lr_cache, pos0, n_seqs,
+                           seq_stride_x, seq_stride_lr, dt, st);
+  return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
+extern "C" size_t lora_attn_decode_workspace_bytes(const la_attn_args* a) {
+  AttnParams p;
+  if (check_attn(a, 1, &p) != LA_OK) return 0;
+  DecodePlan d = plan_decode(p, a->io_dtype);
+  return d.partial_bytes + d.counter_bytes;
+}
+
+extern "C" la_status lora_attn_decode(const la_attn_args* a, void* workspace,
+                                      size_t workspace_bytes, la_stream_t stream) {
+  AttnParams p;
+  la_status s = check_attn(a, 1, &p);
+  if (s != LA_OK) return s;
+  DecodePlan d = plan_decode(p, a->io_dtype);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+      workspace_bytes < d.partial_bytes + d.counter_bytes)
+    return LA_ERR_WORKSPACE;
+  if (p.n_seqs == 0) return LA_OK;
+  if ((int64_t)p.n_seqs * p.n_kv > 65535) return LA_ERR_UNSUPPORTED;
+  p.n_splits = d.n_splits;
+  p.split_len = d.split_len;
+  p.partials = static_cast<float*>(workspace);
+  p.counters = reinterpret_cast<int*>(static_cast<char*>(workspace) + d.partial_bytes);
+  p.err = error_word_ptr();
+  if (!p.err) return LA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = d.kind == 1 ? launch_decode_bf16(p, a->out_dtype, st)
+                              : launch_attn_simt(p, a->io_dtype, a->out_dtype, st);
+  return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
+extern "C" la_status lora_attn_prefill(const la_attn_args* a, la_stream_t stream) {
+  AttnParams p;
+  la_status s = check_attn(a, 0, &p);
+  if (s != LA_OK) return s;
+  if (p.n_seqs == 0 || p.n_q_tokens == 0) return LA_OK;
+  if ((int64_t)p.n_seqs * p.n_kv > 65535) return LA_ERR_UNSUPPORTED;
+  p.err = error_word_ptr();
+  if (!p.err) return LA_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (a->io_dtype == LA_BF16 && bf16_prefill_supported(p))
+    e = launch_prefill_bf16(p, a->out_dtype, st);
+  else
+    e = launch_attn_simt(p, a->io_dtype, a->out_dtype, st);
+  return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
+extern "C" la_status la_device_check(void) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return LA_ERR_CUDA;
+  int* ptr = error_word_ptr();
+  if (!ptr) return LA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, ptr, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return LA_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(ptr, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+      return LA_ERR_CUDA;
+    return LA_ERR_DEVICE_CHECK;
+  }
+  return LA_OK;
+}

@@ -1,0 +1,82 @@
+// Internal declarations shared by the library's translation units.
+// Nothing here is part of the public ABI (include/lora_attn.h).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "lora_attn.h"
+
+namespace la {
+
+constexpr int kMaxRowsSimt = 64;   // agents x GQA group rows one generic CTA holds
+
+// Parameters of one attention launch, resolved on the host.
+struct AttnParams {
+  int n_seqs, n_agents, n_q, n_kv, d, r, g;
+  int rows_per_tok;        // n_agents * g
+  float s;                 // lora_scale
+  float scale;             // softmax_scale
+  double rope_base;
+  int64_t L_max;
+  const void* k_base;
+  const void* v_base;
+  int64_t kv_seq, kv_head, kv_tok;
+  const void* lr;
+  int64_t lr_seq;
+  const void* B_k;
+  const void* B_v;
+  const void* q;
+  void* out;
+  const int32_t* kv_len;   // decode only
+  int64_t max_kv_len;
+  int64_t q_pos0;          // prefill only
+  int n_q_tokens;
+  int decode;              // 1 = decode, 0 = prefill
+  // decode split-K
+  int n_splits;
+  int64_t split_len;       // keys per split (multiple of the key tile)
+  float* partials;         // [units][n_splits][rows][d + r + 2]
+  int* counters;           // [units]
+  int* err;                // device error word
+  int out_bf16;            // tensor-core kernels: 1 = bf16 outputs, 0 = fp32
+};
+
+// Device error word of the library (address on the current device).
+int* error_word_ptr();
+
+// Launchers (return cudaError_t of the launch).
+cudaError_t launch_append_simt(const void* X, int64_t ldx, int64_t n, int64_t H, const void* A,
+                               int r, void* lr, int64_t pos0, int n_seqs, int64_t sx,
+                               int64_t slr, la_dtype dt, cudaStream_t st);
+cudaError_t launch_append_bf16_mma(const void* X, int64_t ldx, int64_t n, int64_t H,
+                                   const void* A, int r, void* lr, int64_t pos0, int n_seqs,
+                                   int64_t sx, int64_t slr, cudaStream_t st);
+cudaError_t launch_attn_simt(const AttnParams& p, la_dtype io, la_dtype out, cudaStream_t st);
+
+// Decode split-K plan shared by the workspace query and the launch.
+struct DecodePlan {
+  int kind;                // 0 = generic SIMT kernel, 1 = bf16 tensor-core kernel
+  int n_splits;
+  int64_t split_len;
+  int rows;                // rows per unit
+  size_t partial_bytes;
+  size_t counter_bytes;
+};
+
+// ---------------------------------------------------------------------------
+// small device helpers
+// ---------------------------------------------------------------------------
+template <typename T> __device__ __forceinline__ float to_f32(T v);
+template <> __device__ __forceinline__ float to_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) {
+  return __bfloat162float(v);
+}
+template <typename T> __device__ __forceinline__ T from_f32(float v);
+template <> __device__ __forceinline__ float from_f32<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float v) {
+  return __float2bfloat16_rn(v);
+}
+
+}  // namespace la

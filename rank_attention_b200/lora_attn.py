@@ -1,0 +1,205 @@
+"""Python binding of liblora_attn.so (ctypes; argument marshalling only).
+
+The names match the C ABI in include/lora_attn.h.  Tensors are torch CUDA
+tensors; the binding passes their data pointers, sizes and strides, and the
+current torch stream.  Every step of the computation runs in the library's
+CUDA kernels.  If the compiled library is missing, importing this module
+raises: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "_lib", "liblora_attn.so")
+
+LA_OK, LA_ERR_INVALID_ARG, LA_ERR_UNSUPPORTED, LA_ERR_CAPACITY = 0, 1, 2, 3
+LA_ERR_WORKSPACE, LA_ERR_CUDA, LA_ERR_DEVICE_CHECK = 4, 5, 6
+LA_F32, LA_BF16 = 0, 1
+
+EXPORTED = ("la_status_string", "lr_cache_append", "lora_attn_prefill", "lora_attn_decode",
+            "lora_attn_decode_workspace_bytes", "la_device_check")
+
+
+class LoraAttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+class AttnArgs(ctypes.Structure):
+    """Mirror of la_attn_args."""
+
+    _fields_ = [
+        ("n_seqs", ctypes.c_int32), ("n_agents", ctypes.c_int32),
+        ("n_q_heads", ctypes.c_int32), ("n_kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32), ("r", ctypes.c_int32),
+        ("lora_scale", ctypes.c_float), ("softmax_scale", ctypes.c_float),
+        ("rope_base", ctypes.c_double),
+        ("L_max", ctypes.c_int64),
+        ("k_base", ctypes.c_void_p), ("v_base", ctypes.c_void_p),
+        ("kv_seq_stride", ctypes.c_int64), ("kv_head_stride", ctypes.c_int64),
+        ("kv_tok_stride", ctypes.c_int64),
+        ("lr_cache", ctypes.c_void_p), ("lr_seq_stride", ctypes.c_int64),
+        ("B_k", ctypes.c_void_p), ("B_v", ctypes.c_void_p),
+        ("q", ctypes.c_void_p), ("out", ctypes.c_void_p),
+        ("kv_len", ctypes.c_void_p),
+        ("max_kv_len", ctypes.c_int64),
+        ("q_pos0", ctypes.c_int64),
+        ("n_q_tokens", ctypes.c_int32),
+        ("io_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int),
+    ]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"liblora_attn.so is not built ({LIB_PATH}); run "
+                          "python -m rank_attention_b200.build_lib")
+    lib = ctypes.CDLL(LIB_PATH)
+    lib.la_status_string.restype = ctypes.c_char_p
+    lib.la_status_string.argtypes = [ctypes.c_int]
+    lib.lr_cache_append.restype = ctypes.c_int
+    lib.lr_cache_append.argtypes = [
+        ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+        ctypes.c_int32, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32,
+        ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_void_p]
+    lib.lora_attn_prefill.restype = ctypes.c_int
+    lib.lora_attn_prefill.argtypes = [ctypes.POINTER(AttnArgs), ctypes.c_void_p]
+    lib.lora_attn_decode.restype = ctypes.c_int
+    lib.lora_attn_decode.argtypes = [ctypes.POINTER(AttnArgs), ctypes.c_void_p, ctypes.c_size_t,
+                                     ctypes.c_void_p]
+    lib.lora_attn_decode_workspace_bytes.restype = ctypes.c_size_t
+    lib.lora_attn_decode_workspace_bytes.argtypes = [ctypes.POINTER(AttnArgs)]
+    lib.la_device_check.restype = ctypes.c_int
+    lib.la_device_check.argtypes = []
+    return lib
+
+
+lib = _load()
+
+
+def status_string(status: int) -> str:
+    return lib.la_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != LA_OK:
+        raise LoraAttnError(status, where)
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return LA_F32
+    if t.dtype == torch.bfloat16:
+        return LA_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def lr_cache_append(X: torch.Tensor, A_kv: torch.Tensor, lr_cache: torch.Tensor, pos0: int,
+                    stream=None) -> None:
+    """lr_cache[:, pos0:pos0+n] = X @ A_kv.
+
+    X [n_seqs, n, H] (last dim contiguous), A_kv [H, 2r] contiguous,
+    lr_cache [n_seqs, L_max, 2r] (last two dims contiguous)."""
+    n_seqs, n, H = X.shape
+    r = A_kv.shape[1] // 2
+    assert X.stride(2) == 1 and A_kv.is_contiguous()
+    assert lr_cache.stride(2) == 1 and lr_cache.stride(1) == 2 * r
+    st = lib.lr_cache_append(X.data_ptr(), X.stride(1), n, H, A_kv.data_ptr(), r,
+                             lr_cache.data_ptr(), lr_cache.shape[1], pos0, n_seqs, X.stride(0),
+                             lr_cache.stride(0), _dt(X), _stream(stream))
+    _check(st, "lr_cache_append")
+
+
+def make_args(k_base, v_base, lr, B_k, B_v, q, out, *, lora_scale: float, rope_base: float,
+              softmax_scale: Optional[float] = None, kv_len: Optional[torch.Tensor] = None,
+              max_kv_len: int = 0, q_pos0: int = 0) -> AttnArgs:
+    """Fill la_attn_args from tensors.
+
+    k_base, v_base [n_seqs, n_kv, L_max, d] (any strides with a unit last
+    stride); lr [n_seqs, L_max, 2r]; B_k, B_v [n_agents, r, n_kv*d];
+    q, out [n_seqs, n_agents, n_tok, n_q, d] contiguous; kv_len int32 [n_seqs]."""
+    n_seqs, n_kv, L_max, d = k_base.shape
+    n_agents, n_tok, n_q = q.shape[1], q.shape[2], q.shape[3]
+    r = lr.shape[2] // 2
+    assert k_base.stride() == v_base.stride() and k_base.stride(3) == 1
+    assert lr.stride(2) == 1 and lr.stride(1) == 2 * r
+    assert B_k.is_contiguous() and B_v.is_contiguous() and q.is_contiguous() and out.is_contiguous()
+    a = AttnArgs()
+    a.n_seqs, a.n_agents, a.n_q_heads, a.n_kv_heads = n_seqs, n_agents, n_q, n_kv
+    a.head_dim, a.r = d, r
+    a.lora_scale = lora_scale
+    a.softmax_scale = softmax_scale if softmax_scale is not None else 1.0 / math.sqrt(d)
+    a.rope_base = rope_base
+    a.L_max = L_max
+    a.k_base, a.v_base = k_base.data_ptr(), v_base.data_ptr()
+    a.kv_seq_stride, a.kv_head_stride, a.kv_tok_stride = (k_base.stride(0), k_base.stride(1),
+                                                          k_base.stride(2))
+    a.lr_cache, a.lr_seq_stride = lr.data_ptr(), lr.stride(0)
+    a.B_k, a.B_v = B_k.data_ptr(), B_v.data_ptr()
+    a.q, a.out = q.data_ptr(), out.data_ptr()
+    a.kv_len = kv_len.data_ptr() if kv_len is not None else None
+    a.max_kv_len = max_kv_len
+    a.q_pos0 = q_pos0
+    a.n_q_tokens = n_tok
+    a.io_dtype, a.out_dtype = _dt(k_base), _dt(out)
+    return a
+
+
+def lora_attn_decode_workspace_bytes(args: AttnArgs) -> int:
+    return int(lib.lora_attn_decode_workspace_bytes(ctypes.byref(args)))
+
+
+def decode_workspace(args: AttnArgs, device) -> torch.Tensor:
+    """A zero-filled workspace large enough for these decode arguments."""
+    n = lora_attn_decode_workspace_bytes(args)
+    if n == 0:
+        raise LoraAttnError(LA_ERR_INVALID_ARG, "lora_attn_decode_workspace_bytes")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def lora_attn_decode(args: AttnArgs, workspace: torch.Tensor, stream=None) -> None:
+    st = lib.lora_attn_decode(ctypes.byref(args), workspace.data_ptr(), workspace.numel(),
+                              _stream(stream))
+    _check(st, "lora_attn_decode")
+
+
+def lora_attn_prefill(args: AttnArgs, stream=None) -> None:
+    st = lib.lora_attn_prefill(ctypes.byref(args), _stream(stream))
+    _check(st, "lora_attn_prefill")
+
+
+def la_device_check() -> int:
+    return int(lib.la_device_check())
+
+
+class DecodeStep:
+    """One decode step of the hot path: append the new token's LR row, then
+    attend every agent's query over the shared caches.
+
+    Holds the argument struct and the zero-filled split-K workspace so that a
+    step is two library calls.  Tensors must stay alive while it is used."""
+
+    def __init__(self, k_base, v_base, lr, B_k, B_v, q, out, kv_len, *, lora_scale, rope_base,
+                 max_kv_len, A_kv=None, x_new=None, pos_new=None):
+        self.args = make_args(k_base, v_base, lr, B_k, B_v, q, out, lora_scale=lora_scale,
+                              rope_base=rope_base, kv_len=kv_len, max_kv_len=max_kv_len)
+        self.workspace = decode_workspace(self.args, q.device)
+        self.lr, self.A_kv, self.x_new, self.pos_new = lr, A_kv, x_new, pos_new
+        self._keep = (k_base, v_base, lr, B_k, B_v, q, out, kv_len)
+
+    def __call__(self, stream=None) -> None:
+        if self.x_new is not None:
+            lr_cache_append(self.x_new, self.A_kv, self.lr, self.pos_new, stream)
+        lora_attn_decode(self.args, self.workspace, stream)

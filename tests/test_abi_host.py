@@ -1,0 +1,156 @@
+"""Host-side checks of the C ABI: the library loads on a machine without a GPU,
+exports every entry point include/lora_attn.h declares, its struct layout
+matches the binding, and invalid arguments are rejected before any launch.
+
+Every call below carries at least one invalid argument, so none of them can
+reach a kernel launch (the fake pointers are never dereferenced)."""
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+
+from rank_attention_b200 import lora_attn as la
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lora_attn.h")
+FAKE = 0x10000  # 16-byte aligned, never dereferenced
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b([a-z_][a-z0-9_]*)\s*\(", text)) -
+                  {"sizeof", "defined"})
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert set(names) == set(la.EXPORTED), names
+    lib = ctypes.CDLL(la.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings():
+    for s in range(7):
+        assert la.status_string(s).startswith("LA_")
+    assert "unknown" in la.status_string(99)
+
+
+def test_struct_layout_matches_header(tmp_path):
+    fields = [f[0] for f in la.AttnArgs._fields_]
+    src = tmp_path / "layout.c"
+    body = "\n".join(f'printf("{f} %zu\\n", offsetof(la_attn_args, {f}));' for f in fields)
+    src.write_text('#include <stdio.h>\n#include <stddef.h>\n#include "lora_attn.h"\n'
+                   "int main(void){" + body +
+                   'printf("sizeof %zu\\n", sizeof(la_attn_args)); return 0;}\n')
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-std=c99", "-I", os.path.join(ROOT, "include"), str(src), "-o",
+                    str(exe)], check=True)
+    out = dict(line.split() for line in subprocess.run([str(exe)], capture_output=True,
+                                                        text=True, check=True).stdout.split("\n")
+               if line)
+    for f in fields:
+        assert int(out[f]) == getattr(la.AttnArgs, f).offset, f
+    assert int(out["sizeof"]) == ctypes.sizeof(la.AttnArgs)
+
+
+def _append(**kw):
+    a = dict(X=FAKE, ldx=256, n=4, H=256, A=FAKE, r=8, lr=FAKE, L_max=16, pos0=0, n_seqs=1,
+             sx=0, slr=0, dt=la.LA_F32)
+    a.update(kw)
+    return la.lib.lr_cache_append(a["X"], a["ldx"], a["n"], a["H"], a["A"], a["r"], a["lr"],
+                                  a["L_max"], a["pos0"], a["n_seqs"], a["sx"], a["slr"], a["dt"],
+                                  None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(X=0), la.LA_ERR_INVALID_ARG),
+    (dict(A=0), la.LA_ERR_INVALID_ARG),
+    (dict(lr=0), la.LA_ERR_INVALID_ARG),
+    (dict(X=FAKE + 4), la.LA_ERR_INVALID_ARG),
+    (dict(r=12), la.LA_ERR_UNSUPPORTED),
+    (dict(dt=7), la.LA_ERR_INVALID_ARG),
+    (dict(ldx=100), la.LA_ERR_INVALID_ARG),
+    (dict(ldx=258), la.LA_ERR_INVALID_ARG),
+    (dict(pos0=13), la.LA_ERR_CAPACITY),
+    (dict(pos0=-1), la.LA_ERR_CAPACITY),
+    (dict(n=-1), la.LA_ERR_INVALID_ARG),
+    (dict(H=0), la.LA_ERR_INVALID_ARG),
+])
+def test_append_rejects(kw, status):
+    assert _append(**kw) == status
+
+
+def _args(**kw):
+    a = la.AttnArgs()
+    a.n_seqs, a.n_agents, a.n_q_heads, a.n_kv_heads, a.head_dim, a.r = 1, 2, 4, 2, 64, 8
+    a.lora_scale, a.softmax_scale, a.rope_base = 2.0, 0.125, 10000.0
+    a.L_max = 256
+    a.k_base = a.v_base = a.lr_cache = a.B_k = a.B_v = a.q = a.out = a.kv_len = FAKE
+    a.kv_seq_stride, a.kv_head_stride, a.kv_tok_stride = 2 * 256 * 64, 256 * 64, 64
+    a.lr_seq_stride = 256 * 16
+    a.max_kv_len = 256
+    a.q_pos0, a.n_q_tokens = 0, 1
+    a.io_dtype = a.out_dtype = la.LA_F32
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+BAD_ATTN = [
+    (dict(head_dim=96), la.LA_ERR_UNSUPPORTED),
+    (dict(r=24), la.LA_ERR_UNSUPPORTED),
+    (dict(n_q_heads=5), la.LA_ERR_INVALID_ARG),
+    (dict(n_agents=0), la.LA_ERR_INVALID_ARG),
+    (dict(k_base=0), la.LA_ERR_INVALID_ARG),
+    (dict(out=FAKE + 8), la.LA_ERR_INVALID_ARG),
+    (dict(kv_tok_stride=32), la.LA_ERR_INVALID_ARG),
+    (dict(kv_head_stride=3), la.LA_ERR_INVALID_ARG),
+    (dict(lr_seq_stride=100), la.LA_ERR_INVALID_ARG),
+    (dict(softmax_scale=0.0), la.LA_ERR_INVALID_ARG),
+    (dict(softmax_scale=float("nan")), la.LA_ERR_INVALID_ARG),
+    (dict(rope_base=0.5), la.LA_ERR_INVALID_ARG),
+    (dict(io_dtype=3), la.LA_ERR_INVALID_ARG),
+    (dict(n_agents=40), la.LA_ERR_UNSUPPORTED),
+]
+
+
+@pytest.mark.parametrize("kw,status", BAD_ATTN + [
+    (dict(n_q_tokens=2), la.LA_ERR_INVALID_ARG),
+    (dict(kv_len=0), la.LA_ERR_INVALID_ARG),
+    (dict(max_kv_len=0), la.LA_ERR_INVALID_ARG),
+    (dict(max_kv_len=257), la.LA_ERR_CAPACITY),
+])
+def test_decode_rejects(kw, status):
+    a = _args(**kw)
+    assert la.lib.lora_attn_decode(ctypes.byref(a), FAKE, 1 << 20, None) == status
+    assert la.lib.lora_attn_decode_workspace_bytes(ctypes.byref(a)) == 0
+
+
+def test_decode_rejects_small_workspace():
+    a = _args()
+    need = la.lib.lora_attn_decode_workspace_bytes(ctypes.byref(a))
+    assert need > 0
+    assert la.lib.lora_attn_decode(ctypes.byref(a), FAKE, need - 1, None) == la.LA_ERR_WORKSPACE
+    assert la.lib.lora_attn_decode(ctypes.byref(a), 0, need, None) == la.LA_ERR_WORKSPACE
+    assert la.lib.lora_attn_decode(ctypes.byref(a), FAKE + 16, need, None) == la.LA_ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("kw,status", BAD_ATTN + [
+    (dict(q_pos0=250, n_q_tokens=7), la.LA_ERR_CAPACITY),
+    (dict(q_pos0=-1), la.LA_ERR_INVALID_ARG),
+    (dict(n_q_tokens=-1), la.LA_ERR_INVALID_ARG),
+])
+def test_prefill_rejects(kw, status):
+    a = _args(**kw)
+    assert la.lib.lora_attn_prefill(ctypes.byref(a), None) == status
+
+
+def test_null_args():
+    assert la.lib.lora_attn_prefill(None, None) == la.LA_ERR_INVALID_ARG
+    assert la.lib.lora_attn_decode(None, FAKE, 1 << 20, None) == la.LA_ERR_INVALID_ARG
+    assert la.lib.lora_attn_decode_workspace_bytes(None) == 0

@@ -1,0 +1,295 @@
+"""CUDA path vs the fp64 oracle, element by element, through the C ABI.
+
+Small cases run the oracle on every output; the LLaMA-shaped cases run the
+CUDA path at full size and compare every output the oracle can afford
+(all of the 8k decode; sampled (agent, KV head, token) units elsewhere)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import impl as oracle
+from rank_attention_b200 import workloads as W
+from tests.helpers import (assert_parity, bf16_ulp, errors, oracle_decode, to_device, to_np)
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module")
+def la():
+    from rank_attention_b200 import lora_attn
+    return lora_attn
+
+
+# ------------------------------------------------------------- LR append ----
+def _append_case(la, n_seqs, n, H, r, dtype, L_max, pos0, seed):
+    inp = W.append_inputs(n, H, r, dtype, seed, n_seqs=n_seqs)
+    sentinel = -123.5
+    lr = torch.full((n_seqs, L_max, 2 * r), sentinel, dtype=dtype, device=DEV)
+    la.lr_cache_append(inp["X"].to(DEV), inp["A_kv"].to(DEV), lr, pos0)
+    torch.cuda.synchronize()
+    got = lr.cpu()
+    ref = oracle.lr_cache_rows(inp["X"], inp["A_kv"])
+    # rows outside [pos0, pos0 + n) untouched, bit for bit
+    outside = torch.ones(L_max, dtype=torch.bool)
+    outside[pos0:pos0 + n] = False
+    assert (got[:, outside] == sentinel).all()
+    rows = to_np(got[:, pos0:pos0 + n])
+    if dtype == torch.float32:
+        mx, _ = errors(rows, ref)
+        assert mx <= 1e-5
+    else:
+        # the fp64 value rounded to bf16, within one bf16 ulp (fp32 accumulation order)
+        bound = np.maximum(bf16_ulp(ref),
+                           1e-6 * (np.abs(to_np(inp["X"])) @ np.abs(to_np(inp["A_kv"]))))
+        assert (np.abs(rows - ref) <= bound).all(), np.abs(rows - ref).max()
+
+
+def test_append_fp32_tiny(la):
+    s = W.TINY_FP32
+    _append_case(la, 1, s.kv_len, s.hidden, s.r, torch.float32, 300, 20, seed=0)
+
+
+@pytest.mark.parametrize("r", [8, 16, 32, 64])
+def test_append_bf16_ragged(la, r):
+    _append_case(la, 2, 333, 4096, r, torch.bfloat16, 1000, 501, seed=r)
+
+
+def test_append_bf16_single_row_and_last_slot(la):
+    _append_case(la, 1, 1, 4096, 16, torch.bfloat16, 8192, 8191, seed=5)
+
+
+def test_append_bf16_stack_chunk(la):
+    # 4096-token chunk through r=64 shared A (one layer of the 32-layer stack)
+    _append_case(la, 1, 4096, 4096, 64, torch.bfloat16, 4096 + 64, 37, seed=6)
+
+
+def test_append_empty_is_noop(la):
+    lr = torch.full((1, 8, 16), 3.0, device=DEV)
+    X = torch.zeros((1, 0, 256), device=DEV)
+    A = torch.zeros((256, 16), device=DEV)
+    la.lr_cache_append(X, A, lr, 8)
+    torch.cuda.synchronize()
+    assert (lr == 3.0).all()
+
+
+# ----------------------------------------------------- tiny fp32 (exact) ----
+def _tiny_caches(shape, L_max=None):
+    w = W.hidden_layer_weights(shape)
+    kb, vb = oracle.base_cache_from_hidden(w["X"], w["W_k"], w["W_v"], shape.n_kv_heads,
+                                           shape.rope_base)
+    L = shape.kv_len
+    L_max = L if L_max is None else L_max
+    k_base = torch.zeros((shape.n_seqs, shape.n_kv_heads, L_max, shape.head_dim))
+    v_base = torch.zeros_like(k_base)
+    k_base[:, :, :L] = torch.from_numpy(kb).float()
+    v_base[:, :, :L] = torch.from_numpy(vb).float()
+    return w, k_base, v_base
+
+
+def _run(la, shape, k_base, v_base, lr, B_k, B_v, q, kv_len=None, mode=None, out_dtype=None):
+    mode = mode or shape.mode
+    out = torch.empty(q.shape, dtype=out_dtype or torch.float32, device=DEV)
+    if mode == "decode":
+        args = la.make_args(k_base, v_base, lr, B_k, B_v, q, out, lora_scale=shape.lora_scale,
+                            rope_base=shape.rope_base, kv_len=kv_len,
+                            max_kv_len=int(kv_len.max().item()))
+        ws = la.decode_workspace(args, DEV)
+        la.lora_attn_decode(args, ws)
+    else:
+        args = la.make_args(k_base, v_base, lr, B_k, B_v, q, out, lora_scale=shape.lora_scale,
+                            rope_base=shape.rope_base, q_pos0=shape.q_pos0)
+        la.lora_attn_prefill(args)
+    torch.cuda.synchronize()
+    assert la.la_device_check() == 0
+    return out
+
+
+def test_tiny_fp32_decode_step_from_hidden(la):
+    """Full step: GPU appends LR = X A, then decodes; oracle works from X in fp64."""
+    s = W.TINY_FP32
+    w, k_base, v_base = _tiny_caches(s)
+    lr = torch.zeros((1, s.kv_len, 2 * s.r), device=DEV)
+    la.lr_cache_append(w["X"].to(DEV), w["A_kv"].to(DEV), lr, 0)
+    kv_len = torch.tensor([s.kv_len], dtype=torch.int32, device=DEV)
+    got = _run(la, s, k_base.to(DEV), v_base.to(DEV), lr, w["B_k"].to(DEV), w["B_v"].to(DEV),
+               w["q"].to(DEV), kv_len)
+    kb, vb = oracle.base_cache_from_hidden(w["X"], w["W_k"], w["W_v"], s.n_kv_heads, s.rope_base)
+    ref = oracle.lora_attention(kb, vb, oracle.lr_cache_rows(w["X"], w["A_kv"]), w["B_k"],
+                                w["B_v"], w["q"], [s.kv_len], lora_scale=s.lora_scale,
+                                softmax_scale=s.softmax_scale, rope_base=s.rope_base,
+                                mode="decode")
+    assert_parity(to_np(got), ref, torch.float32)
+
+
+@pytest.mark.parametrize("kv_len", [1, 2, 31, 33, 200, 256])
+def test_tiny_fp32_decode_lengths(la, kv_len):
+    s = W.TINY_FP32
+    w, k_base, v_base = _tiny_caches(s)
+    lr = torch.from_numpy(oracle.lr_cache_rows(w["X"], w["A_kv"])).float()
+    kvl = torch.tensor([kv_len], dtype=torch.int32)
+    got = _run(la, s, k_base.to(DEV), v_base.to(DEV), lr.to(DEV), w["B_k"].to(DEV),
+               w["B_v"].to(DEV), w["q"].to(DEV), kvl.to(DEV))
+    ref = oracle.lora_attention(k_base, v_base, lr, w["B_k"], w["B_v"], w["q"], kvl,
+                                lora_scale=s.lora_scale, softmax_scale=s.softmax_scale,
+                                rope_base=s.rope_base, mode="decode")
+    assert_parity(to_np(got), ref, torch.float32)
+
+
+@pytest.mark.parametrize("n_tok", [1, 40, 77])
+def test_tiny_fp32_prefill(la, n_tok):
+    s = W.TINY_FP32.replace(n_q_tokens=n_tok, mode="prefill")
+    w, k_base, v_base = _tiny_caches(s)
+    lr = torch.from_numpy(oracle.lr_cache_rows(w["X"], w["A_kv"])).float()
+    got = _run(la, s, k_base.to(DEV), v_base.to(DEV), lr.to(DEV), w["B_k"].to(DEV),
+               w["B_v"].to(DEV), w["q"].to(DEV))
+    ref = oracle.lora_attention(k_base, v_base, lr, w["B_k"], w["B_v"], w["q"], [s.kv_len],
+                                lora_scale=s.lora_scale, softmax_scale=s.softmax_scale,
+                                rope_base=s.rope_base, mode="prefill")
+    assert_parity(to_np(got), ref, torch.float32)
+
+
+# ----------------------------------------------------------- bf16 decode ----
+def test_llama8b_decode_8k_full(la):
+    """The 8192-token, 3-agent, r=16 decode: every output against the oracle."""
+    s = W.LLAMA8B_DECODE_8K
+    inp = W.direct_cache_inputs(s)
+    d = to_device(inp)
+    got = _run(la, s, d["k_base"], d["v_base"], d["lr"], d["B_k"], d["B_v"], d["q"], d["kv_len"])
+    ref = oracle_decode(inp, s)
+    assert_parity(to_np(got), ref, s.dtype)
+    # the LoRA terms matter at this scale: dropping them would fail the bar
+    no_lora = oracle.lora_attention(inp["k_base"], inp["v_base"], inp["lr"], inp["B_k"] * 0,
+                                    inp["B_v"] * 0, inp["q"], inp["kv_len"],
+                                    lora_scale=s.lora_scale, softmax_scale=s.softmax_scale,
+                                    rope_base=s.rope_base, mode="decode")
+    assert errors(no_lora, ref)[0] > 20 * 1e-2
+
+
+@pytest.mark.parametrize("r,n_agents,d,lens", [
+    (16, 3, 128, [1, 37, 1000]),
+    (32, 5, 128, [64, 65, 129]),
+    (64, 2, 128, [513, 2, 300]),
+    (8, 4, 128, [100, 7, 1024]),
+    (16, 3, 64, [1024, 500, 33]),
+])
+def test_bf16_decode_ragged(la, r, n_agents, d, lens):
+    s = W.LLAMA8B_DECODE_8K.replace(n_seqs=len(lens), n_agents=n_agents, head_dim=d, r=r,
+                                    alpha=2.0 * r, kv_len=max(lens), seed=11 + r)
+    inp = W.direct_cache_inputs(s, L_max=max(lens) + 16)
+    inp["kv_len"] = torch.tensor(lens, dtype=torch.int32)
+    dd = to_device(inp)
+    got = _run(la, s, dd["k_base"], dd["v_base"], dd["lr"], dd["B_k"], dd["B_v"], dd["q"],
+               dd["kv_len"])
+    assert_parity(to_np(got), oracle_decode(inp, s), s.dtype)
+
+
+def test_bf16_decode_token_major_layout(la):
+    """Base cache stored [seq][token][head][d]: same result as head-major."""
+    s = W.LLAMA8B_DECODE_8K.replace(kv_len=777, n_seqs=2, seed=21)
+    inp = W.direct_cache_inputs(s)
+    dd = to_device(inp)
+    kt = dd["k_base"].permute(0, 2, 1, 3).contiguous().permute(0, 2, 1, 3)
+    vt = dd["v_base"].permute(0, 2, 1, 3).contiguous().permute(0, 2, 1, 3)
+    a = _run(la, s, dd["k_base"], dd["v_base"], dd["lr"], dd["B_k"], dd["B_v"], dd["q"],
+             dd["kv_len"])
+    b = _run(la, s, kt, vt, dd["lr"], dd["B_k"], dd["B_v"], dd["q"], dd["kv_len"])
+    assert torch.equal(a, b)
+    assert_parity(to_np(b), oracle_decode(inp, s), s.dtype)
+
+
+def test_decode_workspace_reuse_is_deterministic(la):
+    s = W.LLAMA8B_DECODE_8K.replace(kv_len=3000, seed=22)
+    dd = to_device(W.direct_cache_inputs(s))
+    out1 = torch.empty(dd["q"].shape, device=DEV)
+    out2 = torch.empty_like(out1)
+    a1 = la.make_args(dd["k_base"], dd["v_base"], dd["lr"], dd["B_k"], dd["B_v"], dd["q"], out1,
+                      lora_scale=s.lora_scale, rope_base=s.rope_base, kv_len=dd["kv_len"],
+                      max_kv_len=s.kv_len)
+    a2 = la.make_args(dd["k_base"], dd["v_base"], dd["lr"], dd["B_k"], dd["B_v"], dd["q"], out2,
+                      lora_scale=s.lora_scale, rope_base=s.rope_base, kv_len=dd["kv_len"],
+                      max_kv_len=s.kv_len)
+    ws = la.decode_workspace(a1, DEV)
+    la.lora_attn_decode(a1, ws)
+    la.lora_attn_decode(a2, ws)
+    torch.cuda.synchronize()
+    assert torch.equal(out1, out2)
+
+
+def test_decode_kv_len_beyond_bound_is_reported(la):
+    """kv_len above max_kv_len: the kernel's own check skips that sequence and
+    raises the device error word; the other sequence is still computed."""
+    s = W.LLAMA8B_DECODE_8K.replace(kv_len=500, n_seqs=2, seed=23)
+    inp = W.direct_cache_inputs(s, L_max=600)
+    dd = to_device(inp)
+    dd["kv_len"] = torch.tensor([500, 550], dtype=torch.int32, device=DEV)
+    out = torch.full(dd["q"].shape, 7.0, device=DEV)
+    args = la.make_args(dd["k_base"], dd["v_base"], dd["lr"], dd["B_k"], dd["B_v"], dd["q"], out,
+                        lora_scale=s.lora_scale, rope_base=s.rope_base, kv_len=dd["kv_len"],
+                        max_kv_len=500)
+    la.lora_attn_decode(args, la.decode_workspace(args, DEV))
+    assert la.la_device_check() == la.LA_ERR_DEVICE_CHECK
+    assert la.la_device_check() == 0
+    assert (out[1] == 7.0).all()
+    ref = oracle_decode(dict(inp, kv_len=torch.tensor([500, 500])), s)
+    assert_parity(to_np(out[0]), ref[0], s.dtype)
+
+
+# ---------------------------------------------------------- bf16 prefill ----
+@pytest.mark.parametrize("L,n_tok,r,n_agents", [
+    (300, 77, 16, 3),
+    (129, 129, 32, 2),
+    (1000, 256, 64, 4),
+    (65, 1, 8, 1),
+])
+def test_bf16_prefill_small(la, L, n_tok, r, n_agents):
+    s = W.LLAMA8B_PREFILL_16K.replace(kv_len=L, n_q_tokens=n_tok, r=r, alpha=2.0 * r,
+                                      n_agents=n_agents, seed=31 + L)
+    inp = W.direct_cache_inputs(s)
+    dd = to_device(inp)
+    got = _run(la, s, dd["k_base"], dd["v_base"], dd["lr"], dd["B_k"], dd["B_v"], dd["q"])
+    ref = oracle.lora_attention(inp["k_base"], inp["v_base"], inp["lr"], inp["B_k"], inp["B_v"],
+                                inp["q"], inp["kv_len"], lora_scale=s.lora_scale,
+                                softmax_scale=s.softmax_scale, rope_base=s.rope_base,
+                                mode="prefill")
+    assert_parity(to_np(got), ref, s.dtype)
+
+
+def _sampled_units(la, s, inp, got, units, tokens):
+    """Compare sampled (seq, agent, kv head) x query tokens against the oracle."""
+    g = s.group
+    refs, gots = [], []
+    for (seq, agent, kvh) in units:
+        kvl = int(inp["kv_len"][seq])
+        qpos = oracle.query_positions(kvl, s.n_q_tokens, s.mode, s.q_pos0 if s.mode == "prefill"
+                                      else None)
+        ref = oracle.lora_attention_unit(inp["k_base"], inp["v_base"], inp["lr"], inp["B_k"],
+                                         inp["B_v"], inp["q"], seq=seq, agent=agent, kv_head=kvh,
+                                         kv_len=kvl, q_positions=qpos, lora_scale=s.lora_scale,
+                                         softmax_scale=s.softmax_scale, rope_base=s.rope_base,
+                                         q_tokens=tokens)
+        refs.append(ref)
+        gots.append(to_np(got[seq, agent][tokens][:, kvh * g:(kvh + 1) * g]))
+    return assert_parity(np.stack(gots), np.stack(refs), s.dtype)
+
+
+def test_llama8b_prefill_16k_sampled(la):
+    s = W.LLAMA8B_PREFILL_16K
+    inp = W.direct_cache_inputs(s)
+    dd = to_device(inp)
+    got = _run(la, s, dd["k_base"], dd["v_base"], dd["lr"], dd["B_k"], dd["B_v"], dd["q"]).cpu()
+    tokens = np.array([0, 1, 63, 64, 127, 500, 1000, 1022, 1023])
+    _sampled_units(la, s, inp, got, [(0, 0, 0), (0, 1, 3), (0, 2, 7)], tokens)
+
+
+@pytest.mark.parametrize("ctx", [32768])
+def test_llama8b_sweep_decode_sampled(la, ctx):
+    s = W.llama8b_sweep(ctx)
+    inp = W.direct_cache_inputs(s)
+    dd = to_device(inp)
+    got = _run(la, s, dd["k_base"], dd["v_base"], dd["lr"], dd["B_k"], dd["B_v"], dd["q"],
+               dd["kv_len"]).cpu()
+    _sampled_units(la, s, inp, got, [(0, 0, 0), (5, 4, 7), (15, 2, 3)], np.array([0]))
