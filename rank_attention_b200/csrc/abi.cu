@@ -23,6 +23,7 @@ int* error_word_ptr() {
 size_t simt_rows_cap(const AttnParams& p);
 int simt_key_tile();
 bool bf16_decode_supported(const AttnParams& p);
+size_t bf16_decode_partial_bytes(const AttnParams& p);
 void bf16_decode_plan(const AttnParams& p, int* n_splits, int64_t* split_len, int* rows);
 cudaError_t launch_decode_bf16(const AttnParams& p, la_dtype out, cudaStream_t st);
 bool bf16_prefill_supported(const AttnParams& p);
@@ -126,7 +127,10 @@ DecodePlan plan_decode(const AttnParams& p, la_dtype io) {
     d.rows = (int)simt_rows_cap(p);
   }
   const size_t W = (size_t)p.d + p.r + 2;
-  d.partial_bytes = d.n_splits > 1 ? (size_t)units * d.n_splits * d.rows * W * sizeof(float) : 0;
+  if (d.kind == 1)
+    d.partial_bytes = bf16_decode_partial_bytes(p);
+  else
+    d.partial_bytes = d.n_splits > 1 ? (size_t)units * d.n_splits * d.rows * W * sizeof(float) : 0;
   d.partial_bytes = (d.partial_bytes + 255) / 256 * 256;
   d.counter_bytes = ((size_t)units * sizeof(int) + 255) / 256 * 256;
   return d;

@@ -1,0 +1,237 @@
+// lr_cache_append on the tensor cores (bf16 in, fp32 accumulate, bf16 out).
+//
+// PreLRShared precompute (PReCache abstract and blog; LRAgent summary §3
+// BaseLRShared): LR[pos0 + i] = X_i [A_k | A_v], computed once per new chunk
+// through the A every agent shares.  The rows are stored unscaled and
+// unrotated, K part first.
+//
+// A CTA owns 64 chunk rows (16 per warp) and all 2r output columns; TMA
+// stages 64 x 64 slices of X and of A_kv (128/64/32-byte swizzle, no
+// multicast) through a 3-stage mbarrier pipeline, and warp-level bf16 MMAs
+// accumulate in fp32.  The hidden dimension is split over the CTAs of a
+// thread-block cluster so that short chunks (a single decode token) still
+// spread over many SMs; the partial sums meet in distributed shared memory,
+// where each CTA reduces and writes its share of the rows.
+#include <cooperative_groups.h>
+#include <cudaTypedefs.h>
+
+#include "la_internal.cuh"
+#include "ptx.cuh"
+
+namespace la {
+namespace {
+
+namespace cg = cooperative_groups;
+using namespace ptx;
+
+constexpr int TM = 64;     // chunk rows per CTA
+constexpr int KC = 64;     // hidden columns per stage
+constexpr int NTHR = 128;
+constexpr int NSTAGE = 3;
+constexpr int kMaxHS = 16;
+constexpr int kSMs = 148;
+
+constexpr int align1k(int x) { return (x + 1023) / 1024 * 1024; }
+
+template <int R>
+struct ACfg {
+  static constexpr int C = 2 * R;                       // output columns
+  static constexpr int X_TILE = TM * KC * 2;            // 8 KB
+  static constexpr int A_TILE = align1k(KC * C * 2);
+  static constexpr int STAGE = X_TILE + A_TILE;
+  static constexpr int RED = TM * C * 4;                // fp32 partial
+  static constexpr int AREA = NSTAGE * STAGE > RED ? NSTAGE * STAGE : align1k(RED);
+  static constexpr size_t smem = 1024 + AREA + 64;
+};
+
+template <int R>
+__global__ void __launch_bounds__(NTHR, 1)
+    append_bf16_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmA,
+                       __nv_bfloat16* __restrict__ lr, int64_t pos0, int64_t n, int64_t slr,
+                       int hs, int kchunks, int* err) {
+  using Cf = ACfg<R>;
+  constexpr int C = Cf::C;
+  constexpr int NTN = C / 8;       // n-tiles of the output
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t area_u = smem_u32(smem);
+  const uint32_t bar_u = smem_u32(smem + Cf::AREA);
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int gq = lane >> 2, t4 = lane & 3, mi = lane >> 3, rr = lane & 7;
+  const int cr = blockIdx.x % hs;              // rank in the cluster = hidden split
+  const int mtile = blockIdx.x / hs;
+  const int seq = blockIdx.y;
+  const int64_t t0 = (int64_t)mtile * TM;
+  const int kb = cr * kchunks / hs, ke = (cr + 1) * kchunks / hs;
+  const int nk = ke - kb;
+  cg::cluster_group cluster = cg::this_cluster();
+
+  if (tid == 0) {
+    for (int s = 0; s < NSTAGE; ++s) mbar_init(bar_u + 8 * s, 1);
+    fence_mbar_init();
+    tma_prefetch(&tmX);
+    tma_prefetch(&tmA);
+  }
+  __syncthreads();
+  auto issue = [&](int j) {
+    const int s = j % NSTAGE;
+    const uint32_t sb = area_u + s * Cf::STAGE;
+    const uint32_t bar = bar_u + 8 * s;
+    const int h0 = (kb + j) * KC;
+    mbar_expect_tx(bar, Cf::X_TILE + KC * C * 2);
+    tma_load_3d(sb, &tmX, bar, h0, (int)t0, seq);
+    constexpr int AB = C < 64 ? C : 64;
+#pragma unroll
+    for (int b = 0; b < C / AB; ++b) tma_load_2d_(sb + Cf::X_TILE + b * KC * AB * 2, &tmA, bar, AB * b, h0);
+  };
+  if (tid == 0)
+    for (int j = 0; j < NSTAGE && j < nk; ++j) issue(j);
+
+  float acc[NTN][4];
+#pragma unroll
+  for (int q = 0; q < NTN; ++q)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[q][e] = 0.f;
+
+  int fail = 0;
+  for (int j = 0; j < nk; ++j) {
+    const int s = j % NSTAGE;
+    if (!mbar_wait(bar_u + 8 * s, (j / NSTAGE) & 1)) fail = 1;
+    if (__syncthreads_or(fail)) {
+      fail = 1;
+      break;
+    }
+    const uint32_t sX = area_u + s * Cf::STAGE;
+    const uint32_t sA = sX + Cf::X_TILE;
+#pragma unroll
+    for (int ks = 0; ks < KC / 16; ++ks) {
+      uint32_t a[4];
+      ldsm_x4(a, sX + tile_off<KC, TM>(16 * w + rr + (mi & 1) * 8, 16 * ks + (mi >> 1) * 8));
+#pragma unroll
+      for (int q = 0; q < NTN; q += 2) {
+        uint32_t b[4];
+        ldsm_x4_t(b, sA + tile_off<C, KC>(16 * ks + rr + (mi & 1) * 8, 8 * (q + (mi >> 1))));
+        mma16816(acc[q], a, b[0], b[1]);
+        mma16816(acc[q + 1], a, b[2], b[3]);
+      }
+    }
+    __syncthreads();
+    if (tid == 0 && j + NSTAGE < nk) issue(j + NSTAGE);
+  }
+  if (fail && tid == 0) atomicOr(err, 2);
+
+  // partial sums -> shared memory (stage area reused), then reduce over the cluster
+  __syncthreads();
+  float* red = reinterpret_cast<float*>(smem);
+#pragma unroll
+  for (int q = 0; q < NTN; ++q)
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      red[(16 * w + gq + (e >> 1) * 8) * C + 8 * q + 2 * t4 + (e & 1)] = acc[q][e];
+  if (hs > 1) cluster.sync();
+  else __syncthreads();
+  if (!fail) {
+    const int rows_per = (TM + hs - 1) / hs;
+    const int r0 = cr * rows_per;
+    for (int i = tid; i < rows_per * C; i += NTHR) {
+      const int row = r0 + i / C, c = i % C;
+      if (row >= TM || t0 + row >= n) continue;
+      float v = 0.f;
+      for (int k = 0; k < hs; ++k) v += cluster.map_shared_rank(red, k)[row * C + c];
+      lr[seq * slr + (pos0 + t0 + row) * C + c] = __float2bfloat16_rn(v);
+    }
+  }
+  if (hs > 1) cluster.sync();
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+template <int R>
+cudaError_t launch_r(const void* X, int64_t ldx, int64_t n, int64_t H, const void* A, void* lr,
+                     int64_t pos0, int n_seqs, int64_t sx, int64_t slr, int* err, cudaStream_t st) {
+  using Cf = ACfg<R>;
+  constexpr int C = 2 * R;
+  auto enc = encode_fn();
+  if (!enc) return cudaErrorInvalidValue;
+  CUtensorMap mx, ma;
+  cuuint64_t xd[3] = {(cuuint64_t)H, (cuuint64_t)n, (cuuint64_t)n_seqs};
+  cuuint64_t xs[2] = {(cuuint64_t)ldx * 2, (cuuint64_t)(n_seqs > 1 ? sx : n * ldx) * 2};
+  cuuint32_t xb[3] = {KC, TM, 1};
+  cuuint32_t one[3] = {1, 1, 1};
+  if (enc(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(X), xd, xs, xb, one,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  constexpr int AB = C < 64 ? C : 64;
+  cuuint64_t ad[2] = {(cuuint64_t)C, (cuuint64_t)H};
+  cuuint64_t as[1] = {(cuuint64_t)C * 2};
+  cuuint32_t ab[2] = {AB, KC};
+  const CUtensorMapSwizzle sw = AB * 2 == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : AB * 2 == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B;
+  if (enc(&ma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(A), ad, as, ab, one,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  const int kchunks = (int)((H + KC - 1) / KC);
+  const int64_t mtiles = (n + TM - 1) / TM;
+  int hs = (int)(kSMs / (mtiles * n_seqs));
+  if (hs > kMaxHS) hs = kMaxHS;
+  if (hs > kchunks) hs = kchunks;
+  if (hs < 1) hs = 1;
+  auto kern = append_bf16_kernel<R>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cf::smem);
+  if (e != cudaSuccess) return e;
+  if (hs > 8) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(mtiles * hs), n_seqs);
+  cfg.blockDim = dim3(NTHR);
+  cfg.dynamicSmemBytes = Cf::smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = hs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, mx, ma, static_cast<__nv_bfloat16*>(lr), pos0, n, slr, hs,
+                         kchunks, err);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool bf16_append_supported(int64_t H, int r) {
+  return H >= 16 && H < (1ll << 31) && (r == 8 || r == 16 || r == 32 || r == 64);
+}
+
+cudaError_t launch_append_bf16_mma(const void* X, int64_t ldx, int64_t n, int64_t H,
+                                   const void* A, int r, void* lr, int64_t pos0, int n_seqs,
+                                   int64_t sx, int64_t slr, cudaStream_t st) {
+  int* err = error_word_ptr();
+  if (!err) return cudaErrorInvalidValue;
+  switch (r) {
+    case 8: return launch_r<8>(X, ldx, n, H, A, lr, pos0, n_seqs, sx, slr, err, st);
+    case 16: return launch_r<16>(X, ldx, n, H, A, lr, pos0, n_seqs, sx, slr, err, st);
+    case 32: return launch_r<32>(X, ldx, n, H, A, lr, pos0, n_seqs, sx, slr, err, st);
+    default: return launch_r<64>(X, ldx, n, H, A, lr, pos0, n_seqs, sx, slr, err, st);
+  }
+}
+
+}  // namespace la
