@@ -43,6 +43,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", action="store_true",
+                    help="only run the decode kernel a few times on one cache set (for ncu)")
     return ap.parse_args()
 
 
@@ -100,6 +102,64 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+# DRAM bytes per decode launch from an ncu capture of the workload, keyed by the
+# sha256 prefix of the decode kernel's source: reported only while the kernel is
+# unchanged since the counters were taken.
+DECODE_TRAFFIC = {"022d280010462508": 34375936}
+
+
+def decode_source_sha() -> str:
+    import hashlib
+    path = os.path.join(ROOT, "rank_attention_b200", "csrc", "attn_decode_bf16.cu")
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def decode_kernels_per_call(s) -> int:
+    """Kernels one lora_attn_decode call launches for this workload: the decode
+    kernel, plus the split-merge kernel when the keys are split over CTAs (the
+    library splits each (sequence, KV head) over min(32, 148 // units, tiles of
+    128 keys) CTAs)."""
+    units = s.n_seqs * s.n_kv_heads
+    splits = 1 if units >= 148 else min(32, 148 // units, (s.kv_len + 127) // 128)
+    return 2 if splits > 1 else 1
+
+
+def run_profile():
+    """A short, deterministic run of the decode kernel alone, for profilers."""
+    import torch
+    from rank_attention_b200 import lora_attn as la
+    from rank_attention_b200 import workloads as W
+    s = W.LLAMA8B_DECODE_8K
+    dev = torch.device("cuda", 0)
+    inp = {k: v.to(dev) for k, v in W.direct_cache_inputs(s, device=dev).items()}
+    out = torch.empty(inp["q"].shape, dtype=torch.float32, device=dev)
+    args = la.make_args(inp["k_base"], inp["v_base"], inp["lr"], inp["B_k"], inp["B_v"], inp["q"],
+                        out, lora_scale=s.lora_scale, rope_base=s.rope_base,
+                        kv_len=inp["kv_len"], max_kv_len=s.kv_len)
+    ws = la.decode_workspace(args, dev)
+    for _ in range(5):
+        la.lora_attn_decode(args, ws)
+    torch.cuda.synchronize()
+    return 0 if la.la_device_check() == 0 else 1
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """Maximum of a per-rank scalar over all ranks (every rank gets it)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank_step: int, steps: int, world: int, ms_max: float) -> float:
+    """Units processed by all ranks per second, timed by the slowest rank."""
+    return units_per_rank_step * steps * world / (ms_max / 1e3)
+
+
 def decode_bytes(s) -> int:
     """Algorithmic HBM bytes of one decode launch: base K and V read once, LR
     cache read once, every agent's B_k and B_v, the queries and the fp32 outputs."""
@@ -152,23 +212,47 @@ def time_oracle(s, steps: int, budget_s: float):
     return s.n_seqs * s.n_agents / per, len(times), per
 
 
+def oracle_unit_step(inp, new, s, k: int) -> None:
+    """One reference step: the oracle's decode of one (agent, KV head) unit of the
+    workload (unit k cycles through all of them), after appending the new LR row."""
+    from oracle import impl as oracle
+    a = k % s.n_agents
+    j = (k // s.n_agents) % s.n_kv_heads
+    lr = oracle.lr_cache_append(inp["lr"], new["X"], new["A_kv"], s.kv_len - 1)
+    oracle.lora_attention_unit(inp["k_base"], inp["v_base"], lr, inp["B_k"], inp["B_v"],
+                               inp["q"], seq=0, agent=a, kv_head=j, kv_len=s.kv_len,
+                               q_positions=[s.kv_len - 1], lora_scale=s.lora_scale,
+                               softmax_scale=s.softmax_scale, rope_base=s.rope_base)
+
+
 def run_reference(args):
+    """The reference arm: the fp64 oracle on the host cores (rank 0 only)."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
     from rank_attention_b200 import workloads as W
     s = W.LLAMA8B_DECODE_8K
-    # warm-up steps, then the timed steps (a bounded sample: the oracle is slow)
-    time_oracle(s, max(1, min(args.warmup, 1)), 5.0)
-    value, n, per = time_oracle(s, args.steps, 60.0)
+    inp = W.direct_cache_inputs(s)
+    new = W.append_inputs(1, s.hidden, s.r, s.dtype, seed=s.seed + 100, n_seqs=s.n_seqs)
+    for k in range(args.warmup):
+        oracle_unit_step(inp, new, s, k)
+    t0 = time.perf_counter()
+    for k in range(args.steps):
+        oracle_unit_step(inp, new, s, k)
+    per_unit = (time.perf_counter() - t0) / args.steps
+    units = s.n_agents * s.n_kv_heads
+    full_step = per_unit * units          # one whole decode step of the workload
+    value = s.n_seqs * s.n_agents / full_step
     cores = blas_threads()
+    sample = (f"each step = one of the {units} (agent, KV head) units of {s.name} "
+              f"(append + materialised attention), cycled; rate scaled to the whole step")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
-            "n_gpus": args.gpus, "steps": n, "warmup": args.warmup,
-            "ms_per_step": per * 1e3, "higher_is_better": True, "scaling": "weak",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": full_step * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": s.name, "sample": f"{n} full decode steps"},
+            "config": {"workload": s.name, "kv_len": s.kv_len, "agents": s.n_agents, "r": s.r},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
-                             "sample": f"{n} full decode steps of {s.name} (append + attention)"},
+                             "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -237,12 +321,6 @@ def run_ours(args):
         if world > 1:
             dist.barrier()
 
-    def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
 
     clocks = ClockSampler(local)
     clocks.start()
@@ -258,7 +336,7 @@ def run_ours(args):
         ev1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    ms = max_over_ranks(ev0.elapsed_time(ev1))
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
     # decode kernel alone
     d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
@@ -269,8 +347,7 @@ def run_ours(args):
     clk = clocks.stop()
     dec_ms = d0.elapsed_time(d1) / (n_sets * reps)
 
-    agent_tokens = s.n_seqs * s.n_agents * args.steps * world
-    value = agent_tokens / (ms / 1e3)
+    value = whole_job_rate(s.n_seqs * s.n_agents, args.steps, world, ms)
 
     # end to end through the public API with host buffers: H2D of the step's
     # inputs (new hidden row, queries, lengths), the two calls, D2H of outputs
@@ -304,8 +381,8 @@ def run_ours(args):
         e1.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e_ms = max_over_ranks(e0.elapsed_time(e1))
-    e2e_value = s.n_seqs * s.n_agents * e_steps * world / (e_ms / 1e3)
+    e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e_value = whole_job_rate(s.n_seqs * s.n_agents, e_steps, world, e_ms)
 
     hbm, peak_kind = peaks()
     dbytes = decode_bytes(s)
@@ -324,10 +401,10 @@ def run_ours(args):
                      "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                      "peak_kind": f"{peak_kind} copy bandwidth",
                      "algorithmic_bytes_per_launch": dbytes, "launch_us": dec_ms * 1e3,
-                     "traffic": None},
+                     "traffic": DECODE_TRAFFIC.get(decode_source_sha())},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e_steps},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": (1 + decode_kernels_per_call(s)) * args.steps,
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -347,6 +424,8 @@ def main():
     args = parse()
     if args.impl == "reference":
         return run_reference(args)
+    if args.profile:
+        return run_profile()
     return run_ours(args)
 
 

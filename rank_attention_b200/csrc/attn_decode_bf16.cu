@@ -32,6 +32,8 @@
 // forms out = sum_k w_k Z_k / sum_k w_k l_k with w_k = 2^(m_k - max m).
 #include <cudaTypedefs.h>
 
+#include <cmath>
+
 #include "la_internal.cuh"
 #include "ptx.cuh"
 
@@ -52,6 +54,11 @@ constexpr int kSMs = 148;
 constexpr int BAR_MAX = 1, BAR_P = 2, BAR_PFREE = 4, BAR_QP = 6, BAR_END = 8;
 
 constexpr int align1k(int x) { return (x + 1023) / 1024 * 1024; }
+
+// RoPE frequencies theta_i = base^(-2i/d), formed in fp64 on the host
+struct RopeTheta {
+  double theta[64];
+};
 constexpr int imax(int a, int b) { return a > b ? a : b; }
 
 template <int D, int R, int NT>
@@ -80,9 +87,20 @@ struct Cfg {
 __device__ __forceinline__ float2 rope_cs_exact(int64_t t, double theta) {
   const double two_pi = 6.283185307179586476925286766559;
   const double ang = (double)t * theta;
-  const float red = (float)(ang - two_pi * rint(ang / two_pi));
+  const float red = (float)fma(-two_pi, rint(ang * 0.15915494309189533577), ang);
   float s, c;
   sincosf(red, &s, &c);
+  return make_float2(c, s);
+}
+
+// (cos, sin) of a small angle (|ang| < ~200 rad): Cody-Waite reduction with a
+// two-constant split of 2 pi, then the SFU (about 2^-21 absolute on [-pi, pi])
+__device__ __forceinline__ float2 sincos_small(float ang) {
+  const float k = rintf(ang * 0.15915494309189535f);
+  float red = fmaf(-k, 6.28318548202514648f, ang);
+  red = fmaf(-k, -1.7484556000744083e-07f, red);
+  float s, c;
+  __sincosf(red, &s, &c);
   return make_float2(c, s);
 }
 
@@ -111,7 +129,8 @@ template <int D, int R, int NT>
 __global__ void __launch_bounds__(NTHR, 1)
     decode_bf16_kernel(const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV,
-                       const __grid_constant__ CUtensorMap tmL, const AttnParams p) {
+                       const __grid_constant__ CUtensorMap tmL, const AttnParams p,
+                       const __grid_constant__ RopeTheta rt) {
   using C = Cfg<D, R, NT>;
   constexpr int W = C::W, ROWS = C::ROWS;
   extern __shared__ unsigned char smem_raw[];
@@ -222,7 +241,7 @@ __global__ void __launch_bounds__(NTHR, 1)
       }
       *reinterpret_cast<uint4*>(qs + tile_off<D, ROWS>(row, c * 8)) = v;
     }
-    if (tid < D / 2) theta[tid] = exp2(-2.0 * tid / D * log2(p.rope_base));
+    if (tid < D / 2) theta[tid] = rt.theta[tid];
   }
   __syncthreads();
   if (tid < D / 2) rotate_queries<D, ROWS>(qs_u, qp_u, theta, k_lo, p.s, tid);
@@ -241,7 +260,7 @@ __global__ void __launch_bounds__(NTHR, 1)
       for (int f = 0; f < 4; ++f) {
         const int i = 16 * grp + 8 * (f >> 1) + 2 * t4 + (f & 1);
 #pragma unroll
-        for (int kr = 0; kr < 2; ++kr) cj[grp][kr][f] = rope_cs_exact(16 * w + gq + 8 * kr, theta[i]);
+        for (int kr = 0; kr < 2; ++kr) cj[grp][kr][f] = sincos_small((float)(16 * w + gq + 8 * kr) * (float)rt.theta[i]);
       }
     float m_st[NT][2], l_st[NT][2];
 #pragma unroll
@@ -731,6 +750,8 @@ int n_splits_for(const AttnParams& p) {
 template <int D, int R, int NT>
 cudaError_t launch_t(const AttnParams& p, cudaStream_t st) {
   using C = Cfg<D, R, NT>;
+  RopeTheta rt;
+  for (int i = 0; i < 64; ++i) rt.theta[i] = i < D / 2 ? std::pow(p.rope_base, -2.0 * i / D) : 0.0;
   CUtensorMap mk, mv, ml;
   if (!make_maps(p, &mk, &mv, &ml)) return cudaErrorInvalidValue;
   const size_t sm = C::smem(p.n_agents);
@@ -738,7 +759,7 @@ cudaError_t launch_t(const AttnParams& p, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   dim3 grid(p.n_splits, p.n_seqs * p.n_kv);
-  kern<<<grid, NTHR, sm, st>>>(mk, mv, ml, p);
+  kern<<<grid, NTHR, sm, st>>>(mk, mv, ml, p, rt);
   e = cudaGetLastError();
   if (e != cudaSuccess || p.n_splits == 1) return e;
   // merge of the splits, launched early (programmatic dependent launch)
