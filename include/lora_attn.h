@@ -61,7 +61,8 @@ typedef enum {
   LA_ERR_CAPACITY = 3,     /* rows would land at or beyond L_max */
   LA_ERR_WORKSPACE = 4,    /* decode workspace missing or too small */
   LA_ERR_CUDA = 5,         /* a CUDA call or launch failed */
-  LA_ERR_DEVICE_CHECK = 6  /* a kernel's own bounds check fired (see la_device_check) */
+  LA_ERR_DEVICE_CHECK = 6, /* a kernel's own bounds check fired (see la_device_check) */
+  LA_ERR_SCRATCH_LIMIT = 7 /* decode scratch would exceed LA_STATIC_SCRATCH_BYTES */
 } la_status;
 
 typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
@@ -159,6 +160,34 @@ la_status lora_attn_decode(const la_attn_args* args, void* workspace, size_t wor
 
 /* Workspace bytes lora_attn_decode needs for these arguments (0 if invalid). */
 size_t lora_attn_decode_workspace_bytes(const la_attn_args* args);
+
+/*
+ * lora_attn_decode_static_scratch -- lora_attn_decode for callers that cannot
+ * give the library device memory.
+ *
+ * The pages have no counterpart to this entry point: it exists for callers
+ * that cannot allocate device memory.  Examples are a plugin running inside a
+ * serving runtime whose allocator owns every device allocation, and a process
+ * that sizes its device memory once at start-up.
+ *
+ * It computes exactly what lora_attn_decode computes, with the same arguments
+ * and errors, but it takes no workspace and allocates nothing.  The split-K
+ * scratch (per-split partials and arrival counters) lives in one device array
+ * of LA_STATIC_SCRATCH_BYTES that the library holds on every device that loads
+ * it, until the process exits.
+ *   - The first call on a device sets the array up: it looks up the array's
+ *     device address, clears it and synchronises that device.  Make that first
+ *     call before any stream capture.
+ *   - Every call shares the one array, which keeps what the last call left
+ *     in it; each call first clears, on `stream`, the part that must start at
+ *     zero.  Calls whose work overlaps on the GPU (other streams, other host
+ *     threads) race on the array: serialise them, e.g. on one stream.
+ *   - If these arguments need more scratch than LA_STATIC_SCRATCH_BYTES
+ *     (lora_attn_decode_workspace_bytes(args) > LA_STATIC_SCRATCH_BYTES), it
+ *     returns LA_ERR_SCRATCH_LIMIT before launching anything.
+ */
+#define LA_STATIC_SCRATCH_BYTES ((size_t)4 << 20)
+la_status lora_attn_decode_static_scratch(const la_attn_args* args, la_stream_t stream);
 
 /*
  * la_device_check -- synchronises the current device, then reads and clears

@@ -150,6 +150,8 @@ extern "C" const char* la_status_string(la_status s) {
     case LA_ERR_WORKSPACE: return "LA_ERR_WORKSPACE: workspace missing or too small";
     case LA_ERR_CUDA: return "LA_ERR_CUDA: CUDA call or launch failed";
     case LA_ERR_DEVICE_CHECK: return "LA_ERR_DEVICE_CHECK: a kernel bounds check fired";
+    case LA_ERR_SCRATCH_LIMIT:
+      return "LA_ERR_SCRATCH_LIMIT: decode scratch exceeds the library's static array";
   }
   return "unknown la_status";
 }
@@ -181,6 +183,19 @@ extern "C" la_status lr_cache_append(const void* X, int64_t ldx, int64_t n_token
                            seq_stride_x, seq_stride_lr, dt, st);
   return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
 }
+
+namespace la {
+// Byte range of the arrival counters inside a decode workspace for these
+// arguments (they must read zero when a decode starts).  False if invalid.
+bool decode_counter_range(const la_attn_args* a, size_t* offset, size_t* bytes) {
+  AttnParams p;
+  if (check_attn(a, 1, &p) != LA_OK) return false;
+  DecodePlan d = plan_decode(p, a->io_dtype);
+  *offset = d.partial_bytes;
+  *bytes = d.counter_bytes;
+  return true;
+}
+}  // namespace la
 
 extern "C" size_t lora_attn_decode_workspace_bytes(const la_attn_args* a) {
   AttnParams p;

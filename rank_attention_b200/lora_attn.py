@@ -19,11 +19,13 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "_lib", "liblora_attn.so")
 
 LA_OK, LA_ERR_INVALID_ARG, LA_ERR_UNSUPPORTED, LA_ERR_CAPACITY = 0, 1, 2, 3
-LA_ERR_WORKSPACE, LA_ERR_CUDA, LA_ERR_DEVICE_CHECK = 4, 5, 6
+LA_ERR_WORKSPACE, LA_ERR_CUDA, LA_ERR_DEVICE_CHECK, LA_ERR_SCRATCH_LIMIT = 4, 5, 6, 7
+LA_STATIC_SCRATCH_BYTES = 4 << 20
 LA_F32, LA_BF16 = 0, 1
 
 EXPORTED = ("la_status_string", "lr_cache_append", "lora_attn_prefill", "lora_attn_decode",
-            "lora_attn_decode_workspace_bytes", "la_device_check")
+            "lora_attn_decode_workspace_bytes", "la_device_check",
+            "lora_attn_decode_static_scratch")
 
 
 class LoraAttnError(RuntimeError):
@@ -77,6 +79,8 @@ def _load() -> ctypes.CDLL:
     lib.lora_attn_decode_workspace_bytes.argtypes = [ctypes.POINTER(AttnArgs)]
     lib.la_device_check.restype = ctypes.c_int
     lib.la_device_check.argtypes = []
+    lib.lora_attn_decode_static_scratch.restype = ctypes.c_int
+    lib.lora_attn_decode_static_scratch.argtypes = [ctypes.POINTER(AttnArgs), ctypes.c_void_p]
     return lib
 
 
@@ -173,6 +177,13 @@ def lora_attn_decode(args: AttnArgs, workspace: torch.Tensor, stream=None) -> No
     st = lib.lora_attn_decode(ctypes.byref(args), workspace.data_ptr(), workspace.numel(),
                               _stream(stream))
     _check(st, "lora_attn_decode")
+
+
+def lora_attn_decode_static_scratch(args: AttnArgs, stream=None) -> None:
+    """Decode without a workspace: the split scratch is the library's own device
+    array (for callers that cannot allocate device memory; see the header)."""
+    st = lib.lora_attn_decode_static_scratch(ctypes.byref(args), _stream(stream))
+    _check(st, "lora_attn_decode_static_scratch")
 
 
 def lora_attn_prefill(args: AttnArgs, stream=None) -> None:

@@ -22,6 +22,7 @@ FAKE = 0x10000  # 16-byte aligned, never dereferenced
 def declared_functions():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"#define.*", "", text)
     return sorted(set(re.findall(r"\b([a-z_][a-z0-9_]*)\s*\(", text)) -
                   {"sizeof", "defined"})
 
@@ -35,7 +36,7 @@ def test_every_declared_symbol_is_exported():
 
 
 def test_status_strings():
-    for s in range(7):
+    for s in range(8):
         assert la.status_string(s).startswith("LA_")
     assert "unknown" in la.status_string(99)
 

@@ -1,0 +1,89 @@
+"""lora_attn_decode_static_scratch: decode for callers that cannot allocate.
+
+A plugin inside a serving runtime whose allocator owns all device memory, or a
+process that fixes its device memory at start-up, cannot hand the library a
+workspace.  This entry point keeps the decode's split scratch in the library's
+own device array instead.  These tests call it through the C ABI and check that
+two calls in a row give what lora_attn_decode gives with a caller workspace.
+
+The file sorts last so that a run stopping at its first failure has already run
+every other test; it also passes on its own in a fresh process.
+"""
+import ctypes
+
+import pytest
+import torch
+
+from rank_attention_b200 import workloads as W
+from tests.helpers import assert_parity, to_np
+
+DEV = "cuda"
+FAKE = 0x10000  # 16-byte aligned, never dereferenced
+
+
+@pytest.fixture(scope="module")
+def la():
+    from rank_attention_b200 import lora_attn
+    return lora_attn
+
+
+def _compare(la, s, inp):
+    d = {k: v.to(DEV) for k, v in inp.items()}
+    out_ws = torch.empty(d["q"].shape, device=DEV)
+    args = la.make_args(d["k_base"], d["v_base"], d["lr"], d["B_k"], d["B_v"], d["q"], out_ws,
+                        lora_scale=s.lora_scale, rope_base=s.rope_base, kv_len=d["kv_len"],
+                        max_kv_len=int(inp["kv_len"].max()))
+    need = la.lora_attn_decode_workspace_bytes(args)
+    assert 0 < need <= la.LA_STATIC_SCRATCH_BYTES
+    la.lora_attn_decode(args, la.decode_workspace(args, DEV))
+    torch.cuda.synchronize()
+    ref = out_ws.cpu()
+    for _ in range(2):  # two calls in a row share (and reuse) the static scratch
+        out = torch.full(d["q"].shape, float("nan"), device=DEV)
+        a2 = la.make_args(d["k_base"], d["v_base"], d["lr"], d["B_k"], d["B_v"], d["q"], out,
+                          lora_scale=s.lora_scale, rope_base=s.rope_base, kv_len=d["kv_len"],
+                          max_kv_len=int(inp["kv_len"].max()))
+        st = la.lib.lora_attn_decode_static_scratch(ctypes.byref(a2),
+                                                    torch.cuda.current_stream().cuda_stream)
+        assert st == la.LA_OK, la.status_string(st)
+        torch.cuda.synchronize()
+        assert la.la_device_check() == la.LA_OK
+        assert_parity(to_np(out), to_np(ref), s.dtype)
+
+
+@pytest.mark.gpu
+def test_static_scratch_matches_workspace_decode_bf16(la):
+    """The LLaMA-shaped 8192-token decode (tensor-core kernel, split over the keys)."""
+    s = W.LLAMA8B_DECODE_8K
+    _compare(la, s, W.direct_cache_inputs(s))
+
+
+@pytest.mark.gpu
+def test_static_scratch_matches_workspace_decode_fp32(la):
+    """The fp32 generic kernel, whose split merge also uses arrival counters."""
+    s = W.TINY_FP32
+    inp = W.direct_cache_inputs(s.replace(dtype=torch.float32))
+    _compare(la, s, inp)
+
+
+def test_static_scratch_rejects_oversized_request(la):
+    """Arguments needing more scratch than the array are refused before any
+    launch (the fake pointers are never touched)."""
+    a = la.AttnArgs()
+    a.n_seqs, a.n_agents, a.n_q_heads, a.n_kv_heads, a.head_dim, a.r = 1, 16, 4, 1, 128, 64
+    a.lora_scale, a.softmax_scale, a.rope_base = 2.0, 0.088, 10000.0
+    a.L_max = 1 << 20
+    a.k_base = a.v_base = a.lr_cache = a.B_k = a.B_v = a.q = a.out = a.kv_len = FAKE
+    a.kv_seq_stride, a.kv_head_stride, a.kv_tok_stride = (1 << 20) * 128, (1 << 20) * 128, 128
+    a.lr_seq_stride = (1 << 20) * 128
+    a.max_kv_len = 1 << 20
+    a.n_q_tokens = 1
+    a.io_dtype = a.out_dtype = la.LA_F32
+    assert la.lora_attn_decode_workspace_bytes(a) > la.LA_STATIC_SCRATCH_BYTES
+    st = la.lib.lora_attn_decode_static_scratch(ctypes.byref(a), None)
+    assert st == la.LA_ERR_SCRATCH_LIMIT
+    assert "LA_ERR_SCRATCH_LIMIT" in la.status_string(st)
+    bad = la.AttnArgs()
+    ctypes.memmove(ctypes.byref(bad), ctypes.byref(a), ctypes.sizeof(a))
+    bad.head_dim = 96
+    assert la.lib.lora_attn_decode_static_scratch(ctypes.byref(bad), None) == la.LA_ERR_UNSUPPORTED
