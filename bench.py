@@ -116,10 +116,12 @@ def decode_source_sha() -> str:
 
 
 def decode_kernels_per_call(s) -> int:
-    """Kernels one lora_attn_decode call launches for this workload: the decode
-    kernel, plus the split-merge kernel when the keys are split over CTAs (the
-    library splits each (sequence, KV head) over min(32, 148 // units, tiles of
-    128 keys) CTAs)."""
+    """Kernels one lora_attn_decode call launches for this workload.  The
+    tensor-core decode (d = 128, r in {16, 32, 64}, at most three agents) merges
+    its key splits inside the same launch: one kernel.  The other bf16 shapes
+    add a split-merge kernel when the keys are split over CTAs."""
+    if s.head_dim == 128 and s.r in (16, 32, 64) and s.n_agents <= 3:
+        return 1
     units = s.n_seqs * s.n_kv_heads
     splits = 1 if units >= 148 else min(32, 148 // units, (s.kv_len + 127) // 128)
     return 2 if splits > 1 else 1

@@ -144,7 +144,12 @@ la_status lora_attn_prefill(const la_attn_args* args, la_stream_t stream);
 
 /*
  * lora_attn_decode -- one query token per (sequence, agent), split over the
- * sequence (split-K) with the partial results merged inside the same launch.
+ * sequence (split-K).  On the tensor-core path (bf16, head_dim 128, r in
+ * {16, 32, 64}, at most three agents) the partial results are merged inside
+ * the same launch: that launch is cooperative (every CTA resident at once,
+ * at most one per SM), so it fails with LA_ERR_CUDA on a device whose SMs
+ * are partly taken by a context limit.  Other shapes merge in the same
+ * launch (fp32) or in a second kernel (bf16).
  *
  * workspace: device memory of at least lora_attn_decode_workspace_bytes(args)
  * bytes, 256-byte aligned, ZERO-FILLED BEFORE ITS FIRST USE.  Each call

@@ -132,7 +132,8 @@ DecodePlan plan_decode(const AttnParams& p, la_dtype io) {
   else
     d.partial_bytes = d.n_splits > 1 ? (size_t)units * d.n_splits * d.rows * W * sizeof(float) : 0;
   d.partial_bytes = (d.partial_bytes + 255) / 256 * 256;
-  d.counter_bytes = ((size_t)units * sizeof(int) + 255) / 256 * 256;
+  // per unit: an arrival and a departure counter of the split merge
+  d.counter_bytes = ((size_t)2 * units * sizeof(int) + 255) / 256 * 256;
   return d;
 }
 

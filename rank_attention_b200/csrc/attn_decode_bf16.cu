@@ -34,6 +34,8 @@
 
 #include <cmath>
 
+#include <cuda_fp16.h>
+
 #include "la_internal.cuh"
 #include "ptx.cuh"
 
@@ -647,35 +649,833 @@ __global__ void __launch_bounds__(NTHR, 1)
 }
 
 // Merge of a unit's splits: one CTA per (row, unit), one thread per column.
-// out = sum_k 2^(m_k - M) Z_k / sum_k 2^(m_k - M) l_k, M = max_k m_k.
+// out = sum_k 2^(m_k - M) Z_k / sum_k 2^(m_k - M) l_k, M = max_k m_k.  The
+// split weights are formed once per CTA; every thread then issues its column's
+// loads of all splits before using them, so the merge costs a couple of L2
+// round trips, not one per split.
 template <int D>
 __global__ void __launch_bounds__(D) decode_merge_kernel(const AttnParams p) {
-  pdl_wait();  // the partials of the preceding decode grid are complete and visible
   constexpr int WP = D + 4;
+  __shared__ float wts[kMaxSplits];
   const int row = blockIdx.x, unit = blockIdx.y, c = threadIdx.x;
-  {
-    const int64_t kvl = p.kv_len[unit / p.n_kv];
-    if (kvl < 1 || kvl > p.max_kv_len) return;  // reported by the decode grid
-  }
+  const int64_t kvl = p.kv_len[unit / p.n_kv];  // an input: read before the wait
+  pdl_wait();  // the partials of the preceding decode grid are complete and visible
+  if (kvl < 1 || kvl > p.max_kv_len) return;  // reported by the decode grid
   const int ns = p.n_splits, n_rows = p.n_agents * p.g;
   const float* base = p.partials + (size_t)unit * ns * n_rows * WP + (size_t)row * WP;
   const size_t kstr = (size_t)n_rows * WP;
-  float mx = -INFINITY;
-  for (int k = 0; k < ns; ++k) mx = fmaxf(mx, __ldcg(base + k * kstr + D));
-  float l = 0.f, acc = 0.f;
-#pragma unroll 4
-  for (int k = 0; k < ns; ++k) {
-    const float mk = __ldcg(base + k * kstr + D);
-    const float wk = mk == -INFINITY ? 0.f : exp2f(mk - mx);
-    l = fmaf(wk, __ldcg(base + k * kstr + D + 1), l);
-    acc = fmaf(wk, __ldcg(base + k * kstr + c), acc);
+  // every load of this thread is issued before any of them is used
+  float z[kMaxSplits];
+#pragma unroll
+  for (int k = 0; k < kMaxSplits; ++k) z[k] = k < ns ? __ldcg(base + k * kstr + c) : 0.f;
+  float2 ml = make_float2(-INFINITY, 0.f);
+  if (c < ns) ml = __ldcg(reinterpret_cast<const float2*>(base + c * kstr + D));
+  if (c < 32) {
+    float mx = ml.x;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const float wk = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - mx);
+    float l = wk * ml.y;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    if (c < ns) wts[c] = l > 0.f ? wk / l : 0.f;
   }
+  __syncthreads();
+  float acc = 0.f;
+#pragma unroll
+  for (int k = 0; k < kMaxSplits; ++k)
+    if (k < ns) acc = fmaf(wts[k], z[k], acc);
   const int seq = unit / p.n_kv, kvh = unit % p.n_kv;
   const int a = row / p.g, gi = row % p.g;
   const int64_t oi = (((int64_t)seq * p.n_agents + a) * p.n_q + kvh * p.g + gi) * D + c;
-  const float val = l > 0.f ? acc / l : 0.f;
-  if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(val);
-  else reinterpret_cast<float*>(p.out)[oi] = val;
+  if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(acc);
+  else reinterpret_cast<float*>(p.out)[oi] = acc;
+}
+
+// ============================================================================
+// Decode with the 5th-generation tensor cores (tcgen05 / TMEM).
+//
+// The agent-shared GEMMs of a 128-key tile run as single-thread-issued
+// tcgen05 MMAs (M = 128 keys) whose operands are read from shared memory once
+// per CTA: the base scores S_base^T = K_base Q^T (N = the query rows, padded to
+// 16 / 32) and every agent's key delta dK^a = LRk B_k^a (N = d, K = r), all
+// accumulated in TMEM.  Eight score warps -- two per 32-lane TMEM
+// sub-partition, 16 keys each -- read dK^a straight into the mma.sync
+// accumulator layout (tcgen05.ld 16x256b), turn it by R(j), and score it
+// against the tile's rotated queries; the rest (softmax, value side, merge) is
+// as in the kernel above.  Warp 10 stages B_k and the tiles (TMA) and issues
+// the MMAs.
+// ============================================================================
+constexpr int TC_NES = 8;                          // score warps (16 keys each)
+constexpr int TC_NTHR = 32 * (TC_NES + NPV + 1);   // + value warps + TMA / MMA warp
+constexpr int TC_COLS = 512;                        // TMEM columns allocated
+constexpr int TC_SCOL = 384;                        // TMEM column of S_base
+
+template <int D, int R, int NT>
+struct TCfg {
+  static constexpr int ROWS = NT * 8;
+  static constexpr int QPAD = NT <= 2 ? 16 : 32;        // N of the base-score MMA
+  static constexpr int W = D + R + 4;
+  static constexpr int KV_TILE = KT * D * 2;
+  static constexpr int LR_TILE = align1k(KT * 2 * R * 2);
+  static constexpr int STAGE = 2 * KV_TILE + LR_TILE;
+  static constexpr int AREA = imax(ST * STAGE, align1k(ROWS * W * 4));
+  static constexpr int P_TILE = align1k(ROWS * KT * 2);
+  static constexpr int SMALL = 2 * TC_NES * ROWS * 4 + 2 * ROWS * 4 + TC_NES * ROWS * 4 + 64 * 8 + 16 + 64 * 8;
+  static constexpr int QU_BYTES = align1k(QPAD * D * 2);   // Q as the MMA operand
+  static constexpr int QP_BYTES = align1k(ROWS * D * 2);   // each Q' buffer
+  static constexpr int BK_BYTES = R * D * 2;
+  static constexpr int KS = R / 16;
+  static constexpr int MR = R / 16;
+  static constexpr int NG = D / 32;
+  static constexpr int MT = D / 2 / 16;
+  // LR tile: rows of 2r bf16 in boxes of min(2r, 64); its swizzle span
+  static constexpr int LR_ROWB = (2 * R < 64 ? 2 * R : 64) * 2;
+  static constexpr uint32_t LR_LAYOUT = LR_ROWB == 128 ? 2u : (LR_ROWB == 64 ? 4u : 6u);
+  static size_t smem(int n_agents) {
+    return 1024 + AREA + 2 * P_TILE + align1k(SMALL) + QU_BYTES + 2 * QP_BYTES +
+           (size_t)align1k(BK_BYTES) * n_agents + (size_t)BK_BYTES * n_agents + 128;
+  }
+};
+
+template <int D, int SRC_ROWS, int DST_ROWS>
+__device__ __forceinline__ void rotate_queries_tc(uint32_t qs_u, uint32_t qp_u, const double* theta,
+                                                  int64_t t, float s, int i) {
+  const float2 cs = rope_cs_exact(t, theta[i]);
+  const float c = cs.x * s, sn = cs.y * s;
+#pragma unroll 4
+  for (int row = 0; row < DST_ROWS; ++row) {
+    uint16_t a, b;
+    asm volatile("ld.shared.b16 %0, [%1];" : "=h"(a) : "r"(qs_u + tile_off<D, SRC_ROWS>(row, i)));
+    asm volatile("ld.shared.b16 %0, [%1];" : "=h"(b) : "r"(qs_u + tile_off<D, SRC_ROWS>(row, i + D / 2)));
+    const float x1 = __uint_as_float((uint32_t)a << 16), x2 = __uint_as_float((uint32_t)b << 16);
+    const __nv_bfloat16 y1 = __float2bfloat16_rn(fmaf(x1, c, x2 * sn));
+    const __nv_bfloat16 y2 = __float2bfloat16_rn(fmaf(x2, c, -x1 * sn));
+    sts16(qp_u + tile_off<D, DST_ROWS>(row, i), *reinterpret_cast<const uint16_t*>(&y1));
+    sts16(qp_u + tile_off<D, DST_ROWS>(row, i + D / 2), *reinterpret_cast<const uint16_t*>(&y2));
+  }
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float2 v) {
+  __half2 h = __floats2half2_rn(v.x, v.y);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ float2 unpack_half2(uint32_t v) {
+  return __half22float2(*reinterpret_cast<const __half2*>(&v));
+}
+
+template <int D, int R, int NT>
+__global__ void __launch_bounds__(TC_NTHR, 1)
+    decode_tc_kernel(const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV,
+                     const __grid_constant__ CUtensorMap tmL,
+                     const __grid_constant__ CUtensorMap tmB, const AttnParams p,
+                     const __grid_constant__ RopeTheta rt) {
+  using C = TCfg<D, R, NT>;
+  constexpr int W = C::W, ROWS = C::ROWS, QPAD = C::QPAD;
+  constexpr int NB = 32 * (TC_NES + NPV);   // threads in the score / value barriers
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* area = smem;
+  unsigned char* ptile = area + C::AREA;
+  float* Mx = reinterpret_cast<float*>(ptile + 2 * C::P_TILE);   // [2][NES][ROWS]
+  float* Corr = Mx + 2 * TC_NES * ROWS;                          // [2][ROWS]
+  float* Lw = Corr + 2 * ROWS;                                   // [NES][ROWS]
+  double* theta = reinterpret_cast<double*>(Lw + TC_NES * ROWS); // [64]
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(theta + 64);
+  float2* cs0 = reinterpret_cast<float2*>(tslot + 4);             // [64] s (cos, sin)(k_lo theta_i)
+  unsigned char* qu = ptile + 2 * C::P_TILE + align1k(C::SMALL);  // Q (MMA operand)
+  unsigned char* qpb0 = qu + C::QU_BYTES;                          // Q'[2]
+  unsigned char* bks = qpb0 + 2 * C::QP_BYTES;
+  unsigned char* bvs = bks + (size_t)align1k(C::BK_BYTES) * p.n_agents;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(bvs + (size_t)C::BK_BYTES * p.n_agents);
+  __shared__ int s_fail;
+
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int gq = lane >> 2, t4 = lane & 3;
+  const int mi = lane >> 3, rr = lane & 7;
+  const int unit = blockIdx.y;
+  const int seq = unit / p.n_kv, kvh = unit % p.n_kv;
+  const int split = blockIdx.x;
+  const int ns = p.n_splits;
+  const int g = p.g, na = p.n_agents, n_rows = na * g;
+
+  const int64_t total_tiles = (p.max_kv_len + KT - 1) / KT;
+  const int64_t tb = split * total_tiles / ns;
+  const int64_t te = (split + 1) * total_tiles / ns;
+  const int64_t k_lo = tb * KT;
+
+  const uint32_t area_u = smem_u32(area);
+  const uint32_t ptile_u = smem_u32(ptile);
+  const uint32_t qu_u = smem_u32(qu);
+  const uint32_t qp_u = smem_u32(qpb0);
+  const uint32_t bks_u = smem_u32(bks);
+  const uint32_t bvs_u = smem_u32(bvs);
+  const uint32_t full_u = smem_u32(bars);          // [ST]
+  const uint32_t empty_u = full_u + 8 * ST;        // [ST]: MMA commit + value warps
+  const uint32_t tfull = full_u + 16 * ST;         // MMA results of a tile are in TMEM
+  const uint32_t tempty = tfull + 8;               // score warps are done reading TMEM
+  const uint32_t bvbar = tfull + 16;
+  const uint32_t bkbar = tfull + 24;              // B_k^a slices have landed
+  const uint32_t qbar = tfull + 32;               // the queries have landed (staged unswizzled)
+  const int64_t ldB = (int64_t)p.n_kv * D;
+
+  auto issue = [&](int n) {  // TMA of tile n into stage n % ST (one thread)
+    const int s = n % ST;
+    const uint32_t sb = area_u + s * C::STAGE;
+    const uint32_t bar = full_u + 8 * s;
+    const int key0 = (int)(k_lo + (int64_t)n * KT);
+    mbar_expect_tx(bar, 2 * C::KV_TILE + KT * 2 * R * 2);
+#pragma unroll
+    for (int b = 0; b < D / 64; ++b) {
+      tma_load_4d(sb + b * KT * 128, &tmK, bar, 64 * b, key0, kvh, seq);
+      tma_load_4d(sb + C::KV_TILE + b * KT * 128, &tmV, bar, 64 * b, key0, kvh, seq);
+    }
+    constexpr int LB = (2 * R) < 64 ? 2 * R : 64;
+#pragma unroll
+    for (int b = 0; b < (2 * R) / LB; ++b)
+      tma_load_3d(sb + 2 * C::KV_TILE + b * KT * LB * 2, &tmL, bar, LB * b, key0, seq);
+  };
+
+  // ---- first loads (independent of kv_len): queries, B_k^a, the first tiles, B_v^a
+  const int n_spec = (int)min((int64_t)ST, te - tb);
+  if (w == TC_NES + NPV && lane == 0) {
+    s_fail = 0;
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(full_u + 8 * s, 1);
+      mbar_init(empty_u + 8 * s, 1 + NPV);
+    }
+    mbar_init(tfull, 1);
+    mbar_init(tempty, TC_NES);
+    mbar_init(bvbar, 1);
+    mbar_init(bkbar, 1);
+    mbar_init(qbar, 1);
+    fence_mbar_init();
+    // each agent's g query rows of this KV head are contiguous
+    const __nv_bfloat16* Q = reinterpret_cast<const __nv_bfloat16*>(p.q);
+    mbar_expect_tx(qbar, (uint32_t)(n_rows * D * 2));
+    for (int a = 0; a < na; ++a)
+      bulk_load(ptile_u + a * g * D * 2, Q + (((int64_t)seq * na + a) * p.n_q + kvh * g) * D,
+                (uint32_t)(g * D * 2), qbar);
+    tma_prefetch(&tmB);
+    tma_prefetch(&tmK);
+    tma_prefetch(&tmV);
+    tma_prefetch(&tmL);
+    // B_k^a head slices (r rows x 64 d boxes, the MN-major MMA operand)
+    mbar_expect_tx(bkbar, (uint32_t)(na * C::BK_BYTES));
+    for (int a = 0; a < na; ++a)
+#pragma unroll
+      for (int b = 0; b < D / 64; ++b)
+        tma_load_3d(bks_u + a * align1k(C::BK_BYTES) + b * R * 128, &tmB, bkbar, kvh * D + 64 * b, 0, a);
+    // the first stages before kv_len is known: tiles of this split's range
+    // (by max_kv_len) past the sequence's length are loaded but never used
+    for (int n = 0; n < n_spec; ++n) issue(n);
+    const __nv_bfloat16* Bv = reinterpret_cast<const __nv_bfloat16*>(p.B_v);
+    mbar_expect_tx(bvbar, (uint32_t)(na * C::BK_BYTES));
+    for (int i = 0; i < na * R; ++i)
+      bulk_load(bvs_u + i * D * 2, Bv + (int64_t)i * ldB + kvh * D, D * 2, bvbar);
+  }
+  const int64_t kvl = p.kv_len[seq];
+  if (kvl < 1 || kvl > p.max_kv_len) {
+    if (tid == 0 && split == 0) atomicOr(p.err, 1);
+    if (w == TC_NES + NPV && lane == 0) {  // the copies in flight land before the CTA leaves
+      mbar_wait(qbar, 0);
+      mbar_wait(bkbar, 0);
+      mbar_wait(bvbar, 0);
+      for (int n = 0; n < n_spec; ++n) mbar_wait(full_u + 8 * n, 0);
+    }
+    return;
+  }
+  const int64_t k_hi = min(te * KT, kvl);
+  const int n_tiles = k_hi > k_lo ? (int)((k_hi - k_lo + KT - 1) / KT) : 0;
+  if (w == TC_NES + NPV) tmem_alloc(smem_u32(tslot), TC_COLS);
+
+  int fail = 0;
+  // ---- per-CTA constants: Q (the base-score MMA operand), frequencies, and the
+  // score warps' in-tile rotations R(j) while the first loads are in flight
+  const int sp = w & 3, kb = 32 * sp + 16 * (w >> 2);  // score warp: TMEM sub-partition, first key
+  uint32_t cjh[C::NG][2][4];
+  if (w < TC_NES) {
+    // R(j) for this thread's keys j = kb + gq (+8) and its 16 frequencies (f16 pairs)
+#pragma unroll
+    for (int grp = 0; grp < C::NG; ++grp)
+#pragma unroll
+      for (int f = 0; f < 4; ++f) {
+        const int i = 16 * grp + 8 * (f >> 1) + 2 * t4 + (f & 1);
+        const float th = (float)rt.theta[i];
+#pragma unroll
+        for (int kr = 0; kr < 2; ++kr)
+          cjh[grp][kr][f] = pack_half2(sincos_small((float)(kb + gq + 8 * kr) * th));
+      }
+  }
+  if (tid < D / 2) theta[tid] = rt.theta[tid];
+  if (w >= TC_NES && w < TC_NES + NPV) {
+    // the first tile's query rotation R(-k_lo), scaled by s (exact in fp64)
+    for (int i = tid - 32 * TC_NES; i < D / 2; i += 32 * NPV) {
+      const float2 cs = rope_cs_exact(k_lo, rt.theta[i]);
+      cs0[i] = make_float2(cs.x * p.s, cs.y * p.s);
+    }
+  }
+  __syncthreads();  // barriers initialised, cs0 ready
+  if (!mbar_wait(qbar, 0)) fail = 1;
+  // Q (swizzled: the base-score MMA operand) and Q' = s R(-k_lo) Q for the first tile
+  for (int i = tid; i < QPAD * (D / 16); i += TC_NTHR) {
+    const int row = i / (D / 16), c = i % (D / 16);
+    uint4 v1 = make_uint4(0, 0, 0, 0), v2 = v1;
+    if (row < n_rows) {
+      v1 = *reinterpret_cast<const uint4*>(ptile + (size_t)row * D * 2 + c * 16);
+      v2 = *reinterpret_cast<const uint4*>(ptile + (size_t)row * D * 2 + D + c * 16);
+    }
+    *reinterpret_cast<uint4*>(qu + tile_off<D, QPAD>(row, c * 8)) = v1;
+    *reinterpret_cast<uint4*>(qu + tile_off<D, QPAD>(row, c * 8 + D / 2)) = v2;
+    if (row < ROWS) {
+      const uint32_t* x1 = reinterpret_cast<const uint32_t*>(&v1);
+      const uint32_t* x2 = reinterpret_cast<const uint32_t*>(&v2);
+      uint4 y1, y2;
+      uint32_t* o1 = reinterpret_cast<uint32_t*>(&y1);
+      uint32_t* o2 = reinterpret_cast<uint32_t*>(&y2);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 a = unpack_bf16(x1[e]), b = unpack_bf16(x2[e]);
+        const float2 c0 = cs0[8 * c + 2 * e], c1 = cs0[8 * c + 2 * e + 1];
+        o1[e] = pack_bf16(fmaf(a.x, c0.x, b.x * c0.y), fmaf(a.y, c1.x, b.y * c1.y));
+        o2[e] = pack_bf16(fmaf(b.x, c0.x, -a.x * c0.y), fmaf(b.y, c1.x, -a.y * c1.y));
+      }
+      *reinterpret_cast<uint4*>(qpb0 + tile_off<D, ROWS>(row, c * 8)) = y1;
+      *reinterpret_cast<uint4*>(qpb0 + tile_off<D, ROWS>(row, c * 8 + D / 2)) = y2;
+    }
+  }
+  fence_proxy_async_smem();  // the MMA reads Q through the async proxy
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+
+  const float sl2 = p.scale * kLog2e;
+
+  if (w < TC_NES) {
+    // ======================================================== score warps
+    float m_st[NT][2], l_st[NT][2];
+#pragma unroll
+    for (int pt = 0; pt < NT; ++pt) {
+      m_st[pt][0] = m_st[pt][1] = -INFINITY;
+      l_st[pt][0] = l_st[pt][1] = 0.f;
+    }
+    const uint32_t tl = tmem + ((uint32_t)kb << 16);
+    // per agent: the n-tile holding its query rows, and whether this lane's row is one of them
+    int pa_of[3];
+    bool mine[3];
+#pragma unroll
+    for (int a = 0; a < 3; ++a) {
+      pa_of[a] = (a * g) >> 3;
+      mine[a] = (8 * pa_of[a] + gq) / g == a;
+    }
+    for (int n = 0; n < n_tiles; ++n) {
+      const int pb = n & 1;
+      const uint32_t qpb = qp_u + pb * C::QP_BYTES;
+      const int64_t k0 = k_lo + (int64_t)n * KT;
+      const int64_t kw0 = k0 + kb;
+      if (!mbar_wait(tfull, n & 1)) fail = 1;
+      tc_fence_after();
+      bar_sync(BAR_QP + pb, NB);
+
+      float S[NT][4];
+      {
+        uint32_t r4[NT][4];
+#pragma unroll
+        for (int pt = 0; pt < NT; ++pt) tmem_ld16x256_x1(r4[pt], tl + TC_SCOL + 8 * pt);
+        tmem_wait_ld();
+#pragma unroll
+        for (int pt = 0; pt < NT; ++pt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) S[pt][e] = __uint_as_float(r4[pt][e]);
+      }
+      if (kw0 < k_hi) {
+        // agents outer, column groups inner; the TMEM load of the next (agent,
+        // group) is in flight while the current one is turned and scored
+        uint32_t xl[2][8], xh[2][8];   // delta columns i and i + d/2 of a group
+        tmem_ld16x256_x2(xl[0], tl);
+        tmem_ld16x256_x2(xh[0], tl + D / 2);
+        for (int a = 0; a < na; ++a) {
+          const int pa = a == 0 ? pa_of[0] : (a == 1 ? pa_of[1] : pa_of[2]);
+          const bool mn = a == 0 ? mine[0] : (a == 1 ? mine[1] : mine[2]);
+#pragma unroll
+          for (int grp = 0; grp < C::NG; ++grp) {
+            const int cb = grp & 1, nb = cb ^ 1;
+            tmem_wait_ld_regs(xl[cb], xh[cb]);
+            if (grp + 1 < C::NG) {
+              const uint32_t ta = tl + 128 * a + 16 * (grp + 1);
+              tmem_ld16x256_x2(xl[nb], ta);
+              tmem_ld16x256_x2(xh[nb], ta + D / 2);
+            } else if (a + 1 < na) {
+              const uint32_t ta = tl + 128 * (a + 1);
+              tmem_ld16x256_x2(xl[nb], ta);
+              tmem_ld16x256_x2(xh[nb], ta + D / 2);
+            }
+            uint32_t A_lo[4], A_hi[4];
+#pragma unroll
+            for (int q = 0; q < 2; ++q)
+#pragma unroll
+              for (int hh = 0; hh < 2; ++hh) {
+                // R(j) of key row hh at the adjacent frequencies (2 t4, 2 t4 + 1) + 8 q
+                const float2 u = unpack_half2(cjh[grp][hh][2 * q]);
+                const float2 v = unpack_half2(cjh[grp][hh][2 * q + 1]);
+                const uint64_t cc = f2(u.x, v.x), ss = f2(u.y, v.y), nn = f2(-u.y, -v.y);
+                const uint64_t x1 = f2(__uint_as_float(xl[cb][4 * q + 2 * hh]), __uint_as_float(xl[cb][4 * q + 2 * hh + 1]));
+                const uint64_t x2 = f2(__uint_as_float(xh[cb][4 * q + 2 * hh]), __uint_as_float(xh[cb][4 * q + 2 * hh + 1]));
+                const float2 l2 = f2_unpack(fma_f2(x1, cc, mul_f2(x2, nn)));
+                const float2 h2 = f2_unpack(fma_f2(x2, cc, mul_f2(x1, ss)));
+                A_lo[2 * q + hh] = pack_bf16(l2.x, l2.y);
+                A_hi[2 * q + hh] = pack_bf16(h2.x, h2.y);
+              }
+            uint32_t bq[4];
+            ldsm_x4(bq, qpb + tile_off<D, ROWS>(8 * pa + rr, 16 * grp + (mi & 1) * 8 + (mi >> 1) * (D / 2)));
+            if (!mn) bq[0] = bq[1] = bq[2] = bq[3] = 0u;
+#pragma unroll
+            for (int pt = 0; pt < NT; ++pt)
+              if (pt == pa) {
+                mma16816(S[pt], A_lo, bq[0], bq[1]);
+                mma16816(S[pt], A_hi, bq[2], bq[3]);
+              }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty);  // TMEM of this tile may be overwritten
+
+      // tile row maxima over all score warps
+      const bool v0 = kw0 + gq < k_hi, v1 = kw0 + gq + 8 < k_hi;
+      float x[NT][4];
+      float* mxw = Mx + (pb * TC_NES + w) * ROWS;
+#pragma unroll
+      for (int pt = 0; pt < NT; ++pt) {
+        x[pt][0] = v0 ? S[pt][0] * sl2 : -INFINITY;
+        x[pt][1] = v0 ? S[pt][1] * sl2 : -INFINITY;
+        x[pt][2] = v1 ? S[pt][2] * sl2 : -INFINITY;
+        x[pt][3] = v1 ? S[pt][3] * sl2 : -INFINITY;
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          float mt_ = fmaxf(x[pt][e], x[pt][e + 2]);
+          mt_ = fmaxf(mt_, __shfl_xor_sync(0xffffffffu, mt_, 4));
+          mt_ = fmaxf(mt_, __shfl_xor_sync(0xffffffffu, mt_, 8));
+          mt_ = fmaxf(mt_, __shfl_xor_sync(0xffffffffu, mt_, 16));
+          if (gq == 0) mxw[8 * pt + 2 * t4 + e] = mt_;
+        }
+      }
+      bar_sync(BAR_MAX, 32 * TC_NES);
+#pragma unroll
+      for (int pt = 0; pt < NT; ++pt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int row = 8 * pt + 2 * t4 + e;
+          float mt_ = -INFINITY;
+#pragma unroll
+          for (int ww = 0; ww < TC_NES; ++ww) mt_ = fmaxf(mt_, Mx[(pb * TC_NES + ww) * ROWS + row]);
+          const float mo = m_st[pt][e];
+          const float mn = fmaxf(mo, mt_);
+          const float corr = (mo == -INFINITY) ? 0.f : fast_exp2(mo - mn);
+          const float p0 = (mn == -INFINITY) ? 0.f : fast_exp2(x[pt][e] - mn);
+          const float p1 = (mn == -INFINITY) ? 0.f : fast_exp2(x[pt][e + 2] - mn);
+          x[pt][e] = p0;
+          x[pt][e + 2] = p1;
+          l_st[pt][e] = l_st[pt][e] * corr + p0 + p1;
+          m_st[pt][e] = mn;
+          if (w == 0 && gq == 0) Corr[pb * ROWS + row] = corr;
+        }
+      bar_sync(BAR_PFREE + pb, NB);
+      const uint32_t pt_u = ptile_u + pb * C::P_TILE;
+#pragma unroll
+      for (int pt = 0; pt < NT; ++pt) {
+        const uint32_t b0 = movmatrix_t(pack_bf16(x[pt][0], x[pt][1]));
+        const uint32_t b1 = movmatrix_t(pack_bf16(x[pt][2], x[pt][3]));
+        sts32(pt_u + tile_off<KT, ROWS>(8 * pt + gq, kb + 2 * t4), b0);
+        sts32(pt_u + tile_off<KT, ROWS>(8 * pt + gq, kb + 8 + 2 * t4), b1);
+      }
+      bar_arrive(BAR_P + pb, NB);
+    }
+#pragma unroll
+    for (int pt = 0; pt < NT; ++pt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        float l = l_st[pt][e];
+        l += __shfl_xor_sync(0xffffffffu, l, 4);
+        l += __shfl_xor_sync(0xffffffffu, l, 8);
+        l += __shfl_xor_sync(0xffffffffu, l, 16);
+        if (gq == 0) Lw[w * ROWS + 8 * pt + 2 * t4 + e] = l;
+      }
+    tc_fence_before();
+    bar_sync(BAR_END, TC_NTHR);
+    float* Mo = reinterpret_cast<float*>(area);
+    if (w == 0 && gq == 0) {
+#pragma unroll
+      for (int pt = 0; pt < NT; ++pt)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) Mo[(8 * pt + 2 * t4 + e) * W + D + R] = m_st[pt][e];
+    }
+  } else if (w < TC_NES + NPV) {
+    // ======================================================== value warps
+    const int pv = w - TC_NES;
+    float O[C::MT][NT][4];
+    float Olr[C::MR][NT][4];
+#pragma unroll
+    for (int mt = 0; mt < C::MT; ++mt)
+#pragma unroll
+      for (int pt = 0; pt < NT; ++pt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) O[mt][pt][e] = 0.f;
+#pragma unroll
+    for (int mr = 0; mr < C::MR; ++mr)
+#pragma unroll
+      for (int pt = 0; pt < NT; ++pt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) Olr[mr][pt][e] = 0.f;
+    if (n_tiles > 0) {
+      bar_arrive(BAR_QP + 0, NB);
+      bar_arrive(BAR_PFREE + 0, NB);
+    }
+    if (n_tiles > 1) bar_arrive(BAR_PFREE + 1, NB);
+    const int d0 = pv * (D / 2);
+    for (int n = 0; n < n_tiles; ++n) {
+      const int s = n % ST, pb = n & 1;
+      const uint32_t sV = area_u + s * C::STAGE + C::KV_TILE;
+      const uint32_t sL = area_u + s * C::STAGE + 2 * C::KV_TILE;
+      const int64_t k0 = k_lo + (int64_t)n * KT;
+      if (n + 1 < n_tiles) {
+        const int i = pv * 32 + lane;
+        if (i < D / 2)
+          rotate_queries_tc<D, QPAD, ROWS>(qu_u, qp_u + ((n + 1) & 1) * C::QP_BYTES, theta, k0 + KT, p.s, i);
+        bar_arrive(BAR_QP + ((n + 1) & 1), NB);
+      }
+      if (!mbar_wait(full_u + 8 * s, (n / ST) & 1)) fail = 1;
+      if (k0 + KT > k_hi) {
+        unsigned char* vb = area + s * C::STAGE + C::KV_TILE;
+        unsigned char* lb = area + s * C::STAGE + 2 * C::KV_TILE;
+        const int first = (int)(k_hi - k0);
+        for (int i = lane; i < (KT - first) * (D / 4); i += 32) {
+          const int row = first + i / (D / 4), c = d0 + 2 * (i % (D / 4));
+          *reinterpret_cast<uint32_t*>(vb + tile_off<D, KT>(row, c)) = 0u;
+        }
+        if (pv == 0)
+          for (int i = lane; i < (KT - first) * (R / 2); i += 32) {
+            const int row = first + i / (R / 2), c = R + 2 * (i % (R / 2));
+            *reinterpret_cast<uint32_t*>(lb + tile_off<2 * R, KT>(row, c)) = 0u;
+          }
+        fence_proxy_async_smem();
+        __syncwarp();
+      }
+      bar_sync(BAR_P + pb, NB);
+#pragma unroll
+      for (int pt = 0; pt < NT; ++pt) {
+        const float c0 = Corr[pb * ROWS + 8 * pt + 2 * t4];
+        const float c1 = Corr[pb * ROWS + 8 * pt + 2 * t4 + 1];
+#pragma unroll
+        for (int mt = 0; mt < C::MT; ++mt) {
+          O[mt][pt][0] *= c0; O[mt][pt][2] *= c0;
+          O[mt][pt][1] *= c1; O[mt][pt][3] *= c1;
+        }
+#pragma unroll
+        for (int mr = 0; mr < C::MR; ++mr) {
+          Olr[mr][pt][0] *= c0; Olr[mr][pt][2] *= c0;
+          Olr[mr][pt][1] *= c1; Olr[mr][pt][3] *= c1;
+        }
+      }
+      const uint32_t pt_u = ptile_u + pb * C::P_TILE;
+#pragma unroll 2
+      for (int ks = 0; ks < KT / 16; ++ks) {
+        uint32_t bP[NT][2];
+#pragma unroll
+        for (int pt = 0; pt < NT; ++pt)
+          ldsm_x2(bP[pt][0], bP[pt][1], pt_u + tile_off<KT, ROWS>(8 * pt + rr, 16 * ks + ((lane >> 3) & 1) * 8));
+#pragma unroll
+        for (int mt = 0; mt < C::MT; ++mt) {
+          uint32_t aV[4];
+          ldsm_x4_t(aV, sV + tile_off<D, KT>(16 * ks + rr + (mi >> 1) * 8, d0 + 16 * mt + (mi & 1) * 8));
+#pragma unroll
+          for (int pt = 0; pt < NT; ++pt) mma16816(O[mt][pt], aV, bP[pt][0], bP[pt][1]);
+        }
+        if (pv == 0) {
+#pragma unroll
+          for (int mr = 0; mr < C::MR; ++mr) {
+            uint32_t aV[4];
+            ldsm_x4_t(aV, sL + tile_off<2 * R, KT>(16 * ks + rr + (mi >> 1) * 8, R + 16 * mr + (mi & 1) * 8));
+#pragma unroll
+            for (int pt = 0; pt < NT; ++pt) mma16816(Olr[mr][pt], aV, bP[pt][0], bP[pt][1]);
+          }
+        }
+      }
+      __syncwarp();
+      if (n + 2 < n_tiles) bar_arrive(BAR_PFREE + pb, NB);
+      if (lane == 0) mbar_arrive(empty_u + 8 * s);
+    }
+    bar_sync(BAR_END, TC_NTHR);
+    float* Mo = reinterpret_cast<float*>(area);
+#pragma unroll
+    for (int pt = 0; pt < NT; ++pt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int row = 8 * pt + 2 * t4 + (e & 1);
+        const int dd = gq + (e >> 1) * 8;
+#pragma unroll
+        for (int mt = 0; mt < C::MT; ++mt) Mo[row * W + d0 + 16 * mt + dd] = O[mt][pt][e];
+        if (pv == 0) {
+#pragma unroll
+          for (int mr = 0; mr < C::MR; ++mr)
+            if (16 * mr + dd < R) Mo[row * W + D + 16 * mr + dd] = Olr[mr][pt][e];
+        }
+      }
+  } else {
+    // ======================================================== TMA / MMA warp
+    if (lane == 0) {
+      constexpr uint32_t ID_S = umma_idesc_bf16(128, QPAD, 0, 0);
+      constexpr uint32_t ID_E = umma_idesc_bf16(128, D, 0, 1);
+      if (n_tiles > 0 && !mbar_wait(bkbar, 0)) fail = 1;
+      for (int n = 0; n < n_tiles; ++n) {
+        const int s = n % ST;
+        const uint32_t sK = area_u + s * C::STAGE;
+        const uint32_t sL = sK + 2 * C::KV_TILE;
+        if (!mbar_wait(full_u + 8 * s, (n / ST) & 1)) fail = 1;
+        if (n > 0 && !mbar_wait(tempty, (n - 1) & 1)) fail = 1;
+        tc_fence_after();
+        // base scores for every agent's rows: S_base^T = K_base Q^T
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t da = umma_desc(sK + (kk >> 2) * (KT * 128) + (kk & 3) * 32, 16, 1024, 2);
+          const uint64_t db = umma_desc(qu_u + (kk >> 2) * (QPAD * 128) + (kk & 3) * 32, 16, 1024, 2);
+          umma_bf16(tmem + TC_SCOL, da, db, ID_S, kk > 0);
+        }
+        // key deltas dK^a = LRk B_k^a (B_k^a stored r-major: the MN-major operand)
+        for (int a = 0; a < na; ++a) {
+#pragma unroll
+          for (int ks = 0; ks < C::KS; ++ks) {
+            const uint64_t da = umma_desc(sL + ks * 32, 16, 8 * C::LR_ROWB, C::LR_LAYOUT);
+            const uint64_t db = umma_desc(bks_u + a * align1k(C::BK_BYTES) + ks * 16 * 128, R * 128, 1024, 2);
+            umma_bf16(tmem + 128 * a, da, db, ID_E, ks > 0);
+          }
+        }
+        umma_commit(tfull);
+        umma_commit(empty_u + 8 * s);  // K and LRk of this stage have been read
+        if (n >= 1 && n - 1 + ST < n_tiles) {
+          const int sp = (n - 1) % ST;
+          if (!mbar_wait(empty_u + 8 * sp, ((n - 1) / ST) & 1)) fail = 1;
+          issue(n - 1 + ST);
+        }
+      }
+      for (int n = n_tiles; n < n_spec; ++n)  // loaded ahead of kv_len and not used
+        if (!mbar_wait(full_u + 8 * n, 0)) fail = 1;
+    }
+    __syncwarp();
+    bar_sync(BAR_END, TC_NTHR);
+  }
+  if (fail) s_fail = 1;
+  if (!mbar_wait(bvbar, 0)) s_fail = 1;
+  if (!mbar_wait(bkbar, 0)) s_fail = 1;
+  __syncthreads();
+  if (w == TC_NES + NPV) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TC_COLS);
+  }
+  float* Mo = reinterpret_cast<float*>(area);
+  for (int row = tid; row < n_rows; row += TC_NTHR) {
+    float l = 0.f;
+#pragma unroll
+    for (int ww = 0; ww < TC_NES; ++ww) l += Lw[ww * ROWS + row];
+    Mo[row * W + D + R + 1] = l;
+  }
+  if (ns == 1) {  // Z = O_base + s O_lr B_v^a (with split keys the merge applies B_v^a once)
+    const __nv_bfloat16* bv = reinterpret_cast<const __nv_bfloat16*>(bvs);
+    for (int i = tid; i < n_rows * (D / 4); i += TC_NTHR) {
+      const int row = i / (D / 4), c = 4 * (i % (D / 4));
+      const __nv_bfloat16* b = bv + (size_t)(row / g) * R * D + c;
+      float z0 = 0.f, z1 = 0.f, z2 = 0.f, z3 = 0.f;
+#pragma unroll
+      for (int j = 0; j < R; ++j) {
+        const float o = Mo[row * W + D + j];
+        const uint2 bb = *reinterpret_cast<const uint2*>(b + j * D);
+        const float2 f01 = unpack_bf16(bb.x), f23 = unpack_bf16(bb.y);
+        z0 = fmaf(o, f01.x, z0); z1 = fmaf(o, f01.y, z1);
+        z2 = fmaf(o, f23.x, z2); z3 = fmaf(o, f23.y, z3);
+      }
+      float4* zp = reinterpret_cast<float4*>(Mo + row * W + c);
+      float4 zo = *zp;
+      zo.x = fmaf(p.s, z0, zo.x); zo.y = fmaf(p.s, z1, zo.y);
+      zo.z = fmaf(p.s, z2, zo.z); zo.w = fmaf(p.s, z3, zo.w);
+      *zp = zo;
+    }
+  }
+  __syncthreads();
+  if (s_fail && tid == 0) atomicOr(p.err, 2);
+  if (ns == 1) {
+    if (s_fail) return;
+    for (int i = tid; i < n_rows * D; i += TC_NTHR) {
+      const int row = i / D, c = i % D;
+      const int a = row / g, gi = row % g;
+      const float l = Mo[row * W + D + R + 1];
+      const float val = l > 0.f ? Mo[row * W + c] / l : 0.f;
+      const int64_t oi = (((int64_t)seq * na + a) * p.n_q + kvh * g + gi) * D + c;
+      if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(val);
+      else reinterpret_cast<float*>(p.out)[oi] = val;
+    }
+    return;
+  }
+  // ---- split merge, shared by the unit's CTAs.  Each writes its partial
+  // (O_base, O_lr, m, l) to the workspace, waits until every split of the unit
+  // has (the launch is cooperative, so all CTAs are resident; the wait is
+  // bounded), then produces one contiguous share of the unit's output:
+  //   w_k = 2^(m_k - M) / sum_k 2^(m_k - M) l_k,  M = max_k m_k,
+  //   out = sum_k w_k O_base,k + s (sum_k w_k O_lr,k) B_v^a,
+  // B_v^a applied once per row (it is linear, so it commutes with the merge).
+  // A CTA that failed still arrives, so the others never wait for it.
+  float* ws_unit = p.partials + (size_t)unit * ns * n_rows * W;
+  {
+    float* part = ws_unit + (size_t)split * n_rows * W;
+    for (int i = tid; i < n_rows * (W / 4); i += TC_NTHR)
+      reinterpret_cast<float4*>(part)[i] = reinterpret_cast<const float4*>(Mo)[i];
+  }
+  int* arrive = p.counters + unit;
+  int* depart = p.counters + p.n_seqs * p.n_kv + unit;
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    atomicAdd(arrive, 1);
+    int it = 0;
+    while (ld_acquire_gpu(arrive) < ns) {
+      if (++it > (1 << 22)) {
+        atomicOr(p.err, 4);
+        break;
+      }
+      __nanosleep(32);
+    }
+    __threadfence();
+  }
+  __syncthreads();
+  constexpr int CH = D / 4;                        // float4 chunks per output row
+  const int n_items = n_rows * CH;
+  const int ib = (int)((int64_t)split * n_items / ns), ie = (int)((int64_t)(split + 1) * n_items / ns);
+  const int ni = ie - ib;
+  const int rb = ib / CH, nr = ni > 0 ? (ie - 1) / CH + 1 - rb : 0;
+  const int ks = ni > 0 ? max(1, TC_NTHR / ni) : 1;   // subsets of the splits per item
+  float* Wf = Mo;                                  // [nr][kMaxSplits] weights
+  float* Ol = Wf + nr * kMaxSplits;                // [nr][R] merged O_lr
+  float* T = Ol + nr * R;                          // [nr][ns][R] w_k O_lr,k
+  float4* red = reinterpret_cast<float4*>(T + ((nr * ns * R + 3) & ~3));  // [ks][ni]
+  auto part_at = [&](int k, int row, int c) {
+    return reinterpret_cast<const float4*>(ws_unit + ((size_t)k * n_rows + row) * W + c);
+  };
+  // (a) this thread's partial loads, issued before the weights are known
+  float4 v[2][4];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int u = tid + h * TC_NTHR;
+    const int item = ib + u % max(ni, 1), sub = u / max(ni, 1);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int k = sub + j * ks;
+      v[h][j] = (u < ni * ks && k < ns) ? __ldcg(part_at(k, item / CH, 4 * (item % CH)))
+                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  }
+  // (b) per row, one warp: lane k holds split k's (m, l) and O_lr
+  for (int r = w; r < nr; r += TC_NTHR / 32) {
+    const int row = rb + r;
+    float2 ml = make_float2(-INFINITY, 0.f);
+    float4 ol[R / 4];
+    if (lane < ns) {
+      ml = __ldcg(reinterpret_cast<const float2*>(ws_unit + ((size_t)lane * n_rows + row) * W + D + R));
+#pragma unroll
+      for (int j = 0; j < R / 4; ++j) ol[j] = __ldcg(part_at(lane, row, D + 4 * j));
+    }
+    float mx = ml.x;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const float e = (lane < ns && ml.x != -INFINITY) ? exp2f(ml.x - mx) : 0.f;
+    float lt = e * ml.y;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) lt += __shfl_xor_sync(0xffffffffu, lt, o);
+    const float wk = lt > 0.f ? e / lt : 0.f;
+    if (lane < ns) {
+      Wf[r * kMaxSplits + lane] = wk;
+      float4* tr = reinterpret_cast<float4*>(T + ((size_t)r * ns + lane) * R);
+#pragma unroll
+      for (int j = 0; j < R / 4; ++j)
+        tr[j] = make_float4(wk * ol[j].x, wk * ol[j].y, wk * ol[j].z, wk * ol[j].w);
+    }
+  }
+  __syncthreads();
+  // (c) merged O_lr per row; (d) weighted sums of this thread's loads
+  for (int i = tid; i < nr * R; i += TC_NTHR) {
+    const int r = i / R, j = i % R;
+    float acc = 0.f;
+    for (int k = 0; k < ns; ++k) acc += T[((size_t)r * ns + k) * R + j];
+    Ol[i] = acc;
+  }
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int u = tid + h * TC_NTHR;
+    if (u < ni * ks) {
+      const int item = ib + u % ni, sub = u / ni;
+      const int row = item / CH, c = 4 * (item % CH);
+      const float* wr = Wf + (row - rb) * kMaxSplits;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int k = sub + j * ks;
+        const float wk = k < ns ? wr[k] : 0.f;
+        acc.x = fmaf(wk, v[h][j].x, acc.x); acc.y = fmaf(wk, v[h][j].y, acc.y);
+        acc.z = fmaf(wk, v[h][j].z, acc.z); acc.w = fmaf(wk, v[h][j].w, acc.w);
+      }
+      for (int k = sub + 4 * ks; k < ns; k += ks) {  // more splits than four per subset
+        const float4 x = __ldcg(part_at(k, row, c));
+        acc.x = fmaf(wr[k], x.x, acc.x); acc.y = fmaf(wr[k], x.y, acc.y);
+        acc.z = fmaf(wr[k], x.z, acc.z); acc.w = fmaf(wr[k], x.w, acc.w);
+      }
+      red[u] = acc;
+    }
+  }
+  __syncthreads();
+  // (e) out = sum over subsets + s O_lr B_v^a
+  {
+    const __nv_bfloat16* bv = reinterpret_cast<const __nv_bfloat16*>(bvs);
+    for (int i = tid; i < ni; i += TC_NTHR) {
+      float4 acc = red[i];
+      for (int sub = 1; sub < ks; ++sub) {
+        const float4 x = red[sub * ni + i];
+        acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
+      }
+      const int item = ib + i, row = item / CH, c = 4 * (item % CH);
+      const int a = row / g, gi = row % g;
+      const float* ol = Ol + (row - rb) * R;
+      const __nv_bfloat16* bb = bv + (size_t)a * R * D + c;
+      float z0 = 0.f, z1 = 0.f, z2 = 0.f, z3 = 0.f;
+#pragma unroll
+      for (int j = 0; j < R; ++j) {
+        const float o = ol[j];
+        const uint2 b2 = *reinterpret_cast<const uint2*>(bb + j * D);
+        const float2 f01 = unpack_bf16(b2.x), f23 = unpack_bf16(b2.y);
+        z0 = fmaf(o, f01.x, z0); z1 = fmaf(o, f01.y, z1);
+        z2 = fmaf(o, f23.x, z2); z3 = fmaf(o, f23.y, z3);
+      }
+      acc.x = fmaf(p.s, z0, acc.x); acc.y = fmaf(p.s, z1, acc.y);
+      acc.z = fmaf(p.s, z2, acc.z); acc.w = fmaf(p.s, z3, acc.w);
+      const int64_t oi = (((int64_t)seq * na + a) * p.n_q + kvh * g + gi) * D + c;
+      if (p.out_bf16) {
+        uint2 o;
+        o.x = pack_bf16(acc.x, acc.y);
+        o.y = pack_bf16(acc.z, acc.w);
+        *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.out) + oi) = o;
+      } else {
+        *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + oi) = acc;
+      }
+    }
+  }
+  // the last CTA to leave resets the unit's counters for the next call
+  __syncthreads();
+  if (tid == 0 && atomicAdd(depart, 1) == ns - 1) {
+    *arrive = 0;
+    *depart = 0;
+    __threadfence();
+  }
 }
 
 // -------------------------------------------------------------------- host
@@ -737,10 +1537,25 @@ size_t smem_for(const AttnParams& p) {
 }
 
 // Splits per (sequence, KV head): enough CTAs for one CTA per SM.
+// SMs of the current device (148 on B200; also the answer when no device is
+// visible, so that workspace sizes can be planned on a host without a GPU)
+int device_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) {
+    cudaGetLastError();
+    return kSMs;
+  }
+  return n;
+}
+
+// splits of each (sequence, KV head) over the keys: enough CTAs to cover the
+// SMs once (one CTA per SM), so that a split launch is always fully resident
 int n_splits_for(const AttnParams& p) {
   const int units = p.n_seqs * p.n_kv;
   const int64_t total_tiles = (p.max_kv_len + KT - 1) / KT;
-  int64_t ns = units >= kSMs ? 1 : kSMs / units;
+  const int sms = device_sms();
+  int64_t ns = units >= sms ? 1 : sms / units;
   if (ns > kMaxSplits) ns = kMaxSplits;
   if (ns > total_tiles) ns = total_tiles;
   if (ns < 1) ns = 1;
@@ -778,9 +1593,65 @@ cudaError_t launch_t(const AttnParams& p, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+bool tc_supported(const AttnParams& p) {
+  if (p.d != 128 || !(p.r == 16 || p.r == 32 || p.r == 64)) return false;
+  if (!(p.g == 1 || p.g == 2 || p.g == 4 || p.g == 8)) return false;
+  if (p.n_agents > 3) return false;                     // TMEM: 128 columns per agent + scores
+  const int NT = n_rowtiles(p);
+  if (NT > 3) return false;
+  if (p.L_max >= (1ll << 31)) return false;
+  size_t sm = 0;
+  switch (p.r) {
+    case 16: sm = NT == 1 ? TCfg<128, 16, 1>::smem(p.n_agents) : NT == 2 ? TCfg<128, 16, 2>::smem(p.n_agents) : TCfg<128, 16, 3>::smem(p.n_agents); break;
+    case 32: sm = NT == 1 ? TCfg<128, 32, 1>::smem(p.n_agents) : NT == 2 ? TCfg<128, 32, 2>::smem(p.n_agents) : TCfg<128, 32, 3>::smem(p.n_agents); break;
+    default: sm = NT == 1 ? TCfg<128, 64, 1>::smem(p.n_agents) : NT == 2 ? TCfg<128, 64, 2>::smem(p.n_agents) : TCfg<128, 64, 3>::smem(p.n_agents); break;
+  }
+  return sm <= 227 * 1024;
+}
+
+template <int D, int R, int NT>
+cudaError_t launch_tc(const AttnParams& p, cudaStream_t st) {
+  using C = TCfg<D, R, NT>;
+  RopeTheta rt;
+  for (int i = 0; i < 64; ++i) rt.theta[i] = i < D / 2 ? std::pow(p.rope_base, -2.0 * i / D) : 0.0;
+  CUtensorMap mk, mv, ml, mb;
+  if (!make_maps(p, &mk, &mv, &ml)) return cudaErrorInvalidValue;
+  {
+    // B_k as (n_kv*d, r, n_agents): a CTA loads its head's r x 64 slices
+    cuuint64_t dims[3] = {(cuuint64_t)p.n_kv * D, (cuuint64_t)R, (cuuint64_t)p.n_agents};
+    cuuint64_t str[2] = {(cuuint64_t)p.n_kv * D * 2, (cuuint64_t)R * p.n_kv * D * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)R, 1};
+    cuuint32_t one[3] = {1, 1, 1};
+    if (encode_fn()(&mb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(p.B_k), dims, str, box,
+                    one, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
+  const size_t sm = C::smem(p.n_agents);
+  auto kern = decode_tc_kernel<D, R, NT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  if (e != cudaSuccess) return e;
+  dim3 grid(p.n_splits, p.n_seqs * p.n_kv);
+  // with split keys the unit's CTAs wait for one another: all must be resident
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(TC_NTHR);
+  cfg.dynamicSmemBytes = sm;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = p.n_splits > 1 ? 1 : 0;
+  e = cudaLaunchKernelEx(&cfg, kern, mk, mv, ml, mb, p, rt);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 bool bf16_decode_supported(const AttnParams& p) {
+  if (tc_supported(p)) return true;
   if (p.d != 128) return false;
   if (!(p.g == 1 || p.g == 2 || p.g == 4 || p.g == 8)) return false;
   const int NT = n_rowtiles(p);
@@ -800,13 +1671,20 @@ void bf16_decode_plan(const AttnParams& p, int* n_splits, int64_t* split_len, in
 size_t bf16_decode_partial_bytes(const AttnParams& p) {
   const int ns = n_splits_for(p);
   if (ns == 1) return 0;
-  return (size_t)p.n_seqs * p.n_kv * ns * (p.n_agents * p.g) * (p.d + 4) * sizeof(float);
+  return (size_t)p.n_seqs * p.n_kv * ns * (p.n_agents * p.g) * (p.d + p.r + 4) * sizeof(float);
 }
 
 cudaError_t launch_decode_bf16(const AttnParams& pin, la_dtype out, cudaStream_t st) {
   AttnParams p = pin;
   p.out_bf16 = out == LA_BF16;
   const int NT = n_rowtiles(p);
+  if (tc_supported(p)) {
+    switch (p.r) {
+      case 16: return NT == 1 ? launch_tc<128, 16, 1>(p, st) : NT == 2 ? launch_tc<128, 16, 2>(p, st) : launch_tc<128, 16, 3>(p, st);
+      case 32: return NT == 1 ? launch_tc<128, 32, 1>(p, st) : NT == 2 ? launch_tc<128, 32, 2>(p, st) : launch_tc<128, 32, 3>(p, st);
+      default: return NT == 1 ? launch_tc<128, 64, 1>(p, st) : NT == 2 ? launch_tc<128, 64, 2>(p, st) : launch_tc<128, 64, 3>(p, st);
+    }
+  }
   switch (p.r) {
     case 8: return NT == 1 ? launch_t<128, 8, 1>(p, st) : NT == 2 ? launch_t<128, 8, 2>(p, st) : launch_t<128, 8, 3>(p, st);
     case 16: return NT == 1 ? launch_t<128, 16, 1>(p, st) : NT == 2 ? launch_t<128, 16, 2>(p, st) : launch_t<128, 16, 3>(p, st);
