@@ -876,7 +876,36 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
     for (int i = 0; i < na * R; ++i)
       bulk_load(bvs_u + i * D * 2, Bv + (int64_t)i * ldB + kvh * D, D * 2, bvbar);
   }
-  const int64_t kvl = p.kv_len[seq];
+  const int64_t kvl = p.kv_len[seq];  // in flight while the constants are computed
+  const int sp = w & 3, kb = 32 * sp + 16 * (w >> 2);  // score warp: TMEM sub-partition, first key
+  // R(j) for this thread's keys j = kb + gq + 8 hh and its frequencies
+  // i = 16 grp + 8 q + 2 t4 (+1), as (cos, cos) and (sin, sin) pairs over the
+  // two adjacent frequencies: the operands of the packed f32x2 rotation
+  uint64_t RC[C::NG][2][2], RS[C::NG][2][2];
+  if (w < TC_NES) {
+#pragma unroll
+    for (int grp = 0; grp < C::NG; ++grp)
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int i = 16 * grp + 8 * q + 2 * t4;
+        const float th0 = (float)rt.theta[i], th1 = (float)rt.theta[i + 1];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const float j = (float)(kb + gq + 8 * hh);
+          const float2 a = sincos_small(j * th0), b = sincos_small(j * th1);
+          RC[grp][hh][q] = f2(a.x, b.x);
+          RS[grp][hh][q] = f2(a.y, b.y);
+        }
+      }
+  }
+  if (tid < D / 2) theta[tid] = rt.theta[tid];
+  if (w >= TC_NES && w < TC_NES + NPV) {
+    // the first tile's query rotation R(-k_lo), scaled by s (exact in fp64)
+    for (int i = tid - 32 * TC_NES; i < D / 2; i += 32 * NPV) {
+      const float2 cs = rope_cs_exact(k_lo, rt.theta[i]);
+      cs0[i] = make_float2(cs.x * p.s, cs.y * p.s);
+    }
+  }
   if (kvl < 1 || kvl > p.max_kv_len) {
     if (tid == 0 && split == 0) atomicOr(p.err, 1);
     if (w == TC_NES + NPV && lane == 0) {  // the copies in flight land before the CTA leaves
@@ -892,31 +921,6 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
   if (w == TC_NES + NPV) tmem_alloc(smem_u32(tslot), TC_COLS);
 
   int fail = 0;
-  // ---- per-CTA constants: Q (the base-score MMA operand), frequencies, and the
-  // score warps' in-tile rotations R(j) while the first loads are in flight
-  const int sp = w & 3, kb = 32 * sp + 16 * (w >> 2);  // score warp: TMEM sub-partition, first key
-  uint32_t cjh[C::NG][2][4];
-  if (w < TC_NES) {
-    // R(j) for this thread's keys j = kb + gq (+8) and its 16 frequencies (f16 pairs)
-#pragma unroll
-    for (int grp = 0; grp < C::NG; ++grp)
-#pragma unroll
-      for (int f = 0; f < 4; ++f) {
-        const int i = 16 * grp + 8 * (f >> 1) + 2 * t4 + (f & 1);
-        const float th = (float)rt.theta[i];
-#pragma unroll
-        for (int kr = 0; kr < 2; ++kr)
-          cjh[grp][kr][f] = pack_half2(sincos_small((float)(kb + gq + 8 * kr) * th));
-      }
-  }
-  if (tid < D / 2) theta[tid] = rt.theta[tid];
-  if (w >= TC_NES && w < TC_NES + NPV) {
-    // the first tile's query rotation R(-k_lo), scaled by s (exact in fp64)
-    for (int i = tid - 32 * TC_NES; i < D / 2; i += 32 * NPV) {
-      const float2 cs = rope_cs_exact(k_lo, rt.theta[i]);
-      cs0[i] = make_float2(cs.x * p.s, cs.y * p.s);
-    }
-  }
   __syncthreads();  // barriers initialised, cs0 ready
   if (!mbar_wait(qbar, 0)) fail = 1;
   // Q (swizzled: the base-score MMA operand) and Q' = s R(-k_lo) Q for the first tile
@@ -1000,6 +1004,7 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
         for (int a = 0; a < na; ++a) {
           const int pa = a == 0 ? pa_of[0] : (a == 1 ? pa_of[1] : pa_of[2]);
           const bool mn = a == 0 ? mine[0] : (a == 1 ? mine[1] : mine[2]);
+          float Sd[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int grp = 0; grp < C::NG; ++grp) {
             const int cb = grp & 1, nb = cb ^ 1;
@@ -1018,27 +1023,27 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
             for (int q = 0; q < 2; ++q)
 #pragma unroll
               for (int hh = 0; hh < 2; ++hh) {
-                // R(j) of key row hh at the adjacent frequencies (2 t4, 2 t4 + 1) + 8 q
-                const float2 u = unpack_half2(cjh[grp][hh][2 * q]);
-                const float2 v = unpack_half2(cjh[grp][hh][2 * q + 1]);
-                const uint64_t cc = f2(u.x, v.x), ss = f2(u.y, v.y), nn = f2(-u.y, -v.y);
+                // (x1, x2) = delta columns (i, i + d/2) at two adjacent i; R(j) x
                 const uint64_t x1 = f2(__uint_as_float(xl[cb][4 * q + 2 * hh]), __uint_as_float(xl[cb][4 * q + 2 * hh + 1]));
                 const uint64_t x2 = f2(__uint_as_float(xh[cb][4 * q + 2 * hh]), __uint_as_float(xh[cb][4 * q + 2 * hh + 1]));
-                const float2 l2 = f2_unpack(fma_f2(x1, cc, mul_f2(x2, nn)));
-                const float2 h2 = f2_unpack(fma_f2(x2, cc, mul_f2(x1, ss)));
+                const uint64_t c = RC[grp][hh][q], sn = RS[grp][hh][q];
+                const float2 l2 = f2_unpack(sub_f2(mul_f2(x1, c), mul_f2(x2, sn)));
+                const float2 h2 = f2_unpack(fma_f2(x2, c, mul_f2(x1, sn)));
                 A_lo[2 * q + hh] = pack_bf16(l2.x, l2.y);
                 A_hi[2 * q + hh] = pack_bf16(h2.x, h2.y);
               }
             uint32_t bq[4];
             ldsm_x4(bq, qpb + tile_off<D, ROWS>(8 * pa + rr, 16 * grp + (mi & 1) * 8 + (mi >> 1) * (D / 2)));
             if (!mn) bq[0] = bq[1] = bq[2] = bq[3] = 0u;
-#pragma unroll
-            for (int pt = 0; pt < NT; ++pt)
-              if (pt == pa) {
-                mma16816(S[pt], A_lo, bq[0], bq[1]);
-                mma16816(S[pt], A_hi, bq[2], bq[3]);
-              }
+            mma16816(Sd, A_lo, bq[0], bq[1]);
+            mma16816(Sd, A_hi, bq[2], bq[3]);
           }
+#pragma unroll
+          for (int pt = 0; pt < NT; ++pt)
+            if (pt == pa) {
+              S[pt][0] += Sd[0]; S[pt][1] += Sd[1];
+              S[pt][2] += Sd[2]; S[pt][3] += Sd[3];
+            }
         }
       }
       tc_fence_before();
@@ -1256,6 +1261,21 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
         }
         umma_commit(tfull);
         umma_commit(empty_u + 8 * s);  // K and LRk of this stage have been read
+        if (n == 0) {
+          // the split's later tiles stream into L2 from here on (after the first
+          // loads have landed), so that HBM stays busy between stage refills
+          for (int m = ST; m < te - tb; ++m) {
+            const int key0 = (int)(k_lo + (int64_t)m * KT);
+#pragma unroll
+            for (int b = 0; b < D / 64; ++b) {
+              tma_prefetch_l2_4d(&tmK, 64 * b, key0, kvh, seq);
+              tma_prefetch_l2_4d(&tmV, 64 * b, key0, kvh, seq);
+            }
+            constexpr int LB = (2 * R) < 64 ? 2 * R : 64;
+#pragma unroll
+            for (int b = 0; b < (2 * R) / LB; ++b) tma_prefetch_l2_3d(&tmL, LB * b, key0, seq);
+          }
+        }
         if (n >= 1 && n - 1 + ST < n_tiles) {
           const int sp = (n - 1) % ST;
           if (!mbar_wait(empty_u + 8 * sp, ((n - 1) / ST) & 1)) fail = 1;
