@@ -15,6 +15,7 @@
 #include <cooperative_groups.h>
 #include <cudaTypedefs.h>
 
+#include "bf16_common.cuh"
 #include "la_internal.cuh"
 #include "ptx.cuh"
 
@@ -31,7 +32,6 @@ constexpr int NSTAGE = 3;
 constexpr int kMaxHS = 16;
 constexpr int kSMs = 148;
 
-constexpr int align1k(int x) { return (x + 1023) / 1024 * 1024; }
 
 template <int R>
 struct ACfg {
@@ -143,19 +143,6 @@ __global__ void __launch_bounds__(NTHR, 1)
     }
   }
   if (hs > 1) cluster.sync();
-}
-
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
-  return fn;
 }
 
 template <int R>

@@ -36,6 +36,7 @@
 
 #include <cuda_fp16.h>
 
+#include "bf16_common.cuh"
 #include "la_internal.cuh"
 #include "ptx.cuh"
 
@@ -50,17 +51,11 @@ constexpr int NES = 8;              // score warps (16 keys each)
 constexpr int NPV = 2;              // value warps
 constexpr int NTHR = 32 * (NES + NPV);
 constexpr int kMaxSplits = 32;
-constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kSMs = 148;
 // named barriers (0 is __syncthreads)
 constexpr int BAR_MAX = 1, BAR_P = 2, BAR_PFREE = 4, BAR_QP = 6, BAR_END = 8;
 
-constexpr int align1k(int x) { return (x + 1023) / 1024 * 1024; }
 
-// RoPE frequencies theta_i = base^(-2i/d), formed in fp64 on the host
-struct RopeTheta {
-  double theta[64];
-};
 constexpr int imax(int a, int b) { return a > b ? a : b; }
 
 template <int D, int R, int NT>
@@ -84,27 +79,6 @@ struct Cfg {
            (size_t)align1k(BK_BYTES) * n_agents + (size_t)BK_BYTES * n_agents + 64;
   }
 };
-
-// (cos, sin) of t * theta, the angle formed and reduced modulo 2 pi in fp64
-__device__ __forceinline__ float2 rope_cs_exact(int64_t t, double theta) {
-  const double two_pi = 6.283185307179586476925286766559;
-  const double ang = (double)t * theta;
-  const float red = (float)fma(-two_pi, rint(ang * 0.15915494309189533577), ang);
-  float s, c;
-  sincosf(red, &s, &c);
-  return make_float2(c, s);
-}
-
-// (cos, sin) of a small angle (|ang| < ~200 rad): Cody-Waite reduction with a
-// two-constant split of 2 pi, then the SFU (about 2^-21 absolute on [-pi, pi])
-__device__ __forceinline__ float2 sincos_small(float ang) {
-  const float k = rintf(ang * 0.15915494309189535f);
-  float red = fmaf(-k, 6.28318548202514648f, ang);
-  red = fmaf(-k, -1.7484556000744083e-07f, red);
-  float s, c;
-  __sincosf(red, &s, &c);
-  return make_float2(c, s);
-}
 
 // Q'[row] = s R(-t) Q[row] for every row, frequencies i = lane .. of this warp
 // (nw_off: first frequency handled by the calling warp, step 32 per warp)
@@ -1499,24 +1473,6 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
 }
 
 // -------------------------------------------------------------------- host
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
-  return fn;
-}
-
-CUtensorMapSwizzle swizzle_for(int row_bytes) {
-  return row_bytes >= 128 ? CU_TENSOR_MAP_SWIZZLE_128B
-                          : (row_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
-}
-
 bool make_maps(const AttnParams& p, CUtensorMap* mk, CUtensorMap* mv, CUtensorMap* ml) {
   auto enc = encode_fn();
   if (!enc) return false;

@@ -1,0 +1,574 @@
+// Flash-LoRA-Attention prefill on the tcgen05 tensor cores (bf16 storage,
+// fp32 accumulation in TMEM).
+//
+// One CTA = one (sequence, agent, KV head) and a block of 128 query rows: the
+// 128 / g query tokens of the block times the g query heads of the GQA group
+// (row = token * g + head).  Keys stream in tiles of 128.  Per tile (LRAgent
+// summary App. D.1: RoPE blocks reordering on the key side, so the delta is
+// rebuilt in head dimension per tile):
+//   dK   = LRk B_k^a                       tcgen05, M = 128 keys, N = d, K = r
+//   K^a  = K_base + s R(t) dK              CUDA cores, written over K_base in
+//                                          shared memory; R(t) = R(k0) R(j)
+//   S    = Q K^a^T                         tcgen05, M = 128 rows, N = 128 keys
+//   P    = exp2(S log2e / sqrt(d) - m)     CUDA cores, to TMEM as bf16
+//   O   += P V_base,  O_lr += P LR         tcgen05, A = P from TMEM; value side
+//                                          reordered (LRAgent explainer,
+//                                          Metodologia 3): only r wide
+// and once per row at the end out = (O + s O_lr B_v^a) / l.
+// The running max is rescaled lazily: O and l are corrected only when a row's
+// maximum grows by more than 2^8, so P <= 256 and the correction is rare.
+//
+// Warps: 8 compute warps build K^a (16 keys each, the mma fragment layout of
+// the delta) and run the softmax (two warps per TMEM sub-partition, 64 keys
+// each); warp 8 issues TMA loads and MMAs.  The compute warps build tile n+1
+// before the softmax of tile n, so the S MMA of tile n+1 runs during that
+// softmax and the P V MMA of tile n during the next build.
+#include <cmath>
+
+#include <cuda_fp16.h>
+
+#include "bf16_common.cuh"
+#include "la_internal.cuh"
+#include "ptx.cuh"
+
+namespace la {
+namespace {
+
+using namespace ptx;
+
+constexpr int PD = 128;                  // head_dim
+constexpr int PKT = 128;                 // keys per tile
+constexpr int PM = 128;                  // query rows per CTA
+constexpr int PNC = 8;                   // compute warps
+constexpr int PNTHR = 32 * (PNC + 1);
+// TMEM columns
+constexpr int T_DK = 0, T_S = 128, T_P = 256, T_O = 320, T_OL = 448, T_COLS = 512;
+// named barriers (0 is __syncthreads)
+constexpr int PBAR_CW = 1, PBAR_PAIR = 2;  // PBAR_PAIR + sub-partition: the two warps of a row block
+
+template <int R>
+struct PCfg {
+  static constexpr int LRW = 2 * R;                            // LR row, elements
+  static constexpr int LR_ROWB = (LRW < 64 ? LRW : 64) * 2;     // bytes per LR box row
+  static constexpr uint32_t LR_LAYOUT = LR_ROWB == 128 ? 2u : (LR_ROWB == 64 ? 4u : 6u);
+  static constexpr int KV = PKT * PD * 2;                       // a K or V tile
+  static constexpr int LR_TILE = align1k(PKT * LRW * 2);
+  static constexpr int STAGE = KV + LR_TILE;                    // K (or V) tile + LR rows
+  static constexpr int Q_BYTES = PM * PD * 2;
+  static constexpr int B_BYTES = R * PD * 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;                 // [2] stages
+  static constexpr int OFF_V = OFF_K + 2 * STAGE;               // [2] stages
+  static constexpr int OFF_BK = OFF_V + 2 * STAGE;
+  static constexpr int OFF_BV = OFF_BK + align1k(B_BYTES);
+  static constexpr int OFF_MISC = OFF_BV + align1k(B_BYTES);
+  // misc: anchors [2][64] float2, exchange [2][8][32] float, theta [64] double,
+  // 16 mbarriers, the TMEM slot
+  static constexpr int MISC = 1024 + 2048 + 512 + 128 + 16;
+  static constexpr size_t SMEM = 1024 + OFF_MISC + MISC;
+};
+
+template <int R>
+__global__ void __launch_bounds__(PNTHR, 1)
+    prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
+                      const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV,
+                      const __grid_constant__ CUtensorMap tmL,
+                      const __grid_constant__ CUtensorMap tmB, const AttnParams p,
+                      const __grid_constant__ RopeTheta rt) {
+  using C = PCfg<R>;
+  constexpr int D = PD;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sb = smem_u32(smem);
+  const uint32_t q_u = sb + C::OFF_Q, k_u = sb + C::OFF_K, v_u = sb + C::OFF_V;
+  const uint32_t bk_u = sb + C::OFF_BK, bv_u = sb + C::OFF_BV;
+  unsigned char* misc = smem + C::OFF_MISC;
+  float2* anc = reinterpret_cast<float2*>(misc);               // [2][64] s (cos, sin)(k0 theta_i)
+  float* xch = reinterpret_cast<float*>(misc + 1024);          // [2][8][32]
+  double* theta = reinterpret_cast<double*>(misc + 3072);      // [64]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(misc + 3584);   // [16]
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(misc + 3584 + 128);
+  const __nv_bfloat16* bvs = reinterpret_cast<const __nv_bfloat16*>(smem + C::OFF_BV);
+  __shared__ int s_fail;
+
+  const uint32_t b0 = smem_u32(bars);
+  auto kfull = [&](int s) { return b0 + 8 * s; };
+  auto vfull = [&](int s) { return b0 + 16 + 8 * s; };
+  auto kempty = [&](int s) { return b0 + 32 + 8 * s; };
+  auto vempty = [&](int s) { return b0 + 48 + 8 * s; };
+  const uint32_t qbar = b0 + 64, bvbar = b0 + 72, dkfull = b0 + 80, kaready = b0 + 88;
+  const uint32_t sfull = b0 + 96, staken = b0 + 104, pfull = b0 + 112, pvdone = b0 + 120;
+
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int gq = lane >> 2, t4 = lane & 3;
+  const int seq = blockIdx.z;
+  const int agent = blockIdx.y / p.n_kv, kvh = blockIdx.y % p.n_kv;
+  const int g = p.g, na = p.n_agents;
+  const int QB = PM / g;
+  const int tok0 = blockIdx.x * QB;
+  const int ntok = min(QB, p.n_q_tokens - tok0);
+  const int64_t qmin = p.q_pos0 + tok0;               // position of the block's first token
+  const int64_t kend = qmin + ntok;                    // keys [0, kend)
+  const int N = (int)((kend + PKT - 1) / PKT);
+
+  auto load_stage = [&](const CUtensorMap* m, uint32_t base, uint32_t bar, int n) {
+    const int key0 = n * PKT;
+    mbar_expect_tx(bar, (uint32_t)(C::KV + PKT * C::LRW * 2));
+#pragma unroll
+    for (int b = 0; b < D / 64; ++b) tma_load_4d(base + b * PKT * 128, m, bar, 64 * b, key0, kvh, seq);
+    constexpr int LB = C::LR_ROWB / 2;
+#pragma unroll
+    for (int b = 0; b < C::LRW / LB; ++b)
+      tma_load_3d(base + C::KV + b * PKT * C::LR_ROWB, &tmL, bar, LB * b, key0, seq);
+  };
+  auto load_k = [&](int n) { load_stage(&tmK, k_u + (n & 1) * C::STAGE, kfull(n & 1), n); };
+  auto load_v = [&](int n) { load_stage(&tmV, v_u + (n & 1) * C::STAGE, vfull(n & 1), n); };
+
+  if (w == PNC && lane == 0) {
+    s_fail = 0;
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(kfull(s), 1);
+      mbar_init(vfull(s), 1);
+      mbar_init(kempty(s), 1);
+      mbar_init(vempty(s), 1);
+    }
+    mbar_init(qbar, 1);
+    mbar_init(bvbar, 1);
+    mbar_init(dkfull, 1);
+    mbar_init(kaready, PNC);
+    mbar_init(sfull, 1);
+    mbar_init(staken, PNC);
+    mbar_init(pfull, PNC);
+    mbar_init(pvdone, 1);
+    fence_mbar_init();
+    tma_prefetch(&tmQ);
+    tma_prefetch(&tmB);
+    tma_prefetch(&tmK);
+    tma_prefetch(&tmV);
+    tma_prefetch(&tmL);
+    // the block's rows: g heads of each of its tokens, two 64-column boxes
+    mbar_expect_tx(qbar, (uint32_t)(C::Q_BYTES + C::B_BYTES));
+#pragma unroll
+    for (int b = 0; b < D / 64; ++b)
+      tma_load_4d(q_u + b * PM * 128, &tmQ, qbar, 64 * b, kvh * g, tok0, seq * na + agent);
+#pragma unroll
+    for (int b = 0; b < D / 64; ++b)
+      tma_load_3d(bk_u + b * R * 128, &tmB, qbar, kvh * D + 64 * b, 0, agent);
+    load_k(0);
+    load_v(0);
+    if (N > 1) {
+      load_k(1);
+      load_v(1);
+    }
+    const __nv_bfloat16* Bv = reinterpret_cast<const __nv_bfloat16*>(p.B_v);
+    mbar_expect_tx(bvbar, (uint32_t)C::B_BYTES);
+    for (int j = 0; j < R; ++j)
+      bulk_load(bv_u + j * D * 2, Bv + ((int64_t)agent * R + j) * p.n_kv * D + kvh * D, D * 2, bvbar);
+  }
+  if (w == PNC) tmem_alloc(smem_u32(tslot), T_COLS);
+
+  // ---- compute-warp constants: R(j) for the two keys of the build fragment,
+  // frequencies, and the first two tiles' anchors s R(k0)
+  const int sp = w & 3, ch = w >> 2;
+  const int kb = 32 * sp + 16 * ch;   // build: this warp's 16 keys (its TMEM lanes)
+  // (cos, cos) and (sin, sin) over two adjacent frequencies: the operands of
+  // the packed f32x2 rotation
+  uint64_t RC[4][2][2], RS[4][2][2];
+  if (w < PNC) {
+#pragma unroll
+    for (int grp = 0; grp < 4; ++grp)
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int i = 16 * grp + 8 * q + 2 * t4;
+        const float th0 = (float)rt.theta[i], th1 = (float)rt.theta[i + 1];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const float j = (float)(kb + gq + 8 * hh);
+          const float2 a = sincos_small(j * th0), b = sincos_small(j * th1);
+          RC[grp][hh][q] = f2(a.x, b.x);
+          RS[grp][hh][q] = f2(a.y, b.y);
+        }
+      }
+  }
+  if (tid < D / 2) theta[tid] = rt.theta[tid];
+  if (tid < 2 * (D / 2)) {
+    const int n = tid / (D / 2), i = tid % (D / 2);
+    const float2 cs = rope_cs_exact((int64_t)n * PKT, rt.theta[i]);
+    anc[n * 64 + i] = make_float2(cs.x * p.s, cs.y * p.s);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+  int fail = 0;
+
+  if (w == PNC) {
+    // ============================================================ TMA / MMA warp
+    if (lane == 0) {
+      constexpr uint32_t ID_DK = umma_idesc_bf16(128, PD, 0, 1);
+      constexpr uint32_t ID_S = umma_idesc_bf16(128, PKT, 0, 0);
+      constexpr uint32_t ID_PV = umma_idesc_bf16(128, PD, 0, 1);
+      constexpr uint32_t ID_PL = umma_idesc_bf16(128, C::LRW, 0, 1);
+      auto mma_dk = [&](int n) {  // dK = LRk B_k^a
+        if (!mbar_wait(kfull(n & 1), (n >> 1) & 1)) fail = 1;
+        tc_fence_after();
+        const uint32_t lr = k_u + (n & 1) * C::STAGE + C::KV;
+#pragma unroll
+        for (int ks = 0; ks < R / 16; ++ks)
+          umma_bf16(tmem + T_DK, umma_desc(lr + ks * 32, 16, 8 * C::LR_ROWB, C::LR_LAYOUT),
+                    umma_desc(bk_u + ks * 16 * 128, R * 128, 1024, 2), ID_DK, ks > 0);
+        umma_commit(dkfull);
+      };
+      auto mma_pv = [&](int n) {  // O += P V_base, O_lr += P LR
+        if (!mbar_wait(pfull, n & 1)) fail = 1;
+        if (!mbar_wait(vfull(n & 1), (n >> 1) & 1)) fail = 1;
+        tc_fence_after();
+        const uint32_t vs = v_u + (n & 1) * C::STAGE;
+#pragma unroll
+        for (int ks = 0; ks < PKT / 16; ++ks)
+          umma_bf16_ts(tmem + T_O, tmem + T_P + ks * 8, umma_desc(vs + ks * 16 * 128, PKT * 128, 1024, 2),
+                       ID_PV, (n > 0 || ks > 0) ? 1u : 0u);
+#pragma unroll
+        for (int ks = 0; ks < PKT / 16; ++ks)
+          umma_bf16_ts(tmem + T_OL, tmem + T_P + ks * 8,
+                       umma_desc(vs + C::KV + ks * 16 * C::LR_ROWB, PKT * C::LR_ROWB, 8 * C::LR_ROWB,
+                                 C::LR_LAYOUT),
+                       ID_PL, (n > 0 || ks > 0) ? 1u : 0u);
+        umma_commit(pvdone);
+        umma_commit(vempty(n & 1));
+      };
+      if (!mbar_wait(qbar, 0)) fail = 1;
+      mma_dk(0);
+      for (int n = 0; n < N; ++n) {
+        if (!mbar_wait(kaready, n & 1)) fail = 1;
+        if (n > 0 && !mbar_wait(staken, (n - 1) & 1)) fail = 1;
+        tc_fence_after();
+        const uint32_t ks_ = k_u + (n & 1) * C::STAGE;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_bf16(tmem + T_S, umma_desc(q_u + (kk >> 2) * (PM * 128) + (kk & 3) * 32, 16, 1024, 2),
+                    umma_desc(ks_ + (kk >> 2) * (PKT * 128) + (kk & 3) * 32, 16, 1024, 2), ID_S, kk > 0);
+        umma_commit(sfull);
+        umma_commit(kempty(n & 1));
+        if (n + 1 < N) mma_dk(n + 1);
+        if (n > 0) mma_pv(n - 1);
+        if (n + 2 < N) {
+          if (!mbar_wait(kempty(n & 1), (n >> 1) & 1)) fail = 1;
+          load_k(n + 2);
+        }
+        if (n > 0 && n + 1 < N) {
+          if (!mbar_wait(vempty((n - 1) & 1), ((n - 1) >> 1) & 1)) fail = 1;
+          load_v(n + 1);
+        }
+      }
+      mma_pv(N - 1);
+      // loads in flight when the loop ends are all consumed: every issued tile is used
+    }
+    __syncwarp();
+  } else {
+    // ============================================================ compute warps
+    const float sl2 = p.scale * kLog2e;
+    const int row = 32 * sp + lane;          // softmax: this thread's query row (TMEM lane)
+    const int rtok = row / g;
+    const bool rvalid = rtok < ntok;
+    const int64_t qpos = qmin + rtok;
+    float m_ref = -INFINITY, lsum = 0.f;
+
+    auto build = [&](int n) {  // K^a = K_base + s R(k0) R(j) dK, over K_base in place
+      if (!mbar_wait(dkfull, n & 1)) fail = 1;
+      if (!mbar_wait(kfull(n & 1), (n >> 1) & 1)) fail = 1;
+      tc_fence_after();
+      const uint32_t kst = k_u + (n & 1) * C::STAGE;
+      const float2* an = anc + (n & 1) * 64;
+      const uint32_t tl = tmem + T_DK + ((uint32_t)kb << 16);
+      // this lane's pair of K elements in a 128-byte-swizzled row: key kb + gq
+      // (+8), 16-byte chunk (2 grp + q) ^ gq, word t4; columns + d/2 are one box on
+      const uint32_t rowb = kst + (uint32_t)(kb + gq) * 128 + 4 * t4;
+#pragma unroll
+      for (int grp = 0; grp < 4; ++grp) {
+        uint32_t xl[8], xh[8];
+        tmem_ld16x256_x2(xl, tl + 16 * grp);
+        tmem_ld16x256_x2(xh, tl + 16 * grp + D / 2);
+        tmem_wait_ld_regs(xl, xh);
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const int i0 = 16 * grp + 8 * q + 2 * t4;
+          const float2 a0 = an[i0], a1 = an[i0 + 1];
+          const uint64_t ac = f2(a0.x, a1.x), as = f2(a0.y, a1.y);
+          const uint32_t cx = (uint32_t)(((2 * grp + q) ^ gq) << 4);
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            const uint64_t x1 = f2(__uint_as_float(xl[4 * q + 2 * hh]), __uint_as_float(xl[4 * q + 2 * hh + 1]));
+            const uint64_t x2 = f2(__uint_as_float(xh[4 * q + 2 * hh]), __uint_as_float(xh[4 * q + 2 * hh + 1]));
+            const uint64_t c = RC[grp][hh][q], sn = RS[grp][hh][q];
+            const uint64_t y1 = sub_f2(mul_f2(x1, c), mul_f2(x2, sn));   // R(j) dK
+            const uint64_t y2 = fma_f2(x2, c, mul_f2(x1, sn));
+            const float2 z1 = f2_unpack(sub_f2(mul_f2(ac, y1), mul_f2(as, y2)));   // s R(k0) y
+            const float2 z2 = f2_unpack(fma_f2(ac, y2, mul_f2(as, y1)));
+            const uint32_t o1 = rowb + hh * 1024 + cx, o2 = o1 + PKT * 128;
+            sts32(o1, add_bf16x2(lds32(o1), pack_bf16(z1.x, z1.y)));
+            sts32(o2, add_bf16x2(lds32(o2), pack_bf16(z2.x, z2.y)));
+          }
+        }
+      }
+      fence_proxy_async_smem();  // the S MMA reads K^a through the async proxy
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(kaready);
+    };
+
+    auto softmax = [&](int n) {
+      if (!mbar_wait(sfull, n & 1)) fail = 1;
+      tc_fence_after();
+      const uint32_t ts = tmem + T_S + 64 * ch + ((uint32_t)(32 * sp) << 16);
+      uint32_t sv[2][32];
+      tmem_ld32x32b_x32(sv[0], ts);
+      tmem_ld32x32b_x32(sv[1], ts + 32);
+      tmem_wait_ld_r32(sv[0]);
+      tmem_wait_ld_r32(sv[1]);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(staken);  // S may be overwritten by the next tile's MMA
+
+      // row maximum of the raw scores (the scale is positive); keys past a row's
+      // position are set to -inf (only the tiles that reach the block's first
+      // position need it; rows past the chunk are never written out)
+      const int64_t key0 = (int64_t)n * PKT + 64 * ch;
+      if (key0 + 63 > qmin) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int c = 0; c < 32; ++c)
+            if (key0 + 32 * h + c > qpos) sv[h][c] = __float_as_uint(-INFINITY);
+      }
+      float mr[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float m = __uint_as_float(sv[h][0]);
+#pragma unroll
+        for (int c = 1; c < 31; c += 2) m = max3f(m, __uint_as_float(sv[h][c]), __uint_as_float(sv[h][c + 1]));
+        mr[h] = fmaxf(m, __uint_as_float(sv[h][31]));
+      }
+      const float mloc = fmaxf(mr[0], mr[1]) * sl2;
+      float* xb = xch + (n & 1) * 256;
+      xb[w * 32 + lane] = mloc;
+      bar_sync(PBAR_PAIR + sp, 64);
+      const float mt = fmaxf(mloc, xb[(w ^ 4) * 32 + lane]);
+      // lazy rescale: move the reference max only when a row's max grew by > 8
+      const bool need = mt > m_ref + 8.f || (m_ref == -INFINITY && mt != -INFINITY);
+      if (__any_sync(0xffffffffu, need)) {
+        const float m_new = fmaxf(m_ref, mt);
+        const float corr = m_ref == -INFINITY ? 0.f : fast_exp2(m_ref - m_new);
+        if (n > 0 && __any_sync(0xffffffffu, m_ref != -INFINITY)) {
+          if (!mbar_wait(pvdone, (n - 1) & 1)) fail = 1;  // O holds every tile before this one
+          tc_fence_after();
+          const uint32_t to = tmem + T_O + 64 * ch + ((uint32_t)(32 * sp) << 16);
+#pragma unroll 1
+          for (int h = 0; h < 4; ++h) {
+            uint32_t ov[16];
+            tmem_ld32x32b_x16(ov, to + 16 * h);
+            tmem_wait_ld_r16(ov);
+#pragma unroll
+            for (int c = 0; c < 16; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * corr);
+            tmem_st32x32b_x16(to + 16 * h, ov);
+          }
+          if (ch == 0) {
+            const uint32_t tol = tmem + T_OL + ((uint32_t)(32 * sp) << 16);
+#pragma unroll 1
+            for (int h = 0; h < C::LRW / 16; ++h) {
+              uint32_t ov[16];
+              tmem_ld32x32b_x16(ov, tol + 16 * h);
+              tmem_wait_ld_r16(ov);
+#pragma unroll
+              for (int c = 0; c < 16; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * corr);
+              tmem_st32x32b_x16(tol + 16 * h, ov);
+            }
+          }
+          tmem_wait_st();
+        }
+        lsum *= corr;
+        m_ref = m_new;
+      }
+      // p = 2^(S scale log2e - m): one packed fma per pair, then the SFU
+      const float mu = m_ref == -INFINITY ? 0.f : m_ref;   // rows with no visible key yet: p = 0
+      const uint64_t scl = f2(sl2, sl2), nmu = f2(-mu, -mu);
+      uint32_t pk[32];
+      uint64_t acc = f2(0.f, 0.f);
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          const float2 xa = f2_unpack(fma_f2(f2(__uint_as_float(sv[h][c]), __uint_as_float(sv[h][c + 1])), scl, nmu));
+          const float p0 = fast_exp2(xa.x), p1 = fast_exp2(xa.y);
+          acc = add_f2(acc, f2(p0, p1));
+          pk[16 * h + c / 2] = pack_bf16(p0, p1);
+        }
+      const float2 accf = f2_unpack(acc);
+      const float ls = accf.x + accf.y;
+      lsum += ls;
+      if (n > 0 && !mbar_wait(pvdone, (n - 1) & 1)) fail = 1;  // the P V MMA of tile n-1 is done
+      tc_fence_after();
+      tmem_st32x32b_x32(tmem + T_P + 32 * ch + ((uint32_t)(32 * sp) << 16), pk);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(pfull);
+    };
+
+    build(0);
+    for (int i = 0; i < N; ++i) {
+      bar_sync(PBAR_CW, 32 * PNC);  // anchors of tile i+1 are in place
+      if (i + 1 < N) build(i + 1);
+      softmax(i);
+      if (tid < D / 2 && i + 2 < N) {
+        const float2 cs = rope_cs_exact((int64_t)(i + 2) * PKT, theta[tid]);
+        anc[(i & 1) * 64 + tid] = make_float2(cs.x * p.s, cs.y * p.s);
+      }
+    }
+
+    // ---- epilogue: out = (O + s O_lr B_v^a) / l for this warp's 64 columns
+    if (!mbar_wait(pvdone, (N - 1) & 1)) fail = 1;
+    if (!mbar_wait(bvbar, 0)) fail = 1;
+    tc_fence_after();
+    float* lx = xch + (N & 1) * 256;  // the exchange buffer the last softmax did not use
+    lx[w * 32 + lane] = lsum;
+    bar_sync(PBAR_PAIR + sp, 64);
+    const float l = lsum + lx[(w ^ 4) * 32 + lane];
+    const float inv_l = l > 0.f ? 1.f / l : 0.f;
+    uint32_t olr[32];
+    tmem_ld32x32b_x32(olr, tmem + T_OL + ((uint32_t)(32 * sp) << 16) + (C::LRW > 32 ? 32 : 0));
+    tmem_wait_ld_r32(olr);
+    const int lro = C::LRW > 32 ? R - 32 : R;   // column of O_lr's value part in olr
+    const int head = kvh * g + row % g;
+    const int64_t obase = (((int64_t)seq * na + agent) * p.n_q_tokens + tok0 + rtok) * p.n_q + head;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t ov[32];
+      tmem_ld32x32b_x32(ov, tmem + T_O + 64 * ch + 32 * h + ((uint32_t)(32 * sp) << 16));
+      tmem_wait_ld_r32(ov);
+      float z[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) z[c] = 0.f;
+#pragma unroll
+      for (int j = 0; j < R; ++j) {
+        const float o = __uint_as_float(olr[lro + j]);
+        const __nv_bfloat16* brow = bvs + j * D + 64 * ch + 32 * h;
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          const float2 bb = unpack_bf16(*reinterpret_cast<const uint32_t*>(brow + c));
+          z[c] = fmaf(o, bb.x, z[c]);
+          z[c + 1] = fmaf(o, bb.y, z[c + 1]);
+        }
+      }
+      if (rvalid) {
+        const int64_t oi = obase * D + 64 * ch + 32 * h;
+        if (p.out_bf16) {
+          uint32_t* o = reinterpret_cast<uint32_t*>(reinterpret_cast<__nv_bfloat16*>(p.out) + oi);
+#pragma unroll
+          for (int c = 0; c < 32; c += 2)
+            o[c / 2] = pack_bf16(fmaf(p.s, z[c], __uint_as_float(ov[c])) * inv_l,
+                                 fmaf(p.s, z[c + 1], __uint_as_float(ov[c + 1])) * inv_l);
+        } else {
+          float4* o = reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + oi);
+#pragma unroll
+          for (int c = 0; c < 32; c += 4)
+            o[c / 4] = make_float4(fmaf(p.s, z[c], __uint_as_float(ov[c])) * inv_l,
+                                   fmaf(p.s, z[c + 1], __uint_as_float(ov[c + 1])) * inv_l,
+                                   fmaf(p.s, z[c + 2], __uint_as_float(ov[c + 2])) * inv_l,
+                                   fmaf(p.s, z[c + 3], __uint_as_float(ov[c + 3])) * inv_l);
+        }
+      }
+    }
+  }
+  if (fail) s_fail = 1;
+  tc_fence_before();
+  __syncthreads();
+  if (w == PNC) {
+    tc_fence_after();
+    tmem_dealloc(tmem, T_COLS);
+  }
+  if (s_fail && tid == 0) atomicOr(p.err, 2);
+}
+
+// ------------------------------------------------------------------ host
+bool prefill_maps(const AttnParams& p, CUtensorMap* mq, CUtensorMap* mk, CUtensorMap* mv,
+                  CUtensorMap* ml, CUtensorMap* mb) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  const int D = PD, R = p.r, g = p.g;
+  cuuint32_t one[4] = {1, 1, 1, 1};
+  // queries [n_seqs * n_agents][n_tok][n_q][d]: boxes of 64 columns x g heads x 128/g tokens
+  cuuint64_t qd[4] = {(cuuint64_t)D, (cuuint64_t)p.n_q, (cuuint64_t)p.n_q_tokens,
+                      (cuuint64_t)p.n_seqs * p.n_agents};
+  cuuint64_t qs[3] = {(cuuint64_t)D * 2, (cuuint64_t)p.n_q * D * 2,
+                      (cuuint64_t)p.n_q_tokens * p.n_q * D * 2};
+  cuuint32_t qb[4] = {64, (cuuint32_t)g, (cuuint32_t)(PM / g), 1};
+  if (enc(mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(p.q), qd, qs, qb, one,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  cuuint64_t kd[4] = {(cuuint64_t)D, (cuuint64_t)p.L_max, (cuuint64_t)p.n_kv, (cuuint64_t)p.n_seqs};
+  cuuint64_t ks[3] = {(cuuint64_t)p.kv_tok * 2, (cuuint64_t)p.kv_head * 2, (cuuint64_t)p.kv_seq * 2};
+  cuuint32_t kb[4] = {64, (cuuint32_t)PKT, 1, 1};
+  if (enc(mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(p.k_base), kd, ks, kb, one,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  if (enc(mv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(p.v_base), kd, ks, kb, one,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  const int lb = 2 * R < 64 ? 2 * R : 64;
+  cuuint64_t ld[3] = {(cuuint64_t)(2 * R), (cuuint64_t)p.L_max, (cuuint64_t)p.n_seqs};
+  cuuint64_t ls[2] = {(cuuint64_t)(2 * R * 2), (cuuint64_t)p.lr_seq * 2};
+  cuuint32_t lbx[3] = {(cuuint32_t)lb, (cuuint32_t)PKT, 1};
+  if (enc(ml, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(p.lr), ld, ls, lbx, one,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(lb * 2), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  // B_k as (n_kv * d, r, n_agents): r x 64 slices of one head
+  cuuint64_t bd[3] = {(cuuint64_t)p.n_kv * D, (cuuint64_t)R, (cuuint64_t)p.n_agents};
+  cuuint64_t bs[2] = {(cuuint64_t)p.n_kv * D * 2, (cuuint64_t)R * p.n_kv * D * 2};
+  cuuint32_t bb[3] = {64, (cuuint32_t)R, 1};
+  if (enc(mb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(p.B_k), bd, bs, bb, one,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  return true;
+}
+
+template <int R>
+cudaError_t launch_prefill_tc(const AttnParams& p, cudaStream_t st) {
+  using C = PCfg<R>;
+  RopeTheta rt;
+  for (int i = 0; i < 64; ++i) rt.theta[i] = std::pow(p.rope_base, -2.0 * i / PD);
+  CUtensorMap mq, mk, mv, ml, mb;
+  if (!prefill_maps(p, &mq, &mk, &mv, &ml, &mb)) return cudaErrorInvalidValue;
+  auto kern = prefill_tc_kernel<R>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+  if (e != cudaSuccess) return e;
+  const int QB = PM / p.g;
+  dim3 grid((p.n_q_tokens + QB - 1) / QB, p.n_agents * p.n_kv, p.n_seqs);
+  kern<<<grid, PNTHR, C::SMEM, st>>>(mq, mk, mv, ml, mb, p, rt);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool bf16_prefill_supported(const AttnParams& p) {
+  if (p.d != PD || p.r != 16) return false;
+  if (!(p.g == 1 || p.g == 2 || p.g == 4 || p.g == 8)) return false;
+  if (p.L_max >= (1ll << 31) || p.n_q_tokens < 1) return false;
+  if ((int64_t)p.n_agents * p.n_kv > 65535 || p.n_seqs > 65535) return false;
+  return PCfg<16>::SMEM <= 227 * 1024;
+}
+
+cudaError_t launch_prefill_bf16(const AttnParams& pin, la_dtype out, cudaStream_t st) {
+  AttnParams p = pin;
+  p.out_bf16 = out == LA_BF16;
+  return launch_prefill_tc<16>(p, st);
+}
+
+}  // namespace la

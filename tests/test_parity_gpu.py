@@ -258,6 +258,80 @@ def test_bf16_prefill_small(la, L, n_tok, r, n_agents):
     assert_parity(to_np(got), ref, s.dtype)
 
 
+def _prefill_vs_oracle(la, s, inp, out_dtype=None):
+    dd = to_device(inp)
+    got = _run(la, s, dd["k_base"], dd["v_base"], dd["lr"], dd["B_k"], dd["B_v"], dd["q"],
+               out_dtype=out_dtype)
+    ref = oracle.lora_attention(inp["k_base"], inp["v_base"], inp["lr"], inp["B_k"], inp["B_v"],
+                                inp["q"], inp["kv_len"], lora_scale=s.lora_scale,
+                                softmax_scale=s.softmax_scale, rope_base=s.rope_base,
+                                mode="prefill")
+    return assert_parity(to_np(got.float()), ref, s.dtype)
+
+
+@pytest.mark.parametrize("n_q,n_kv,L,n_tok,n_seqs", [
+    (32, 8, 200, 200, 1),     # g = 4, self-attention of a fresh chunk (q_pos0 = 0), ragged block
+    (32, 4, 700, 45, 2),      # g = 8: 16 tokens per block, two sequences
+    (8, 8, 390, 260, 1),      # g = 1: 128 tokens per block, chunk over a prefix
+    (16, 8, 129, 64, 1),      # g = 2, one key past a tile
+    (32, 8, 100, 1, 1),       # one query token, one partial tile
+])
+def test_bf16_prefill_tensor_core_shapes(la, n_q, n_kv, L, n_tok, n_seqs):
+    """The tcgen05 prefill (r = 16): GQA groups 1..8, blocks cut by the chunk's
+    end, keys cut inside a tile, several sequences."""
+    s = W.LLAMA8B_PREFILL_16K.replace(n_q_heads=n_q, n_kv_heads=n_kv, kv_len=L, n_q_tokens=n_tok,
+                                      n_seqs=n_seqs, seed=400 + L)
+    _prefill_vs_oracle(la, s, W.direct_cache_inputs(s))
+
+
+def test_bf16_prefill_bf16_output(la):
+    s = W.LLAMA8B_PREFILL_16K.replace(kv_len=333, n_q_tokens=96, seed=77)
+    _prefill_vs_oracle(la, s, W.direct_cache_inputs(s), out_dtype=torch.bfloat16)
+
+
+def _ramped_keys(s, inp, lo, hi):
+    ramp = torch.linspace(lo, hi, s.kv_len).view(1, 1, -1, 1)
+    inp["k_base"] = (inp["k_base"].float() * ramp).to(torch.bfloat16)
+    return inp
+
+
+def test_bf16_prefill_growing_scores(la):
+    """Keys whose scale grows tenfold along the sequence move every row's
+    maximum up by many units of log2: the lazy rescale of O and l engages
+    repeatedly.  Exact oracle."""
+    s = W.LLAMA8B_PREFILL_16K.replace(kv_len=1200, n_q_tokens=128, seed=78)
+    _prefill_vs_oracle(la, s, _ramped_keys(s, W.direct_cache_inputs(s), 0.25, 2.5))
+
+
+def test_bf16_prefill_growing_scores_bf16_keys(la):
+    """A thirtyfold ramp.  The tensor cores take each agent's keys
+    K^a = K_base + RoPE(s LRk B_k^a) rounded to bf16, an error that grows with
+    |K| (at six times the configs' key scale it alone exceeds the 1e-2 bound),
+    so here the reference applies that one rounding to the oracle's K^a and
+    the comparison isolates the online softmax and its rescaling."""
+    s = W.LLAMA8B_PREFILL_16K.replace(kv_len=1200, n_q_tokens=128, seed=79)
+    inp = _ramped_keys(s, W.direct_cache_inputs(s), 0.2, 6.0)
+    dd = to_device(inp)
+    got = to_np(_run(la, s, dd["k_base"], dd["v_base"], dd["lr"], dd["B_k"], dd["B_v"], dd["q"]))
+    g, d, r = s.group, s.head_dim, s.r
+    qpos = oracle.query_positions(s.kv_len, s.n_q_tokens, "prefill")
+    kpos = np.arange(s.kv_len)
+    lr = to_np(inp["lr"][0])
+    ref = np.empty_like(got)
+    for a in range(s.n_agents):
+        for kvh in range(s.n_kv_heads):
+            cols = slice(kvh * d, (kvh + 1) * d)
+            Ka = oracle.agent_keys(inp["k_base"][0, kvh], lr[:, :r], to_np(inp["B_k"][a])[:, cols],
+                                   s.lora_scale, kpos, s.rope_base)
+            Ka = to_np(torch.from_numpy(Ka).to(torch.bfloat16))
+            Va = oracle.agent_values(inp["v_base"][0, kvh], lr[:, r:], to_np(inp["B_v"][a])[:, cols],
+                                     s.lora_scale)
+            for h in range(kvh * g, (kvh + 1) * g):
+                ref[0, a, :, h] = oracle.attention(to_np(inp["q"][0, a, :, h]), Ka, Va,
+                                                   s.softmax_scale, qpos, kpos)
+    assert_parity(got, ref, s.dtype)
+
+
 def _sampled_units(la, s, inp, got, units, tokens):
     """Compare sampled (seq, agent, kv head) x query tokens against the oracle."""
     g = s.group
