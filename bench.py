@@ -43,8 +43,10 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--profile", action="store_true",
-                    help="only run the decode kernel a few times on one cache set (for ncu)")
+    ap.add_argument("--profile", nargs="?", const="decode", choices=["decode", "prefill"],
+                    help="a short deterministic run of one kernel for profilers "
+                         "(decode: the 8192-token decode five times; prefill: the "
+                         "16384 + 1024-token prefill three times); prints nothing")
     return ap.parse_args()
 
 
@@ -55,6 +57,65 @@ def peaks():
         return float(p["hbm_gbs"]), "measured"
     except Exception:
         return 6650.0, "fallback"
+
+
+def tc_peak():
+    """Dense bf16 tensor-core peak (TFLOP/s) for a kernel timed on its own."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured cuBLAS bf16 burst"
+    except Exception:
+        return 1590.0, "fallback"
+
+
+def prefill_flops(s):
+    """4 d flops per unmasked (query, key) pair (Q K^T and P V), plus the
+    LoRA-inclusive count: 2 r per pair for P LR_v, 2 r d per (agent, KV head,
+    key) for the key delta, 2 r d per query row for the epilogue."""
+    pairs = s.n_agents * s.n_q_heads * sum(s.q_pos0 + j + 1 for j in range(s.n_q_tokens))
+    base = 4 * s.head_dim * pairs
+    keys = s.n_agents * s.n_kv_heads * (s.q_pos0 + s.n_q_tokens)
+    lora = 2 * s.r * pairs + 2 * s.r * s.head_dim * keys + \
+        2 * s.r * s.head_dim * s.n_agents * s.n_q_heads * s.n_q_tokens
+    return base, base + lora
+
+
+def time_prefill(dev, reps=5, warmup=3):
+    """The chunked prefill workload (16384-token prefix + 1024-token chunk per
+    agent, 3 agents, r = 16): one lora_attn_prefill per launch, CUDA events
+    around each launch, L2 flushed (256 MB written) before each."""
+    import torch
+    from rank_attention_b200 import lora_attn as la
+    from rank_attention_b200 import workloads as W
+    s = W.LLAMA8B_PREFILL_16K
+    inp = W.direct_cache_inputs(s, device=dev)
+    out = torch.empty(inp["q"].shape, dtype=torch.bfloat16, device=dev)
+    args = la.make_args(inp["k_base"], inp["v_base"], inp["lr"], inp["B_k"], inp["B_v"],
+                        inp["q"], out, lora_scale=s.lora_scale, rope_base=s.rope_base,
+                        q_pos0=s.q_pos0)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(warmup):
+        la.lora_attn_prefill(args)
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(reps):
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        la.lora_attn_prefill(args)
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    if la.la_device_check() != 0:
+        raise RuntimeError("prefill device check failed")
+    ms = statistics.median(times)
+    base, lora = prefill_flops(s)
+    peak, kind = tc_peak()
+    tf = base / (ms / 1e3) / 1e12
+    return {"workload": s.name, "value": tf, "unit": "TFLOP/s", "ms": ms,
+            "flops_per_launch": base, "lora_inclusive_tflops": lora / (ms / 1e3) / 1e12,
+            "peak": peak, "peak_kind": kind, "frac": tf / peak, "out_dtype": "bf16",
+            "timing": f"median of {reps} launches, CUDA events, L2 flushed before each"}
 
 
 class ClockSampler:
@@ -127,21 +188,28 @@ def decode_kernels_per_call(s) -> int:
     return 2 if splits > 1 else 1
 
 
-def run_profile():
-    """A short, deterministic run of the decode kernel alone, for profilers."""
+def run_profile(kind: str = "decode"):
+    """A short, deterministic run of one kernel alone, for profilers."""
     import torch
     from rank_attention_b200 import lora_attn as la
     from rank_attention_b200 import workloads as W
-    s = W.LLAMA8B_DECODE_8K
     dev = torch.device("cuda", 0)
+    s = W.LLAMA8B_DECODE_8K if kind == "decode" else W.LLAMA8B_PREFILL_16K
     inp = {k: v.to(dev) for k, v in W.direct_cache_inputs(s, device=dev).items()}
     out = torch.empty(inp["q"].shape, dtype=torch.float32, device=dev)
-    args = la.make_args(inp["k_base"], inp["v_base"], inp["lr"], inp["B_k"], inp["B_v"], inp["q"],
-                        out, lora_scale=s.lora_scale, rope_base=s.rope_base,
-                        kv_len=inp["kv_len"], max_kv_len=s.kv_len)
-    ws = la.decode_workspace(args, dev)
-    for _ in range(5):
-        la.lora_attn_decode(args, ws)
+    if kind == "decode":
+        args = la.make_args(inp["k_base"], inp["v_base"], inp["lr"], inp["B_k"], inp["B_v"],
+                            inp["q"], out, lora_scale=s.lora_scale, rope_base=s.rope_base,
+                            kv_len=inp["kv_len"], max_kv_len=s.kv_len)
+        ws = la.decode_workspace(args, dev)
+        for _ in range(5):
+            la.lora_attn_decode(args, ws)
+    else:
+        args = la.make_args(inp["k_base"], inp["v_base"], inp["lr"], inp["B_k"], inp["B_v"],
+                            inp["q"], out, lora_scale=s.lora_scale, rope_base=s.rope_base,
+                            q_pos0=s.q_pos0)
+        for _ in range(3):
+            la.lora_attn_prefill(args)
     torch.cuda.synchronize()
     return 0 if la.la_device_check() == 0 else 1
 
@@ -386,6 +454,8 @@ def run_ours(args):
     e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     e2e_value = whole_job_rate(s.n_seqs * s.n_agents, e_steps, world, e_ms)
 
+    prefill = time_prefill(dev)
+
     hbm, peak_kind = peaks()
     dbytes = decode_bytes(s)
     achieved = dbytes / (dec_ms / 1e3) / 1e9
@@ -408,6 +478,7 @@ def run_ours(args):
                 "d2h_bytes_per_step": d2h, "steps": e_steps},
         "gpu_launches": (1 + decode_kernels_per_call(s)) * args.steps,
         "clocks": clk,
+        "prefill": prefill,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, n, per = time_oracle(s, 20, 15.0)
@@ -427,7 +498,7 @@ def main():
     if args.impl == "reference":
         return run_reference(args)
     if args.profile:
-        return run_profile()
+        return run_profile(args.profile)
     return run_ours(args)
 
 
