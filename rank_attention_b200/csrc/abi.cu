@@ -24,7 +24,7 @@ size_t simt_rows_cap(const AttnParams& p);
 int simt_key_tile();
 bool bf16_decode_supported(const AttnParams& p);
 size_t bf16_decode_partial_bytes(const AttnParams& p);
-void bf16_decode_plan(const AttnParams& p, int* n_splits, int64_t* split_len, int* rows);
+void bf16_decode_plan(const AttnParams& p, int* n_splits, int64_t* split_len, int* rows, int* groups);
 cudaError_t launch_decode_bf16(const AttnParams& p, la_dtype out, cudaStream_t st);
 bool bf16_prefill_supported(const AttnParams& p);
 cudaError_t launch_prefill_bf16(const AttnParams& p, la_dtype out, cudaStream_t st);
@@ -113,9 +113,10 @@ DecodePlan plan_decode(const AttnParams& p, la_dtype io) {
   const int units = p.n_seqs * p.n_kv;
   if (io == LA_BF16 && bf16_decode_supported(p)) {
     d.kind = 1;
-    bf16_decode_plan(p, &d.n_splits, &d.split_len, &d.rows);
+    bf16_decode_plan(p, &d.n_splits, &d.split_len, &d.rows, &d.groups);
   } else {
     d.kind = 0;
+    d.groups = 1;
     const int tk = simt_key_tile();
     const int64_t max_tiles = (p.max_kv_len + tk - 1) / tk;
     int64_t want = (2 * kNumSMs + units - 1) / (units > 0 ? units : 1);
@@ -133,7 +134,7 @@ DecodePlan plan_decode(const AttnParams& p, la_dtype io) {
     d.partial_bytes = d.n_splits > 1 ? (size_t)units * d.n_splits * d.rows * W * sizeof(float) : 0;
   d.partial_bytes = (d.partial_bytes + 255) / 256 * 256;
   // per unit: an arrival and a departure counter of the split merge
-  d.counter_bytes = ((size_t)2 * units * sizeof(int) + 255) / 256 * 256;
+  d.counter_bytes = ((size_t)2 * units * d.groups * sizeof(int) + 255) / 256 * 256;
   return d;
 }
 

@@ -706,9 +706,9 @@ struct TCfg {
   // LR tile: rows of 2r bf16 in boxes of min(2r, 64); its swizzle span
   static constexpr int LR_ROWB = (2 * R < 64 ? 2 * R : 64) * 2;
   static constexpr uint32_t LR_LAYOUT = LR_ROWB == 128 ? 2u : (LR_ROWB == 64 ? 4u : 6u);
-  static size_t smem(int n_agents) {
+  static size_t smem(int n_agents) {  // n_agents: the agents of one CTA
     return 1024 + AREA + 2 * P_TILE + align1k(SMALL) + QU_BYTES + 2 * QP_BYTES +
-           (size_t)align1k(BK_BYTES) * n_agents + (size_t)BK_BYTES * n_agents + 128;
+           (size_t)align1k(BK_BYTES) * n_agents + 128;
   }
 };
 
@@ -762,18 +762,23 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
   unsigned char* qu = ptile + 2 * C::P_TILE + align1k(C::SMALL);  // Q (MMA operand)
   unsigned char* qpb0 = qu + C::QU_BYTES;                          // Q'[2]
   unsigned char* bks = qpb0 + 2 * C::QP_BYTES;
-  unsigned char* bvs = bks + (size_t)align1k(C::BK_BYTES) * p.n_agents;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(bvs + (size_t)C::BK_BYTES * p.n_agents);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(bks + (size_t)align1k(C::BK_BYTES) * p.agent_group);
   __shared__ int s_fail;
 
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int gq = lane >> 2, t4 = lane & 3;
   const int mi = lane >> 3, rr = lane & 7;
-  const int unit = blockIdx.y;
+  const int unit = blockIdx.z;
   const int seq = unit / p.n_kv, kvh = unit % p.n_kv;
   const int split = blockIdx.x;
   const int ns = p.n_splits;
-  const int g = p.g, na = p.n_agents, n_rows = na * g;
+  // this CTA's agents: group blockIdx.y of p.agent_group agents (the groups of a
+  // unit are adjacent in launch order, so its cache tiles are read from HBM once
+  // and are L2 hits for the other groups)
+  const int agent0 = blockIdx.y * p.agent_group;
+  const int g = p.g, na = min(p.agent_group, p.n_agents - agent0), n_rows = na * g;
+  const int na_tot = p.n_agents;
+  const int unitg = blockIdx.y * (p.n_seqs * p.n_kv) + unit;   // (agent group, unit)
 
   const int64_t total_tiles = (p.max_kv_len + KT - 1) / KT;
   const int64_t tb = split * total_tiles / ns;
@@ -785,12 +790,10 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
   const uint32_t qu_u = smem_u32(qu);
   const uint32_t qp_u = smem_u32(qpb0);
   const uint32_t bks_u = smem_u32(bks);
-  const uint32_t bvs_u = smem_u32(bvs);
   const uint32_t full_u = smem_u32(bars);          // [ST]
   const uint32_t empty_u = full_u + 8 * ST;        // [ST]: MMA commit + value warps
   const uint32_t tfull = full_u + 16 * ST;         // MMA results of a tile are in TMEM
   const uint32_t tempty = tfull + 8;               // score warps are done reading TMEM
-  const uint32_t bvbar = tfull + 16;
   const uint32_t bkbar = tfull + 24;              // B_k^a slices have landed
   const uint32_t qbar = tfull + 32;               // the queries have landed (staged unswizzled)
   const int64_t ldB = (int64_t)p.n_kv * D;
@@ -822,7 +825,6 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
     }
     mbar_init(tfull, 1);
     mbar_init(tempty, TC_NES);
-    mbar_init(bvbar, 1);
     mbar_init(bkbar, 1);
     mbar_init(qbar, 1);
     fence_mbar_init();
@@ -830,7 +832,7 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
     const __nv_bfloat16* Q = reinterpret_cast<const __nv_bfloat16*>(p.q);
     mbar_expect_tx(qbar, (uint32_t)(n_rows * D * 2));
     for (int a = 0; a < na; ++a)
-      bulk_load(ptile_u + a * g * D * 2, Q + (((int64_t)seq * na + a) * p.n_q + kvh * g) * D,
+      bulk_load(ptile_u + a * g * D * 2, Q + (((int64_t)seq * na_tot + agent0 + a) * p.n_q + kvh * g) * D,
                 (uint32_t)(g * D * 2), qbar);
     tma_prefetch(&tmB);
     tma_prefetch(&tmK);
@@ -841,14 +843,10 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
     for (int a = 0; a < na; ++a)
 #pragma unroll
       for (int b = 0; b < D / 64; ++b)
-        tma_load_3d(bks_u + a * align1k(C::BK_BYTES) + b * R * 128, &tmB, bkbar, kvh * D + 64 * b, 0, a);
+        tma_load_3d(bks_u + a * align1k(C::BK_BYTES) + b * R * 128, &tmB, bkbar, kvh * D + 64 * b, 0, agent0 + a);
     // the first stages before kv_len is known: tiles of this split's range
     // (by max_kv_len) past the sequence's length are loaded but never used
     for (int n = 0; n < n_spec; ++n) issue(n);
-    const __nv_bfloat16* Bv = reinterpret_cast<const __nv_bfloat16*>(p.B_v);
-    mbar_expect_tx(bvbar, (uint32_t)(na * C::BK_BYTES));
-    for (int i = 0; i < na * R; ++i)
-      bulk_load(bvs_u + i * D * 2, Bv + (int64_t)i * ldB + kvh * D, D * 2, bvbar);
   }
   const int64_t kvl = p.kv_len[seq];  // in flight while the constants are computed
   const int sp = w & 3, kb = 32 * sp + 16 * (w >> 2);  // score warp: TMEM sub-partition, first key
@@ -885,7 +883,6 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
     if (w == TC_NES + NPV && lane == 0) {  // the copies in flight land before the CTA leaves
       mbar_wait(qbar, 0);
       mbar_wait(bkbar, 0);
-      mbar_wait(bvbar, 0);
       for (int n = 0; n < n_spec; ++n) mbar_wait(full_u + 8 * n, 0);
     }
     return;
@@ -1210,6 +1207,20 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
       constexpr uint32_t ID_S = umma_idesc_bf16(128, QPAD, 0, 0);
       constexpr uint32_t ID_E = umma_idesc_bf16(128, D, 0, 1);
       if (n_tiles > 0 && !mbar_wait(bkbar, 0)) fail = 1;
+      // the split's later tiles stream into L2 from here on (the queries and the
+      // first stages were requested first), so that HBM stays busy between
+      // stage refills
+      for (int m = ST; m < n_tiles; ++m) {
+        const int key0 = (int)(k_lo + (int64_t)m * KT);
+#pragma unroll
+        for (int b = 0; b < D / 64; ++b) {
+          tma_prefetch_l2_4d(&tmK, 64 * b, key0, kvh, seq);
+          tma_prefetch_l2_4d(&tmV, 64 * b, key0, kvh, seq);
+        }
+        constexpr int LB = (2 * R) < 64 ? 2 * R : 64;
+#pragma unroll
+        for (int b = 0; b < (2 * R) / LB; ++b) tma_prefetch_l2_3d(&tmL, LB * b, key0, seq);
+      }
       for (int n = 0; n < n_tiles; ++n) {
         const int s = n % ST;
         const uint32_t sK = area_u + s * C::STAGE;
@@ -1235,21 +1246,6 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
         }
         umma_commit(tfull);
         umma_commit(empty_u + 8 * s);  // K and LRk of this stage have been read
-        if (n == 0) {
-          // the split's later tiles stream into L2 from here on (after the first
-          // loads have landed), so that HBM stays busy between stage refills
-          for (int m = ST; m < te - tb; ++m) {
-            const int key0 = (int)(k_lo + (int64_t)m * KT);
-#pragma unroll
-            for (int b = 0; b < D / 64; ++b) {
-              tma_prefetch_l2_4d(&tmK, 64 * b, key0, kvh, seq);
-              tma_prefetch_l2_4d(&tmV, 64 * b, key0, kvh, seq);
-            }
-            constexpr int LB = (2 * R) < 64 ? 2 * R : 64;
-#pragma unroll
-            for (int b = 0; b < (2 * R) / LB; ++b) tma_prefetch_l2_3d(&tmL, LB * b, key0, seq);
-          }
-        }
         if (n >= 1 && n - 1 + ST < n_tiles) {
           const int sp = (n - 1) % ST;
           if (!mbar_wait(empty_u + 8 * sp, ((n - 1) / ST) & 1)) fail = 1;
@@ -1263,7 +1259,6 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
     bar_sync(BAR_END, TC_NTHR);
   }
   if (fail) s_fail = 1;
-  if (!mbar_wait(bvbar, 0)) s_fail = 1;
   if (!mbar_wait(bkbar, 0)) s_fail = 1;
   __syncthreads();
   if (w == TC_NES + NPV) {
@@ -1278,15 +1273,15 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
     Mo[row * W + D + R + 1] = l;
   }
   if (ns == 1) {  // Z = O_base + s O_lr B_v^a (with split keys the merge applies B_v^a once)
-    const __nv_bfloat16* bv = reinterpret_cast<const __nv_bfloat16*>(bvs);
+    const __nv_bfloat16* bv = reinterpret_cast<const __nv_bfloat16*>(p.B_v) + (int64_t)agent0 * R * ldB + kvh * D;
     for (int i = tid; i < n_rows * (D / 4); i += TC_NTHR) {
       const int row = i / (D / 4), c = 4 * (i % (D / 4));
-      const __nv_bfloat16* b = bv + (size_t)(row / g) * R * D + c;
+      const __nv_bfloat16* b = bv + (size_t)(row / g) * R * ldB + c;
       float z0 = 0.f, z1 = 0.f, z2 = 0.f, z3 = 0.f;
 #pragma unroll
       for (int j = 0; j < R; ++j) {
         const float o = Mo[row * W + D + j];
-        const uint2 bb = *reinterpret_cast<const uint2*>(b + j * D);
+        const uint2 bb = __ldg(reinterpret_cast<const uint2*>(b + j * ldB));
         const float2 f01 = unpack_bf16(bb.x), f23 = unpack_bf16(bb.y);
         z0 = fmaf(o, f01.x, z0); z1 = fmaf(o, f01.y, z1);
         z2 = fmaf(o, f23.x, z2); z3 = fmaf(o, f23.y, z3);
@@ -1307,7 +1302,7 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
       const int a = row / g, gi = row % g;
       const float l = Mo[row * W + D + R + 1];
       const float val = l > 0.f ? Mo[row * W + c] / l : 0.f;
-      const int64_t oi = (((int64_t)seq * na + a) * p.n_q + kvh * g + gi) * D + c;
+      const int64_t oi = (((int64_t)seq * na_tot + agent0 + a) * p.n_q + kvh * g + gi) * D + c;
       if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(val);
       else reinterpret_cast<float*>(p.out)[oi] = val;
     }
@@ -1321,14 +1316,14 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
   //   out = sum_k w_k O_base,k + s (sum_k w_k O_lr,k) B_v^a,
   // B_v^a applied once per row (it is linear, so it commutes with the merge).
   // A CTA that failed still arrives, so the others never wait for it.
-  float* ws_unit = p.partials + (size_t)unit * ns * n_rows * W;
+  float* ws_unit = p.partials + (size_t)unitg * ns * (p.agent_group * g) * W;
   {
     float* part = ws_unit + (size_t)split * n_rows * W;
     for (int i = tid; i < n_rows * (W / 4); i += TC_NTHR)
       reinterpret_cast<float4*>(part)[i] = reinterpret_cast<const float4*>(Mo)[i];
   }
-  int* arrive = p.counters + unit;
-  int* depart = p.counters + p.n_seqs * p.n_kv + unit;
+  int* arrive = p.counters + unitg;
+  int* depart = p.counters + gridDim.y * (p.n_seqs * p.n_kv) + unitg;
   __threadfence();
   __syncthreads();
   if (tid == 0) {
@@ -1383,7 +1378,7 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
     float mx = ml.x;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    const float e = (lane < ns && ml.x != -INFINITY) ? exp2f(ml.x - mx) : 0.f;
+    const float e = (lane < ns && ml.x != -INFINITY) ? fast_exp2(ml.x - mx) : 0.f;
     float lt = e * ml.y;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) lt += __shfl_xor_sync(0xffffffffu, lt, o);
@@ -1430,7 +1425,7 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
   __syncthreads();
   // (e) out = sum over subsets + s O_lr B_v^a
   {
-    const __nv_bfloat16* bv = reinterpret_cast<const __nv_bfloat16*>(bvs);
+    const __nv_bfloat16* bv = reinterpret_cast<const __nv_bfloat16*>(p.B_v) + (int64_t)agent0 * R * ldB + kvh * D;
     for (int i = tid; i < ni; i += TC_NTHR) {
       float4 acc = red[i];
       for (int sub = 1; sub < ks; ++sub) {
@@ -1440,19 +1435,19 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
       const int item = ib + i, row = item / CH, c = 4 * (item % CH);
       const int a = row / g, gi = row % g;
       const float* ol = Ol + (row - rb) * R;
-      const __nv_bfloat16* bb = bv + (size_t)a * R * D + c;
+      const __nv_bfloat16* bb = bv + (size_t)a * R * ldB + c;
       float z0 = 0.f, z1 = 0.f, z2 = 0.f, z3 = 0.f;
 #pragma unroll
       for (int j = 0; j < R; ++j) {
         const float o = ol[j];
-        const uint2 b2 = *reinterpret_cast<const uint2*>(bb + j * D);
+        const uint2 b2 = __ldg(reinterpret_cast<const uint2*>(bb + j * ldB));
         const float2 f01 = unpack_bf16(b2.x), f23 = unpack_bf16(b2.y);
         z0 = fmaf(o, f01.x, z0); z1 = fmaf(o, f01.y, z1);
         z2 = fmaf(o, f23.x, z2); z3 = fmaf(o, f23.y, z3);
       }
       acc.x = fmaf(p.s, z0, acc.x); acc.y = fmaf(p.s, z1, acc.y);
       acc.z = fmaf(p.s, z2, acc.z); acc.w = fmaf(p.s, z3, acc.w);
-      const int64_t oi = (((int64_t)seq * na + a) * p.n_q + kvh * g + gi) * D + c;
+      const int64_t oi = (((int64_t)seq * na_tot + agent0 + a) * p.n_q + kvh * g + gi) * D + c;
       if (p.out_bf16) {
         uint2 o;
         o.x = pack_bf16(acc.x, acc.y);
@@ -1525,16 +1520,30 @@ int device_sms() {
   return n;
 }
 
-// splits of each (sequence, KV head) over the keys: enough CTAs to cover the
-// SMs once (one CTA per SM), so that a split launch is always fully resident
+bool tc_fits(const AttnParams& p, int G);
+int tc_group_size(const AttnParams& p);
+
+// agent groups of the tensor-core decode (each CTA holds one group), else 1
+int decode_groups(const AttnParams& p) {
+  const int G = tc_group_size(p);
+  return G > 0 ? (p.n_agents + G - 1) / G : 1;
+}
+
+// splits of each (sequence, KV head, agent group) over the keys: enough CTAs
+// to cover the SMs once (one CTA per SM), so that a split launch is always
+// fully resident
 int n_splits_for(const AttnParams& p) {
-  const int units = p.n_seqs * p.n_kv;
+  const int units = p.n_seqs * p.n_kv * decode_groups(p);
   const int64_t total_tiles = (p.max_kv_len + KT - 1) / KT;
   const int sms = device_sms();
   int64_t ns = units >= sms ? 1 : sms / units;
   if (ns > kMaxSplits) ns = kMaxSplits;
   if (ns > total_tiles) ns = total_tiles;
   if (ns < 1) ns = 1;
+  // as few splits as give the same longest split: the split with the most tiles
+  // sets the time, fewer splits mean less to merge
+  const int64_t per = (total_tiles + ns - 1) / ns;
+  ns = (total_tiles + per - 1) / per;
   return (int)ns;
 }
 
@@ -1569,21 +1578,36 @@ cudaError_t launch_t(const AttnParams& p, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-bool tc_supported(const AttnParams& p) {
-  if (p.d != 128 || !(p.r == 16 || p.r == 32 || p.r == 64)) return false;
-  if (!(p.g == 1 || p.g == 2 || p.g == 4 || p.g == 8)) return false;
-  if (p.n_agents > 3) return false;                     // TMEM: 128 columns per agent + scores
-  const int NT = n_rowtiles(p);
+// the tensor-core decode with G agents per CTA: TMEM holds G key deltas of
+// 128 columns and the scores; rows G g in at most three m16 row tiles; shared
+// memory within 227 KB
+bool tc_fits(const AttnParams& p, int G) {
+  if (G < 1 || G > 3) return false;
+  const int NT = (G * p.g + 7) / 8;
   if (NT > 3) return false;
-  if (p.L_max >= (1ll << 31)) return false;
   size_t sm = 0;
   switch (p.r) {
-    case 16: sm = NT == 1 ? TCfg<128, 16, 1>::smem(p.n_agents) : NT == 2 ? TCfg<128, 16, 2>::smem(p.n_agents) : TCfg<128, 16, 3>::smem(p.n_agents); break;
-    case 32: sm = NT == 1 ? TCfg<128, 32, 1>::smem(p.n_agents) : NT == 2 ? TCfg<128, 32, 2>::smem(p.n_agents) : TCfg<128, 32, 3>::smem(p.n_agents); break;
-    default: sm = NT == 1 ? TCfg<128, 64, 1>::smem(p.n_agents) : NT == 2 ? TCfg<128, 64, 2>::smem(p.n_agents) : TCfg<128, 64, 3>::smem(p.n_agents); break;
+    case 16: sm = NT == 1 ? TCfg<128, 16, 1>::smem(G) : NT == 2 ? TCfg<128, 16, 2>::smem(G) : TCfg<128, 16, 3>::smem(G); break;
+    case 32: sm = NT == 1 ? TCfg<128, 32, 1>::smem(G) : NT == 2 ? TCfg<128, 32, 2>::smem(G) : TCfg<128, 32, 3>::smem(G); break;
+    default: sm = NT == 1 ? TCfg<128, 64, 1>::smem(G) : NT == 2 ? TCfg<128, 64, 2>::smem(G) : TCfg<128, 64, 3>::smem(G); break;
   }
   return sm <= 227 * 1024;
 }
+
+// agents per CTA of the tensor-core decode (0: the shape does not run on it).
+// The largest group that fits: more agents per CTA read the shared caches
+// fewer times; the groups of a launch run side by side, so a cache tile read
+// by one group is mostly an L2 hit for the others.
+int tc_group_size(const AttnParams& p) {
+  if (p.d != 128 || !(p.r == 16 || p.r == 32 || p.r == 64)) return 0;
+  if (!(p.g == 1 || p.g == 2 || p.g == 4 || p.g == 8)) return 0;
+  if (p.L_max >= (1ll << 31)) return 0;
+  for (int G = p.n_agents < 3 ? p.n_agents : 3; G >= 1; --G)
+    if (tc_fits(p, G)) return G;
+  return 0;
+}
+
+bool tc_supported(const AttnParams& p) { return tc_group_size(p) > 0; }
 
 template <int D, int R, int NT>
 cudaError_t launch_tc(const AttnParams& p, cudaStream_t st) {
@@ -1603,11 +1627,11 @@ cudaError_t launch_tc(const AttnParams& p, cudaStream_t st) {
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  const size_t sm = C::smem(p.n_agents);
+  const size_t sm = C::smem(p.agent_group);
   auto kern = decode_tc_kernel<D, R, NT>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.n_splits, p.n_seqs * p.n_kv);
+  dim3 grid(p.n_splits, (p.n_agents + p.agent_group - 1) / p.agent_group, p.n_seqs * p.n_kv);
   // with split keys the unit's CTAs wait for one another: all must be resident
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
@@ -1638,29 +1662,35 @@ bool bf16_decode_supported(const AttnParams& p) {
   return true;
 }
 
-void bf16_decode_plan(const AttnParams& p, int* n_splits, int64_t* split_len, int* rows) {
+void bf16_decode_plan(const AttnParams& p, int* n_splits, int64_t* split_len, int* rows, int* groups) {
+  const int G = tc_group_size(p);
   *n_splits = n_splits_for(p);
   *split_len = KT;
-  *rows = p.n_agents * p.g;
+  *rows = (G > 0 ? G : p.n_agents) * p.g;
+  *groups = decode_groups(p);
 }
 
 size_t bf16_decode_partial_bytes(const AttnParams& p) {
   const int ns = n_splits_for(p);
   if (ns == 1) return 0;
-  return (size_t)p.n_seqs * p.n_kv * ns * (p.n_agents * p.g) * (p.d + p.r + 4) * sizeof(float);
+  const int G = tc_group_size(p);
+  const int rows = (G > 0 ? G : p.n_agents) * p.g;
+  return (size_t)p.n_seqs * p.n_kv * decode_groups(p) * ns * rows * (p.d + p.r + 4) * sizeof(float);
 }
 
 cudaError_t launch_decode_bf16(const AttnParams& pin, la_dtype out, cudaStream_t st) {
   AttnParams p = pin;
   p.out_bf16 = out == LA_BF16;
-  const int NT = n_rowtiles(p);
-  if (tc_supported(p)) {
+  p.agent_group = tc_group_size(p);
+  if (p.agent_group > 0) {
+    const int NT = (p.agent_group * p.g + 7) / 8;
     switch (p.r) {
       case 16: return NT == 1 ? launch_tc<128, 16, 1>(p, st) : NT == 2 ? launch_tc<128, 16, 2>(p, st) : launch_tc<128, 16, 3>(p, st);
       case 32: return NT == 1 ? launch_tc<128, 32, 1>(p, st) : NT == 2 ? launch_tc<128, 32, 2>(p, st) : launch_tc<128, 32, 3>(p, st);
       default: return NT == 1 ? launch_tc<128, 64, 1>(p, st) : NT == 2 ? launch_tc<128, 64, 2>(p, st) : launch_tc<128, 64, 3>(p, st);
     }
   }
+  const int NT = n_rowtiles(p);
   switch (p.r) {
     case 8: return NT == 1 ? launch_t<128, 8, 1>(p, st) : NT == 2 ? launch_t<128, 8, 2>(p, st) : launch_t<128, 8, 3>(p, st);
     case 16: return NT == 1 ? launch_t<128, 16, 1>(p, st) : NT == 2 ? launch_t<128, 16, 2>(p, st) : launch_t<128, 16, 3>(p, st);

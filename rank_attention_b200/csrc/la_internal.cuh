@@ -41,6 +41,7 @@ struct AttnParams {
   int* counters;           // [units]
   int* err;                // device error word
   int out_bf16;            // tensor-core kernels: 1 = bf16 outputs, 0 = fp32
+  int agent_group;         // tensor-core decode: agents per CTA (grid z runs over the groups)
 };
 
 // Device error word of the library (address on the current device).
@@ -63,6 +64,7 @@ struct DecodePlan {
   int rows;                // rows per unit
   size_t partial_bytes;
   size_t counter_bytes;
+  int groups;              // agent groups of the tensor-core decode (1 otherwise)
 };
 
 // ---------------------------------------------------------------------------

@@ -187,6 +187,23 @@ def test_bf16_decode_ragged(la, r, n_agents, d, lens):
     assert_parity(to_np(got), oracle_decode(inp, s), s.dtype)
 
 
+@pytest.mark.parametrize("r,n_agents,n_q,L,n_seqs,out_bf16", [
+    (16, 5, 32, 3000, 1, False),   # groups of 3 + 2 agents, keys split over CTAs
+    (64, 4, 32, 2000, 1, True),    # r = 64: one agent per CTA, four groups
+    (32, 7, 16, 1500, 2, False),   # g = 2: groups of 3 + 3 + 1, two sequences
+])
+def test_bf16_decode_agent_groups(la, r, n_agents, n_q, L, n_seqs, out_bf16):
+    """More agents than one CTA holds: the agents are split into groups that run
+    side by side, each with its own split merge."""
+    s = W.LLAMA8B_DECODE_8K.replace(n_seqs=n_seqs, n_agents=n_agents, n_q_heads=n_q, r=r,
+                                    alpha=2.0 * r, kv_len=L, seed=90 + n_agents)
+    inp = W.direct_cache_inputs(s)
+    dd = to_device(inp)
+    got = _run(la, s, dd["k_base"], dd["v_base"], dd["lr"], dd["B_k"], dd["B_v"], dd["q"],
+               dd["kv_len"], out_dtype=torch.bfloat16 if out_bf16 else None)
+    assert_parity(to_np(got.float()), oracle_decode(inp, s), s.dtype)
+
+
 def test_bf16_decode_token_major_layout(la):
     """Base cache stored [seq][token][head][d]: same result as head-major."""
     s = W.LLAMA8B_DECODE_8K.replace(kv_len=777, n_seqs=2, seed=21)
