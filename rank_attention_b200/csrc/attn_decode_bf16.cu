@@ -1,35 +1,40 @@
 // Flash-LoRA-Attention decode on the tensor cores (bf16 storage, fp32 accumulate).
 //
-// One CTA = one (sequence, KV head, split of the keys); the splits of a
-// (sequence, KV head) form one thread-block cluster.  A CTA's rows are every
-// agent x every query head of the GQA group, so each base and LR tile is read
-// from HBM once for all agents (LRAgent summary §3 BaseLRShared: one base and
-// one LR cache shared by the whole system).  128-key tiles of K_base, V_base
-// and the LR rows are staged in shared memory by TMA (128/64/32-byte swizzle,
-// no multicast) through a two-stage full/empty mbarrier pipeline.
+// Two kernels share this file.
 //
-// Warp roles (320 threads):
-//  * 8 score warps, 16 keys each.  Key side (LRAgent summary App. D.1: RoPE
-//    blocks the reordering, so the delta is rebuilt in head dimension).  A key
-//    at position t = k0 + j of a tile starting at k0 is rotated by
+// decode_tc_kernel (the main path).  One CTA = one (sequence, KV head, agent
+// group, split of the keys).  Its rows are the group's agents x the query
+// heads of the GQA group, so each base and LR tile is read from HBM once for
+// all of them (LRAgent summary §3 BaseLRShared: one base and one LR cache
+// shared by the whole system).  128-key tiles of K_base, V_base and the LR
+// rows are staged in shared memory by TMA (128/64/32-byte swizzle, no
+// multicast) through a two-stage full/empty mbarrier pipeline.
+//  * Warp 10 issues the TMA loads and, per tile, the tcgen05 MMAs (M = 128
+//    keys): the base scores S_base^T = K_base Q^T for every row, and each
+//    agent's key delta dK^a = LRk B_k^a (N = d, K = r), all into TMEM.
+//  * 8 score warps, 16 keys each (LRAgent summary App. D.1: RoPE blocks the
+//    reordering, so the delta is rebuilt in head dimension).  A key at
+//    position t = k0 + j of a tile starting at k0 is rotated by
 //    R(t) = R(k0) R(j), so
 //      q . K^a_t = q . K_base,t + (s R(-k0) q) . R(j) (LRk_t B_k^a):
-//    the base scores are one MMA over all agents' rows, the delta dK = LRk B_k^a
-//    is an MMA per agent (M = 16 keys, N = d, K = r) turned in registers by
+//    dK^a comes out of TMEM in the mma.sync fragment layout, is turned by
 //    R(j) -- whose cos / sin are per-thread constants, j being fixed per
-//    thread -- and scored against the tile's rotated queries Q' = s R(-k0) Q.
-//    Two agents are interleaved for ILP.  The tile's row maxima meet in
-//    shared memory; the warps write P^T (bf16) and the rescale factors.
+//    thread -- and scored (mma.sync) against the tile's rotated queries
+//    Q' = s R(-k0) Q.  The tile's row maxima meet in shared memory; the warps
+//    write P^T (bf16) and the rescale factors.
 //  * 2 value warps own O_base^T (half of d each) and O_lr^T: value side
 //    reordered (LRAgent explainer, Metodologia 3; summary App. B),
 //    O_base^T += V_base^T P^T and O_lr^T += LRv^T P^T, so the LoRA value path
-//    stays r wide inside the loop.  They also rotate the queries for the next
-//    tile and refill the pipeline.
-// Epilogue: each CTA applies B_v^a once per row to its partial,
-// Z = O_base + s O_lr B_v^a (linear, so it commutes with the merge).  With one
-// split the CTA writes out = Z / l; otherwise it writes (Z, m, l) to the
-// workspace and a small merge kernel, chained by programmatic dependent launch,
-// forms out = sum_k w_k Z_k / sum_k w_k l_k with w_k = 2^(m_k - max m).
+//    stays r wide inside the loop.  They also rotate the queries per tile.
+//  Split keys merge inside the same launch: each CTA writes (O_base, O_lr, m,
+//  l), the unit's CTAs wait for one another (cooperative launch, bounded
+//  wait), and each merges a share of the unit's rows, applying B_v^a once per
+//  row: out = (sum_k w_k O_base,k + s (sum_k w_k O_lr,k) B_v^a) with
+//  w_k = 2^(m_k - M) / sum_k 2^(m_k - M) l_k.
+//
+// decode_bf16_kernel + decode_merge_kernel (shapes the first kernel does not
+// take: d = 64, r = 8).  The same tiling with mma.sync for every product and a
+// second kernel, chained by programmatic dependent launch, for the merge.
 #include <cudaTypedefs.h>
 
 #include <cmath>
