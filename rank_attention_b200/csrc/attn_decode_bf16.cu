@@ -865,7 +865,7 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
         const int i = 16 * grp + 8 * q + 2 * t4;
-        const float th0 = (float)rt.theta[i], th1 = (float)rt.theta[i + 1];
+        const float th0 = rt.thetaf[i], th1 = rt.thetaf[i + 1];
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           const float j = (float)(kb + gq + 8 * hh);
@@ -1556,7 +1556,10 @@ template <int D, int R, int NT>
 cudaError_t launch_t(const AttnParams& p, cudaStream_t st) {
   using C = Cfg<D, R, NT>;
   RopeTheta rt;
-  for (int i = 0; i < 64; ++i) rt.theta[i] = i < D / 2 ? std::pow(p.rope_base, -2.0 * i / D) : 0.0;
+  for (int i = 0; i < 64; ++i) {
+    rt.theta[i] = i < D / 2 ? std::pow(p.rope_base, -2.0 * i / D) : 0.0;
+    rt.thetaf[i] = (float)rt.theta[i];
+  }
   CUtensorMap mk, mv, ml;
   if (!make_maps(p, &mk, &mv, &ml)) return cudaErrorInvalidValue;
   const size_t sm = C::smem(p.n_agents);
@@ -1618,7 +1621,10 @@ template <int D, int R, int NT>
 cudaError_t launch_tc(const AttnParams& p, cudaStream_t st) {
   using C = TCfg<D, R, NT>;
   RopeTheta rt;
-  for (int i = 0; i < 64; ++i) rt.theta[i] = i < D / 2 ? std::pow(p.rope_base, -2.0 * i / D) : 0.0;
+  for (int i = 0; i < 64; ++i) {
+    rt.theta[i] = i < D / 2 ? std::pow(p.rope_base, -2.0 * i / D) : 0.0;
+    rt.thetaf[i] = (float)rt.theta[i];
+  }
   CUtensorMap mk, mv, ml, mb;
   if (!make_maps(p, &mk, &mv, &ml)) return cudaErrorInvalidValue;
   {

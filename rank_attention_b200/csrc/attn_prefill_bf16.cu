@@ -182,7 +182,7 @@ __global__ void __launch_bounds__(PNTHR, 1)
 #pragma unroll
       for (int q = 0; q < 2; ++q) {
         const int i = 16 * grp + 8 * q + 2 * t4;
-        const float th0 = (float)rt.theta[i], th1 = (float)rt.theta[i + 1];
+        const float th0 = rt.thetaf[i], th1 = rt.thetaf[i + 1];
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           const float j = (float)(kb + gq + 8 * hh);
@@ -543,7 +543,10 @@ template <int R>
 cudaError_t launch_prefill_tc(const AttnParams& p, cudaStream_t st) {
   using C = PCfg<R>;
   RopeTheta rt;
-  for (int i = 0; i < 64; ++i) rt.theta[i] = std::pow(p.rope_base, -2.0 * i / PD);
+  for (int i = 0; i < 64; ++i) {
+    rt.theta[i] = std::pow(p.rope_base, -2.0 * i / PD);
+    rt.thetaf[i] = (float)rt.theta[i];
+  }
   CUtensorMap mq, mk, mv, ml, mb;
   if (!prefill_maps(p, &mq, &mk, &mv, &ml, &mb)) return cudaErrorInvalidValue;
   auto kern = prefill_tc_kernel<R>;

@@ -16,6 +16,7 @@ constexpr int align1k(int x) { return (x + 1023) / 1024 * 1024; }
 // RoPE frequencies theta_i = base^(-2i/d), formed in fp64 on the host
 struct RopeTheta {
   double theta[64];
+  float thetaf[64];   // the same, rounded to fp32 (small in-tile angles)
 };
 
 // (cos, sin) of t * theta, the angle formed and reduced modulo 2 pi in fp64
