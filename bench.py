@@ -80,6 +80,85 @@ def prefill_flops(s):
     return base, base + lora
 
 
+def non_shared_setup(la, s, inp, dev):
+    """The non-shared baseline of one decode step: every agent's K^a, V^a
+    materialised (lora_materialize_agent_kv), then plain attention over the
+    per-agent caches -- the same decode kernel with n_seqs * n_agents
+    sequences of one agent and B = 0, so it reads n_agents x the base cache.
+    Returns (materialise, decode, outputs [n_seqs, n_agents, 1, n_q, d])."""
+    import torch
+    n, na, nkv, d, r = s.n_seqs, s.n_agents, s.n_kv_heads, s.head_dim, s.r
+    L = inp["k_base"].shape[2]
+    kout = torch.empty((n, na, nkv, L, d), dtype=inp["k_base"].dtype, device=dev)
+    vout = torch.empty_like(kout)
+    q = inp["q"]
+    out = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    margs = la.make_args(inp["k_base"], inp["v_base"], inp["lr"], inp["B_k"], inp["B_v"], q, out,
+                         lora_scale=s.lora_scale, rope_base=s.rope_base, kv_len=inp["kv_len"],
+                         max_kv_len=int(s.kv_len))
+    zlr = torch.zeros((n * na, L, 2 * r), dtype=inp["lr"].dtype, device=dev)
+    zb = torch.zeros((1, r, nkv * d), dtype=inp["B_k"].dtype, device=dev)
+    kv_len = inp["kv_len"].repeat_interleave(na)
+    q1 = q.reshape(n * na, 1, q.shape[2], q.shape[3], d)
+    out1 = out.view(n * na, 1, q.shape[2], q.shape[3], d)
+    dargs = la.make_args(kout.view(n * na, nkv, L, d), vout.view(n * na, nkv, L, d), zlr, zb, zb,
+                         q1, out1, lora_scale=s.lora_scale, rope_base=s.rope_base, kv_len=kv_len,
+                         max_kv_len=int(s.kv_len))
+    ws = la.decode_workspace(dargs, dev)
+    keep = (kout, vout, zlr, zb, kv_len, q1, out1, ws)
+
+    def materialise(stream=None):
+        la.lora_materialize_agent_kv(margs, kout, vout, stream)
+
+    def decode(stream=None):
+        la.lora_attn_decode(dargs, ws, stream)
+
+    materialise.keep = keep
+    return materialise, decode, out
+
+
+def time_non_shared(dev, shared_decode_us, reps=5):
+    """Time the non-shared baseline on the decode workload (L2 flushed before
+    each timed launch) and report its bytes beside the shared path's."""
+    import torch
+    from rank_attention_b200 import lora_attn as la
+    from rank_attention_b200 import workloads as W
+    s = W.LLAMA8B_DECODE_8K
+    inp = W.direct_cache_inputs(s, device=dev)
+    mat, dec, _ = non_shared_setup(la, s, inp, dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    mat()
+    dec()
+    torch.cuda.synchronize()
+
+    def timed(fn):
+        ts = []
+        for _ in range(reps):
+            flush.fill_(1)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return statistics.median(ts) * 1e3
+
+    mat_us, dec_us = timed(mat), timed(dec)
+    if la.la_device_check() != 0:
+        raise RuntimeError("non-shared baseline device check failed")
+    shared = decode_bytes(s)
+    e = 2
+    ns_bytes = (2 * s.n_seqs * s.n_agents * s.n_kv_heads * s.kv_len * s.head_dim * e
+                + s.n_seqs * s.n_agents * s.n_q_heads * s.head_dim * (e + 4))
+    return {"workload": s.name, "decode_us": dec_us, "materialise_us": mat_us,
+            "bytes_per_decode": ns_bytes, "shared_bytes_per_decode": shared,
+            "bytes_saved_frac": 1.0 - shared / ns_bytes,
+            "shared_speedup": dec_us / shared_decode_us,
+            "what": "per-agent K^a, V^a materialised once (materialise_us, not per step), then "
+                    "attention over n_agents separate caches (decode_us): the same decode kernel "
+                    "with B = 0"}
+
+
 def time_prefill(dev, reps=5, warmup=3):
     """The chunked prefill workload (16384-token prefix + 1024-token chunk per
     agent, 3 agents, r = 16): one lora_attn_prefill per launch, CUDA events
@@ -455,6 +534,7 @@ def run_ours(args):
     e2e_value = whole_job_rate(s.n_seqs * s.n_agents, e_steps, world, e_ms)
 
     prefill = time_prefill(dev)
+    non_shared = time_non_shared(dev, dec_ms * 1e3)
 
     hbm, peak_kind = peaks()
     dbytes = decode_bytes(s)
@@ -479,6 +559,7 @@ def run_ours(args):
         "gpu_launches": (1 + decode_kernels_per_call(s)) * args.steps,
         "clocks": clk,
         "prefill": prefill,
+        "non_shared_baseline": non_shared,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, n, per = time_oracle(s, 20, 15.0)

@@ -191,6 +191,26 @@ size_t lora_attn_decode_workspace_bytes(const la_attn_args* args);
  *     (lora_attn_decode_workspace_bytes(args) > LA_STATIC_SCRATCH_BYTES), it
  *     returns LA_ERR_SCRATCH_LIMIT before launching anything.
  */
+/*
+ * lora_materialize_agent_kv -- the non-shared baseline's caches.
+ *
+ * Writes every agent's full keys and values
+ *   K^a_t = K_base_t + RoPE_t(s LRk_t B_k^a),  V^a_t = V_base_t + s LRv_t B_v^a
+ * for positions [0, max_kv_len) of every sequence and KV head: what a system
+ * without cache sharing keeps per agent (LRAgent summary §3, Non-Shared).
+ * Attention over them (lora_attn_decode with n_seqs * n_agents sequences of
+ * one agent and B = 0) reads n_agents times the base cache; the library's
+ * shared path never writes these.  It exists to measure that baseline.
+ *
+ * args: as for lora_attn_decode (q, out and the workspace are not used).
+ * k_out, v_out: device, [n_seqs][n_agents][n_kv_heads][L_max][head_dim],
+ *   contiguous, io_dtype; rows at or past max_kv_len are not written.
+ * Errors: as lora_attn_decode's argument errors, and LA_ERR_INVALID_ARG for
+ * a null or misaligned k_out / v_out.
+ */
+la_status lora_materialize_agent_kv(const la_attn_args* args, void* k_out, void* v_out,
+                                    la_stream_t stream);
+
 #define LA_STATIC_SCRATCH_BYTES ((size_t)4 << 20)
 la_status lora_attn_decode_static_scratch(const la_attn_args* args, la_stream_t stream);
 

@@ -246,6 +246,18 @@ extern "C" la_status lora_attn_prefill(const la_attn_args* a, la_stream_t stream
   return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
 }
 
+extern "C" la_status lora_materialize_agent_kv(const la_attn_args* a, void* k_out, void* v_out,
+                                               la_stream_t stream) {
+  AttnParams p;
+  la_status s = check_attn(a, 1, &p);
+  if (s != LA_OK) return s;
+  if (!k_out || !v_out || !aligned16(k_out) || !aligned16(v_out)) return LA_ERR_INVALID_ARG;
+  if (p.n_seqs == 0) return LA_OK;
+  if (p.n_seqs > 65535 || (p.max_kv_len + 3) / 4 > 0x7fffffff) return LA_ERR_UNSUPPORTED;
+  cudaError_t e = launch_materialize(p, a->io_dtype, k_out, v_out, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
 extern "C" la_status la_device_check(void) {
   if (cudaDeviceSynchronize() != cudaSuccess) return LA_ERR_CUDA;
   int* ptr = error_word_ptr();

@@ -55,6 +55,7 @@ cudaError_t launch_append_bf16_mma(const void* X, int64_t ldx, int64_t n, int64_
                                    const void* A, int r, void* lr, int64_t pos0, int n_seqs,
                                    int64_t sx, int64_t slr, cudaStream_t st);
 cudaError_t launch_attn_simt(const AttnParams& p, la_dtype io, la_dtype out, cudaStream_t st);
+cudaError_t launch_materialize(const AttnParams& p, la_dtype io, void* kout, void* vout, cudaStream_t st);
 
 // Decode split-K plan shared by the workspace query and the launch.
 struct DecodePlan {

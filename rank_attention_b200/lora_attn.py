@@ -25,7 +25,7 @@ LA_F32, LA_BF16 = 0, 1
 
 EXPORTED = ("la_status_string", "lr_cache_append", "lora_attn_prefill", "lora_attn_decode",
             "lora_attn_decode_workspace_bytes", "la_device_check",
-            "lora_attn_decode_static_scratch")
+            "lora_attn_decode_static_scratch", "lora_materialize_agent_kv")
 
 
 class LoraAttnError(RuntimeError):
@@ -81,6 +81,9 @@ def _load() -> ctypes.CDLL:
     lib.la_device_check.argtypes = []
     lib.lora_attn_decode_static_scratch.restype = ctypes.c_int
     lib.lora_attn_decode_static_scratch.argtypes = [ctypes.POINTER(AttnArgs), ctypes.c_void_p]
+    lib.lora_materialize_agent_kv.restype = ctypes.c_int
+    lib.lora_materialize_agent_kv.argtypes = [ctypes.POINTER(AttnArgs), ctypes.c_void_p,
+                                              ctypes.c_void_p, ctypes.c_void_p]
     return lib
 
 
@@ -184,6 +187,16 @@ def lora_attn_decode_static_scratch(args: AttnArgs, stream=None) -> None:
     array (for callers that cannot allocate device memory; see the header)."""
     st = lib.lora_attn_decode_static_scratch(ctypes.byref(args), _stream(stream))
     _check(st, "lora_attn_decode_static_scratch")
+
+
+def lora_materialize_agent_kv(args: AttnArgs, k_out: torch.Tensor, v_out: torch.Tensor,
+                              stream=None) -> None:
+    """Every agent's full K^a, V^a ([n_seqs, n_agents, n_kv, L_max, d] each): the
+    non-shared baseline's caches (see the header)."""
+    assert k_out.is_contiguous() and v_out.is_contiguous()
+    st = lib.lora_materialize_agent_kv(ctypes.byref(args), k_out.data_ptr(), v_out.data_ptr(),
+                                       _stream(stream))
+    _check(st, "lora_materialize_agent_kv")
 
 
 def lora_attn_prefill(args: AttnArgs, stream=None) -> None:

@@ -384,3 +384,38 @@ def test_llama8b_sweep_decode_sampled(la, ctx):
     got = _run(la, s, dd["k_base"], dd["v_base"], dd["lr"], dd["B_k"], dd["B_v"], dd["q"],
                dd["kv_len"]).cpu()
     _sampled_units(la, s, inp, got, [(0, 0, 0), (5, 4, 7), (15, 2, 3)], np.array([0]))
+
+
+# ------------------------------------------------------ non-shared baseline ----
+def test_materialized_agent_caches_and_non_shared_decode(la):
+    """The non-shared baseline: every agent's K^a, V^a written out equal the
+    oracle's materialised caches (one bf16 rounding), and plain attention over
+    them gives the shared path's outputs."""
+    import bench
+    s = W.LLAMA8B_DECODE_8K.replace(kv_len=700, n_seqs=2, seed=55)
+    inp = W.direct_cache_inputs(s)
+    dd = to_device(inp)
+    mat, dec, out_ns = bench.non_shared_setup(la, s, dd, DEV)
+    mat()
+    kout, vout = mat.keep[0].cpu(), mat.keep[1].cpu()
+    d, r = s.head_dim, s.r
+    kpos = np.arange(s.kv_len)
+    for seq in range(s.n_seqs):
+        lr = to_np(inp["lr"][seq])
+        for a in range(s.n_agents):
+            for j in (0, s.n_kv_heads - 1):
+                cols = slice(j * d, (j + 1) * d)
+                Ka = oracle.agent_keys(inp["k_base"][seq, j], lr[:, :r], to_np(inp["B_k"][a])[:, cols],
+                                       s.lora_scale, kpos, s.rope_base)
+                Va = oracle.agent_values(inp["v_base"][seq, j], lr[:, r:], to_np(inp["B_v"][a])[:, cols],
+                                         s.lora_scale)
+                for got, ref in ((kout[seq, a, j, :s.kv_len], Ka), (vout[seq, a, j, :s.kv_len], Va)):
+                    err = np.abs(to_np(got) - ref)
+                    assert (err <= bf16_ulp(ref) + 1e-3 * np.abs(ref).max()).all(), err.max()
+    dec()
+    torch.cuda.synchronize()
+    assert la.la_device_check() == 0
+    shared = _run(la, s, dd["k_base"], dd["v_base"], dd["lr"], dd["B_k"], dd["B_v"], dd["q"],
+                  dd["kv_len"])
+    assert_parity(to_np(out_ns), oracle_decode(inp, s), s.dtype)
+    assert_parity(to_np(out_ns), to_np(shared), s.dtype)
