@@ -48,18 +48,20 @@ constexpr int PBAR_CW = 1, PBAR_PAIR = 2;  // PBAR_PAIR + sub-partition: the two
 
 template <int R>
 struct PCfg {
-  static constexpr int LRW = 2 * R;                            // LR row, elements
-  static constexpr int LR_ROWB = (LRW < 64 ? LRW : 64) * 2;     // bytes per LR box row
+  // a K stage holds the K_base tile and the tile's LRk columns, a V stage the
+  // V_base tile and its LRv columns: r columns of the LR rows, one TMA box
+  static constexpr int LR_ROWB = R * 2;                         // bytes per LRk / LRv row
   static constexpr uint32_t LR_LAYOUT = LR_ROWB == 128 ? 2u : (LR_ROWB == 64 ? 4u : 6u);
   static constexpr int KV = PKT * PD * 2;                       // a K or V tile
-  static constexpr int LR_TILE = align1k(PKT * LRW * 2);
-  static constexpr int STAGE = KV + LR_TILE;                    // K (or V) tile + LR rows
+  static constexpr int LR_TILE = align1k(PKT * R * 2);
+  static constexpr int STAGE = KV + LR_TILE;
+  static constexpr int NV = R >= 64 ? 1 : 2;                    // V stages (one at r = 64: room)
   static constexpr int Q_BYTES = PM * PD * 2;
   static constexpr int B_BYTES = R * PD * 2;
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + Q_BYTES;                 // [2] stages
-  static constexpr int OFF_V = OFF_K + 2 * STAGE;               // [2] stages
-  static constexpr int OFF_BK = OFF_V + 2 * STAGE;
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;                 // [2] K stages
+  static constexpr int OFF_V = OFF_K + 2 * STAGE;               // [NV] V stages
+  static constexpr int OFF_BK = OFF_V + NV * STAGE;
   static constexpr int OFF_BV = OFF_BK + align1k(B_BYTES);
   static constexpr int OFF_MISC = OFF_BV + align1k(B_BYTES);
   // misc: anchors [2][64] float2, exchange [2][8][32] float, theta [64] double,
@@ -113,18 +115,16 @@ __global__ void __launch_bounds__(PNTHR, 1)
   const int64_t kend = qmin + ntok;                    // keys [0, kend)
   const int N = (int)((kend + PKT - 1) / PKT);
 
-  auto load_stage = [&](const CUtensorMap* m, uint32_t base, uint32_t bar, int n) {
+  // lr_col: 0 for the LRk columns (with K), r for LRv (with V)
+  auto load_stage = [&](const CUtensorMap* m, uint32_t base, uint32_t bar, int n, int lr_col) {
     const int key0 = n * PKT;
-    mbar_expect_tx(bar, (uint32_t)(C::KV + PKT * C::LRW * 2));
+    mbar_expect_tx(bar, (uint32_t)(C::KV + PKT * R * 2));
 #pragma unroll
     for (int b = 0; b < D / 64; ++b) tma_load_4d(base + b * PKT * 128, m, bar, 64 * b, key0, kvh, seq);
-    constexpr int LB = C::LR_ROWB / 2;
-#pragma unroll
-    for (int b = 0; b < C::LRW / LB; ++b)
-      tma_load_3d(base + C::KV + b * PKT * C::LR_ROWB, &tmL, bar, LB * b, key0, seq);
+    tma_load_3d(base + C::KV, &tmL, bar, lr_col, key0, seq);
   };
-  auto load_k = [&](int n) { load_stage(&tmK, k_u + (n & 1) * C::STAGE, kfull(n & 1), n); };
-  auto load_v = [&](int n) { load_stage(&tmV, v_u + (n & 1) * C::STAGE, vfull(n & 1), n); };
+  auto load_k = [&](int n) { load_stage(&tmK, k_u + (n & 1) * C::STAGE, kfull(n & 1), n, 0); };
+  auto load_v = [&](int n) { load_stage(&tmV, v_u + (n % C::NV) * C::STAGE, vfull(n % C::NV), n, R); };
 
   if (w == PNC && lane == 0) {
     s_fail = 0;
@@ -160,7 +160,7 @@ __global__ void __launch_bounds__(PNTHR, 1)
     load_v(0);
     if (N > 1) {
       load_k(1);
-      load_v(1);
+      if (C::NV > 1) load_v(1);
     }
     const __nv_bfloat16* Bv = reinterpret_cast<const __nv_bfloat16*>(p.B_v);
     mbar_expect_tx(bvbar, (uint32_t)C::B_BYTES);
@@ -210,7 +210,7 @@ __global__ void __launch_bounds__(PNTHR, 1)
       constexpr uint32_t ID_DK = umma_idesc_bf16(128, PD, 0, 1);
       constexpr uint32_t ID_S = umma_idesc_bf16(128, PKT, 0, 0);
       constexpr uint32_t ID_PV = umma_idesc_bf16(128, PD, 0, 1);
-      constexpr uint32_t ID_PL = umma_idesc_bf16(128, C::LRW, 0, 1);
+      constexpr uint32_t ID_PL = umma_idesc_bf16(128, R, 0, 1);
       auto mma_dk = [&](int n) {  // dK = LRk B_k^a
         if (!mbar_wait(kfull(n & 1), (n >> 1) & 1)) fail = 1;
         tc_fence_after();
@@ -223,9 +223,9 @@ __global__ void __launch_bounds__(PNTHR, 1)
       };
       auto mma_pv = [&](int n) {  // O += P V_base, O_lr += P LR
         if (!mbar_wait(pfull, n & 1)) fail = 1;
-        if (!mbar_wait(vfull(n & 1), (n >> 1) & 1)) fail = 1;
+        if (!mbar_wait(vfull(n % C::NV), (n / C::NV) & 1)) fail = 1;
         tc_fence_after();
-        const uint32_t vs = v_u + (n & 1) * C::STAGE;
+        const uint32_t vs = v_u + (n % C::NV) * C::STAGE;
 #pragma unroll
         for (int ks = 0; ks < PKT / 16; ++ks)
           umma_bf16_ts(tmem + T_O, tmem + T_P + ks * 8, umma_desc(vs + ks * 16 * 128, PKT * 128, 1024, 2),
@@ -237,7 +237,7 @@ __global__ void __launch_bounds__(PNTHR, 1)
                                  C::LR_LAYOUT),
                        ID_PL, (n > 0 || ks > 0) ? 1u : 0u);
         umma_commit(pvdone);
-        umma_commit(vempty(n & 1));
+        umma_commit(vempty(n % C::NV));
       };
       if (!mbar_wait(qbar, 0)) fail = 1;
       mma_dk(0);
@@ -258,9 +258,9 @@ __global__ void __launch_bounds__(PNTHR, 1)
           if (!mbar_wait(kempty(n & 1), (n >> 1) & 1)) fail = 1;
           load_k(n + 2);
         }
-        if (n > 0 && n + 1 < N) {
-          if (!mbar_wait(vempty((n - 1) & 1), ((n - 1) >> 1) & 1)) fail = 1;
-          load_v(n + 1);
+        if (n > 0 && n - 1 + C::NV < N) {  // V stage of tile n-1 is free once its P V is done
+          if (!mbar_wait(vempty((n - 1) % C::NV), ((n - 1) / C::NV) & 1)) fail = 1;
+          load_v(n - 1 + C::NV);
         }
       }
       mma_pv(N - 1);
@@ -377,7 +377,7 @@ __global__ void __launch_bounds__(PNTHR, 1)
           if (ch == 0) {
             const uint32_t tol = tmem + T_OL + ((uint32_t)(32 * sp) << 16);
 #pragma unroll 1
-            for (int h = 0; h < C::LRW / 16; ++h) {
+            for (int h = 0; h < R / 16; ++h) {
               uint32_t ov[16];
               tmem_ld32x32b_x16(ov, tol + 16 * h);
               tmem_wait_ld_r16(ov);
@@ -437,10 +437,15 @@ __global__ void __launch_bounds__(PNTHR, 1)
     bar_sync(PBAR_PAIR + sp, 64);
     const float l = lsum + lx[(w ^ 4) * 32 + lane];
     const float inv_l = l > 0.f ? 1.f / l : 0.f;
-    uint32_t olr[32];
-    tmem_ld32x32b_x32(olr, tmem + T_OL + ((uint32_t)(32 * sp) << 16) + (C::LRW > 32 ? 32 : 0));
-    tmem_wait_ld_r32(olr);
-    const int lro = C::LRW > 32 ? R - 32 : R;   // column of O_lr's value part in olr
+    uint32_t olr[R];   // P LRv, this thread's row
+#pragma unroll
+    for (int h = 0; h < R / 16; ++h) {
+      uint32_t t16[16];
+      tmem_ld32x32b_x16(t16, tmem + T_OL + 16 * h + ((uint32_t)(32 * sp) << 16));
+      tmem_wait_ld_r16(t16);
+#pragma unroll
+      for (int c = 0; c < 16; ++c) olr[16 * h + c] = t16[c];
+    }
     const int head = kvh * g + row % g;
     const int64_t obase = (((int64_t)seq * na + agent) * p.n_q_tokens + tok0 + rtok) * p.n_q + head;
 #pragma unroll
@@ -453,7 +458,7 @@ __global__ void __launch_bounds__(PNTHR, 1)
       for (int c = 0; c < 32; ++c) z[c] = 0.f;
 #pragma unroll
       for (int j = 0; j < R; ++j) {
-        const float o = __uint_as_float(olr[lro + j]);
+        const float o = __uint_as_float(olr[j]);
         const __nv_bfloat16* brow = bvs + j * D + 64 * ch + 32 * h;
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
@@ -520,12 +525,12 @@ bool prefill_maps(const AttnParams& p, CUtensorMap* mq, CUtensorMap* mk, CUtenso
           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return false;
-  const int lb = 2 * R < 64 ? 2 * R : 64;
+  // LR rows [2r]: boxes of r columns (LRk at column 0, LRv at column r)
   cuuint64_t ld[3] = {(cuuint64_t)(2 * R), (cuuint64_t)p.L_max, (cuuint64_t)p.n_seqs};
   cuuint64_t ls[2] = {(cuuint64_t)(2 * R * 2), (cuuint64_t)p.lr_seq * 2};
-  cuuint32_t lbx[3] = {(cuuint32_t)lb, (cuuint32_t)PKT, 1};
+  cuuint32_t lbx[3] = {(cuuint32_t)R, (cuuint32_t)PKT, 1};
   if (enc(ml, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(p.lr), ld, ls, lbx, one,
-          CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(lb * 2), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(R * 2), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return false;
   // B_k as (n_kv * d, r, n_agents): r x 64 slices of one head
@@ -561,17 +566,22 @@ cudaError_t launch_prefill_tc(const AttnParams& p, cudaStream_t st) {
 }  // namespace
 
 bool bf16_prefill_supported(const AttnParams& p) {
-  if (p.d != PD || p.r != 16) return false;
+  // r = 8 would make the P LRv MMA N = 8, below the M = 128 minimum of 16
+  if (p.d != PD || !(p.r == 16 || p.r == 32 || p.r == 64)) return false;
   if (!(p.g == 1 || p.g == 2 || p.g == 4 || p.g == 8)) return false;
   if (p.L_max >= (1ll << 31) || p.n_q_tokens < 1) return false;
   if ((int64_t)p.n_agents * p.n_kv > 65535 || p.n_seqs > 65535) return false;
-  return PCfg<16>::SMEM <= 227 * 1024;
+  return PCfg<16>::SMEM <= 227 * 1024 && PCfg<32>::SMEM <= 227 * 1024 && PCfg<64>::SMEM <= 227 * 1024;
 }
 
 cudaError_t launch_prefill_bf16(const AttnParams& pin, la_dtype out, cudaStream_t st) {
   AttnParams p = pin;
   p.out_bf16 = out == LA_BF16;
-  return launch_prefill_tc<16>(p, st);
+  switch (p.r) {
+    case 16: return launch_prefill_tc<16>(p, st);
+    case 32: return launch_prefill_tc<32>(p, st);
+    default: return launch_prefill_tc<64>(p, st);
+  }
 }
 
 }  // namespace la

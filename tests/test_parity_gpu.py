@@ -286,18 +286,20 @@ def _prefill_vs_oracle(la, s, inp, out_dtype=None):
     return assert_parity(to_np(got.float()), ref, s.dtype)
 
 
-@pytest.mark.parametrize("n_q,n_kv,L,n_tok,n_seqs", [
-    (32, 8, 200, 200, 1),     # g = 4, self-attention of a fresh chunk (q_pos0 = 0), ragged block
-    (32, 4, 700, 45, 2),      # g = 8: 16 tokens per block, two sequences
-    (8, 8, 390, 260, 1),      # g = 1: 128 tokens per block, chunk over a prefix
-    (16, 8, 129, 64, 1),      # g = 2, one key past a tile
-    (32, 8, 100, 1, 1),       # one query token, one partial tile
+@pytest.mark.parametrize("n_q,n_kv,L,n_tok,n_seqs,r", [
+    (32, 8, 200, 200, 1, 16),     # g = 4, self-attention of a fresh chunk (q_pos0 = 0), ragged block
+    (32, 8, 600, 300, 1, 32),     # r = 32
+    (32, 8, 700, 200, 1, 64),     # r = 64: one V stage
+    (32, 4, 700, 45, 2, 16),      # g = 8: 16 tokens per block, two sequences
+    (8, 8, 390, 260, 1, 16),      # g = 1: 128 tokens per block, chunk over a prefix
+    (16, 8, 129, 64, 1, 16),      # g = 2, one key past a tile
+    (32, 8, 100, 1, 1, 16),       # one query token, one partial tile
 ])
-def test_bf16_prefill_tensor_core_shapes(la, n_q, n_kv, L, n_tok, n_seqs):
-    """The tcgen05 prefill (r = 16): GQA groups 1..8, blocks cut by the chunk's
-    end, keys cut inside a tile, several sequences."""
+def test_bf16_prefill_tensor_core_shapes(la, n_q, n_kv, L, n_tok, n_seqs, r):
+    """The tcgen05 prefill (r = 16, 32, 64): GQA groups 1..8, blocks cut by the
+    chunk's end, keys cut inside a tile, several sequences."""
     s = W.LLAMA8B_PREFILL_16K.replace(n_q_heads=n_q, n_kv_heads=n_kv, kv_len=L, n_q_tokens=n_tok,
-                                      n_seqs=n_seqs, seed=400 + L)
+                                      n_seqs=n_seqs, r=r, alpha=2.0 * r, seed=400 + L)
     _prefill_vs_oracle(la, s, W.direct_cache_inputs(s))
 
 
@@ -374,6 +376,17 @@ def test_llama8b_prefill_16k_sampled(la):
     got = _run(la, s, dd["k_base"], dd["v_base"], dd["lr"], dd["B_k"], dd["B_v"], dd["q"]).cpu()
     tokens = np.array([0, 1, 63, 64, 127, 500, 1000, 1022, 1023])
     _sampled_units(la, s, inp, got, [(0, 0, 0), (0, 1, 3), (0, 2, 7)], tokens)
+
+
+def test_llama8b_stack_prefill_sampled(la):
+    """One layer of the 32-layer stack: a 4096-token chunk over a 32768-token
+    prefix, 4 agents, r = 64 (the tensor-core prefill with one V stage)."""
+    s = W.llama8b_stack_prefill(0)
+    inp = W.direct_cache_inputs(s)
+    dd = to_device(inp)
+    got = _run(la, s, dd["k_base"], dd["v_base"], dd["lr"], dd["B_k"], dd["B_v"], dd["q"]).cpu()
+    tokens = np.array([0, 1, 127, 128, 2047, 4095])
+    _sampled_units(la, s, inp, got, [(0, 0, 0), (0, 3, 5)], tokens)
 
 
 @pytest.mark.parametrize("ctx", [32768])
