@@ -1211,6 +1211,8 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
     if (lane == 0) {
       constexpr uint32_t ID_S = umma_idesc_bf16(128, QPAD, 0, 0);
       constexpr uint32_t ID_E = umma_idesc_bf16(128, D, 0, 1);
+      const uint64_t dQ = umma_desc(qu_u, 16, 1024, 2);
+      const uint64_t dBk = umma_desc(bks_u, R * 128, 1024, 2);
       if (n_tiles > 0 && !mbar_wait(bkbar, 0)) fail = 1;
       // the split's later tiles stream into L2 from here on (the queries and the
       // first stages were requested first), so that HBM stays busy between
@@ -1234,20 +1236,18 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
         if (n > 0 && !mbar_wait(tempty, (n - 1) & 1)) fail = 1;
         tc_fence_after();
         // base scores for every agent's rows: S_base^T = K_base Q^T
+        const uint64_t dK = umma_desc(sK, 16, 1024, 2);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t da = umma_desc(sK + (kk >> 2) * (KT * 128) + (kk & 3) * 32, 16, 1024, 2);
-          const uint64_t db = umma_desc(qu_u + (kk >> 2) * (QPAD * 128) + (kk & 3) * 32, 16, 1024, 2);
-          umma_bf16(tmem + TC_SCOL, da, db, ID_S, kk > 0);
-        }
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_bf16(tmem + TC_SCOL, umma_desc_add(dK, (kk >> 2) * (KT * 128) + (kk & 3) * 32),
+                    umma_desc_add(dQ, (kk >> 2) * (QPAD * 128) + (kk & 3) * 32), ID_S, kk > 0);
         // key deltas dK^a = LRk B_k^a (B_k^a stored r-major: the MN-major operand)
+        const uint64_t dL = umma_desc(sL, 16, 8 * C::LR_ROWB, C::LR_LAYOUT);
         for (int a = 0; a < na; ++a) {
+          const uint64_t dB = umma_desc_add(dBk, a * align1k(C::BK_BYTES));
 #pragma unroll
-          for (int ks = 0; ks < C::KS; ++ks) {
-            const uint64_t da = umma_desc(sL + ks * 32, 16, 8 * C::LR_ROWB, C::LR_LAYOUT);
-            const uint64_t db = umma_desc(bks_u + a * align1k(C::BK_BYTES) + ks * 16 * 128, R * 128, 1024, 2);
-            umma_bf16(tmem + 128 * a, da, db, ID_E, ks > 0);
-          }
+          for (int ks = 0; ks < C::KS; ++ks)
+            umma_bf16(tmem + 128 * a, umma_desc_add(dL, ks * 32), umma_desc_add(dB, ks * 16 * 128), ID_E, ks > 0);
         }
         umma_commit(tfull);
         umma_commit(empty_u + 8 * s);  // K and LRk of this stage have been read

@@ -211,31 +211,37 @@ __global__ void __launch_bounds__(PNTHR, 1)
       constexpr uint32_t ID_S = umma_idesc_bf16(128, PKT, 0, 0);
       constexpr uint32_t ID_PV = umma_idesc_bf16(128, PD, 0, 1);
       constexpr uint32_t ID_PL = umma_idesc_bf16(128, R, 0, 1);
+      // operand descriptors of stage 0; the others are fixed byte offsets on
+      const uint64_t dQ = umma_desc(q_u, 16, 1024, 2);
+      const uint64_t dK = umma_desc(k_u, 16, 1024, 2);
+      const uint64_t dLRk = umma_desc(k_u + C::KV, 16, 8 * C::LR_ROWB, C::LR_LAYOUT);
+      const uint64_t dBk = umma_desc(bk_u, R * 128, 1024, 2);
+      const uint64_t dV = umma_desc(v_u, PKT * 128, 1024, 2);
+      const uint64_t dLRv = umma_desc(v_u + C::KV, PKT * C::LR_ROWB, 8 * C::LR_ROWB, C::LR_LAYOUT);
       auto mma_dk = [&](int n) {  // dK = LRk B_k^a
         if (!mbar_wait(kfull(n & 1), (n >> 1) & 1)) fail = 1;
         tc_fence_after();
-        const uint32_t lr = k_u + (n & 1) * C::STAGE + C::KV;
+        const uint64_t lr = umma_desc_add(dLRk, (n & 1) * C::STAGE);
 #pragma unroll
         for (int ks = 0; ks < R / 16; ++ks)
-          umma_bf16(tmem + T_DK, umma_desc(lr + ks * 32, 16, 8 * C::LR_ROWB, C::LR_LAYOUT),
-                    umma_desc(bk_u + ks * 16 * 128, R * 128, 1024, 2), ID_DK, ks > 0);
+          umma_bf16(tmem + T_DK, umma_desc_add(lr, ks * 32), umma_desc_add(dBk, ks * 16 * 128), ID_DK, ks > 0);
         umma_commit(dkfull);
       };
       auto mma_pv = [&](int n) {  // O += P V_base, O_lr += P LR
         if (!mbar_wait(pfull, n & 1)) fail = 1;
         if (!mbar_wait(vfull(n % C::NV), (n / C::NV) & 1)) fail = 1;
         tc_fence_after();
-        const uint32_t vs = v_u + (n % C::NV) * C::STAGE;
+        const uint64_t vd = umma_desc_add(dV, (n % C::NV) * C::STAGE);
+        const uint64_t ld = umma_desc_add(dLRv, (n % C::NV) * C::STAGE);
+        const uint32_t acc = n > 0 ? 1u : 0u;
 #pragma unroll
         for (int ks = 0; ks < PKT / 16; ++ks)
-          umma_bf16_ts(tmem + T_O, tmem + T_P + ks * 8, umma_desc(vs + ks * 16 * 128, PKT * 128, 1024, 2),
-                       ID_PV, (n > 0 || ks > 0) ? 1u : 0u);
+          umma_bf16_ts(tmem + T_O, tmem + T_P + ks * 8, umma_desc_add(vd, ks * 16 * 128), ID_PV,
+                       ks > 0 ? 1u : acc);
 #pragma unroll
         for (int ks = 0; ks < PKT / 16; ++ks)
-          umma_bf16_ts(tmem + T_OL, tmem + T_P + ks * 8,
-                       umma_desc(vs + C::KV + ks * 16 * C::LR_ROWB, PKT * C::LR_ROWB, 8 * C::LR_ROWB,
-                                 C::LR_LAYOUT),
-                       ID_PL, (n > 0 || ks > 0) ? 1u : 0u);
+          umma_bf16_ts(tmem + T_OL, tmem + T_P + ks * 8, umma_desc_add(ld, ks * 16 * C::LR_ROWB), ID_PL,
+                       ks > 0 ? 1u : acc);
         umma_commit(pvdone);
         umma_commit(vempty(n % C::NV));
       };
@@ -245,11 +251,11 @@ __global__ void __launch_bounds__(PNTHR, 1)
         if (!mbar_wait(kaready, n & 1)) fail = 1;
         if (n > 0 && !mbar_wait(staken, (n - 1) & 1)) fail = 1;
         tc_fence_after();
-        const uint32_t ks_ = k_u + (n & 1) * C::STAGE;
+        const uint64_t kd = umma_desc_add(dK, (n & 1) * C::STAGE);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          umma_bf16(tmem + T_S, umma_desc(q_u + (kk >> 2) * (PM * 128) + (kk & 3) * 32, 16, 1024, 2),
-                    umma_desc(ks_ + (kk >> 2) * (PKT * 128) + (kk & 3) * 32, 16, 1024, 2), ID_S, kk > 0);
+          umma_bf16(tmem + T_S, umma_desc_add(dQ, (kk >> 2) * (PM * 128) + (kk & 3) * 32),
+                    umma_desc_add(kd, (kk >> 2) * (PKT * 128) + (kk & 3) * 32), ID_S, kk > 0);
         umma_commit(sfull);
         umma_commit(kempty(n & 1));
         if (n + 1 < N) mma_dk(n + 1);

@@ -186,6 +186,11 @@ __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint
   return (uint64_t)((saddr >> 4) & 0x3FFF) | ((uint64_t)((lbo >> 4) & 0x3FFF) << 16) |
          ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46) | ((uint64_t)layout << 61);
 }
+// The descriptor of the same operand `bytes` further on (a multiple of 16; the
+// address field is addr >> 4 and shared memory stays below 256 KB, so no carry)
+__host__ __device__ constexpr uint64_t umma_desc_add(uint64_t desc, uint32_t bytes) {
+  return desc + (bytes >> 4);
+}
 // Instruction descriptor of kind::f16: bf16 x bf16 -> f32, M x N, operand majors.
 __host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N, int a_mn, int b_mn) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
