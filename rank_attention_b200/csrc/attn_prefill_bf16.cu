@@ -20,7 +20,8 @@
 //
 // Warps: 8 compute warps build K^a (16 keys each, the mma fragment layout of
 // the delta) and run the softmax (two warps per TMEM sub-partition, 64 keys
-// each); warp 8 issues TMA loads and MMAs.  The compute warps build tile n+1
+// each); warp 8 issues the MMAs (and the first loads), warp 9 the TMA
+// refills.  The compute warps build tile n+1
 // before the softmax of tile n, so the S MMA of tile n+1 runs during that
 // softmax and the P V MMA of tile n during the next build.
 #include <cmath>
@@ -40,7 +41,7 @@ constexpr int PD = 128;                  // head_dim
 constexpr int PKT = 128;                 // keys per tile
 constexpr int PM = 128;                  // query rows per CTA
 constexpr int PNC = 8;                   // compute warps
-constexpr int PNTHR = 32 * (PNC + 1);
+constexpr int PNTHR = 32 * (PNC + 2);  // + the MMA warp + the TMA refill warp
 // TMEM columns
 constexpr int T_DK = 0, T_S = 128, T_P = 256, T_O = 320, T_OL = 448, T_COLS = 512;
 // named barriers (0 is __syncthreads)
@@ -260,8 +261,19 @@ __global__ void __launch_bounds__(PNTHR, 1)
         umma_commit(kempty(n & 1));
         if (n + 1 < N) mma_dk(n + 1);
         if (n > 0) mma_pv(n - 1);
+      }
+      mma_pv(N - 1);
+      // loads in flight when the loop ends are all consumed: every issued tile is used
+    }
+    __syncwarp();
+  } else if (w == PNC + 1) {
+    // ============================================================ TMA refill warp
+    // refills in the order the MMAs free the stages (S of tile n, then P V of
+    // tile n-1), so that the MMA warp never waits for an MMA to finish
+    if (lane == 0) {
+      for (int n = 0; n < N; ++n) {
         if (n + 2 < N) {
-          if (!mbar_wait(kempty(n & 1), (n >> 1) & 1)) fail = 1;
+          if (!mbar_wait(kempty(n & 1), (n >> 1) & 1)) fail = 1;   // S_n has read K^a_n
           load_k(n + 2);
         }
         if (n > 0 && n - 1 + C::NV < N) {  // V stage of tile n-1 is free once its P V is done
@@ -269,8 +281,6 @@ __global__ void __launch_bounds__(PNTHR, 1)
           load_v(n - 1 + C::NV);
         }
       }
-      mma_pv(N - 1);
-      // loads in flight when the loop ends are all consumed: every issued tile is used
     }
     __syncwarp();
   } else {
