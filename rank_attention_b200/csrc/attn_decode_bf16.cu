@@ -51,6 +51,9 @@ namespace {
 using namespace ptx;
 
 constexpr int ST = 2;               // pipeline stages
+// tiles requested into L2 ahead of the stage loads: enough to keep HBM busy
+// between refills, few enough that 148 CTAs' windows stay resident in L2
+constexpr int kL2Ahead = 4;
 constexpr int KT = 128;             // keys per tile
 constexpr int NES = 8;              // score warps (16 keys each)
 constexpr int NPV = 2;              // value warps
@@ -1214,10 +1217,10 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
       const uint64_t dQ = umma_desc(qu_u, 16, 1024, 2);
       const uint64_t dBk = umma_desc(bks_u, R * 128, 1024, 2);
       if (n_tiles > 0 && !mbar_wait(bkbar, 0)) fail = 1;
-      // the split's later tiles stream into L2 from here on (the queries and the
+      // the split's next tiles stream into L2 from here on (the queries and the
       // first stages were requested first), so that HBM stays busy between
-      // stage refills
-      for (int m = ST; m < n_tiles; ++m) {
+      // stage refills; the window moves one tile per tile consumed
+      auto prefetch = [&](int m) {
         const int key0 = (int)(k_lo + (int64_t)m * KT);
 #pragma unroll
         for (int b = 0; b < D / 64; ++b) {
@@ -1227,7 +1230,8 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
         constexpr int LB = (2 * R) < 64 ? 2 * R : 64;
 #pragma unroll
         for (int b = 0; b < (2 * R) / LB; ++b) tma_prefetch_l2_3d(&tmL, LB * b, key0, seq);
-      }
+      };
+      for (int m = ST; m < n_tiles && m < ST + kL2Ahead; ++m) prefetch(m);
       for (int n = 0; n < n_tiles; ++n) {
         const int s = n % ST;
         const uint32_t sK = area_u + s * C::STAGE;
@@ -1255,6 +1259,7 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
           const int sp = (n - 1) % ST;
           if (!mbar_wait(empty_u + 8 * sp, ((n - 1) / ST) & 1)) fail = 1;
           issue(n - 1 + ST);
+          if (n - 1 + ST + kL2Ahead < n_tiles) prefetch(n - 1 + ST + kL2Ahead);
         }
       }
       for (int n = n_tiles; n < n_spec; ++n)  // loaded ahead of kv_len and not used

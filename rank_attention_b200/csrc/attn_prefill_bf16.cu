@@ -71,7 +71,7 @@ struct PCfg {
   static constexpr size_t SMEM = 1024 + OFF_MISC + MISC;
 };
 
-template <int R>
+template <int R, int KS>
 __global__ void __launch_bounds__(PNTHR, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmK,
@@ -79,6 +79,7 @@ __global__ void __launch_bounds__(PNTHR, 1)
                       const __grid_constant__ CUtensorMap tmL,
                       const __grid_constant__ CUtensorMap tmB, const AttnParams p,
                       const __grid_constant__ RopeTheta rt) {
+  constexpr int ksplit = KS;   // 1, or 2: the keys of a block split over a cluster of two CTAs
   using C = PCfg<R>;
   constexpr int D = PD;
   extern __shared__ unsigned char smem_raw[];
@@ -110,15 +111,22 @@ __global__ void __launch_bounds__(PNTHR, 1)
   const int agent = blockIdx.y / p.n_kv, kvh = blockIdx.y % p.n_kv;
   const int g = p.g, na = p.n_agents;
   const int QB = PM / g;
-  const int tok0 = blockIdx.x * QB;
+  const int tok0 = (int)(blockIdx.x / ksplit) * QB;
   const int ntok = min(QB, p.n_q_tokens - tok0);
   const int64_t qmin = p.q_pos0 + tok0;               // position of the block's first token
   const int64_t kend = qmin + ntok;                    // keys [0, kend)
   const int N = (int)((kend + PKT - 1) / PKT);
+  // key split over a CTA pair (a cluster of two): half 0 takes tiles [0, T0),
+  // half 1 tiles [T0, N) and hands its partial (O, O_lr, m, l) to half 0
+  const int half = ksplit > 1 ? (int)cluster_ctarank() : 0;
+  const int T0 = ksplit > 1 ? max(1, N / 2) : N;
+  const int nb = half ? T0 : 0;          // first tile of this CTA
+  const int NT = half ? N - T0 : T0;     // tiles of this CTA (local index 0 .. NT-1)
+  const bool work = KS == 1 || NT > 0;   // half 1 of a one-tile block has no keys
 
   // lr_col: 0 for the LRk columns (with K), r for LRv (with V)
   auto load_stage = [&](const CUtensorMap* m, uint32_t base, uint32_t bar, int n, int lr_col) {
-    const int key0 = n * PKT;
+    const int key0 = (nb + n) * PKT;
     mbar_expect_tx(bar, (uint32_t)(C::KV + PKT * R * 2));
 #pragma unroll
     for (int b = 0; b < D / 64; ++b) tma_load_4d(base + b * PKT * 128, m, bar, 64 * b, key0, kvh, seq);
@@ -149,24 +157,28 @@ __global__ void __launch_bounds__(PNTHR, 1)
     tma_prefetch(&tmK);
     tma_prefetch(&tmV);
     tma_prefetch(&tmL);
-    // the block's rows: g heads of each of its tokens, two 64-column boxes
-    mbar_expect_tx(qbar, (uint32_t)(C::Q_BYTES + C::B_BYTES));
+    if (work) {
+      // the block's rows: g heads of each of its tokens, two 64-column boxes
+      mbar_expect_tx(qbar, (uint32_t)(C::Q_BYTES + C::B_BYTES));
 #pragma unroll
-    for (int b = 0; b < D / 64; ++b)
-      tma_load_4d(q_u + b * PM * 128, &tmQ, qbar, 64 * b, kvh * g, tok0, seq * na + agent);
+      for (int b = 0; b < D / 64; ++b)
+        tma_load_4d(q_u + b * PM * 128, &tmQ, qbar, 64 * b, kvh * g, tok0, seq * na + agent);
 #pragma unroll
-    for (int b = 0; b < D / 64; ++b)
-      tma_load_3d(bk_u + b * R * 128, &tmB, qbar, kvh * D + 64 * b, 0, agent);
-    load_k(0);
-    load_v(0);
-    if (N > 1) {
-      load_k(1);
-      if (C::NV > 1) load_v(1);
+      for (int b = 0; b < D / 64; ++b)
+        tma_load_3d(bk_u + b * R * 128, &tmB, qbar, kvh * D + 64 * b, 0, agent);
+      load_k(0);
+      load_v(0);
+      if (NT > 1) {
+        load_k(1);
+        if (C::NV > 1) load_v(1);
+      }
     }
-    const __nv_bfloat16* Bv = reinterpret_cast<const __nv_bfloat16*>(p.B_v);
-    mbar_expect_tx(bvbar, (uint32_t)C::B_BYTES);
-    for (int j = 0; j < R; ++j)
-      bulk_load(bv_u + j * D * 2, Bv + ((int64_t)agent * R + j) * p.n_kv * D + kvh * D, D * 2, bvbar);
+    if (half == 0) {  // B_v^a: only the CTA that writes the output
+      const __nv_bfloat16* Bv = reinterpret_cast<const __nv_bfloat16*>(p.B_v);
+      mbar_expect_tx(bvbar, (uint32_t)C::B_BYTES);
+      for (int j = 0; j < R; ++j)
+        bulk_load(bv_u + j * D * 2, Bv + ((int64_t)agent * R + j) * p.n_kv * D + kvh * D, D * 2, bvbar);
+    }
   }
   if (w == PNC) tmem_alloc(smem_u32(tslot), T_COLS);
 
@@ -196,7 +208,7 @@ __global__ void __launch_bounds__(PNTHR, 1)
   if (tid < D / 2) theta[tid] = rt.theta[tid];
   if (tid < 2 * (D / 2)) {
     const int n = tid / (D / 2), i = tid % (D / 2);
-    const float2 cs = rope_cs_exact((int64_t)n * PKT, rt.theta[i]);
+    const float2 cs = rope_cs_exact((int64_t)(nb + n) * PKT, rt.theta[i]);
     anc[n * 64 + i] = make_float2(cs.x * p.s, cs.y * p.s);
   }
   tc_fence_before();
@@ -207,7 +219,7 @@ __global__ void __launch_bounds__(PNTHR, 1)
 
   if (w == PNC) {
     // ============================================================ TMA / MMA warp
-    if (lane == 0) {
+    if (lane == 0 && work) {
       constexpr uint32_t ID_DK = umma_idesc_bf16(128, PD, 0, 1);
       constexpr uint32_t ID_S = umma_idesc_bf16(128, PKT, 0, 0);
       constexpr uint32_t ID_PV = umma_idesc_bf16(128, PD, 0, 1);
@@ -248,7 +260,7 @@ __global__ void __launch_bounds__(PNTHR, 1)
       };
       if (!mbar_wait(qbar, 0)) fail = 1;
       mma_dk(0);
-      for (int n = 0; n < N; ++n) {
+      for (int n = 0; n < NT; ++n) {
         if (!mbar_wait(kaready, n & 1)) fail = 1;
         if (n > 0 && !mbar_wait(staken, (n - 1) & 1)) fail = 1;
         tc_fence_after();
@@ -259,30 +271,38 @@ __global__ void __launch_bounds__(PNTHR, 1)
                     umma_desc_add(kd, (kk >> 2) * (PKT * 128) + (kk & 3) * 32), ID_S, kk > 0);
         umma_commit(sfull);
         umma_commit(kempty(n & 1));
-        if (n + 1 < N) mma_dk(n + 1);
+        if (n + 1 < NT) mma_dk(n + 1);
         if (n > 0) mma_pv(n - 1);
       }
-      mma_pv(N - 1);
+      mma_pv(NT - 1);
       // loads in flight when the loop ends are all consumed: every issued tile is used
     }
     __syncwarp();
+    if (ksplit > 1) {
+      cluster_sync_all();
+      cluster_sync_all();
+    }
   } else if (w == PNC + 1) {
     // ============================================================ TMA refill warp
     // refills in the order the MMAs free the stages (S of tile n, then P V of
     // tile n-1), so that the MMA warp never waits for an MMA to finish
     if (lane == 0) {
-      for (int n = 0; n < N; ++n) {
-        if (n + 2 < N) {
+      for (int n = 0; n < NT; ++n) {
+        if (n + 2 < NT) {
           if (!mbar_wait(kempty(n & 1), (n >> 1) & 1)) fail = 1;   // S_n has read K^a_n
           load_k(n + 2);
         }
-        if (n > 0 && n - 1 + C::NV < N) {  // V stage of tile n-1 is free once its P V is done
+        if (n > 0 && n - 1 + C::NV < NT) {  // V stage of tile n-1 is free once its P V is done
           if (!mbar_wait(vempty((n - 1) % C::NV), ((n - 1) / C::NV) & 1)) fail = 1;
           load_v(n - 1 + C::NV);
         }
       }
     }
     __syncwarp();
+    if (ksplit > 1) {
+      cluster_sync_all();
+      cluster_sync_all();
+    }
   } else {
     // ============================================================ compute warps
     const float sl2 = p.scale * kLog2e;
@@ -351,7 +371,7 @@ __global__ void __launch_bounds__(PNTHR, 1)
       // row maximum of the raw scores (the scale is positive); keys past a row's
       // position are set to -inf (only the tiles that reach the block's first
       // position need it; rows past the chunk are never written out)
-      const int64_t key0 = (int64_t)n * PKT + 64 * ch;
+      const int64_t key0 = (int64_t)(nb + n) * PKT + 64 * ch;
       if (key0 + 63 > qmin) {
 #pragma unroll
         for (int h = 0; h < 2; ++h)
@@ -433,26 +453,67 @@ __global__ void __launch_bounds__(PNTHR, 1)
       if (lane == 0) mbar_arrive(pfull);
     };
 
-    build(0);
-    for (int i = 0; i < N; ++i) {
+    if (work) build(0);
+    for (int i = 0; i < NT; ++i) {
       bar_sync(PBAR_CW, 32 * PNC);  // anchors of tile i+1 are in place
-      if (i + 1 < N) build(i + 1);
+      if (i + 1 < NT) build(i + 1);
       softmax(i);
-      if (tid < D / 2 && i + 2 < N) {
-        const float2 cs = rope_cs_exact((int64_t)(i + 2) * PKT, theta[tid]);
+      if (tid < D / 2 && i + 2 < NT) {
+        const float2 cs = rope_cs_exact((int64_t)(nb + i + 2) * PKT, theta[tid]);
         anc[(i & 1) * 64 + tid] = make_float2(cs.x * p.s, cs.y * p.s);
       }
     }
 
+    // half 1's partial goes to its drained K / V stages: O as float4 [d/4][128
+    // rows], O_lr as float4 [r/4][128 rows], then m_ref and l per row
+    const uint32_t xo = k_u, xl = xo + PM * PD * 4, xm = xl + PM * R * 4, xs = xm + PM * 4;
+    if constexpr (KS > 1) {
+      if (half == 1) {
+        if (work) {
+          if (!mbar_wait(pvdone, (NT - 1) & 1)) fail = 1;
+          tc_fence_after();
+          float* lx = xch + (NT & 1) * 256;  // the exchange buffer the last softmax did not use
+          lx[w * 32 + lane] = lsum;
+          bar_sync(PBAR_PAIR + sp, 64);
+          const float l = lsum + lx[(w ^ 4) * 32 + lane];
+#pragma unroll 1
+          for (int h = 0; h < 4; ++h) {
+            uint32_t ov[16];
+            tmem_ld32x32b_x16(ov, tmem + T_O + 64 * ch + 16 * h + ((uint32_t)(32 * sp) << 16));
+            tmem_wait_ld_r16(ov);
+#pragma unroll
+            for (int c = 0; c < 16; c += 4)
+              sts128(xo + (uint32_t)(((64 * ch + 16 * h + c) / 4) * PM + row) * 16, ov[c], ov[c + 1], ov[c + 2],
+                     ov[c + 3]);
+          }
+          if (ch == 0) {
+#pragma unroll 1
+            for (int h = 0; h < R / 16; ++h) {
+              uint32_t t16[16];
+              tmem_ld32x32b_x16(t16, tmem + T_OL + 16 * h + ((uint32_t)(32 * sp) << 16));
+              tmem_wait_ld_r16(t16);
+#pragma unroll
+              for (int c = 0; c < 16; c += 4)
+                sts128(xl + (uint32_t)(((16 * h + c) / 4) * PM + row) * 16, t16[c], t16[c + 1], t16[c + 2],
+                       t16[c + 3]);
+            }
+            sts32(xm + row * 4, __float_as_uint(m_ref));
+            sts32(xs + row * 4, __float_as_uint(l));
+          }
+        }
+        cluster_sync_all();  // the partial is in place
+        cluster_sync_all();  // half 0 has read it
+      }
+    }
+    if (half == 0) {
     // ---- epilogue: out = (O + s O_lr B_v^a) / l for this warp's 64 columns
-    if (!mbar_wait(pvdone, (N - 1) & 1)) fail = 1;
+    if (!mbar_wait(pvdone, (NT - 1) & 1)) fail = 1;
     if (!mbar_wait(bvbar, 0)) fail = 1;
     tc_fence_after();
-    float* lx = xch + (N & 1) * 256;  // the exchange buffer the last softmax did not use
+    float* lx = xch + (NT & 1) * 256;  // the exchange buffer the last softmax did not use
     lx[w * 32 + lane] = lsum;
     bar_sync(PBAR_PAIR + sp, 64);
-    const float l = lsum + lx[(w ^ 4) * 32 + lane];
-    const float inv_l = l > 0.f ? 1.f / l : 0.f;
+    float l = lsum + lx[(w ^ 4) * 32 + lane];
     uint32_t olr[R];   // P LRv, this thread's row
 #pragma unroll
     for (int h = 0; h < R / 16; ++h) {
@@ -462,6 +523,31 @@ __global__ void __launch_bounds__(PNTHR, 1)
 #pragma unroll
       for (int c = 0; c < 16; ++c) olr[16 * h + c] = t16[c];
     }
+    // with split keys: merge with half 1's partial, both rescaled to the larger
+    // of the two reference maxima
+    float a0 = 1.f, a1 = 0.f;
+    bool merge = false;
+    if constexpr (KS > 1) {
+      cluster_sync_all();
+      merge = N - T0 > 0;
+      if (merge) {
+        const float m1 = dsmem_ld(dsmem_addr(xm + row * 4, 1));
+        const float l1 = dsmem_ld(dsmem_addr(xs + row * 4, 1));
+        const float M = fmaxf(m_ref, m1);
+        a0 = m_ref == -INFINITY ? 0.f : fast_exp2(m_ref - M);
+        a1 = m1 == -INFINITY ? 0.f : fast_exp2(m1 - M);
+        l = a0 * l + a1 * l1;
+#pragma unroll
+        for (int j = 0; j < R; j += 4) {
+          const float4 r4 = dsmem_ld4(dsmem_addr(xl + (uint32_t)((j / 4) * PM + row) * 16, 1));
+          olr[j] = __float_as_uint(fmaf(a0, __uint_as_float(olr[j]), a1 * r4.x));
+          olr[j + 1] = __float_as_uint(fmaf(a0, __uint_as_float(olr[j + 1]), a1 * r4.y));
+          olr[j + 2] = __float_as_uint(fmaf(a0, __uint_as_float(olr[j + 2]), a1 * r4.z));
+          olr[j + 3] = __float_as_uint(fmaf(a0, __uint_as_float(olr[j + 3]), a1 * r4.w));
+        }
+      }
+    }
+    const float inv_l = l > 0.f ? 1.f / l : 0.f;
     const int head = kvh * g + row % g;
     const int64_t obase = (((int64_t)seq * na + agent) * p.n_q_tokens + tok0 + rtok) * p.n_q + head;
 #pragma unroll
@@ -469,6 +555,19 @@ __global__ void __launch_bounds__(PNTHR, 1)
       uint32_t ov[32];
       tmem_ld32x32b_x32(ov, tmem + T_O + 64 * ch + 32 * h + ((uint32_t)(32 * sp) << 16));
       tmem_wait_ld_r32(ov);
+      if constexpr (KS > 1) {
+        if (merge) {
+#pragma unroll
+          for (int c = 0; c < 32; c += 4) {
+            const float4 r4 =
+                dsmem_ld4(dsmem_addr(xo + (uint32_t)(((64 * ch + 32 * h + c) / 4) * PM + row) * 16, 1));
+            ov[c] = __float_as_uint(fmaf(a0, __uint_as_float(ov[c]), a1 * r4.x));
+            ov[c + 1] = __float_as_uint(fmaf(a0, __uint_as_float(ov[c + 1]), a1 * r4.y));
+            ov[c + 2] = __float_as_uint(fmaf(a0, __uint_as_float(ov[c + 2]), a1 * r4.z));
+            ov[c + 3] = __float_as_uint(fmaf(a0, __uint_as_float(ov[c + 3]), a1 * r4.w));
+          }
+        }
+      }
       float z[32];
 #pragma unroll
       for (int c = 0; c < 32; ++c) z[c] = 0.f;
@@ -501,6 +600,8 @@ __global__ void __launch_bounds__(PNTHR, 1)
                                    fmaf(p.s, z[c + 3], __uint_as_float(ov[c + 3])) * inv_l);
         }
       }
+    }
+    if constexpr (KS > 1) cluster_sync_all();
     }
   }
   if (fail) s_fail = 1;
@@ -560,6 +661,53 @@ bool prefill_maps(const AttnParams& p, CUtensorMap* mq, CUtensorMap* mk, CUtenso
   return true;
 }
 
+// Key split: 1 (one CTA per block of rows) or 2 (a cluster of two CTAs per
+// block, each over half of the keys).  The CTAs of one wave run about equally
+// long, so the launch takes ceil(CTAs / resident CTAs) waves.  A half costs
+// more than half a CTA (its own start-up, pipeline fill and the merge: about
+// 15% measured at 65 tiles a half), so the split pays where the CTAs leave
+// SMs idle: fewer CTAs than SMs, or a last wave that is mostly empty.
+template <int R>
+int prefill_ksplit(const AttnParams& p, int nblk) {
+  using C = PCfg<R>;
+  const int64_t tiles = (p.q_pos0 + p.n_q_tokens + PKT - 1) / PKT;
+  if (tiles < 4) return 1;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) {
+    cudaGetLastError();
+    return 1;
+  }
+  static int pairs[64] = {};   // resident CTA pairs per device (0: not queried yet)
+  int& np = pairs[dev & 63];
+  if (np == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (unsigned)sms, 1, 1);
+    cfg.blockDim = dim3(PNTHR);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaFuncSetAttribute(prefill_tc_kernel<R, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)C::SMEM) != cudaSuccess ||
+        cudaOccupancyMaxActiveClusters(&n, prefill_tc_kernel<R, 2>, &cfg) != cudaSuccess || n < 1) {
+      cudaGetLastError();
+      n = -1;
+    }
+    np = n;
+  }
+  if (np < 1) return 1;
+  const double ctas = (double)nblk * p.n_agents * p.n_kv * p.n_seqs;
+  const double t1 = std::ceil(ctas / sms);              // waves of whole CTAs
+  const double t2 = 0.5 * std::ceil(ctas / np) * 1.15;  // half-length waves, + their overhead
+  return t2 < t1 ? 2 : 1;
+}
+
 template <int R>
 cudaError_t launch_prefill_tc(const AttnParams& p, cudaStream_t st) {
   using C = PCfg<R>;
@@ -570,12 +718,26 @@ cudaError_t launch_prefill_tc(const AttnParams& p, cudaStream_t st) {
   }
   CUtensorMap mq, mk, mv, ml, mb;
   if (!prefill_maps(p, &mq, &mk, &mv, &ml, &mb)) return cudaErrorInvalidValue;
-  auto kern = prefill_tc_kernel<R>;
+  const int QB = PM / p.g;
+  const int nblk = (p.n_q_tokens + QB - 1) / QB;
+  const int ks = prefill_ksplit<R>(p, nblk);
+  auto kern = ks > 1 ? prefill_tc_kernel<R, 2> : prefill_tc_kernel<R, 1>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
   if (e != cudaSuccess) return e;
-  const int QB = PM / p.g;
-  dim3 grid((p.n_q_tokens + QB - 1) / QB, p.n_agents * p.n_kv, p.n_seqs);
-  kern<<<grid, PNTHR, C::SMEM, st>>>(mq, mk, mv, ml, mb, p, rt);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(nblk * ks), p.n_agents * p.n_kv, p.n_seqs);
+  cfg.blockDim = dim3(PNTHR);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)ks;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = ks > 1 ? 1 : 0;
+  e = cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, ml, mb, p, rt);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -585,7 +747,7 @@ bool bf16_prefill_supported(const AttnParams& p) {
   // r = 8 would make the P LRv MMA N = 8, below the M = 128 minimum of 16
   if (p.d != PD || !(p.r == 16 || p.r == 32 || p.r == 64)) return false;
   if (!(p.g == 1 || p.g == 2 || p.g == 4 || p.g == 8)) return false;
-  if (p.L_max >= (1ll << 31) || p.n_q_tokens < 1) return false;
+  if (p.L_max >= (1ll << 31) || p.n_q_tokens < 1 || p.n_q_tokens > (1 << 29)) return false;
   if ((int64_t)p.n_agents * p.n_kv > 65535 || p.n_seqs > 65535) return false;
   return PCfg<16>::SMEM <= 227 * 1024 && PCfg<32>::SMEM <= 227 * 1024 && PCfg<64>::SMEM <= 227 * 1024;
 }

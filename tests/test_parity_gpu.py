@@ -294,6 +294,7 @@ def _prefill_vs_oracle(la, s, inp, out_dtype=None):
     (8, 8, 390, 260, 1, 16),      # g = 1: 128 tokens per block, chunk over a prefix
     (16, 8, 129, 64, 1, 16),      # g = 2, one key past a tile
     (32, 8, 100, 1, 1, 16),       # one query token, one partial tile
+    (4, 1, 512, 512, 1, 16),      # few CTAs: key halves on CTA pairs; blocks of one tile leave half 1 empty
 ])
 def test_bf16_prefill_tensor_core_shapes(la, n_q, n_kv, L, n_tok, n_seqs, r):
     """The tcgen05 prefill (r = 16, 32, 64): GQA groups 1..8, blocks cut by the
