@@ -692,6 +692,7 @@ constexpr int TC_NES = 8;                          // score warps (16 keys each)
 constexpr int TC_NTHR = 32 * (TC_NES + NPV + 1);   // + value warps + TMA / MMA warp
 constexpr int TC_COLS = 512;                        // TMEM columns allocated
 constexpr int TC_SCOL = 384;                        // TMEM column of S_base
+constexpr int TC_OCOL = 448;                        // TMEM column of O_base^T (d lanes x query rows)
 
 template <int D, int R, int NT>
 struct TCfg {
@@ -710,7 +711,6 @@ struct TCfg {
   static constexpr int KS = R / 16;
   static constexpr int MR = R / 16;
   static constexpr int NG = D / 32;
-  static constexpr int MT = D / 2 / 16;
   // LR tile: rows of 2r bf16 in boxes of min(2r, 64); its swizzle span
   static constexpr int LR_ROWB = (2 * R < 64 ? 2 * R : 64) * 2;
   static constexpr uint32_t LR_LAYOUT = LR_ROWB == 128 ? 2u : (LR_ROWB == 64 ? 4u : 6u);
@@ -804,6 +804,8 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
   const uint32_t tempty = tfull + 8;               // score warps are done reading TMEM
   const uint32_t bkbar = tfull + 24;              // B_k^a slices have landed
   const uint32_t qbar = tfull + 32;               // the queries have landed (staged unswizzled)
+  const uint32_t pfull = tfull + 40;              // P of a tile is written, its V rows are final
+  const uint32_t pvdone = tfull + 48;             // the P V_base MMA of a tile has completed
   const int64_t ldB = (int64_t)p.n_kv * D;
 
   auto issue = [&](int n) {  // TMA of tile n into stage n % ST (one thread)
@@ -835,6 +837,8 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
     mbar_init(tempty, TC_NES);
     mbar_init(bkbar, 1);
     mbar_init(qbar, 1);
+    mbar_init(pfull, TC_NES + NPV);
+    mbar_init(pvdone, 1);
     fence_mbar_init();
     // each agent's g query rows of this KV head are contiguous
     const __nv_bfloat16* Q = reinterpret_cast<const __nv_bfloat16*>(p.q);
@@ -1069,6 +1073,9 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
           if (w == 0 && gq == 0) Corr[pb * ROWS + row] = corr;
         }
       bar_sync(BAR_PFREE + pb, NB);
+      // O^T holds every tile before this one (and P buffer pb, last read by the
+      // P V MMA of tile n-2, is free)
+      if (n > 0 && !mbar_wait(pvdone, (n - 1) & 1)) fail = 1;
       const uint32_t pt_u = ptile_u + pb * C::P_TILE;
 #pragma unroll
       for (int pt = 0; pt < NT; ++pt) {
@@ -1078,6 +1085,31 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
         sts32(pt_u + tile_off<KT, ROWS>(8 * pt + gq, kb + 8 + 2 * t4), b1);
       }
       bar_arrive(BAR_P + pb, NB);
+      // the running maxima moved: O^T (TMEM lanes = d, columns = query rows)
+      // times corr, by one warp per sub-partition
+      if (n > 0 && w < 4) {
+        bool any = false;
+        for (int row = 0; row < n_rows; ++row) any |= Corr[pb * ROWS + row] != 1.f;
+        if (any) {
+          tc_fence_after();
+#pragma unroll
+          for (int c0 = 0; c0 < QPAD; c0 += 16) {
+            uint32_t ov[16];
+            const uint32_t ta = tmem + TC_OCOL + c0 + ((uint32_t)(32 * w) << 16);
+            tmem_ld32x32b_x16(ov, ta);
+            tmem_wait_ld_r16(ov);
+#pragma unroll
+            for (int c = 0; c < 16; ++c)
+              if (c0 + c < ROWS) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * Corr[pb * ROWS + c0 + c]);
+            tmem_st32x32b_x16(ta, ov);
+          }
+          tmem_wait_st();
+        }
+      }
+      fence_proxy_async_smem();  // the MMA reads P through the async proxy
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(pfull);
     }
 #pragma unroll
     for (int pt = 0; pt < NT; ++pt)
@@ -1089,6 +1121,7 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
         l += __shfl_xor_sync(0xffffffffu, l, 16);
         if (gq == 0) Lw[w * ROWS + 8 * pt + 2 * t4 + e] = l;
       }
+    if (n_tiles > 0 && !mbar_wait(pvdone, (n_tiles - 1) & 1)) fail = 1;  // O^T is complete
     tc_fence_before();
     bar_sync(BAR_END, TC_NTHR);
     float* Mo = reinterpret_cast<float*>(area);
@@ -1098,17 +1131,29 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
 #pragma unroll
         for (int e = 0; e < 2; ++e) Mo[(8 * pt + 2 * t4 + e) * W + D + R] = m_st[pt][e];
     }
+    if (w < 4) {  // O_base, this lane's d = 32 w + lane, every query row
+      tc_fence_after();
+#pragma unroll
+      for (int c0 = 0; c0 < QPAD; c0 += 16) {
+        uint32_t ov[16];
+        if (n_tiles > 0) {
+          tmem_ld32x32b_x16(ov, tmem + TC_OCOL + c0 + ((uint32_t)(32 * w) << 16));
+          tmem_wait_ld_r16(ov);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 16; ++c) ov[c] = 0u;
+        }
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          if (c0 + c < ROWS) Mo[(c0 + c) * W + 32 * w + lane] = __uint_as_float(ov[c]);
+      }
+    }
   } else if (w < TC_NES + NPV) {
     // ======================================================== value warps
+    // the next tile's rotated queries, the tail rows of a tile past the
+    // sequence's end, and O_lr^T += LRv^T P^T (mma.sync; r columns)
     const int pv = w - TC_NES;
-    float O[C::MT][NT][4];
     float Olr[C::MR][NT][4];
-#pragma unroll
-    for (int mt = 0; mt < C::MT; ++mt)
-#pragma unroll
-      for (int pt = 0; pt < NT; ++pt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) O[mt][pt][e] = 0.f;
 #pragma unroll
     for (int mr = 0; mr < C::MR; ++mr)
 #pragma unroll
@@ -1123,7 +1168,6 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
     const int d0 = pv * (D / 2);
     for (int n = 0; n < n_tiles; ++n) {
       const int s = n % ST, pb = n & 1;
-      const uint32_t sV = area_u + s * C::STAGE + C::KV_TILE;
       const uint32_t sL = area_u + s * C::STAGE + 2 * C::KV_TILE;
       const int64_t k0 = k_lo + (int64_t)n * KT;
       if (n + 1 < n_tiles) {
@@ -1133,7 +1177,7 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
         bar_arrive(BAR_QP + ((n + 1) & 1), NB);
       }
       if (!mbar_wait(full_u + 8 * s, (n / ST) & 1)) fail = 1;
-      if (k0 + KT > k_hi) {
+      if (k0 + KT > k_hi) {  // rows past the end: zero, so that P (0 there) meets no stale NaN
         unsigned char* vb = area + s * C::STAGE + C::KV_TILE;
         unsigned char* lb = area + s * C::STAGE + 2 * C::KV_TILE;
         const int first = (int)(k_hi - k0);
@@ -1146,40 +1190,29 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
             const int row = first + i / (R / 2), c = R + 2 * (i % (R / 2));
             *reinterpret_cast<uint32_t*>(lb + tile_off<2 * R, KT>(row, c)) = 0u;
           }
-        fence_proxy_async_smem();
-        __syncwarp();
+        fence_proxy_async_smem();  // the P V MMA reads V through the async proxy
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(pfull);
       bar_sync(BAR_P + pb, NB);
+      if (pv == 0) {
 #pragma unroll
-      for (int pt = 0; pt < NT; ++pt) {
-        const float c0 = Corr[pb * ROWS + 8 * pt + 2 * t4];
-        const float c1 = Corr[pb * ROWS + 8 * pt + 2 * t4 + 1];
+        for (int pt = 0; pt < NT; ++pt) {
+          const float c0 = Corr[pb * ROWS + 8 * pt + 2 * t4];
+          const float c1 = Corr[pb * ROWS + 8 * pt + 2 * t4 + 1];
 #pragma unroll
-        for (int mt = 0; mt < C::MT; ++mt) {
-          O[mt][pt][0] *= c0; O[mt][pt][2] *= c0;
-          O[mt][pt][1] *= c1; O[mt][pt][3] *= c1;
+          for (int mr = 0; mr < C::MR; ++mr) {
+            Olr[mr][pt][0] *= c0; Olr[mr][pt][2] *= c0;
+            Olr[mr][pt][1] *= c1; Olr[mr][pt][3] *= c1;
+          }
         }
-#pragma unroll
-        for (int mr = 0; mr < C::MR; ++mr) {
-          Olr[mr][pt][0] *= c0; Olr[mr][pt][2] *= c0;
-          Olr[mr][pt][1] *= c1; Olr[mr][pt][3] *= c1;
-        }
-      }
-      const uint32_t pt_u = ptile_u + pb * C::P_TILE;
+        const uint32_t pt_u = ptile_u + pb * C::P_TILE;
 #pragma unroll 2
-      for (int ks = 0; ks < KT / 16; ++ks) {
-        uint32_t bP[NT][2];
+        for (int ks = 0; ks < KT / 16; ++ks) {
+          uint32_t bP[NT][2];
 #pragma unroll
-        for (int pt = 0; pt < NT; ++pt)
-          ldsm_x2(bP[pt][0], bP[pt][1], pt_u + tile_off<KT, ROWS>(8 * pt + rr, 16 * ks + ((lane >> 3) & 1) * 8));
-#pragma unroll
-        for (int mt = 0; mt < C::MT; ++mt) {
-          uint32_t aV[4];
-          ldsm_x4_t(aV, sV + tile_off<D, KT>(16 * ks + rr + (mi >> 1) * 8, d0 + 16 * mt + (mi & 1) * 8));
-#pragma unroll
-          for (int pt = 0; pt < NT; ++pt) mma16816(O[mt][pt], aV, bP[pt][0], bP[pt][1]);
-        }
-        if (pv == 0) {
+          for (int pt = 0; pt < NT; ++pt)
+            ldsm_x2(bP[pt][0], bP[pt][1], pt_u + tile_off<KT, ROWS>(8 * pt + rr, 16 * ks + ((lane >> 3) & 1) * 8));
 #pragma unroll
           for (int mr = 0; mr < C::MR; ++mr) {
             uint32_t aV[4];
@@ -1195,25 +1228,24 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
     }
     bar_sync(BAR_END, TC_NTHR);
     float* Mo = reinterpret_cast<float*>(area);
+    if (pv == 0) {
 #pragma unroll
-    for (int pt = 0; pt < NT; ++pt)
+      for (int pt = 0; pt < NT; ++pt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int row = 8 * pt + 2 * t4 + (e & 1);
-        const int dd = gq + (e >> 1) * 8;
-#pragma unroll
-        for (int mt = 0; mt < C::MT; ++mt) Mo[row * W + d0 + 16 * mt + dd] = O[mt][pt][e];
-        if (pv == 0) {
+        for (int e = 0; e < 4; ++e) {
+          const int row = 8 * pt + 2 * t4 + (e & 1);
+          const int dd = gq + (e >> 1) * 8;
 #pragma unroll
           for (int mr = 0; mr < C::MR; ++mr)
             if (16 * mr + dd < R) Mo[row * W + D + 16 * mr + dd] = Olr[mr][pt][e];
         }
-      }
+    }
   } else {
     // ======================================================== TMA / MMA warp
     if (lane == 0) {
       constexpr uint32_t ID_S = umma_idesc_bf16(128, QPAD, 0, 0);
       constexpr uint32_t ID_E = umma_idesc_bf16(128, D, 0, 1);
+      constexpr uint32_t ID_PV = umma_idesc_bf16(128, QPAD, 1, 0);   // O^T += V^T P^T, A = V MN-major
       const uint64_t dQ = umma_desc(qu_u, 16, 1024, 2);
       const uint64_t dBk = umma_desc(bks_u, R * 128, 1024, 2);
       if (n_tiles > 0 && !mbar_wait(bkbar, 0)) fail = 1;
@@ -1232,6 +1264,23 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
         for (int b = 0; b < (2 * R) / LB; ++b) tma_prefetch_l2_3d(&tmL, LB * b, key0, seq);
       };
       for (int m = ST; m < n_tiles && m < ST + kL2Ahead; ++m) prefetch(m);
+      auto mma_pv = [&](int m) {  // O^T (d x query rows) += V_base^T P^T over the tile's keys
+        const int sm = m % ST;
+        if (!mbar_wait(pfull, m & 1)) fail = 1;
+        tc_fence_after();
+        // P^T as the K-major B operand: the P tile's ROWS rows in 64-key boxes
+        // (ROWS * 128 bytes apart); with N = QPAD > ROWS the MMA also reads the
+        // next rows' bytes (the next box, the next buffer or the softmax
+        // scratch, all inside shared memory) into O^T columns that are never read
+        const uint64_t dV = umma_desc(area_u + sm * C::STAGE + C::KV_TILE, KT * 128, 1024, 2);
+        const uint64_t dP = umma_desc(ptile_u + (m & 1) * C::P_TILE, 16, 1024, 2);
+#pragma unroll
+        for (int kk = 0; kk < KT / 16; ++kk)
+          umma_bf16(tmem + TC_OCOL, umma_desc_add(dV, kk * 16 * 128),
+                    umma_desc_add(dP, (kk >> 2) * (ROWS * 128) + (kk & 3) * 32), ID_PV, (m > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(pvdone);
+        umma_commit(empty_u + 8 * sm);  // the stage's K, LRk and V have been read
+      };
       for (int n = 0; n < n_tiles; ++n) {
         const int s = n % ST;
         const uint32_t sK = area_u + s * C::STAGE;
@@ -1254,7 +1303,7 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
             umma_bf16(tmem + 128 * a, umma_desc_add(dL, ks * 32), umma_desc_add(dB, ks * 16 * 128), ID_E, ks > 0);
         }
         umma_commit(tfull);
-        umma_commit(empty_u + 8 * s);  // K and LRk of this stage have been read
+        if (n > 0) mma_pv(n - 1);
         if (n >= 1 && n - 1 + ST < n_tiles) {
           const int sp = (n - 1) % ST;
           if (!mbar_wait(empty_u + 8 * sp, ((n - 1) / ST) & 1)) fail = 1;
@@ -1262,6 +1311,7 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
           if (n - 1 + ST + kL2Ahead < n_tiles) prefetch(n - 1 + ST + kL2Ahead);
         }
       }
+      if (n_tiles > 0) mma_pv(n_tiles - 1);
       for (int n = n_tiles; n < n_spec; ++n)  // loaded ahead of kv_len and not used
         if (!mbar_wait(full_u + 8 * n, 0)) fail = 1;
     }
