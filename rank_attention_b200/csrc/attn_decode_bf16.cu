@@ -720,11 +720,10 @@ struct TCfg {
   }
 };
 
+// Q' = R(-k0) Q scaled by s for one frequency i of every row, from the
+// scaled (cos, sin)(k0 theta_i) (bf16 in, bf16 out; swizzled 64-column boxes).
 template <int D, int SRC_ROWS, int DST_ROWS>
-__device__ __forceinline__ void rotate_queries_tc(uint32_t qs_u, uint32_t qp_u, const double* theta,
-                                                  int64_t t, float s, int i) {
-  const float2 cs = rope_cs_exact(t, theta[i]);
-  const float c = cs.x * s, sn = cs.y * s;
+__device__ __forceinline__ void rotate_queries_cs(uint32_t qs_u, uint32_t qp_u, float c, float sn, int i) {
 #pragma unroll 4
   for (int row = 0; row < DST_ROWS; ++row) {
     uint16_t a, b;
@@ -761,7 +760,8 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* area = smem;
   unsigned char* ptile = area + C::AREA;
-  float* Mx = reinterpret_cast<float*>(ptile + 2 * C::P_TILE);   // [2][NES][ROWS]
+  float* Mx = reinterpret_cast<float*>(ptile + 2 * C::P_TILE);   // [2][ROWS][NES]
+  static_assert(TC_NES == 8, "a row's maxima are read as two float4");
   float* Corr = Mx + 2 * TC_NES * ROWS;                          // [2][ROWS]
   float* Lw = Corr + 2 * ROWS;                                   // [NES][ROWS]
   double* theta = reinterpret_cast<double*>(Lw + TC_NES * ROWS); // [64]
@@ -1036,7 +1036,6 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
       // tile row maxima over all score warps
       const bool v0 = kw0 + gq < k_hi, v1 = kw0 + gq + 8 < k_hi;
       float x[NT][4];
-      float* mxw = Mx + (pb * TC_NES + w) * ROWS;
 #pragma unroll
       for (int pt = 0; pt < NT; ++pt) {
         x[pt][0] = v0 ? S[pt][0] * sl2 : -INFINITY;
@@ -1049,18 +1048,19 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
           mt_ = fmaxf(mt_, __shfl_xor_sync(0xffffffffu, mt_, 4));
           mt_ = fmaxf(mt_, __shfl_xor_sync(0xffffffffu, mt_, 8));
           mt_ = fmaxf(mt_, __shfl_xor_sync(0xffffffffu, mt_, 16));
-          if (gq == 0) mxw[8 * pt + 2 * t4 + e] = mt_;
+          if (gq == 0) Mx[(pb * ROWS + 8 * pt + 2 * t4 + e) * TC_NES + w] = mt_;
         }
       }
       bar_sync(BAR_MAX, 32 * TC_NES);
+      bool moved = false;   // a running maximum of this lane's rows grew
 #pragma unroll
       for (int pt = 0; pt < NT; ++pt)
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int row = 8 * pt + 2 * t4 + e;
-          float mt_ = -INFINITY;
-#pragma unroll
-          for (int ww = 0; ww < TC_NES; ++ww) mt_ = fmaxf(mt_, Mx[(pb * TC_NES + ww) * ROWS + row]);
+          const float4 ma = *reinterpret_cast<const float4*>(Mx + (pb * ROWS + row) * TC_NES);
+          const float4 mb = *reinterpret_cast<const float4*>(Mx + (pb * ROWS + row) * TC_NES + 4);
+          const float mt_ = fmaxf(max3f(ma.x, ma.y, ma.z), max3f(ma.w, max3f(mb.x, mb.y, mb.z), mb.w));
           const float mo = m_st[pt][e];
           const float mn = fmaxf(mo, mt_);
           const float corr = (mo == -INFINITY) ? 0.f : fast_exp2(mo - mn);
@@ -1070,8 +1070,10 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
           x[pt][e + 2] = p1;
           l_st[pt][e] = l_st[pt][e] * corr + p0 + p1;
           m_st[pt][e] = mn;
+          moved |= corr != 1.f;
           if (w == 0 && gq == 0) Corr[pb * ROWS + row] = corr;
         }
+      const bool any_moved = __any_sync(0xffffffffu, moved);   // over every row (the lanes' t4)
       bar_sync(BAR_PFREE + pb, NB);
       // O^T holds every tile before this one (and P buffer pb, last read by the
       // P V MMA of tile n-2, is free)
@@ -1088,9 +1090,7 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
       // the running maxima moved: O^T (TMEM lanes = d, columns = query rows)
       // times corr, by one warp per sub-partition
       if (n > 0 && w < 4) {
-        bool any = false;
-        for (int row = 0; row < n_rows; ++row) any |= Corr[pb * ROWS + row] != 1.f;
-        if (any) {
+        if (any_moved) {
           tc_fence_after();
 #pragma unroll
           for (int c0 = 0; c0 < QPAD; c0 += 16) {
@@ -1166,14 +1166,29 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
     }
     if (n_tiles > 1) bar_arrive(BAR_PFREE + 1, NB);
     const int d0 = pv * (D / 2);
+    // this lane's frequency i: s (cos, sin)(k0 theta_i) of the tile being
+    // rotated, advanced one tile at a time by the rotation through KT theta_i
+    // in fp32 and taken exactly (fp64) again every 16 tiles
+    const int qi = pv * 32 + lane;
+    float2 qcs = make_float2(0.f, 0.f), qstep = qcs;
+    if (qi < D / 2) {
+      qcs = cs0[qi];
+      qstep = rope_cs_exact(KT, theta[qi]);
+    }
     for (int n = 0; n < n_tiles; ++n) {
       const int s = n % ST, pb = n & 1;
       const uint32_t sL = area_u + s * C::STAGE + 2 * C::KV_TILE;
       const int64_t k0 = k_lo + (int64_t)n * KT;
       if (n + 1 < n_tiles) {
-        const int i = pv * 32 + lane;
-        if (i < D / 2)
-          rotate_queries_tc<D, QPAD, ROWS>(qu_u, qp_u + ((n + 1) & 1) * C::QP_BYTES, theta, k0 + KT, p.s, i);
+        if (qi < D / 2) {
+          if (((n + 1) & 15) == 0) {
+            const float2 cs = rope_cs_exact(k0 + KT, theta[qi]);
+            qcs = make_float2(cs.x * p.s, cs.y * p.s);
+          } else {
+            qcs = make_float2(fmaf(qcs.x, qstep.x, -qcs.y * qstep.y), fmaf(qcs.y, qstep.x, qcs.x * qstep.y));
+          }
+          rotate_queries_cs<D, QPAD, ROWS>(qu_u, qp_u + ((n + 1) & 1) * C::QP_BYTES, qcs.x, qcs.y, qi);
+        }
         bar_arrive(BAR_QP + ((n + 1) & 1), NB);
       }
       if (!mbar_wait(full_u + 8 * s, (n / ST) & 1)) fail = 1;
