@@ -43,6 +43,9 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--all-configs", action="store_true",
+                    help="also time the long-context decode sweep and one layer of the "
+                         "32-layer stack (decode and prefill), reported under other_configs")
     ap.add_argument("--profile", nargs="?", const="decode", choices=["decode", "prefill"],
                     help="a short deterministic run of one kernel for profilers "
                          "(decode: the 8192-token decode five times; prefill: the "
@@ -159,14 +162,14 @@ def time_non_shared(dev, shared_decode_us, reps=5):
                     "with B = 0"}
 
 
-def time_prefill(dev, reps=5, warmup=3):
-    """The chunked prefill workload (16384-token prefix + 1024-token chunk per
-    agent, 3 agents, r = 16): one lora_attn_prefill per launch, CUDA events
-    around each launch, L2 flushed (256 MB written) before each."""
+def time_prefill(dev, reps=5, warmup=3, s=None):
+    """A chunked prefill workload (default: 16384-token prefix + 1024-token
+    chunk per agent, 3 agents, r = 16): one lora_attn_prefill per launch, CUDA
+    events around each launch, L2 flushed (256 MB written) before each."""
     import torch
     from rank_attention_b200 import lora_attn as la
     from rank_attention_b200 import workloads as W
-    s = W.LLAMA8B_PREFILL_16K
+    s = s or W.LLAMA8B_PREFILL_16K
     inp = W.direct_cache_inputs(s, device=dev)
     out = torch.empty(inp["q"].shape, dtype=torch.bfloat16, device=dev)
     args = la.make_args(inp["k_base"], inp["v_base"], inp["lr"], inp["B_k"], inp["B_v"],
@@ -195,6 +198,62 @@ def time_prefill(dev, reps=5, warmup=3):
             "flops_per_launch": base, "lora_inclusive_tflops": lora / (ms / 1e3) / 1e12,
             "peak": peak, "peak_kind": kind, "frac": tf / peak, "out_dtype": "bf16",
             "timing": f"median of {reps} launches, CUDA events, L2 flushed before each"}
+
+
+def time_decode_shape(dev, s, reps=5, warmup=3):
+    """One lora_attn_decode launch of a decode workload, CUDA events around
+    each launch, L2 flushed before each; HBM roofline on its algorithmic bytes."""
+    import torch
+    from rank_attention_b200 import lora_attn as la
+    from rank_attention_b200 import workloads as W
+    inp = W.direct_cache_inputs(s, device=dev)
+    out = torch.empty(inp["q"].shape, dtype=torch.bfloat16, device=dev)
+    args = la.make_args(inp["k_base"], inp["v_base"], inp["lr"], inp["B_k"], inp["B_v"],
+                        inp["q"], out, lora_scale=s.lora_scale, rope_base=s.rope_base,
+                        kv_len=inp["kv_len"], max_kv_len=s.kv_len)
+    ws = la.decode_workspace(args, dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(warmup):
+        la.lora_attn_decode(args, ws)
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(reps):
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        la.lora_attn_decode(args, ws)
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    if la.la_device_check() != 0:
+        raise RuntimeError("decode device check failed")
+    ms = statistics.median(times)
+    hbm, kind = peaks()
+    b = decode_bytes(s)
+    gbs = b / (ms / 1e3) / 1e9
+    return {"workload": s.name, "kind": "decode", "us": ms * 1e3,
+            "agent_tokens_per_s": s.n_seqs * s.n_agents / (ms / 1e3),
+            "algorithmic_bytes": b, "GB/s": gbs, "peak": hbm, "frac": gbs / hbm,
+            "timing": f"median of {reps} launches, CUDA events, L2 flushed before each"}
+
+
+def time_other_configs(dev):
+    """The long-context batched decode sweep (16 requests x 5 agents, r = 32)
+    and one layer of the 32-layer stack (4096-token chunk over a 32768-token
+    prefix, 4 agents, r = 64: prefill, then decode over the 36864 keys)."""
+    import torch
+    from rank_attention_b200 import workloads as W
+    res = []
+    for ctx in W.SWEEP_CTX:
+        res.append(time_decode_shape(dev, W.llama8b_sweep(ctx)))
+        torch.cuda.empty_cache()
+    pf = time_prefill(dev, s=W.llama8b_stack_prefill(0))
+    pf["kind"] = "prefill"
+    res.append(pf)
+    torch.cuda.empty_cache()
+    res.append(time_decode_shape(dev, W.llama8b_stack_decode(0)))
+    torch.cuda.empty_cache()
+    return res
 
 
 class ClockSampler:
@@ -245,7 +304,7 @@ class ClockSampler:
 # DRAM bytes per decode launch from an ncu capture of the workload, keyed by the
 # sha256 prefix of the decode kernel's source: reported only while the kernel is
 # unchanged since the counters were taken.
-DECODE_TRAFFIC = {"620567e7b5bcb3ce": 34402816}
+DECODE_TRAFFIC = {"0118cb326e4aeb7f": 34415104}
 
 
 def decode_source_sha() -> str:
@@ -561,6 +620,8 @@ def run_ours(args):
         "prefill": prefill,
         "non_shared_baseline": non_shared,
     }
+    if args.all_configs:
+        line["other_configs"] = time_other_configs(dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, n, per = time_oracle(s, 20, 15.0)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": blas_threads(),
