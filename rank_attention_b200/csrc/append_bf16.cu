@@ -67,6 +67,9 @@ __global__ void __launch_bounds__(NTHR, 1)
   const int nk = ke - kb;
   cg::cluster_group cluster = cg::this_cluster();
 
+  // the next kernel of the stream (the decode of the step) may start its
+  // set-up now; it waits for this grid's completion before reading the LR cache
+  pdl_launch_dependents();
   if (tid == 0) {
     for (int s = 0; s < NSTAGE; ++s) mbar_init(bar_u + 8 * s, 1);
     fence_mbar_init();

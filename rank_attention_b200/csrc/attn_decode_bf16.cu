@@ -840,16 +840,20 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
     mbar_init(pfull, TC_NES + NPV);
     mbar_init(pvdone, 1);
     fence_mbar_init();
+    tma_prefetch(&tmB);
+    tma_prefetch(&tmK);
+    tma_prefetch(&tmV);
+    tma_prefetch(&tmL);
+    // launched as a programmatic dependent of the preceding kernel (the LR
+    // append of the step): everything above overlaps its tail; every read of
+    // an input comes after the wait (a no-op without a preceding kernel)
+    pdl_wait();
     // each agent's g query rows of this KV head are contiguous
     const __nv_bfloat16* Q = reinterpret_cast<const __nv_bfloat16*>(p.q);
     mbar_expect_tx(qbar, (uint32_t)(n_rows * D * 2));
     for (int a = 0; a < na; ++a)
       bulk_load(ptile_u + a * g * D * 2, Q + (((int64_t)seq * na_tot + agent0 + a) * p.n_q + kvh * g) * D,
                 (uint32_t)(g * D * 2), qbar);
-    tma_prefetch(&tmB);
-    tma_prefetch(&tmK);
-    tma_prefetch(&tmV);
-    tma_prefetch(&tmL);
     // B_k^a head slices (r rows x 64 d boxes, the MN-major MMA operand)
     mbar_expect_tx(bkbar, (uint32_t)(na * C::BK_BYTES));
     for (int a = 0; a < na; ++a)
@@ -860,6 +864,7 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
     // (by max_kv_len) past the sequence's length are loaded but never used
     for (int n = 0; n < n_spec; ++n) issue(n);
   }
+  pdl_wait();
   const int64_t kvl = p.kv_len[seq];  // in flight while the constants are computed
   const int sp = w & 3, kb = 32 * sp + 16 * (w >> 2);  // score warp: TMEM sub-partition, first key
   // R(j) for this thread's keys j = kb + gq + 8 hh and its frequencies
@@ -1719,13 +1724,26 @@ cudaError_t launch_tc(const AttnParams& p, cudaStream_t st) {
   cfg.blockDim = dim3(TC_NTHR);
   cfg.dynamicSmemBytes = sm;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
+  // the set-up may overlap the preceding kernel (programmatic dependent
+  // launch; the kernel waits for it before reading any input)
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[na++].val.programmaticStreamSerializationAllowed = 1;
+  if (p.n_splits > 1) {
+    attr[na].id = cudaLaunchAttributeCooperative;
+    attr[na++].val.cooperative = 1;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = p.n_splits > 1 ? 1 : 0;
+  cfg.numAttrs = na;
   e = cudaLaunchKernelEx(&cfg, kern, mk, mv, ml, mb, p, rt);
-  if (e != cudaSuccess) return e;
+  if (e != cudaSuccess) {  // without the overlap where the runtime refuses the pair of attributes
+    cudaGetLastError();
+    cfg.attrs = attr + 1;
+    cfg.numAttrs = na - 1;
+    e = cudaLaunchKernelEx(&cfg, kern, mk, mv, ml, mb, p, rt);
+    if (e != cudaSuccess) return e;
+  }
   return cudaGetLastError();
 }
 
