@@ -23,6 +23,12 @@ What it computes, and from which passage:
   V^a_t = V_base,t + s LRv_t B_v^a, with s = alpha / r.
 * Attention of one head over accumulated length L = L_p + L_c with a causal
   mask -- LRAgent summary App. B "Flash-LoRA-Attention".
+* Optionally one LR cache per agent, X A_a, when every agent owns its own
+  down-projection A_a (BaseShared: only the base cache is shared) -- LRAgent
+  summary §3 "BaseShared"; LRAgent explainer, "Esquemas de Compartilhamento",
+  BaseShared.  PreLRShared fills every agent's cache when a chunk first passes
+  through the model -- PReCache blog (rit.work), how PReCache precomputes each
+  role's cache.
 
 The oracle MATERIALISES every agent's full K^a and V^a and runs a naive
 two-pass softmax (max, then exp / sum).  It does not use the reordered value
@@ -95,6 +101,14 @@ def lr_cache_append(lr_cache, X, A_kv, pos0: int) -> np.ndarray:
     n = rows.shape[-2]
     out[:, pos0:pos0 + n, :] = rows
     return out
+
+
+def lr_cache_append_agents(lr_caches, X, A_kv_agents, pos0: int) -> np.ndarray:
+    """Every agent's own LR cache (BaseShared, filled by PreLRShared): a copy of
+    lr_caches [n_agents, n_seqs, L_max, 2r] whose agent a has rows
+    pos0..pos0+n-1 replaced by X @ A_kv_agents[a] ([H, 2r])."""
+    return np.stack([lr_cache_append(lr_caches[a], X, A_kv_agents[a], pos0)
+                     for a in range(len(A_kv_agents))])
 
 
 # ----------------------------------------------------------------------------
@@ -177,7 +191,8 @@ def lora_attention_unit(k_base, v_base, lr, B_k, B_v, q, *, seq: int, agent: int
     g = n_q // k_base.shape[1]
     L = int(kv_len)
     kpos = np.arange(L)
-    lr_s = _np64(lr[seq, :L])
+    # the agent's own LR cache (BaseShared), or the one shared by all agents
+    lr_s = _np64(lr[agent, seq, :L] if lr.ndim == 4 else lr[seq, :L])
     cols = slice(kv_head * d, (kv_head + 1) * d)
     Ka = agent_keys(k_base[seq, kv_head, :L], lr_s[:, :r], _np64(B_k[agent])[:, cols],
                     lora_scale, kpos, rope_base)
@@ -199,7 +214,8 @@ def lora_attention(k_base, v_base, lr, B_k, B_v, q, kv_len, *, lora_scale: float
                    q_pos0: int = None) -> np.ndarray:
     """Every agent's attention output over the shared base and LR caches.
 
-    k_base, v_base [n_seqs, n_kv, L_max, d]; lr [n_seqs, L_max, 2r];
+    k_base, v_base [n_seqs, n_kv, L_max, d]; lr [n_seqs, L_max, 2r] shared by
+    every agent, or [n_agents, n_seqs, L_max, 2r], one cache per agent;
     B_k, B_v [n_agents, r, n_kv*d]; q [n_seqs, n_agents, n_tok, n_q, d];
     kv_len [n_seqs].  Returns out [n_seqs, n_agents, n_tok, n_q, d] in fp64.
     """

@@ -51,6 +51,7 @@ class AttnShape:
     dtype: torch.dtype   # storage dtype of caches, weights and queries
     seed: int
     mode: str            # "decode" or "prefill"
+    lr_per_agent: bool = False   # one LR cache per agent (own A_a: BaseShared) instead of one shared
 
     @property
     def group(self) -> int:
@@ -174,7 +175,9 @@ def direct_cache_inputs(shape: AttnShape, device="cpu", L_max: Optional[int] = N
     """Base K/V, LR cache, B_k, B_v and queries drawn directly (LLaMA-shaped cases).
 
     Layouts: k_base, v_base [n_seqs, n_kv, L_max, d]; lr [n_seqs, L_max, 2r]
-    (LR_k columns first); B_k, B_v [n_agents, r, n_kv*d];
+    (LR_k columns first), or [n_agents, n_seqs, L_max, 2r] with
+    shape.lr_per_agent (agent a's cache drawn after agent a-1's);
+    B_k, B_v [n_agents, r, n_kv*d];
     q [n_seqs, n_agents, n_q_tokens, n_q_heads, d]; kv_len int32 [n_seqs].
     Rows at or beyond kv_len are left at zero.
     """
@@ -184,11 +187,15 @@ def direct_cache_inputs(shape: AttnShape, device="cpu", L_max: Optional[int] = N
     dt = shape.dtype
     k_base = torch.zeros((shape.n_seqs, n_kv, L_max, d), dtype=dt, device=device)
     v_base = torch.zeros_like(k_base)
-    lr = torch.zeros((shape.n_seqs, L_max, 2 * r), dtype=dt, device=device)
+    n_lr = shape.n_agents if shape.lr_per_agent else 1
+    lr = torch.zeros((n_lr, shape.n_seqs, L_max, 2 * r), dtype=dt, device=device)
     L = shape.kv_len
     k_base[:, :, :L] = _normal((shape.n_seqs, n_kv, L, d), CACHE_STD, dt, g, device)
     v_base[:, :, :L] = _normal((shape.n_seqs, n_kv, L, d), CACHE_STD, dt, g, device)
-    lr[:, :L] = _normal((shape.n_seqs, L, 2 * r), CACHE_STD, dt, g, device)
+    for a in range(n_lr):
+        lr[a, :, :L] = _normal((shape.n_seqs, L, 2 * r), CACHE_STD, dt, g, device)
+    if not shape.lr_per_agent:
+        lr = lr[0]
     b_std = 0.02 if with_lora else 0.0
     B_k = _normal((shape.n_agents, r, n_kv * d), b_std, dt, g, device)
     B_v = _normal((shape.n_agents, r, n_kv * d), b_std, dt, g, device)

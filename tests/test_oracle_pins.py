@@ -187,6 +187,90 @@ def test_brute_force_llama_like_rope_base():
     assert brute_force_error(seed=2, d=16, r=4, L=9, n_tok=4, base=500000.0) < 1e-12
 
 
+# ------------------------------------------------ one LR cache per agent ----
+def per_agent_problem(seed=3, **kw):
+    """The tiny problem with a down-projection A_a of its own for every agent
+    (BaseShared: only the base cache is shared)."""
+    p = tiny_problem(seed=seed, **kw)
+    rng = np.random.default_rng(100 + seed)
+    n_agents, H, r = p["B_k"].shape[0], p["X"].shape[-1], p["B_k"].shape[1]
+    p["A_k"] = rng.standard_normal((n_agents, H, r)) / math.sqrt(H)
+    p["A_v"] = rng.standard_normal((n_agents, H, r)) / math.sqrt(H)
+    return p
+
+
+def per_agent_brute_force_error(mode="prefill", seed=3, **kw):
+    """Per-agent merged weights W + s A_a B_a against the oracle fed every agent's
+    own LR cache X A_a (filled by the per-agent append)."""
+    p = per_agent_problem(seed=seed, **kw)
+    n_agents = p["B_k"].shape[0]
+    q = p["q"] if mode == "prefill" else p["q"][:, :, -1:]
+    ref = np.empty(q.shape)
+    for a in range(n_agents):
+        pa = dict(p, A_k=p["A_k"][a], A_v=p["A_v"][a], B_k=p["B_k"][a:a + 1],
+                  B_v=p["B_v"][a:a + 1], q=q[:, a:a + 1])
+        ref[:, a:a + 1] = brute_force(pa, mode)
+    k_base, v_base = impl.base_cache_from_hidden(p["X"], p["W_k"], p["W_v"], p["n_kv"], p["base"])
+    A_kv = np.concatenate([p["A_k"], p["A_v"]], axis=2)       # [n_agents, H, 2r]
+    n_seqs, L = p["X"].shape[0], p["L"]
+    lr = impl.lr_cache_append_agents(np.zeros((n_agents, n_seqs, L, A_kv.shape[2])), p["X"], A_kv, 0)
+    got = impl.lora_attention(k_base, v_base, lr, p["B_k"], p["B_v"], q, np.full(n_seqs, L),
+                              lora_scale=p["s"], softmax_scale=1 / math.sqrt(p["d"]),
+                              rope_base=p["base"], mode=mode)
+    return np.abs(got - ref).max() / np.abs(ref).max()
+
+
+@pytest.mark.parametrize("mode", ["prefill", "decode"])
+def test_brute_force_per_agent_down_projections(mode):
+    assert per_agent_brute_force_error(mode=mode) < 1e-12
+
+
+def test_per_agent_caches_all_equal_reduce_to_the_shared_cache():
+    rng = np.random.default_rng(7)
+    n_seqs, n_agents, n_q, n_kv, d, L, r = 2, 3, 4, 2, 8, 9, 2
+    k_base = rng.standard_normal((n_seqs, n_kv, L, d))
+    v_base = rng.standard_normal((n_seqs, n_kv, L, d))
+    lr = rng.standard_normal((n_seqs, L, 2 * r))
+    B_k, B_v = rng.standard_normal((2, n_agents, r, n_kv * d))
+    q = rng.standard_normal((n_seqs, n_agents, 3, n_q, d))
+    kw = dict(lora_scale=1.5, softmax_scale=0.3, rope_base=100.0, mode="prefill")
+    shared = impl.lora_attention(k_base, v_base, lr, B_k, B_v, q, np.full(n_seqs, L), **kw)
+    each = impl.lora_attention(k_base, v_base, np.stack([lr] * n_agents), B_k, B_v, q,
+                               np.full(n_seqs, L), **kw)
+    np.testing.assert_array_equal(shared, each)
+
+
+def test_per_agent_append_against_python_loops():
+    rng = np.random.default_rng(8)
+    n_agents, n_seqs, L, H, r, n, pos0 = 2, 2, 6, 5, 2, 3, 2
+    X = rng.standard_normal((n_seqs, n, H))
+    A = rng.standard_normal((n_agents, H, 2 * r))
+    old = rng.standard_normal((n_agents, n_seqs, L, 2 * r))
+    got = impl.lr_cache_append_agents(old, X, A, pos0)
+    for a in range(n_agents):
+        for q in range(n_seqs):
+            for t in range(L):
+                for c in range(2 * r):
+                    if pos0 <= t < pos0 + n:
+                        want = sum(X[q, t - pos0, k] * A[a, k, c] for k in range(H))
+                    else:
+                        want = old[a, q, t, c]
+                    assert abs(got[a, q, t, c] - want) <= 1e-12 * (1 + abs(want))
+
+
+def _bad_unit_first_agents_cache(k_base, v_base, lr, B_k, B_v, q, **kw):
+    # reads agent 0's LR cache for every agent
+    lr2 = np.asarray(impl._np64(lr))
+    if lr2.ndim == 4:
+        lr2 = np.stack([lr2[0]] * lr2.shape[0])
+    return _orig_unit(k_base, v_base, lr2, B_k, B_v, q, **kw)
+
+
+def test_planted_per_agent_cache_mistake_is_caught(monkeypatch):
+    monkeypatch.setattr(impl, "lora_attention_unit", _bad_unit_first_agents_cache)
+    assert per_agent_brute_force_error(mode="prefill") > 1e-6
+
+
 def test_reordered_value_path_identity():
     rng = np.random.default_rng(5)
     L, d, r, s = 13, 16, 4, 2.0
