@@ -95,6 +95,30 @@ la_status lr_cache_append(const void* X, int64_t ldx, int64_t n_tokens, int64_t 
                           int64_t pos0, int32_t n_seqs, int64_t seq_stride_x,
                           int64_t seq_stride_lr, la_dtype dt, la_stream_t stream);
 
+/*
+ * lr_cache_append_agents -- PreLRShared precompute of every agent's own LR
+ * cache when each agent a has its own down-projection A_a (BaseShared): the
+ * new chunk's hidden states are multiplied by every agent's A_a as they first
+ * pass through the model (PReCache blog, how PReCache precomputes each role's
+ * cache; LRAgent summary §3 "BaseShared": Y_lr,a = X A_a).
+ *
+ * For every agent a in [0, n_agents), sequence q and chunk row i:
+ *   lr_cache[a][q][pos0 + i][c] = sum_k X[q][i][k] * A_kv[a][k][c]
+ * with the layout, rounding and untouched rows of lr_cache_append.
+ *
+ *   A_kv      [n_agents][hidden][2r], each agent's [A_k,a | A_v,a] contiguous.
+ *   lr_cache  agent a's cache starts at lr_cache + a * lr_agent_stride
+ *             (elements; a multiple of 16 bytes, at least
+ *             (n_seqs - 1) * seq_stride_lr + L_max * 2r).
+ * Other arguments and errors as lr_cache_append; n_agents < 1 or a bad
+ * lr_agent_stride is LA_ERR_INVALID_ARG.
+ */
+la_status lr_cache_append_agents(const void* X, int64_t ldx, int64_t n_tokens, int64_t hidden,
+                                 const void* A_kv, int32_t n_agents, int32_t r, void* lr_cache,
+                                 int64_t lr_agent_stride, int64_t L_max, int64_t pos0,
+                                 int32_t n_seqs, int64_t seq_stride_x, int64_t seq_stride_lr,
+                                 la_dtype dt, la_stream_t stream);
+
 /* Arguments shared by lora_attn_prefill and lora_attn_decode. */
 typedef struct {
   int32_t n_seqs;       /* independent sequences, each with its own caches */
@@ -132,6 +156,16 @@ typedef struct {
   int32_t n_q_tokens;   /* decode: must be 1 */
   la_dtype io_dtype;    /* dtype of k_base, v_base, lr_cache, B_k, B_v and q */
   la_dtype out_dtype;   /* dtype of out */
+  /* Elements between two agents' LR caches.  0: one LR cache shared by every
+   * agent (shared A: BaseLRShared).  > 0: agent a owns its down-projection A_a
+   * and reads its own LR cache X A_a (BaseShared; filled for every agent at
+   * once by lr_cache_append_agents, PreLRShared), laid out as above and
+   * starting at lr_cache + a * lr_agent_stride; a multiple of 16 bytes, at
+   * least (n_seqs - 1) * lr_seq_stride + L_max * 2r (the caches do not
+   * overlap).  LRAgent summary §3 "BaseShared"; LRAgent explainer, "Esquemas
+   * de Compartilhamento"; PReCache blog, how PReCache precomputes each
+   * role's cache.  The base cache stays shared in both cases. */
+  int64_t lr_agent_stride;
 } la_attn_args;
 
 /*

@@ -22,6 +22,7 @@ int* error_word_ptr() {
 
 size_t simt_rows_cap(const AttnParams& p);
 int simt_key_tile();
+size_t simt_smem_bytes(const AttnParams& p);
 bool bf16_decode_supported(const AttnParams& p);
 size_t bf16_decode_partial_bytes(const AttnParams& p);
 void bf16_decode_plan(const AttnParams& p, int* n_splits, int64_t* split_len, int* rows, int* groups);
@@ -62,6 +63,10 @@ la_status check_attn(const la_attn_args* a, int decode, AttnParams* p) {
     return LA_ERR_INVALID_ARG;
   if (a->lr_seq_stride < a->L_max * 2 * a->r || !stride_ok(a->lr_seq_stride, io))
     return LA_ERR_INVALID_ARG;
+  if (a->lr_agent_stride != 0 &&
+      (!stride_ok(a->lr_agent_stride, io) ||
+       a->lr_agent_stride < (int64_t)(a->n_seqs > 0 ? a->n_seqs - 1 : 0) * a->lr_seq_stride + a->L_max * 2 * a->r))
+    return LA_ERR_INVALID_ARG;
   const int g = a->n_q_heads / a->n_kv_heads;
   if ((int64_t)a->n_agents * g > kMaxRowsSimt) return LA_ERR_UNSUPPORTED;
   if (decode) {
@@ -93,6 +98,7 @@ la_status check_attn(const la_attn_args* a, int decode, AttnParams* p) {
   p->kv_tok = a->kv_tok_stride;
   p->lr = a->lr_cache;
   p->lr_seq = a->lr_seq_stride;
+  p->lr_agent = a->lr_agent_stride;
   p->B_k = a->B_k;
   p->B_v = a->B_v;
   p->q = a->q;
@@ -186,6 +192,32 @@ extern "C" la_status lr_cache_append(const void* X, int64_t ldx, int64_t n_token
   return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
 }
 
+extern "C" la_status lr_cache_append_agents(const void* X, int64_t ldx, int64_t n_tokens,
+                                            int64_t hidden, const void* A_kv, int32_t n_agents,
+                                            int32_t r, void* lr_cache, int64_t lr_agent_stride,
+                                            int64_t L_max, int64_t pos0, int32_t n_seqs,
+                                            int64_t seq_stride_x, int64_t seq_stride_lr,
+                                            la_dtype dt, la_stream_t stream) {
+  if (!dtype_ok(dt) || n_agents < 1) return LA_ERR_INVALID_ARG;
+  if (n_agents > 1) {
+    if (!stride_ok(lr_agent_stride, dt)) return LA_ERR_INVALID_ARG;
+    if (rank_ok(r) && n_seqs >= 1 && L_max >= 1 &&
+        lr_agent_stride < (int64_t)(n_seqs - 1) * seq_stride_lr + L_max * 2 * r)
+      return LA_ERR_INVALID_ARG;
+  }
+  // agent a: the single-A append of X A_a into its own cache; the checks of
+  // the first call cover every agent (same shapes, strides and alignment)
+  const size_t a_bytes = (size_t)hidden * 2 * r * esize(dt);
+  for (int32_t a = 0; a < n_agents; ++a) {
+    const la_status st = lr_cache_append(
+        X, ldx, n_tokens, hidden, A_kv ? static_cast<const char*>(A_kv) + a * a_bytes : nullptr, r,
+        lr_cache ? static_cast<char*>(lr_cache) + (size_t)a * lr_agent_stride * esize(dt) : nullptr,
+        L_max, pos0, n_seqs, seq_stride_x, seq_stride_lr, dt, stream);
+    if (st != LA_OK) return st;
+  }
+  return LA_OK;
+}
+
 namespace la {
 // Byte range of the arrival counters inside a decode workspace for these
 // arguments (they must read zero when a decode starts).  False if invalid.
@@ -217,6 +249,7 @@ extern "C" la_status lora_attn_decode(const la_attn_args* a, void* workspace,
     return LA_ERR_WORKSPACE;
   if (p.n_seqs == 0) return LA_OK;
   if ((int64_t)p.n_seqs * p.n_kv > 65535) return LA_ERR_UNSUPPORTED;
+  if (d.kind == 0 && simt_smem_bytes(p) > 227 * 1024) return LA_ERR_UNSUPPORTED;
   p.n_splits = d.n_splits;
   p.split_len = d.split_len;
   p.partials = static_cast<float*>(workspace);
@@ -235,14 +268,13 @@ extern "C" la_status lora_attn_prefill(const la_attn_args* a, la_stream_t stream
   if (s != LA_OK) return s;
   if (p.n_seqs == 0 || p.n_q_tokens == 0) return LA_OK;
   if ((int64_t)p.n_seqs * p.n_kv > 65535) return LA_ERR_UNSUPPORTED;
+  const bool tc = a->io_dtype == LA_BF16 && bf16_prefill_supported(p);
+  if (!tc && simt_smem_bytes(p) > 227 * 1024) return LA_ERR_UNSUPPORTED;
   p.err = error_word_ptr();
   if (!p.err) return LA_ERR_CUDA;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e;
-  if (a->io_dtype == LA_BF16 && bf16_prefill_supported(p))
-    e = launch_prefill_bf16(p, a->out_dtype, st);
-  else
-    e = launch_attn_simt(p, a->io_dtype, a->out_dtype, st);
+  const cudaError_t e = tc ? launch_prefill_bf16(p, a->out_dtype, st)
+                           : launch_attn_simt(p, a->io_dtype, a->out_dtype, st);
   return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
 }
 

@@ -194,7 +194,7 @@ __global__ void __launch_bounds__(NTHR, 1)
     constexpr int LB = (2 * R) < 64 ? 2 * R : 64;
 #pragma unroll
     for (int b = 0; b < (2 * R) / LB; ++b)
-      tma_load_3d(sb + 2 * C::KV_TILE + b * KT * LB * 2, &tmL, bar, LB * b, key0, seq);
+      tma_load_4d(sb + 2 * C::KV_TILE + b * KT * LB * 2, &tmL, bar, LB * b, key0, seq, 0);
   };
   if (tid == 0) {
     for (int n = 0; n < ST && n < n_tiles; ++n) issue(n);
@@ -784,6 +784,7 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
   // unit are adjacent in launch order, so its cache tiles are read from HBM once
   // and are L2 hits for the other groups)
   const int agent0 = blockIdx.y * p.agent_group;
+  const int lra = p.lr_agent ? agent0 : 0;   // LR cache of the CTA's agent (one per CTA then)
   const int g = p.g, na = min(p.agent_group, p.n_agents - agent0), n_rows = na * g;
   const int na_tot = p.n_agents;
   const int unitg = blockIdx.y * (p.n_seqs * p.n_kv) + unit;   // (agent group, unit)
@@ -822,7 +823,7 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
     constexpr int LB = (2 * R) < 64 ? 2 * R : 64;
 #pragma unroll
     for (int b = 0; b < (2 * R) / LB; ++b)
-      tma_load_3d(sb + 2 * C::KV_TILE + b * KT * LB * 2, &tmL, bar, LB * b, key0, seq);
+      tma_load_4d(sb + 2 * C::KV_TILE + b * KT * LB * 2, &tmL, bar, LB * b, key0, seq, lra);
   };
 
   // ---- first loads (independent of kv_len): queries, B_k^a, the first tiles, B_v^a
@@ -1281,7 +1282,7 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
         }
         constexpr int LB = (2 * R) < 64 ? 2 * R : 64;
 #pragma unroll
-        for (int b = 0; b < (2 * R) / LB; ++b) tma_prefetch_l2_3d(&tmL, LB * b, key0, seq);
+        for (int b = 0; b < (2 * R) / LB; ++b) tma_prefetch_l2_4d(&tmL, LB * b, key0, seq, lra);
       };
       for (int m = ST; m < n_tiles && m < ST + kL2Ahead; ++m) prefetch(m);
       auto mma_pv = [&](int m) {  // O^T (d x query rows) += V_base^T P^T over the tile's keys
@@ -1564,11 +1565,14 @@ bool make_maps(const AttnParams& p, CUtensorMap* mk, CUtensorMap* mv, CUtensorMa
           one, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return false;
+  // LR caches [n_lr][n_seqs][L_max][2r]: one shared cache, or one per agent
   const int lb = 2 * R < 64 ? 2 * R : 64;
-  cuuint64_t ldims[3] = {(cuuint64_t)(2 * R), (cuuint64_t)p.L_max, (cuuint64_t)p.n_seqs};
-  cuuint64_t lstr[2] = {(cuuint64_t)(2 * R * 2), (cuuint64_t)p.lr_seq * 2};
-  cuuint32_t lbox[3] = {(cuuint32_t)lb, (cuuint32_t)KT, 1};
-  if (enc(ml, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(p.lr), ldims, lstr, lbox, one,
+  const int64_t n_lr = p.lr_agent ? p.n_agents : 1;
+  const int64_t lr_agent_b = p.lr_agent ? p.lr_agent * 2 : p.lr_seq * 2 * p.n_seqs;
+  cuuint64_t ldims[4] = {(cuuint64_t)(2 * R), (cuuint64_t)p.L_max, (cuuint64_t)p.n_seqs, (cuuint64_t)n_lr};
+  cuuint64_t lstr[3] = {(cuuint64_t)(2 * R * 2), (cuuint64_t)p.lr_seq * 2, (cuuint64_t)lr_agent_b};
+  cuuint32_t lbox[4] = {(cuuint32_t)lb, (cuuint32_t)KT, 1, 1};
+  if (enc(ml, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(p.lr), ldims, lstr, lbox, one,
           CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(lb * 2), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return false;
@@ -1685,7 +1689,10 @@ int tc_group_size(const AttnParams& p) {
   if (p.d != 128 || !(p.r == 16 || p.r == 32 || p.r == 64)) return 0;
   if (!(p.g == 1 || p.g == 2 || p.g == 4 || p.g == 8)) return 0;
   if (p.L_max >= (1ll << 31)) return 0;
-  for (int G = p.n_agents < 3 ? p.n_agents : 3; G >= 1; --G)
+  // with one LR cache per agent a CTA holds one agent (its tiles are the
+  // agent's own LR rows beside the shared base tiles)
+  const int gmax = p.lr_agent ? 1 : 3;
+  for (int G = p.n_agents < gmax ? p.n_agents : gmax; G >= 1; --G)
     if (tc_fits(p, G)) return G;
   return 0;
 }
@@ -1751,6 +1758,7 @@ cudaError_t launch_tc(const AttnParams& p, cudaStream_t st) {
 
 bool bf16_decode_supported(const AttnParams& p) {
   if (tc_supported(p)) return true;
+  if (p.lr_agent) return false;   // the generic kernel serves per-agent LR caches otherwise
   if (p.d != 128) return false;
   if (!(p.g == 1 || p.g == 2 || p.g == 4 || p.g == 8)) return false;
   const int NT = n_rowtiles(p);

@@ -109,6 +109,7 @@ __global__ void __launch_bounds__(PNTHR, 1)
   const int gq = lane >> 2, t4 = lane & 3;
   const int seq = blockIdx.z;
   const int agent = blockIdx.y / p.n_kv, kvh = blockIdx.y % p.n_kv;
+  const int lra = p.lr_agent ? agent : 0;   // the agent's own LR cache, or the shared one
   const int g = p.g, na = p.n_agents;
   const int QB = PM / g;
   const int tok0 = (int)(blockIdx.x / ksplit) * QB;
@@ -130,7 +131,7 @@ __global__ void __launch_bounds__(PNTHR, 1)
     mbar_expect_tx(bar, (uint32_t)(C::KV + PKT * R * 2));
 #pragma unroll
     for (int b = 0; b < D / 64; ++b) tma_load_4d(base + b * PKT * 128, m, bar, 64 * b, key0, kvh, seq);
-    tma_load_3d(base + C::KV, &tmL, bar, lr_col, key0, seq);
+    tma_load_4d(base + C::KV, &tmL, bar, lr_col, key0, seq, lra);
   };
   auto load_k = [&](int n) { load_stage(&tmK, k_u + (n & 1) * C::STAGE, kfull(n & 1), n, 0); };
   auto load_v = [&](int n) { load_stage(&tmV, v_u + (n % C::NV) * C::STAGE, vfull(n % C::NV), n, R); };
@@ -642,11 +643,14 @@ bool prefill_maps(const AttnParams& p, CUtensorMap* mq, CUtensorMap* mk, CUtenso
           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return false;
-  // LR rows [2r]: boxes of r columns (LRk at column 0, LRv at column r)
-  cuuint64_t ld[3] = {(cuuint64_t)(2 * R), (cuuint64_t)p.L_max, (cuuint64_t)p.n_seqs};
-  cuuint64_t ls[2] = {(cuuint64_t)(2 * R * 2), (cuuint64_t)p.lr_seq * 2};
-  cuuint32_t lbx[3] = {(cuuint32_t)R, (cuuint32_t)PKT, 1};
-  if (enc(ml, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(p.lr), ld, ls, lbx, one,
+  // LR rows [2r]: boxes of r columns (LRk at column 0, LRv at column r), in
+  // [n_lr][n_seqs][L_max][2r]: one shared cache, or one per agent
+  const int64_t n_lr = p.lr_agent ? p.n_agents : 1;
+  const int64_t lr_agent_b = p.lr_agent ? p.lr_agent * 2 : p.lr_seq * 2 * p.n_seqs;
+  cuuint64_t ld[4] = {(cuuint64_t)(2 * R), (cuuint64_t)p.L_max, (cuuint64_t)p.n_seqs, (cuuint64_t)n_lr};
+  cuuint64_t ls[3] = {(cuuint64_t)(2 * R * 2), (cuuint64_t)p.lr_seq * 2, (cuuint64_t)lr_agent_b};
+  cuuint32_t lbx[4] = {(cuuint32_t)R, (cuuint32_t)PKT, 1, 1};
+  if (enc(ml, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(p.lr), ld, ls, lbx, one,
           CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(R * 2), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return false;

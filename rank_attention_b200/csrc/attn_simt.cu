@@ -36,7 +36,8 @@ constexpr int NW = NT / 32;
 struct SmemLayout {
   int rows, D, R;
   size_t theta, cs, q, kb, vb, ka, lr, s, o, m, l, alpha, pos, total;
-  __host__ __device__ SmemLayout(int rows_, int D_, int R_) : rows(rows_), D(D_), R(R_) {
+  // n_lr: LR tiles staged per key tile (1 shared cache, or one per agent)
+  __host__ __device__ SmemLayout(int rows_, int D_, int R_, int n_lr) : rows(rows_), D(D_), R(R_) {
     size_t off = 0;
     auto take = [&](size_t bytes) { size_t o = off; off += (bytes + 15) / 16 * 16; return o; };
     theta = take(sizeof(double) * 64);
@@ -45,7 +46,7 @@ struct SmemLayout {
     kb = take(sizeof(float) * TK * D);
     vb = take(sizeof(float) * TK * D);
     ka = take(sizeof(float) * TK * D);
-    lr = take(sizeof(float) * TK * 2 * R);
+    lr = take(sizeof(float) * TK * 2 * R * n_lr);
     s = take(sizeof(float) * rows * TK);
     o = take(sizeof(float) * rows * (D + R));
     m = take(sizeof(float) * rows);
@@ -92,7 +93,8 @@ __global__ void __launch_bounds__(NT) attn_simt_kernel(const AttnParams p, const
   const int split = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
-  SmemLayout L(rows_cap, D, R);
+  const int n_lr = p.lr_agent ? na : 1;
+  SmemLayout L(rows_cap, D, R, n_lr);
   double* theta = reinterpret_cast<double*>(smem + L.theta);
   float2* CS = reinterpret_cast<float2*>(smem + L.cs);
   float* Qs = reinterpret_cast<float*>(smem + L.q);
@@ -159,10 +161,11 @@ __global__ void __launch_bounds__(NT) attn_simt_kernel(const AttnParams p, const
       Kb[i] = kv;
       Vb[i] = vv;
     }
-    for (int i = tid; i < TK * 2 * R; i += NT) {
-      const int t = i / (2 * R), c = i % (2 * R);
+    // LR tile [n_lr][TK][2r]: the shared cache, or agent a's own (BaseShared)
+    for (int i = tid; i < n_lr * TK * 2 * R; i += NT) {
+      const int al = i / (TK * 2 * R), t = (i / (2 * R)) % TK, c = i % (2 * R);
       const int64_t key = k0 + t;
-      LRs[i] = key < k_end ? to_f32(lrp[key * 2 * R + c]) : 0.f;
+      LRs[i] = key < k_end ? to_f32(lrp[al * p.lr_agent + key * 2 * R + c]) : 0.f;
     }
     for (int i = tid; i < TK * H2; i += NT) {
       const int t = i / H2, c = i % H2;
@@ -173,11 +176,12 @@ __global__ void __launch_bounds__(NT) attn_simt_kernel(const AttnParams p, const
     for (int a = 0; a < na; ++a) {
       // 2a. key expansion for agent a: K^a = K_base + RoPE(s * LRk * B_k^a)
       const IO* Bk = reinterpret_cast<const IO*>(p.B_k) + (int64_t)a * R * ldB + kvh * D;
+      const float* LRa = LRs + (n_lr > 1 ? a : 0) * TK * 2 * R;
       for (int i = tid; i < TK * H2; i += NT) {
         const int t = i / H2, c = i % H2;
         float x1 = 0.f, x2 = 0.f;
         for (int j = 0; j < R; ++j) {
-          const float lv = LRs[t * 2 * R + j];
+          const float lv = LRa[t * 2 * R + j];
           x1 = fmaf(lv, to_f32(Bk[j * ldB + c]), x1);
           x2 = fmaf(lv, to_f32(Bk[j * ldB + c + H2]), x2);
         }
@@ -233,7 +237,8 @@ __global__ void __launch_bounds__(NT) attn_simt_kernel(const AttnParams p, const
         for (int t = 0; t < TK; ++t) acc = fmaf(Pr[t], Vb[t * D + c], acc);
       } else {
         const int j = R + (c - D);
-        for (int t = 0; t < TK; ++t) acc = fmaf(Pr[t], LRs[t * 2 * R + j], acc);
+        const float* LRa = LRs + (n_lr > 1 ? (row / g) % na : 0) * TK * 2 * R;   // the row's agent
+        for (int t = 0; t < TK; ++t) acc = fmaf(Pr[t], LRa[t * 2 * R + j], acc);
       }
       O[i] = acc;
     }
@@ -308,7 +313,8 @@ template <typename IO, typename OUT>
 cudaError_t launch_typed(const AttnParams& p, cudaStream_t st) {
   const int qb = p.decode ? 1 : max(1, kMaxRowsSimt / p.rows_per_tok);
   const int rows_cap = qb * p.rows_per_tok;
-  SmemLayout L(rows_cap, p.d, p.r);
+  SmemLayout L(rows_cap, p.d, p.r, p.lr_agent ? p.n_agents : 1);
+  if (L.total > 227 * 1024) return cudaErrorInvalidConfiguration;
   cudaError_t e = cudaFuncSetAttribute(attn_simt_kernel<IO, OUT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
   if (e != cudaSuccess) return e;
@@ -326,6 +332,10 @@ size_t simt_rows_cap(const AttnParams& p) {
 }
 
 int simt_key_tile() { return TK; }
+
+size_t simt_smem_bytes(const AttnParams& p) {
+  return SmemLayout((int)simt_rows_cap(p), p.d, p.r, p.lr_agent ? p.n_agents : 1).total;
+}
 
 cudaError_t launch_attn_simt(const AttnParams& p, la_dtype io, la_dtype out, cudaStream_t st) {
   if (io == LA_F32 && out == LA_F32) return launch_typed<float, float>(p, st);

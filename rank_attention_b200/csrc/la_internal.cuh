@@ -25,6 +25,7 @@ struct AttnParams {
   int64_t kv_seq, kv_head, kv_tok;
   const void* lr;
   int64_t lr_seq;
+  int64_t lr_agent;        // elements between agents' LR caches; 0 = one shared cache
   const void* B_k;
   const void* B_v;
   const void* q;

@@ -46,15 +46,17 @@ __global__ void __launch_bounds__(kMatThreads) materialize_kernel(AttnParams p, 
   const float2 cs = rope_cs_exact(t, rt.theta[i]);
   const IO* lr = reinterpret_cast<const IO*>(p.lr) + seq * p.lr_seq + t * 2 * R;
   float lk[R], lv[R];
-#pragma unroll
-  for (int m = 0; m < R; ++m) {
-    lk[m] = ld_io(lr + m);
-    lv[m] = ld_io(lr + R + m);
-  }
   const int64_t ldB = (int64_t)p.n_kv * D;
   const IO* Bk = reinterpret_cast<const IO*>(p.B_k);
   const IO* Bv = reinterpret_cast<const IO*>(p.B_v);
   for (int a = 0; a < p.n_agents; ++a) {
+    if (a == 0 || p.lr_agent) {  // the shared LR row, or agent a's own
+#pragma unroll
+      for (int m = 0; m < R; ++m) {
+        lk[m] = ld_io(lr + a * p.lr_agent + m);
+        lv[m] = ld_io(lr + a * p.lr_agent + R + m);
+      }
+    }
     for (int j = 0; j < p.n_kv; ++j) {
       const IO* bk = Bk + (int64_t)a * R * ldB + j * D + i;
       const IO* bv = Bv + (int64_t)a * R * ldB + j * D + i;

@@ -25,7 +25,8 @@ LA_F32, LA_BF16 = 0, 1
 
 EXPORTED = ("la_status_string", "lr_cache_append", "lora_attn_prefill", "lora_attn_decode",
             "lora_attn_decode_workspace_bytes", "la_device_check",
-            "lora_attn_decode_static_scratch", "lora_materialize_agent_kv")
+            "lora_attn_decode_static_scratch", "lora_materialize_agent_kv",
+            "lr_cache_append_agents")
 
 
 class LoraAttnError(RuntimeError):
@@ -55,6 +56,7 @@ class AttnArgs(ctypes.Structure):
         ("q_pos0", ctypes.c_int64),
         ("n_q_tokens", ctypes.c_int32),
         ("io_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int),
+        ("lr_agent_stride", ctypes.c_int64),
     ]
 
 
@@ -70,6 +72,11 @@ def _load() -> ctypes.CDLL:
         ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
         ctypes.c_int32, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int32,
         ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_void_p]
+    lib.lr_cache_append_agents.restype = ctypes.c_int
+    lib.lr_cache_append_agents.argtypes = [
+        ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+        ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+        ctypes.c_int64, ctypes.c_int32, ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_void_p]
     lib.lora_attn_prefill.restype = ctypes.c_int
     lib.lora_attn_prefill.argtypes = [ctypes.POINTER(AttnArgs), ctypes.c_void_p]
     lib.lora_attn_decode.restype = ctypes.c_int
@@ -129,16 +136,39 @@ def lr_cache_append(X: torch.Tensor, A_kv: torch.Tensor, lr_cache: torch.Tensor,
     _check(st, "lr_cache_append")
 
 
+def lr_cache_append_agents(X: torch.Tensor, A_kv: torch.Tensor, lr_cache: torch.Tensor,
+                           pos0: int, stream=None) -> None:
+    """lr_cache[a, :, pos0:pos0+n] = X @ A_kv[a] for every agent a.
+
+    X [n_seqs, n, H] (last dim contiguous), A_kv [n_agents, H, 2r] contiguous,
+    lr_cache [n_agents, n_seqs, L_max, 2r] (last two dims contiguous)."""
+    n_seqs, n, H = X.shape
+    n_agents, r = A_kv.shape[0], A_kv.shape[2] // 2
+    assert X.stride(2) == 1 and A_kv.is_contiguous()
+    assert lr_cache.stride(3) == 1 and lr_cache.stride(2) == 2 * r
+    st = lib.lr_cache_append_agents(X.data_ptr(), X.stride(1), n, H, A_kv.data_ptr(), n_agents, r,
+                                    lr_cache.data_ptr(), lr_cache.stride(0), lr_cache.shape[2],
+                                    pos0, n_seqs, X.stride(0), lr_cache.stride(1), _dt(X),
+                                    _stream(stream))
+    _check(st, "lr_cache_append_agents")
+
+
 def make_args(k_base, v_base, lr, B_k, B_v, q, out, *, lora_scale: float, rope_base: float,
               softmax_scale: Optional[float] = None, kv_len: Optional[torch.Tensor] = None,
               max_kv_len: int = 0, q_pos0: int = 0) -> AttnArgs:
     """Fill la_attn_args from tensors.
 
     k_base, v_base [n_seqs, n_kv, L_max, d] (any strides with a unit last
-    stride); lr [n_seqs, L_max, 2r]; B_k, B_v [n_agents, r, n_kv*d];
+    stride); lr [n_seqs, L_max, 2r], one LR cache shared by every agent, or
+    [n_agents, n_seqs, L_max, 2r], one per agent; B_k, B_v [n_agents, r, n_kv*d];
     q, out [n_seqs, n_agents, n_tok, n_q, d] contiguous; kv_len int32 [n_seqs]."""
     n_seqs, n_kv, L_max, d = k_base.shape
     n_agents, n_tok, n_q = q.shape[1], q.shape[2], q.shape[3]
+    per_agent = lr.dim() == 4
+    lr_agent_stride = lr.stride(0) if per_agent else 0
+    if per_agent:
+        assert lr.shape[0] == n_agents
+        lr = lr[0]
     r = lr.shape[2] // 2
     assert k_base.stride() == v_base.stride() and k_base.stride(3) == 1
     assert lr.stride(2) == 1 and lr.stride(1) == 2 * r
@@ -161,6 +191,7 @@ def make_args(k_base, v_base, lr, B_k, B_v, q, out, *, lora_scale: float, rope_b
     a.q_pos0 = q_pos0
     a.n_q_tokens = n_tok
     a.io_dtype, a.out_dtype = _dt(k_base), _dt(out)
+    a.lr_agent_stride = lr_agent_stride
     return a
 
 

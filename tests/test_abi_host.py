@@ -117,6 +117,9 @@ BAD_ATTN = [
     (dict(rope_base=0.5), la.LA_ERR_INVALID_ARG),
     (dict(io_dtype=3), la.LA_ERR_INVALID_ARG),
     (dict(n_agents=40), la.LA_ERR_UNSUPPORTED),
+    (dict(lr_agent_stride=-4096), la.LA_ERR_INVALID_ARG),
+    (dict(lr_agent_stride=4097), la.LA_ERR_INVALID_ARG),   # not a multiple of 16 bytes
+    (dict(lr_agent_stride=2048), la.LA_ERR_INVALID_ARG),   # overlaps the next agent's cache
 ]
 
 
@@ -149,6 +152,44 @@ def test_decode_rejects_small_workspace():
 def test_prefill_rejects(kw, status):
     a = _args(**kw)
     assert la.lib.lora_attn_prefill(ctypes.byref(a), None) == status
+
+
+def test_per_agent_lr_stride_accepted():
+    # one LR cache per agent, laid out back to back: a valid plan
+    a = _args(lr_agent_stride=256 * 16)
+    assert la.lib.lora_attn_decode_workspace_bytes(ctypes.byref(a)) > 0
+
+
+def test_per_agent_lr_too_large_for_the_generic_kernel():
+    # fp32 runs on the generic kernel, which stages every agent's LR tile:
+    # 16 agents at r = 64, d = 128 exceed its shared memory, refused before launch
+    a = _args(n_agents=16, head_dim=128, r=64, lr_seq_stride=256 * 128,
+              kv_seq_stride=2 * 256 * 128, kv_head_stride=256 * 128, kv_tok_stride=128,
+              lr_agent_stride=256 * 128)
+    assert la.lib.lora_attn_decode(ctypes.byref(a), FAKE, 1 << 26, None) == la.LA_ERR_UNSUPPORTED
+    a.n_q_tokens = 1
+    assert la.lib.lora_attn_prefill(ctypes.byref(a), None) == la.LA_ERR_UNSUPPORTED
+
+
+def _append_agents(**kw):
+    a = dict(X=FAKE, ldx=256, n=4, H=256, A=FAKE, na=2, r=8, lr=FAKE, ls=16 * 16, L_max=16,
+             pos0=0, n_seqs=1, sx=0, slr=0, dt=la.LA_F32)
+    a.update(kw)
+    return la.lib.lr_cache_append_agents(a["X"], a["ldx"], a["n"], a["H"], a["A"], a["na"],
+                                         a["r"], a["lr"], a["ls"], a["L_max"], a["pos0"],
+                                         a["n_seqs"], a["sx"], a["slr"], a["dt"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(na=0), la.LA_ERR_INVALID_ARG),
+    (dict(ls=101), la.LA_ERR_INVALID_ARG),       # not a multiple of 16 bytes
+    (dict(ls=16), la.LA_ERR_INVALID_ARG),        # overlaps the next agent's cache
+    (dict(X=0), la.LA_ERR_INVALID_ARG),
+    (dict(r=12), la.LA_ERR_UNSUPPORTED),
+    (dict(pos0=13), la.LA_ERR_CAPACITY),
+])
+def test_append_agents_rejects(kw, status):
+    assert _append_agents(**kw) == status
 
 
 def test_null_args():

@@ -433,3 +433,105 @@ def test_materialized_agent_caches_and_non_shared_decode(la):
                   dd["kv_len"])
     assert_parity(to_np(out_ns), oracle_decode(inp, s), s.dtype)
     assert_parity(to_np(out_ns), to_np(shared), s.dtype)
+
+
+# ------------------------------ one LR cache per agent (BaseShared) ----
+# Each agent owns its down-projection A_a and reads its own LR cache X A_a
+# beside the shared base cache (LRAgent summary §3 "BaseShared"); the LR
+# tensor is [n_agents, n_seqs, L_max, 2r] and la_attn_args.lr_agent_stride
+# points each agent at its own.
+@pytest.mark.parametrize("n_q,n_kv,L,n_tok,n_seqs,r,n_agents", [
+    (32, 8, 600, 300, 1, 16, 3),     # tensor-core prefill, r = 16
+    (32, 8, 700, 200, 1, 64, 4),     # r = 64: one V stage
+    (8, 8, 390, 260, 2, 32, 2),      # g = 1, two sequences
+    (4, 1, 512, 512, 1, 16, 3),      # few CTAs: key halves on CTA pairs
+])
+def test_base_shared_prefill_tensor_cores(la, n_q, n_kv, L, n_tok, n_seqs, r, n_agents):
+    s = W.LLAMA8B_PREFILL_16K.replace(n_q_heads=n_q, n_kv_heads=n_kv, kv_len=L, n_q_tokens=n_tok,
+                                      n_seqs=n_seqs, r=r, alpha=2.0 * r, n_agents=n_agents,
+                                      seed=600 + L, lr_per_agent=True)
+    _prefill_vs_oracle(la, s, W.direct_cache_inputs(s))
+
+
+@pytest.mark.parametrize("kv_len,n_seqs,n_agents,r", [
+    (1500, 1, 3, 16),     # the 3-agent layer, one agent per CTA
+    (700, 2, 5, 32),      # the batched sweep's agents and rank, short
+    (300, 1, 4, 64),      # the stack's rank
+])
+def test_base_shared_decode_tensor_cores(la, kv_len, n_seqs, n_agents, r):
+    s = W.LLAMA8B_DECODE_8K.replace(kv_len=kv_len, n_seqs=n_seqs, n_agents=n_agents, r=r,
+                                    alpha=2.0 * r, seed=700 + kv_len, lr_per_agent=True)
+    inp = W.direct_cache_inputs(s)
+    dd = to_device(inp)
+    got = _run(la, s, dd["k_base"], dd["v_base"], dd["lr"], dd["B_k"], dd["B_v"], dd["q"],
+               dd["kv_len"])
+    assert_parity(to_np(got), oracle_decode(inp, s), s.dtype)
+
+
+@pytest.mark.parametrize("mode,n_tok", [("decode", 1), ("prefill", 37)])
+def test_base_shared_fp32_generic_kernel(la, mode, n_tok):
+    s = W.TINY_FP32.replace(kv_len=200, n_q_tokens=n_tok, mode=mode, n_agents=3, seed=71,
+                            lr_per_agent=True)
+    inp = W.direct_cache_inputs(s)
+    dd = to_device(inp)
+    got = _run(la, s, dd["k_base"], dd["v_base"], dd["lr"], dd["B_k"], dd["B_v"], dd["q"],
+               dd["kv_len"])
+    ref = oracle.lora_attention(inp["k_base"], inp["v_base"], inp["lr"], inp["B_k"], inp["B_v"],
+                                inp["q"], inp["kv_len"], lora_scale=s.lora_scale,
+                                softmax_scale=s.softmax_scale, rope_base=s.rope_base, mode=mode)
+    assert_parity(to_np(got), ref, s.dtype)
+
+
+@pytest.mark.parametrize("dtype,r", [(torch.bfloat16, 16), (torch.bfloat16, 64), (torch.float32, 8)])
+def test_append_agents_equals_one_append_per_agent(la, dtype, r):
+    """Every agent's cache X A_a: bit-identical to one single-A append per agent,
+    rows outside the chunk untouched, and within one rounding of the oracle."""
+    n_agents, n_seqs, n, H, L_max, pos0 = 3, 2, 45, 512, 64, 7
+    g = torch.Generator().manual_seed(90 + r)
+    X = torch.randn(n_seqs, n, H, generator=g).to(dtype)
+    A = (0.05 * torch.randn(n_agents, H, 2 * r, generator=g)).to(dtype)
+    guard = torch.full((n_agents, n_seqs, L_max, 2 * r), 7.0, dtype=dtype)
+    lr = guard.to(DEV)
+    la.lr_cache_append_agents(X.to(DEV), A.to(DEV), lr, pos0)
+    one = guard.to(DEV)
+    for a in range(n_agents):
+        la.lr_cache_append(X.to(DEV), A[a].to(DEV), one[a], pos0)
+    torch.cuda.synchronize()
+    assert torch.equal(lr.cpu(), one.cpu())
+    got = lr.cpu()
+    assert torch.equal(got[:, :, :pos0], guard[:, :, :pos0])
+    assert torch.equal(got[:, :, pos0 + n:], guard[:, :, pos0 + n:])
+    ref = oracle.lr_cache_append_agents(guard.to(torch.float64).numpy(), X, A, pos0)
+    err = np.abs(to_np(got) - ref)
+    tol = bf16_ulp(ref) if dtype == torch.bfloat16 else 1e-5 * (1 + np.abs(ref))
+    assert (err <= tol).all(), err.max()
+
+
+def test_base_shared_materialized_caches(la):
+    """The non-shared baseline over per-agent LR caches: agent a's K^a, V^a are
+    built from its own LR rows."""
+    import bench
+    s = W.LLAMA8B_DECODE_8K.replace(kv_len=400, n_seqs=1, seed=57, lr_per_agent=True)
+    inp = W.direct_cache_inputs(s)
+    dd = to_device(inp)
+    mat, dec, out_ns = bench.non_shared_setup(la, s, dd, DEV)
+    mat()
+    torch.cuda.synchronize()
+    kout, vout = mat.keep[0].cpu(), mat.keep[1].cpu()
+    d, r = s.head_dim, s.r
+    kpos = np.arange(s.kv_len)
+    for a in range(s.n_agents):
+        lr = to_np(inp["lr"][a, 0])
+        j = a % s.n_kv_heads
+        cols = slice(j * d, (j + 1) * d)
+        Ka = oracle.agent_keys(inp["k_base"][0, j], lr[:, :r], to_np(inp["B_k"][a])[:, cols],
+                               s.lora_scale, kpos, s.rope_base)
+        Va = oracle.agent_values(inp["v_base"][0, j], lr[:, r:], to_np(inp["B_v"][a])[:, cols],
+                                 s.lora_scale)
+        for got, ref in ((kout[0, a, j, :s.kv_len], Ka), (vout[0, a, j, :s.kv_len], Va)):
+            err = np.abs(to_np(got) - ref)
+            assert (err <= bf16_ulp(ref) + 1e-3 * np.abs(ref).max()).all(), err.max()
+    dec()
+    torch.cuda.synchronize()
+    assert la.la_device_check() == 0
+    assert_parity(to_np(out_ns), oracle_decode(inp, s), s.dtype)
