@@ -132,6 +132,32 @@ def base_cache_from_hidden(X, W_k, W_v, n_kv_heads: int, rope_base: float):
 
 
 # ----------------------------------------------------------------------------
+# LoRA on the query and output projections (the qkvo setting of LRAgent
+# summary App. D.1 "Ablation on LoRA Application"; Y = X W_0 + (X A) B as in
+# App. A.3)
+# ----------------------------------------------------------------------------
+def lora_queries(q_base, lr_q, B_q, lora_scale: float, positions, rope_base: float) -> np.ndarray:
+    """Agent queries with a query-side LoRA, rotated at their positions:
+    q^a_t = RoPE_t(X_t W_q + s (X_t A_q) B_q^a), head by head.
+
+    q_base [n_tok, n_q, d]: the base projection X W_q, not yet rotated;
+    lr_q [n_tok, r]: X A_q, unscaled; B_q [r, n_q*d]: the agent's up-projection.
+    The delta joins the projection before RoPE (RoPE rotates what the
+    projection produces).  Returns [n_tok, n_q, d]."""
+    qb = _np64(q_base)
+    n_tok, n_q, d = qb.shape
+    delta = lora_scale * (_np64(lr_q) @ _np64(B_q))            # [n_tok, n_q*d]
+    pre = qb + delta.reshape(n_tok, n_q, d)
+    return rope(pre.transpose(1, 0, 2), positions, rope_base).transpose(1, 0, 2)
+
+
+def lora_output(y_base, o, A_o, B_o, lora_scale: float) -> np.ndarray:
+    """Output projection with LoRA: y^a = O W_o + s (O A_o) B_o^a, given the
+    base part y_base = O W_o.  o [n_tok, D_in]; A_o [D_in, r]; B_o [r, D_out]."""
+    return _np64(y_base) + lora_scale * ((_np64(o) @ _np64(A_o)) @ _np64(B_o))
+
+
+# ----------------------------------------------------------------------------
 # Per-agent keys and values (materialised)
 # ----------------------------------------------------------------------------
 def agent_keys(k_base_h, lr_k, B_k_h, lora_scale: float, positions, rope_base: float):

@@ -271,6 +271,53 @@ def test_planted_per_agent_cache_mistake_is_caught(monkeypatch):
     assert per_agent_brute_force_error(mode="prefill") > 1e-6
 
 
+# --------------------------------------- query- and output-side LoRA ----
+def qo_problem(seed=11, n_tok=5, H=12, n_q=4, d=8, r=3, D_out=10, alpha=4.5):
+    rng = np.random.default_rng(seed)
+    return dict(X=rng.standard_normal((n_tok, H)), W_q=rng.standard_normal((H, n_q * d)),
+                A_q=rng.standard_normal((H, r)), B_q=rng.standard_normal((r, n_q * d)),
+                W_o=rng.standard_normal((n_q * d, D_out)), A_o=rng.standard_normal((n_q * d, r)),
+                B_o=rng.standard_normal((r, D_out)), s=alpha / r, n_q=n_q, d=d,
+                pos=np.arange(7, 7 + n_tok))
+
+
+def query_lora_error(seed=11, base=100.0):
+    """Merged weights W_q + s A_q B_q, projected and rotated with the complex
+    RoPE, against the decomposed oracle."""
+    p = qo_problem(seed)
+    n_tok = p["X"].shape[0]
+    merged = (p["X"] @ (p["W_q"] + p["s"] * p["A_q"] @ p["B_q"])).reshape(n_tok, p["n_q"], p["d"])
+    ref = complex_rope(merged.transpose(1, 0, 2), p["pos"], base).transpose(1, 0, 2)
+    got = impl.lora_queries((p["X"] @ p["W_q"]).reshape(n_tok, p["n_q"], p["d"]),
+                            p["X"] @ p["A_q"], p["B_q"], p["s"], p["pos"], base)
+    return np.abs(got - ref).max() / np.abs(ref).max()
+
+
+def test_query_lora_against_merged_weights():
+    assert query_lora_error() < 1e-12
+    assert query_lora_error(seed=12, base=500000.0) < 1e-12
+
+
+def test_output_lora_against_merged_weights():
+    p = qo_problem(13)
+    o = p["X"] @ p["W_q"]                                   # any [n_tok, n_q*d] attention output
+    ref = o @ (p["W_o"] + p["s"] * p["A_o"] @ p["B_o"])
+    got = impl.lora_output(o @ p["W_o"], o, p["A_o"], p["B_o"], p["s"])
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+
+
+def _bad_queries_delta_after_rope(q_base, lr_q, B_q, lora_scale, positions, rope_base):
+    qb = impl._np64(q_base)
+    n_tok, n_q, d = qb.shape
+    rot = impl.rope(qb.transpose(1, 0, 2), positions, rope_base).transpose(1, 0, 2)
+    return rot + lora_scale * (impl._np64(lr_q) @ impl._np64(B_q)).reshape(n_tok, n_q, d)
+
+
+def test_planted_query_lora_mistake_is_caught(monkeypatch):
+    monkeypatch.setattr(impl, "lora_queries", _bad_queries_delta_after_rope)
+    assert query_lora_error() > 1e-6
+
+
 def test_reordered_value_path_identity():
     rng = np.random.default_rng(5)
     L, d, r, s = 13, 16, 4, 2.0
