@@ -237,6 +237,88 @@ def time_decode_shape(dev, s, reps=5, warmup=3):
             "timing": f"median of {reps} launches, CUDA events, L2 flushed before each"}
 
 
+def time_base_shared(dev):
+    """The decode workload with one LR cache per agent (each agent's own A_a,
+    BaseShared) beside the same decode over one shared LR cache, both timed
+    alike (single launches, L2 flushed), with the caches' sizes."""
+    from rank_attention_b200 import workloads as W
+    s = W.LLAMA8B_DECODE_8K
+    own = time_decode_shape(dev, s.replace(lr_per_agent=True))
+    shared = time_decode_shape(dev, s)
+    lr_one = s.n_seqs * s.kv_len * 2 * s.r * 2
+    base = 2 * s.n_seqs * s.n_kv_heads * s.kv_len * s.head_dim * 2
+    return {"workload": s.name + "_lr_per_agent", "decode_us": own["us"], "GB/s": own["GB/s"],
+            "frac": own["frac"], "algorithmic_bytes": own["algorithmic_bytes"],
+            "shared_lr_decode_us": shared["us"],
+            "cache_bytes": {"base": base, "lr_per_agent_total": s.n_agents * lr_one,
+                            "lr_shared": lr_one},
+            "what": "each agent reads its own LR cache X A_a beside the shared base cache "
+                    "(one agent per CTA); shared_lr_decode_us: the same decode with one "
+                    "LR cache (shared A), timed the same way",
+            "timing": own["timing"]}
+
+
+def _time_launches(fn, flush, reps=5, warmup=3):
+    """Median CUDA-event time (ms) of single launches, L2 flushed before each."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(reps):
+        flush.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    return statistics.median(times)
+
+
+def time_qkvo(dev):
+    """Query- and output-side LoRA (the qkvo setting) on the 3-agent layer: one
+    decode token per agent, and a 1024-token chunk per agent.  HBM roofline on
+    the bytes each kernel must move (inputs once, outputs once)."""
+    import torch
+    from rank_attention_b200 import lora_attn as la
+    from rank_attention_b200 import workloads as W
+    s = W.LLAMA8B_DECODE_8K
+    na, nq, d, r, e = s.n_agents, s.n_q_heads, s.head_dim, s.r, 2
+    D = nq * d
+    hbm, _ = peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(5)
+    res = {}
+    for n_tok in (1, 1024):
+        qb = torch.randn(1, na, n_tok, nq, d, generator=g, device=dev).to(torch.bfloat16)
+        lrq = torch.randn(1, na, n_tok, r, generator=g, device=dev).to(torch.bfloat16)
+        Bq = (0.02 * torch.randn(na, r, D, generator=g, device=dev)).to(torch.bfloat16)
+        qo = torch.empty_like(qb)
+        pe = torch.full((1,), s.kv_len, dtype=torch.int32, device=dev)
+        o = torch.randn(1, na, n_tok, D, generator=g, device=dev).to(torch.bfloat16)
+        Ao = (0.02 * torch.randn(D, r, generator=g, device=dev)).to(torch.bfloat16)
+        Bo = (0.02 * torch.randn(na, r, D, generator=g, device=dev)).to(torch.bfloat16)
+        y = torch.randn(1, na, n_tok, D, generator=g, device=dev).to(torch.bfloat16)
+        q_ms = _time_launches(lambda: la.lora_query_expand(qb, lrq, Bq, qo, pe, lora_scale=s.lora_scale,
+                                                           rope_base=s.rope_base), flush)
+        o_ms = _time_launches(lambda: la.lora_output_delta(o, Ao, Bo, y, lora_scale=s.lora_scale),
+                              flush)
+        if la.la_device_check() != 0:
+            raise RuntimeError("qkvo device check failed")
+        qbytes = (2 * na * n_tok * D + na * n_tok * r + na * r * D) * e
+        obytes = (na * n_tok * D + D * r + na * r * D + 2 * na * n_tok * D) * e
+        res[f"{n_tok}_tok"] = {
+            "query_expand_us": q_ms * 1e3, "query_expand_GB/s": qbytes / (q_ms / 1e3) / 1e9,
+            "query_expand_frac": qbytes / (q_ms / 1e3) / 1e9 / hbm, "query_expand_bytes": qbytes,
+            "output_delta_us": o_ms * 1e3, "output_delta_GB/s": obytes / (o_ms / 1e3) / 1e9,
+            "output_delta_frac": obytes / (o_ms / 1e3) / 1e9 / hbm, "output_delta_bytes": obytes}
+    res["workload"] = f"{s.name}: {na} agents, n_q*d = {D}, r = {r}; one decode token and a 1024-token chunk per agent"
+    res["timing"] = "median of 5 launches, CUDA events, L2 flushed before each"
+    return res
+
+
 def time_other_configs(dev):
     """The long-context batched decode sweep (16 requests x 5 agents, r = 32)
     and one layer of the 32-layer stack (4096-token chunk over a 32768-token
@@ -369,11 +451,12 @@ def whole_job_rate(units_per_rank_step: int, steps: int, world: int, ms_max: flo
 
 
 def decode_bytes(s) -> int:
-    """Algorithmic HBM bytes of one decode launch: base K and V read once, LR
-    cache read once, every agent's B_k and B_v, the queries and the fp32 outputs."""
+    """Algorithmic HBM bytes of one decode launch: base K and V read once, the
+    LR cache read once (every agent's own with one cache per agent), every
+    agent's B_k and B_v, the queries and the fp32 outputs."""
     e = 2  # bf16
     base = 2 * s.n_seqs * s.n_kv_heads * s.kv_len * s.head_dim * e
-    lr = s.n_seqs * s.kv_len * 2 * s.r * e
+    lr = s.n_seqs * s.kv_len * 2 * s.r * e * (s.n_agents if s.lr_per_agent else 1)
     Bw = 2 * s.n_agents * s.r * s.n_kv_heads * s.head_dim * e
     q = s.n_seqs * s.n_agents * s.n_q_heads * s.head_dim * e
     out = s.n_seqs * s.n_agents * s.n_q_heads * s.head_dim * 4
@@ -594,6 +677,8 @@ def run_ours(args):
 
     prefill = time_prefill(dev)
     non_shared = time_non_shared(dev, dec_ms * 1e3)
+    base_shared = time_base_shared(dev)
+    qkvo = time_qkvo(dev)
 
     hbm, peak_kind = peaks()
     dbytes = decode_bytes(s)
@@ -619,6 +704,8 @@ def run_ours(args):
         "clocks": clk,
         "prefill": prefill,
         "non_shared_baseline": non_shared,
+        "base_shared": base_shared,
+        "qkvo": qkvo,
     }
     if args.all_configs:
         line["other_configs"] = time_other_configs(dev)

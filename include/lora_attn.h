@@ -226,6 +226,54 @@ size_t lora_attn_decode_workspace_bytes(const la_attn_args* args);
  *     returns LA_ERR_SCRATCH_LIMIT before launching anything.
  */
 /*
+ * lora_query_expand -- query-side LoRA and RoPE (the qkvo setting: LoRA on
+ * the query, key, value and output projections; LRAgent summary App. D.1
+ * "Ablation on LoRA Application"), producing the rotated per-agent queries
+ * that lora_attn_prefill / lora_attn_decode take:
+ *   q_out[q][a][j][h][:] = RoPE_pos( q_base[q][a][j][h][:]
+ *                                    + s * lr_q[q][a][j][:] B_q[a][:, h*d:(h+1)*d] )
+ * at position pos = pos_end[q] - n_tok + j (decode: pos_end = kv_len; prefill:
+ * q_pos0 + n_tok), RoPE as for the keys.  The delta joins the projection
+ * before the rotation.
+ *
+ *   q_base  [n_seqs][n_agents][n_tok][n_q_heads][d], X^a W_q of the base model,
+ *           not yet rotated, contiguous.
+ *   lr_q    [n_seqs][n_agents][n_tok][r], X^a A_q (unscaled), contiguous.
+ *   B_q     [n_agents][r][n_q_heads * d], contiguous.
+ *   q_out   layout of q_base; may be q_base itself (each element is read
+ *           before it is written, by the same thread).
+ *   pos_end device int32 [n_seqs].
+ * All of dtype dt; fp32 accumulation.  Errors: LA_ERR_INVALID_ARG (null or
+ * misaligned pointer, non-positive size), LA_ERR_UNSUPPORTED (head_dim not 64
+ * or 128, r not in {8,16,32,64}, grid limits).
+ */
+la_status lora_query_expand(const void* q_base, const void* lr_q, const void* B_q, void* q_out,
+                            int32_t n_seqs, int32_t n_agents, int32_t n_tok, int32_t n_q_heads,
+                            int32_t head_dim, int32_t r, float lora_scale, double rope_base,
+                            const int32_t* pos_end, la_dtype dt, la_stream_t stream);
+
+/*
+ * lora_output_delta -- output-side LoRA of the qkvo setting (LRAgent summary
+ * App. D.1), added to the base model's output projection:
+ *   y[q][a][j][:] += s * ( o[q][a][j][:] A_o[a] ) B_o[a]
+ * so that y = O W_o + s (O A_o) B_o^a when y holds O W_o on entry.
+ *
+ *   o     [n_seqs][n_agents][n_tok][d_in], the attention outputs, contiguous.
+ *   A_o   [d_in][r]; agent a's at A_o + a * a_agent_stride elements
+ *         (a_agent_stride = 0: one A_o shared by every agent, shared-A).
+ *   B_o   [n_agents][r][d_out], contiguous.
+ *   y     [n_seqs][n_agents][n_tok][d_out], read and written.
+ * All of dtype dt; fp32 accumulation.  Errors: LA_ERR_INVALID_ARG (null or
+ * misaligned pointer, non-positive size, negative stride),
+ * LA_ERR_UNSUPPORTED (r not in {8,16,32,64}, d_out not a multiple of 8,
+ * grid limits).
+ */
+la_status lora_output_delta(const void* o, const void* A_o, int64_t a_agent_stride, const void* B_o,
+                            void* y, int32_t n_seqs, int32_t n_agents, int32_t n_tok, int32_t d_in,
+                            int32_t d_out, int32_t r, float lora_scale, la_dtype dt,
+                            la_stream_t stream);
+
+/*
  * lora_materialize_agent_kv -- the non-shared baseline's caches.
  *
  * Writes every agent's full keys and values

@@ -218,6 +218,46 @@ extern "C" la_status lr_cache_append_agents(const void* X, int64_t ldx, int64_t 
   return LA_OK;
 }
 
+extern "C" la_status lora_query_expand(const void* q_base, const void* lr_q, const void* B_q,
+                                       void* q_out, int32_t n_seqs, int32_t n_agents,
+                                       int32_t n_tok, int32_t n_q_heads, int32_t head_dim,
+                                       int32_t r, float lora_scale, double rope_base,
+                                       const int32_t* pos_end, la_dtype dt, la_stream_t stream) {
+  if (!dtype_ok(dt)) return LA_ERR_INVALID_ARG;
+  if (n_seqs < 1 || n_agents < 1 || n_tok < 1 || n_q_heads < 1) return LA_ERR_INVALID_ARG;
+  if (!isfinite(lora_scale) || !isfinite(rope_base) || !(rope_base > 1.0)) return LA_ERR_INVALID_ARG;
+  if (head_dim != 64 && head_dim != 128) return LA_ERR_UNSUPPORTED;
+  if (!rank_ok(r)) return LA_ERR_UNSUPPORTED;
+  if (!q_base || !lr_q || !B_q || !q_out || !pos_end) return LA_ERR_INVALID_ARG;
+  if (!aligned16(q_base) || !aligned16(lr_q) || !aligned16(B_q) || !aligned16(q_out) ||
+      (reinterpret_cast<uintptr_t>(pos_end) & 3u) != 0)
+    return LA_ERR_INVALID_ARG;
+  if (n_agents > 65535 || n_seqs > 65535) return LA_ERR_UNSUPPORTED;
+  if ((int64_t)n_tok * ((n_q_heads + 7) / 8) > 0x7fffffff) return LA_ERR_UNSUPPORTED;
+  const cudaError_t e = la::launch_query_expand(q_base, lr_q, B_q, q_out, n_seqs, n_agents, n_tok,
+                                                n_q_heads, head_dim, r, lora_scale, rope_base,
+                                                pos_end, dt, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
+extern "C" la_status lora_output_delta(const void* o, const void* A_o, int64_t a_agent_stride,
+                                       const void* B_o, void* y, int32_t n_seqs, int32_t n_agents,
+                                       int32_t n_tok, int32_t d_in, int32_t d_out, int32_t r,
+                                       float lora_scale, la_dtype dt, la_stream_t stream) {
+  if (!dtype_ok(dt)) return LA_ERR_INVALID_ARG;
+  if (n_seqs < 1 || n_agents < 1 || n_tok < 1 || d_in < 1 || d_out < 1) return LA_ERR_INVALID_ARG;
+  if (a_agent_stride < 0 || !isfinite(lora_scale)) return LA_ERR_INVALID_ARG;
+  if ((a_agent_stride * (int64_t)esize(dt)) % 16 != 0) return LA_ERR_INVALID_ARG;
+  if (!rank_ok(r) || d_out % 8 != 0) return LA_ERR_UNSUPPORTED;   // 8-column vectors of B_o and y
+  if (!o || !A_o || !B_o || !y) return LA_ERR_INVALID_ARG;
+  if (!aligned16(o) || !aligned16(A_o) || !aligned16(B_o) || !aligned16(y)) return LA_ERR_INVALID_ARG;
+  if (n_agents > 65535 || n_seqs > 65535) return LA_ERR_UNSUPPORTED;
+  const cudaError_t e = la::launch_output_delta(o, A_o, a_agent_stride, B_o, y, n_seqs, n_agents,
+                                                n_tok, d_in, d_out, r, lora_scale, dt,
+                                                static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+
 namespace la {
 // Byte range of the arrival counters inside a decode workspace for these
 // arguments (they must read zero when a decode starts).  False if invalid.

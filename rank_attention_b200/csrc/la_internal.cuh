@@ -56,6 +56,13 @@ cudaError_t launch_append_bf16_mma(const void* X, int64_t ldx, int64_t n, int64_
                                    const void* A, int r, void* lr, int64_t pos0, int n_seqs,
                                    int64_t sx, int64_t slr, cudaStream_t st);
 cudaError_t launch_attn_simt(const AttnParams& p, la_dtype io, la_dtype out, cudaStream_t st);
+cudaError_t launch_query_expand(const void* q_base, const void* lr_q, const void* B_q, void* q_out,
+                                int n_seqs, int n_agents, int n_tok, int n_q, int d, int r, float s,
+                                double rope_base, const int32_t* pos_end, la_dtype dt,
+                                cudaStream_t st);
+cudaError_t launch_output_delta(const void* o, const void* A_o, int64_t a_agent_stride,
+                                const void* B_o, void* y, int n_seqs, int n_agents, int n_tok,
+                                int d_in, int d_out, int r, float s, la_dtype dt, cudaStream_t st);
 cudaError_t launch_materialize(const AttnParams& p, la_dtype io, void* kout, void* vout, cudaStream_t st);
 
 // Decode split-K plan shared by the workspace query and the launch.

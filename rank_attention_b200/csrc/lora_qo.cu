@@ -1,0 +1,267 @@
+// LoRA on the query and output projections (the qkvo setting: LoRA on the
+// query, key, value and output projections; LRAgent summary App. D.1
+// "Ablation on LoRA Application"), around the attention, with the cache
+// decomposition Y = X W_0 + (X A) B of App. A.3:
+//
+//   query side   q^a_t = RoPE_t( X^a_t W_q + s (X^a_t A_q) B_q^a )
+//   output side  y^a   = O^a W_o + s (O^a A_o) B_o^a
+//
+// The base products X W_q and O W_o are the base model's; these kernels take
+// them as inputs and add the rank-r parts.  Both are HBM-bound: every input
+// element is read once and every output element written once, the r-wide
+// rows X A_q and O A_o stay in shared memory, the up-projections B^a are read
+// coalesced and reused from L1 / L2 across a CTA's tokens.
+#include <cmath>
+
+#include <cuda_bf16.h>
+
+#include "bf16_common.cuh"
+#include "la_internal.cuh"
+
+namespace la {
+namespace {
+
+template <typename IO>
+__device__ __forceinline__ float ldf(const IO* p);
+template <>
+__device__ __forceinline__ float ldf<float>(const float* p) { return *p; }
+template <>
+__device__ __forceinline__ float ldf<__nv_bfloat16>(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+template <typename IO>
+__device__ __forceinline__ IO stf(float x);
+template <>
+__device__ __forceinline__ float stf<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 stf<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+constexpr int kQThreads = 256;  // one (head, frequency) pair each: 4 heads a CTA at d = 128
+constexpr int kQTok = 16;     // tokens per CTA: each B_q^a value is loaded once for them
+
+// One CTA per (16 tokens x 4 heads, agent, sequence); a thread owns one
+// (head, frequency) pair, x_i and x_{i+d/2}, for all the CTA's tokens: it
+// loads its r B_q^a pairs once, accumulates the deltas of every token, then
+// adds each token's base projection and rotates (the delta joins before the
+// rotation; every element is written once, so q_out may alias q_base).
+// (cos, sin) per (token, frequency) are formed once per CTA, angle reduced in
+// fp64.
+template <typename IO>
+__global__ void __launch_bounds__(kQThreads) query_expand_kernel(
+    const IO* __restrict__ q_base, const IO* __restrict__ lr_q, const IO* __restrict__ B_q,
+    IO* q_out, int n_agents, int n_tok, int n_q, int d, int r, float s, RopeTheta rt,
+    const int32_t* __restrict__ pos_end) {
+  __shared__ float lr[kQTok][64];
+  __shared__ float2 cs[kQTok][64];
+  const int h2 = d / 2, ld = n_q * d;
+  const int hpb = kQThreads / h2;                     // heads per CTA (4 at d = 128, 8 at d = 64)
+  const int hblocks = (n_q + hpb - 1) / hpb;
+  const int tb = (blockIdx.x / hblocks) * kQTok, h0 = (blockIdx.x % hblocks) * hpb;
+  const int agent = blockIdx.y, seq = blockIdx.z;
+  const int nt = min(kQTok, n_tok - tb);
+  const int64_t row0 = ((int64_t)seq * n_agents + agent) * n_tok + tb;
+  const int64_t pos0 = (int64_t)pos_end[seq] - n_tok + tb;
+  for (int u = threadIdx.x; u < nt * r; u += kQThreads)
+    lr[u / r][u % r] = ldf(lr_q + (row0 + u / r) * r + u % r);
+  for (int u = threadIdx.x; u < nt * h2; u += kQThreads)
+    cs[u / h2][u % h2] = rope_cs_exact(pos0 + u / h2, rt.theta[u % h2]);
+  __syncthreads();
+  const int h = h0 + threadIdx.x / h2, i = threadIdx.x % h2;
+  if (h >= n_q) return;
+  const int c1 = h * d + i, c2 = c1 + h2;
+  const IO* B = B_q + (int64_t)agent * r * ld;
+  float x1[kQTok], x2[kQTok];
+#pragma unroll
+  for (int tt = 0; tt < kQTok; ++tt) x1[tt] = x2[tt] = 0.f;
+#pragma unroll 16
+  for (int m = 0; m < r; ++m) {
+    const float b1 = ldf(B + (int64_t)m * ld + c1), b2 = ldf(B + (int64_t)m * ld + c2);
+#pragma unroll
+    for (int tt = 0; tt < kQTok; ++tt) {
+      x1[tt] = fmaf(lr[tt][m], b1, x1[tt]);
+      x2[tt] = fmaf(lr[tt][m], b2, x2[tt]);
+    }
+  }
+#pragma unroll
+  for (int tt = 0; tt < kQTok; ++tt) {
+    if (tt < nt) {
+      const IO* qb = q_base + (row0 + tt) * ld;
+      IO* qo = q_out + (row0 + tt) * ld;
+      const float y1 = fmaf(s, x1[tt], ldf(qb + c1)), y2 = fmaf(s, x2[tt], ldf(qb + c2));
+      const float2 c = cs[tt][i];
+      qo[c1] = stf<IO>(y1 * c.x - y2 * c.y);
+      qo[c2] = stf<IO>(y2 * c.x + y1 * c.y);
+    }
+  }
+}
+
+constexpr int kOThreads = 256;
+constexpr int kOWarps = kOThreads / 32;
+constexpr int kOTok = 8;      // tokens per CTA: A_o and B_o^a are read once for them
+constexpr int kOCols = 8;     // output columns per thread (one 16-byte load of bf16)
+constexpr int kOColBlock = kOThreads * kOCols;
+
+template <typename IO>
+struct Vec8 {
+  float v[8];
+};
+template <typename IO>
+__device__ __forceinline__ Vec8<IO> ld8(const IO* p);
+template <>
+__device__ __forceinline__ Vec8<__nv_bfloat16> ld8<__nv_bfloat16>(const __nv_bfloat16* p) {
+  Vec8<__nv_bfloat16> r;
+  const uint4 u = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    r.v[2 * j] = __uint_as_float(w[j] << 16);
+    r.v[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+  }
+  return r;
+}
+template <>
+__device__ __forceinline__ Vec8<float> ld8<float>(const float* p) {
+  Vec8<float> r;
+  const float4 a = *reinterpret_cast<const float4*>(p), b = *reinterpret_cast<const float4*>(p + 4);
+  r.v[0] = a.x; r.v[1] = a.y; r.v[2] = a.z; r.v[3] = a.w;
+  r.v[4] = b.x; r.v[5] = b.y; r.v[6] = b.z; r.v[7] = b.w;
+  return r;
+}
+
+// One CTA per (8 tokens x 2048 output columns, agent, sequence).  Shrink
+// t = O A_o for the CTA's tokens (each column block recomputes it: O(D_in r)
+// per token, small against the expand): thread j takes rows j, j + 256, ...
+// of A_o, 16 columns at a time as two 16-byte vectors, multiplies them by
+// the tokens' o values of the same rows, and the block sums the partials
+// (warp shuffles, then shared memory).  Expand y += s t B_o^a: a thread owns
+// 8 consecutive output columns, read as one 16-byte vector per row of B_o^a.
+template <typename IO>
+__global__ void __launch_bounds__(kOThreads) output_delta_kernel(
+    const IO* __restrict__ o, const IO* __restrict__ A_o, int64_t a_agent_stride,
+    const IO* __restrict__ B_o, IO* y, int n_agents, int n_tok, int d_in, int d_out, int r,
+    float s) {
+  __shared__ float part[kOWarps][kOTok][16];
+  __shared__ float t[kOTok][64];
+  const int cblocks = (d_out + kOColBlock - 1) / kOColBlock;
+  const int tb = (blockIdx.x / cblocks) * kOTok, cb = blockIdx.x % cblocks;
+  const int agent = blockIdx.y, seq = blockIdx.z;
+  const int nt = min(kOTok, n_tok - tb);
+  const int64_t row0 = ((int64_t)seq * n_agents + agent) * n_tok + tb;
+  const IO* A = A_o + agent * a_agent_stride;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  for (int m0 = 0; m0 < r; m0 += 16) {     // 16 columns of A_o per pass
+    const int mw = min(16, r - m0);          // 8 at r = 8
+    float acc[kOTok][16];
+#pragma unroll
+    for (int tt = 0; tt < kOTok; ++tt)
+#pragma unroll
+      for (int m = 0; m < 16; ++m) acc[tt][m] = 0.f;
+#pragma unroll 4
+    for (int k = threadIdx.x; k < d_in; k += kOThreads) {
+      const Vec8<IO> a0 = ld8<IO>(A + (int64_t)k * r + m0);
+      Vec8<IO> a1;
+      if (mw > 8) a1 = ld8<IO>(A + (int64_t)k * r + m0 + 8);
+      else
+#pragma unroll
+        for (int j = 0; j < 8; ++j) a1.v[j] = 0.f;
+#pragma unroll
+      for (int tt = 0; tt < kOTok; ++tt) {
+        const float x = tt < nt ? ldf(o + (row0 + tt) * d_in + k) : 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          acc[tt][j] = fmaf(x, a0.v[j], acc[tt][j]);
+          acc[tt][8 + j] = fmaf(x, a1.v[j], acc[tt][8 + j]);
+        }
+      }
+    }
+#pragma unroll
+    for (int tt = 0; tt < kOTok; ++tt) {
+      if (tt >= nt) break;   // the block's last tokens (one in a decode step)
+#pragma unroll
+      for (int m = 0; m < 16; ++m) {
+        float v = acc[tt][m];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+        if (lane == 0) part[w][tt][m] = v;
+      }
+    }
+    __syncthreads();
+    if (threadIdx.x < kOTok * 16) {
+      const int tt = threadIdx.x / 16, m = threadIdx.x % 16;
+      float v = 0.f;
+#pragma unroll
+      for (int ww = 0; ww < kOWarps; ++ww) v += part[ww][tt][m];
+      if (m < mw) t[tt][m0 + m] = v;
+    }
+    __syncthreads();
+  }
+  const int c0 = cb * kOColBlock + threadIdx.x * kOCols;
+  if (c0 >= d_out) return;
+  const IO* B = B_o + (int64_t)agent * r * d_out + c0;
+  float z[kOTok][kOCols];
+#pragma unroll
+  for (int tt = 0; tt < kOTok; ++tt)
+#pragma unroll
+    for (int j = 0; j < kOCols; ++j) z[tt][j] = 0.f;
+#pragma unroll 4
+  for (int m = 0; m < r; ++m) {
+    const Vec8<IO> b = ld8<IO>(B + (int64_t)m * d_out);
+#pragma unroll
+    for (int tt = 0; tt < kOTok; ++tt)
+#pragma unroll
+      for (int j = 0; j < kOCols; ++j) z[tt][j] = fmaf(t[tt][m], b.v[j], z[tt][j]);
+  }
+#pragma unroll
+  for (int tt = 0; tt < kOTok; ++tt) {
+    if (tt < nt) {
+      IO* yp = y + (row0 + tt) * d_out + c0;
+#pragma unroll
+      for (int j = 0; j < kOCols; ++j) yp[j] = stf<IO>(fmaf(s, z[tt][j], ldf(yp + j)));
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_query_expand(const void* q_base, const void* lr_q, const void* B_q, void* q_out,
+                                int n_seqs, int n_agents, int n_tok, int n_q, int d, int r, float s,
+                                double rope_base, const int32_t* pos_end, la_dtype dt,
+                                cudaStream_t st) {
+  RopeTheta rt;
+  for (int i = 0; i < 64; ++i) {
+    rt.theta[i] = i < d / 2 ? std::pow(rope_base, -2.0 * i / d) : 0.0;
+    rt.thetaf[i] = (float)rt.theta[i];
+  }
+  const int hblocks = (n_q + kQThreads / (d / 2) - 1) / (kQThreads / (d / 2));
+  const dim3 grid((unsigned)(((int64_t)n_tok + kQTok - 1) / kQTok * hblocks), (unsigned)n_agents,
+                  (unsigned)n_seqs);
+  if (dt == LA_BF16)
+    query_expand_kernel<__nv_bfloat16><<<grid, kQThreads, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(q_base), static_cast<const __nv_bfloat16*>(lr_q),
+        static_cast<const __nv_bfloat16*>(B_q), static_cast<__nv_bfloat16*>(q_out), n_agents, n_tok,
+        n_q, d, r, s, rt, pos_end);
+  else
+    query_expand_kernel<float><<<grid, kQThreads, 0, st>>>(
+        static_cast<const float*>(q_base), static_cast<const float*>(lr_q),
+        static_cast<const float*>(B_q), static_cast<float*>(q_out), n_agents, n_tok, n_q, d, r, s, rt,
+        pos_end);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_output_delta(const void* o, const void* A_o, int64_t a_agent_stride,
+                                const void* B_o, void* y, int n_seqs, int n_agents, int n_tok,
+                                int d_in, int d_out, int r, float s, la_dtype dt, cudaStream_t st) {
+  const int cblocks = (d_out + kOColBlock - 1) / kOColBlock;
+  const dim3 grid((unsigned)((int64_t)(n_tok + kOTok - 1) / kOTok * cblocks), (unsigned)n_agents,
+                  (unsigned)n_seqs);
+  if (dt == LA_BF16)
+    output_delta_kernel<__nv_bfloat16><<<grid, kOThreads, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(A_o), a_agent_stride,
+        static_cast<const __nv_bfloat16*>(B_o), static_cast<__nv_bfloat16*>(y), n_agents, n_tok,
+        d_in, d_out, r, s);
+  else
+    output_delta_kernel<float><<<grid, kOThreads, 0, st>>>(
+        static_cast<const float*>(o), static_cast<const float*>(A_o), a_agent_stride,
+        static_cast<const float*>(B_o), static_cast<float*>(y), n_agents, n_tok, d_in, d_out, r, s);
+  return cudaGetLastError();
+}
+
+}  // namespace la

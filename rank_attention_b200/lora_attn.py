@@ -26,7 +26,7 @@ LA_F32, LA_BF16 = 0, 1
 EXPORTED = ("la_status_string", "lr_cache_append", "lora_attn_prefill", "lora_attn_decode",
             "lora_attn_decode_workspace_bytes", "la_device_check",
             "lora_attn_decode_static_scratch", "lora_materialize_agent_kv",
-            "lr_cache_append_agents")
+            "lr_cache_append_agents", "lora_query_expand", "lora_output_delta")
 
 
 class LoraAttnError(RuntimeError):
@@ -77,6 +77,16 @@ def _load() -> ctypes.CDLL:
         ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
         ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
         ctypes.c_int64, ctypes.c_int32, ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_void_p]
+    lib.lora_query_expand.restype = ctypes.c_int
+    lib.lora_query_expand.argtypes = [
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
+        ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+        ctypes.c_float, ctypes.c_double, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p]
+    lib.lora_output_delta.restype = ctypes.c_int
+    lib.lora_output_delta.argtypes = [
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
+        ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+        ctypes.c_int32, ctypes.c_float, ctypes.c_int, ctypes.c_void_p]
     lib.lora_attn_prefill.restype = ctypes.c_int
     lib.lora_attn_prefill.argtypes = [ctypes.POINTER(AttnArgs), ctypes.c_void_p]
     lib.lora_attn_decode.restype = ctypes.c_int
@@ -151,6 +161,40 @@ def lr_cache_append_agents(X: torch.Tensor, A_kv: torch.Tensor, lr_cache: torch.
                                     pos0, n_seqs, X.stride(0), lr_cache.stride(1), _dt(X),
                                     _stream(stream))
     _check(st, "lr_cache_append_agents")
+
+
+def lora_query_expand(q_base: torch.Tensor, lr_q: torch.Tensor, B_q: torch.Tensor,
+                      q_out: torch.Tensor, pos_end: torch.Tensor, *, lora_scale: float,
+                      rope_base: float, stream=None) -> None:
+    """q_out = RoPE(q_base + s lr_q B_q^a) per agent and head.
+
+    q_base, q_out [n_seqs, n_agents, n_tok, n_q, d] contiguous (may be the same
+    tensor); lr_q [n_seqs, n_agents, n_tok, r]; B_q [n_agents, r, n_q*d];
+    pos_end int32 [n_seqs]: token j sits at pos_end - n_tok + j."""
+    n_seqs, n_agents, n_tok, n_q, d = q_base.shape
+    r = lr_q.shape[-1]
+    assert q_base.is_contiguous() and q_out.is_contiguous() and lr_q.is_contiguous()
+    assert B_q.is_contiguous() and pos_end.dtype == torch.int32
+    st = lib.lora_query_expand(q_base.data_ptr(), lr_q.data_ptr(), B_q.data_ptr(),
+                               q_out.data_ptr(), n_seqs, n_agents, n_tok, n_q, d, r, lora_scale,
+                               rope_base, pos_end.data_ptr(), _dt(q_base), _stream(stream))
+    _check(st, "lora_query_expand")
+
+
+def lora_output_delta(o: torch.Tensor, A_o: torch.Tensor, B_o: torch.Tensor, y: torch.Tensor, *,
+                      lora_scale: float, stream=None) -> None:
+    """y += s (o A_o) B_o^a per agent.
+
+    o [n_seqs, n_agents, n_tok, d_in]; A_o [d_in, r] shared, or [n_agents, d_in, r];
+    B_o [n_agents, r, d_out]; y [n_seqs, n_agents, n_tok, d_out]; all contiguous."""
+    n_seqs, n_agents, n_tok, d_in = o.shape
+    r, d_out = B_o.shape[1], B_o.shape[2]
+    a_stride = A_o.stride(0) if A_o.dim() == 3 else 0
+    assert o.is_contiguous() and A_o.is_contiguous() and B_o.is_contiguous() and y.is_contiguous()
+    st = lib.lora_output_delta(o.data_ptr(), A_o.data_ptr(), a_stride, B_o.data_ptr(), y.data_ptr(),
+                               n_seqs, n_agents, n_tok, d_in, d_out, r, lora_scale, _dt(o),
+                               _stream(stream))
+    _check(st, "lora_output_delta")
 
 
 def make_args(k_base, v_base, lr, B_k, B_v, q, out, *, lora_scale: float, rope_base: float,

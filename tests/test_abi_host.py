@@ -192,6 +192,51 @@ def test_append_agents_rejects(kw, status):
     assert _append_agents(**kw) == status
 
 
+def _qexp(**kw):
+    a = dict(qb=FAKE, lr=FAKE, B=FAKE, qo=FAKE, n=1, na=3, nt=1, nq=32, d=128, r=16, s=2.0,
+             base=500000.0, pe=FAKE, dt=la.LA_BF16)
+    a.update(kw)
+    return la.lib.lora_query_expand(a["qb"], a["lr"], a["B"], a["qo"], a["n"], a["na"], a["nt"],
+                                    a["nq"], a["d"], a["r"], a["s"], a["base"], a["pe"], a["dt"],
+                                    None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(qb=0), la.LA_ERR_INVALID_ARG),
+    (dict(pe=0), la.LA_ERR_INVALID_ARG),
+    (dict(qo=FAKE + 2), la.LA_ERR_INVALID_ARG),
+    (dict(nt=0), la.LA_ERR_INVALID_ARG),
+    (dict(base=1.0), la.LA_ERR_INVALID_ARG),
+    (dict(d=96), la.LA_ERR_UNSUPPORTED),
+    (dict(r=12), la.LA_ERR_UNSUPPORTED),
+    (dict(dt=5), la.LA_ERR_INVALID_ARG),
+])
+def test_query_expand_rejects(kw, status):
+    assert _qexp(**kw) == status
+
+
+def _odelta(**kw):
+    a = dict(o=FAKE, A=FAKE, As=0, B=FAKE, y=FAKE, n=1, na=3, nt=1, di=4096, do=4096, r=16,
+             s=2.0, dt=la.LA_BF16)
+    a.update(kw)
+    return la.lib.lora_output_delta(a["o"], a["A"], a["As"], a["B"], a["y"], a["n"], a["na"],
+                                    a["nt"], a["di"], a["do"], a["r"], a["s"], a["dt"], None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(y=0), la.LA_ERR_INVALID_ARG),
+    (dict(A=FAKE + 4), la.LA_ERR_INVALID_ARG),
+    (dict(As=-1), la.LA_ERR_INVALID_ARG),
+    (dict(As=4100), la.LA_ERR_INVALID_ARG),      # agents' A_o not 16-byte aligned
+    (dict(di=0), la.LA_ERR_INVALID_ARG),
+    (dict(r=3), la.LA_ERR_UNSUPPORTED),
+    (dict(do=4100), la.LA_ERR_UNSUPPORTED),
+    (dict(s=float("inf")), la.LA_ERR_INVALID_ARG),
+])
+def test_output_delta_rejects(kw, status):
+    assert _odelta(**kw) == status
+
+
 def test_null_args():
     assert la.lib.lora_attn_prefill(None, None) == la.LA_ERR_INVALID_ARG
     assert la.lib.lora_attn_decode(None, FAKE, 1 << 20, None) == la.LA_ERR_INVALID_ARG

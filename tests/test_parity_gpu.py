@@ -535,3 +535,79 @@ def test_base_shared_materialized_caches(la):
     torch.cuda.synchronize()
     assert la.la_device_check() == 0
     assert_parity(to_np(out_ns), oracle_decode(inp, s), s.dtype)
+
+
+# --------------------------- query- and output-side LoRA (qkvo setting) ----
+def _qo_inputs(n_seqs, n_agents, n_tok, n_q, d, r, dtype, seed):
+    g = torch.Generator().manual_seed(seed)
+    q_base = (W.CACHE_STD * torch.randn(n_seqs, n_agents, n_tok, n_q, d, generator=g)).to(dtype)
+    lr_q = (W.CACHE_STD * torch.randn(n_seqs, n_agents, n_tok, r, generator=g)).to(dtype)
+    B_q = (0.02 * torch.randn(n_agents, r, n_q * d, generator=g)).to(dtype)
+    return q_base, lr_q, B_q
+
+
+@pytest.mark.parametrize("dtype,n_seqs,n_agents,n_tok,n_q,d,r,in_place", [
+    (torch.bfloat16, 1, 3, 1, 32, 128, 16, False),    # one decode step of the 3-agent layer
+    (torch.bfloat16, 2, 2, 37, 32, 128, 64, True),    # a ragged prefill chunk, in place
+    (torch.float32, 2, 3, 5, 4, 64, 8, False),        # the tiny fp32 shape
+])
+def test_query_expand_against_oracle(la, dtype, n_seqs, n_agents, n_tok, n_q, d, r, in_place):
+    q_base, lr_q, B_q = _qo_inputs(n_seqs, n_agents, n_tok, n_q, d, r, dtype, 300 + r)
+    pos_end = torch.tensor([5000 + 977 * i for i in range(n_seqs)], dtype=torch.int32)
+    s, base = 2.0, 500000.0
+    qb = q_base.to(DEV)
+    out = qb if in_place else torch.empty_like(qb)
+    la.lora_query_expand(qb, lr_q.to(DEV), B_q.to(DEV), out, pos_end.to(DEV), lora_scale=s,
+                         rope_base=base)
+    torch.cuda.synchronize()
+    ref = np.empty(q_base.shape)
+    for q in range(n_seqs):
+        pos = int(pos_end[q]) - n_tok + np.arange(n_tok)
+        for a in range(n_agents):
+            ref[q, a] = oracle.lora_queries(q_base[q, a], lr_q[q, a], B_q[a], s, pos, base)
+    assert_parity(to_np(out), ref, dtype)
+
+
+@pytest.mark.parametrize("dtype,n_seqs,n_agents,n_tok,r,per_agent_A", [
+    (torch.bfloat16, 1, 3, 1, 16, False),     # a decode step, shared A_o
+    (torch.bfloat16, 2, 2, 19, 64, True),     # ragged token blocks, per-agent A_o
+    (torch.float32, 1, 2, 9, 8, False),
+])
+def test_output_delta_against_oracle(la, dtype, n_seqs, n_agents, n_tok, r, per_agent_A):
+    d_in, d_out = 4096, 4096
+    g = torch.Generator().manual_seed(400 + r)
+    o = torch.randn(n_seqs, n_agents, n_tok, d_in, generator=g).to(dtype)
+    A_shape = (n_agents, d_in, r) if per_agent_A else (d_in, r)
+    A_o = (0.02 * torch.randn(*A_shape, generator=g)).to(dtype)
+    B_o = (0.02 * torch.randn(n_agents, r, d_out, generator=g)).to(dtype)
+    y0 = torch.randn(n_seqs, n_agents, n_tok, d_out, generator=g).to(dtype)
+    y = y0.to(DEV)
+    s = 2.0
+    la.lora_output_delta(o.to(DEV), A_o.to(DEV), B_o.to(DEV), y, lora_scale=s)
+    torch.cuda.synchronize()
+    ref = np.empty(y0.shape)
+    for q in range(n_seqs):
+        for a in range(n_agents):
+            Aa = A_o[a] if per_agent_A else A_o
+            ref[q, a] = oracle.lora_output(y0[q, a], o[q, a], Aa, B_o[a], s)
+    assert_parity(to_np(y), ref, dtype)
+    if dtype == torch.float32:   # the delta alone too (fp32 keeps it exact enough to isolate)
+        assert_parity(to_np(y) - to_np(y0), ref - to_np(y0), dtype)
+
+
+def test_query_expand_then_decode(la):
+    """The decode step with a query-side LoRA: expanded queries feed the
+    attention; the oracle rotates its own q^a and attends."""
+    s = W.LLAMA8B_DECODE_8K.replace(kv_len=900, seed=61)
+    inp = W.direct_cache_inputs(s)
+    q_base, lr_q, B_q = _qo_inputs(s.n_seqs, s.n_agents, 1, s.n_q_heads, s.head_dim, s.r,
+                                   s.dtype, 62)
+    dd = to_device(inp)
+    q = torch.empty_like(dd["q"])
+    la.lora_query_expand(q_base.to(DEV), lr_q.to(DEV), B_q.to(DEV), q, dd["kv_len"],
+                         lora_scale=s.lora_scale, rope_base=s.rope_base)
+    got = _run(la, s, dd["k_base"], dd["v_base"], dd["lr"], dd["B_k"], dd["B_v"], q, dd["kv_len"])
+    qa = np.stack([oracle.lora_queries(q_base[0, a], lr_q[0, a], B_q[a], s.lora_scale,
+                                       [s.kv_len - 1], s.rope_base) for a in range(s.n_agents)])
+    inp_q = dict(inp, q=torch.from_numpy(qa[None]).to(s.dtype))   # the kernel's queries are bf16
+    assert_parity(to_np(got), oracle_decode(inp_q, s), s.dtype)
