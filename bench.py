@@ -46,7 +46,8 @@ def parse():
     ap.add_argument("--all-configs", action="store_true",
                     help="also time the long-context decode sweep and one layer of the "
                          "32-layer stack (decode and prefill), reported under other_configs")
-    ap.add_argument("--profile", nargs="?", const="decode", choices=["decode", "prefill"],
+    ap.add_argument("--profile", nargs="?", const="decode",
+                    choices=["decode", "prefill", "append", "qkvo"],
                     help="a short deterministic run of one kernel for profilers "
                          "(decode: the 8192-token decode five times; prefill: the "
                          "16384 + 1024-token prefill three times); prints nothing")
@@ -414,6 +415,17 @@ def run_profile(kind: str = "decode"):
     from rank_attention_b200 import lora_attn as la
     from rank_attention_b200 import workloads as W
     dev = torch.device("cuda", 0)
+    if kind == "append":   # one layer of the stack: a 4096-token chunk through r = 64 shared A
+        s = W.llama8b_stack_prefill(0)
+        inp = W.append_inputs(s.n_q_tokens, s.hidden, s.r, torch.bfloat16, seed=9, device=dev)
+        lr = torch.zeros((1, s.kv_len, 2 * s.r), dtype=torch.bfloat16, device=dev)
+        for _ in range(3):
+            la.lr_cache_append(inp["X"], inp["A_kv"], lr, s.kv_len - s.n_q_tokens)
+        torch.cuda.synchronize()
+        return 0 if la.la_device_check() == 0 else 1
+    if kind == "qkvo":     # query expand and output delta, 1024 tokens per agent
+        timed = time_qkvo(dev)
+        return 0 if timed else 1
     s = W.LLAMA8B_DECODE_8K if kind == "decode" else W.LLAMA8B_PREFILL_16K
     inp = {k: v.to(dev) for k, v in W.direct_cache_inputs(s, device=dev).items()}
     out = torch.empty(inp["q"].shape, dtype=torch.float32, device=dev)
