@@ -387,7 +387,7 @@ class ClockSampler:
 # DRAM bytes per decode launch from an ncu capture of the workload, keyed by the
 # sha256 prefix of the decode kernel's source: reported only while the kernel is
 # unchanged since the counters were taken.
-DECODE_TRAFFIC = {"0118cb326e4aeb7f": 34415104}
+DECODE_TRAFFIC = {"de1f4b62b2e1f47a": 34417664}
 
 
 def decode_source_sha() -> str:
