@@ -67,6 +67,22 @@ typedef enum {
 
 typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
 
+/* How the value side is computed (la_attn_args.value_path).  The three give
+ * the same outputs up to rounding; 1 and 2 exist to measure the reordering
+ * (the naive-reconstruction ablation of LRAgent summary App. B / explainer,
+ * Metodologia 3):
+ *   LA_VALUE_REORDERED          O = P V_base + (P LRv) s B_v^a, B_v applied once
+ *                               per row; the fastest kernel for the shape.
+ *   LA_VALUE_REORDERED_GENERIC  the same on the generic CUDA-core kernel.
+ *   LA_VALUE_PER_TILE           naive: per key tile and agent, V^a = V_base +
+ *                               s LRv B_v^a rebuilt in head dimension, then
+ *                               O += P V^a; the generic CUDA-core kernel. */
+typedef enum {
+  LA_VALUE_REORDERED = 0,
+  LA_VALUE_REORDERED_GENERIC = 1,
+  LA_VALUE_PER_TILE = 2
+} la_value_path;
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* la_status_string(la_status s);
 
@@ -166,6 +182,7 @@ typedef struct {
    * de Compartilhamento"; PReCache blog, how PReCache precomputes each
    * role's cache.  The base cache stays shared in both cases. */
   int64_t lr_agent_stride;
+  int32_t value_path;   /* la_value_path; 0 (zeroed struct) = LA_VALUE_REORDERED */
 } la_attn_args;
 
 /*

@@ -67,6 +67,7 @@ la_status check_attn(const la_attn_args* a, int decode, AttnParams* p) {
       (!stride_ok(a->lr_agent_stride, io) ||
        a->lr_agent_stride < (int64_t)(a->n_seqs > 0 ? a->n_seqs - 1 : 0) * a->lr_seq_stride + a->L_max * 2 * a->r))
     return LA_ERR_INVALID_ARG;
+  if (a->value_path < LA_VALUE_REORDERED || a->value_path > LA_VALUE_PER_TILE) return LA_ERR_INVALID_ARG;
   const int g = a->n_q_heads / a->n_kv_heads;
   if ((int64_t)a->n_agents * g > kMaxRowsSimt) return LA_ERR_UNSUPPORTED;
   if (decode) {
@@ -99,6 +100,7 @@ la_status check_attn(const la_attn_args* a, int decode, AttnParams* p) {
   p->lr = a->lr_cache;
   p->lr_seq = a->lr_seq_stride;
   p->lr_agent = a->lr_agent_stride;
+  p->value_path = a->value_path;
   p->B_k = a->B_k;
   p->B_v = a->B_v;
   p->q = a->q;
@@ -117,7 +119,7 @@ DecodePlan plan_decode(const AttnParams& p, la_dtype io) {
   DecodePlan d;
   memset(&d, 0, sizeof(d));
   const int units = p.n_seqs * p.n_kv;
-  if (io == LA_BF16 && bf16_decode_supported(p)) {
+  if (io == LA_BF16 && p.value_path == LA_VALUE_REORDERED && bf16_decode_supported(p)) {
     d.kind = 1;
     bf16_decode_plan(p, &d.n_splits, &d.split_len, &d.rows, &d.groups);
   } else {
@@ -308,7 +310,7 @@ extern "C" la_status lora_attn_prefill(const la_attn_args* a, la_stream_t stream
   if (s != LA_OK) return s;
   if (p.n_seqs == 0 || p.n_q_tokens == 0) return LA_OK;
   if ((int64_t)p.n_seqs * p.n_kv > 65535) return LA_ERR_UNSUPPORTED;
-  const bool tc = a->io_dtype == LA_BF16 && bf16_prefill_supported(p);
+  const bool tc = a->io_dtype == LA_BF16 && p.value_path == LA_VALUE_REORDERED && bf16_prefill_supported(p);
   if (!tc && simt_smem_bytes(p) > 227 * 1024) return LA_ERR_UNSUPPORTED;
   p.err = error_word_ptr();
   if (!p.err) return LA_ERR_CUDA;

@@ -80,7 +80,10 @@ __device__ __forceinline__ float2 rope_cs(int64_t t, double theta) {
   return make_float2(cs, sn);
 }
 
-template <typename IO, typename OUT>
+// NAIVE: the value side rebuilt in head dimension per tile and agent,
+// V^a = V_base + s LRv B_v^a, then O += P V^a (no rank-r partial; the
+// naive-reconstruction baseline the reordering is measured against).
+template <typename IO, typename OUT, bool NAIVE>
 __global__ void __launch_bounds__(NT) attn_simt_kernel(const AttnParams p, const int qb) {
   extern __shared__ __align__(16) unsigned char smem[];
   const int D = p.d, R = p.r, H2 = D / 2, g = p.g, na = p.n_agents;
@@ -227,8 +230,34 @@ __global__ void __launch_bounds__(NT) attn_simt_kernel(const AttnParams p, const
     }
     __syncthreads();
 
-    // 4. O_base += P V_base ; O_lr += P LRv
     const int W = D + R;
+    if constexpr (NAIVE) {
+      // 4'. per agent: V^a tile in head dimension (over the key buffer), then
+      // O_base += P V^a for the agent's rows; O_lr stays zero
+      for (int a = 0; a < na; ++a) {
+        const IO* Bv = reinterpret_cast<const IO*>(p.B_v) + (int64_t)a * R * ldB + kvh * D;
+        const float* LRa = LRs + (n_lr > 1 ? a : 0) * TK * 2 * R;
+        for (int i = tid; i < TK * D; i += NT) {
+          const int t = i / D, c = i % D;
+          float x = 0.f;
+          for (int j = 0; j < R; ++j) x = fmaf(LRa[t * 2 * R + R + j], to_f32(Bv[j * ldB + c]), x);
+          Ka[i] = fmaf(p.s, x, Vb[i]);
+        }
+        __syncthreads();
+        const int rows_a = ntok * g;
+        for (int i = tid; i < rows_a * D; i += NT) {
+          const int ra = i / D, c = i % D;
+          const int row = ((ra / g) * na + a) * g + (ra % g);
+          float acc = O[row * W + c] * Al[row];
+          const float* Pr = S + row * TK;
+          for (int t = 0; t < TK; ++t) acc = fmaf(Pr[t], Ka[t * D + c], acc);
+          O[row * W + c] = acc;
+        }
+        __syncthreads();
+      }
+      continue;
+    }
+    // 4. O_base += P V_base ; O_lr += P LRv
     for (int i = tid; i < rows * W; i += NT) {
       const int row = i / W, c = i % W;
       float acc = O[i] * Al[row];
@@ -309,18 +338,18 @@ __global__ void __launch_bounds__(NT) attn_simt_kernel(const AttnParams p, const
   }
 }
 
-template <typename IO, typename OUT>
+template <typename IO, typename OUT, bool NAIVE>
 cudaError_t launch_typed(const AttnParams& p, cudaStream_t st) {
   const int qb = p.decode ? 1 : max(1, kMaxRowsSimt / p.rows_per_tok);
   const int rows_cap = qb * p.rows_per_tok;
   SmemLayout L(rows_cap, p.d, p.r, p.lr_agent ? p.n_agents : 1);
   if (L.total > 227 * 1024) return cudaErrorInvalidConfiguration;
-  cudaError_t e = cudaFuncSetAttribute(attn_simt_kernel<IO, OUT>,
+  cudaError_t e = cudaFuncSetAttribute(attn_simt_kernel<IO, OUT, NAIVE>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.total);
   if (e != cudaSuccess) return e;
   const int units = p.n_seqs * p.n_kv;
   dim3 grid(p.decode ? p.n_splits : 1, p.decode ? 1 : (p.n_q_tokens + qb - 1) / qb, units);
-  attn_simt_kernel<IO, OUT><<<grid, NT, L.total, st>>>(p, qb);
+  attn_simt_kernel<IO, OUT, NAIVE><<<grid, NT, L.total, st>>>(p, qb);
   return cudaGetLastError();
 }
 
@@ -337,11 +366,17 @@ size_t simt_smem_bytes(const AttnParams& p) {
   return SmemLayout((int)simt_rows_cap(p), p.d, p.r, p.lr_agent ? p.n_agents : 1).total;
 }
 
+template <bool NAIVE>
+cudaError_t launch_io(const AttnParams& p, la_dtype io, la_dtype out, cudaStream_t st) {
+  if (io == LA_F32 && out == LA_F32) return launch_typed<float, float, NAIVE>(p, st);
+  if (io == LA_F32 && out == LA_BF16) return launch_typed<float, __nv_bfloat16, NAIVE>(p, st);
+  if (io == LA_BF16 && out == LA_F32) return launch_typed<__nv_bfloat16, float, NAIVE>(p, st);
+  return launch_typed<__nv_bfloat16, __nv_bfloat16, NAIVE>(p, st);
+}
+
 cudaError_t launch_attn_simt(const AttnParams& p, la_dtype io, la_dtype out, cudaStream_t st) {
-  if (io == LA_F32 && out == LA_F32) return launch_typed<float, float>(p, st);
-  if (io == LA_F32 && out == LA_BF16) return launch_typed<float, __nv_bfloat16>(p, st);
-  if (io == LA_BF16 && out == LA_F32) return launch_typed<__nv_bfloat16, float>(p, st);
-  return launch_typed<__nv_bfloat16, __nv_bfloat16>(p, st);
+  return p.value_path == LA_VALUE_PER_TILE ? launch_io<true>(p, io, out, st)
+                                           : launch_io<false>(p, io, out, st);
 }
 
 }  // namespace la

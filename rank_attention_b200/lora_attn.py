@@ -22,6 +22,7 @@ LA_OK, LA_ERR_INVALID_ARG, LA_ERR_UNSUPPORTED, LA_ERR_CAPACITY = 0, 1, 2, 3
 LA_ERR_WORKSPACE, LA_ERR_CUDA, LA_ERR_DEVICE_CHECK, LA_ERR_SCRATCH_LIMIT = 4, 5, 6, 7
 LA_STATIC_SCRATCH_BYTES = 4 << 20
 LA_F32, LA_BF16 = 0, 1
+LA_VALUE_REORDERED, LA_VALUE_REORDERED_GENERIC, LA_VALUE_PER_TILE = 0, 1, 2
 
 EXPORTED = ("la_status_string", "lr_cache_append", "lora_attn_prefill", "lora_attn_decode",
             "lora_attn_decode_workspace_bytes", "la_device_check",
@@ -57,6 +58,7 @@ class AttnArgs(ctypes.Structure):
         ("n_q_tokens", ctypes.c_int32),
         ("io_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int),
         ("lr_agent_stride", ctypes.c_int64),
+        ("value_path", ctypes.c_int32),
     ]
 
 
@@ -199,7 +201,7 @@ def lora_output_delta(o: torch.Tensor, A_o: torch.Tensor, B_o: torch.Tensor, y: 
 
 def make_args(k_base, v_base, lr, B_k, B_v, q, out, *, lora_scale: float, rope_base: float,
               softmax_scale: Optional[float] = None, kv_len: Optional[torch.Tensor] = None,
-              max_kv_len: int = 0, q_pos0: int = 0) -> AttnArgs:
+              max_kv_len: int = 0, q_pos0: int = 0, value_path: int = LA_VALUE_REORDERED) -> AttnArgs:
     """Fill la_attn_args from tensors.
 
     k_base, v_base [n_seqs, n_kv, L_max, d] (any strides with a unit last
@@ -236,6 +238,7 @@ def make_args(k_base, v_base, lr, B_k, B_v, q, out, *, lora_scale: float, rope_b
     a.n_q_tokens = n_tok
     a.io_dtype, a.out_dtype = _dt(k_base), _dt(out)
     a.lr_agent_stride = lr_agent_stride
+    a.value_path = value_path
     return a
 
 

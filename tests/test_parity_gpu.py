@@ -611,3 +611,40 @@ def test_query_expand_then_decode(la):
                                        [s.kv_len - 1], s.rope_base) for a in range(s.n_agents)])
     inp_q = dict(inp, q=torch.from_numpy(qa[None]).to(s.dtype))   # the kernel's queries are bf16
     assert_parity(to_np(got), oracle_decode(inp_q, s), s.dtype)
+
+
+# -------------------- value side: reordered vs rebuilt per tile (ablation) ----
+def _run_path(la, s, dd, value_path):
+    out = torch.empty(dd["q"].shape, dtype=torch.float32, device=DEV)
+    if s.mode == "decode":
+        args = la.make_args(dd["k_base"], dd["v_base"], dd["lr"], dd["B_k"], dd["B_v"], dd["q"], out,
+                            lora_scale=s.lora_scale, rope_base=s.rope_base, kv_len=dd["kv_len"],
+                            max_kv_len=s.kv_len, value_path=value_path)
+        la.lora_attn_decode(args, la.decode_workspace(args, DEV))
+    else:
+        args = la.make_args(dd["k_base"], dd["v_base"], dd["lr"], dd["B_k"], dd["B_v"], dd["q"], out,
+                            lora_scale=s.lora_scale, rope_base=s.rope_base, q_pos0=s.q_pos0,
+                            value_path=value_path)
+        la.lora_attn_prefill(args)
+    torch.cuda.synchronize()
+    assert la.la_device_check() == 0
+    return out
+
+
+@pytest.mark.parametrize("shape", [
+    W.LLAMA8B_DECODE_8K.replace(kv_len=700, seed=81),
+    W.LLAMA8B_PREFILL_16K.replace(kv_len=300, n_q_tokens=45, seed=82),
+    W.LLAMA8B_DECODE_8K.replace(kv_len=500, seed=83, lr_per_agent=True),
+    W.TINY_FP32.replace(kv_len=150, seed=84),
+])
+@pytest.mark.parametrize("value_path", [1, 2])
+def test_value_paths_match_the_oracle(la, shape, value_path):
+    """The generic kernel with the reordered value side (1) and with V^a rebuilt
+    per tile (2): both equal the oracle (which materialises V^a)."""
+    inp = W.direct_cache_inputs(shape)
+    got = _run_path(la, shape, to_device(inp), value_path)
+    ref = oracle.lora_attention(inp["k_base"], inp["v_base"], inp["lr"], inp["B_k"], inp["B_v"],
+                                inp["q"], inp["kv_len"], lora_scale=shape.lora_scale,
+                                softmax_scale=shape.softmax_scale, rope_base=shape.rope_base,
+                                mode=shape.mode)
+    assert_parity(to_np(got), ref, shape.dtype)
