@@ -17,9 +17,12 @@
 
 #include "bf16_common.cuh"
 #include "la_internal.cuh"
+#include "ptx.cuh"
 
 namespace la {
 namespace {
+
+using ptx::pack_bf16;
 
 template <typename IO>
 __device__ __forceinline__ float ldf(const IO* p);
@@ -34,16 +37,47 @@ __device__ __forceinline__ float stf<float>(float x) { return x; }
 template <>
 __device__ __forceinline__ __nv_bfloat16 stf<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
 
-constexpr int kQThreads = 256;  // one (head, frequency) pair each: 4 heads a CTA at d = 128
-constexpr int kQTok = 16;     // tokens per CTA: each B_q^a value is loaded once for them
+constexpr int kQThreads = 256;
+constexpr int kQTok = 8;      // tokens per CTA: each B_q^a value is loaded once for them
+constexpr int kQF = 4;        // adjacent frequencies per thread (one 8-byte bf16 access)
 
-// One CTA per (16 tokens x 4 heads, agent, sequence); a thread owns one
-// (head, frequency) pair, x_i and x_{i+d/2}, for all the CTA's tokens: it
-// loads its r B_q^a pairs once, accumulates the deltas of every token, then
-// adds each token's base projection and rotates (the delta joins before the
-// rotation; every element is written once, so q_out may alias q_base).
-// (cos, sin) per (token, frequency) are formed once per CTA, angle reduced in
-// fp64.
+template <typename IO>
+struct Vec4 {
+  float v[4];
+};
+template <typename IO>
+__device__ __forceinline__ Vec4<IO> ld4(const IO* p);
+template <>
+__device__ __forceinline__ Vec4<__nv_bfloat16> ld4<__nv_bfloat16>(const __nv_bfloat16* p) {
+  Vec4<__nv_bfloat16> r;
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  r.v[0] = __uint_as_float(u.x << 16);
+  r.v[1] = __uint_as_float(u.x & 0xffff0000u);
+  r.v[2] = __uint_as_float(u.y << 16);
+  r.v[3] = __uint_as_float(u.y & 0xffff0000u);
+  return r;
+}
+template <>
+__device__ __forceinline__ Vec4<float> ld4<float>(const float* p) {
+  Vec4<float> r;
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  r.v[0] = a.x; r.v[1] = a.y; r.v[2] = a.z; r.v[3] = a.w;
+  return r;
+}
+__device__ __forceinline__ void st4(__nv_bfloat16* p, const float (&v)[4]) {
+  *reinterpret_cast<uint2*>(p) = make_uint2(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]));
+}
+__device__ __forceinline__ void st4(float* p, const float (&v)[4]) {
+  *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+}
+
+// One CTA per (8 tokens x a block of heads, agent, sequence); a thread owns
+// 4 adjacent frequencies i of one head -- elements i and i + d/2, the RoPE
+// pairs -- for all the CTA's tokens: it loads its slices of the r rows of
+// B_q^a once, accumulates every token's delta, then adds the token's base
+// projection and rotates (the delta joins before the rotation; every element
+// is written once, so q_out may alias q_base).  (cos, sin) per (token,
+// frequency) are formed once per CTA, angle reduced in fp64.
 template <typename IO>
 __global__ void __launch_bounds__(kQThreads) query_expand_kernel(
     const IO* __restrict__ q_base, const IO* __restrict__ lr_q, const IO* __restrict__ B_q,
@@ -52,7 +86,8 @@ __global__ void __launch_bounds__(kQThreads) query_expand_kernel(
   __shared__ float lr[kQTok][64];
   __shared__ float2 cs[kQTok][64];
   const int h2 = d / 2, ld = n_q * d;
-  const int hpb = kQThreads / h2;                     // heads per CTA (4 at d = 128, 8 at d = 64)
+  const int tph = h2 / kQF;                           // threads per head
+  const int hpb = kQThreads / tph;                    // heads per CTA (16 at d = 128)
   const int hblocks = (n_q + hpb - 1) / hpb;
   const int tb = (blockIdx.x / hblocks) * kQTok, h0 = (blockIdx.x % hblocks) * hpb;
   const int agent = blockIdx.y, seq = blockIdx.z;
@@ -64,20 +99,26 @@ __global__ void __launch_bounds__(kQThreads) query_expand_kernel(
   for (int u = threadIdx.x; u < nt * h2; u += kQThreads)
     cs[u / h2][u % h2] = rope_cs_exact(pos0 + u / h2, rt.theta[u % h2]);
   __syncthreads();
-  const int h = h0 + threadIdx.x / h2, i = threadIdx.x % h2;
+  const int h = h0 + threadIdx.x / tph, i0 = (threadIdx.x % tph) * kQF;
   if (h >= n_q) return;
-  const int c1 = h * d + i, c2 = c1 + h2;
+  const int c1 = h * d + i0, c2 = c1 + h2;
   const IO* B = B_q + (int64_t)agent * r * ld;
-  float x1[kQTok], x2[kQTok];
+  float x1[kQTok][kQF], x2[kQTok][kQF];
 #pragma unroll
-  for (int tt = 0; tt < kQTok; ++tt) x1[tt] = x2[tt] = 0.f;
-#pragma unroll 16
+  for (int tt = 0; tt < kQTok; ++tt)
+#pragma unroll
+    for (int j = 0; j < kQF; ++j) x1[tt][j] = x2[tt][j] = 0.f;
+#pragma unroll 4
   for (int m = 0; m < r; ++m) {
-    const float b1 = ldf(B + (int64_t)m * ld + c1), b2 = ldf(B + (int64_t)m * ld + c2);
+    const Vec4<IO> b1 = ld4<IO>(B + (int64_t)m * ld + c1), b2 = ld4<IO>(B + (int64_t)m * ld + c2);
 #pragma unroll
     for (int tt = 0; tt < kQTok; ++tt) {
-      x1[tt] = fmaf(lr[tt][m], b1, x1[tt]);
-      x2[tt] = fmaf(lr[tt][m], b2, x2[tt]);
+      const float l = lr[tt][m];
+#pragma unroll
+      for (int j = 0; j < kQF; ++j) {
+        x1[tt][j] = fmaf(l, b1.v[j], x1[tt][j]);
+        x2[tt][j] = fmaf(l, b2.v[j], x2[tt][j]);
+      }
     }
   }
 #pragma unroll
@@ -85,17 +126,24 @@ __global__ void __launch_bounds__(kQThreads) query_expand_kernel(
     if (tt < nt) {
       const IO* qb = q_base + (row0 + tt) * ld;
       IO* qo = q_out + (row0 + tt) * ld;
-      const float y1 = fmaf(s, x1[tt], ldf(qb + c1)), y2 = fmaf(s, x2[tt], ldf(qb + c2));
-      const float2 c = cs[tt][i];
-      qo[c1] = stf<IO>(y1 * c.x - y2 * c.y);
-      qo[c2] = stf<IO>(y2 * c.x + y1 * c.y);
+      const Vec4<IO> a1 = ld4<IO>(qb + c1), a2 = ld4<IO>(qb + c2);
+      float o1[kQF], o2[kQF];
+#pragma unroll
+      for (int j = 0; j < kQF; ++j) {
+        const float y1 = fmaf(s, x1[tt][j], a1.v[j]), y2 = fmaf(s, x2[tt][j], a2.v[j]);
+        const float2 c = cs[tt][i0 + j];
+        o1[j] = y1 * c.x - y2 * c.y;
+        o2[j] = y2 * c.x + y1 * c.y;
+      }
+      st4(qo + c1, o1);
+      st4(qo + c2, o2);
     }
   }
 }
 
 constexpr int kOThreads = 256;
 constexpr int kOWarps = kOThreads / 32;
-constexpr int kOTok = 8;      // tokens per CTA: A_o and B_o^a are read once for them
+constexpr int kOTok = 4;      // tokens per CTA: A_o and B_o^a are read once for them
 constexpr int kOCols = 8;     // output columns per thread (one 16-byte load of bf16)
 constexpr int kOColBlock = kOThreads * kOCols;
 
@@ -126,7 +174,7 @@ __device__ __forceinline__ Vec8<float> ld8<float>(const float* p) {
   return r;
 }
 
-// One CTA per (8 tokens x 2048 output columns, agent, sequence).  Shrink
+// One CTA per (4 tokens x 2048 output columns, agent, sequence).  Shrink
 // t = O A_o for the CTA's tokens (each column block recomputes it: O(D_in r)
 // per token, small against the expand): thread j takes rows j, j + 256, ...
 // of A_o, 16 columns at a time as two 16-byte vectors, multiplies them by
@@ -213,8 +261,12 @@ __global__ void __launch_bounds__(kOThreads) output_delta_kernel(
   for (int tt = 0; tt < kOTok; ++tt) {
     if (tt < nt) {
       IO* yp = y + (row0 + tt) * d_out + c0;
+      const Vec8<IO> y0 = ld8<IO>(yp);
+      float o[kOCols];
 #pragma unroll
-      for (int j = 0; j < kOCols; ++j) yp[j] = stf<IO>(fmaf(s, z[tt][j], ldf(yp + j)));
+      for (int j = 0; j < kOCols; ++j) o[j] = fmaf(s, z[tt][j], y0.v[j]);
+      st4(yp, *reinterpret_cast<const float(*)[4]>(o));
+      st4(yp + 4, *reinterpret_cast<const float(*)[4]>(o + 4));
     }
   }
 }
@@ -230,7 +282,8 @@ cudaError_t launch_query_expand(const void* q_base, const void* lr_q, const void
     rt.theta[i] = i < d / 2 ? std::pow(rope_base, -2.0 * i / d) : 0.0;
     rt.thetaf[i] = (float)rt.theta[i];
   }
-  const int hblocks = (n_q + kQThreads / (d / 2) - 1) / (kQThreads / (d / 2));
+  const int hpb = kQThreads / (d / 2 / kQF);
+  const int hblocks = (n_q + hpb - 1) / hpb;
   const dim3 grid((unsigned)(((int64_t)n_tok + kQTok - 1) / kQTok * hblocks), (unsigned)n_agents,
                   (unsigned)n_seqs);
   if (dt == LA_BF16)
