@@ -274,8 +274,9 @@ def time_base_shared(dev):
             "cache_bytes": {"base": base, "lr_per_agent_total": s.n_agents * lr_one,
                             "lr_shared": lr_one},
             "what": "each agent reads its own LR cache X A_a beside the shared base cache "
-                    "(one agent per CTA); shared_lr_decode_us: the same decode with one "
-                    "LR cache (shared A), timed the same way",
+                    "(at r = 16 up to three agents a CTA, each stage holding every agent's LR "
+                    "tile); shared_lr_decode_us: the same decode with one LR cache (shared A), "
+                    "timed the same way",
             "timing": own["timing"]}
 
 

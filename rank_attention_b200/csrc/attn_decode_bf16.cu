@@ -694,14 +694,17 @@ constexpr int TC_COLS = 512;                        // TMEM columns allocated
 constexpr int TC_SCOL = 384;                        // TMEM column of S_base
 constexpr int TC_OCOL = 448;                        // TMEM column of O_base^T (d lanes x query rows)
 
-template <int D, int R, int NT>
+// PA: one LR cache per agent with several agents per CTA -- every stage holds
+// each agent's LR tile beside the shared base tiles (r = 16: up to 3 agents)
+template <int D, int R, int NT, bool PA = false>
 struct TCfg {
   static constexpr int ROWS = NT * 8;
+  static constexpr int NLR = PA ? 3 : 1;               // LR tiles per stage
   static constexpr int QPAD = NT <= 2 ? 16 : 32;        // N of the base-score MMA
   static constexpr int W = D + R + 4;
   static constexpr int KV_TILE = KT * D * 2;
   static constexpr int LR_TILE = align1k(KT * 2 * R * 2);
-  static constexpr int STAGE = 2 * KV_TILE + LR_TILE;
+  static constexpr int STAGE = 2 * KV_TILE + NLR * LR_TILE;
   static constexpr int AREA = imax(ST * STAGE, align1k(ROWS * W * 4));
   static constexpr int P_TILE = align1k(ROWS * KT * 2);
   static constexpr int SMALL = 2 * TC_NES * ROWS * 4 + 2 * ROWS * 4 + TC_NES * ROWS * 4 + 64 * 8 + 16 + 64 * 8;
@@ -745,14 +748,14 @@ __device__ __forceinline__ float2 unpack_half2(uint32_t v) {
   return __half22float2(*reinterpret_cast<const __half2*>(&v));
 }
 
-template <int D, int R, int NT>
+template <int D, int R, int NT, bool PA>
 __global__ void __launch_bounds__(TC_NTHR, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV,
                      const __grid_constant__ CUtensorMap tmL,
                      const __grid_constant__ CUtensorMap tmB, const AttnParams p,
                      const __grid_constant__ RopeTheta rt) {
-  using C = TCfg<D, R, NT>;
+  using C = TCfg<D, R, NT, PA>;
   constexpr int W = C::W, ROWS = C::ROWS, QPAD = C::QPAD;
   constexpr int NB = 32 * (TC_NES + NPV);   // threads in the score / value barriers
   extern __shared__ unsigned char smem_raw[];
@@ -814,16 +817,19 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
     const uint32_t sb = area_u + s * C::STAGE;
     const uint32_t bar = full_u + 8 * s;
     const int key0 = (int)(k_lo + (int64_t)n * KT);
-    mbar_expect_tx(bar, 2 * C::KV_TILE + KT * 2 * R * 2);
+    const int nlr = PA ? na : 1;   // the agents' own LR tiles, or the shared one
+    mbar_expect_tx(bar, 2 * C::KV_TILE + nlr * KT * 2 * R * 2);
 #pragma unroll
     for (int b = 0; b < D / 64; ++b) {
       tma_load_4d(sb + b * KT * 128, &tmK, bar, 64 * b, key0, kvh, seq);
       tma_load_4d(sb + C::KV_TILE + b * KT * 128, &tmV, bar, 64 * b, key0, kvh, seq);
     }
     constexpr int LB = (2 * R) < 64 ? 2 * R : 64;
+    for (int al = 0; al < nlr; ++al)
 #pragma unroll
-    for (int b = 0; b < (2 * R) / LB; ++b)
-      tma_load_4d(sb + 2 * C::KV_TILE + b * KT * LB * 2, &tmL, bar, LB * b, key0, seq, lra);
+      for (int b = 0; b < (2 * R) / LB; ++b)
+        tma_load_4d(sb + 2 * C::KV_TILE + al * C::LR_TILE + b * KT * LB * 2, &tmL, bar, LB * b, key0, seq,
+                    PA ? agent0 + al : lra);
   };
 
   // ---- first loads (independent of kv_len): queries, B_k^a, the first tiles, B_v^a
@@ -1207,10 +1213,11 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
           *reinterpret_cast<uint32_t*>(vb + tile_off<D, KT>(row, c)) = 0u;
         }
         if (pv == 0)
-          for (int i = lane; i < (KT - first) * (R / 2); i += 32) {
-            const int row = first + i / (R / 2), c = R + 2 * (i % (R / 2));
-            *reinterpret_cast<uint32_t*>(lb + tile_off<2 * R, KT>(row, c)) = 0u;
-          }
+          for (int al = 0; al < (PA ? na : 1); ++al)
+            for (int i = lane; i < (KT - first) * (R / 2); i += 32) {
+              const int row = first + i / (R / 2), c = R + 2 * (i % (R / 2));
+              *reinterpret_cast<uint32_t*>(lb + al * C::LR_TILE + tile_off<2 * R, KT>(row, c)) = 0u;
+            }
         fence_proxy_async_smem();  // the P V MMA reads V through the async proxy
       }
       __syncwarp();
@@ -1234,12 +1241,30 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
 #pragma unroll
           for (int pt = 0; pt < NT; ++pt)
             ldsm_x2(bP[pt][0], bP[pt][1], pt_u + tile_off<KT, ROWS>(8 * pt + rr, 16 * ks + ((lane >> 3) & 1) * 8));
+          if constexpr (PA) {
+            // each agent's rows against its own LRv: the other agents' P
+            // columns of the fragment (its query rows, n = lane / 4) are zeroed
+            for (int al = 0; al < na; ++al) {
 #pragma unroll
-          for (int mr = 0; mr < C::MR; ++mr) {
-            uint32_t aV[4];
-            ldsm_x4_t(aV, sL + tile_off<2 * R, KT>(16 * ks + rr + (mi >> 1) * 8, R + 16 * mr + (mi & 1) * 8));
+              for (int mr = 0; mr < C::MR; ++mr) {
+                uint32_t aV[4];
+                ldsm_x4_t(aV, sL + al * C::LR_TILE +
+                                  tile_off<2 * R, KT>(16 * ks + rr + (mi >> 1) * 8, R + 16 * mr + (mi & 1) * 8));
 #pragma unroll
-            for (int pt = 0; pt < NT; ++pt) mma16816(Olr[mr][pt], aV, bP[pt][0], bP[pt][1]);
+                for (int pt = 0; pt < NT; ++pt) {
+                  const bool mine = (8 * pt + gq) / g == al;
+                  mma16816(Olr[mr][pt], aV, mine ? bP[pt][0] : 0u, mine ? bP[pt][1] : 0u);
+                }
+              }
+            }
+          } else {
+#pragma unroll
+            for (int mr = 0; mr < C::MR; ++mr) {
+              uint32_t aV[4];
+              ldsm_x4_t(aV, sL + tile_off<2 * R, KT>(16 * ks + rr + (mi >> 1) * 8, R + 16 * mr + (mi & 1) * 8));
+#pragma unroll
+              for (int pt = 0; pt < NT; ++pt) mma16816(Olr[mr][pt], aV, bP[pt][0], bP[pt][1]);
+            }
           }
         }
       }
@@ -1282,7 +1307,9 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
         }
         constexpr int LB = (2 * R) < 64 ? 2 * R : 64;
 #pragma unroll
-        for (int b = 0; b < (2 * R) / LB; ++b) tma_prefetch_l2_4d(&tmL, LB * b, key0, seq, lra);
+        for (int al = 0; al < (PA ? na : 1); ++al)
+          for (int b = 0; b < (2 * R) / LB; ++b)
+            tma_prefetch_l2_4d(&tmL, LB * b, key0, seq, PA ? agent0 + al : lra);
       };
       for (int m = ST; m < n_tiles && m < ST + kL2Ahead; ++m) prefetch(m);
       auto mma_pv = [&](int m) {  // O^T (d x query rows) += V_base^T P^T over the tile's keys
@@ -1319,9 +1346,10 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
         const uint64_t dL = umma_desc(sL, 16, 8 * C::LR_ROWB, C::LR_LAYOUT);
         for (int a = 0; a < na; ++a) {
           const uint64_t dB = umma_desc_add(dBk, a * align1k(C::BK_BYTES));
+          const uint64_t dLa = PA ? umma_desc_add(dL, a * C::LR_TILE) : dL;
 #pragma unroll
           for (int ks = 0; ks < C::KS; ++ks)
-            umma_bf16(tmem + 128 * a, umma_desc_add(dL, ks * 32), umma_desc_add(dB, ks * 16 * 128), ID_E, ks > 0);
+            umma_bf16(tmem + 128 * a, umma_desc_add(dLa, ks * 32), umma_desc_add(dB, ks * 16 * 128), ID_E, ks > 0);
         }
         umma_commit(tfull);
         if (n > 0) mma_pv(n - 1);
@@ -1673,6 +1701,12 @@ bool tc_fits(const AttnParams& p, int G) {
   const int NT = (G * p.g + 7) / 8;
   if (NT > 3) return false;
   size_t sm = 0;
+  if (p.lr_agent && G > 1) {   // per-agent LR tiles in every stage: r = 16 only
+    if (p.r != 16) return false;
+    sm = NT == 1 ? TCfg<128, 16, 1, true>::smem(G) : NT == 2 ? TCfg<128, 16, 2, true>::smem(G)
+                                                    : TCfg<128, 16, 3, true>::smem(G);
+    return sm <= 227 * 1024;
+  }
   switch (p.r) {
     case 16: sm = NT == 1 ? TCfg<128, 16, 1>::smem(G) : NT == 2 ? TCfg<128, 16, 2>::smem(G) : TCfg<128, 16, 3>::smem(G); break;
     case 32: sm = NT == 1 ? TCfg<128, 32, 1>::smem(G) : NT == 2 ? TCfg<128, 32, 2>::smem(G) : TCfg<128, 32, 3>::smem(G); break;
@@ -1689,9 +1723,9 @@ int tc_group_size(const AttnParams& p) {
   if (p.d != 128 || !(p.r == 16 || p.r == 32 || p.r == 64)) return 0;
   if (!(p.g == 1 || p.g == 2 || p.g == 4 || p.g == 8)) return 0;
   if (p.L_max >= (1ll << 31)) return 0;
-  // with one LR cache per agent a CTA holds one agent (its tiles are the
-  // agent's own LR rows beside the shared base tiles)
-  const int gmax = p.lr_agent ? 1 : 3;
+  // with one LR cache per agent every stage holds each agent's LR tile: up to
+  // three agents a CTA at r = 16 (shared memory), one at r = 32 and 64
+  const int gmax = p.lr_agent && p.r != 16 ? 1 : 3;
   for (int G = p.n_agents < gmax ? p.n_agents : gmax; G >= 1; --G)
     if (tc_fits(p, G)) return G;
   return 0;
@@ -1699,9 +1733,9 @@ int tc_group_size(const AttnParams& p) {
 
 bool tc_supported(const AttnParams& p) { return tc_group_size(p) > 0; }
 
-template <int D, int R, int NT>
+template <int D, int R, int NT, bool PA = false>
 cudaError_t launch_tc(const AttnParams& p, cudaStream_t st) {
-  using C = TCfg<D, R, NT>;
+  using C = TCfg<D, R, NT, PA>;
   RopeTheta rt;
   for (int i = 0; i < 64; ++i) {
     rt.theta[i] = i < D / 2 ? std::pow(p.rope_base, -2.0 * i / D) : 0.0;
@@ -1721,7 +1755,7 @@ cudaError_t launch_tc(const AttnParams& p, cudaStream_t st) {
       return cudaErrorInvalidValue;
   }
   const size_t sm = C::smem(p.agent_group);
-  auto kern = decode_tc_kernel<D, R, NT>;
+  auto kern = decode_tc_kernel<D, R, NT, PA>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
   dim3 grid(p.n_splits, (p.n_agents + p.agent_group - 1) / p.agent_group, p.n_seqs * p.n_kv);
@@ -1791,6 +1825,9 @@ cudaError_t launch_decode_bf16(const AttnParams& pin, la_dtype out, cudaStream_t
   p.agent_group = tc_group_size(p);
   if (p.agent_group > 0) {
     const int NT = (p.agent_group * p.g + 7) / 8;
+    if (p.lr_agent && p.agent_group > 1)   // r = 16 (tc_fits)
+      return NT == 1 ? launch_tc<128, 16, 1, true>(p, st) : NT == 2 ? launch_tc<128, 16, 2, true>(p, st)
+                                                         : launch_tc<128, 16, 3, true>(p, st);
     switch (p.r) {
       case 16: return NT == 1 ? launch_tc<128, 16, 1>(p, st) : NT == 2 ? launch_tc<128, 16, 2>(p, st) : launch_tc<128, 16, 3>(p, st);
       case 32: return NT == 1 ? launch_tc<128, 32, 1>(p, st) : NT == 2 ? launch_tc<128, 32, 2>(p, st) : launch_tc<128, 32, 3>(p, st);

@@ -453,14 +453,17 @@ def test_base_shared_prefill_tensor_cores(la, n_q, n_kv, L, n_tok, n_seqs, r, n_
     _prefill_vs_oracle(la, s, W.direct_cache_inputs(s))
 
 
-@pytest.mark.parametrize("kv_len,n_seqs,n_agents,r", [
-    (1500, 1, 3, 16),     # the 3-agent layer, one agent per CTA
-    (700, 2, 5, 32),      # the batched sweep's agents and rank, short
-    (300, 1, 4, 64),      # the stack's rank
+@pytest.mark.parametrize("kv_len,n_seqs,n_agents,r,n_kv", [
+    (1500, 1, 3, 16, 8),     # the 3-agent layer: 3 agents a CTA, each with its own LR tiles
+    (900, 1, 5, 16, 8),      # groups of 3 + 2 agents
+    (650, 2, 3, 16, 4),      # g = 8: 24 rows, three row tiles
+    (700, 2, 5, 32, 8),      # the batched sweep's agents and rank, short: one agent a CTA
+    (300, 1, 4, 64, 8),      # the stack's rank
 ])
-def test_base_shared_decode_tensor_cores(la, kv_len, n_seqs, n_agents, r):
+def test_base_shared_decode_tensor_cores(la, kv_len, n_seqs, n_agents, r, n_kv):
     s = W.LLAMA8B_DECODE_8K.replace(kv_len=kv_len, n_seqs=n_seqs, n_agents=n_agents, r=r,
-                                    alpha=2.0 * r, seed=700 + kv_len, lr_per_agent=True)
+                                    alpha=2.0 * r, seed=700 + kv_len, lr_per_agent=True,
+                                    n_kv_heads=n_kv)
     inp = W.direct_cache_inputs(s)
     dd = to_device(inp)
     got = _run(la, s, dd["k_base"], dd["v_base"], dd["lr"], dd["B_k"], dd["B_v"], dd["q"],
