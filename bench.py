@@ -408,7 +408,7 @@ class ClockSampler:
 # DRAM bytes per decode launch from an ncu capture of the workload, keyed by the
 # sha256 prefix of the decode kernel's source: reported only while the kernel is
 # unchanged since the counters were taken.
-DECODE_TRAFFIC = {"de1f4b62b2e1f47a": 34417664}
+DECODE_TRAFFIC = {"6e250726839f6d4a": 34417408}
 
 
 def decode_source_sha() -> str:
