@@ -408,14 +408,21 @@ class ClockSampler:
 # DRAM bytes per decode launch from an ncu capture of the workload, keyed by the
 # sha256 prefix of the decode kernel's source: reported only while the kernel is
 # unchanged since the counters were taken.
-DECODE_TRAFFIC = {"6e250726839f6d4a": 34417408}
+DECODE_TRAFFIC = {"87bbd0a7ac4ecf2f": 34417408}
 
 
 def decode_source_sha() -> str:
+    """sha256 prefix of the decode source's code: comments, blank lines and
+    trailing spaces removed, so that an edit of the comments keeps the key."""
     import hashlib
+    import re
     path = os.path.join(ROOT, "rank_attention_b200", "csrc", "attn_decode_bf16.cu")
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    with open(path) as f:
+        src = f.read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    code = "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
+    return hashlib.sha256(code.encode()).hexdigest()[:16]
 
 
 def decode_kernels_per_call(s) -> int:

@@ -6,12 +6,15 @@
 // group, split of the keys).  Its rows are the group's agents x the query
 // heads of the GQA group, so each base and LR tile is read from HBM once for
 // all of them (LRAgent summary §3 BaseLRShared: one base and one LR cache
-// shared by the whole system).  128-key tiles of K_base, V_base and the LR
-// rows are staged in shared memory by TMA (128/64/32-byte swizzle, no
-// multicast) through a two-stage full/empty mbarrier pipeline.
+// shared by the whole system; with one LR cache per agent -- BaseShared --
+// each stage holds every agent's own LR tile).  128-key tiles of K_base,
+// V_base and the LR rows are staged in shared memory by TMA (128/64/32-byte
+// swizzle, no multicast) through a two-stage full/empty mbarrier pipeline,
+// with a window of later tiles requested into L2.
 //  * Warp 10 issues the TMA loads and, per tile, the tcgen05 MMAs (M = 128
-//    keys): the base scores S_base^T = K_base Q^T for every row, and each
-//    agent's key delta dK^a = LRk B_k^a (N = d, K = r), all into TMEM.
+//    keys): the base scores S_base^T = K_base Q^T for every row and each
+//    agent's key delta dK^a = LRk B_k^a (N = d, K = r), into TMEM; then the
+//    previous tile's O_base^T += V_base^T P^T (M = d, N = the query rows).
 //  * 8 score warps, 16 keys each (LRAgent summary App. D.1: RoPE blocks the
 //    reordering, so the delta is rebuilt in head dimension).  A key at
 //    position t = k0 + j of a tile starting at k0 is rotated by
@@ -21,16 +24,18 @@
 //    R(j) -- whose cos / sin are per-thread constants, j being fixed per
 //    thread -- and scored (mma.sync) against the tile's rotated queries
 //    Q' = s R(-k0) Q.  The tile's row maxima meet in shared memory; the warps
-//    write P^T (bf16) and the rescale factors.
-//  * 2 value warps own O_base^T (half of d each) and O_lr^T: value side
-//    reordered (LRAgent explainer, Metodologia 3; summary App. B),
-//    O_base^T += V_base^T P^T and O_lr^T += LRv^T P^T, so the LoRA value path
-//    stays r wide inside the loop.  They also rotate the queries per tile.
+//    write P (bf16) and rescale O_base^T in TMEM when a row's maximum moved.
+//  * 2 value warps: the value side reordered (LRAgent explainer, Metodologia
+//    3; summary App. B) keeps the LoRA path r wide inside the loop, O_lr^T +=
+//    LRv^T P^T (mma.sync); they also rotate the next tile's queries and zero
+//    the rows of a tile past the sequence's end.
 //  Split keys merge inside the same launch: each CTA writes (O_base, O_lr, m,
 //  l), the unit's CTAs wait for one another (cooperative launch, bounded
 //  wait), and each merges a share of the unit's rows, applying B_v^a once per
 //  row: out = (sum_k w_k O_base,k + s (sum_k w_k O_lr,k) B_v^a) with
-//  w_k = 2^(m_k - M) / sum_k 2^(m_k - M) l_k.
+//  w_k = 2^(m_k - M) / sum_k 2^(m_k - M) l_k.  The launch is a programmatic
+//  dependent of the kernel before it (the step's LR append): the set-up runs
+//  while that kernel finishes, every input is read after griddepcontrol.wait.
 //
 // decode_bf16_kernel + decode_merge_kernel (shapes the first kernel does not
 // take: d = 64, r = 8).  The same tiling with mma.sync for every product and a
@@ -681,12 +686,12 @@ __global__ void __launch_bounds__(D) decode_merge_kernel(const AttnParams p) {
 // tcgen05 MMAs (M = 128 keys) whose operands are read from shared memory once
 // per CTA: the base scores S_base^T = K_base Q^T (N = the query rows, padded to
 // 16 / 32) and every agent's key delta dK^a = LRk B_k^a (N = d, K = r), all
-// accumulated in TMEM.  Eight score warps -- two per 32-lane TMEM
-// sub-partition, 16 keys each -- read dK^a straight into the mma.sync
-// accumulator layout (tcgen05.ld 16x256b), turn it by R(j), and score it
-// against the tile's rotated queries; the rest (softmax, value side, merge) is
-// as in the kernel above.  Warp 10 stages B_k and the tiles (TMA) and issues
-// the MMAs.
+// accumulated in TMEM, and O_base^T += V_base^T P^T.  Eight score warps --
+// two per 32-lane TMEM sub-partition, 16 keys each -- read dK^a straight into
+// the mma.sync accumulator layout (tcgen05.ld 16x256b), turn it by R(j), score
+// it against the tile's rotated queries and run the softmax; two value warps
+// keep the r-wide O_lr; warp 10 stages B_k and the tiles (TMA) and issues the
+// MMAs.
 // ============================================================================
 constexpr int TC_NES = 8;                          // score warps (16 keys each)
 constexpr int TC_NTHR = 32 * (TC_NES + NPV + 1);   // + value warps + TMA / MMA warp

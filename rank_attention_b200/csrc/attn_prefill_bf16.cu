@@ -24,6 +24,10 @@
 // refills.  The compute warps build tile n+1
 // before the softmax of tile n, so the S MMA of tile n+1 runs during that
 // softmax and the P V MMA of tile n during the next build.
+// Where whole CTAs would leave SMs idle, the launch runs each block as a
+// cluster of two CTAs over the two halves of its key tiles (template KS = 2),
+// merged over distributed shared memory.  With one LR cache per agent the LR
+// tiles are the CTA's agent's own (an agent coordinate of the LR tensor map).
 #include <cmath>
 
 #include <cuda_fp16.h>

@@ -22,6 +22,10 @@
 // Epilogue: out = (O_base + s O_lr B_v^a) / l, the single up-projection per
 // query block.  Decode splits the keys over CTAs; the last CTA of a unit to
 // arrive merges the (m, l, O_base, O_lr) partials and runs the epilogue.
+// With one LR cache per agent (BaseShared) every agent's LR tile is staged.
+// A second instance rebuilds V^a = V_base + s LRv B_v^a per tile instead of
+// step 4's rank-r partial (the naive reconstruction, measured against the
+// reordering).
 #include "la_internal.cuh"
 
 #include <math.h>
