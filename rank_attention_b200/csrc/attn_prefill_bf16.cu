@@ -116,7 +116,8 @@ __global__ void __launch_bounds__(PNTHR, 1)
   const int lra = p.lr_agent ? agent : 0;   // the agent's own LR cache, or the shared one
   const int g = p.g, na = p.n_agents;
   const int QB = PM / g;
-  const int tok0 = (int)(blockIdx.x / ksplit) * QB;
+  // the split launch covers the blocks from p.blk0 on (the whole-CTA launch from 0)
+  const int tok0 = ((KS > 1 ? p.blk0 : 0) + (int)(blockIdx.x / ksplit)) * QB;
   const int ntok = min(QB, p.n_q_tokens - tok0);
   const int64_t qmin = p.q_pos0 + tok0;               // position of the block's first token
   const int64_t kend = qmin + ntok;                    // keys [0, kend)
@@ -669,22 +670,25 @@ bool prefill_maps(const AttnParams& p, CUtensorMap* mq, CUtensorMap* mk, CUtenso
   return true;
 }
 
-// Key split: 1 (one CTA per block of rows) or 2 (a cluster of two CTAs per
-// block, each over half of the keys).  The CTAs of one wave run about equally
-// long, so the launch takes ceil(CTAs / resident CTAs) waves.  A half costs
-// more than half a CTA (its own start-up, pipeline fill and the merge: about
-// 15% measured at 65 tiles a half), so the split pays where the CTAs leave
-// SMs idle: fewer CTAs than SMs, or a last wave that is mostly empty.
+// Which blocks of rows run as whole CTAs and which as key halves on CTA pairs
+// (KS = 2): the first nA blocks whole, the rest split, in two launches.  The
+// CTAs of one wave run about equally long, so a launch takes ceil(CTAs /
+// resident CTAs) waves; a half costs more than half a CTA (its own start-up,
+// pipeline fill and the merge: about 15 % measured at 65 tiles a half).  The
+// split pays where whole CTAs would leave SMs idle -- fewer CTAs than SMs, or
+// a last wave that is mostly empty (768 CTAs on 148 SMs: 720 whole in 5 waves,
+// the last two blocks' 48 as 96 halves in one half-length wave, instead of
+// 6 waves).  Returns nA in [0, nblk].
 template <int R>
-int prefill_ksplit(const AttnParams& p, int nblk) {
+int prefill_whole_blocks(const AttnParams& p, int nblk) {
   using C = PCfg<R>;
   const int64_t tiles = (p.q_pos0 + p.n_q_tokens + PKT - 1) / PKT;
-  if (tiles < 4) return 1;
+  if (tiles < 4) return nblk;
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) {
     cudaGetLastError();
-    return 1;
+    return nblk;
   }
   static int pairs[64] = {};   // resident CTA pairs per device (0: not queried yet)
   int& np = pairs[dev & 63];
@@ -709,11 +713,18 @@ int prefill_ksplit(const AttnParams& p, int nblk) {
     }
     np = n;
   }
-  if (np < 1) return 1;
-  const double ctas = (double)nblk * p.n_agents * p.n_kv * p.n_seqs;
-  const double t1 = std::ceil(ctas / sms);              // waves of whole CTAs
-  const double t2 = 0.5 * std::ceil(ctas / np) * 1.15;  // half-length waves, + their overhead
-  return t2 < t1 ? 2 : 1;
+  if (np < 1) return nblk;
+  const double per_blk = (double)p.n_agents * p.n_kv * p.n_seqs;   // CTAs (or pairs) per block
+  int best = nblk;
+  double best_t = std::ceil(nblk * per_blk / sms);
+  for (int na = nblk - 1; na >= 0; --na) {
+    const double t = std::ceil(na * per_blk / sms) + 0.5 * 1.15 * std::ceil((nblk - na) * per_blk / np);
+    if (t < best_t - 1e-9) {
+      best_t = t;
+      best = na;
+    }
+  }
+  return best;
 }
 
 template <int R>
@@ -728,24 +739,31 @@ cudaError_t launch_prefill_tc(const AttnParams& p, cudaStream_t st) {
   if (!prefill_maps(p, &mq, &mk, &mv, &ml, &mb)) return cudaErrorInvalidValue;
   const int QB = PM / p.g;
   const int nblk = (p.n_q_tokens + QB - 1) / QB;
-  const int ks = prefill_ksplit<R>(p, nblk);
-  auto kern = ks > 1 ? prefill_tc_kernel<R, 2> : prefill_tc_kernel<R, 1>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
-  if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(nblk * ks), p.n_agents * p.n_kv, p.n_seqs);
-  cfg.blockDim = dim3(PNTHR);
-  cfg.dynamicSmemBytes = C::SMEM;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)ks;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = ks > 1 ? 1 : 0;
-  e = cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, ml, mb, p, rt);
-  if (e != cudaSuccess) return e;
+  const int nA = prefill_whole_blocks<R>(p, nblk);
+  // blocks [0, nA) as whole CTAs, blocks [nA, nblk) as key halves on CTA pairs
+  for (int ks = 1; ks <= 2; ++ks) {
+    const int nb = ks == 1 ? nA : nblk - nA;
+    if (nb == 0) continue;
+    auto kern = ks > 1 ? prefill_tc_kernel<R, 2> : prefill_tc_kernel<R, 1>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
+    if (e != cudaSuccess) return e;
+    AttnParams pk = p;
+    pk.blk0 = ks > 1 ? nA : 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(nb * ks), p.n_agents * p.n_kv, p.n_seqs);
+    cfg.blockDim = dim3(PNTHR);
+    cfg.dynamicSmemBytes = C::SMEM;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)ks;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = ks > 1 ? 1 : 0;
+    e = cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, ml, mb, pk, rt);
+    if (e != cudaSuccess) return e;
+  }
   return cudaGetLastError();
 }
 

@@ -44,6 +44,7 @@ struct AttnParams {
   int out_bf16;            // tensor-core kernels: 1 = bf16 outputs, 0 = fp32
   int agent_group;         // tensor-core decode: agents per CTA (grid z runs over the groups)
   int value_path;          // la_value_path: 0 fastest reordered, 1 generic reordered, 2 per tile
+  int blk0;                // tensor-core prefill, split launch: the first block of rows it covers
 };
 
 // Device error word of the library (address on the current device).

@@ -295,6 +295,7 @@ def _prefill_vs_oracle(la, s, inp, out_dtype=None):
     (16, 8, 129, 64, 1, 16),      # g = 2, one key past a tile
     (32, 8, 100, 1, 1, 16),       # one query token, one partial tile
     (4, 1, 512, 512, 1, 16),      # few CTAs: key halves on CTA pairs; blocks of one tile leave half 1 empty
+    (32, 8, 600, 224, 1, 16),     # 168 CTAs: 6 blocks whole, the last one as key halves (two launches)
 ])
 def test_bf16_prefill_tensor_core_shapes(la, n_q, n_kv, L, n_tok, n_seqs, r):
     """The tcgen05 prefill (r = 16, 32, 64): GQA groups 1..8, blocks cut by the
