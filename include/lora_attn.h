@@ -316,9 +316,24 @@ la_status lora_attn_decode_static_scratch(const la_attn_args* args, la_stream_t 
 /*
  * la_device_check -- synchronises the current device, then reads and clears
  * the library's device error word.  Returns LA_OK, LA_ERR_DEVICE_CHECK if a
- * kernel's bounds check fired since the last call, or LA_ERR_CUDA.
+ * kernel's own check fired since the last call, or LA_ERR_CUDA.
+ *
+ * la_device_check_word -- the same, and writes the word's bits to *word
+ * (host pointer; 0 when nothing fired):
+ *   LA_DEV_KV_LEN     a decode kv_len[q] outside [1, max_kv_len]
+ *   LA_DEV_PIPE_WAIT  a tensor-core kernel's wait on its copy/MMA pipeline
+ *                     gave up after its iteration limit (the CTA skipped its
+ *                     output and, holding TMEM, freed it)
+ *   LA_DEV_MERGE_WAIT a decode CTA's wait for the other splits of its unit
+ *                     gave up after its iteration limit (about a second);
+ *                     that unit's output is not to be trusted
+ * No check traps: every kernel returns and the context stays usable.
  */
+#define LA_DEV_KV_LEN 1
+#define LA_DEV_PIPE_WAIT 2
+#define LA_DEV_MERGE_WAIT 4
 la_status la_device_check(void);
+la_status la_device_check_word(int32_t* word);
 
 #ifdef __cplusplus
 }

@@ -332,7 +332,8 @@ extern "C" la_status lora_materialize_agent_kv(const la_attn_args* a, void* k_ou
   return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
 }
 
-extern "C" la_status la_device_check(void) {
+extern "C" la_status la_device_check_word(int32_t* word) {
+  if (word) *word = 0;
   if (cudaDeviceSynchronize() != cudaSuccess) return LA_ERR_CUDA;
   int* ptr = error_word_ptr();
   if (!ptr) return LA_ERR_CUDA;
@@ -342,7 +343,10 @@ extern "C" la_status la_device_check(void) {
     const int zero = 0;
     if (cudaMemcpy(ptr, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
       return LA_ERR_CUDA;
+    if (word) *word = v;
     return LA_ERR_DEVICE_CHECK;
   }
   return LA_OK;
 }
+
+extern "C" la_status la_device_check(void) { return la_device_check_word(nullptr); }

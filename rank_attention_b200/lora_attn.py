@@ -23,11 +23,13 @@ LA_ERR_WORKSPACE, LA_ERR_CUDA, LA_ERR_DEVICE_CHECK, LA_ERR_SCRATCH_LIMIT = 4, 5,
 LA_STATIC_SCRATCH_BYTES = 4 << 20
 LA_F32, LA_BF16 = 0, 1
 LA_VALUE_REORDERED, LA_VALUE_REORDERED_GENERIC, LA_VALUE_PER_TILE = 0, 1, 2
+LA_DEV_KV_LEN, LA_DEV_PIPE_WAIT, LA_DEV_MERGE_WAIT = 1, 2, 4
 
 EXPORTED = ("la_status_string", "lr_cache_append", "lora_attn_prefill", "lora_attn_decode",
             "lora_attn_decode_workspace_bytes", "la_device_check",
             "lora_attn_decode_static_scratch", "lora_materialize_agent_kv",
-            "lr_cache_append_agents", "lora_query_expand", "lora_output_delta")
+            "lr_cache_append_agents", "lora_query_expand", "lora_output_delta",
+            "la_device_check_word")
 
 
 class LoraAttnError(RuntimeError):
@@ -98,6 +100,8 @@ def _load() -> ctypes.CDLL:
     lib.lora_attn_decode_workspace_bytes.argtypes = [ctypes.POINTER(AttnArgs)]
     lib.la_device_check.restype = ctypes.c_int
     lib.la_device_check.argtypes = []
+    lib.la_device_check_word.restype = ctypes.c_int
+    lib.la_device_check_word.argtypes = [ctypes.POINTER(ctypes.c_int32)]
     lib.lora_attn_decode_static_scratch.restype = ctypes.c_int
     lib.lora_attn_decode_static_scratch.argtypes = [ctypes.POINTER(AttnArgs), ctypes.c_void_p]
     lib.lora_materialize_agent_kv.restype = ctypes.c_int
@@ -284,6 +288,13 @@ def lora_attn_prefill(args: AttnArgs, stream=None) -> None:
 
 def la_device_check() -> int:
     return int(lib.la_device_check())
+
+
+def la_device_check_word() -> tuple:
+    """(status, bits of the device error word that fired); reads and clears it."""
+    w = ctypes.c_int32(0)
+    st = int(lib.la_device_check_word(ctypes.byref(w)))
+    return st, int(w.value)
 
 
 class DecodeStep:

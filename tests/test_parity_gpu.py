@@ -255,6 +255,34 @@ def test_decode_kv_len_beyond_bound_is_reported(la):
     assert_parity(to_np(out[0]), ref[0], s.dtype)
 
 
+def test_decode_merge_wait_runs_out_and_is_reported(la):
+    """The in-launch split merge waits, bounded, for every split of its unit to
+    arrive.  A workspace whose arrival counters start at -1 (all bytes 0xFF)
+    never reaches the split count: every CTA's wait gives up after its
+    iteration limit, the launch still ends, the merge-wait bit of the device
+    error word is set, and the same context then computes a correct decode on
+    a zeroed workspace."""
+    s = W.LLAMA8B_DECODE_8K.replace(kv_len=4096, n_seqs=1, seed=29)
+    inp = W.direct_cache_inputs(s)
+    dd = to_device(inp)
+    out = torch.zeros(dd["q"].shape, device=DEV)
+    args = la.make_args(dd["k_base"], dd["v_base"], dd["lr"], dd["B_k"], dd["B_v"], dd["q"], out,
+                        lora_scale=s.lora_scale, rope_base=s.rope_base, kv_len=dd["kv_len"],
+                        max_kv_len=s.kv_len)
+    ws = la.decode_workspace(args, DEV)
+    assert la.la_device_check() == 0
+    ws.fill_(0xFF)
+    la.lora_attn_decode(args, ws)
+    st, word = la.la_device_check_word()
+    assert st == la.LA_ERR_DEVICE_CHECK
+    assert word == la.LA_DEV_MERGE_WAIT
+    assert la.la_device_check_word() == (0, 0)
+    ws.zero_()
+    la.lora_attn_decode(args, ws)
+    assert la.la_device_check_word() == (0, 0)
+    assert_parity(to_np(out), oracle_decode(inp, s), s.dtype)
+
+
 # ---------------------------------------------------------- bf16 prefill ----
 @pytest.mark.parametrize("L,n_tok,r,n_agents", [
     (300, 77, 16, 3),
