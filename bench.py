@@ -680,8 +680,9 @@ def run_ours(args):
 
     value = whole_job_rate(s.n_seqs * s.n_agents, args.steps, world, ms)
 
-    # end to end through the public API with host buffers: H2D of the step's
-    # inputs (new hidden row, queries, lengths), the two calls, D2H of outputs
+    # end to end through the public API with host buffers: lora_decode_step_host
+    # copies the step's inputs in (new hidden row, queries, lengths), appends,
+    # decodes and copies the outputs back
     h_x = [x.cpu().pin_memory() for (_, x, _) in sets]
     h_q = [i["q"].cpu().pin_memory() for (i, _, _) in sets]
     h_len = [i["kv_len"].cpu().pin_memory() for (i, _, _) in sets]
@@ -690,14 +691,9 @@ def run_ours(args):
     d2h = h_out[0].numel() * 4
     e_steps = min(args.steps, 100)
 
-    def e2e_step(k):
+    def e2e_step(k):  # one library call: copies in, append, decode, copy out
         i = k % n_sets
-        inp, x, out = sets[i]
-        x.copy_(h_x[i], non_blocking=True)
-        inp["q"].copy_(h_q[i], non_blocking=True)
-        inp["kv_len"].copy_(h_len[i], non_blocking=True)
-        steps_fn[i]()
-        h_out[i].copy_(out, non_blocking=True)
+        steps_fn[i].from_host(h_x[i], h_q[i], h_len[i], h_out[i], stream)
 
     with torch.cuda.stream(stream):
         for k in range(3):

@@ -186,6 +186,43 @@ typedef struct {
 } la_attn_args;
 
 /*
+ * lora_decode_step_host -- one whole decode step with the step's inputs and
+ * outputs in HOST memory, as a serving loop runs it.  Queued on `stream`, in
+ * this order, with nothing synchronised:
+ *   1. copies x_host -> x_dev, q_host -> args->q, kv_len_host -> args->kv_len;
+ *   2. appends the new token's LR row of every sequence q at position
+ *      kv_len_host[q] - 1 (lr_cache_append; with args->lr_agent_stride > 0,
+ *      one row per agent into that agent's own cache, X A_a, as
+ *      lr_cache_append_agents);
+ *   3. lora_attn_decode(args, workspace, ...);
+ *   4. copies args->out -> out_host.
+ * out_host holds the step's outputs once the stream has been synchronised.
+ * Pinned (page-locked) host buffers make the copies asynchronous; pageable
+ * ones are still correct, with the copies staged by the CUDA runtime.
+ *
+ *   args        as lora_attn_decode; args->q, args->kv_len and args->lr_cache
+ *               are device buffers this call writes (the copies and the
+ *               append), args->out the device buffer it copies back.
+ *   A_kv        device, [hidden][2r] (shared A) or [n_agents][hidden][2r]
+ *               (args->lr_agent_stride > 0), io dtype.
+ *   x_dev       device staging of n_seqs * hidden elements (io dtype), 16-byte
+ *               aligned; hidden * element size a multiple of 16 bytes.
+ *   x_host      host [n_seqs][hidden]: the new token's hidden row per sequence.
+ *   q_host      host [n_seqs][n_agents][1][n_q_heads][d], io dtype.
+ *   kv_len_host host int32 [n_seqs], each in [1, max_kv_len] (read by this
+ *               call on the host and copied to args->kv_len).
+ *   out_host    host [n_seqs][n_agents][1][n_q_heads][d], out dtype.
+ * Errors, all before anything is queued: those of lora_attn_decode and
+ * lr_cache_append, and LA_ERR_INVALID_ARG for a null host or staging pointer
+ * or a kv_len_host[q] outside [1, max_kv_len].  LA_ERR_CUDA if a copy or a
+ * launch fails to queue (the steps before it may have been queued).
+ */
+la_status lora_decode_step_host(const la_attn_args* args, void* workspace,
+                                size_t workspace_bytes, const void* A_kv, int64_t hidden,
+                                void* x_dev, const void* x_host, const void* q_host,
+                                const int32_t* kv_len_host, void* out_host, la_stream_t stream);
+
+/*
  * lora_attn_prefill -- causal Flash-LoRA-Attention for a chunk of n_q_tokens
  * query tokens per (sequence, agent) over prefix + chunk.
  * Errors: LA_ERR_INVALID_ARG, LA_ERR_UNSUPPORTED, LA_ERR_CAPACITY

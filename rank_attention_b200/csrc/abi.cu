@@ -166,15 +166,21 @@ extern "C" const char* la_status_string(la_status s) {
   return "unknown la_status";
 }
 
-extern "C" la_status lr_cache_append(const void* X, int64_t ldx, int64_t n_tokens, int64_t hidden,
-                                     const void* A_kv, int32_t r, void* lr_cache, int64_t L_max,
-                                     int64_t pos0, int32_t n_seqs, int64_t seq_stride_x,
-                                     int64_t seq_stride_lr, la_dtype dt, la_stream_t stream) {
+namespace {
+// The checks of lr_cache_append; *empty: valid, but nothing to read or write.
+la_status append_check(const void* X, int64_t ldx, int64_t n_tokens, int64_t hidden,
+                       const void* A_kv, int32_t r, const void* lr_cache, int64_t L_max,
+                       int64_t pos0, int32_t n_seqs, int64_t seq_stride_x, int64_t seq_stride_lr,
+                       la_dtype dt, bool* empty) {
+  *empty = false;
   if (!dtype_ok(dt)) return LA_ERR_INVALID_ARG;
   if (n_tokens < 0 || n_seqs < 0 || hidden < 1 || L_max < 1) return LA_ERR_INVALID_ARG;
   if (!rank_ok(r)) return LA_ERR_UNSUPPORTED;
   if (pos0 < 0 || pos0 + n_tokens > L_max) return LA_ERR_CAPACITY;
-  if (n_tokens == 0 || n_seqs == 0) return LA_OK;  // nothing is read or written
+  if (n_tokens == 0 || n_seqs == 0) {  // nothing is read or written
+    *empty = true;
+    return LA_OK;
+  }
   if (!X || !A_kv || !lr_cache) return LA_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(A_kv) || !aligned16(lr_cache)) return LA_ERR_INVALID_ARG;
   if (ldx < hidden || !stride_ok(ldx, dt)) return LA_ERR_INVALID_ARG;
@@ -183,7 +189,14 @@ extern "C" la_status lr_cache_append(const void* X, int64_t ldx, int64_t n_token
   if (n_seqs > 1 && seq_stride_lr < L_max * 2 * r) return LA_ERR_INVALID_ARG;
   if ((hidden * (int64_t)esize(dt)) % 16 != 0) return LA_ERR_INVALID_ARG;
   if (n_seqs > 65535) return LA_ERR_UNSUPPORTED;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return LA_OK;
+}
+
+// lr_cache_append's launch, after append_check passed with *empty false.
+la_status append_launch(const void* X, int64_t ldx, int64_t n_tokens, int64_t hidden,
+                        const void* A_kv, int32_t r, void* lr_cache, int64_t pos0,
+                        int32_t n_seqs, int64_t seq_stride_x, int64_t seq_stride_lr, la_dtype dt,
+                        cudaStream_t st) {
   cudaError_t e;
   if (dt == LA_BF16 && bf16_append_supported(hidden, r))
     e = launch_append_bf16_mma(X, ldx, n_tokens, hidden, A_kv, r, lr_cache, pos0, n_seqs,
@@ -192,6 +205,19 @@ extern "C" la_status lr_cache_append(const void* X, int64_t ldx, int64_t n_token
     e = launch_append_simt(X, ldx, n_tokens, hidden, A_kv, r, lr_cache, pos0, n_seqs,
                            seq_stride_x, seq_stride_lr, dt, st);
   return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+}  // namespace
+
+extern "C" la_status lr_cache_append(const void* X, int64_t ldx, int64_t n_tokens, int64_t hidden,
+                                     const void* A_kv, int32_t r, void* lr_cache, int64_t L_max,
+                                     int64_t pos0, int32_t n_seqs, int64_t seq_stride_x,
+                                     int64_t seq_stride_lr, la_dtype dt, la_stream_t stream) {
+  bool empty = false;
+  const la_status s = append_check(X, ldx, n_tokens, hidden, A_kv, r, lr_cache, L_max, pos0,
+                                   n_seqs, seq_stride_x, seq_stride_lr, dt, &empty);
+  if (s != LA_OK || empty) return s;
+  return append_launch(X, ldx, n_tokens, hidden, A_kv, r, lr_cache, pos0, n_seqs, seq_stride_x,
+                       seq_stride_lr, dt, static_cast<cudaStream_t>(stream));
 }
 
 extern "C" la_status lr_cache_append_agents(const void* X, int64_t ldx, int64_t n_tokens,
@@ -280,28 +306,109 @@ extern "C" size_t lora_attn_decode_workspace_bytes(const la_attn_args* a) {
   return d.partial_bytes + d.counter_bytes;
 }
 
-extern "C" la_status lora_attn_decode(const la_attn_args* a, void* workspace,
-                                      size_t workspace_bytes, la_stream_t stream) {
-  AttnParams p;
-  la_status s = check_attn(a, 1, &p);
+namespace {
+// The checks and the plan of lora_attn_decode.  On LA_OK with *empty false,
+// *p is ready to launch as *kind (1: tensor-core decode, 0: generic kernel).
+la_status decode_prepare(const la_attn_args* a, void* workspace, size_t workspace_bytes,
+                         AttnParams* p, int* kind, bool* empty) {
+  *empty = false;
+  la_status s = check_attn(a, 1, p);
   if (s != LA_OK) return s;
-  DecodePlan d = plan_decode(p, a->io_dtype);
+  DecodePlan d = plan_decode(*p, a->io_dtype);
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
       workspace_bytes < d.partial_bytes + d.counter_bytes)
     return LA_ERR_WORKSPACE;
-  if (p.n_seqs == 0) return LA_OK;
-  if ((int64_t)p.n_seqs * p.n_kv > 65535) return LA_ERR_UNSUPPORTED;
-  if (d.kind == 0 && simt_smem_bytes(p) > 227 * 1024) return LA_ERR_UNSUPPORTED;
-  p.n_splits = d.n_splits;
-  p.split_len = d.split_len;
-  p.partials = static_cast<float*>(workspace);
-  p.counters = reinterpret_cast<int*>(static_cast<char*>(workspace) + d.partial_bytes);
+  if (p->n_seqs == 0) {
+    *empty = true;
+    return LA_OK;
+  }
+  if ((int64_t)p->n_seqs * p->n_kv > 65535) return LA_ERR_UNSUPPORTED;
+  if (d.kind == 0 && simt_smem_bytes(*p) > 227 * 1024) return LA_ERR_UNSUPPORTED;
+  p->n_splits = d.n_splits;
+  p->split_len = d.split_len;
+  p->partials = static_cast<float*>(workspace);
+  p->counters = reinterpret_cast<int*>(static_cast<char*>(workspace) + d.partial_bytes);
+  *kind = d.kind;
+  return LA_OK;
+}
+
+la_status decode_launch(AttnParams& p, int kind, const la_attn_args* a, cudaStream_t st) {
   p.err = error_word_ptr();
   if (!p.err) return LA_ERR_CUDA;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = d.kind == 1 ? launch_decode_bf16(p, a->out_dtype, st)
-                              : launch_attn_simt(p, a->io_dtype, a->out_dtype, st);
+  cudaError_t e = kind == 1 ? launch_decode_bf16(p, a->out_dtype, st)
+                            : launch_attn_simt(p, a->io_dtype, a->out_dtype, st);
   return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
+}
+}  // namespace
+
+extern "C" la_status lora_attn_decode(const la_attn_args* a, void* workspace,
+                                      size_t workspace_bytes, la_stream_t stream) {
+  AttnParams p;
+  int kind = 0;
+  bool empty = false;
+  const la_status s = decode_prepare(a, workspace, workspace_bytes, &p, &kind, &empty);
+  if (s != LA_OK || empty) return s;
+  return decode_launch(p, kind, a, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" la_status lora_decode_step_host(const la_attn_args* a, void* workspace,
+                                           size_t workspace_bytes, const void* A_kv,
+                                           int64_t hidden, void* x_dev, const void* x_host,
+                                           const void* q_host, const int32_t* kv_len_host,
+                                           void* out_host, la_stream_t stream) {
+  AttnParams p;
+  int kind = 0;
+  bool empty = false;
+  la_status s = decode_prepare(a, workspace, workspace_bytes, &p, &kind, &empty);
+  if (s != LA_OK || empty) return s;
+  if (!x_dev || !x_host || !q_host || !kv_len_host || !out_host || !a->lr_cache)
+    return LA_ERR_INVALID_ARG;
+  const la_dtype dt = a->io_dtype;
+  const int32_t n_seqs = a->n_seqs;
+  // the new token of sequence q sits at position kv_len_host[q] - 1
+  bool same_pos = true;
+  for (int32_t q = 0; q < n_seqs; ++q) {
+    if (kv_len_host[q] < 1 || kv_len_host[q] > a->max_kv_len) return LA_ERR_INVALID_ARG;
+    same_pos = same_pos && kv_len_host[q] == kv_len_host[0];
+  }
+  // every append below has the shapes, strides and alignment this check sees
+  s = append_check(x_dev, hidden, 1, hidden, A_kv, a->r, a->lr_cache, a->L_max,
+                   kv_len_host[0] - 1, n_seqs, hidden, a->lr_seq_stride, dt, &empty);
+  if (s != LA_OK) return s;
+  const size_t es = esize(dt), eo = esize(a->out_dtype);
+  const size_t x_bytes = (size_t)n_seqs * hidden * es;
+  const size_t q_elems = (size_t)n_seqs * a->n_agents * a->n_q_heads * a->head_dim;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(x_dev, x_host, x_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+      cudaMemcpyAsync(const_cast<void*>(a->q), q_host, q_elems * es, cudaMemcpyHostToDevice,
+                      st) != cudaSuccess ||
+      cudaMemcpyAsync(const_cast<int32_t*>(a->kv_len), kv_len_host, (size_t)n_seqs * 4,
+                      cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return LA_ERR_CUDA;
+  // the new rows: into the shared LR cache, or into every agent's own (X A_a)
+  const int n_lr = a->lr_agent_stride > 0 ? a->n_agents : 1;
+  const size_t a_bytes = (size_t)hidden * 2 * a->r * es;
+  for (int l = 0; l < n_lr; ++l) {
+    const char* A_l = static_cast<const char*>(A_kv) + l * a_bytes;
+    char* lr_l = static_cast<char*>(const_cast<void*>(a->lr_cache)) + (size_t)l * a->lr_agent_stride * es;
+    if (same_pos) {
+      s = append_launch(x_dev, hidden, 1, hidden, A_l, a->r, lr_l, kv_len_host[0] - 1, n_seqs,
+                        hidden, a->lr_seq_stride, dt, st);
+      if (s != LA_OK) return s;
+    } else {
+      for (int32_t q = 0; q < n_seqs; ++q) {
+        s = append_launch(static_cast<const char*>(x_dev) + (size_t)q * hidden * es, hidden, 1,
+                          hidden, A_l, a->r, lr_l + (size_t)q * a->lr_seq_stride * es,
+                          kv_len_host[q] - 1, 1, hidden, a->lr_seq_stride, dt, st);
+        if (s != LA_OK) return s;
+      }
+    }
+  }
+  s = decode_launch(p, kind, a, st);
+  if (s != LA_OK) return s;
+  if (cudaMemcpyAsync(out_host, a->out, q_elems * eo, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return LA_ERR_CUDA;
+  return LA_OK;
 }
 
 extern "C" la_status lora_attn_prefill(const la_attn_args* a, la_stream_t stream) {

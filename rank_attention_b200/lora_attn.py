@@ -29,7 +29,7 @@ EXPORTED = ("la_status_string", "lr_cache_append", "lora_attn_prefill", "lora_at
             "lora_attn_decode_workspace_bytes", "la_device_check",
             "lora_attn_decode_static_scratch", "lora_materialize_agent_kv",
             "lr_cache_append_agents", "lora_query_expand", "lora_output_delta",
-            "la_device_check_word")
+            "la_device_check_word", "lora_decode_step_host")
 
 
 class LoraAttnError(RuntimeError):
@@ -101,6 +101,11 @@ def _load() -> ctypes.CDLL:
     lib.la_device_check.restype = ctypes.c_int
     lib.la_device_check.argtypes = []
     lib.la_device_check_word.restype = ctypes.c_int
+    lib.lora_decode_step_host.restype = ctypes.c_int
+    lib.lora_decode_step_host.argtypes = [
+        ctypes.POINTER(AttnArgs), ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p,
+        ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+        ctypes.c_void_p, ctypes.c_void_p]
     lib.la_device_check_word.argtypes = [ctypes.POINTER(ctypes.c_int32)]
     lib.lora_attn_decode_static_scratch.restype = ctypes.c_int
     lib.lora_attn_decode_static_scratch.argtypes = [ctypes.POINTER(AttnArgs), ctypes.c_void_p]
@@ -264,6 +269,23 @@ def lora_attn_decode(args: AttnArgs, workspace: torch.Tensor, stream=None) -> No
     _check(st, "lora_attn_decode")
 
 
+def lora_decode_step_host(args: AttnArgs, workspace: torch.Tensor, A_kv: torch.Tensor,
+                          x_dev: torch.Tensor, x_host: torch.Tensor, q_host: torch.Tensor,
+                          kv_len_host: torch.Tensor, out_host: torch.Tensor, stream=None) -> None:
+    """One decode step from host buffers (copies in, LR append, decode, copy
+    out), queued on the stream by one library call.  x_dev is the device
+    staging [n_seqs, hidden]; the host tensors are CPU tensors, pinned for
+    asynchronous copies."""
+    for t in (x_host, q_host, kv_len_host, out_host):
+        assert t.device.type == "cpu" and t.is_contiguous()
+    assert x_dev.is_contiguous() and kv_len_host.dtype == torch.int32
+    st = lib.lora_decode_step_host(ctypes.byref(args), workspace.data_ptr(), workspace.numel(),
+                                   A_kv.data_ptr(), x_dev.shape[-1], x_dev.data_ptr(),
+                                   x_host.data_ptr(), q_host.data_ptr(), kv_len_host.data_ptr(),
+                                   out_host.data_ptr(), _stream(stream))
+    _check(st, "lora_decode_step_host")
+
+
 def lora_attn_decode_static_scratch(args: AttnArgs, stream=None) -> None:
     """Decode without a workspace: the split scratch is the library's own device
     array (for callers that cannot allocate device memory; see the header)."""
@@ -316,3 +338,10 @@ class DecodeStep:
         if self.x_new is not None:
             lr_cache_append(self.x_new, self.A_kv, self.lr, self.pos_new, stream)
         lora_attn_decode(self.args, self.workspace, stream)
+
+    def from_host(self, x_host, q_host, kv_len_host, out_host, stream=None) -> None:
+        """The same step with its inputs and outputs in host memory: one call
+        that copies them in and out around the append and the decode; the new
+        rows land at kv_len_host - 1."""
+        lora_decode_step_host(self.args, self.workspace, self.A_kv, self.x_new, x_host, q_host,
+                              kv_len_host, out_host, stream)

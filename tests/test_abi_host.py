@@ -243,3 +243,38 @@ def test_null_args():
     assert la.lib.lora_attn_prefill(None, None) == la.LA_ERR_INVALID_ARG
     assert la.lib.lora_attn_decode(None, FAKE, 1 << 20, None) == la.LA_ERR_INVALID_ARG
     assert la.lib.lora_attn_decode_workspace_bytes(None) == 0
+    assert la.lib.lora_decode_step_host(None, FAKE, 1 << 20, FAKE, 64, FAKE, FAKE, FAKE, FAKE,
+                                        FAKE, None) == la.LA_ERR_INVALID_ARG
+
+
+def _step(a=None, ws_bytes=1 << 20, A_kv=FAKE, hidden=64, x_dev=FAKE, x_host=FAKE, q_host=FAKE,
+          kv_len=(5,), out_host=FAKE):
+    a = a if a is not None else _args()
+    kv = (ctypes.c_int32 * len(kv_len))(*kv_len) if kv_len is not None else None
+    return la.lib.lora_decode_step_host(ctypes.byref(a), FAKE, ws_bytes, A_kv, hidden, x_dev,
+                                        x_host, q_host, kv, out_host, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(kv_len=(0,)), la.LA_ERR_INVALID_ARG),        # no key: the new token has no row
+    (dict(kv_len=(257,)), la.LA_ERR_INVALID_ARG),      # above max_kv_len
+    (dict(kv_len=None), la.LA_ERR_INVALID_ARG),
+    (dict(x_host=0), la.LA_ERR_INVALID_ARG),
+    (dict(q_host=0), la.LA_ERR_INVALID_ARG),
+    (dict(out_host=0), la.LA_ERR_INVALID_ARG),
+    (dict(x_dev=0), la.LA_ERR_INVALID_ARG),
+    (dict(x_dev=FAKE + 8), la.LA_ERR_INVALID_ARG),     # staging not 16-byte aligned
+    (dict(A_kv=0), la.LA_ERR_INVALID_ARG),
+    (dict(hidden=0), la.LA_ERR_INVALID_ARG),
+    (dict(hidden=6), la.LA_ERR_INVALID_ARG),           # 24-byte rows
+    (dict(ws_bytes=16), la.LA_ERR_WORKSPACE),
+] + [(dict(a=_args(**kw)), st) for kw, st in BAD_ATTN])
+def test_decode_step_host_rejects(kw, status):
+    """Every check of the host-buffer step runs before anything is queued."""
+    assert _step(**kw) == status
+
+
+def test_decode_step_host_second_sequence_checked():
+    # the second sequence's length is checked too, before any copy
+    a = _args(n_seqs=2)
+    assert _step(a=a, kv_len=(5, 300)) == la.LA_ERR_INVALID_ARG

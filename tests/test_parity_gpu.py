@@ -283,6 +283,60 @@ def test_decode_merge_wait_runs_out_and_is_reported(la):
     assert_parity(to_np(out), oracle_decode(inp, s), s.dtype)
 
 
+@pytest.mark.parametrize("kv_lens,per_agent", [
+    ((8192,), False),           # the LLaMA-8B decode step: one sequence, shared A
+    ((700, 650, 700), False),   # unequal lengths: one append per sequence
+    ((640, 640), True),         # BaseShared: every agent's own A_a and LR cache
+])
+def test_decode_step_from_host_equals_device_step(la, kv_lens, per_agent):
+    """lora_decode_step_host (copies in, append at kv_len - 1, decode, copy out)
+    gives the same LR rows and outputs, bit for bit, as the same step on
+    device buffers (the append then the decode), and the outputs match the
+    oracle over the updated caches."""
+    n_seqs, L_max = len(kv_lens), max(kv_lens)
+    s = W.LLAMA8B_DECODE_8K.replace(kv_len=L_max, n_seqs=n_seqs, seed=37, lr_per_agent=per_agent)
+    inp = W.direct_cache_inputs(s, L_max=L_max)
+    inp["kv_len"] = torch.tensor(kv_lens, dtype=torch.int32)
+    x = W.append_inputs(1, s.hidden, s.r, s.dtype, seed=41, n_seqs=n_seqs)["X"]
+    if per_agent:
+        A_kv = torch.stack([W.append_inputs(1, s.hidden, s.r, s.dtype, seed=43 + a)["A_kv"]
+                            for a in range(s.n_agents)])
+    else:
+        A_kv = W.append_inputs(1, s.hidden, s.r, s.dtype, seed=43)["A_kv"]
+    outs, lrs = [], []
+    for from_host in (False, True):
+        dd = to_device(inp)
+        out = torch.zeros(dd["q"].shape, device=DEV)
+        x_dev, A_dev = x.to(DEV), A_kv.to(DEV)
+        step = la.DecodeStep(dd["k_base"], dd["v_base"], dd["lr"], dd["B_k"], dd["B_v"], dd["q"],
+                             out, dd["kv_len"], lora_scale=s.lora_scale, rope_base=s.rope_base,
+                             max_kv_len=L_max, A_kv=A_dev, x_new=x_dev)
+        if from_host:
+            x_dev.zero_()
+            dd["q"].zero_()
+            dd["kv_len"].zero_()
+            out_host = torch.full(out.shape, 7.0).pin_memory()
+            step.from_host(x.pin_memory(), inp["q"].pin_memory(),
+                           inp["kv_len"].pin_memory(), out_host)
+            torch.cuda.synchronize()
+            outs.append(out_host.clone())
+        else:
+            for q, n in enumerate(kv_lens):
+                if per_agent:
+                    la.lr_cache_append_agents(x_dev[q:q + 1], A_dev, dd["lr"][:, q:q + 1], n - 1)
+                else:
+                    la.lr_cache_append(x_dev[q:q + 1], A_dev, dd["lr"][q:q + 1], n - 1)
+            la.lora_attn_decode(step.args, step.workspace)
+            torch.cuda.synchronize()
+            outs.append(out.cpu())
+        lrs.append(dd["lr"].cpu())
+    assert la.la_device_check() == 0
+    assert torch.equal(lrs[0], lrs[1])
+    assert not torch.equal(lrs[1], inp["lr"])   # the new rows did land
+    assert torch.equal(outs[0], outs[1])
+    assert_parity(to_np(outs[1]), oracle_decode(inp, s, lr=lrs[1].double()), s.dtype)
+
+
 # ---------------------------------------------------------- bf16 prefill ----
 @pytest.mark.parametrize("L,n_tok,r,n_agents", [
     (300, 77, 16, 3),
