@@ -615,7 +615,14 @@ def run_ours(args):
     for i in range(n_sets):
         si = s.replace(seed=s.seed + 1000 * (rank + 1) + i)
         inp = {k: v.to(dev) for k, v in W.direct_cache_inputs(si, device=dev).items()}
-        x_new = W.append_inputs(1, s.hidden, s.r, s.dtype, seed=si.seed + 7, device=dev)["X"]
+        x0 = W.append_inputs(1, s.hidden, s.r, s.dtype, seed=si.seed + 7, device=dev)["X"]
+        # the step's inputs back to back in one device buffer (one H2D copy a step)
+        _, x_new, q, kv_len = la.packed_step_inputs(x0.shape, inp["q"].shape, s.n_seqs, s.dtype,
+                                                    dev)
+        x_new.copy_(x0)
+        q.copy_(inp["q"])
+        kv_len.copy_(inp["kv_len"])
+        inp["q"], inp["kv_len"] = q, kv_len
         out = torch.empty(inp["q"].shape, dtype=torch.float32, device=dev)
         st = la.DecodeStep(inp["k_base"], inp["v_base"], inp["lr"], inp["B_k"], inp["B_v"],
                            inp["q"], out, inp["kv_len"], lora_scale=s.lora_scale,
@@ -683,9 +690,16 @@ def run_ours(args):
     # end to end through the public API with host buffers: lora_decode_step_host
     # copies the step's inputs in (new hidden row, queries, lengths), appends,
     # decodes and copies the outputs back
-    h_x = [x.cpu().pin_memory() for (_, x, _) in sets]
-    h_q = [i["q"].cpu().pin_memory() for (i, _, _) in sets]
-    h_len = [i["kv_len"].cpu().pin_memory() for (i, _, _) in sets]
+    h_x, h_q, h_len = [], [], []
+    for (i, x, _) in sets:  # pinned, back to back as on the device
+        _, hx, hq, hl = la.packed_step_inputs(x.shape, i["q"].shape, s.n_seqs, s.dtype, "cpu",
+                                              pin=True)
+        hx.copy_(x)
+        hq.copy_(i["q"])
+        hl.copy_(i["kv_len"])
+        h_x.append(hx)
+        h_q.append(hq)
+        h_len.append(hl)
     h_out = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for (_, _, o) in sets]
     h2d = h_x[0].numel() * 2 + h_q[0].numel() * 2 + h_len[0].numel() * 4
     d2h = h_out[0].numel() * 4

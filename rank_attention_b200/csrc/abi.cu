@@ -378,13 +378,27 @@ extern "C" la_status lora_decode_step_host(const la_attn_args* a, void* workspac
   const size_t es = esize(dt), eo = esize(a->out_dtype);
   const size_t x_bytes = (size_t)n_seqs * hidden * es;
   const size_t q_elems = (size_t)n_seqs * a->n_agents * a->n_q_heads * a->head_dim;
+  const size_t q_bytes = q_elems * es, kv_bytes = (size_t)n_seqs * 4;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (cudaMemcpyAsync(x_dev, x_host, x_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
-      cudaMemcpyAsync(const_cast<void*>(a->q), q_host, q_elems * es, cudaMemcpyHostToDevice,
-                      st) != cudaSuccess ||
-      cudaMemcpyAsync(const_cast<int32_t*>(a->kv_len), kv_len_host, (size_t)n_seqs * 4,
-                      cudaMemcpyHostToDevice, st) != cudaSuccess)
+  // x, q and kv_len back to back in one host and one device buffer: one copy
+  // (each copy on the stream costs microseconds of latency, whatever its size)
+  const char* xh = static_cast<const char*>(x_host);
+  const char* xd = static_cast<const char*>(x_dev);
+  const bool packed = xh + x_bytes == static_cast<const char*>(q_host) &&
+                      xh + x_bytes + q_bytes == reinterpret_cast<const char*>(kv_len_host) &&
+                      xd + x_bytes == static_cast<const char*>(a->q) &&
+                      xd + x_bytes + q_bytes == reinterpret_cast<const char*>(a->kv_len);
+  if (packed) {
+    if (cudaMemcpyAsync(x_dev, x_host, x_bytes + q_bytes + kv_bytes, cudaMemcpyHostToDevice,
+                        st) != cudaSuccess)
+      return LA_ERR_CUDA;
+  } else if (cudaMemcpyAsync(x_dev, x_host, x_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+             cudaMemcpyAsync(const_cast<void*>(a->q), q_host, q_bytes, cudaMemcpyHostToDevice,
+                             st) != cudaSuccess ||
+             cudaMemcpyAsync(const_cast<int32_t*>(a->kv_len), kv_len_host, kv_bytes,
+                             cudaMemcpyHostToDevice, st) != cudaSuccess) {
     return LA_ERR_CUDA;
+  }
   // the new rows: into the shared LR cache, or into every agent's own (X A_a)
   const int n_lr = a->lr_agent_stride > 0 ? a->n_agents : 1;
   const size_t a_bytes = (size_t)hidden * 2 * a->r * es;

@@ -286,6 +286,19 @@ def lora_decode_step_host(args: AttnArgs, workspace: torch.Tensor, A_kv: torch.T
     _check(st, "lora_decode_step_host")
 
 
+def packed_step_inputs(x_shape, q_shape, n_seqs: int, dtype: torch.dtype, device,
+                       pin: bool = False):
+    """x [x_shape], q [q_shape] (dtype) and kv_len int32 [n_seqs] as back-to-back
+    views of one buffer: laid out so on both sides, lora_decode_step_host moves
+    a step's inputs in one copy.  Returns (buffer, x, q, kv_len)."""
+    es = torch.empty(0, dtype=dtype).element_size()
+    nx, nq = math.prod(x_shape) * es, math.prod(q_shape) * es
+    buf = torch.empty(nx + nq + 4 * n_seqs, dtype=torch.uint8, device=device,
+                      pin_memory=pin)
+    return (buf, buf[:nx].view(dtype).view(x_shape), buf[nx:nx + nq].view(dtype).view(q_shape),
+            buf[nx + nq:].view(torch.int32))
+
+
 def lora_attn_decode_static_scratch(args: AttnArgs, stream=None) -> None:
     """Decode without a workspace: the split scratch is the library's own device
     array (for callers that cannot allocate device memory; see the header)."""

@@ -278,3 +278,15 @@ def test_decode_step_host_second_sequence_checked():
     # the second sequence's length is checked too, before any copy
     a = _args(n_seqs=2)
     assert _step(a=a, kv_len=(5, 300)) == la.LA_ERR_INVALID_ARG
+
+
+def test_packed_step_inputs_back_to_back():
+    """The helper's views sit in the order and with no gap that let
+    lora_decode_step_host move a step's inputs in one copy."""
+    import torch
+    buf, x, q, kv = la.packed_step_inputs((2, 1, 64), (2, 3, 1, 4, 64), 2, torch.bfloat16, "cpu")
+    assert x.data_ptr() == buf.data_ptr()
+    assert q.data_ptr() == x.data_ptr() + x.numel() * 2
+    assert kv.data_ptr() == q.data_ptr() + q.numel() * 2
+    assert kv.dtype == torch.int32 and kv.numel() == 2
+    assert buf.numel() == (x.numel() + q.numel()) * 2 + 8

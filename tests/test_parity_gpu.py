@@ -283,12 +283,13 @@ def test_decode_merge_wait_runs_out_and_is_reported(la):
     assert_parity(to_np(out), oracle_decode(inp, s), s.dtype)
 
 
-@pytest.mark.parametrize("kv_lens,per_agent", [
-    ((8192,), False),           # the LLaMA-8B decode step: one sequence, shared A
-    ((700, 650, 700), False),   # unequal lengths: one append per sequence
-    ((640, 640), True),         # BaseShared: every agent's own A_a and LR cache
+@pytest.mark.parametrize("kv_lens,per_agent,packed", [
+    ((8192,), False, False),          # the LLaMA-8B decode step: one sequence, shared A
+    ((8192,), False, True),           # the same with x, q, kv_len back to back: one copy
+    ((700, 650, 700), False, True),   # unequal lengths: one append per sequence
+    ((640, 640), True, False),        # BaseShared: every agent's own A_a and LR cache
 ])
-def test_decode_step_from_host_equals_device_step(la, kv_lens, per_agent):
+def test_decode_step_from_host_equals_device_step(la, kv_lens, per_agent, packed):
     """lora_decode_step_host (copies in, append at kv_len - 1, decode, copy out)
     gives the same LR rows and outputs, bit for bit, as the same step on
     device buffers (the append then the decode), and the outputs match the
@@ -308,6 +309,15 @@ def test_decode_step_from_host_equals_device_step(la, kv_lens, per_agent):
         dd = to_device(inp)
         out = torch.zeros(dd["q"].shape, device=DEV)
         x_dev, A_dev = x.to(DEV), A_kv.to(DEV)
+        h_x, h_q, h_len = x.pin_memory(), inp["q"].pin_memory(), inp["kv_len"].pin_memory()
+        if from_host and packed:
+            _, x_dev, dd["q"], dd["kv_len"] = la.packed_step_inputs(
+                x.shape, inp["q"].shape, n_seqs, s.dtype, DEV)
+            _, h_x, h_q, h_len = la.packed_step_inputs(x.shape, inp["q"].shape, n_seqs, s.dtype,
+                                                       "cpu", pin=True)
+            h_x.copy_(x)
+            h_q.copy_(inp["q"])
+            h_len.copy_(inp["kv_len"])
         step = la.DecodeStep(dd["k_base"], dd["v_base"], dd["lr"], dd["B_k"], dd["B_v"], dd["q"],
                              out, dd["kv_len"], lora_scale=s.lora_scale, rope_base=s.rope_base,
                              max_kv_len=L_max, A_kv=A_dev, x_new=x_dev)
@@ -316,8 +326,7 @@ def test_decode_step_from_host_equals_device_step(la, kv_lens, per_agent):
             dd["q"].zero_()
             dd["kv_len"].zero_()
             out_host = torch.full(out.shape, 7.0).pin_memory()
-            step.from_host(x.pin_memory(), inp["q"].pin_memory(),
-                           inp["kv_len"].pin_memory(), out_host)
+            step.from_host(h_x, h_q, h_len, out_host)
             torch.cuda.synchronize()
             outs.append(out_host.clone())
         else:
