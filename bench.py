@@ -503,6 +503,36 @@ def decode_bytes(s) -> int:
     return base + lr + Bw + q + out
 
 
+CACHE_SCHEMES = ("non_shared", "base_shared", "base_lr_shared")
+
+
+def kv_cache_bytes(s, scheme: str) -> int:
+    """Bytes of the KV caches of one layer that serve all n_agents agents of
+    the shape's sequences, at its context length, under a cache-sharing scheme
+    (LRAgent summary, §3 Methodology, BaseShared and BaseLRShared):
+      non_shared      every agent its own K^a and V^a, each [n_kv][L][d] (the
+                      buffers lora_materialize_agent_kv writes);
+      base_shared     one base K and V [n_kv][L][d], and every agent its own LR
+                      cache X A_a [L][2r] (lr_agent_stride > 0);
+      base_lr_shared  one base K and V, and one LR cache X A [L][2r] that all
+                      agents read (shared A).
+    Counted from the layouts the library reads, per sequence, in bf16."""
+    e = 2
+    base = 2 * s.n_kv_heads * s.kv_len * s.head_dim * e
+    lr = s.kv_len * 2 * s.r * e
+    per_seq = {"non_shared": s.n_agents * base,
+               "base_shared": base + s.n_agents * lr,
+               "base_lr_shared": base + lr}[scheme]
+    return s.n_seqs * per_seq
+
+
+def kv_cache_report(s) -> dict:
+    """kv_cache_bytes of every scheme for a shape, and each against non-shared."""
+    b = {k: kv_cache_bytes(s, k) for k in CACHE_SCHEMES}
+    return {"workload": s.name, "bytes": b,
+            "vs_non_shared": {k: b[k] / b["non_shared"] for k in CACHE_SCHEMES}}
+
+
 def append_bytes(s, n_tok: int) -> int:
     return s.n_seqs * (n_tok * s.hidden * 2 + n_tok * 2 * s.r * 2) + s.hidden * 2 * s.r * 2
 
@@ -755,6 +785,7 @@ def run_ours(args):
         "clocks": clk,
         "prefill": prefill,
         "non_shared_baseline": non_shared,
+        "kv_cache_memory": kv_cache_report(s),
         "base_shared": base_shared,
         "qkvo": qkvo,
         "value_ablation": value_ablation,
