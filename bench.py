@@ -63,6 +63,10 @@ def peaks():
         return 6650.0, "fallback"
 
 
+NOMINAL_HBM_GBS = 8000.0      # B200 HBM3e, nominal (7.7 TB/s in the HGX figure)
+NOMINAL_BF16_TFLOPS = 2250.0  # B200 dense bf16 tensor cores, nominal
+
+
 def tc_peak():
     """Dense bf16 tensor-core peak (TFLOP/s) for a kernel timed on its own."""
     try:
@@ -197,7 +201,8 @@ def time_prefill(dev, reps=5, warmup=3, s=None):
     tf = base / (ms / 1e3) / 1e12
     return {"workload": s.name, "value": tf, "unit": "TFLOP/s", "ms": ms,
             "flops_per_launch": base, "lora_inclusive_tflops": lora / (ms / 1e3) / 1e12,
-            "peak": peak, "peak_kind": kind, "frac": tf / peak, "out_dtype": "bf16",
+            "peak": peak, "peak_kind": kind, "frac": tf / peak,
+            "frac_of_nominal": tf / NOMINAL_BF16_TFLOPS, "out_dtype": "bf16",
             "timing": f"median of {reps} launches, CUDA events, L2 flushed before each"}
 
 
@@ -778,7 +783,9 @@ def run_ours(args):
                      "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                      "peak_kind": f"{peak_kind} copy bandwidth",
                      "algorithmic_bytes_per_launch": dbytes, "launch_us": dec_ms * 1e3,
-                     "traffic": DECODE_TRAFFIC.get(decode_source_sha())},
+                     "traffic": DECODE_TRAFFIC.get(decode_source_sha()),
+                     "frac_of_nominal": achieved / NOMINAL_HBM_GBS,
+                     "nominal_peak": NOMINAL_HBM_GBS},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e_steps},
         "gpu_launches": (1 + decode_kernels_per_call(s)) * args.steps,
