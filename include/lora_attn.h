@@ -31,9 +31,10 @@
  * rotated.  Per-agent K^a / V^a are never written to memory.
  *
  * Conventions for every entry point:
- *   - All tensor pointers are DEVICE pointers owned by the caller.  Nothing
- *     is retained after return.  The library never allocates device memory;
- *     decode scratch comes from the caller's workspace.
+ *   - All tensor pointers are DEVICE pointers owned by the caller, except
+ *     the *_host buffers of lora_decode_step_host.  Nothing is retained
+ *     after return.  The library never allocates device memory; decode
+ *     scratch comes from the caller's workspace.
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
  *     stream) and runs asynchronously; the library does not synchronise.
  *   - Argument errors are reported synchronously, BEFORE anything is
