@@ -578,21 +578,23 @@ def time_oracle(s, steps: int, budget_s: float):
     return s.n_seqs * s.n_agents / per, len(times), per
 
 
-def oracle_unit_step(inp, new, s, k: int) -> None:
-    """One reference step: the oracle's decode of one (agent, KV head) unit of the
-    workload (unit k cycles through all of them), after appending the new LR row."""
-    from oracle import impl as oracle
-    a = k % s.n_agents
-    j = (k // s.n_agents) % s.n_kv_heads
-    lr = oracle.lr_cache_append(inp["lr"], new["X"], new["A_kv"], s.kv_len - 1)
-    oracle.lora_attention_unit(inp["k_base"], inp["v_base"], lr, inp["B_k"], inp["B_v"],
-                               inp["q"], seq=0, agent=a, kv_head=j, kv_len=s.kv_len,
-                               q_positions=[s.kv_len - 1], lora_scale=s.lora_scale,
-                               softmax_scale=s.softmax_scale, rope_base=s.rope_base)
+def step_config(s, world: int) -> dict:
+    """The `config` of the JSON line, identical for both arms: the workload, the
+    step, how the inputs exceed L2 and how the step is timed."""
+    step_bytes = decode_bytes(s) + append_bytes(s, 1)
+    n_sets = max(2, math.ceil(2 * L2_BYTES / step_bytes))
+    return {"workload": s.name, "kv_len": s.kv_len, "agents": s.n_agents, "r": s.r,
+            "step": "lr_cache_append(1 token) + lora_attn_decode",
+            "l2": f"inputs larger than L2: {n_sets} rotating cache sets of "
+                  f"{step_bytes / 1e6:.1f} MB ({n_sets * step_bytes / 1e6:.0f} MB > 126 MB)",
+            "timing": "CUDA graphs of the steps, CUDA events on the launch stream",
+            "parallelism": f"replicas x{world}"}
 
 
 def run_reference(args):
-    """The reference arm: the fp64 oracle on the host cores (rank 0 only)."""
+    """The reference arm: the fp64 oracle on the host cores (rank 0 only), each
+    step one whole decode step of the workload (LR append of the new token,
+    then every agent's materialised attention), as the GPU arm's step."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
@@ -600,23 +602,23 @@ def run_reference(args):
     s = W.LLAMA8B_DECODE_8K
     inp = W.direct_cache_inputs(s)
     new = W.append_inputs(1, s.hidden, s.r, s.dtype, seed=s.seed + 100, n_seqs=s.n_seqs)
-    for k in range(args.warmup):
-        oracle_unit_step(inp, new, s, k)
+    for _ in range(args.warmup):
+        oracle_step(inp, new, s)
     t0 = time.perf_counter()
-    for k in range(args.steps):
-        oracle_unit_step(inp, new, s, k)
-    per_unit = (time.perf_counter() - t0) / args.steps
-    units = s.n_agents * s.n_kv_heads
-    full_step = per_unit * units          # one whole decode step of the workload
+    for _ in range(args.steps):
+        oracle_step(inp, new, s)
+    full_step = (time.perf_counter() - t0) / args.steps
     value = s.n_seqs * s.n_agents / full_step
     cores = blas_threads()
-    sample = (f"each step = one of the {units} (agent, KV head) units of {s.name} "
-              f"(append + materialised attention), cycled; rate scaled to the whole step")
+    sample = (f"{args.steps} whole decode steps of {s.name} on the host (append of the new "
+              f"token's LR row, then all {s.n_agents * s.n_kv_heads} (agent, KV head) units' "
+              f"materialised attention), after {args.warmup} untimed")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": full_step * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": s.name, "kv_len": s.kv_len, "agents": s.n_agents, "r": s.r},
+            "config": step_config(s, world),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -773,12 +775,7 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": s.name, "kv_len": s.kv_len, "agents": s.n_agents, "r": s.r,
-                   "step": "lr_cache_append(1 token) + lora_attn_decode",
-                   "l2": f"inputs larger than L2: {n_sets} rotating cache sets of "
-                         f"{step_bytes / 1e6:.1f} MB ({n_sets * step_bytes / 1e6:.0f} MB > 126 MB)",
-                   "timing": "CUDA graphs of the steps, CUDA events on the launch stream",
-                   "parallelism": f"replicas x{world}"},
+        "config": step_config(s, world),
         "roofline": {"kernel": "lora_attn_decode", "bound": "hbm", "achieved": achieved,
                      "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
                      "peak_kind": f"{peak_kind} copy bandwidth",

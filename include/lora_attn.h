@@ -245,7 +245,8 @@ la_status lora_attn_prefill(const la_attn_args* args, la_stream_t stream);
  * launch (fp32) or in a second kernel (bf16).
  *
  * workspace: device memory of at least lora_attn_decode_workspace_bytes(args)
- * bytes, 256-byte aligned, ZERO-FILLED BEFORE ITS FIRST USE.  Each call
+ * bytes, 256-byte aligned, ZERO-FILLED BEFORE ITS FIRST USE (may be NULL for
+ * an empty batch, n_seqs = 0, which returns LA_OK and launches nothing).  Each call
  * leaves the arrival counters it used back at zero, so a workspace can be
  * reused by later calls on the same stream; calls that run concurrently
  * need separate workspaces.
@@ -273,9 +274,10 @@ size_t lora_attn_decode_workspace_bytes(const la_attn_args* args);
  * scratch (per-split partials and arrival counters) lives in one device array
  * of LA_STATIC_SCRATCH_BYTES that the library holds on every device that loads
  * it, until the process exits.
- *   - The first call on a device sets the array up: it looks up the array's
- *     device address, clears it and synchronises that device.  Make that first
- *     call before any stream capture.
+ *   - Each call looks up the array's device address on the current device
+ *     (a host-side query) and allocates nothing.
+ *   - An empty batch (n_seqs = 0) returns LA_OK and launches nothing; invalid
+ *     arguments return the status lora_attn_decode would return.
  *   - Every call shares the one array, which keeps what the last call left
  *     in it; each call first clears, on `stream`, the part that must start at
  *     zero.  Calls whose work overlaps on the GPU (other streams, other host

@@ -297,6 +297,13 @@ bool decode_counter_range(const la_attn_args* a, size_t* offset, size_t* bytes) 
   *bytes = d.counter_bytes;
   return true;
 }
+
+// What lora_attn_decode's argument checks say about these arguments alone
+// (no workspace considered): LA_OK for valid arguments.
+la_status decode_args_status(const la_attn_args* a) {
+  AttnParams p;
+  return check_attn(a, 1, &p);
+}
 }  // namespace la
 
 extern "C" size_t lora_attn_decode_workspace_bytes(const la_attn_args* a) {
@@ -314,14 +321,14 @@ la_status decode_prepare(const la_attn_args* a, void* workspace, size_t workspac
   *empty = false;
   la_status s = check_attn(a, 1, p);
   if (s != LA_OK) return s;
+  if (p->n_seqs == 0) {  // an empty batch needs no workspace (its size is 0)
+    *empty = true;
+    return LA_OK;
+  }
   DecodePlan d = plan_decode(*p, a->io_dtype);
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
       workspace_bytes < d.partial_bytes + d.counter_bytes)
     return LA_ERR_WORKSPACE;
-  if (p->n_seqs == 0) {
-    *empty = true;
-    return LA_OK;
-  }
   if ((int64_t)p->n_seqs * p->n_kv > 65535) return LA_ERR_UNSUPPORTED;
   if (d.kind == 0 && simt_smem_bytes(*p) > 227 * 1024) return LA_ERR_UNSUPPORTED;
   p->n_splits = d.n_splits;

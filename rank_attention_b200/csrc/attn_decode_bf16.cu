@@ -1651,6 +1651,7 @@ int decode_groups(const AttnParams& p) {
 // fully resident
 int n_splits_for(const AttnParams& p) {
   const int units = p.n_seqs * p.n_kv * decode_groups(p);
+  if (units < 1) return 1;   // an empty batch
   const int64_t total_tiles = (p.max_kv_len + KT - 1) / KT;
   const int sms = device_sms();
   int64_t ns = units >= sms ? 1 : sms / units;

@@ -471,25 +471,61 @@ def test_llama8b_prefill_16k_sampled(la):
     _sampled_units(la, s, inp, got, [(0, 0, 0), (0, 1, 3), (0, 2, 7)], tokens)
 
 
-def test_llama8b_stack_prefill_sampled(la):
-    """One layer of the 32-layer stack: a 4096-token chunk over a 32768-token
-    prefix, 4 agents, r = 64 (the tensor-core prefill with one V stage)."""
-    s = W.llama8b_stack_prefill(0)
-    inp = W.direct_cache_inputs(s)
-    dd = to_device(inp)
-    got = _run(la, s, dd["k_base"], dd["v_base"], dd["lr"], dd["B_k"], dd["B_v"], dd["q"]).cpu()
-    tokens = np.array([0, 1, 127, 128, 2047, 4095])
-    _sampled_units(la, s, inp, got, [(0, 0, 0), (0, 3, 5)], tokens)
+@pytest.mark.parametrize("layer", [0, 15, 31])
+def test_llama8b_stack_prefill_sampled(la, layer):
+    """Layers 0, 15 and 31 of the 32-layer stack (each its own seeded inputs):
+    a 4096-token chunk over a 32768-token prefix, 4 agents, r = 64 (the
+    tensor-core prefill with one V stage).  Every agent and KV head is
+    sampled across the layers, at tokens on tile and block edges and the last."""
+    s = W.llama8b_stack_prefill(layer)
+    inp = W.direct_cache_inputs(s, device=DEV)
+    got = _run(la, s, inp["k_base"], inp["v_base"], inp["lr"], inp["B_k"], inp["B_v"],
+               inp["q"]).cpu()
+    tokens = np.array([0, 1, 31, 32, 127, 128, 1000, 2047, 2048, 3071, 4094, 4095])
+    units = [((0, (layer + k) % s.n_agents, (3 * layer + 5 * k) % s.n_kv_heads)) for k in range(4)]
+    _sampled_units(la, s, inp, got, units, tokens)
 
 
-@pytest.mark.parametrize("ctx", [32768])
+@pytest.mark.parametrize("layer", [0, 15, 31])
+def test_llama8b_stack_decode_full(la, layer):
+    """The stack's decode over the 36864 cached keys (prefix + chunk), 4 agents,
+    r = 64, layers 0, 15 and 31: every output against the oracle."""
+    s = W.llama8b_stack_decode(layer)
+    inp = W.direct_cache_inputs(s, device=DEV)
+    got = _run(la, s, inp["k_base"], inp["v_base"], inp["lr"], inp["B_k"], inp["B_v"], inp["q"],
+               inp["kv_len"])
+    assert_parity(to_np(got), oracle_decode(inp, s), s.dtype)
+
+
+@pytest.mark.parametrize("ctx", W.SWEEP_CTX)
 def test_llama8b_sweep_decode_sampled(la, ctx):
+    """The batched long-context decode (16 requests x 5 agents, r = 32) at
+    32768, 65536 and 131072 keys; inputs drawn on the device, sampled
+    (sequence, agent, KV head) units copied to the host for the oracle."""
     s = W.llama8b_sweep(ctx)
-    inp = W.direct_cache_inputs(s)
-    dd = to_device(inp)
-    got = _run(la, s, dd["k_base"], dd["v_base"], dd["lr"], dd["B_k"], dd["B_v"], dd["q"],
-               dd["kv_len"]).cpu()
-    _sampled_units(la, s, inp, got, [(0, 0, 0), (5, 4, 7), (15, 2, 3)], np.array([0]))
+    inp = W.direct_cache_inputs(s, device=DEV)
+    got = _run(la, s, inp["k_base"], inp["v_base"], inp["lr"], inp["B_k"], inp["B_v"], inp["q"],
+               inp["kv_len"]).cpu()
+    _sampled_units(la, s, inp, got, [(0, 0, 0), (5, 4, 7), (15, 2, 3), (9, 3, 1)], np.array([0]))
+    del inp
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("ctx,n_agents,r", [(131072, 5, 32), (36864, 4, 64)])
+def test_decode_dominated_by_the_last_keys(la, ctx, n_agents, r):
+    """The largest positions decide the output: the LR rows of the last 200
+    keys are scaled fourfold, so their rotated key deltas lead the scores and
+    their values the output.  A rotation off by one position at the tail then
+    moves the outputs by about 5e-2 of their maximum (1e-2 rad of drift by
+    about 5e-3), where with unscaled rows it would be averaged away over the
+    131072 keys (3e-3)."""
+    s = W.llama8b_sweep(ctx).replace(n_seqs=1, n_agents=n_agents, r=r, alpha=2.0 * r,
+                                     seed=ctx + r)
+    inp = W.direct_cache_inputs(s, device=DEV)
+    inp["lr"][:, ctx - 200:] *= 4
+    got = _run(la, s, inp["k_base"], inp["v_base"], inp["lr"], inp["B_k"], inp["B_v"], inp["q"],
+               inp["kv_len"])
+    assert_parity(to_np(got), oracle_decode(inp, s), s.dtype)
 
 
 # ------------------------------------------------------ non-shared baseline ----
