@@ -25,6 +25,7 @@ int simt_key_tile();
 size_t simt_smem_bytes(const AttnParams& p);
 bool bf16_decode_supported(const AttnParams& p);
 size_t bf16_decode_partial_bytes(const AttnParams& p);
+size_t bf16_decode_counter_ints(const AttnParams& p);
 void bf16_decode_plan(const AttnParams& p, int* n_splits, int64_t* split_len, int* rows, int* groups);
 cudaError_t launch_decode_bf16(const AttnParams& p, la_dtype out, cudaStream_t st);
 bool bf16_prefill_supported(const AttnParams& p);
@@ -141,8 +142,10 @@ DecodePlan plan_decode(const AttnParams& p, la_dtype io) {
   else
     d.partial_bytes = d.n_splits > 1 ? (size_t)units * d.n_splits * d.rows * W * sizeof(float) : 0;
   d.partial_bytes = (d.partial_bytes + 255) / 256 * 256;
-  // per unit: an arrival and a departure counter of the split merge
-  d.counter_bytes = ((size_t)2 * units * d.groups * sizeof(int) + 255) / 256 * 256;
+  // the split merge's counters: per unit an arrival and a departure counter
+  // (generic kernel), or the bf16 decode's own
+  const size_t ints = d.kind == 1 ? bf16_decode_counter_ints(p) : (size_t)2 * units * d.groups;
+  d.counter_bytes = (ints * sizeof(int) + 255) / 256 * 256;
   return d;
 }
 

@@ -1,0 +1,883 @@
+// Flash-LoRA-Attention decode with the key-side LoRA scored on the tensor
+// cores through a cos/sin table (bf16 storage, fp32 accumulate).
+//
+// The key of agent a at position t is K^a_t = K_base,t + RoPE_t(s LRk_t B_k^a)
+// (LRAgent summary App. D.1: the delta is rebuilt in head dimension because
+// RoPE blocks the reordering on the key side).  RoPE pairs element i with
+// i + d/2 and turns the pair by t theta_i, so for a query row q the delta's
+// share of the score is
+//   q . RoPE_t(s LRk_t B) = sum_rho LRk_t[rho] W[t, rho],
+//   W[t, rho] = sum_{i < d/2} cos(t theta_i) U[rho, i] + sin(t theta_i) V[rho, i],
+//   U[rho, i] = s (q_i B[rho, i] + q_{i+d/2} B[rho, i+d/2]),
+//   V[rho, i] = s (q_{i+d/2} B[rho, i] - q_i B[rho, i+d/2]).
+// U and V depend on the row's query and its agent's B_k^a only, so a CTA
+// builds them once ([U | V] is the d-deep B operand, one row per (query row,
+// rho)), and per 128-key tile the tensor cores compute W = CS UV^T from the
+// tile's table CS[j] = [cos | sin]((k0 + j) theta) (A operand, in TMEM).  What
+// is left on the CUDA cores per key is an r-wide dot with LRk_t; no key delta
+// is rotated element by element.
+//
+// One CTA = one (sequence, KV head, agent group, key split).  Its rows are the
+// group's agents x the GQA group's query heads, so every base and LR tile
+// crosses HBM once for all of them (LRAgent summary §3 BaseLRShared).
+//  * warp 9 (one thread) issues per tile S = K_base Q^T and W = CS UV^T, and
+//    for the previous tile O^T += V_base^T P^T (tcgen05, fp32 in TMEM);
+//  * warps 0-7 (key j = 32 (w % 4) + lane, half w / 4 of the rows) add the
+//    r-wide dots to S, run the online softmax and write P (bf16); they also
+//    write the next tile's table CS into TMEM: (cos, sin)((k0 + j) theta) from
+//    the exact (cos, sin)(k0 theta) (angle reduced in fp64) and per-thread
+//    (cos, sin)(j theta);
+//  * warp 8 keeps the value side reordered (LRAgent explainer, Metodologia 3;
+//    summary App. B): O_lr^T += LRv^T P^T stays r wide (mma.sync); it also
+//    streams K_base, V_base and the LR rows of each tile by TMA into a
+//    two-stage ring, with a window of later tiles requested into L2.
+// The softmax rescales lazily: a row's reference maximum moves only when a
+// tile's maximum passes it by more than 2^8, so O and O_lr are rescaled only
+// then; out = O / l holds for any reference.
+// Splits of the keys merge in the same launch without waiting: each CTA takes
+// a ticket when its partial (O_base, O_lr, m, l) is ready; all but the last
+// publish it and leave, and the last one merges them all,
+//   w_k = 2^(m_k - M) / sum_k 2^(m_k - M) l_k,
+//   out = sum_k w_k O_base,k + s (sum_k w_k O_lr,k) B_v^a,
+// B_v^a applied once per row.  No CTA waits for one that has not arrived, so
+// the launch needs no co-residency and may run in several waves.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+
+#include "bf16_common.cuh"
+#include "la_internal.cuh"
+#include "ptx.cuh"
+
+namespace la {
+namespace {
+
+using namespace ptx;
+
+constexpr int KT = 128;            // keys per tile
+constexpr int ST = 2;              // pipeline stages
+constexpr int D = 128;             // head_dim
+constexpr int QP = 16;             // padded query rows: N of S and of P V
+constexpr int NSW = 8;             // score warps
+constexpr int WV = 8, WM = 9;
+constexpr int NTHR = 32 * 10;
+constexpr int kL2Ahead = 4;        // tiles requested into L2 ahead of the stage loads
+constexpr int kMaxSplits = 32;
+constexpr int kSMs = 148;
+
+// TMEM columns
+constexpr uint32_t T_W = 0, T_CS = 256, T_S = 320, T_O = 352, T_COLS = 512;
+
+// barriers (mbarrier slots)
+enum { B_FULL = 0, B_EMPTY = ST, B_TFULL = 2 * ST, B_WFREE, B_CSFULL, B_PFULL, B_PFREE, B_ODONE, B_NUM };
+
+template <int R, int RP>
+struct Cfg {
+  static constexpr int NW = RP * R;                     // W columns: (row, rho)
+  static constexpr int RH = RP / 2;                     // rows per score-warp half
+  static constexpr int KV_TILE = KT * D * 2;            // a K or V tile: 2 boxes of 64 d
+  static constexpr int LB = 2 * R < 64 ? 2 * R : 64;     // LR box columns
+  static constexpr int LR_TILE = align1k(KT * 2 * R * 2);
+  static constexpr int STAGE = 2 * KV_TILE + LR_TILE;
+  static constexpr int UV_BYTES = align1k(NW * D * 2);
+  static constexpr int Q_BYTES = align1k(QP * D * 2);
+  static constexpr int P_BYTES = align1k(QP * KT * 2);
+  static constexpr int WP = D + R + 4;                  // partial row: O | O_lr | m | l | pad
+  static constexpr int MR = R / 16;                     // m16 tiles of O_lr^T
+  // small area: Mx [2][8][4] f32, Corr [2][QP] f32, cs0 [2][64] f32x2,
+  // Lsum [QP][4] f32, Mfin [QP] f32, theta [64] f64, barriers, slots
+  static constexpr int SMALL = 2 * 8 * 4 * 4 + 2 * QP * 4 + 2 * 64 * 8 + QP * 4 * 4 + QP * 4 + 64 * 8 +
+                               B_NUM * 8 + 64;
+  static constexpr size_t smem() {
+    return 1024 + (size_t)ST * STAGE + UV_BYTES + Q_BYTES + P_BYTES + align1k(SMALL);
+  }
+  static_assert(NW <= 256, "W is one MMA of N <= 256");
+  static_assert(RP % 4 == 0 && RP <= QP, "rows");
+  static_assert((size_t)RP * WP * 4 <= (size_t)UV_BYTES, "partial staging fits the UV area");
+};
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ int ld_acquire(const int* p) { return ld_acquire_gpu(p); }
+
+template <int R, int RP>
+__global__ void __launch_bounds__(NTHR, 1)
+    decode_cs_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                     const __grid_constant__ CUtensorMap tmL, const AttnParams p,
+                     const __grid_constant__ RopeTheta rt) {
+  using C = Cfg<R, RP>;
+  constexpr int NW = C::NW, RH = C::RH, WP = C::WP;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char* stages = smem;
+  unsigned char* uv = stages + ST * C::STAGE;
+  unsigned char* qop = uv + C::UV_BYTES;
+  unsigned char* pbuf = qop + C::Q_BYTES;
+  float* Mx = reinterpret_cast<float*>(pbuf + C::P_BYTES);   // [2 halves][8 rows][4 sub-partitions]
+  float* Corr = Mx + 2 * 8 * 4;                                // [2][QP]
+  float2* cs0 = reinterpret_cast<float2*>(Corr + 2 * QP);      // [2][64]: (cos, sin)(k0 theta_i)
+  float* Lsum = reinterpret_cast<float*>(cs0 + 2 * 64);        // [QP][4]
+  float* Mfin = Lsum + QP * 4;                                 // [QP]
+  double* theta = reinterpret_cast<double*>(Mfin + QP);        // [64]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(theta + 64);
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + B_NUM);
+  int* s_misc = reinterpret_cast<int*>(tslot + 2);             // [0] fail, [1] ticket
+  float* Part = reinterpret_cast<float*>(uv);                  // [RP][WP], after the last MMA
+
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int unit = blockIdx.z;
+  const int seq = unit / p.n_kv, kvh = unit % p.n_kv;
+  const int split = blockIdx.x, ns = p.n_splits;
+  const int agent0 = blockIdx.y * p.agent_group;
+  const int g = p.g, na = min(p.agent_group, p.n_agents - agent0), n_rows = na * g;
+  const int na_tot = p.n_agents;
+  const int lra = p.lr_agent ? agent0 : 0;   // one LR cache per agent: one agent per CTA
+  const int unitg = blockIdx.y * (p.n_seqs * p.n_kv) + unit;
+  const int n_units_g = gridDim.y * p.n_seqs * p.n_kv;
+
+  const int64_t total_tiles = (p.max_kv_len + KT - 1) / KT;
+  const int64_t tb = split * total_tiles / ns;
+  const int64_t te = (split + 1) * total_tiles / ns;
+  const int64_t k_lo = tb * KT;
+  const int n_spec = (int)min((int64_t)ST, te - tb);
+
+  const uint32_t st_u = smem_u32(stages);
+  const uint32_t uv_u = smem_u32(uv);
+  const uint32_t q_u = smem_u32(qop);
+  const uint32_t p_u = smem_u32(pbuf);
+  const uint32_t bar_u = smem_u32(bars);
+  auto bar = [&](int i) { return bar_u + 8u * (uint32_t)i; };
+  const int64_t ldB = (int64_t)p.n_kv * D;
+
+  auto issue = [&](int n) {  // TMA of tile n into stage n % ST (one thread)
+    const int s = n % ST;
+    const uint32_t sb = st_u + s * C::STAGE;
+    const int key0 = (int)(k_lo + (int64_t)n * KT);
+    mbar_expect_tx(bar(B_FULL + s), 2 * C::KV_TILE + KT * 2 * R * 2);
+#pragma unroll
+    for (int b = 0; b < D / 64; ++b) {
+      tma_load_4d(sb + b * KT * 128, &tmK, bar(B_FULL + s), 64 * b, key0, kvh, seq);
+      tma_load_4d(sb + C::KV_TILE + b * KT * 128, &tmV, bar(B_FULL + s), 64 * b, key0, kvh, seq);
+    }
+#pragma unroll
+    for (int b = 0; b < (2 * R) / C::LB; ++b)
+      tma_load_4d(sb + 2 * C::KV_TILE + b * KT * C::LB * 2, &tmL, bar(B_FULL + s), C::LB * b, key0, seq, lra);
+  };
+  auto prefetch = [&](int n) {  // tile n into L2 only
+    const int key0 = (int)(k_lo + (int64_t)n * KT);
+#pragma unroll
+    for (int b = 0; b < D / 64; ++b) {
+      tma_prefetch_l2_4d(&tmK, 64 * b, key0, kvh, seq);
+      tma_prefetch_l2_4d(&tmV, 64 * b, key0, kvh, seq);
+    }
+#pragma unroll
+    for (int b = 0; b < (2 * R) / C::LB; ++b) tma_prefetch_l2_4d(&tmL, C::LB * b, key0, seq, lra);
+  };
+
+  // ---- barriers, then the first tiles (by max_kv_len: independent of kv_len)
+  if (w == WV && lane == 0) {
+    s_misc[0] = 0;
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(bar(B_FULL + s), 1);
+      mbar_init(bar(B_EMPTY + s), 2);      // the P V MMA's commit + the value warp
+    }
+    mbar_init(bar(B_TFULL), 1);
+    mbar_init(bar(B_WFREE), NSW);
+    mbar_init(bar(B_CSFULL), NSW);
+    mbar_init(bar(B_PFULL), NSW + 1);
+    mbar_init(bar(B_PFREE), 2);
+    mbar_init(bar(B_ODONE), 1);
+    fence_mbar_init();
+    tma_prefetch(&tmK);
+    tma_prefetch(&tmV);
+    tma_prefetch(&tmL);
+    // a programmatic dependent of the preceding kernel (the step's LR append):
+    // everything above overlaps its tail, every input is read after the wait
+    pdl_wait();
+    for (int n = 0; n < n_spec; ++n) issue(n);
+  }
+  if (tid < D / 2) theta[tid] = rt.theta[tid];
+  if (tid < 2 * QP) Corr[tid] = 1.f;
+  pdl_wait();
+  const int64_t kvl = p.kv_len[seq];
+  const bool bad_len = kvl < 1 || kvl > p.max_kv_len;
+  const int64_t k_hi = bad_len ? k_lo : min(te * KT, kvl);
+  const int n_tiles = k_hi > k_lo ? (int)((k_hi - k_lo + KT - 1) / KT) : 0;
+  if (w == WM) tmem_alloc(smem_u32(tslot), T_COLS);
+
+  // ---- per-CTA operands: [U | V] (B of W = CS UV^T), the queries (B of S), P zeroed
+  {
+    const __nv_bfloat16* Q = reinterpret_cast<const __nv_bfloat16*>(p.q);
+    const __nv_bfloat16* Bk = reinterpret_cast<const __nv_bfloat16*>(p.B_k);
+    const float s = p.s;
+    for (int it = tid; it < NW * 8; it += NTHR) {   // (row, rho) x 8 frequencies
+      const int n = it >> 3, i0 = (it & 7) * 8;
+      const int row = n / R, rho = n % R;
+      uint4 u4 = make_uint4(0, 0, 0, 0), v4 = u4;
+      if (row < n_rows && !bad_len) {
+        const int a = row / g, gi = row % g;
+        const __nv_bfloat16* qr = Q + (((int64_t)seq * na_tot + agent0 + a) * p.n_q + kvh * g + gi) * D;
+        const __nv_bfloat16* br = Bk + ((int64_t)(agent0 + a) * R + rho) * ldB + kvh * D;
+        const uint4 q1 = __ldg(reinterpret_cast<const uint4*>(qr + i0));
+        const uint4 q2 = __ldg(reinterpret_cast<const uint4*>(qr + D / 2 + i0));
+        const uint4 b1 = __ldg(reinterpret_cast<const uint4*>(br + i0));
+        const uint4 b2 = __ldg(reinterpret_cast<const uint4*>(br + D / 2 + i0));
+        const uint32_t* q1w = reinterpret_cast<const uint32_t*>(&q1);
+        const uint32_t* q2w = reinterpret_cast<const uint32_t*>(&q2);
+        const uint32_t* b1w = reinterpret_cast<const uint32_t*>(&b1);
+        const uint32_t* b2w = reinterpret_cast<const uint32_t*>(&b2);
+        uint32_t* uw = reinterpret_cast<uint32_t*>(&u4);
+        uint32_t* vw = reinterpret_cast<uint32_t*>(&v4);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 x1 = unpack_bf16(q1w[e]), x2 = unpack_bf16(q2w[e]);
+          const float2 c1 = unpack_bf16(b1w[e]), c2 = unpack_bf16(b2w[e]);
+          uw[e] = pack_bf16(s * fmaf(x1.x, c1.x, x2.x * c2.x), s * fmaf(x1.y, c1.y, x2.y * c2.y));
+          vw[e] = pack_bf16(s * fmaf(x2.x, c1.x, -x1.x * c2.x), s * fmaf(x2.y, c1.y, -x1.y * c2.y));
+        }
+      }
+      *reinterpret_cast<uint4*>(uv + tile_off<D, NW>(n, i0)) = u4;
+      *reinterpret_cast<uint4*>(uv + tile_off<D, NW>(n, D / 2 + i0)) = v4;
+    }
+    for (int it = tid; it < QP * (D / 8); it += NTHR) {
+      const int row = it / (D / 8), c = (it % (D / 8)) * 8;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (row < n_rows && !bad_len) {
+        const int a = row / g, gi = row % g;
+        v = __ldg(reinterpret_cast<const uint4*>(Q + (((int64_t)seq * na_tot + agent0 + a) * p.n_q + kvh * g + gi) * D + c));
+      }
+      *reinterpret_cast<uint4*>(qop + tile_off<D, QP>(row, c)) = v;
+    }
+    for (int it = tid; it < C::P_BYTES / 16; it += NTHR)
+      *reinterpret_cast<uint4*>(pbuf + it * 16) = make_uint4(0, 0, 0, 0);
+  }
+
+  // ---- score warps: per-thread (cos, sin)(j theta_i) for their 32 frequencies,
+  // and the exact (cos, sin)(k0 theta_i) of the first two tiles
+  const int sp = w & 3, hh = (w >> 2) & 1;
+  const int jk = 32 * sp + lane;                  // this thread's key in a tile (its TMEM lane)
+  const uint32_t lane_off = (uint32_t)(32 * sp) << 16;
+  uint64_t CJ[16], SJ[16];
+  if (w < NSW) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const int i0 = 32 * hh + 2 * e;
+      const float2 a = sincos_small((float)jk * rt.thetaf[i0]);
+      const float2 b = sincos_small((float)jk * rt.thetaf[i0 + 1]);
+      CJ[e] = f2(a.x, b.x);
+      SJ[e] = f2(a.y, b.y);
+    }
+    if (sp == 0) {
+      const int i = 32 * hh + lane;
+      cs0[i] = rope_cs_exact(k_lo, rt.theta[i]);
+      cs0[64 + i] = rope_cs_exact(k_lo + KT, rt.theta[i]);
+    }
+  }
+
+  fence_proxy_async_smem();   // UV, Q and P are read by the tensor cores (async proxy)
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+  int fail = 0;
+  const float sl2 = p.scale * kLog2e;
+
+  // CS of tile n into TMEM: lane j, columns 16 hh.. (cos) and 32 + 16 hh.. (sin)
+  auto write_cs = [&](int n) {
+    const float4* c0 = reinterpret_cast<const float4*>(cs0 + (n & 1) * 64 + 32 * hh);
+    uint32_t cw[16], sw[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const float4 v = c0[e];   // (cos, sin) of frequencies 2e, 2e + 1 of this half
+      const uint64_t cc = f2(v.x, v.z), ss = f2(v.y, v.w), nss = f2(-v.y, -v.w);
+      const float2 co = f2_unpack(fma_f2(cc, CJ[e], mul_f2(nss, SJ[e])));
+      const float2 si = f2_unpack(fma_f2(ss, CJ[e], mul_f2(cc, SJ[e])));
+      cw[e] = pack_bf16(co.x, co.y);
+      sw[e] = pack_bf16(si.x, si.y);
+    }
+    tmem_st32x32b_x16(tmem + T_CS + 16 * hh + lane_off, cw);
+    tmem_st32x32b_x16(tmem + T_CS + 32 + 16 * hh + lane_off, sw);
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar(B_CSFULL));
+  };
+
+  if (w < NSW) {
+    // ======================================================== score warps
+    if (n_tiles > 0) write_cs(0);
+    float m_ref[RH], l_st[RH];
+#pragma unroll
+    for (int r = 0; r < RH; ++r) {
+      m_ref[r] = -INFINITY;
+      l_st[r] = 0.f;
+    }
+    for (int n = 0; n < n_tiles; ++n) {
+      const int s = n % ST;
+      const int64_t k0 = k_lo + (int64_t)n * KT;
+      const bool valid = k0 + jk < k_hi;
+      if (!mbar_wait(bar(B_FULL + s), (n / ST) & 1)) fail = 1;
+      if (!mbar_wait(bar(B_TFULL), n & 1)) fail = 1;
+      tc_fence_after();
+      // S (every row), this half's W columns, this key's LRk
+      uint32_t sv[16];
+      tmem_ld32x32b_x16(sv, tmem + T_S + lane_off);
+      float lk[R];
+      {
+        const unsigned char* lrow = stages + s * C::STAGE + 2 * C::KV_TILE;
+#pragma unroll
+        for (int c = 0; c < R; c += 8) {
+          const uint4 v = *reinterpret_cast<const uint4*>(lrow + tile_off<2 * R, KT>(jk, c));
+          const float2 a0 = unpack_bf16(v.x), a1 = unpack_bf16(v.y), a2 = unpack_bf16(v.z), a3 = unpack_bf16(v.w);
+          lk[c] = a0.x; lk[c + 1] = a0.y; lk[c + 2] = a1.x; lk[c + 3] = a1.y;
+          lk[c + 4] = a2.x; lk[c + 5] = a2.y; lk[c + 6] = a3.x; lk[c + 7] = a3.y;
+        }
+      }
+      float dsc[RH];
+      constexpr int RPC = 32 / R;   // rows per 32-column chunk
+#pragma unroll
+      for (int ch = 0; ch < RH / RPC; ++ch) {
+        uint32_t wv[32];
+        tmem_ld32x32b_x32(wv, tmem + T_W + (uint32_t)(hh * RH * R + 32 * ch) + lane_off);
+        tmem_wait_ld_r32(wv);
+#pragma unroll
+        for (int rr = 0; rr < RPC; ++rr) {
+          uint64_t acc = f2(0.f, 0.f);
+#pragma unroll
+          for (int rho = 0; rho < R; rho += 2)
+            acc = fma_f2(f2(lk[rho], lk[rho + 1]),
+                         f2(__uint_as_float(wv[rr * R + rho]), __uint_as_float(wv[rr * R + rho + 1])), acc);
+          const float2 a2 = f2_unpack(acc);
+          dsc[ch * RPC + rr] = a2.x + a2.y;
+        }
+      }
+      tmem_wait_ld_r16(sv);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_WFREE));   // S and W of this tile are in registers
+      if (n + 1 < n_tiles) write_cs(n + 1);        // W of this tile has read CS: refill it
+      if (sp == 0 && n + 2 < n_tiles) {            // exact (cos, sin)(k0 theta) two tiles ahead
+        const int i = 32 * hh + lane;
+        cs0[(n & 1) * 64 + i] = rope_cs_exact(k0 + 2 * KT, theta[i]);
+      }
+      // scores (log2 units) and this tile's row maxima
+      float x[RH];
+#pragma unroll
+      for (int r = 0; r < RH; ++r) {
+        const float sb = __uint_as_float(hh ? sv[RH + r] : sv[r]);
+        x[r] = valid ? (sb + dsc[r]) * sl2 : -INFINITY;
+        const float mt = warp_max(x[r]);
+        if (lane == 0) Mx[(hh * 8 + r) * 4 + sp] = mt;
+      }
+      bar_sync(1 + hh, 128);
+      bool moved = false;
+      float corr[RH];
+#pragma unroll
+      for (int r = 0; r < RH; ++r) {
+        const float4 m4 = *reinterpret_cast<const float4*>(Mx + (hh * 8 + r) * 4);
+        const float tmax = fmaxf(fmaxf(m4.x, m4.y), fmaxf(m4.z, m4.w));
+        corr[r] = 1.f;
+        if (tmax > m_ref[r] + 8.f) {   // lazy: move the reference only when it is 2^8 behind
+          corr[r] = m_ref[r] == -INFINITY ? 0.f : fast_exp2(m_ref[r] - tmax);
+          m_ref[r] = tmax;
+          l_st[r] *= corr[r];
+          moved = true;
+        }
+        if (sp == 0 && lane == 0) Corr[(n & 1) * QP + hh * RH + r] = corr[r];
+      }
+      // P V and O_lr of the previous tile are done: P is free, O^T is final
+      if (n > 0 && !mbar_wait(bar(B_PFREE), (n - 1) & 1)) fail = 1;
+      if (moved && n > 0) {   // O^T (TMEM lanes = d, columns = rows) times corr
+        tc_fence_after();
+#pragma unroll
+        for (int r = 0; r < RH; ++r)
+          if (corr[r] != 1.f) {
+            const uint32_t ta = tmem + T_O + (uint32_t)(hh * RH + r) + lane_off;
+            uint32_t o = tmem_ld32x32b_x1(ta);
+            tmem_wait_ld_r1(o);
+            tmem_st32x32b_x1(ta, __float_as_uint(__uint_as_float(o) * corr[r]));
+          }
+        tmem_wait_st();
+      }
+#pragma unroll
+      for (int r = 0; r < RH; ++r) {
+        const float pr = m_ref[r] == -INFINITY ? 0.f : fast_exp2(x[r] - m_ref[r]);
+        l_st[r] += pr;
+        const __nv_bfloat16 pb = __float2bfloat16_rn(pr);
+        sts16(p_u + tile_off<KT, QP>(hh * RH + r, jk), *reinterpret_cast<const uint16_t*>(&pb));
+      }
+      fence_proxy_async_smem();   // the P V MMA reads P through the async proxy
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_PFULL));
+    }
+    // ---- partial of this CTA: l (over the keys), m, O^T
+#pragma unroll
+    for (int r = 0; r < RH; ++r) {
+      const float lt = warp_sum(l_st[r]);
+      if (lane == 0) Lsum[(hh * RH + r) * 4 + sp] = lt;
+      if (sp == 0 && lane == 0) Mfin[hh * RH + r] = m_ref[r];
+    }
+    uint32_t ov[16];
+    if (n_tiles > 0) {
+      if (!mbar_wait(bar(B_ODONE), 0)) fail = 1;
+      tc_fence_after();
+      tmem_ld32x32b_x16(ov, tmem + T_O + lane_off);
+      tmem_wait_ld_r16(ov);
+    } else {
+#pragma unroll
+      for (int c = 0; c < 16; ++c) ov[c] = 0u;
+    }
+#pragma unroll
+    for (int r = 0; r < RH; ++r) Part[(hh * RH + r) * WP + jk] = __uint_as_float(hh ? ov[RH + r] : ov[r]);
+  } else if (w == WV) {
+    // ======================================================== value warp
+    // O_lr^T (r x rows) += LRv^T P^T over the tile's keys (mma.sync), and the
+    // rows of a tile past the sequence's end zeroed in V and LRv
+    float Olr[C::MR][2][4];
+#pragma unroll
+    for (int mr = 0; mr < C::MR; ++mr)
+#pragma unroll
+      for (int pt = 0; pt < 2; ++pt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) Olr[mr][pt][e] = 0.f;
+    const int mi = lane >> 3, rr = lane & 7, t4 = lane & 3;
+    if (lane == 0)
+      for (int m = ST; m < n_tiles && m < ST + kL2Ahead; ++m) prefetch(m);
+    for (int n = 0; n < n_tiles; ++n) {
+      const int s = n % ST;
+      const int64_t k0 = k_lo + (int64_t)n * KT;
+      unsigned char* sb = stages + s * C::STAGE;
+      if (!mbar_wait(bar(B_FULL + s), (n / ST) & 1)) fail = 1;
+      if (k0 + KT > k_hi) {   // P is 0 there; zeroed rows keep stale NaN out of P V
+        const int first = (int)(k_hi - k0);
+        for (int i = lane; i < (KT - first) * (D / 8); i += 32) {
+          const int row = first + i / (D / 8), c = 8 * (i % (D / 8));
+          *reinterpret_cast<uint4*>(sb + C::KV_TILE + tile_off<D, KT>(row, c)) = make_uint4(0, 0, 0, 0);
+        }
+        for (int i = lane; i < (KT - first) * (R / 8); i += 32) {
+          const int row = first + i / (R / 8), c = R + 8 * (i % (R / 8));
+          *reinterpret_cast<uint4*>(sb + 2 * C::KV_TILE + tile_off<2 * R, KT>(row, c)) = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_PFULL));
+      if (!mbar_wait(bar(B_PFULL), n & 1)) fail = 1;
+#pragma unroll
+      for (int pt = 0; pt < 2; ++pt) {
+        const float c0 = Corr[(n & 1) * QP + 8 * pt + 2 * t4];
+        const float c1 = Corr[(n & 1) * QP + 8 * pt + 2 * t4 + 1];
+#pragma unroll
+        for (int mr = 0; mr < C::MR; ++mr) {
+          Olr[mr][pt][0] *= c0; Olr[mr][pt][2] *= c0;
+          Olr[mr][pt][1] *= c1; Olr[mr][pt][3] *= c1;
+        }
+      }
+      const uint32_t sl = smem_u32(sb + 2 * C::KV_TILE);
+#pragma unroll 2
+      for (int ks = 0; ks < KT / 16; ++ks) {
+        uint32_t bP[2][2];
+#pragma unroll
+        for (int pt = 0; pt < 2; ++pt)
+          ldsm_x2(bP[pt][0], bP[pt][1], p_u + tile_off<KT, QP>(8 * pt + rr, 16 * ks + ((lane >> 3) & 1) * 8));
+#pragma unroll
+        for (int mr = 0; mr < C::MR; ++mr) {
+          uint32_t aV[4];
+          ldsm_x4_t(aV, sl + tile_off<2 * R, KT>(16 * ks + rr + (mi >> 1) * 8, R + 16 * mr + (mi & 1) * 8));
+#pragma unroll
+          for (int pt = 0; pt < 2; ++pt) mma16816(Olr[mr][pt], aV, bP[pt][0], bP[pt][1]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(bar(B_PFREE));
+        mbar_arrive(bar(B_EMPTY + s));
+        if (n + ST < n_tiles) {   // the stage's refill once the P V MMA has read it
+          if (!mbar_wait(bar(B_EMPTY + s), (n / ST) & 1)) fail = 1;
+          issue(n + ST);
+          if (n + ST + kL2Ahead < n_tiles) prefetch(n + ST + kL2Ahead);
+        }
+      }
+      __syncwarp();
+    }
+    if (lane == 0)
+      for (int n = n_tiles; n < n_spec; ++n)   // loaded ahead of kv_len and not used
+        if (!mbar_wait(bar(B_FULL + n), 0)) fail = 1;
+    // the partial's O_lr (the UV area is free once every MMA has completed)
+    if (n_tiles > 0 && !mbar_wait(bar(B_ODONE), 0)) fail = 1;
+#pragma unroll
+    for (int mr = 0; mr < C::MR; ++mr)
+#pragma unroll
+      for (int pt = 0; pt < 2; ++pt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int row = 8 * pt + 2 * t4 + (e & 1);
+          const int rho = 16 * mr + (lane >> 2) + (e >> 1) * 8;
+          if (row < RP) Part[row * WP + D + rho] = Olr[mr][pt][e];
+        }
+  } else if (w == WM) {
+    // ======================================================== MMA warp
+    if (lane == 0 && n_tiles > 0) {
+      constexpr uint32_t ID_S = umma_idesc_bf16(128, QP, 0, 0);
+      constexpr uint32_t ID_W = umma_idesc_bf16(128, NW, 0, 0);
+      constexpr uint32_t ID_PV = umma_idesc_bf16(128, QP, 1, 0);   // O^T += V^T P^T, A = V MN-major
+      const uint64_t dQ = umma_desc(q_u, 16, 1024, 2);
+      const uint64_t dUV = umma_desc(uv_u, 16, 1024, 2);
+      const uint64_t dP = umma_desc(p_u, 16, 1024, 2);
+      auto mma_pv = [&](int m) {
+        if (!mbar_wait(bar(B_PFULL), m & 1)) fail = 1;
+        tc_fence_after();
+        const uint64_t dV = umma_desc(st_u + (m % ST) * C::STAGE + C::KV_TILE, KT * 128, 1024, 2);
+#pragma unroll
+        for (int kk = 0; kk < KT / 16; ++kk)
+          umma_bf16(tmem + T_O, umma_desc_add(dV, kk * 16 * 128),
+                    umma_desc_add(dP, (kk >> 2) * (QP * 128) + (kk & 3) * 32), ID_PV, (m > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(bar(B_PFREE));
+        umma_commit(bar(B_EMPTY + m % ST));
+      };
+      for (int n = 0; n < n_tiles; ++n) {
+        const int s = n % ST;
+        if (!mbar_wait(bar(B_FULL + s), (n / ST) & 1)) fail = 1;
+        if (n > 0 && !mbar_wait(bar(B_WFREE), (n - 1) & 1)) fail = 1;
+        if (!mbar_wait(bar(B_CSFULL), n & 1)) fail = 1;
+        tc_fence_after();
+        const uint64_t dK = umma_desc(st_u + s * C::STAGE, 16, 1024, 2);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_bf16(tmem + T_S, umma_desc_add(dK, (kk >> 2) * (KT * 128) + (kk & 3) * 32),
+                    umma_desc_add(dQ, (kk >> 2) * (QP * 128) + (kk & 3) * 32), ID_S, kk > 0);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_bf16_ts(tmem + T_W, tmem + T_CS + kk * 8,
+                       umma_desc_add(dUV, (kk >> 2) * (NW * 128) + (kk & 3) * 32), ID_W, kk > 0);
+        umma_commit(bar(B_TFULL));
+        if (n > 0) mma_pv(n - 1);
+      }
+      mma_pv(n_tiles - 1);
+      umma_commit(bar(B_ODONE));
+    }
+    __syncwarp();
+  }
+  if (fail) s_misc[0] = 1;
+  tc_fence_before();
+  __syncthreads();
+  if (w == WM) {
+    tc_fence_after();
+    tmem_dealloc(tmem, T_COLS);
+  }
+  if (bad_len) {
+    if (tid == 0 && split == 0) atomicOr(p.err, 1);
+    return;
+  }
+  for (int row = tid; row < RP; row += NTHR) {
+    Part[row * WP + D + R] = Mfin[row];
+    Part[row * WP + D + R + 1] = Lsum[row * 4] + Lsum[row * 4 + 1] + Lsum[row * 4 + 2] + Lsum[row * 4 + 3];
+  }
+  if (s_misc[0] && tid == 0) atomicOr(p.err, 2);
+  __syncthreads();
+
+  const __nv_bfloat16* bv = reinterpret_cast<const __nv_bfloat16*>(p.B_v) + (int64_t)agent0 * R * ldB + kvh * D;
+  // out[row][c..c+3] = (O + s O_lr B_v^a) / l from a merged row record
+  auto emit = [&](const float* rec, int row, int c) {
+    const int a = row / g, gi = row % g;
+    const float* ol = rec + D;
+    const __nv_bfloat16* bb = bv + (size_t)a * R * ldB + c;
+    float z0 = 0.f, z1 = 0.f, z2 = 0.f, z3 = 0.f;
+#pragma unroll
+    for (int j = 0; j < R; ++j) {
+      const float o = ol[j];
+      const uint2 b2 = __ldg(reinterpret_cast<const uint2*>(bb + j * ldB));
+      const float2 f01 = unpack_bf16(b2.x), f23 = unpack_bf16(b2.y);
+      z0 = fmaf(o, f01.x, z0); z1 = fmaf(o, f01.y, z1);
+      z2 = fmaf(o, f23.x, z2); z3 = fmaf(o, f23.y, z3);
+    }
+    const float l = rec[D + R + 1];
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    float4 acc = *reinterpret_cast<const float4*>(rec + c);
+    acc.x = fmaf(p.s, z0, acc.x) * inv; acc.y = fmaf(p.s, z1, acc.y) * inv;
+    acc.z = fmaf(p.s, z2, acc.z) * inv; acc.w = fmaf(p.s, z3, acc.w) * inv;
+    const int64_t oi = (((int64_t)seq * na_tot + agent0 + a) * p.n_q + kvh * g + gi) * D + c;
+    if (p.out_bf16) {
+      uint2 o;
+      o.x = pack_bf16(acc.x, acc.y);
+      o.y = pack_bf16(acc.z, acc.w);
+      *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(p.out) + oi) = o;
+    } else {
+      *reinterpret_cast<float4*>(reinterpret_cast<float*>(p.out) + oi) = acc;
+    }
+  };
+
+  if (ns == 1) {
+    if (s_misc[0]) return;
+    for (int i = tid; i < n_rows * (D / 4); i += NTHR) {
+      const int row = i / (D / 4), c = 4 * (i % (D / 4));
+      emit(Part + row * WP, row, c);
+    }
+    return;
+  }
+
+  // ---- split merge: a ticket per CTA; all but the last publish their partial
+  int* ctr = p.counters + unitg;
+  int* flags = p.counters + n_units_g + (size_t)unitg * kMaxSplits;
+  float* ws_unit = p.partials + (size_t)unitg * ns * RP * WP;
+  if (tid == 0) s_misc[1] = atomicAdd(ctr, 1);
+  __syncthreads();
+  if (s_misc[1] != ns - 1) {
+    float4* dst = reinterpret_cast<float4*>(ws_unit + (size_t)split * RP * WP);
+    for (int i = tid; i < RP * WP / 4; i += NTHR) __stcg(dst + i, reinterpret_cast<const float4*>(Part)[i]);
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) atomicExch(flags + split, 1);
+    return;
+  }
+  // the last CTA: every other split has taken its ticket; wait (bounded) until
+  // each has published, then merge
+  if (tid < ns && tid != split) {
+    int it = 0;
+    while (ld_acquire(flags + tid) == 0) {
+      if (++it > (1 << 22)) {
+        atomicOr(p.err, 4);
+        break;
+      }
+      __nanosleep(32);
+    }
+  }
+  __threadfence();
+  __syncthreads();
+  // this CTA's partial stays in shared memory; the others are read from L2
+  auto part = [&](int k, int row) -> const float* {
+    return k == split ? Part + row * WP : ws_unit + ((size_t)k * RP + row) * WP;
+  };
+  // (a) per row: M = max_k m_k, weights w_k = 2^(m_k - M) / sum_k 2^(m_k - M) l_k
+  float* Wt = reinterpret_cast<float*>(stages);     // [RP][kMaxSplits] (the stages are drained)
+  float* Mg = Wt + RP * kMaxSplits;                  // merged rows [RP][WP]
+  for (int row = w; row < n_rows; row += NTHR / 32) {
+    float2 ml = make_float2(-INFINITY, 0.f);
+    if (lane < ns) {
+      const float* pr = part(lane, row);
+      ml = lane == split ? make_float2(pr[D + R], pr[D + R + 1])
+                         : __ldcg(reinterpret_cast<const float2*>(pr + D + R));
+    }
+    const float M = warp_max(ml.x);
+    const float e = (lane < ns && ml.x != -INFINITY) ? fast_exp2(ml.x - M) : 0.f;
+    const float L = warp_sum(e * ml.y);
+    if (lane < ns) Wt[row * kMaxSplits + lane] = e;
+    if (lane == 0) Mg[row * WP + D + R + 1] = L;
+  }
+  __syncthreads();
+  // (b) merged O and O_lr, unnormalised (emit divides by L)
+  for (int i = tid; i < n_rows * ((D + R) / 4); i += NTHR) {
+    const int row = i / ((D + R) / 4), c = 4 * (i % ((D + R) / 4));
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int k = 0; k < ns; ++k) {
+      const float wk = Wt[row * kMaxSplits + k];
+      if (wk == 0.f) continue;
+      const float* pr = part(k, row) + c;
+      const float4 v = k == split ? *reinterpret_cast<const float4*>(pr) : __ldcg(reinterpret_cast<const float4*>(pr));
+      acc.x = fmaf(wk, v.x, acc.x); acc.y = fmaf(wk, v.y, acc.y);
+      acc.z = fmaf(wk, v.z, acc.z); acc.w = fmaf(wk, v.w, acc.w);
+    }
+    *reinterpret_cast<float4*>(Mg + row * WP + c) = acc;
+  }
+  __syncthreads();
+  if (!s_misc[0])
+    for (int i = tid; i < n_rows * (D / 4); i += NTHR) {
+      const int row = i / (D / 4), c = 4 * (i % (D / 4));
+      emit(Mg + row * WP, row, c);
+    }
+  // reset the unit's counter and flags for the next call on this workspace
+  if (tid < ns) flags[tid] = 0;
+  if (tid == 0) *ctr = 0;
+}
+
+// -------------------------------------------------------------------- host
+bool make_maps(const AttnParams& p, CUtensorMap* mk, CUtensorMap* mv, CUtensorMap* ml) {
+  auto enc = encode_fn();
+  if (!enc) return false;
+  const int R = p.r;
+  cuuint64_t kdims[4] = {(cuuint64_t)D, (cuuint64_t)p.L_max, (cuuint64_t)p.n_kv, (cuuint64_t)p.n_seqs};
+  cuuint64_t kstr[3] = {(cuuint64_t)p.kv_tok * 2, (cuuint64_t)p.kv_head * 2, (cuuint64_t)p.kv_seq * 2};
+  cuuint32_t kbox[4] = {64, (cuuint32_t)KT, 1, 1};
+  cuuint32_t one[4] = {1, 1, 1, 1};
+  if (enc(mk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(p.k_base), kdims, kstr, kbox, one,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  if (enc(mv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(p.v_base), kdims, kstr, kbox, one,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  const int lb = 2 * R < 64 ? 2 * R : 64;
+  const int64_t n_lr = p.lr_agent ? p.n_agents : 1;
+  const int64_t lr_agent_b = p.lr_agent ? p.lr_agent * 2 : p.lr_seq * 2 * p.n_seqs;
+  cuuint64_t ldims[4] = {(cuuint64_t)(2 * R), (cuuint64_t)p.L_max, (cuuint64_t)p.n_seqs, (cuuint64_t)n_lr};
+  cuuint64_t lstr[3] = {(cuuint64_t)(2 * R * 2), (cuuint64_t)p.lr_seq * 2, (cuuint64_t)lr_agent_b};
+  cuuint32_t lbox[4] = {(cuuint32_t)lb, (cuuint32_t)KT, 1, 1};
+  if (enc(ml, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(p.lr), ldims, lstr, lbox, one,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(lb * 2), CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  return true;
+}
+
+int device_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) {
+    cudaGetLastError();
+    return kSMs;
+  }
+  return n;
+}
+
+// padded rows of a group of G agents (a multiple of 4), 0 if no instance holds it
+int rows_padded(const AttnParams& p, int G) {
+  const int rows = G * p.g;
+  const int rp = (rows + 3) / 4 * 4;
+  if (p.r == 16) return rp <= 16 ? rp : 0;
+  if (p.r == 32) return rp <= 4 ? rp : 0;
+  return 0;
+}
+
+size_t smem_of(int r, int rp) {
+  if (r == 32) return Cfg<32, 4>::smem();
+  switch (rp) {
+    case 4: return Cfg<16, 4>::smem();
+    case 8: return Cfg<16, 8>::smem();
+    case 12: return Cfg<16, 12>::smem();
+    default: return Cfg<16, 16>::smem();
+  }
+}
+
+template <int R, int RP>
+cudaError_t launch_t(const AttnParams& p, cudaStream_t st) {
+  using Cf = Cfg<R, RP>;
+  RopeTheta rt;
+  for (int i = 0; i < 64; ++i) {
+    rt.theta[i] = i < D / 2 ? std::pow(p.rope_base, -2.0 * i / D) : 0.0;
+    rt.thetaf[i] = (float)rt.theta[i];
+  }
+  CUtensorMap mk, mv, ml;
+  if (!make_maps(p, &mk, &mv, &ml)) return cudaErrorInvalidValue;
+  const size_t sm = Cf::smem();
+  auto kern = decode_cs_kernel<R, RP>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.n_splits, (p.n_agents + p.agent_group - 1) / p.agent_group, p.n_seqs * p.n_kv);
+  cfg.blockDim = dim3(NTHR);
+  cfg.dynamicSmemBytes = sm;
+  cfg.stream = st;
+  // the set-up may overlap the preceding kernel (programmatic dependent launch;
+  // the kernel waits for it before reading any input)
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, mk, mv, ml, p, rt);
+  if (e != cudaSuccess) {   // without the overlap where the runtime refuses it
+    cudaGetLastError();
+    cfg.numAttrs = 0;
+    e = cudaLaunchKernelEx(&cfg, kern, mk, mv, ml, p, rt);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+// Agents per CTA of the cos/sin-table decode (0: the shape does not run on
+// it): the largest group whose padded rows fit an instance and whose shared
+// memory fits; one LR cache per agent takes one agent per CTA.
+int cs_group_size(const AttnParams& p) {
+  if (p.d != 128 || !(p.r == 16 || p.r == 32)) return 0;
+  if (!(p.g == 1 || p.g == 2 || p.g == 4 || p.g == 8)) return 0;
+  if (p.L_max >= (1ll << 31)) return 0;
+  const int gmax = p.lr_agent ? 1 : 4;
+  for (int G = p.n_agents < gmax ? p.n_agents : gmax; G >= 1; --G) {
+    const int rp = rows_padded(p, G);
+    if (rp && smem_of(p.r, rp) <= 227 * 1024) return G;
+  }
+  return 0;
+}
+
+// Splits of each (sequence, KV head, agent group) over the keys.  Fewer units
+// than SMs: one wave, as many splits as keep every SM busy (but as few as give
+// the same longest split).  More: the split count (up to 4) whose waves are
+// fullest, so that the last wave does not leave most SMs idle.
+int cs_splits(const AttnParams& p, int G) {
+  const int groups = (p.n_agents + G - 1) / G;
+  const int units = p.n_seqs * p.n_kv * groups;
+  if (units < 1) return 1;
+  const int64_t total_tiles = (p.max_kv_len + KT - 1) / KT;
+  const int sms = device_sms();
+  int64_t ns;
+  if (units < sms) {
+    ns = sms / units;
+    if (ns > kMaxSplits) ns = kMaxSplits;
+    if (ns > total_tiles) ns = total_tiles;
+    if (ns < 1) ns = 1;
+    const int64_t per = (total_tiles + ns - 1) / ns;
+    ns = (total_tiles + per - 1) / per;
+  } else {
+    double best = -1.0;
+    ns = 1;
+    for (int s = 1; s <= 4 && s * 8 <= total_tiles; ++s) {
+      const int64_t ctas = (int64_t)units * s;
+      const int64_t waves = (ctas + sms - 1) / sms;
+      const double eff = (double)ctas / (double)(waves * sms) - 0.01 * s;
+      if (eff > best) {
+        best = eff;
+        ns = s;
+      }
+    }
+  }
+  return (int)ns;
+}
+
+cudaError_t launch_decode_cs(const AttnParams& pin, la_dtype out, cudaStream_t st) {
+  AttnParams p = pin;
+  p.out_bf16 = out == LA_BF16;
+  p.agent_group = cs_group_size(p);
+  if (p.agent_group < 1) return cudaErrorInvalidValue;
+  if (p.n_splits > kMaxSplits) return cudaErrorInvalidValue;
+  if (p.r == 32) return launch_t<32, 4>(p, st);
+  switch (rows_padded(p, p.agent_group)) {
+    case 4: return launch_t<16, 4>(p, st);
+    case 8: return launch_t<16, 8>(p, st);
+    case 12: return launch_t<16, 12>(p, st);
+    default: return launch_t<16, 16>(p, st);
+  }
+}
+
+// Workspace of the cos/sin-table decode: per (agent group, unit) its splits'
+// partials [splits][rows padded][d + r + 4] fp32, then one arrival counter per
+// (group, unit) and a flag per split.
+size_t cs_partial_bytes(const AttnParams& p) {
+  const int G = cs_group_size(p);
+  if (G < 1) return 0;
+  const int ns = cs_splits(p, G);
+  if (ns == 1) return 0;
+  const int groups = (p.n_agents + G - 1) / G;
+  return (size_t)p.n_seqs * p.n_kv * groups * ns * rows_padded(p, G) * (p.d + p.r + 4) * sizeof(float);
+}
+
+size_t cs_counter_ints(const AttnParams& p) {
+  const int G = cs_group_size(p);
+  if (G < 1) return 0;
+  const int groups = (p.n_agents + G - 1) / G;
+  return (size_t)p.n_seqs * p.n_kv * groups * (1 + kMaxSplits);
+}
+
+}  // namespace la

@@ -297,6 +297,18 @@ __device__ __forceinline__ void tmem_st32x32b_x32(uint32_t taddr, const uint32_t
                : "memory");
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+// 32 TMEM lanes x 1 column: thread t gets / puts lane t of one column
+__device__ __forceinline__ uint32_t tmem_ld32x32b_x1(uint32_t taddr) {
+  uint32_t r;
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
+  return r;
+}
+__device__ __forceinline__ void tmem_st32x32b_x1(uint32_t taddr, uint32_t v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void tmem_wait_ld_r1(uint32_t& r) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" : "+r"(r) : : "memory");
+}
 // 16 TMEM lanes x 8 columns: thread t gets lanes t/4 and t/4+8, columns 2(t%4), 2(t%4)+1
 // (the mma.sync m16n8 accumulator layout); .x2 repeats over the next 8 columns.
 __device__ __forceinline__ void tmem_ld16x256_x1(uint32_t (&r)[4], uint32_t taddr) {

@@ -82,17 +82,18 @@ def test_static_scratch_after_a_larger_call_clears_its_counters(la):
         a = la.make_args(d["k_base"], d["v_base"], d["lr"], d["B_k"], d["B_v"], d["q"], out,
                          lora_scale=s.lora_scale, rope_base=s.rope_base, kv_len=d["kv_len"],
                          max_kv_len=s.kv_len)
-        outs.append((s, inp, out, a, la.lora_attn_decode_workspace_bytes(a)))
-    (_, _, _, a_big, need_big), (_, _, _, a_small, _) = outs
+        # d stays referenced: the arguments hold raw pointers into its tensors
+        outs.append((s, inp, out, a, la.lora_attn_decode_workspace_bytes(a), d))
+    (_, _, _, a_big, need_big, _), (_, _, _, a_small, _, _) = outs
     # the small decode's counters start before the big decode's scratch ends
     assert need_big > 0 and la.lora_attn_decode_workspace_bytes(a_small) < need_big
-    for s, inp, out, a, _ in outs:
+    for s, inp, out, a, _, _ in outs:
         st = la.lib.lora_attn_decode_static_scratch(ctypes.byref(a),
                                                     torch.cuda.current_stream().cuda_stream)
         assert st == la.LA_OK, la.status_string(st)
     torch.cuda.synchronize()
     assert la.la_device_check() == la.LA_OK
-    for s, inp, out, _, _ in outs:
+    for s, inp, out, _, _, _ in outs:
         assert_parity(to_np(out), oracle_decode(inp, s), s.dtype)
 
 
