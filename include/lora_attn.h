@@ -368,9 +368,12 @@ la_status lora_attn_decode_static_scratch(const la_attn_args* args, la_stream_t 
  *   LA_DEV_PIPE_WAIT  a tensor-core kernel's wait on its copy/MMA pipeline
  *                     gave up after its iteration limit (the CTA skipped its
  *                     output and, holding TMEM, freed it)
- *   LA_DEV_MERGE_WAIT a decode CTA's wait for the other splits of its unit
- *                     gave up after its iteration limit (about a second);
- *                     that unit's output is not to be trusted
+ *   LA_DEV_MERGE_WAIT the split merge of a decode unit failed: a wait for
+ *                     another split of the unit gave up after its iteration
+ *                     limit (about a second), or the unit's arrival counter
+ *                     held a value no call leaves there (a workspace not
+ *                     zero-filled before its first use); that unit's output
+ *                     is not to be trusted and may be left unwritten
  * No check traps: every kernel returns and the context stays usable.
  */
 #define LA_DEV_KV_LEN 1

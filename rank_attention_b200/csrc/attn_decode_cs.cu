@@ -632,7 +632,12 @@ __global__ void __launch_bounds__(NTHR, 1)
   float* ws_unit = p.partials + (size_t)unitg * ns * RP * WP;
   if (tid == 0) s_misc[1] = atomicAdd(ctr, 1);
   __syncthreads();
-  if (s_misc[1] != ns - 1) {
+  const int ticket = s_misc[1];
+  if (ticket < 0 || ticket >= ns) {   // a counter no call leaves behind: not a zeroed workspace
+    if (tid == 0) atomicOr(p.err, 4);
+    return;
+  }
+  if (ticket != ns - 1) {
     float4* dst = reinterpret_cast<float4*>(ws_unit + (size_t)split * RP * WP);
     for (int i = tid; i < RP * WP / 4; i += NTHR) __stcg(dst + i, reinterpret_cast<const float4*>(Part)[i]);
     __threadfence();

@@ -41,6 +41,13 @@ namespace {
 
 using namespace ptx;
 
+// bf16 pair + fp32 pair, rounded once to an fp16 pair (the K^a operand)
+__device__ __forceinline__ uint32_t add_to_f16x2(uint32_t base_bf16x2, float2 d) {
+  const float2 b = unpack_bf16(base_bf16x2);
+  __half2 h = __floats2half2_rn(b.x + d.x, b.y + d.y);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
 constexpr int PD = 128;                  // head_dim
 constexpr int PKT = 128;                 // keys per tile
 constexpr int PM = 128;                  // query rows per CTA
@@ -227,7 +234,7 @@ __global__ void __launch_bounds__(PNTHR, 1)
     // ============================================================ TMA / MMA warp
     if (lane == 0 && work) {
       constexpr uint32_t ID_DK = umma_idesc_bf16(128, PD, 0, 1);
-      constexpr uint32_t ID_S = umma_idesc_bf16(128, PKT, 0, 0);
+      constexpr uint32_t ID_S = umma_idesc_f16(128, PKT, 0, 0);   // Q and K^a in fp16
       constexpr uint32_t ID_PV = umma_idesc_bf16(128, PD, 0, 1);
       constexpr uint32_t ID_PL = umma_idesc_bf16(128, R, 0, 1);
       // operand descriptors of stage 0; the others are fixed byte offsets on
@@ -350,8 +357,8 @@ __global__ void __launch_bounds__(PNTHR, 1)
             const float2 z1 = f2_unpack(sub_f2(mul_f2(ac, y1), mul_f2(as, y2)));   // s R(k0) y
             const float2 z2 = f2_unpack(fma_f2(ac, y2, mul_f2(as, y1)));
             const uint32_t o1 = rowb + hh * 1024 + cx, o2 = o1 + PKT * 128;
-            sts32(o1, add_bf16x2(lds32(o1), pack_bf16(z1.x, z1.y)));
-            sts32(o2, add_bf16x2(lds32(o2), pack_bf16(z2.x, z2.y)));
+            sts32(o1, add_to_f16x2(lds32(o1), z1));
+            sts32(o2, add_to_f16x2(lds32(o2), z2));
           }
         }
       }
@@ -459,7 +466,22 @@ __global__ void __launch_bounds__(PNTHR, 1)
       if (lane == 0) mbar_arrive(pfull);
     };
 
-    if (work) build(0);
+    if (work) {
+      // the queries to fp16 in place: the S MMA takes Q and K^a in fp16, whose
+      // 11-bit significand keeps the rounding of K^a = K_base + delta small
+      // against |K| (bf16 values convert exactly within fp16's range)
+      if (!mbar_wait(qbar, 0)) fail = 1;
+      for (int i = tid; i < C::Q_BYTES / 16; i += 32 * PNC) {
+        uint4* qp = reinterpret_cast<uint4*>(smem + C::OFF_Q) + i;
+        uint4 v = *qp;
+        v.x = add_to_f16x2(v.x, make_float2(0.f, 0.f));
+        v.y = add_to_f16x2(v.y, make_float2(0.f, 0.f));
+        v.z = add_to_f16x2(v.z, make_float2(0.f, 0.f));
+        v.w = add_to_f16x2(v.w, make_float2(0.f, 0.f));
+        *qp = v;
+      }
+      build(0);   // its proxy fence also covers the queries
+    }
     for (int i = 0; i < NT; ++i) {
       bar_sync(PBAR_CW, 32 * PNC);  // anchors of tile i+1 are in place
       if (i + 1 < NT) build(i + 1);
