@@ -43,9 +43,6 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--all-configs", action="store_true",
-                    help="also time the long-context decode sweep and one layer of the "
-                         "32-layer stack (decode and prefill), reported under other_configs")
     ap.add_argument("--profile", nargs="?", const="decode",
                     choices=["decode", "prefill", "append", "qkvo"],
                     help="a short deterministic run of one kernel for profilers "
@@ -365,6 +362,163 @@ def time_other_configs(dev):
     return res
 
 
+STACK_STEPS = 16   # decode steps per layer after the chunk's prefill
+
+
+class StackLayer:
+    """One layer of the 32-layer stack workload (4 agents, r = 64, hidden 4096):
+    the PreLRShared append of a 4096-token chunk, the prefill of that chunk
+    over the 32768-token prefix, then STACK_STEPS decode steps, each appending
+    its token's LR row and attending over prefix + chunk + the steps so far.
+    Inputs are drawn on the device from the layer's own seed; the base K/V
+    rows of the decode tokens are drawn like the cache (the base model's).
+    Calls queue on the current stream; tensors live as long as the object."""
+
+    def __init__(self, layer: int, dev, pf_out=None, dec_out=None):
+        import torch
+        from rank_attention_b200 import lora_attn as la
+        from rank_attention_b200 import workloads as W
+        s = W.llama8b_stack_prefill(layer)
+        self.shape, self.layer = s, layer
+        n_pre, n_chunk = s.kv_len - s.n_q_tokens, s.n_q_tokens
+        L_max = s.kv_len + STACK_STEPS
+        inp = W.direct_cache_inputs(s, device=dev, L_max=L_max)
+        g = torch.Generator(device=dev)
+        g.manual_seed(s.seed + 500)
+        for k in ("k_base", "v_base"):
+            inp[k][:, :, s.kv_len:] = (W.CACHE_STD * torch.randn(
+                inp[k][:, :, s.kv_len:].shape, generator=g, device=dev)).to(s.dtype)
+        ch = W.append_inputs(n_chunk, s.hidden, s.r, s.dtype, seed=s.seed + 600, device=dev)
+        xs = W.append_inputs(STACK_STEPS, s.hidden, s.r, s.dtype, seed=s.seed + 700, device=dev)["X"]
+        q_dec = (W.CACHE_STD * torch.randn((STACK_STEPS, 1, s.n_agents, 1, s.n_q_heads, s.head_dim),
+                                           generator=g, device=dev)).to(s.dtype)
+        self.pf_out = pf_out if pf_out is not None else torch.empty(inp["q"].shape, dtype=s.dtype,
+                                                                    device=dev)
+        self.dec_out = dec_out if dec_out is not None else torch.empty(
+            (STACK_STEPS,) + tuple(q_dec.shape[1:]), dtype=torch.float32, device=dev)
+        self.kv_lens = [torch.full((1,), s.kv_len + t + 1, dtype=torch.int32, device=dev)
+                        for t in range(STACK_STEPS)]
+        self.inp, self.chunk, self.xs, self.q_dec = inp, ch, xs, q_dec
+        self.n_pre, self.n_chunk = n_pre, n_chunk
+        self.pf_args = la.make_args(inp["k_base"], inp["v_base"], inp["lr"], inp["B_k"], inp["B_v"],
+                                    inp["q"], self.pf_out, lora_scale=s.lora_scale,
+                                    rope_base=s.rope_base, q_pos0=n_pre)
+        self.dec_args = [la.make_args(inp["k_base"], inp["v_base"], inp["lr"], inp["B_k"],
+                                      inp["B_v"], q_dec[t], self.dec_out[t],
+                                      lora_scale=s.lora_scale, rope_base=s.rope_base,
+                                      kv_len=self.kv_lens[t], max_kv_len=L_max)
+                         for t in range(STACK_STEPS)]
+        self.ws = la.decode_workspace(self.dec_args[0], dev)
+
+    def append(self, stream=None):
+        from rank_attention_b200 import lora_attn as la
+        la.lr_cache_append(self.chunk["X"], self.chunk["A_kv"], self.inp["lr"], self.n_pre, stream)
+
+    def prefill(self, stream=None):
+        from rank_attention_b200 import lora_attn as la
+        la.lora_attn_prefill(self.pf_args, stream)
+
+    def decode_step(self, t: int, stream=None):
+        from rank_attention_b200 import lora_attn as la
+        la.lr_cache_append(self.xs[:, t:t + 1], self.chunk["A_kv"], self.inp["lr"],
+                           self.shape.kv_len + t, stream)
+        la.lora_attn_decode(self.dec_args[t], self.ws, stream)
+
+    def run(self, stream=None):
+        self.append(stream)
+        self.prefill(stream)
+        for t in range(STACK_STEPS):
+            self.decode_step(t, stream)
+
+
+def time_stack(dev, reps=3):
+    """The full 32-layer stack (append, prefill, STACK_STEPS decode steps per
+    layer) in one CUDA graph, and each phase alone over all 32 layers; per-step
+    and per-token figures across the 32 layers.  The stack's inputs (about
+    11 GB) exceed L2 many times over."""
+    import torch
+    from rank_attention_b200 import lora_attn as la
+    from rank_attention_b200 import workloads as W
+    pf_out = dec_out = None
+    layers = []
+    for l in range(W.STACK_LAYERS):
+        layers.append(StackLayer(l, dev, pf_out, dec_out))
+        pf_out, dec_out = layers[0].pf_out, layers[0].dec_out   # outputs shared, not read
+    st = torch.cuda.Stream(device=dev)
+    torch.cuda.synchronize()
+
+    def graph(fn):
+        with torch.cuda.stream(st):
+            fn()   # warm-up, outside the capture
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=st):
+            fn()
+        return g
+
+    def timed(g):
+        ts = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(st):
+                e0.record(st)
+                g.replay()
+                e1.record(st)
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1))
+        return statistics.median(ts)
+
+    def all_layers(f):
+        def fn():
+            for L in layers:
+                f(L)
+        return fn
+
+    g_all = graph(all_layers(lambda L: L.run(st)))
+    g_app = graph(all_layers(lambda L: L.append(st)))
+    g_pf = graph(all_layers(lambda L: L.prefill(st)))
+    g_dec = graph(all_layers(lambda L: [L.decode_step(t, st) for t in range(STACK_STEPS)]))
+    ms_all, ms_app, ms_pf, ms_dec = timed(g_all), timed(g_app), timed(g_pf), timed(g_dec)
+    if la.la_device_check() != 0:
+        raise RuntimeError("stack device check failed")
+    del g_all, g_app, g_pf, g_dec
+    s = layers[0].shape
+    nl = len(layers)
+    base, lora = prefill_flops(s)
+    tc, tc_kind = tc_peak()
+    hbm, _ = peaks()
+    dec_step_ms = ms_dec / STACK_STEPS                        # one decode step, all layers
+    kv_mid = s.kv_len + STACK_STEPS // 2
+    dshape = s.replace(kv_len=kv_mid, n_q_tokens=1, mode="decode")
+    dbytes = decode_bytes(dshape) + append_bytes(dshape, 1)
+    abytes = append_bytes(s, s.n_q_tokens)
+    res = {
+        "workload": f"{nl}-layer stack: per layer append of a {s.n_q_tokens}-token chunk (r = {s.r}), "
+                    f"its prefill over {s.kv_len - s.n_q_tokens} + {s.n_q_tokens} keys, "
+                    f"{STACK_STEPS} decode steps of {s.n_agents} agents (append + decode)",
+        "layers": nl, "decode_steps": STACK_STEPS,
+        "stack_ms": ms_all, "append_ms": ms_app, "prefill_ms": ms_pf, "decode_ms": ms_dec,
+        "append_per_layer_us": ms_app / nl * 1e3,
+        "append_GB/s": abytes * nl / (ms_app / 1e3) / 1e9,
+        "append_frac": abytes * nl / (ms_app / 1e3) / 1e9 / hbm,
+        "prefill_per_layer_ms": ms_pf / nl,
+        "prefill_TFLOP/s": base * nl / (ms_pf / 1e3) / 1e12,
+        "prefill_frac": base * nl / (ms_pf / 1e3) / 1e12 / tc,
+        "decode_step_all_layers_us": dec_step_ms * 1e3,
+        "decode_step_per_layer_us": dec_step_ms / nl * 1e3,
+        "decode_agent_tokens_per_s": s.n_agents / (dec_step_ms / 1e3),
+        "decode_GB/s": dbytes * nl / (dec_step_ms / 1e3) / 1e9,
+        "decode_frac": dbytes * nl / (dec_step_ms / 1e3) / 1e9 / hbm,
+        "peaks": {"hbm_GB/s": hbm, "bf16_TFLOP/s": tc, "tc_kind": tc_kind},
+        "timing": f"CUDA graphs over all {nl} layers, median of {reps} replays, CUDA events",
+        "what": "decode_agent_tokens_per_s: agent tokens through all layers per second "
+                "(n_agents / one decode step over the stack); decode bytes: base K, V and LR "
+                "read once per layer and step plus the step's append"}
+    del layers
+    torch.cuda.empty_cache()
+    return res
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle sampling during the timed region."""
 
@@ -540,6 +694,36 @@ def kv_cache_report(s) -> dict:
 
 def append_bytes(s, n_tok: int) -> int:
     return s.n_seqs * (n_tok * s.hidden * 2 + n_tok * 2 * s.r * 2) + s.hidden * 2 * s.r * 2
+
+
+def time_oracle_tiny(reps: int = 50) -> dict:
+    """The oracle on the tiny fp32 case (one decode step from hidden states:
+    base cache, LR rows, attention), on one host thread and on all of them."""
+    from threadpoolctl import threadpool_limits
+    from oracle import impl as oracle
+    from rank_attention_b200 import workloads as W
+    s = W.TINY_FP32
+    w = W.hidden_layer_weights(s)
+
+    def step():
+        kb, vb = oracle.base_cache_from_hidden(w["X"], w["W_k"], w["W_v"], s.n_kv_heads, s.rope_base)
+        lr = oracle.lr_cache_rows(w["X"], w["A_kv"])
+        oracle.lora_attention(kb, vb, lr, w["B_k"], w["B_v"], w["q"], [s.kv_len],
+                              lora_scale=s.lora_scale, softmax_scale=s.softmax_scale,
+                              rope_base=s.rope_base, mode="decode")
+
+    res = {"workload": s.name}
+    for label, limit in (("one_thread", 1), ("all_threads", None)):
+        with threadpool_limits(limits=limit):
+            step()
+            t0 = time.perf_counter()
+            for _ in range(reps):
+                step()
+            per = (time.perf_counter() - t0) / reps
+        res[label] = {"ms_per_step": per * 1e3,
+                      "agent_tokens_per_s": s.n_seqs * s.n_agents / per}
+    res["cores_all"] = blas_threads()
+    return res
 
 
 def oracle_step(inp, new, s):
@@ -794,13 +978,14 @@ def run_ours(args):
         "qkvo": qkvo,
         "value_ablation": value_ablation,
     }
-    if args.all_configs:
-        line["other_configs"] = time_other_configs(dev)
+    line["other_configs"] = time_other_configs(dev)
+    line["stack"] = time_stack(dev)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, n, per = time_oracle(s, 20, 15.0)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": blas_threads(),
                                 "kind": "oracle",
-                                "sample": f"{n} full decode steps of {s.name} on the host"}
+                                "sample": f"{n} full decode steps of {s.name} on the host",
+                                "tiny_fp32": time_oracle_tiny()}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -288,7 +288,14 @@ __global__ void __launch_bounds__(NTHR, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
+  // Every wait is bounded in time.  After one has run out, a thread skips its
+  // later waits but keeps every arrive, commit and named barrier of its role,
+  // so the other roles finish too (their own waits may run out once) and the
+  // CTA reaches its end quickly, reporting the failure.
   int fail = 0;
+  auto wt = [&](int b, uint32_t parity) {
+    if (!fail && !mbar_wait_ns(bar(b), parity)) fail = 1;
+  };
   const float sl2 = p.scale * kLog2e;
 
   // CS of tile n into TMEM: lane j, columns 16 hh.. (cos) and 32 + 16 hh.. (sin)
@@ -325,8 +332,8 @@ __global__ void __launch_bounds__(NTHR, 1)
       const int s = n % ST;
       const int64_t k0 = k_lo + (int64_t)n * KT;
       const bool valid = k0 + jk < k_hi;
-      if (!mbar_wait(bar(B_FULL + s), (n / ST) & 1)) fail = 1;
-      if (!mbar_wait(bar(B_TFULL), n & 1)) fail = 1;
+      wt(B_FULL + s, (n / ST) & 1);
+      wt(B_TFULL, n & 1);
       tc_fence_after();
       // S (every row), this half's W columns, this key's LRk
       uint32_t sv[16];
@@ -395,7 +402,7 @@ __global__ void __launch_bounds__(NTHR, 1)
         if (sp == 0 && lane == 0) Corr[(n & 1) * QP + hh * RH + r] = corr[r];
       }
       // P V and O_lr of the previous tile are done: P is free, O^T is final
-      if (n > 0 && !mbar_wait(bar(B_PFREE), (n - 1) & 1)) fail = 1;
+      if (n > 0) wt(B_PFREE, (n - 1) & 1);
       if (moved && n > 0) {   // O^T (TMEM lanes = d, columns = rows) times corr
         tc_fence_after();
 #pragma unroll
@@ -429,7 +436,7 @@ __global__ void __launch_bounds__(NTHR, 1)
     }
     uint32_t ov[16];
     if (n_tiles > 0) {
-      if (!mbar_wait(bar(B_ODONE), 0)) fail = 1;
+      wt(B_ODONE, 0);
       tc_fence_after();
       tmem_ld32x32b_x16(ov, tmem + T_O + lane_off);
       tmem_wait_ld_r16(ov);
@@ -451,13 +458,15 @@ __global__ void __launch_bounds__(NTHR, 1)
 #pragma unroll
         for (int e = 0; e < 4; ++e) Olr[mr][pt][e] = 0.f;
     const int mi = lane >> 3, rr = lane & 7, t4 = lane & 3;
+    int n_issued = n_spec, n_seen = 0;   // tiles requested / observed landed (lane 0)
     if (lane == 0)
       for (int m = ST; m < n_tiles && m < ST + kL2Ahead; ++m) prefetch(m);
     for (int n = 0; n < n_tiles; ++n) {
       const int s = n % ST;
       const int64_t k0 = k_lo + (int64_t)n * KT;
       unsigned char* sb = stages + s * C::STAGE;
-      if (!mbar_wait(bar(B_FULL + s), (n / ST) & 1)) fail = 1;
+      wt(B_FULL + s, (n / ST) & 1);
+      if (lane == 0 && !fail) n_seen = n + 1;
       if (k0 + KT > k_hi) {   // P is 0 there; zeroed rows keep stale NaN out of P V
         const int first = (int)(k_hi - k0);
         for (int i = lane; i < (KT - first) * (D / 8); i += 32) {
@@ -472,7 +481,7 @@ __global__ void __launch_bounds__(NTHR, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(B_PFULL));
-      if (!mbar_wait(bar(B_PFULL), n & 1)) fail = 1;
+      wt(B_PFULL, n & 1);
 #pragma unroll
       for (int pt = 0; pt < 2; ++pt) {
         const float c0 = Corr[(n & 1) * QP + 8 * pt + 2 * t4];
@@ -503,18 +512,23 @@ __global__ void __launch_bounds__(NTHR, 1)
         mbar_arrive(bar(B_PFREE));
         mbar_arrive(bar(B_EMPTY + s));
         if (n + ST < n_tiles) {   // the stage's refill once the P V MMA has read it
-          if (!mbar_wait(bar(B_EMPTY + s), (n / ST) & 1)) fail = 1;
-          issue(n + ST);
-          if (n + ST + kL2Ahead < n_tiles) prefetch(n + ST + kL2Ahead);
+          wt(B_EMPTY + s, (n / ST) & 1);
+          if (!fail) {
+            issue(n + ST);
+            n_issued = n + ST + 1;
+            if (n + ST + kL2Ahead < n_tiles) prefetch(n + ST + kL2Ahead);
+          }
         }
       }
       __syncwarp();
     }
+    // every requested tile lands before the CTA leaves: those loaded ahead of
+    // kv_len and not used, and those still in flight after a wait ran out
     if (lane == 0)
-      for (int n = n_tiles; n < n_spec; ++n)   // loaded ahead of kv_len and not used
-        if (!mbar_wait(bar(B_FULL + n), 0)) fail = 1;
+      for (int m = max(n_seen, n_issued - ST); m < n_issued; ++m)
+        if (!mbar_wait_ns(bar(B_FULL + m % ST), (m / ST) & 1)) fail = 1;
     // the partial's O_lr (the UV area is free once every MMA has completed)
-    if (n_tiles > 0 && !mbar_wait(bar(B_ODONE), 0)) fail = 1;
+    if (n_tiles > 0) wt(B_ODONE, 0);
 #pragma unroll
     for (int mr = 0; mr < C::MR; ++mr)
 #pragma unroll
@@ -535,7 +549,7 @@ __global__ void __launch_bounds__(NTHR, 1)
       const uint64_t dUV = umma_desc(uv_u, 16, 1024, 2);
       const uint64_t dP = umma_desc(p_u, 16, 1024, 2);
       auto mma_pv = [&](int m) {
-        if (!mbar_wait(bar(B_PFULL), m & 1)) fail = 1;
+        wt(B_PFULL, m & 1);
         tc_fence_after();
         const uint64_t dV = umma_desc(st_u + (m % ST) * C::STAGE + C::KV_TILE, KT * 128, 1024, 2);
 #pragma unroll
@@ -547,9 +561,9 @@ __global__ void __launch_bounds__(NTHR, 1)
       };
       for (int n = 0; n < n_tiles; ++n) {
         const int s = n % ST;
-        if (!mbar_wait(bar(B_FULL + s), (n / ST) & 1)) fail = 1;
-        if (n > 0 && !mbar_wait(bar(B_WFREE), (n - 1) & 1)) fail = 1;
-        if (!mbar_wait(bar(B_CSFULL), n & 1)) fail = 1;
+        wt(B_FULL + s, (n / ST) & 1);
+        if (n > 0) wt(B_WFREE, (n - 1) & 1);
+        wt(B_CSFULL, n & 1);
         tc_fence_after();
         const uint64_t dK = umma_desc(st_u + s * C::STAGE, 16, 1024, 2);
 #pragma unroll
@@ -565,6 +579,9 @@ __global__ void __launch_bounds__(NTHR, 1)
       }
       mma_pv(n_tiles - 1);
       umma_commit(bar(B_ODONE));
+      // TMEM is freed below: every MMA has completed first (an MMA always
+      // completes, so this wait does not run out)
+      if (!mbar_wait_ns(bar(B_ODONE), 0)) fail = 1;
     }
     __syncwarp();
   }

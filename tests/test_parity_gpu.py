@@ -477,6 +477,45 @@ def test_llama8b_stack_decode_full(la, layer):
     assert_parity(to_np(got), oracle_decode(inp, s), s.dtype)
 
 
+@pytest.mark.parametrize("layer", [0, 15, 31])
+def test_llama8b_stack_layer_append_and_decode_steps(la, layer):
+    """Layers 0, 15 and 31 of the 32-layer stack as the bench runs them: the
+    chunk's LR rows appended (X A), then every one of the decode steps appends
+    its token's row and attends over prefix + chunk + the steps so far.  The
+    oracle forms the LR rows from X and A itself (fp64); two (agent, KV head)
+    units are checked at every step, every agent and head over the steps."""
+    import bench
+    L = bench.StackLayer(layer, DEV)
+    s = L.shape
+    L.append()
+    outs = []
+    for t in range(bench.STACK_STEPS):
+        L.decode_step(t)
+        outs.append(L.dec_out[t].clone())
+    torch.cuda.synchronize()
+    assert la.la_device_check() == 0
+    lr = oracle.lr_cache_append(L.inp["lr"][:, :s.kv_len].cpu(), L.chunk["X"].cpu(),
+                                L.chunk["A_kv"].cpu(), L.n_pre)
+    steps = oracle.lr_cache_rows(L.xs.cpu(), L.chunk["A_kv"].cpu())      # [1, steps, 2r]
+    lr = np.concatenate([lr, steps], axis=1)
+    kb, vb = L.inp["k_base"].cpu(), L.inp["v_base"].cpu()
+    g = s.group
+    gots, refs = [], []
+    for t in range(bench.STACK_STEPS):
+        kvl = s.kv_len + t + 1
+        q = L.q_dec[t].cpu()
+        for u in range(2):
+            agent = (t + 2 * u + layer) % s.n_agents
+            kvh = (3 * t + 5 * u + layer) % s.n_kv_heads
+            refs.append(oracle.lora_attention_unit(kb, vb, lr, L.inp["B_k"].cpu(), L.inp["B_v"].cpu(),
+                                                   q, seq=0, agent=agent, kv_head=kvh, kv_len=kvl,
+                                                   q_positions=[kvl - 1], lora_scale=s.lora_scale,
+                                                   softmax_scale=s.softmax_scale,
+                                                   rope_base=s.rope_base))
+            gots.append(to_np(outs[t][0, agent][:, kvh * g:(kvh + 1) * g]))
+    assert_parity(np.stack(gots), np.stack(refs), s.dtype)
+
+
 @pytest.mark.parametrize("ctx", W.SWEEP_CTX)
 def test_llama8b_sweep_decode_sampled(la, ctx):
     """The batched long-context decode (16 requests x 5 agents, r = 32) at
