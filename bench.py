@@ -847,8 +847,7 @@ def run_ours(args):
         out = torch.empty(inp["q"].shape, dtype=torch.float32, device=dev)
         st = la.DecodeStep(inp["k_base"], inp["v_base"], inp["lr"], inp["B_k"], inp["B_v"],
                            inp["q"], out, inp["kv_len"], lora_scale=s.lora_scale,
-                           rope_base=s.rope_base, max_kv_len=s.kv_len, A_kv=A_kv, x_new=x_new,
-                           pos_new=s.kv_len - 1)
+                           rope_base=s.rope_base, max_kv_len=s.kv_len, A_kv=A_kv, x_new=x_new)
         sets.append((inp, x_new, out))
         steps_fn.append(st)
 

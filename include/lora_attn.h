@@ -187,16 +187,41 @@ typedef struct {
 } la_attn_args;
 
 /*
+ * lora_attn_decode_step -- a decode step on device buffers: for every
+ * sequence q the new token's LR row
+ *   lr_cache[q][kv_len[q] - 1][c] = sum_k x_new[q][k] A_kv[k][c],  c in [0, 2r)
+ * (with args->lr_agent_stride > 0 every agent's own cache, from its own
+ * A_kv[a]; rounding as lr_cache_append), then lora_attn_decode over
+ * [0, kv_len[q]), that row included.  Where the tensor-core decode takes the
+ * shape (bf16, head_dim 128, r in {16, 32}) this is ONE launch: the CTAs whose
+ * keys hold position kv_len[q] - 1 form the row themselves, use it and write
+ * it to the cache; otherwise a row-append kernel runs before the decode.
+ * The new token's base K and V rows must already be in k_base / v_base.
+ *
+ *   A_kv    device, [hidden][2r] (shared A), or [n_agents][hidden][2r] with
+ *           args->lr_agent_stride > 0; io dtype, 16-byte aligned.
+ *   x_new   device, [n_seqs][hidden], io dtype, 16-byte aligned.
+ *   hidden  > 0; hidden * element size a multiple of 16 bytes.
+ * Other arguments, workspace and errors as lora_attn_decode, plus
+ * LA_ERR_INVALID_ARG for a null or misaligned A_kv / x_new or a bad hidden.
+ * (The pages have PreLRShared fill the LR rows when a chunk first passes
+ * through the model, PReCache blog; for a decode token that chunk is the
+ * token itself.)
+ */
+la_status lora_attn_decode_step(const la_attn_args* args, const void* A_kv, const void* x_new,
+                                int64_t hidden, void* workspace, size_t workspace_bytes,
+                                la_stream_t stream);
+
+/*
  * lora_decode_step_host -- one whole decode step with the step's inputs and
  * outputs in HOST memory, as a serving loop runs it.  Queued on `stream`, in
  * this order, with nothing synchronised:
  *   1. copies x_host -> x_dev, q_host -> args->q, kv_len_host -> args->kv_len;
- *   2. appends the new token's LR row of every sequence q at position
- *      kv_len_host[q] - 1 (lr_cache_append; with args->lr_agent_stride > 0,
- *      one row per agent into that agent's own cache, X A_a, as
- *      lr_cache_append_agents);
- *   3. lora_attn_decode(args, workspace, ...);
- *   4. copies args->out -> out_host.
+ *   2. lora_attn_decode_step(args, A_kv, x_dev, hidden, workspace, ...): the
+ *      new token's LR row of every sequence q at position kv_len_host[q] - 1
+ *      (with args->lr_agent_stride > 0, one row per agent into that agent's
+ *      own cache, X A_a), then the decode;
+ *   3. copies args->out -> out_host.
  * out_host holds the step's outputs once the stream has been synchronised.
  * Pinned (page-locked) host buffers make the copies asynchronous; pageable
  * ones are still correct, with the copies staged by the CUDA runtime.  When

@@ -31,6 +31,7 @@ cudaError_t launch_decode_bf16(const AttnParams& p, la_dtype out, cudaStream_t s
 bool bf16_prefill_supported(const AttnParams& p);
 cudaError_t launch_prefill_bf16(const AttnParams& p, la_dtype out, cudaStream_t st);
 bool bf16_append_supported(int64_t H, int r);
+int cs_group_size(const AttnParams& p);
 
 namespace {
 
@@ -349,7 +350,51 @@ la_status decode_launch(AttnParams& p, int kind, const la_attn_args* a, cudaStre
                             : launch_attn_simt(p, a->io_dtype, a->out_dtype, st);
   return e == cudaSuccess ? LA_OK : LA_ERR_CUDA;
 }
+
+// The checks of a decode step's new-row inputs.
+la_status step_check(const la_attn_args* a, const void* A_kv, const void* x_new, int64_t hidden) {
+  if (!A_kv || !x_new || hidden < 1) return LA_ERR_INVALID_ARG;
+  if (!aligned16(A_kv) || !aligned16(x_new)) return LA_ERR_INVALID_ARG;
+  if ((hidden * (int64_t)esize(a->io_dtype)) % 16 != 0) return LA_ERR_INVALID_ARG;
+  return LA_OK;
+}
+
+// A decode step after decode_prepare: the new token's LR row at kv_len[q] - 1
+// of every LR cache, then the decode.  One launch where the cos/sin-table
+// decode takes the shape (it forms and writes the row itself), else the
+// row append and the decode.
+la_status step_launch(AttnParams& p, int kind, const la_attn_args* a, const void* A_kv,
+                      const void* x_new, int64_t hidden, cudaStream_t st) {
+  p.err = error_word_ptr();
+  if (!p.err) return LA_ERR_CUDA;
+  if (kind == 1 && a->io_dtype == LA_BF16 && cs_group_size(p) > 0) {
+    p.x_new = x_new;
+    p.A_kv = A_kv;
+    p.hidden = hidden;
+    return decode_launch(p, kind, a, st);
+  }
+  const int n_lr = a->lr_agent_stride > 0 ? a->n_agents : 1;
+  const cudaError_t e = launch_append_row_at_len(x_new, A_kv, hidden * 2 * a->r,
+                                                 const_cast<void*>(a->lr_cache), a->lr_seq_stride,
+                                                 a->lr_agent_stride, n_lr, a->kv_len, a->max_kv_len,
+                                                 a->n_seqs, hidden, a->r, a->io_dtype, p.err, st);
+  if (e != cudaSuccess) return LA_ERR_CUDA;
+  return decode_launch(p, kind, a, st);
+}
 }  // namespace
+
+extern "C" la_status lora_attn_decode_step(const la_attn_args* a, const void* A_kv,
+                                           const void* x_new, int64_t hidden, void* workspace,
+                                           size_t workspace_bytes, la_stream_t stream) {
+  AttnParams p;
+  int kind = 0;
+  bool empty = false;
+  la_status s = decode_prepare(a, workspace, workspace_bytes, &p, &kind, &empty);
+  if (s != LA_OK || empty) return s;
+  s = step_check(a, A_kv, x_new, hidden);
+  if (s != LA_OK) return s;
+  return step_launch(p, kind, a, A_kv, x_new, hidden, static_cast<cudaStream_t>(stream));
+}
 
 extern "C" la_status lora_attn_decode(const la_attn_args* a, void* workspace,
                                       size_t workspace_bytes, la_stream_t stream) {
@@ -373,18 +418,13 @@ extern "C" la_status lora_decode_step_host(const la_attn_args* a, void* workspac
   if (s != LA_OK || empty) return s;
   if (!x_dev || !x_host || !q_host || !kv_len_host || !out_host || !a->lr_cache)
     return LA_ERR_INVALID_ARG;
+  // the new token of sequence q sits at position kv_len_host[q] - 1
+  for (int32_t q = 0; q < a->n_seqs; ++q)
+    if (kv_len_host[q] < 1 || kv_len_host[q] > a->max_kv_len) return LA_ERR_INVALID_ARG;
+  s = step_check(a, A_kv, x_dev, hidden);
+  if (s != LA_OK) return s;
   const la_dtype dt = a->io_dtype;
   const int32_t n_seqs = a->n_seqs;
-  // the new token of sequence q sits at position kv_len_host[q] - 1
-  bool same_pos = true;
-  for (int32_t q = 0; q < n_seqs; ++q) {
-    if (kv_len_host[q] < 1 || kv_len_host[q] > a->max_kv_len) return LA_ERR_INVALID_ARG;
-    same_pos = same_pos && kv_len_host[q] == kv_len_host[0];
-  }
-  // every append below has the shapes, strides and alignment this check sees
-  s = append_check(x_dev, hidden, 1, hidden, A_kv, a->r, a->lr_cache, a->L_max,
-                   kv_len_host[0] - 1, n_seqs, hidden, a->lr_seq_stride, dt, &empty);
-  if (s != LA_OK) return s;
   const size_t es = esize(dt), eo = esize(a->out_dtype);
   const size_t x_bytes = (size_t)n_seqs * hidden * es;
   const size_t q_elems = (size_t)n_seqs * a->n_agents * a->n_q_heads * a->head_dim;
@@ -409,26 +449,8 @@ extern "C" la_status lora_decode_step_host(const la_attn_args* a, void* workspac
                              cudaMemcpyHostToDevice, st) != cudaSuccess) {
     return LA_ERR_CUDA;
   }
-  // the new rows: into the shared LR cache, or into every agent's own (X A_a)
-  const int n_lr = a->lr_agent_stride > 0 ? a->n_agents : 1;
-  const size_t a_bytes = (size_t)hidden * 2 * a->r * es;
-  for (int l = 0; l < n_lr; ++l) {
-    const char* A_l = static_cast<const char*>(A_kv) + l * a_bytes;
-    char* lr_l = static_cast<char*>(const_cast<void*>(a->lr_cache)) + (size_t)l * a->lr_agent_stride * es;
-    if (same_pos) {
-      s = append_launch(x_dev, hidden, 1, hidden, A_l, a->r, lr_l, kv_len_host[0] - 1, n_seqs,
-                        hidden, a->lr_seq_stride, dt, st);
-      if (s != LA_OK) return s;
-    } else {
-      for (int32_t q = 0; q < n_seqs; ++q) {
-        s = append_launch(static_cast<const char*>(x_dev) + (size_t)q * hidden * es, hidden, 1,
-                          hidden, A_l, a->r, lr_l + (size_t)q * a->lr_seq_stride * es,
-                          kv_len_host[q] - 1, 1, hidden, a->lr_seq_stride, dt, st);
-        if (s != LA_OK) return s;
-      }
-    }
-  }
-  s = decode_launch(p, kind, a, st);
+  // the new rows (shared LR cache, or every agent's own) and the decode
+  s = step_launch(p, kind, a, A_kv, x_dev, hidden, st);
   if (s != LA_OK) return s;
   if (cudaMemcpyAsync(out_host, a->out, q_elems * eo, cudaMemcpyDeviceToHost, st) != cudaSuccess)
     return LA_ERR_CUDA;

@@ -82,7 +82,63 @@ cudaError_t launch_r(const void* X, int64_t ldx, int64_t n, int64_t H, const voi
   return cudaGetLastError();
 }
 
+// The one new row of a decode step for every sequence q, at row kv_len[q] - 1
+// of every LR cache l (one shared, or one per agent with its own A):
+// lr[l][q][kv_len[q] - 1] = x[q] A[l].  Eight warps split the hidden rows; a
+// lane keeps columns lane, lane + 32, ...; the warps' sums meet in shared
+// memory.  A kv_len[q] outside [1, max_kv_len] is reported, nothing written.
+template <typename T>
+__global__ void __launch_bounds__(NT) append_row_at_len_kernel(
+    const T* __restrict__ x, const T* __restrict__ A, int64_t a_stride, T* __restrict__ lr,
+    int64_t lr_seq, int64_t lr_agent, const int32_t* __restrict__ kv_len, int64_t max_kv_len,
+    int64_t H, int C, int* err) {
+  __shared__ float part[NT / 32][128];
+  const int q = blockIdx.x, l = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int64_t len = kv_len[q];
+  if (len < 1 || len > max_kv_len) {
+    if (tid == 0) atomicOr(err, 1);
+    return;
+  }
+  const T* xq = x + (int64_t)q * H;
+  const T* Al = A + (int64_t)l * a_stride;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int64_t h = w; h < H; h += NT / 32) {
+    const float xv = to_f32(xq[h]);
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      if (lane + 32 * k < C) acc[k] = fmaf(xv, to_f32(Al[h * C + lane + 32 * k]), acc[k]);
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    if (lane + 32 * k < C) part[w][lane + 32 * k] = acc[k];
+  __syncthreads();
+  if (tid < C) {
+    float v = 0.f;
+#pragma unroll
+    for (int ww = 0; ww < NT / 32; ++ww) v += part[ww][tid];
+    lr[(int64_t)l * lr_agent + (int64_t)q * lr_seq + (len - 1) * C + tid] = from_f32<T>(v);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_append_row_at_len(const void* x, const void* A, int64_t a_stride, void* lr,
+                                     int64_t lr_seq, int64_t lr_agent, int n_lr,
+                                     const int32_t* kv_len, int64_t max_kv_len, int n_seqs,
+                                     int64_t H, int r, la_dtype dt, int* err, cudaStream_t st) {
+  if (2 * r > 128 || n_seqs < 1 || n_lr < 1) return cudaErrorInvalidValue;
+  dim3 grid(n_seqs, n_lr);
+  if (dt == LA_F32)
+    append_row_at_len_kernel<float><<<grid, NT, 0, st>>>(
+        static_cast<const float*>(x), static_cast<const float*>(A), a_stride, static_cast<float*>(lr),
+        lr_seq, lr_agent, kv_len, max_kv_len, H, 2 * r, err);
+  else
+    append_row_at_len_kernel<__nv_bfloat16><<<grid, NT, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(A), a_stride,
+        static_cast<__nv_bfloat16*>(lr), lr_seq, lr_agent, kv_len, max_kv_len, H, 2 * r, err);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_append_simt(const void* X, int64_t ldx, int64_t n, int64_t H, const void* A,
                                int r, void* lr, int64_t pos0, int n_seqs, int64_t sx,

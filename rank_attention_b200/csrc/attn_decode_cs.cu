@@ -69,7 +69,8 @@ constexpr int kSMs = 148;
 constexpr uint32_t T_W = 0, T_CS = 256, T_S = 320, T_O = 352, T_COLS = 512;
 
 // barriers (mbarrier slots)
-enum { B_FULL = 0, B_EMPTY = ST, B_TFULL = 2 * ST, B_WFREE, B_CSFULL, B_PFULL, B_PFREE, B_ODONE, B_NUM };
+enum { B_FULL = 0, B_EMPTY = ST, B_TFULL = 2 * ST, B_WFREE, B_CSFULL, B_PFULL, B_PFREE, B_ODONE, B_PATCH,
+       B_NUM };
 
 template <int R, int RP>
 struct Cfg {
@@ -87,7 +88,7 @@ struct Cfg {
   // small area: Mx [2][8][4] f32, Corr [2][QP] f32, cs0 [2][64] f32x2,
   // Lsum [QP][4] f32, Mfin [QP] f32, theta [64] f64, barriers, slots
   static constexpr int SMALL = 2 * 8 * 4 * 4 + 2 * QP * 4 + 2 * 64 * 8 + QP * 4 * 4 + QP * 4 + 64 * 8 +
-                               B_NUM * 8 + 64;
+                               B_NUM * 8 + 64 + 64 + 16 + 10 * 2 * R * 4 + 2 * R * 2;
   static constexpr size_t smem() {
     return 1024 + (size_t)ST * STAGE + UV_BYTES + Q_BYTES + P_BYTES + align1k(SMALL);
   }
@@ -131,6 +132,9 @@ __global__ void __launch_bounds__(NTHR, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(theta + 64);
   uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + B_NUM);
   int* s_misc = reinterpret_cast<int*>(tslot + 2);             // [0] fail, [1] ticket
+  float* red = reinterpret_cast<float*>(                        // [10 warps][2R]: the new LR row's sums
+      (reinterpret_cast<uintptr_t>(s_misc + 16) + 15) & ~uintptr_t(15));
+  __nv_bfloat16* newrow = reinterpret_cast<__nv_bfloat16*>(red + 10 * 2 * R);   // [2R]
   float* Part = reinterpret_cast<float*>(uv);                  // [RP][WP], after the last MMA
 
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
@@ -196,6 +200,7 @@ __global__ void __launch_bounds__(NTHR, 1)
     mbar_init(bar(B_PFULL), NSW + 1);
     mbar_init(bar(B_PFREE), 2);
     mbar_init(bar(B_ODONE), 1);
+    mbar_init(bar(B_PATCH), 1);
     fence_mbar_init();
     tma_prefetch(&tmK);
     tma_prefetch(&tmV);
@@ -259,6 +264,54 @@ __global__ void __launch_bounds__(NTHR, 1)
     }
     for (int it = tid; it < C::P_BYTES / 16; it += NTHR)
       *reinterpret_cast<uint4*>(pbuf + it * 16) = make_uint4(0, 0, 0, 0);
+  }
+
+  // ---- decode step in one launch: the CTA whose keys hold position kv_len - 1
+  // forms that token's LR row x_new [A_k | A_v] (fp32 sums, rounded to bf16
+  // as the append rounds them); one CTA per LR cache writes it to the cache
+  const int64_t p_new = kvl - 1;
+  const bool has_new = p.x_new != nullptr && !bad_len && p_new >= k_lo && p_new < k_hi;
+  if (has_new) {
+    constexpr int CH = 2 * R / 8;            // 16-byte column chunks of an A row
+    constexpr int RPI = 32 / CH;             // A rows per warp and iteration
+    const __nv_bfloat16* x = reinterpret_cast<const __nv_bfloat16*>(p.x_new) + (int64_t)seq * p.hidden;
+    const __nv_bfloat16* A = reinterpret_cast<const __nv_bfloat16*>(p.A_kv) +
+                             (p.lr_agent ? (int64_t)agent0 * p.hidden * 2 * R : 0);
+    const int ch = lane % CH, rs = lane / CH;
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+    for (int64_t h = (int64_t)w * RPI + rs; h < p.hidden; h += (int64_t)(NTHR / 32) * RPI) {
+      const float xv = __bfloat162float(x[h]);
+      const uint4 a = __ldg(reinterpret_cast<const uint4*>(A + h * 2 * R + 8 * ch));
+      const uint32_t* aw = reinterpret_cast<const uint32_t*>(&a);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = unpack_bf16(aw[e]);
+        acc[2 * e] = fmaf(xv, f.x, acc[2 * e]);
+        acc[2 * e + 1] = fmaf(xv, f.y, acc[2 * e + 1]);
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+#pragma unroll
+      for (int o = CH; o < 32; o <<= 1) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
+    if (rs == 0)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) red[w * 2 * R + 8 * ch + e] = acc[e];
+  }
+  __syncthreads();
+  if (has_new && tid < 2 * R) {
+    float v = 0.f;
+#pragma unroll
+    for (int ww = 0; ww < NTHR / 32; ++ww) v += red[ww * 2 * R + tid];
+    const __nv_bfloat16 b = __float2bfloat16_rn(v);
+    newrow[tid] = b;
+    if (kvh == 0 && (p.lr_agent || blockIdx.y == 0)) {   // the cache's one writer
+      __nv_bfloat16* lr = reinterpret_cast<__nv_bfloat16*>(const_cast<void*>(p.lr)) +
+                          (p.lr_agent ? (int64_t)agent0 * p.lr_agent : 0) + (int64_t)seq * p.lr_seq;
+      lr[p_new * 2 * R + tid] = b;
+    }
   }
 
   // ---- score warps: per-thread (cos, sin)(j theta_i) for their 32 frequencies,
@@ -334,6 +387,7 @@ __global__ void __launch_bounds__(NTHR, 1)
       const bool valid = k0 + jk < k_hi;
       wt(B_FULL + s, (n / ST) & 1);
       wt(B_TFULL, n & 1);
+      if (has_new && p_new >= k0 && p_new < k0 + KT) wt(B_PATCH, 0);   // the new LR row is in place
       tc_fence_after();
       // S (every row), this half's W columns, this key's LRk
       uint32_t sv[16];
@@ -467,6 +521,13 @@ __global__ void __launch_bounds__(NTHR, 1)
       unsigned char* sb = stages + s * C::STAGE;
       wt(B_FULL + s, (n / ST) & 1);
       if (lane == 0 && !fail) n_seen = n + 1;
+      if (has_new && p_new >= k0 && p_new < k0 + KT) {   // the new token's LR row over the loaded one
+        for (int c = lane; c < 2 * R / 8; c += 32)
+          *reinterpret_cast<uint4*>(sb + 2 * C::KV_TILE + tile_off<2 * R, KT>((int)(p_new - k0), 8 * c)) =
+              reinterpret_cast<const uint4*>(newrow)[c];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(B_PATCH));
+      }
       if (k0 + KT > k_hi) {   // P is 0 there; zeroed rows keep stale NaN out of P V
         const int first = (int)(k_hi - k0);
         for (int i = lane; i < (KT - first) * (D / 8); i += 32) {

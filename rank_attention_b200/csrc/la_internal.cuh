@@ -45,6 +45,11 @@ struct AttnParams {
   int agent_group;         // tensor-core decode: agents per CTA (grid z runs over the groups)
   int value_path;          // la_value_path: 0 fastest reordered, 1 generic reordered, 2 per tile
   int blk0;                // tensor-core prefill, split launch: the first block of rows it covers
+  // decode step in one launch: the new token's LR row x_new[q] A_kv written at
+  // row kv_len[q] - 1 (and used) by the decode itself; null x_new: no append
+  const void* x_new;       // [n_seqs][hidden]
+  const void* A_kv;        // [hidden][2r], or [n_agents][hidden][2r] with per-agent caches
+  int64_t hidden;
 };
 
 // Device error word of the library (address on the current device).
@@ -58,6 +63,10 @@ cudaError_t launch_append_bf16_mma(const void* X, int64_t ldx, int64_t n, int64_
                                    const void* A, int r, void* lr, int64_t pos0, int n_seqs,
                                    int64_t sx, int64_t slr, cudaStream_t st);
 cudaError_t launch_attn_simt(const AttnParams& p, la_dtype io, la_dtype out, cudaStream_t st);
+cudaError_t launch_append_row_at_len(const void* x, const void* A, int64_t a_stride, void* lr,
+                                     int64_t lr_seq, int64_t lr_agent, int n_lr,
+                                     const int32_t* kv_len, int64_t max_kv_len, int n_seqs,
+                                     int64_t H, int r, la_dtype dt, int* err, cudaStream_t st);
 cudaError_t launch_query_expand(const void* q_base, const void* lr_q, const void* B_q, void* q_out,
                                 int n_seqs, int n_agents, int n_tok, int n_q, int d, int r, float s,
                                 double rope_base, const int32_t* pos_end, la_dtype dt,

@@ -29,7 +29,7 @@ EXPORTED = ("la_status_string", "lr_cache_append", "lora_attn_prefill", "lora_at
             "lora_attn_decode_workspace_bytes", "la_device_check",
             "lora_attn_decode_static_scratch", "lora_materialize_agent_kv",
             "lr_cache_append_agents", "lora_query_expand", "lora_output_delta",
-            "la_device_check_word", "lora_decode_step_host")
+            "la_device_check_word", "lora_decode_step_host", "lora_attn_decode_step")
 
 
 class LoraAttnError(RuntimeError):
@@ -107,6 +107,10 @@ def _load() -> ctypes.CDLL:
         ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
         ctypes.c_void_p, ctypes.c_void_p]
     lib.la_device_check_word.argtypes = [ctypes.POINTER(ctypes.c_int32)]
+    lib.lora_attn_decode_step.restype = ctypes.c_int
+    lib.lora_attn_decode_step.argtypes = [ctypes.POINTER(AttnArgs), ctypes.c_void_p, ctypes.c_void_p,
+                                          ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t,
+                                          ctypes.c_void_p]
     lib.lora_attn_decode_static_scratch.restype = ctypes.c_int
     lib.lora_attn_decode_static_scratch.argtypes = [ctypes.POINTER(AttnArgs), ctypes.c_void_p]
     lib.lora_materialize_agent_kv.restype = ctypes.c_int
@@ -269,6 +273,19 @@ def lora_attn_decode(args: AttnArgs, workspace: torch.Tensor, stream=None) -> No
     _check(st, "lora_attn_decode")
 
 
+def lora_attn_decode_step(args: AttnArgs, A_kv: torch.Tensor, x_new: torch.Tensor,
+                          workspace: torch.Tensor, stream=None) -> None:
+    """A decode step on device buffers: the new token's LR row x_new[q] A_kv at
+    kv_len[q] - 1 of the LR cache(s), then the decode (one launch where the
+    tensor-core decode takes the shape).  x_new [n_seqs, hidden] contiguous;
+    A_kv [hidden, 2r], or [n_agents, hidden, 2r] with per-agent caches."""
+    assert x_new.is_contiguous() and A_kv.is_contiguous()
+    st = lib.lora_attn_decode_step(ctypes.byref(args), A_kv.data_ptr(), x_new.data_ptr(),
+                                   x_new.shape[-1], workspace.data_ptr(), workspace.numel(),
+                                   _stream(stream))
+    _check(st, "lora_attn_decode_step")
+
+
 def lora_decode_step_host(args: AttnArgs, workspace: torch.Tensor, A_kv: torch.Tensor,
                           x_dev: torch.Tensor, x_host: torch.Tensor, q_host: torch.Tensor,
                           kv_len_host: torch.Tensor, out_host: torch.Tensor, stream=None) -> None:
@@ -333,24 +350,28 @@ def la_device_check_word() -> tuple:
 
 
 class DecodeStep:
-    """One decode step of the hot path: append the new token's LR row, then
-    attend every agent's query over the shared caches.
+    """One decode step of the hot path: the new token's LR row at kv_len - 1,
+    then every agent's query over the shared caches (lora_attn_decode_step:
+    one library call, one launch where the tensor-core decode takes the shape).
 
-    Holds the argument struct and the zero-filled split-K workspace so that a
-    step is two library calls.  Tensors must stay alive while it is used."""
+    Holds the argument struct and the zero-filled split-K workspace.  Tensors
+    must stay alive while it is used.  Without x_new / A_kv it is the decode
+    alone."""
 
     def __init__(self, k_base, v_base, lr, B_k, B_v, q, out, kv_len, *, lora_scale, rope_base,
-                 max_kv_len, A_kv=None, x_new=None, pos_new=None):
+                 max_kv_len, A_kv=None, x_new=None):
         self.args = make_args(k_base, v_base, lr, B_k, B_v, q, out, lora_scale=lora_scale,
                               rope_base=rope_base, kv_len=kv_len, max_kv_len=max_kv_len)
         self.workspace = decode_workspace(self.args, q.device)
-        self.lr, self.A_kv, self.x_new, self.pos_new = lr, A_kv, x_new, pos_new
-        self._keep = (k_base, v_base, lr, B_k, B_v, q, out, kv_len)
+        self.lr, self.A_kv = lr, A_kv
+        self.x_new = None if x_new is None else x_new.reshape(x_new.shape[0], -1)
+        self._keep = (k_base, v_base, lr, B_k, B_v, q, out, kv_len, x_new)
 
     def __call__(self, stream=None) -> None:
         if self.x_new is not None:
-            lr_cache_append(self.x_new, self.A_kv, self.lr, self.pos_new, stream)
-        lora_attn_decode(self.args, self.workspace, stream)
+            lora_attn_decode_step(self.args, self.A_kv, self.x_new, self.workspace, stream)
+        else:
+            lora_attn_decode(self.args, self.workspace, stream)
 
     def from_host(self, x_host, q_host, kv_len_host, out_host, stream=None) -> None:
         """The same step with its inputs and outputs in host memory: one call

@@ -290,10 +290,11 @@ def test_decode_merge_wait_runs_out_and_is_reported(la):
     ((640, 640), True, False),        # BaseShared: every agent's own A_a and LR cache
 ])
 def test_decode_step_from_host_equals_device_step(la, kv_lens, per_agent, packed):
-    """lora_decode_step_host (copies in, append at kv_len - 1, decode, copy out)
-    gives the same LR rows and outputs, bit for bit, as the same step on
-    device buffers (the append then the decode), and the outputs match the
-    oracle over the updated caches."""
+    """lora_decode_step_host (copies in, the step, copy out) gives the same LR
+    rows and outputs, bit for bit, as lora_attn_decode_step on device buffers.
+    The new rows are X A within one bf16 ulp of the oracle's fp64 rows (fp32
+    accumulation order), every other row is untouched, and the outputs match
+    the oracle over the updated caches."""
     n_seqs, L_max = len(kv_lens), max(kv_lens)
     s = W.LLAMA8B_DECODE_8K.replace(kv_len=L_max, n_seqs=n_seqs, seed=37, lr_per_agent=per_agent)
     inp = W.direct_cache_inputs(s, L_max=L_max)
@@ -330,20 +331,69 @@ def test_decode_step_from_host_equals_device_step(la, kv_lens, per_agent, packed
             torch.cuda.synchronize()
             outs.append(out_host.clone())
         else:
+            step()
+            torch.cuda.synchronize()
+            outs.append(out.cpu())
+        lrs.append(dd["lr"].cpu())
+    assert la.la_device_check() == 0
+    assert torch.equal(lrs[0], lrs[1])
+    assert torch.equal(outs[0], outs[1])
+    # the new rows, and nothing else, changed
+    got = lrs[1] if per_agent else lrs[1][None]
+    before = inp["lr"] if per_agent else inp["lr"][None]
+    A_list = [A_kv[a] for a in range(s.n_agents)] if per_agent else [A_kv]
+    for l, A in enumerate(A_list):
+        ref = oracle.lr_cache_rows(x, A)[:, 0]                      # [n_seqs, 2r]
+        for q, n in enumerate(kv_lens):
+            row = to_np(got[l, q, n - 1])
+            bound = np.maximum(bf16_ulp(ref[q]), 1e-6 * (np.abs(to_np(x[q, 0])) @ np.abs(to_np(A))))
+            assert (np.abs(row - ref[q]) <= bound).all(), np.abs(row - ref[q]).max()
+            keep = torch.ones(got.shape[2], dtype=torch.bool)
+            keep[n - 1] = False
+            assert torch.equal(got[l, q, keep], before[l, q, keep])
+    assert_parity(to_np(outs[1]), oracle_decode(inp, s, lr=lrs[1].double()), s.dtype)
+
+
+@pytest.mark.parametrize("r,n_agents,per_agent", [(16, 3, False), (32, 5, False), (16, 3, True),
+                                                  (64, 4, False)])
+def test_decode_step_equals_append_then_decode(la, r, n_agents, per_agent):
+    """The one-launch step (the decode forms the new token's LR row itself; r =
+    16, 32) and its two-launch form (r = 64: a row-append kernel, then the
+    decode) against lr_cache_append followed by lora_attn_decode: the rows
+    agree within one bf16 ulp, the outputs within the parity bar."""
+    kv_lens = (1000, 777)
+    s = W.LLAMA8B_DECODE_8K.replace(kv_len=1000, n_seqs=2, r=r, alpha=2.0 * r, n_agents=n_agents,
+                                    seed=48 + r, lr_per_agent=per_agent)
+    inp = W.direct_cache_inputs(s)
+    inp["kv_len"] = torch.tensor(kv_lens, dtype=torch.int32)
+    x = W.append_inputs(1, s.hidden, r, s.dtype, seed=49, n_seqs=2)["X"]
+    A_kv = (torch.stack([W.append_inputs(1, s.hidden, r, s.dtype, seed=50 + a)["A_kv"]
+                         for a in range(n_agents)]) if per_agent
+            else W.append_inputs(1, s.hidden, r, s.dtype, seed=50)["A_kv"])
+    res = []
+    for fused in (True, False):
+        dd = to_device(inp)
+        out = torch.zeros(dd["q"].shape, device=DEV)
+        x_dev, A_dev = x.to(DEV), A_kv.to(DEV)
+        step = la.DecodeStep(dd["k_base"], dd["v_base"], dd["lr"], dd["B_k"], dd["B_v"], dd["q"],
+                             out, dd["kv_len"], lora_scale=s.lora_scale, rope_base=s.rope_base,
+                             max_kv_len=1000, A_kv=A_dev, x_new=x_dev)
+        if fused:
+            step()
+        else:
             for q, n in enumerate(kv_lens):
                 if per_agent:
                     la.lr_cache_append_agents(x_dev[q:q + 1], A_dev, dd["lr"][:, q:q + 1], n - 1)
                 else:
                     la.lr_cache_append(x_dev[q:q + 1], A_dev, dd["lr"][q:q + 1], n - 1)
             la.lora_attn_decode(step.args, step.workspace)
-            torch.cuda.synchronize()
-            outs.append(out.cpu())
-        lrs.append(dd["lr"].cpu())
-    assert la.la_device_check() == 0
-    assert torch.equal(lrs[0], lrs[1])
-    assert not torch.equal(lrs[1], inp["lr"])   # the new rows did land
-    assert torch.equal(outs[0], outs[1])
-    assert_parity(to_np(outs[1]), oracle_decode(inp, s, lr=lrs[1].double()), s.dtype)
+        torch.cuda.synchronize()
+        assert la.la_device_check() == 0
+        res.append((to_np(out), to_np(dd["lr"])))
+    (o1, l1), (o2, l2) = res
+    assert (np.abs(l1 - l2) <= 2 * bf16_ulp(l2)).all()
+    assert_parity(o1, o2, s.dtype)
+    assert_parity(o1, oracle_decode(inp, s, lr=torch.from_numpy(l1)), s.dtype)
 
 
 # ---------------------------------------------------------- bf16 prefill ----
