@@ -584,12 +584,26 @@ def decode_source_sha() -> str:
     return hashlib.sha256(code.encode()).hexdigest()[:16]
 
 
+def step_kernels_per_call(s) -> int:
+    """Kernels one decode step (lora_attn_decode_step) launches: one where the
+    tensor-core decode forms the new LR row itself (bf16, d = 128, r = 16 or
+    32), else a row append before the decode's kernels."""
+    if s.dtype != torch_bf16() or s.head_dim != 128:
+        return 1 + decode_kernels_per_call(s)
+    return 1 if s.r in (16, 32) else 1 + decode_kernels_per_call(s)
+
+
+def torch_bf16():
+    import torch
+    return torch.bfloat16
+
+
 def decode_kernels_per_call(s) -> int:
     """Kernels one lora_attn_decode call launches for this workload.  The
-    tensor-core decode (d = 128, r in {16, 32, 64}, at most three agents) merges
-    its key splits inside the same launch: one kernel.  The other bf16 shapes
-    add a split-merge kernel when the keys are split over CTAs."""
-    if s.head_dim == 128 and s.r in (16, 32, 64) and s.n_agents <= 3:
+    tensor-core decodes (d = 128: r in {16, 32} any agent count; r = 64)
+    merge their key splits inside the same launch: one kernel.  The other bf16
+    shapes add a split-merge kernel when the keys are split over CTAs."""
+    if s.head_dim == 128 and (s.r in (16, 32) or (s.r == 64 and s.n_agents <= 3)):
         return 1
     units = s.n_seqs * s.n_kv_heads
     splits = 1 if units >= 148 else min(32, 148 // units, (s.kv_len + 127) // 128)
@@ -768,7 +782,7 @@ def step_config(s, world: int) -> dict:
     step_bytes = decode_bytes(s) + append_bytes(s, 1)
     n_sets = max(2, math.ceil(2 * L2_BYTES / step_bytes))
     return {"workload": s.name, "kv_len": s.kv_len, "agents": s.n_agents, "r": s.r,
-            "step": "lr_cache_append(1 token) + lora_attn_decode",
+            "step": "lora_attn_decode_step: the new token's LR row and the decode",
             "l2": f"inputs larger than L2: {n_sets} rotating cache sets of "
                   f"{step_bytes / 1e6:.1f} MB ({n_sets * step_bytes / 1e6:.0f} MB > 126 MB)",
             "timing": "CUDA graphs of the steps, CUDA events on the launch stream",
@@ -968,7 +982,7 @@ def run_ours(args):
                      "nominal_peak": NOMINAL_HBM_GBS},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e_steps},
-        "gpu_launches": (1 + decode_kernels_per_call(s)) * args.steps,
+        "gpu_launches": step_kernels_per_call(s) * args.steps,
         "clocks": clk,
         "prefill": prefill,
         "non_shared_baseline": non_shared,

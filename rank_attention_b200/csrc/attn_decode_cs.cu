@@ -23,10 +23,10 @@
 //  * warp 9 (one thread) issues per tile S = K_base Q^T and W = CS UV^T, and
 //    for the previous tile O^T += V_base^T P^T (tcgen05, fp32 in TMEM);
 //  * warps 0-7 (key j = 32 (w % 4) + lane, half w / 4 of the rows) add the
-//    r-wide dots to S, run the online softmax and write P (bf16); they also
-//    write the next tile's table CS into TMEM: (cos, sin)((k0 + j) theta) from
-//    the exact (cos, sin)(k0 theta) (angle reduced in fp64) and per-thread
-//    (cos, sin)(j theta);
+//    r-wide dots to S, run the online softmax and write P (bf16); two tiles
+//    ahead they also write the table CS into TMEM (two buffers):
+//    (cos, sin)((k0 + j) theta) from the exact (cos, sin)(k0 theta) (angle
+//    reduced in fp64) and (cos, sin)(j theta), a per-lane table kept in TMEM;
 //  * warp 8 keeps the value side reordered (LRAgent explainer, Metodologia 3;
 //    summary App. B): O_lr^T += LRv^T P^T stays r wide (mma.sync); it also
 //    streams K_base, V_base and the LR rows of each tile by TMA into a
@@ -65,12 +65,14 @@ constexpr int kL2Ahead = 4;        // tiles requested into L2 ahead of the stage
 constexpr int kMaxSplits = 32;
 constexpr int kSMs = 148;
 
-// TMEM columns
-constexpr uint32_t T_W = 0, T_CS = 256, T_S = 320, T_O = 352, T_COLS = 512;
+// TMEM columns: W (at most 192), the two CS buffers (64 each, bf16 pairs),
+// the (cos, sin)(j theta) table (fp32: per half of the frequencies 32 cos,
+// then 32 sin), S, O^T
+constexpr uint32_t T_W = 0, T_CS = 192, T_CSJ = 320, T_S = 448, T_O = 464, T_COLS = 512;
 
 // barriers (mbarrier slots)
-enum { B_FULL = 0, B_EMPTY = ST, B_TFULL = 2 * ST, B_WFREE, B_CSFULL, B_PFULL, B_PFREE, B_ODONE, B_PATCH,
-       B_NUM };
+enum { B_FULL = 0, B_EMPTY = ST, B_TFULL = 2 * ST, B_WFREE, B_CSFULL, B_CSFULL1, B_PFULL, B_PFREE,
+       B_ODONE, B_PATCH, B_NUM };
 
 template <int R, int RP>
 struct Cfg {
@@ -85,16 +87,18 @@ struct Cfg {
   static constexpr int P_BYTES = align1k(QP * KT * 2);
   static constexpr int WP = D + R + 4;                  // partial row: O | O_lr | m | l | pad
   static constexpr int MR = R / 16;                     // m16 tiles of O_lr^T
-  // small area: Mx [2][8][4] f32, Corr [2][QP] f32, cs0 [2][64] f32x2,
+  // small area: Mx [2][8][4] f32, Corr [2][QP] f32, cs0 [4][64] f32x2,
   // Lsum [QP][4] f32, Mfin [QP] f32, theta [64] f64, barriers, slots
-  static constexpr int SMALL = 2 * 8 * 4 * 4 + 2 * QP * 4 + 2 * 64 * 8 + QP * 4 * 4 + QP * 4 + 64 * 8 +
+  static constexpr int SMALL = 2 * 8 * 4 * 4 + 2 * QP * 4 + 4 * 64 * 8 + QP * 4 * 4 + QP * 4 + 64 * 8 +
                                B_NUM * 8 + 64 + 64 + 16 + 10 * 2 * R * 4 + 2 * R * 2;
   static constexpr size_t smem() {
     return 1024 + (size_t)ST * STAGE + UV_BYTES + Q_BYTES + P_BYTES + align1k(SMALL);
   }
-  static_assert(NW <= 256, "W is one MMA of N <= 256");
+  static_assert(NW <= 192, "W is one MMA of N <= 192 (TMEM columns 0..191)");
   static_assert(RP % 4 == 0 && RP <= QP, "rows");
-  static_assert((size_t)RP * WP * 4 <= (size_t)UV_BYTES, "partial staging fits the UV area");
+  // after the loop the UV area holds the partial, the merge's weights, (m, l)
+  // pairs and merged rows; the drained stages the other splits' partials
+  static_assert((size_t)RP * (2 * WP + 3 * kMaxSplits) * 4 <= (size_t)UV_BYTES, "merge area");
 };
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -125,8 +129,8 @@ __global__ void __launch_bounds__(NTHR, 1)
   unsigned char* pbuf = qop + C::Q_BYTES;
   float* Mx = reinterpret_cast<float*>(pbuf + C::P_BYTES);   // [2 halves][8 rows][4 sub-partitions]
   float* Corr = Mx + 2 * 8 * 4;                                // [2][QP]
-  float2* cs0 = reinterpret_cast<float2*>(Corr + 2 * QP);      // [2][64]: (cos, sin)(k0 theta_i)
-  float* Lsum = reinterpret_cast<float*>(cs0 + 2 * 64);        // [QP][4]
+  float2* cs0 = reinterpret_cast<float2*>(Corr + 2 * QP);      // [4][64]: (cos, sin)(k0 theta_i)
+  float* Lsum = reinterpret_cast<float*>(cs0 + 4 * 64);        // [QP][4]
   float* Mfin = Lsum + QP * 4;                                 // [QP]
   double* theta = reinterpret_cast<double*>(Mfin + QP);        // [64]
   uint64_t* bars = reinterpret_cast<uint64_t*>(theta + 64);
@@ -197,6 +201,7 @@ __global__ void __launch_bounds__(NTHR, 1)
     mbar_init(bar(B_TFULL), 1);
     mbar_init(bar(B_WFREE), NSW);
     mbar_init(bar(B_CSFULL), NSW);
+    mbar_init(bar(B_CSFULL1), NSW);
     mbar_init(bar(B_PFULL), NSW + 1);
     mbar_init(bar(B_PFREE), 2);
     mbar_init(bar(B_ODONE), 1);
@@ -217,42 +222,10 @@ __global__ void __launch_bounds__(NTHR, 1)
   const bool bad_len = kvl < 1 || kvl > p.max_kv_len;
   const int64_t k_hi = bad_len ? k_lo : min(te * KT, kvl);
   const int n_tiles = k_hi > k_lo ? (int)((k_hi - k_lo + KT - 1) / KT) : 0;
-  if (w == WM) tmem_alloc(smem_u32(tslot), T_COLS);
 
-  // ---- per-CTA operands: [U | V] (B of W = CS UV^T), the queries (B of S), P zeroed
+  // ---- the queries: the B operand of S (swizzled), read back by the [U | V] build
   {
     const __nv_bfloat16* Q = reinterpret_cast<const __nv_bfloat16*>(p.q);
-    const __nv_bfloat16* Bk = reinterpret_cast<const __nv_bfloat16*>(p.B_k);
-    const float s = p.s;
-    for (int it = tid; it < NW * 8; it += NTHR) {   // (row, rho) x 8 frequencies
-      const int n = it >> 3, i0 = (it & 7) * 8;
-      const int row = n / R, rho = n % R;
-      uint4 u4 = make_uint4(0, 0, 0, 0), v4 = u4;
-      if (row < n_rows && !bad_len) {
-        const int a = row / g, gi = row % g;
-        const __nv_bfloat16* qr = Q + (((int64_t)seq * na_tot + agent0 + a) * p.n_q + kvh * g + gi) * D;
-        const __nv_bfloat16* br = Bk + ((int64_t)(agent0 + a) * R + rho) * ldB + kvh * D;
-        const uint4 q1 = __ldg(reinterpret_cast<const uint4*>(qr + i0));
-        const uint4 q2 = __ldg(reinterpret_cast<const uint4*>(qr + D / 2 + i0));
-        const uint4 b1 = __ldg(reinterpret_cast<const uint4*>(br + i0));
-        const uint4 b2 = __ldg(reinterpret_cast<const uint4*>(br + D / 2 + i0));
-        const uint32_t* q1w = reinterpret_cast<const uint32_t*>(&q1);
-        const uint32_t* q2w = reinterpret_cast<const uint32_t*>(&q2);
-        const uint32_t* b1w = reinterpret_cast<const uint32_t*>(&b1);
-        const uint32_t* b2w = reinterpret_cast<const uint32_t*>(&b2);
-        uint32_t* uw = reinterpret_cast<uint32_t*>(&u4);
-        uint32_t* vw = reinterpret_cast<uint32_t*>(&v4);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 x1 = unpack_bf16(q1w[e]), x2 = unpack_bf16(q2w[e]);
-          const float2 c1 = unpack_bf16(b1w[e]), c2 = unpack_bf16(b2w[e]);
-          uw[e] = pack_bf16(s * fmaf(x1.x, c1.x, x2.x * c2.x), s * fmaf(x1.y, c1.y, x2.y * c2.y));
-          vw[e] = pack_bf16(s * fmaf(x2.x, c1.x, -x1.x * c2.x), s * fmaf(x2.y, c1.y, -x1.y * c2.y));
-        }
-      }
-      *reinterpret_cast<uint4*>(uv + tile_off<D, NW>(n, i0)) = u4;
-      *reinterpret_cast<uint4*>(uv + tile_off<D, NW>(n, D / 2 + i0)) = v4;
-    }
     for (int it = tid; it < QP * (D / 8); it += NTHR) {
       const int row = it / (D / 8), c = (it % (D / 8)) * 8;
       uint4 v = make_uint4(0, 0, 0, 0);
@@ -265,7 +238,6 @@ __global__ void __launch_bounds__(NTHR, 1)
     for (int it = tid; it < C::P_BYTES / 16; it += NTHR)
       *reinterpret_cast<uint4*>(pbuf + it * 16) = make_uint4(0, 0, 0, 0);
   }
-
   // ---- decode step in one launch: the CTA whose keys hold position kv_len - 1
   // forms that token's LR row x_new [A_k | A_v] (fp32 sums, rounded to bf16
   // as the append rounds them); one CTA per LR cache writes it to the cache
@@ -300,7 +272,11 @@ __global__ void __launch_bounds__(NTHR, 1)
 #pragma unroll
       for (int e = 0; e < 8; ++e) red[w * 2 * R + 8 * ch + e] = acc[e];
   }
-  __syncthreads();
+  if (w == WM) tmem_alloc(smem_u32(tslot), T_COLS);
+  tc_fence_before();
+  __syncthreads();   // queries staged, the new row's partial sums, the TMEM address
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
   if (has_new && tid < 2 * R) {
     float v = 0.f;
 #pragma unroll
@@ -314,25 +290,81 @@ __global__ void __launch_bounds__(NTHR, 1)
     }
   }
 
-  // ---- score warps: per-thread (cos, sin)(j theta_i) for their 32 frequencies,
-  // and the exact (cos, sin)(k0 theta_i) of the first two tiles
+  // ---- [U | V]: the B operand of W = CS UV^T, a row per (query row, rho):
+  // U = s (q_i B_i + q_{i+d/2} B_{i+d/2}) in K columns i, V = s (q_{i+d/2} B_i -
+  // q_i B_{i+d/2}) in K columns d/2 + i.  An item is (agent, rho, 8
+  // frequencies): its B_k^a chunks are loaded (all of a thread's items at
+  // once), then combined with each of the agent's g staged query rows.
+  {
+    const __nv_bfloat16* Bk = reinterpret_cast<const __nv_bfloat16*>(p.B_k);
+    const float s = p.s;
+    const int n_ag = (RP + g - 1) / g;          // agents whose rows fall within RP
+    const int items = n_ag * R * 8;
+    constexpr int MAXK = 4;                     // items per thread (at most 4 agents x 32 x 8)
+    uint4 b1[MAXK], b2[MAXK];
+#pragma unroll
+    for (int k = 0; k < MAXK; ++k) {
+      const int it = tid + k * NTHR;
+      b1[k] = b2[k] = make_uint4(0, 0, 0, 0);
+      const int a = it / (R * 8), rho = (it / 8) % R, i0 = (it & 7) * 8;
+      if (it < items && a < na && !bad_len) {
+        const __nv_bfloat16* br = Bk + ((int64_t)(agent0 + a) * R + rho) * ldB + kvh * D;
+        b1[k] = __ldg(reinterpret_cast<const uint4*>(br + i0));
+        b2[k] = __ldg(reinterpret_cast<const uint4*>(br + D / 2 + i0));
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < MAXK; ++k) {
+      const int it = tid + k * NTHR;
+      if (it >= items) continue;
+      const int a = it / (R * 8), rho = (it / 8) % R, i0 = (it & 7) * 8;
+      const uint32_t* b1w = reinterpret_cast<const uint32_t*>(&b1[k]);
+      const uint32_t* b2w = reinterpret_cast<const uint32_t*>(&b2[k]);
+      for (int gi = 0; gi < g; ++gi) {
+        const int row = a * g + gi;
+        if (row >= RP) break;
+        const uint4 q1 = *reinterpret_cast<const uint4*>(qop + tile_off<D, QP>(row, i0));
+        const uint4 q2 = *reinterpret_cast<const uint4*>(qop + tile_off<D, QP>(row, D / 2 + i0));
+        const uint32_t* q1w = reinterpret_cast<const uint32_t*>(&q1);
+        const uint32_t* q2w = reinterpret_cast<const uint32_t*>(&q2);
+        uint4 u4, v4;
+        uint32_t* uw = reinterpret_cast<uint32_t*>(&u4);
+        uint32_t* vw = reinterpret_cast<uint32_t*>(&v4);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 x1 = unpack_bf16(q1w[e]), x2 = unpack_bf16(q2w[e]);
+          const float2 c1 = unpack_bf16(b1w[e]), c2 = unpack_bf16(b2w[e]);
+          uw[e] = pack_bf16(s * fmaf(x1.x, c1.x, x2.x * c2.x), s * fmaf(x1.y, c1.y, x2.y * c2.y));
+          vw[e] = pack_bf16(s * fmaf(x2.x, c1.x, -x1.x * c2.x), s * fmaf(x2.y, c1.y, -x1.y * c2.y));
+        }
+        const int n = row * R + rho;
+        *reinterpret_cast<uint4*>(uv + tile_off<D, NW>(n, i0)) = u4;
+        *reinterpret_cast<uint4*>(uv + tile_off<D, NW>(n, D / 2 + i0)) = v4;
+      }
+    }
+  }
+
+  // ---- score warps: the per-lane table (cos, sin)(j theta_i) of their 32
+  // frequencies into TMEM, and the exact (cos, sin)(k0 theta_i) of the first
+  // three tiles
   const int sp = w & 3, hh = (w >> 2) & 1;
   const int jk = 32 * sp + lane;                  // this thread's key in a tile (its TMEM lane)
   const uint32_t lane_off = (uint32_t)(32 * sp) << 16;
-  uint64_t CJ[16], SJ[16];
   if (w < NSW) {
+    uint32_t cj[32], sj[32];
 #pragma unroll
-    for (int e = 0; e < 16; ++e) {
-      const int i0 = 32 * hh + 2 * e;
-      const float2 a = sincos_small((float)jk * rt.thetaf[i0]);
-      const float2 b = sincos_small((float)jk * rt.thetaf[i0 + 1]);
-      CJ[e] = f2(a.x, b.x);
-      SJ[e] = f2(a.y, b.y);
+    for (int e = 0; e < 32; ++e) {
+      const float2 a = sincos_small((float)jk * rt.thetaf[32 * hh + e]);
+      cj[e] = __float_as_uint(a.x);
+      sj[e] = __float_as_uint(a.y);
     }
+    tmem_st32x32b_x32(tmem + T_CSJ + 64 * hh + lane_off, cj);
+    tmem_st32x32b_x32(tmem + T_CSJ + 64 * hh + 32 + lane_off, sj);
+    tmem_wait_st();
     if (sp == 0) {
       const int i = 32 * hh + lane;
-      cs0[i] = rope_cs_exact(k_lo, rt.theta[i]);
-      cs0[64 + i] = rope_cs_exact(k_lo + KT, rt.theta[i]);
+#pragma unroll
+      for (int t = 0; t < 3; ++t) cs0[t * 64 + i] = rope_cs_exact(k_lo + (int64_t)t * KT, rt.theta[i]);
     }
   }
 
@@ -340,41 +372,51 @@ __global__ void __launch_bounds__(NTHR, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *tslot;
   // Every wait is bounded in time.  After one has run out, a thread skips its
   // later waits but keeps every arrive, commit and named barrier of its role,
   // so the other roles finish too (their own waits may run out once) and the
   // CTA reaches its end quickly, reporting the failure.
   int fail = 0;
   auto wt = [&](int b, uint32_t parity) {
-    if (!fail && !mbar_wait_ns(bar(b), parity)) fail = 1;
+    if (!fail && !mbar_wait_clk(bar(b), parity)) fail = 1;
   };
   const float sl2 = p.scale * kLog2e;
 
-  // CS of tile n into TMEM: lane j, columns 16 hh.. (cos) and 32 + 16 hh.. (sin)
+  // CS of tile n into TMEM buffer n & 1: lane j, columns 16 hh.. (cos) and
+  // 32 + 16 hh.. (sin), bf16 pairs; (cos, sin)((k0 + j) theta) by the angle
+  // sum from cs0 slot n & 3 and this lane's table
   auto write_cs = [&](int n) {
-    const float4* c0 = reinterpret_cast<const float4*>(cs0 + (n & 1) * 64 + 32 * hh);
+    uint32_t cj[32], sj[32];
+    tmem_ld32x32b_x32(cj, tmem + T_CSJ + 64 * hh + lane_off);
+    tmem_ld32x32b_x32(sj, tmem + T_CSJ + 64 * hh + 32 + lane_off);
+    tmem_wait_ld_r32(cj);
+    tmem_wait_ld_r32(sj);
+    const float4* c0 = reinterpret_cast<const float4*>(cs0 + (n & 3) * 64 + 32 * hh);
     uint32_t cw[16], sw[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e) {
       const float4 v = c0[e];   // (cos, sin) of frequencies 2e, 2e + 1 of this half
       const uint64_t cc = f2(v.x, v.z), ss = f2(v.y, v.w), nss = f2(-v.y, -v.w);
-      const float2 co = f2_unpack(fma_f2(cc, CJ[e], mul_f2(nss, SJ[e])));
-      const float2 si = f2_unpack(fma_f2(ss, CJ[e], mul_f2(cc, SJ[e])));
+      const uint64_t CJ = f2(__uint_as_float(cj[2 * e]), __uint_as_float(cj[2 * e + 1]));
+      const uint64_t SJ = f2(__uint_as_float(sj[2 * e]), __uint_as_float(sj[2 * e + 1]));
+      const float2 co = f2_unpack(fma_f2(cc, CJ, mul_f2(nss, SJ)));
+      const float2 si = f2_unpack(fma_f2(ss, CJ, mul_f2(cc, SJ)));
       cw[e] = pack_bf16(co.x, co.y);
       sw[e] = pack_bf16(si.x, si.y);
     }
-    tmem_st32x32b_x16(tmem + T_CS + 16 * hh + lane_off, cw);
-    tmem_st32x32b_x16(tmem + T_CS + 32 + 16 * hh + lane_off, sw);
+    const uint32_t tb = tmem + T_CS + 64 * (n & 1) + lane_off;
+    tmem_st32x32b_x16(tb + 16 * hh, cw);
+    tmem_st32x32b_x16(tb + 32 + 16 * hh, sw);
     tmem_wait_st();
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(bar(B_CSFULL));
+    if (lane == 0) mbar_arrive(bar(B_CSFULL + (n & 1)));
   };
 
   if (w < NSW) {
     // ======================================================== score warps
     if (n_tiles > 0) write_cs(0);
+    if (n_tiles > 1) write_cs(1);
     float m_ref[RH], l_st[RH];
 #pragma unroll
     for (int r = 0; r < RH; ++r) {
@@ -389,46 +431,50 @@ __global__ void __launch_bounds__(NTHR, 1)
       wt(B_TFULL, n & 1);
       if (has_new && p_new >= k0 && p_new < k0 + KT) wt(B_PATCH, 0);   // the new LR row is in place
       tc_fence_after();
-      // S (every row), this half's W columns, this key's LRk
+      // S (every row), this half's W columns (every load in flight before one
+      // wait), this key's LRk
+      constexpr int NCH = RH * R / 32;   // 32-column chunks of this half's W
       uint32_t sv[16];
+      uint32_t wv[NCH][32];
       tmem_ld32x32b_x16(sv, tmem + T_S + lane_off);
-      float lk[R];
+#pragma unroll
+      for (int ch = 0; ch < NCH; ++ch)
+        tmem_ld32x32b_x32(wv[ch], tmem + T_W + (uint32_t)(hh * RH * R + 32 * ch) + lane_off);
+      uint32_t lkw[R / 2];   // LRk of this key as bf16 pairs
       {
         const unsigned char* lrow = stages + s * C::STAGE + 2 * C::KV_TILE;
 #pragma unroll
         for (int c = 0; c < R; c += 8) {
           const uint4 v = *reinterpret_cast<const uint4*>(lrow + tile_off<2 * R, KT>(jk, c));
-          const float2 a0 = unpack_bf16(v.x), a1 = unpack_bf16(v.y), a2 = unpack_bf16(v.z), a3 = unpack_bf16(v.w);
-          lk[c] = a0.x; lk[c + 1] = a0.y; lk[c + 2] = a1.x; lk[c + 3] = a1.y;
-          lk[c + 4] = a2.x; lk[c + 5] = a2.y; lk[c + 6] = a3.x; lk[c + 7] = a3.y;
+          lkw[c / 2] = v.x; lkw[c / 2 + 1] = v.y; lkw[c / 2 + 2] = v.z; lkw[c / 2 + 3] = v.w;
         }
       }
+      tmem_wait_ld_r16(sv);
+#pragma unroll
+      for (int ch = 0; ch < NCH; ++ch) reg_after_wait32(wv[ch]);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(B_WFREE));   // S and W of this tile are in registers
       float dsc[RH];
       constexpr int RPC = 32 / R;   // rows per 32-column chunk
 #pragma unroll
-      for (int ch = 0; ch < RH / RPC; ++ch) {
-        uint32_t wv[32];
-        tmem_ld32x32b_x32(wv, tmem + T_W + (uint32_t)(hh * RH * R + 32 * ch) + lane_off);
-        tmem_wait_ld_r32(wv);
+      for (int ch = 0; ch < NCH; ++ch)
 #pragma unroll
         for (int rr = 0; rr < RPC; ++rr) {
           uint64_t acc = f2(0.f, 0.f);
 #pragma unroll
-          for (int rho = 0; rho < R; rho += 2)
-            acc = fma_f2(f2(lk[rho], lk[rho + 1]),
-                         f2(__uint_as_float(wv[rr * R + rho]), __uint_as_float(wv[rr * R + rho + 1])), acc);
+          for (int rho = 0; rho < R; rho += 2) {
+            const float2 l2 = unpack_bf16(lkw[rho / 2]);
+            acc = fma_f2(f2(l2.x, l2.y),
+                         f2(__uint_as_float(wv[ch][rr * R + rho]), __uint_as_float(wv[ch][rr * R + rho + 1])), acc);
+          }
           const float2 a2 = f2_unpack(acc);
           dsc[ch * RPC + rr] = a2.x + a2.y;
         }
-      }
-      tmem_wait_ld_r16(sv);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(B_WFREE));   // S and W of this tile are in registers
-      if (n + 1 < n_tiles) write_cs(n + 1);        // W of this tile has read CS: refill it
-      if (sp == 0 && n + 2 < n_tiles) {            // exact (cos, sin)(k0 theta) two tiles ahead
+      if (n + 2 < n_tiles) write_cs(n + 2);        // W of this tile has read its CS buffer
+      if (sp == 0 && n + 3 < n_tiles) {            // exact (cos, sin)(k0 theta) three tiles ahead
         const int i = 32 * hh + lane;
-        cs0[(n & 1) * 64 + i] = rope_cs_exact(k0 + 2 * KT, theta[i]);
+        cs0[((n + 3) & 3) * 64 + i] = rope_cs_exact(k0 + 3 * KT, theta[i]);
       }
       // scores (log2 units) and this tile's row maxima
       float x[RH];
@@ -587,7 +633,7 @@ __global__ void __launch_bounds__(NTHR, 1)
     // kv_len and not used, and those still in flight after a wait ran out
     if (lane == 0)
       for (int m = max(n_seen, n_issued - ST); m < n_issued; ++m)
-        if (!mbar_wait_ns(bar(B_FULL + m % ST), (m / ST) & 1)) fail = 1;
+        if (!mbar_wait_clk(bar(B_FULL + m % ST), (m / ST) & 1)) fail = 1;
     // the partial's O_lr (the UV area is free once every MMA has completed)
     if (n_tiles > 0) wt(B_ODONE, 0);
 #pragma unroll
@@ -624,7 +670,7 @@ __global__ void __launch_bounds__(NTHR, 1)
         const int s = n % ST;
         wt(B_FULL + s, (n / ST) & 1);
         if (n > 0) wt(B_WFREE, (n - 1) & 1);
-        wt(B_CSFULL, n & 1);
+        wt(B_CSFULL + (n & 1), (n >> 1) & 1);
         tc_fence_after();
         const uint64_t dK = umma_desc(st_u + s * C::STAGE, 16, 1024, 2);
 #pragma unroll
@@ -633,7 +679,7 @@ __global__ void __launch_bounds__(NTHR, 1)
                     umma_desc_add(dQ, (kk >> 2) * (QP * 128) + (kk & 3) * 32), ID_S, kk > 0);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          umma_bf16_ts(tmem + T_W, tmem + T_CS + kk * 8,
+          umma_bf16_ts(tmem + T_W, tmem + T_CS + 64 * (n & 1) + kk * 8,
                        umma_desc_add(dUV, (kk >> 2) * (NW * 128) + (kk & 3) * 32), ID_W, kk > 0);
         umma_commit(bar(B_TFULL));
         if (n > 0) mma_pv(n - 1);
@@ -642,7 +688,7 @@ __global__ void __launch_bounds__(NTHR, 1)
       umma_commit(bar(B_ODONE));
       // TMEM is freed below: every MMA has completed first (an MMA always
       // completes, so this wait does not run out)
-      if (!mbar_wait_ns(bar(B_ODONE), 0)) fail = 1;
+      if (!mbar_wait_clk(bar(B_ODONE), 0)) fail = 1;
     }
     __syncwarp();
   }
@@ -737,40 +783,61 @@ __global__ void __launch_bounds__(NTHR, 1)
   }
   __threadfence();
   __syncthreads();
-  // this CTA's partial stays in shared memory; the others are read from L2
-  auto part = [&](int k, int row) -> const float* {
-    return k == split ? Part + row * WP : ws_unit + ((size_t)k * RP + row) * WP;
-  };
-  // (a) per row: M = max_k m_k, weights w_k = 2^(m_k - M) / sum_k 2^(m_k - M) l_k
-  float* Wt = reinterpret_cast<float*>(stages);     // [RP][kMaxSplits] (the stages are drained)
-  float* Mg = Wt + RP * kMaxSplits;                  // merged rows [RP][WP]
+  // this CTA's partial stays in shared memory; the others are staged into the
+  // drained stages by cp.async, as many splits at a time as fit
+  constexpr int PF = RP * WP;                        // floats of one split's partial
+  float* Wt = Part + PF;                             // [RP][kMaxSplits] 2^(m_k - M)
+  float2* ML = reinterpret_cast<float2*>(Wt + RP * kMaxSplits);   // [RP][kMaxSplits] (m, l)
+  float* Mg = reinterpret_cast<float*>(ML + RP * kMaxSplits);     // [RP][WP] merged rows
+  float* Sp = reinterpret_cast<float*>(stages);
+  const int kchunk = max(1, min(ns, (int)((size_t)ST * C::STAGE / (PF * 4))));
+  // (a) every split's (m, l) of every row (one round of independent loads)
+  for (int i = tid; i < ns * n_rows; i += NTHR) {
+    const int k = i / n_rows, row = i % n_rows;
+    ML[row * kMaxSplits + k] = k == split ? make_float2(Part[row * WP + D + R], Part[row * WP + D + R + 1])
+                                          : __ldcg(reinterpret_cast<const float2*>(ws_unit + (size_t)k * PF + row * WP + D + R));
+  }
+  __syncthreads();
+  // (b) per row, one warp: M = max_k m_k, w_k = 2^(m_k - M), L = sum_k w_k l_k
   for (int row = w; row < n_rows; row += NTHR / 32) {
-    float2 ml = make_float2(-INFINITY, 0.f);
-    if (lane < ns) {
-      const float* pr = part(lane, row);
-      ml = lane == split ? make_float2(pr[D + R], pr[D + R + 1])
-                         : __ldcg(reinterpret_cast<const float2*>(pr + D + R));
-    }
+    const float2 ml = lane < ns ? ML[row * kMaxSplits + lane] : make_float2(-INFINITY, 0.f);
     const float M = warp_max(ml.x);
     const float e = (lane < ns && ml.x != -INFINITY) ? fast_exp2(ml.x - M) : 0.f;
     const float L = warp_sum(e * ml.y);
     if (lane < ns) Wt[row * kMaxSplits + lane] = e;
     if (lane == 0) Mg[row * WP + D + R + 1] = L;
   }
-  __syncthreads();
-  // (b) merged O and O_lr, unnormalised (emit divides by L)
-  for (int i = tid; i < n_rows * ((D + R) / 4); i += NTHR) {
-    const int row = i / ((D + R) / 4), c = 4 * (i % ((D + R) / 4));
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int k = 0; k < ns; ++k) {
-      const float wk = Wt[row * kMaxSplits + k];
-      if (wk == 0.f) continue;
-      const float* pr = part(k, row) + c;
-      const float4 v = k == split ? *reinterpret_cast<const float4*>(pr) : __ldcg(reinterpret_cast<const float4*>(pr));
-      acc.x = fmaf(wk, v.x, acc.x); acc.y = fmaf(wk, v.y, acc.y);
-      acc.z = fmaf(wk, v.z, acc.z); acc.w = fmaf(wk, v.w, acc.w);
+  // (c) sum_k w_k (O_base,k | O_lr,k), a thread per 4 columns of a row
+  constexpr int CI = (D + R) / 4;
+  const int n_items = n_rows * CI;
+  float4 acc[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
+  for (int kc0 = 0; kc0 < ns; kc0 += kchunk) {
+    const int kc1 = min(ns, kc0 + kchunk);
+    __syncthreads();   // the weights are in place; the previous chunk is consumed
+    for (int i = tid; i < (kc1 - kc0) * (PF / 4); i += NTHR) {
+      const int k = kc0 + i / (PF / 4);
+      if (k != split) cp_async16(smem_u32(Sp + (size_t)i * 4), ws_unit + (size_t)k * PF + (i % (PF / 4)) * 4);
     }
-    *reinterpret_cast<float4*>(Mg + row * WP + c) = acc;
+    cp_async_wait_all();
+    __syncthreads();
+#pragma unroll
+    for (int j2 = 0; j2 < 2; ++j2) {
+      const int it = tid + j2 * NTHR;
+      if (it >= n_items) continue;
+      const int row = it / CI, c = 4 * (it % CI);
+      for (int k = kc0; k < kc1; ++k) {
+        const float wk = Wt[row * kMaxSplits + k];
+        const float4 v = *reinterpret_cast<const float4*>(
+            k == split ? Part + row * WP + c : Sp + (size_t)(k - kc0) * PF + row * WP + c);
+        acc[j2].x = fmaf(wk, v.x, acc[j2].x); acc[j2].y = fmaf(wk, v.y, acc[j2].y);
+        acc[j2].z = fmaf(wk, v.z, acc[j2].z); acc[j2].w = fmaf(wk, v.w, acc[j2].w);
+      }
+    }
+  }
+#pragma unroll
+  for (int j2 = 0; j2 < 2; ++j2) {
+    const int it = tid + j2 * NTHR;
+    if (it < n_items) *reinterpret_cast<float4*>(Mg + (it / CI) * WP + 4 * (it % CI)) = acc[j2];
   }
   __syncthreads();
   if (!s_misc[0])
@@ -827,7 +894,7 @@ int device_sms() {
 int rows_padded(const AttnParams& p, int G) {
   const int rows = G * p.g;
   const int rp = (rows + 3) / 4 * 4;
-  if (p.r == 16) return rp <= 16 ? rp : 0;
+  if (p.r == 16) return rp <= 12 ? rp : 0;
   if (p.r == 32) return rp <= 4 ? rp : 0;
   return 0;
 }
@@ -837,8 +904,7 @@ size_t smem_of(int r, int rp) {
   switch (rp) {
     case 4: return Cfg<16, 4>::smem();
     case 8: return Cfg<16, 8>::smem();
-    case 12: return Cfg<16, 12>::smem();
-    default: return Cfg<16, 16>::smem();
+    default: return Cfg<16, 12>::smem();
   }
 }
 
@@ -939,8 +1005,7 @@ cudaError_t launch_decode_cs(const AttnParams& pin, la_dtype out, cudaStream_t s
   switch (rows_padded(p, p.agent_group)) {
     case 4: return launch_t<16, 4>(p, st);
     case 8: return launch_t<16, 8>(p, st);
-    case 12: return launch_t<16, 12>(p, st);
-    default: return launch_t<16, 16>(p, st);
+    default: return launch_t<16, 12>(p, st);
   }
 }
 
