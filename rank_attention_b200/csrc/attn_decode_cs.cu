@@ -72,7 +72,7 @@ constexpr uint32_t T_W = 0, T_CS = 192, T_CSJ = 320, T_S = 448, T_O = 464, T_COL
 
 // barriers (mbarrier slots)
 enum { B_FULL = 0, B_EMPTY = ST, B_TFULL = 2 * ST, B_WFREE, B_CSFULL, B_CSFULL1, B_PFULL, B_PFREE,
-       B_ODONE, B_PATCH, B_NUM };
+       B_ODONE, B_PATCH, B_OPS, B_NUM };
 
 template <int R, int RP>
 struct Cfg {
@@ -206,6 +206,7 @@ __global__ void __launch_bounds__(NTHR, 1)
     mbar_init(bar(B_PFREE), 2);
     mbar_init(bar(B_ODONE), 1);
     mbar_init(bar(B_PATCH), 1);
+    mbar_init(bar(B_OPS), 1);
     fence_mbar_init();
     tma_prefetch(&tmK);
     tma_prefetch(&tmV);
@@ -213,6 +214,17 @@ __global__ void __launch_bounds__(NTHR, 1)
     // a programmatic dependent of the preceding kernel (the step's LR append):
     // everything above overlaps its tail, every input is read after the wait
     pdl_wait();
+    // the queries (rows a g + gi, unswizzled, into the P buffer) and the B_k^a
+    // head slices (rows a R + rho, into the [U | V] area) before the tiles, so
+    // that these few kilobytes do not queue behind the tiles' megabytes
+    const __nv_bfloat16* Q = reinterpret_cast<const __nv_bfloat16*>(p.q);
+    const __nv_bfloat16* Bk = reinterpret_cast<const __nv_bfloat16*>(p.B_k);
+    mbar_expect_tx(bar(B_OPS), (uint32_t)(na * g * D * 2 + na * R * D * 2));
+    for (int a = 0; a < na; ++a)
+      bulk_load(p_u + a * g * D * 2, Q + (((int64_t)seq * na_tot + agent0 + a) * p.n_q + kvh * g) * D,
+                (uint32_t)(g * D * 2), bar(B_OPS));
+    for (int i = 0; i < na * R; ++i)
+      bulk_load(uv_u + i * D * 2, Bk + ((int64_t)agent0 * R + i) * ldB + kvh * D, D * 2, bar(B_OPS));
     for (int n = 0; n < n_spec; ++n) issue(n);
   }
   if (tid < D / 2) theta[tid] = rt.theta[tid];
@@ -223,20 +235,32 @@ __global__ void __launch_bounds__(NTHR, 1)
   const int64_t k_hi = bad_len ? k_lo : min(te * KT, kvl);
   const int n_tiles = k_hi > k_lo ? (int)((k_hi - k_lo + KT - 1) / KT) : 0;
 
-  // ---- the queries: the B operand of S (swizzled), read back by the [U | V] build
+  // ---- the staged queries into the B operand of S (swizzled); this thread's
+  // B_k^a chunks of the [U | V] build into registers.  An item of the build is
+  // (agent, rho, 8 frequencies).
+  const bool ops_ok = mbar_wait_clk(bar(B_OPS), 0);
+  const int n_ag = (RP + g - 1) / g;            // agents whose rows fall within RP
+  const int items = n_ag * R * 8;
+  constexpr int MAXK = 4;                       // items per thread (at most 4 agents x 32 x 8)
+  uint4 b1[MAXK], b2[MAXK];
   {
-    const __nv_bfloat16* Q = reinterpret_cast<const __nv_bfloat16*>(p.q);
     for (int it = tid; it < QP * (D / 8); it += NTHR) {
       const int row = it / (D / 8), c = (it % (D / 8)) * 8;
       uint4 v = make_uint4(0, 0, 0, 0);
-      if (row < n_rows && !bad_len) {
-        const int a = row / g, gi = row % g;
-        v = __ldg(reinterpret_cast<const uint4*>(Q + (((int64_t)seq * na_tot + agent0 + a) * p.n_q + kvh * g + gi) * D + c));
-      }
+      if (row < n_rows && !bad_len) v = *reinterpret_cast<const uint4*>(pbuf + row * D * 2 + c * 2);
       *reinterpret_cast<uint4*>(qop + tile_off<D, QP>(row, c)) = v;
     }
-    for (int it = tid; it < C::P_BYTES / 16; it += NTHR)
-      *reinterpret_cast<uint4*>(pbuf + it * 16) = make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int k = 0; k < MAXK; ++k) {
+      const int it = tid + k * NTHR;
+      b1[k] = b2[k] = make_uint4(0, 0, 0, 0);
+      const int a = it / (R * 8), rho = (it / 8) % R, i0 = (it & 7) * 8;
+      if (it < items && a < na && !bad_len) {
+        const unsigned char* br = uv + (a * R + rho) * D * 2;
+        b1[k] = *reinterpret_cast<const uint4*>(br + i0 * 2);
+        b2[k] = *reinterpret_cast<const uint4*>(br + (D / 2 + i0) * 2);
+      }
+    }
   }
   // ---- decode step in one launch: the CTA whose keys hold position kv_len - 1
   // forms that token's LR row x_new [A_k | A_v] (fp32 sums, rounded to bf16
@@ -292,27 +316,11 @@ __global__ void __launch_bounds__(NTHR, 1)
 
   // ---- [U | V]: the B operand of W = CS UV^T, a row per (query row, rho):
   // U = s (q_i B_i + q_{i+d/2} B_{i+d/2}) in K columns i, V = s (q_{i+d/2} B_i -
-  // q_i B_{i+d/2}) in K columns d/2 + i.  An item is (agent, rho, 8
-  // frequencies): its B_k^a chunks are loaded (all of a thread's items at
-  // once), then combined with each of the agent's g staged query rows.
+  // q_i B_{i+d/2}) in K columns d/2 + i, over each of the agent's g query rows
+  for (int it = tid; it < C::P_BYTES / 16; it += NTHR)
+    *reinterpret_cast<uint4*>(pbuf + it * 16) = make_uint4(0, 0, 0, 0);
   {
-    const __nv_bfloat16* Bk = reinterpret_cast<const __nv_bfloat16*>(p.B_k);
     const float s = p.s;
-    const int n_ag = (RP + g - 1) / g;          // agents whose rows fall within RP
-    const int items = n_ag * R * 8;
-    constexpr int MAXK = 4;                     // items per thread (at most 4 agents x 32 x 8)
-    uint4 b1[MAXK], b2[MAXK];
-#pragma unroll
-    for (int k = 0; k < MAXK; ++k) {
-      const int it = tid + k * NTHR;
-      b1[k] = b2[k] = make_uint4(0, 0, 0, 0);
-      const int a = it / (R * 8), rho = (it / 8) % R, i0 = (it & 7) * 8;
-      if (it < items && a < na && !bad_len) {
-        const __nv_bfloat16* br = Bk + ((int64_t)(agent0 + a) * R + rho) * ldB + kvh * D;
-        b1[k] = __ldg(reinterpret_cast<const uint4*>(br + i0));
-        b2[k] = __ldg(reinterpret_cast<const uint4*>(br + D / 2 + i0));
-      }
-    }
 #pragma unroll
     for (int k = 0; k < MAXK; ++k) {
       const int it = tid + k * NTHR;
@@ -692,7 +700,7 @@ __global__ void __launch_bounds__(NTHR, 1)
     }
     __syncwarp();
   }
-  if (fail) s_misc[0] = 1;
+  if (fail || !ops_ok) s_misc[0] = 1;
   tc_fence_before();
   __syncthreads();
   if (w == WM) {
