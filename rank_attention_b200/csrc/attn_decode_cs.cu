@@ -116,8 +116,8 @@ __device__ __forceinline__ int ld_acquire(const int* p) { return ld_acquire_gpu(
 template <int R, int RP>
 __global__ void __launch_bounds__(NTHR, 1)
     decode_cs_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                     const __grid_constant__ CUtensorMap tmL, const AttnParams p,
-                     const __grid_constant__ RopeTheta rt) {
+                     const __grid_constant__ CUtensorMap tmL, const __grid_constant__ CUtensorMap tmB,
+                     const AttnParams p, const __grid_constant__ RopeTheta rt) {
   using C = Cfg<R, RP>;
   constexpr int NW = C::NW, RH = C::RH, WP = C::WP;
   extern __shared__ unsigned char smem_raw[];
@@ -211,20 +211,23 @@ __global__ void __launch_bounds__(NTHR, 1)
     tma_prefetch(&tmK);
     tma_prefetch(&tmV);
     tma_prefetch(&tmL);
+    tma_prefetch(&tmB);
     // a programmatic dependent of the preceding kernel (the step's LR append):
     // everything above overlaps its tail, every input is read after the wait
     pdl_wait();
     // the queries (rows a g + gi, unswizzled, into the P buffer) and the B_k^a
-    // head slices (rows a R + rho, into the [U | V] area) before the tiles, so
-    // that these few kilobytes do not queue behind the tiles' megabytes
+    // head slices (per agent R rows x two 64-column boxes, 128-byte swizzle,
+    // into the [U | V] area) before the tiles, so that these few kilobytes do
+    // not queue behind the tiles' megabytes
     const __nv_bfloat16* Q = reinterpret_cast<const __nv_bfloat16*>(p.q);
-    const __nv_bfloat16* Bk = reinterpret_cast<const __nv_bfloat16*>(p.B_k);
     mbar_expect_tx(bar(B_OPS), (uint32_t)(na * g * D * 2 + na * R * D * 2));
     for (int a = 0; a < na; ++a)
       bulk_load(p_u + a * g * D * 2, Q + (((int64_t)seq * na_tot + agent0 + a) * p.n_q + kvh * g) * D,
                 (uint32_t)(g * D * 2), bar(B_OPS));
-    for (int i = 0; i < na * R; ++i)
-      bulk_load(uv_u + i * D * 2, Bk + ((int64_t)agent0 * R + i) * ldB + kvh * D, D * 2, bar(B_OPS));
+    for (int a = 0; a < na; ++a)
+#pragma unroll
+      for (int b = 0; b < D / 64; ++b)
+        tma_load_3d(uv_u + a * R * D * 2 + b * R * 128, &tmB, bar(B_OPS), kvh * D + 64 * b, 0, agent0 + a);
     for (int n = 0; n < n_spec; ++n) issue(n);
   }
   if (tid < D / 2) theta[tid] = rt.theta[tid];
@@ -256,9 +259,9 @@ __global__ void __launch_bounds__(NTHR, 1)
       b1[k] = b2[k] = make_uint4(0, 0, 0, 0);
       const int a = it / (R * 8), rho = (it / 8) % R, i0 = (it & 7) * 8;
       if (it < items && a < na && !bad_len) {
-        const unsigned char* br = uv + (a * R + rho) * D * 2;
-        b1[k] = *reinterpret_cast<const uint4*>(br + i0 * 2);
-        b2[k] = *reinterpret_cast<const uint4*>(br + (D / 2 + i0) * 2);
+        const unsigned char* br = uv + a * R * D * 2;
+        b1[k] = *reinterpret_cast<const uint4*>(br + tile_off<D, R>(rho, i0));
+        b2[k] = *reinterpret_cast<const uint4*>(br + tile_off<D, R>(rho, D / 2 + i0));
       }
     }
   }
@@ -372,7 +375,7 @@ __global__ void __launch_bounds__(NTHR, 1)
     if (sp == 0) {
       const int i = 32 * hh + lane;
 #pragma unroll
-      for (int t = 0; t < 3; ++t) cs0[t * 64 + i] = rope_cs_exact(k_lo + (int64_t)t * KT, rt.theta[i]);
+      for (int t = 0; t < 3; ++t) cs0[t * 64 + i] = rope_cs_sfu(k_lo + (int64_t)t * KT, rt.theta[i]);
     }
   }
 
@@ -425,6 +428,12 @@ __global__ void __launch_bounds__(NTHR, 1)
     // ======================================================== score warps
     if (n_tiles > 0) write_cs(0);
     if (n_tiles > 1) write_cs(1);
+    // the incremental (cos, sin)(k0 theta) of this lane's frequency (sp == 0)
+    float2 cs_cur = make_float2(1.f, 0.f), cs_step = cs_cur;
+    if (sp == 0) {
+      cs_cur = cs0[2 * 64 + 32 * hh + lane];
+      cs_step = rope_cs_sfu(KT, theta[32 * hh + lane]);
+    }
     float m_ref[RH], l_st[RH];
 #pragma unroll
     for (int r = 0; r < RH; ++r) {
@@ -479,11 +488,6 @@ __global__ void __launch_bounds__(NTHR, 1)
           const float2 a2 = f2_unpack(acc);
           dsc[ch * RPC + rr] = a2.x + a2.y;
         }
-      if (n + 2 < n_tiles) write_cs(n + 2);        // W of this tile has read its CS buffer
-      if (sp == 0 && n + 3 < n_tiles) {            // exact (cos, sin)(k0 theta) three tiles ahead
-        const int i = 32 * hh + lane;
-        cs0[((n + 3) & 3) * 64 + i] = rope_cs_exact(k0 + 3 * KT, theta[i]);
-      }
       // scores (log2 units) and this tile's row maxima
       float x[RH];
 #pragma unroll
@@ -534,6 +538,17 @@ __global__ void __launch_bounds__(NTHR, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(B_PFULL));
+      // off the tile's critical path: CS two tiles ahead (W of this tile has read
+      // its buffer), and (cos, sin)(k0 theta) three tiles ahead: the previous
+      // one turned by KT theta in fp32, taken exactly again every 16 tiles
+      if (n + 2 < n_tiles) write_cs(n + 2);
+      if (sp == 0 && n + 3 < n_tiles) {
+        const int m = n + 3;
+        cs_cur = (m & 15) == 0 ? rope_cs_sfu(k_lo + (int64_t)m * KT, theta[32 * hh + lane])
+                               : make_float2(fmaf(cs_cur.x, cs_step.x, -cs_cur.y * cs_step.y),
+                                             fmaf(cs_cur.y, cs_step.x, cs_cur.x * cs_step.y));
+        cs0[(m & 3) * 64 + 32 * hh + lane] = cs_cur;
+      }
     }
     // ---- partial of this CTA: l (over the keys), m, O^T
 #pragma unroll
@@ -569,6 +584,10 @@ __global__ void __launch_bounds__(NTHR, 1)
     int n_issued = n_spec, n_seen = 0;   // tiles requested / observed landed (lane 0)
     if (lane == 0)
       for (int m = ST; m < n_tiles && m < ST + kL2Ahead; ++m) prefetch(m);
+    {   // B_v^a head slices for the epilogue, into L2 while the keys stream
+      const __nv_bfloat16* bvp = reinterpret_cast<const __nv_bfloat16*>(p.B_v) + (int64_t)agent0 * R * ldB + kvh * D;
+      for (int i = lane; i < na * R * 2; i += 32) prefetch_l2(bvp + (int64_t)(i >> 1) * ldB + 64 * (i & 1));
+    }
     for (int n = 0; n < n_tiles; ++n) {
       const int s = n % ST;
       const int64_t k0 = k_lo + (int64_t)n * KT;
@@ -758,10 +777,14 @@ __global__ void __launch_bounds__(NTHR, 1)
     return;
   }
 
-  // ---- split merge: a ticket per CTA; all but the last publish their partial
-  int* ctr = p.counters + unitg;
-  int* flags = p.counters + n_units_g + (size_t)unitg * kMaxSplits;
+  // ---- split merge.  Each CTA takes a ticket; the last merge_ctas tickets
+  // merge (each a share of the rows), the others publish their partial and
+  // leave.  A merging CTA waits only for CTAs that have taken a ticket or, with
+  // several merging CTAs (a launch of one wave), for CTAs of that wave.
+  int* ctr = p.counters + 2 * unitg;                 // [arrivals, mergers done]
+  int* flags = p.counters + 2 * n_units_g + (size_t)unitg * kMaxSplits;
   float* ws_unit = p.partials + (size_t)unitg * ns * RP * WP;
+  const int nm = max(1, min(p.merge_ctas, ns));
   if (tid == 0) s_misc[1] = atomicAdd(ctr, 1);
   __syncthreads();
   const int ticket = s_misc[1];
@@ -769,16 +792,16 @@ __global__ void __launch_bounds__(NTHR, 1)
     if (tid == 0) atomicOr(p.err, 4);
     return;
   }
-  if (ticket != ns - 1) {
+  const int mi = ticket - (ns - nm);                 // this CTA's share of the merge, if >= 0
+  if (mi < 0 || nm > 1) {                            // publish (the other merging CTAs read it too)
     float4* dst = reinterpret_cast<float4*>(ws_unit + (size_t)split * RP * WP);
     for (int i = tid; i < RP * WP / 4; i += NTHR) __stcg(dst + i, reinterpret_cast<const float4*>(Part)[i]);
     __threadfence();
     __syncthreads();
     if (tid == 0) atomicExch(flags + split, 1);
-    return;
+    if (mi < 0) return;
   }
-  // the last CTA: every other split has taken its ticket; wait (bounded) until
-  // each has published, then merge
+  // wait (bounded) until every other split has published
   if (tid < ns && tid != split) {
     int it = 0;
     while (ld_acquire(flags + tid) == 0) {
@@ -791,6 +814,8 @@ __global__ void __launch_bounds__(NTHR, 1)
   }
   __threadfence();
   __syncthreads();
+  const int r0 = mi * n_rows / nm, r1 = (mi + 1) * n_rows / nm;   // this CTA's rows
+  const int nr = r1 - r0;
   // this CTA's partial stays in shared memory; the others are staged into the
   // drained stages by cp.async, as many splits at a time as fit
   constexpr int PF = RP * WP;                        // floats of one split's partial
@@ -798,16 +823,16 @@ __global__ void __launch_bounds__(NTHR, 1)
   float2* ML = reinterpret_cast<float2*>(Wt + RP * kMaxSplits);   // [RP][kMaxSplits] (m, l)
   float* Mg = reinterpret_cast<float*>(ML + RP * kMaxSplits);     // [RP][WP] merged rows
   float* Sp = reinterpret_cast<float*>(stages);
-  const int kchunk = max(1, min(ns, (int)((size_t)ST * C::STAGE / (PF * 4))));
-  // (a) every split's (m, l) of every row (one round of independent loads)
-  for (int i = tid; i < ns * n_rows; i += NTHR) {
-    const int k = i / n_rows, row = i % n_rows;
+  const int kchunk = max(1, min(ns, (int)((size_t)ST * C::STAGE / (nr > 0 ? nr * WP * 4 : 1))));
+  // (a) every split's (m, l) of this CTA's rows (one round of independent loads)
+  for (int i = tid; i < ns * nr; i += NTHR) {
+    const int k = i / nr, row = r0 + i % nr;
     ML[row * kMaxSplits + k] = k == split ? make_float2(Part[row * WP + D + R], Part[row * WP + D + R + 1])
                                           : __ldcg(reinterpret_cast<const float2*>(ws_unit + (size_t)k * PF + row * WP + D + R));
   }
   __syncthreads();
   // (b) per row, one warp: M = max_k m_k, w_k = 2^(m_k - M), L = sum_k w_k l_k
-  for (int row = w; row < n_rows; row += NTHR / 32) {
+  for (int row = r0 + w; row < r1; row += NTHR / 32) {
     const float2 ml = lane < ns ? ML[row * kMaxSplits + lane] : make_float2(-INFINITY, 0.f);
     const float M = warp_max(ml.x);
     const float e = (lane < ns && ml.x != -INFINITY) ? fast_exp2(ml.x - M) : 0.f;
@@ -817,14 +842,15 @@ __global__ void __launch_bounds__(NTHR, 1)
   }
   // (c) sum_k w_k (O_base,k | O_lr,k), a thread per 4 columns of a row
   constexpr int CI = (D + R) / 4;
-  const int n_items = n_rows * CI;
+  const int n_items = nr * CI;
   float4 acc[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
   for (int kc0 = 0; kc0 < ns; kc0 += kchunk) {
     const int kc1 = min(ns, kc0 + kchunk);
     __syncthreads();   // the weights are in place; the previous chunk is consumed
-    for (int i = tid; i < (kc1 - kc0) * (PF / 4); i += NTHR) {
-      const int k = kc0 + i / (PF / 4);
-      if (k != split) cp_async16(smem_u32(Sp + (size_t)i * 4), ws_unit + (size_t)k * PF + (i % (PF / 4)) * 4);
+    for (int i = tid; i < (kc1 - kc0) * nr * (WP / 4); i += NTHR) {   // staged as [k][row][WP]
+      const int k = kc0 + i / (nr * (WP / 4)), rem = i % (nr * (WP / 4));
+      if (k != split)
+        cp_async16(smem_u32(Sp + (size_t)i * 4), ws_unit + (size_t)k * PF + (size_t)(r0 + rem / (WP / 4)) * WP + (rem % (WP / 4)) * 4);
     }
     cp_async_wait_all();
     __syncthreads();
@@ -832,11 +858,11 @@ __global__ void __launch_bounds__(NTHR, 1)
     for (int j2 = 0; j2 < 2; ++j2) {
       const int it = tid + j2 * NTHR;
       if (it >= n_items) continue;
-      const int row = it / CI, c = 4 * (it % CI);
+      const int rl = it / CI, row = r0 + rl, c = 4 * (it % CI);
       for (int k = kc0; k < kc1; ++k) {
         const float wk = Wt[row * kMaxSplits + k];
         const float4 v = *reinterpret_cast<const float4*>(
-            k == split ? Part + row * WP + c : Sp + (size_t)(k - kc0) * PF + row * WP + c);
+            k == split ? Part + row * WP + c : Sp + ((size_t)(k - kc0) * nr + rl) * WP + c);
         acc[j2].x = fmaf(wk, v.x, acc[j2].x); acc[j2].y = fmaf(wk, v.y, acc[j2].y);
         acc[j2].z = fmaf(wk, v.z, acc[j2].z); acc[j2].w = fmaf(wk, v.w, acc[j2].w);
       }
@@ -845,17 +871,26 @@ __global__ void __launch_bounds__(NTHR, 1)
 #pragma unroll
   for (int j2 = 0; j2 < 2; ++j2) {
     const int it = tid + j2 * NTHR;
-    if (it < n_items) *reinterpret_cast<float4*>(Mg + (it / CI) * WP + 4 * (it % CI)) = acc[j2];
+    if (it < n_items) *reinterpret_cast<float4*>(Mg + (r0 + it / CI) * WP + 4 * (it % CI)) = acc[j2];
   }
   __syncthreads();
   if (!s_misc[0])
-    for (int i = tid; i < n_rows * (D / 4); i += NTHR) {
-      const int row = i / (D / 4), c = 4 * (i % (D / 4));
+    for (int i = tid; i < nr * (D / 4); i += NTHR) {
+      const int row = r0 + i / (D / 4), c = 4 * (i % (D / 4));
       emit(Mg + row * WP, row, c);
     }
-  // reset the unit's counter and flags for the next call on this workspace
-  if (tid < ns) flags[tid] = 0;
-  if (tid == 0) *ctr = 0;
+  // the last merging CTA to finish resets the unit's counters and flags for
+  // the next call on this workspace
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    if (atomicAdd(ctr + 1, 1) == nm - 1) {
+      for (int k = 0; k < ns; ++k) flags[k] = 0;
+      ctr[1] = 0;
+      ctr[0] = 0;
+      __threadfence();
+    }
+  }
 }
 
 // -------------------------------------------------------------------- host
@@ -924,8 +959,19 @@ cudaError_t launch_t(const AttnParams& p, cudaStream_t st) {
     rt.theta[i] = i < D / 2 ? std::pow(p.rope_base, -2.0 * i / D) : 0.0;
     rt.thetaf[i] = (float)rt.theta[i];
   }
-  CUtensorMap mk, mv, ml;
+  CUtensorMap mk, mv, ml, mb;
   if (!make_maps(p, &mk, &mv, &ml)) return cudaErrorInvalidValue;
+  {
+    // B_k as (n_kv*d, r, n_agents): a CTA loads its head's r x 64 slices
+    cuuint64_t dims[3] = {(cuuint64_t)p.n_kv * D, (cuuint64_t)R, (cuuint64_t)p.n_agents};
+    cuuint64_t str[2] = {(cuuint64_t)p.n_kv * D * 2, (cuuint64_t)R * p.n_kv * D * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)R, 1};
+    cuuint32_t one[3] = {1, 1, 1};
+    if (encode_fn()(&mb, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(p.B_k), dims, str, box, one,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
   const size_t sm = Cf::smem();
   auto kern = decode_cs_kernel<R, RP>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
@@ -942,11 +988,11 @@ cudaError_t launch_t(const AttnParams& p, cudaStream_t st) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, kern, mk, mv, ml, p, rt);
+  e = cudaLaunchKernelEx(&cfg, kern, mk, mv, ml, mb, p, rt);
   if (e != cudaSuccess) {   // without the overlap where the runtime refuses it
     cudaGetLastError();
     cfg.numAttrs = 0;
-    e = cudaLaunchKernelEx(&cfg, kern, mk, mv, ml, p, rt);
+    e = cudaLaunchKernelEx(&cfg, kern, mk, mv, ml, mb, p, rt);
     if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
@@ -1009,6 +1055,11 @@ cudaError_t launch_decode_cs(const AttnParams& pin, la_dtype out, cudaStream_t s
   p.agent_group = cs_group_size(p);
   if (p.agent_group < 1) return cudaErrorInvalidValue;
   if (p.n_splits > kMaxSplits) return cudaErrorInvalidValue;
+  // several CTAs share a unit's merge only in a launch of one wave, where
+  // every CTA the merging ones wait for is running or about to run
+  const int64_t ctas = (int64_t)p.n_splits * ((p.n_agents + p.agent_group - 1) / p.agent_group) *
+                       p.n_seqs * p.n_kv;
+  p.merge_ctas = ctas <= device_sms() ? 4 : 1;
   if (p.r == 32) return launch_t<32, 4>(p, st);
   switch (rows_padded(p, p.agent_group)) {
     case 4: return launch_t<16, 4>(p, st);
@@ -1018,8 +1069,8 @@ cudaError_t launch_decode_cs(const AttnParams& pin, la_dtype out, cudaStream_t s
 }
 
 // Workspace of the cos/sin-table decode: per (agent group, unit) its splits'
-// partials [splits][rows padded][d + r + 4] fp32, then one arrival counter per
-// (group, unit) and a flag per split.
+// partials [splits][rows padded][d + r + 4] fp32, then per (group, unit) an
+// arrival and a merged counter, then per (group, unit) a flag per split.
 size_t cs_partial_bytes(const AttnParams& p) {
   const int G = cs_group_size(p);
   if (G < 1) return 0;
@@ -1033,7 +1084,7 @@ size_t cs_counter_ints(const AttnParams& p) {
   const int G = cs_group_size(p);
   if (G < 1) return 0;
   const int groups = (p.n_agents + G - 1) / G;
-  return (size_t)p.n_seqs * p.n_kv * groups * (1 + kMaxSplits);
+  return (size_t)p.n_seqs * p.n_kv * groups * (2 + kMaxSplits);
 }
 
 }  // namespace la

@@ -331,6 +331,10 @@ __device__ __forceinline__ void reg_after_wait32(uint32_t (&r)[32]) {
                :
                : "memory");
 }
+// a hint: bring the 128-byte line holding `ptr` into L2
+__device__ __forceinline__ void prefetch_l2(const void* ptr) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
+}
 // 16-byte copy global -> shared that bypasses L1 (cp.async), and the wait for
 // every such copy this thread has issued
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
