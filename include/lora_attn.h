@@ -255,6 +255,10 @@ la_status lora_decode_step_host(const la_attn_args* args, void* workspace,
 /*
  * lora_attn_prefill -- causal Flash-LoRA-Attention for a chunk of n_q_tokens
  * query tokens per (sequence, agent) over prefix + chunk.
+ * On the tensor-core path (bf16, head_dim 128, r in {16, 32, 64}) the score
+ * product takes the queries and each agent's keys K^a = K_base + delta in
+ * fp16 (the sum rounded once): queries and keys must stay below 65504 in
+ * magnitude there.
  * Errors: LA_ERR_INVALID_ARG, LA_ERR_UNSUPPORTED, LA_ERR_CAPACITY
  * (q_pos0 + n_q_tokens > L_max), LA_ERR_CUDA.
  */

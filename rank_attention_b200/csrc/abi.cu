@@ -147,6 +147,9 @@ DecodePlan plan_decode(const AttnParams& p, la_dtype io) {
   // (generic kernel), or the bf16 decode's own
   const size_t ints = d.kind == 1 ? bf16_decode_counter_ints(p) : (size_t)2 * units * d.groups;
   d.counter_bytes = (ints * sizeof(int) + 255) / 256 * 256;
+  // at least 256 bytes, so that the size query is nonzero for any valid call
+  // (the cos/sin-table decode merges inside its clusters and uses none of it)
+  if (d.partial_bytes + d.counter_bytes == 0 && units > 0) d.counter_bytes = 256;
   return d;
 }
 
@@ -330,8 +333,9 @@ la_status decode_prepare(const la_attn_args* a, void* workspace, size_t workspac
     return LA_OK;
   }
   DecodePlan d = plan_decode(*p, a->io_dtype);
-  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
-      workspace_bytes < d.partial_bytes + d.counter_bytes)
+  const size_t need = d.partial_bytes + d.counter_bytes;   // 0: no workspace, NULL allowed
+  if (need > 0 && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+                   workspace_bytes < need))
     return LA_ERR_WORKSPACE;
   if ((int64_t)p->n_seqs * p->n_kv > 65535) return LA_ERR_UNSUPPORTED;
   if (d.kind == 0 && simt_smem_bytes(*p) > 227 * 1024) return LA_ERR_UNSUPPORTED;

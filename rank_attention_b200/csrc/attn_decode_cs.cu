@@ -62,7 +62,7 @@ constexpr int NSW = 8;             // score warps
 constexpr int WV = 8, WM = 9;
 constexpr int NTHR = 32 * 10;
 constexpr int kL2Ahead = 4;        // tiles requested into L2 ahead of the stage loads
-constexpr int kMaxSplits = 32;
+constexpr int kMaxSplits = 16;    // splits of a unit: one cluster (16: non-portable size)
 constexpr int kSMs = 148;
 
 // TMEM columns: W (at most 192), the two CS buffers (64 each, bf16 pairs),
@@ -96,9 +96,8 @@ struct Cfg {
   }
   static_assert(NW <= 192, "W is one MMA of N <= 192 (TMEM columns 0..191)");
   static_assert(RP % 4 == 0 && RP <= QP, "rows");
-  // after the loop the UV area holds the partial, the merge's weights, (m, l)
-  // pairs and merged rows; the drained stages the other splits' partials
-  static_assert((size_t)RP * (2 * WP + 3 * kMaxSplits) * 4 <= (size_t)UV_BYTES, "merge area");
+  // after the loop the UV area holds the CTA's partial (read by the cluster)
+  static_assert((size_t)RP * WP * 4 <= (size_t)UV_BYTES, "partial area");
 };
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -726,10 +725,7 @@ __global__ void __launch_bounds__(NTHR, 1)
     tc_fence_after();
     tmem_dealloc(tmem, T_COLS);
   }
-  if (bad_len) {
-    if (tid == 0 && split == 0) atomicOr(p.err, 1);
-    return;
-  }
+  if (bad_len && tid == 0 && split == 0) atomicOr(p.err, 1);
   for (int row = tid; row < RP; row += NTHR) {
     Part[row * WP + D + R] = Mfin[row];
     Part[row * WP + D + R + 1] = Lsum[row * 4] + Lsum[row * 4 + 1] + Lsum[row * 4 + 2] + Lsum[row * 4 + 3];
@@ -769,7 +765,7 @@ __global__ void __launch_bounds__(NTHR, 1)
   };
 
   if (ns == 1) {
-    if (s_misc[0]) return;
+    if (s_misc[0] || bad_len) return;
     for (int i = tid; i < n_rows * (D / 4); i += NTHR) {
       const int row = i / (D / 4), c = 4 * (i % (D / 4));
       emit(Part + row * WP, row, c);
@@ -777,120 +773,49 @@ __global__ void __launch_bounds__(NTHR, 1)
     return;
   }
 
-  // ---- split merge.  Each CTA takes a ticket; the last merge_ctas tickets
-  // merge (each a share of the rows), the others publish their partial and
-  // leave.  A merging CTA waits only for CTAs that have taken a ticket or, with
-  // several merging CTAs (a launch of one wave), for CTAs of that wave.
-  int* ctr = p.counters + 2 * unitg;                 // [arrivals, mergers done]
-  int* flags = p.counters + 2 * n_units_g + (size_t)unitg * kMaxSplits;
-  float* ws_unit = p.partials + (size_t)unitg * ns * RP * WP;
-  const int nm = max(1, min(p.merge_ctas, ns));
-  if (tid == 0) s_misc[1] = atomicAdd(ctr, 1);
-  __syncthreads();
-  const int ticket = s_misc[1];
-  if (ticket < 0 || ticket >= ns) {   // a counter no call leaves behind: not a zeroed workspace
-    if (tid == 0) atomicOr(p.err, 4);
-    return;
-  }
-  const int mi = ticket - (ns - nm);                 // this CTA's share of the merge, if >= 0
-  if (mi < 0 || nm > 1) {                            // publish (the other merging CTAs read it too)
-    float4* dst = reinterpret_cast<float4*>(ws_unit + (size_t)split * RP * WP);
-    for (int i = tid; i < RP * WP / 4; i += NTHR) __stcg(dst + i, reinterpret_cast<const float4*>(Part)[i]);
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) atomicExch(flags + split, 1);
-    if (mi < 0) return;
-  }
-  // wait (bounded) until every other split has published
-  if (tid < ns && tid != split) {
-    int it = 0;
-    while (ld_acquire(flags + tid) == 0) {
-      if (++it > (1 << 22)) {
-        atomicOr(p.err, 4);
-        break;
+  // ---- split merge over the cluster.  The unit's splits are one thread-block
+  // cluster (rank = split); each CTA's partial (O_base, O_lr, m, l) stays in
+  // its own shared memory, and after a cluster barrier every CTA merges a share
+  // of the unit's (row, 32-column quarter) pieces, reading the partials of all
+  // splits over distributed shared memory, one warp per piece:
+  //   w_k = 2^(m_k - M) / sum_k 2^(m_k - M) l_k,  M = max_k m_k,
+  //   out = sum_k w_k O_base,k + s (sum_k w_k O_lr,k) B_v^a  (B_v^a once per row)
+  cluster_sync_all();   // every split's partial is in place
+  if (!s_misc[0] && !bad_len) {
+    const uint32_t part_u = smem_u32(Part);
+    for (int piece = split + ns * w; piece < n_rows * 4; piece += ns * (NTHR / 32)) {
+      const int row = piece >> 2, c0 = 32 * (piece & 3);
+      const uint32_t rowb = part_u + (uint32_t)(row * WP) * 4;
+      // lane k: split k's (m, l)
+      float2 ml = make_float2(-INFINITY, 0.f);
+      if (lane < ns) ml = dsmem_ld2(dsmem_addr(rowb + (D + R) * 4, lane));
+      const float M = warp_max(ml.x);
+      const float e = (lane < ns && ml.x != -INFINITY) ? fast_exp2(ml.x - M) : 0.f;
+      const float L = warp_sum(e * ml.y);
+      const float inv = L > 0.f ? 1.f / L : 0.f;
+      // lane c: the merged O_base of column c0 + c; lane rho: O_lr[rho] (R <= 32)
+      float o = 0.f, olr = 0.f;
+      for (int k = 0; k < ns; ++k) {
+        const float wk = __shfl_sync(0xffffffffu, e, k);
+        if (wk == 0.f) continue;
+        const uint32_t rk = dsmem_addr(rowb, k);
+        o = fmaf(wk, dsmem_ld(rk + (c0 + lane) * 4), o);
+        if (lane < R) olr = fmaf(wk, dsmem_ld(rk + (D + lane) * 4), olr);
       }
-      __nanosleep(32);
-    }
-  }
-  __threadfence();
-  __syncthreads();
-  const int r0 = mi * n_rows / nm, r1 = (mi + 1) * n_rows / nm;   // this CTA's rows
-  const int nr = r1 - r0;
-  // this CTA's partial stays in shared memory; the others are staged into the
-  // drained stages by cp.async, as many splits at a time as fit
-  constexpr int PF = RP * WP;                        // floats of one split's partial
-  float* Wt = Part + PF;                             // [RP][kMaxSplits] 2^(m_k - M)
-  float2* ML = reinterpret_cast<float2*>(Wt + RP * kMaxSplits);   // [RP][kMaxSplits] (m, l)
-  float* Mg = reinterpret_cast<float*>(ML + RP * kMaxSplits);     // [RP][WP] merged rows
-  float* Sp = reinterpret_cast<float*>(stages);
-  const int kchunk = max(1, min(ns, (int)((size_t)ST * C::STAGE / (nr > 0 ? nr * WP * 4 : 1))));
-  // (a) every split's (m, l) of this CTA's rows (one round of independent loads)
-  for (int i = tid; i < ns * nr; i += NTHR) {
-    const int k = i / nr, row = r0 + i % nr;
-    ML[row * kMaxSplits + k] = k == split ? make_float2(Part[row * WP + D + R], Part[row * WP + D + R + 1])
-                                          : __ldcg(reinterpret_cast<const float2*>(ws_unit + (size_t)k * PF + row * WP + D + R));
-  }
-  __syncthreads();
-  // (b) per row, one warp: M = max_k m_k, w_k = 2^(m_k - M), L = sum_k w_k l_k
-  for (int row = r0 + w; row < r1; row += NTHR / 32) {
-    const float2 ml = lane < ns ? ML[row * kMaxSplits + lane] : make_float2(-INFINITY, 0.f);
-    const float M = warp_max(ml.x);
-    const float e = (lane < ns && ml.x != -INFINITY) ? fast_exp2(ml.x - M) : 0.f;
-    const float L = warp_sum(e * ml.y);
-    if (lane < ns) Wt[row * kMaxSplits + lane] = e;
-    if (lane == 0) Mg[row * WP + D + R + 1] = L;
-  }
-  // (c) sum_k w_k (O_base,k | O_lr,k), a thread per 4 columns of a row
-  constexpr int CI = (D + R) / 4;
-  const int n_items = nr * CI;
-  float4 acc[2] = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
-  for (int kc0 = 0; kc0 < ns; kc0 += kchunk) {
-    const int kc1 = min(ns, kc0 + kchunk);
-    __syncthreads();   // the weights are in place; the previous chunk is consumed
-    for (int i = tid; i < (kc1 - kc0) * nr * (WP / 4); i += NTHR) {   // staged as [k][row][WP]
-      const int k = kc0 + i / (nr * (WP / 4)), rem = i % (nr * (WP / 4));
-      if (k != split)
-        cp_async16(smem_u32(Sp + (size_t)i * 4), ws_unit + (size_t)k * PF + (size_t)(r0 + rem / (WP / 4)) * WP + (rem % (WP / 4)) * 4);
-    }
-    cp_async_wait_all();
-    __syncthreads();
+      // out = (O + s O_lr B_v^a) / L for this lane's column
+      const int a = row / g, gi = row % g;
+      const __nv_bfloat16* bb = bv + (size_t)a * R * ldB + c0 + lane;
+      float z = 0.f;
 #pragma unroll
-    for (int j2 = 0; j2 < 2; ++j2) {
-      const int it = tid + j2 * NTHR;
-      if (it >= n_items) continue;
-      const int rl = it / CI, row = r0 + rl, c = 4 * (it % CI);
-      for (int k = kc0; k < kc1; ++k) {
-        const float wk = Wt[row * kMaxSplits + k];
-        const float4 v = *reinterpret_cast<const float4*>(
-            k == split ? Part + row * WP + c : Sp + ((size_t)(k - kc0) * nr + rl) * WP + c);
-        acc[j2].x = fmaf(wk, v.x, acc[j2].x); acc[j2].y = fmaf(wk, v.y, acc[j2].y);
-        acc[j2].z = fmaf(wk, v.z, acc[j2].z); acc[j2].w = fmaf(wk, v.w, acc[j2].w);
-      }
+      for (int rho = 0; rho < R; ++rho)
+        z = fmaf(__shfl_sync(0xffffffffu, olr, rho), __bfloat162float(bb[(size_t)rho * ldB]), z);
+      const float val = fmaf(p.s, z, o) * inv;
+      const int64_t oi = (((int64_t)seq * na_tot + agent0 + a) * p.n_q + kvh * g + gi) * D + c0 + lane;
+      if (p.out_bf16) reinterpret_cast<__nv_bfloat16*>(p.out)[oi] = __float2bfloat16_rn(val);
+      else reinterpret_cast<float*>(p.out)[oi] = val;
     }
   }
-#pragma unroll
-  for (int j2 = 0; j2 < 2; ++j2) {
-    const int it = tid + j2 * NTHR;
-    if (it < n_items) *reinterpret_cast<float4*>(Mg + (r0 + it / CI) * WP + 4 * (it % CI)) = acc[j2];
-  }
-  __syncthreads();
-  if (!s_misc[0])
-    for (int i = tid; i < nr * (D / 4); i += NTHR) {
-      const int row = r0 + i / (D / 4), c = 4 * (i % (D / 4));
-      emit(Mg + row * WP, row, c);
-    }
-  // the last merging CTA to finish resets the unit's counters and flags for
-  // the next call on this workspace
-  __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    if (atomicAdd(ctr + 1, 1) == nm - 1) {
-      for (int k = 0; k < ns; ++k) flags[k] = 0;
-      ctr[1] = 0;
-      ctr[0] = 0;
-      __threadfence();
-    }
-  }
+  cluster_sync_all();   // no CTA leaves while the others read its partial
 }
 
 // -------------------------------------------------------------------- host
@@ -952,7 +877,8 @@ size_t smem_of(int r, int rp) {
 }
 
 template <int R, int RP>
-cudaError_t launch_t(const AttnParams& p, cudaStream_t st) {
+cudaError_t launch_t(const AttnParams& pin, cudaStream_t st) {
+  AttnParams p = pin;
   using Cf = Cfg<R, RP>;
   RopeTheta rt;
   for (int i = 0; i < 64; ++i) {
@@ -976,22 +902,39 @@ cudaError_t launch_t(const AttnParams& p, cudaStream_t st) {
   auto kern = decode_cs_kernel<R, RP>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
+  if (p.n_splits > 8) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.n_splits, (p.n_agents + p.agent_group - 1) / p.agent_group, p.n_seqs * p.n_kv);
   cfg.blockDim = dim3(NTHR);
   cfg.dynamicSmemBytes = sm;
   cfg.stream = st;
-  // the set-up may overlap the preceding kernel (programmatic dependent launch;
-  // the kernel waits for it before reading any input)
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  // the splits of a unit form one cluster (they merge over distributed shared
+  // memory); the set-up may overlap the preceding kernel (programmatic
+  // dependent launch: the kernel waits for it before reading any input)
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  // as many splits as a resident cluster can hold: halve until one fits
+  for (;;) {
+    attr[0].val.clusterDim.x = (unsigned)p.n_splits;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(p.n_splits, (p.n_agents + p.agent_group - 1) / p.agent_group, p.n_seqs * p.n_kv);
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int nc = 0;
+    if (p.n_splits == 1 || (cudaOccupancyMaxActiveClusters(&nc, kern, &cfg) == cudaSuccess && nc >= 1)) break;
+    cudaGetLastError();
+    p.n_splits = p.n_splits / 2;
+  }
+  cfg.numAttrs = 2;
   e = cudaLaunchKernelEx(&cfg, kern, mk, mv, ml, mb, p, rt);
   if (e != cudaSuccess) {   // without the overlap where the runtime refuses it
     cudaGetLastError();
-    cfg.numAttrs = 0;
+    cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, kern, mk, mv, ml, mb, p, rt);
     if (e != cudaSuccess) return e;
   }
@@ -1055,11 +998,6 @@ cudaError_t launch_decode_cs(const AttnParams& pin, la_dtype out, cudaStream_t s
   p.agent_group = cs_group_size(p);
   if (p.agent_group < 1) return cudaErrorInvalidValue;
   if (p.n_splits > kMaxSplits) return cudaErrorInvalidValue;
-  // several CTAs share a unit's merge only in a launch of one wave, where
-  // every CTA the merging ones wait for is running or about to run
-  const int64_t ctas = (int64_t)p.n_splits * ((p.n_agents + p.agent_group - 1) / p.agent_group) *
-                       p.n_seqs * p.n_kv;
-  p.merge_ctas = ctas <= device_sms() ? 4 : 1;
   if (p.r == 32) return launch_t<32, 4>(p, st);
   switch (rows_padded(p, p.agent_group)) {
     case 4: return launch_t<16, 4>(p, st);
@@ -1068,23 +1006,9 @@ cudaError_t launch_decode_cs(const AttnParams& pin, la_dtype out, cudaStream_t s
   }
 }
 
-// Workspace of the cos/sin-table decode: per (agent group, unit) its splits'
-// partials [splits][rows padded][d + r + 4] fp32, then per (group, unit) an
-// arrival and a merged counter, then per (group, unit) a flag per split.
-size_t cs_partial_bytes(const AttnParams& p) {
-  const int G = cs_group_size(p);
-  if (G < 1) return 0;
-  const int ns = cs_splits(p, G);
-  if (ns == 1) return 0;
-  const int groups = (p.n_agents + G - 1) / G;
-  return (size_t)p.n_seqs * p.n_kv * groups * ns * rows_padded(p, G) * (p.d + p.r + 4) * sizeof(float);
-}
-
-size_t cs_counter_ints(const AttnParams& p) {
-  const int G = cs_group_size(p);
-  if (G < 1) return 0;
-  const int groups = (p.n_agents + G - 1) / G;
-  return (size_t)p.n_seqs * p.n_kv * groups * (2 + kMaxSplits);
-}
+// The cos/sin-table decode merges its splits inside each cluster: it needs no
+// workspace.
+size_t cs_partial_bytes(const AttnParams&) { return 0; }
+size_t cs_counter_ints(const AttnParams&) { return 0; }
 
 }  // namespace la

@@ -35,9 +35,12 @@ void* scratch_on_current_device() {
 
 extern "C" la_status lora_attn_decode_static_scratch(const la_attn_args* args, la_stream_t stream) {
   const size_t need = lora_attn_decode_workspace_bytes(args);
-  // no scratch needed: invalid arguments (reported as lora_attn_decode would)
-  // or an empty batch, which has nothing to do
-  if (need == 0) return la::decode_args_status(args);
+  // no scratch needed: invalid arguments (reported as lora_attn_decode would),
+  // an empty batch, or a decode that needs no workspace (run as it is)
+  if (need == 0) {
+    const la_status st = la::decode_args_status(args);
+    return st != LA_OK ? st : lora_attn_decode(args, nullptr, 0, stream);
+  }
   if (need > la::kStaticScratchBytes) return LA_ERR_SCRATCH_LIMIT;
   void* ptr = la::scratch_on_current_device();
   if (!ptr) return LA_ERR_CUDA;

@@ -50,7 +50,6 @@ struct AttnParams {
   const void* x_new;       // [n_seqs][hidden]
   const void* A_kv;        // [hidden][2r], or [n_agents][hidden][2r] with per-agent caches
   int64_t hidden;
-  int merge_ctas;          // cos/sin-table decode: CTAs of a unit that share its split merge
 };
 
 // Device error word of the library (address on the current device).

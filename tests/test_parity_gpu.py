@@ -256,13 +256,14 @@ def test_decode_kv_len_beyond_bound_is_reported(la):
 
 
 def test_decode_merge_wait_runs_out_and_is_reported(la):
-    """The in-launch split merge hands each split of a unit a ticket from the
-    unit's arrival counter; the last ticket merges.  A workspace whose counters
-    start at -1 (all bytes 0xFF, never zero-filled) hands out a ticket no call
-    can produce: the launch still ends, the merge bit of the device error word
-    is set, and the same context then computes a correct decode on a zeroed
-    workspace."""
-    s = W.LLAMA8B_DECODE_8K.replace(kv_len=4096, n_seqs=1, seed=29)
+    """The in-launch split merge of the r = 64 decode waits, bounded, for every
+    split of its unit to arrive on the unit's counter in the workspace.  A
+    workspace whose counters start at -1 (all bytes 0xFF, never zero-filled)
+    never reaches the split count: every CTA's wait gives up, the launch still
+    ends, the merge bit of the device error word is set, and the same context
+    then computes a correct decode on a zeroed workspace."""
+    # r = 64: the decode whose split merge counts arrivals in the workspace
+    s = W.llama8b_stack_decode(0).replace(kv_len=4096, seed=29)
     inp = W.direct_cache_inputs(s)
     dd = to_device(inp)
     out = torch.zeros(dd["q"].shape, device=DEV)

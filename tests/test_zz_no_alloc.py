@@ -53,8 +53,12 @@ def _compare(la, s, inp):
 
 @pytest.mark.gpu
 def test_static_scratch_matches_workspace_decode_bf16(la):
-    """The LLaMA-shaped 8192-token decode (tensor-core kernel, split over the keys)."""
+    """The LLaMA-shaped 8192-token decode (r = 16: the splits merge inside their
+    cluster, no scratch used) and the stack's r = 64 decode (split partials and
+    arrival counters in the scratch)."""
     s = W.LLAMA8B_DECODE_8K
+    _compare(la, s, W.direct_cache_inputs(s))
+    s = W.llama8b_stack_decode(0).replace(kv_len=4096, seed=17)
     _compare(la, s, W.direct_cache_inputs(s))
 
 
@@ -72,8 +76,8 @@ def test_static_scratch_after_a_larger_call_clears_its_counters(la):
     bytes where the first left its split partials (nonzero floats), so the
     call must clear them before it launches.  Checked against the oracle."""
     from tests.helpers import oracle_decode
-    big = W.LLAMA8B_DECODE_8K
-    small = W.LLAMA8B_DECODE_8K.replace(kv_len=1000, seed=91)
+    big = W.llama8b_stack_decode(0).replace(kv_len=8192)
+    small = W.llama8b_stack_decode(0).replace(kv_len=300, seed=91)
     outs = []
     for s in (big, small):
         inp = W.direct_cache_inputs(s)
