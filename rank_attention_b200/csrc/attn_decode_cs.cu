@@ -211,6 +211,14 @@ __global__ void __launch_bounds__(NTHR, 1)
     tma_prefetch(&tmV);
     tma_prefetch(&tmL);
     tma_prefetch(&tmB);
+  }
+  if (tid < D / 2) theta[tid] = rt.theta[tid];
+  if (tid < 2 * QP) Corr[tid] = 1.f;
+  // the barriers are initialised before any thread polls one: the shared
+  // memory still holds what the SM's previous CTA left there, and a stale
+  // barrier word may read as a completed phase
+  __syncthreads();
+  if (w == WV && lane == 0) {
     // a programmatic dependent of the preceding kernel (the step's LR append):
     // everything above overlaps its tail, every input is read after the wait
     pdl_wait();
@@ -229,8 +237,6 @@ __global__ void __launch_bounds__(NTHR, 1)
         tma_load_3d(uv_u + a * R * D * 2 + b * R * 128, &tmB, bar(B_OPS), kvh * D + 64 * b, 0, agent0 + a);
     for (int n = 0; n < n_spec; ++n) issue(n);
   }
-  if (tid < D / 2) theta[tid] = rt.theta[tid];
-  if (tid < 2 * QP) Corr[tid] = 1.f;
   pdl_wait();
   const int64_t kvl = p.kv_len[seq];
   const bool bad_len = kvl < 1 || kvl > p.max_kv_len;
