@@ -585,12 +585,9 @@ def decode_source_sha() -> str:
 
 
 def step_kernels_per_call(s) -> int:
-    """Kernels one decode step (lora_attn_decode_step) launches: one where the
-    tensor-core decode forms the new LR row itself (bf16, d = 128, r = 16 or
-    32), else a row append before the decode's kernels."""
-    if s.dtype != torch_bf16() or s.head_dim != 128:
-        return 1 + decode_kernels_per_call(s)
-    return 1 if s.r in (16, 32) else 1 + decode_kernels_per_call(s)
+    """Kernels one decode step (lora_attn_decode_step) launches: the new LR
+    row's append, then the decode's kernels."""
+    return 1 + decode_kernels_per_call(s)
 
 
 def torch_bf16():
@@ -600,10 +597,10 @@ def torch_bf16():
 
 def decode_kernels_per_call(s) -> int:
     """Kernels one lora_attn_decode call launches for this workload.  The
-    tensor-core decodes (d = 128: r in {16, 32} any agent count; r = 64)
-    merge their key splits inside the same launch: one kernel.  The other bf16
-    shapes add a split-merge kernel when the keys are split over CTAs."""
-    if s.head_dim == 128 and (s.r in (16, 32) or (s.r == 64 and s.n_agents <= 3)):
+    tensor-core decode (d = 128, r in {16, 32, 64}, agents in groups of up to
+    three a CTA) merges its key splits inside the same launch: one kernel.  The
+    other bf16 shapes add a split-merge kernel when the keys are split over CTAs."""
+    if s.head_dim == 128 and s.r in (16, 32, 64):
         return 1
     units = s.n_seqs * s.n_kv_heads
     splits = 1 if units >= 148 else min(32, 148 // units, (s.kv_len + 127) // 128)

@@ -192,10 +192,9 @@ typedef struct {
  *   lr_cache[q][kv_len[q] - 1][c] = sum_k x_new[q][k] A_kv[k][c],  c in [0, 2r)
  * (with args->lr_agent_stride > 0 every agent's own cache, from its own
  * A_kv[a]; rounding as lr_cache_append), then lora_attn_decode over
- * [0, kv_len[q]), that row included.  Where the tensor-core decode takes the
- * shape (bf16, head_dim 128, r in {16, 32}) this is ONE launch: the CTAs whose
- * keys hold position kv_len[q] - 1 form the row themselves, use it and write
- * it to the cache; otherwise a row-append kernel runs before the decode.
+ * [0, kv_len[q]), that row included: a small row-append kernel (positions
+ * read from kv_len on the device), then the decode, whose set-up overlaps the
+ * append's tail (programmatic dependent launch).
  * The new token's base K and V rows must already be in k_base / v_base.
  *
  *   A_kv    device, [hidden][2r] (shared A), or [n_agents][hidden][2r] with

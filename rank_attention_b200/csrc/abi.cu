@@ -31,7 +31,6 @@ cudaError_t launch_decode_bf16(const AttnParams& p, la_dtype out, cudaStream_t s
 bool bf16_prefill_supported(const AttnParams& p);
 cudaError_t launch_prefill_bf16(const AttnParams& p, la_dtype out, cudaStream_t st);
 bool bf16_append_supported(int64_t H, int r);
-int cs_group_size(const AttnParams& p);
 
 namespace {
 
@@ -147,9 +146,6 @@ DecodePlan plan_decode(const AttnParams& p, la_dtype io) {
   // (generic kernel), or the bf16 decode's own
   const size_t ints = d.kind == 1 ? bf16_decode_counter_ints(p) : (size_t)2 * units * d.groups;
   d.counter_bytes = (ints * sizeof(int) + 255) / 256 * 256;
-  // at least 256 bytes, so that the size query is nonzero for any valid call
-  // (the cos/sin-table decode merges inside its clusters and uses none of it)
-  if (d.partial_bytes + d.counter_bytes == 0 && units > 0) d.counter_bytes = 256;
   return d;
 }
 
@@ -364,19 +360,12 @@ la_status step_check(const la_attn_args* a, const void* A_kv, const void* x_new,
 }
 
 // A decode step after decode_prepare: the new token's LR row at kv_len[q] - 1
-// of every LR cache, then the decode.  One launch where the cos/sin-table
-// decode takes the shape (it forms and writes the row itself), else the
-// row append and the decode.
+// of every LR cache (one small kernel), then the decode, a programmatic
+// dependent of it (its set-up overlaps the row's write).
 la_status step_launch(AttnParams& p, int kind, const la_attn_args* a, const void* A_kv,
                       const void* x_new, int64_t hidden, cudaStream_t st) {
   p.err = error_word_ptr();
   if (!p.err) return LA_ERR_CUDA;
-  if (kind == 1 && a->io_dtype == LA_BF16 && cs_group_size(p) > 0) {
-    p.x_new = x_new;
-    p.A_kv = A_kv;
-    p.hidden = hidden;
-    return decode_launch(p, kind, a, st);
-  }
   const int n_lr = a->lr_agent_stride > 0 ? a->n_agents : 1;
   const cudaError_t e = launch_append_row_at_len(x_new, A_kv, hidden * 2 * a->r,
                                                  const_cast<void*>(a->lr_cache), a->lr_seq_stride,

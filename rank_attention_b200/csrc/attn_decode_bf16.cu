@@ -1796,14 +1796,7 @@ cudaError_t launch_tc(const AttnParams& p, cudaStream_t st) {
 
 }  // namespace
 
-int cs_group_size(const AttnParams& p);
-int cs_splits(const AttnParams& p, int G);
-size_t cs_partial_bytes(const AttnParams& p);
-size_t cs_counter_ints(const AttnParams& p);
-cudaError_t launch_decode_cs(const AttnParams& p, la_dtype out, cudaStream_t st);
-
 bool bf16_decode_supported(const AttnParams& p) {
-  if (cs_group_size(p) > 0) return true;
   if (tc_supported(p)) return true;
   if (p.lr_agent) return false;   // the generic kernel serves per-agent LR caches otherwise
   if (p.d != 128) return false;
@@ -1817,14 +1810,6 @@ bool bf16_decode_supported(const AttnParams& p) {
 }
 
 void bf16_decode_plan(const AttnParams& p, int* n_splits, int64_t* split_len, int* rows, int* groups) {
-  const int Gc = cs_group_size(p);
-  if (Gc > 0) {   // the cos/sin-table decode
-    *n_splits = cs_splits(p, Gc);
-    *split_len = KT;
-    *rows = Gc * p.g;
-    *groups = (p.n_agents + Gc - 1) / Gc;
-    return;
-  }
   const int G = tc_group_size(p);
   *n_splits = n_splits_for(p);
   *split_len = KT;
@@ -1833,7 +1818,6 @@ void bf16_decode_plan(const AttnParams& p, int* n_splits, int64_t* split_len, in
 }
 
 size_t bf16_decode_partial_bytes(const AttnParams& p) {
-  if (cs_group_size(p) > 0) return cs_partial_bytes(p);
   const int ns = n_splits_for(p);
   if (ns == 1) return 0;
   const int G = tc_group_size(p);
@@ -1843,12 +1827,10 @@ size_t bf16_decode_partial_bytes(const AttnParams& p) {
 
 // arrival counters (and flags) of the split merge, in ints, per workspace
 size_t bf16_decode_counter_ints(const AttnParams& p) {
-  if (cs_group_size(p) > 0) return cs_counter_ints(p);
   return (size_t)2 * p.n_seqs * p.n_kv * decode_groups(p);
 }
 
 cudaError_t launch_decode_bf16(const AttnParams& pin, la_dtype out, cudaStream_t st) {
-  if (cs_group_size(pin) > 0) return launch_decode_cs(pin, out, st);
   AttnParams p = pin;
   p.out_bf16 = out == LA_BF16;
   p.agent_group = tc_group_size(p);

@@ -29,17 +29,6 @@ __device__ __forceinline__ float2 rope_cs_exact(int64_t t, double theta) {
   return make_float2(c, s);
 }
 
-// The same angle, reduced modulo 2 pi in fp64, then the SFU (about 2^-21
-// absolute on [-pi, pi]): the accuracy of a bf16 operand built from it
-__device__ __forceinline__ float2 rope_cs_sfu(int64_t t, double theta) {
-  const double two_pi = 6.283185307179586476925286766559;
-  const double ang = (double)t * theta;
-  const float red = (float)fma(-two_pi, rint(ang * 0.15915494309189533577), ang);
-  float s, c;
-  __sincosf(red, &s, &c);
-  return make_float2(c, s);
-}
-
 // (cos, sin) of a small angle (|ang| < ~200 rad): Cody-Waite reduction with a
 // two-constant split of 2 pi, then the SFU (about 2^-21 absolute on [-pi, pi])
 __device__ __forceinline__ float2 sincos_small(float ang) {

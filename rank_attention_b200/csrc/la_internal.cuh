@@ -45,11 +45,6 @@ struct AttnParams {
   int agent_group;         // tensor-core decode: agents per CTA (grid z runs over the groups)
   int value_path;          // la_value_path: 0 fastest reordered, 1 generic reordered, 2 per tile
   int blk0;                // tensor-core prefill, split launch: the first block of rows it covers
-  // decode step in one launch: the new token's LR row x_new[q] A_kv written at
-  // row kv_len[q] - 1 (and used) by the decode itself; null x_new: no append
-  const void* x_new;       // [n_seqs][hidden]
-  const void* A_kv;        // [hidden][2r], or [n_agents][hidden][2r] with per-agent caches
-  int64_t hidden;
 };
 
 // Device error word of the library (address on the current device).

@@ -40,20 +40,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, int lim
     if (mbar_try_wait(bar, parity)) return true;
   return false;
 }
-// Wait bounded in time: gives up once `limit` SM clock cycles have passed
-// (about a second at the default; checked every 256 polls), whatever each
-// poll's own suspend time is.  clock64 is the SM's own cycle counter: cheap to
-// read and monotonic while the CTA runs.
-__device__ __forceinline__ bool mbar_wait_clk(uint32_t bar, uint32_t parity,
-                                             long long limit = 2000000000ll) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const long long t0 = clock64();
-  for (;;) {
-    for (int i = 0; i < 256; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
-    if (clock64() - t0 > limit) return false;
-  }
-}
 // Orders this thread's generic-proxy shared-memory writes before later
 // async-proxy (TMA) accesses of the same memory.
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -156,11 +142,6 @@ __device__ __forceinline__ uint32_t dsmem_addr(uint32_t local, uint32_t rank) {
 __device__ __forceinline__ float dsmem_ld(uint32_t addr) {
   float v;
   asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-  return v;
-}
-__device__ __forceinline__ float2 dsmem_ld2(uint32_t addr) {
-  float2 v;
-  asm volatile("ld.shared::cluster.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr) : "memory");
   return v;
 }
 __device__ __forceinline__ float4 dsmem_ld4(uint32_t addr) {
@@ -316,44 +297,9 @@ __device__ __forceinline__ void tmem_st32x32b_x32(uint32_t taddr, const uint32_t
                : "memory");
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-// After one tcgen05.wait::ld for several loads: the registers of the other
-// loads are named here (an empty statement, ordered after the wait), so that
-// the compiler reads none of them before the wait
-__device__ __forceinline__ void reg_after_wait16(uint32_t (&r)[16]) {
-  asm volatile(""
-               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
-               :
-               : "memory");
-}
-__device__ __forceinline__ void reg_after_wait32(uint32_t (&r)[32]) {
-  asm volatile(""
-               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
-               :
-               : "memory");
-}
 // a hint: bring the 128-byte line holding `ptr` into L2
 __device__ __forceinline__ void prefetch_l2(const void* ptr) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr));
-}
-// 16-byte copy global -> shared that bypasses L1 (cp.async), and the wait for
-// every such copy this thread has issued
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-}
-// 32 TMEM lanes x 1 column: thread t gets / puts lane t of one column
-__device__ __forceinline__ uint32_t tmem_ld32x32b_x1(uint32_t taddr) {
-  uint32_t r;
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
-  return r;
-}
-__device__ __forceinline__ void tmem_st32x32b_x1(uint32_t taddr, uint32_t v) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v) : "memory");
-}
-__device__ __forceinline__ void tmem_wait_ld_r1(uint32_t& r) {
-  asm volatile("tcgen05.wait::ld.sync.aligned;" : "+r"(r) : : "memory");
 }
 // 16 TMEM lanes x 8 columns: thread t gets lanes t/4 and t/4+8, columns 2(t%4), 2(t%4)+1
 // (the mma.sync m16n8 accumulator layout); .x2 repeats over the next 8 columns.

@@ -276,8 +276,7 @@ def lora_attn_decode(args: AttnArgs, workspace: torch.Tensor, stream=None) -> No
 def lora_attn_decode_step(args: AttnArgs, A_kv: torch.Tensor, x_new: torch.Tensor,
                           workspace: torch.Tensor, stream=None) -> None:
     """A decode step on device buffers: the new token's LR row x_new[q] A_kv at
-    kv_len[q] - 1 of the LR cache(s), then the decode (one launch where the
-    tensor-core decode takes the shape).  x_new [n_seqs, hidden] contiguous;
+    kv_len[q] - 1 of the LR cache(s), then the decode.  x_new [n_seqs, hidden] contiguous;
     A_kv [hidden, 2r], or [n_agents, hidden, 2r] with per-agent caches."""
     assert x_new.is_contiguous() and A_kv.is_contiguous()
     st = lib.lora_attn_decode_step(ctypes.byref(args), A_kv.data_ptr(), x_new.data_ptr(),
@@ -352,7 +351,7 @@ def la_device_check_word() -> tuple:
 class DecodeStep:
     """One decode step of the hot path: the new token's LR row at kv_len - 1,
     then every agent's query over the shared caches (lora_attn_decode_step:
-    one library call, one launch where the tensor-core decode takes the shape).
+    one library call: the row append, then the decode).
 
     Holds the argument struct and the zero-filled split-K workspace.  Tensors
     must stay alive while it is used.  Without x_new / A_kv it is the decode

@@ -53,9 +53,8 @@ def _compare(la, s, inp):
 
 @pytest.mark.gpu
 def test_static_scratch_matches_workspace_decode_bf16(la):
-    """The LLaMA-shaped 8192-token decode (r = 16: the splits merge inside their
-    cluster, no scratch used) and the stack's r = 64 decode (split partials and
-    arrival counters in the scratch)."""
+    """The LLaMA-shaped 8192-token decode (r = 16) and the stack's r = 64 decode,
+    both with split partials and arrival counters in the scratch."""
     s = W.LLAMA8B_DECODE_8K
     _compare(la, s, W.direct_cache_inputs(s))
     s = W.llama8b_stack_decode(0).replace(kv_len=4096, seed=17)
