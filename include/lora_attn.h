@@ -68,20 +68,25 @@ typedef enum {
 
 typedef enum { LA_F32 = 0, LA_BF16 = 1 } la_dtype;
 
-/* How the value side is computed (la_attn_args.value_path).  The three give
- * the same outputs up to rounding; 1 and 2 exist to measure the reordering
- * (the naive-reconstruction ablation of LRAgent summary App. B / explainer,
+/* How the value side is computed (la_attn_args.value_path).  All give the
+ * same outputs up to rounding; 1 to 3 exist to measure the reordering (the
+ * naive-reconstruction ablation of LRAgent summary App. B / explainer,
  * Metodologia 3):
  *   LA_VALUE_REORDERED          O = P V_base + (P LRv) s B_v^a, B_v applied once
  *                               per row; the fastest kernel for the shape.
  *   LA_VALUE_REORDERED_GENERIC  the same on the generic CUDA-core kernel.
  *   LA_VALUE_PER_TILE           naive: per key tile and agent, V^a = V_base +
- *                               s LRv B_v^a rebuilt in head dimension, then
- *                               O += P V^a; the generic CUDA-core kernel. */
+ *                               s LRv B_v^a rebuilt in head dimension (rounded
+ *                               to the io dtype), then O += P V^a.  The
+ *                               tensor-core prefill has this arm at r = 16
+ *                               (bf16, head_dim 128); the decode and other
+ *                               shapes run it on the generic kernel.
+ *   LA_VALUE_PER_TILE_GENERIC   the per-tile arm on the generic kernel. */
 typedef enum {
   LA_VALUE_REORDERED = 0,
   LA_VALUE_REORDERED_GENERIC = 1,
-  LA_VALUE_PER_TILE = 2
+  LA_VALUE_PER_TILE = 2,
+  LA_VALUE_PER_TILE_GENERIC = 3
 } la_value_path;
 
 /* Human-readable name of a status code (static string, never NULL). */

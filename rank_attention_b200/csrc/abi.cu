@@ -29,6 +29,7 @@ size_t bf16_decode_counter_ints(const AttnParams& p);
 void bf16_decode_plan(const AttnParams& p, int* n_splits, int64_t* split_len, int* rows, int* groups);
 cudaError_t launch_decode_bf16(const AttnParams& p, la_dtype out, cudaStream_t st);
 bool bf16_prefill_supported(const AttnParams& p);
+bool bf16_prefill_per_tile_supported(const AttnParams& p);
 cudaError_t launch_prefill_bf16(const AttnParams& p, la_dtype out, cudaStream_t st);
 bool bf16_append_supported(int64_t H, int r);
 
@@ -68,7 +69,7 @@ la_status check_attn(const la_attn_args* a, int decode, AttnParams* p) {
       (!stride_ok(a->lr_agent_stride, io) ||
        a->lr_agent_stride < (int64_t)(a->n_seqs > 0 ? a->n_seqs - 1 : 0) * a->lr_seq_stride + a->L_max * 2 * a->r))
     return LA_ERR_INVALID_ARG;
-  if (a->value_path < LA_VALUE_REORDERED || a->value_path > LA_VALUE_PER_TILE) return LA_ERR_INVALID_ARG;
+  if (a->value_path < LA_VALUE_REORDERED || a->value_path > LA_VALUE_PER_TILE_GENERIC) return LA_ERR_INVALID_ARG;
   const int g = a->n_q_heads / a->n_kv_heads;
   if ((int64_t)a->n_agents * g > kMaxRowsSimt) return LA_ERR_UNSUPPORTED;
   if (decode) {
@@ -456,7 +457,9 @@ extern "C" la_status lora_attn_prefill(const la_attn_args* a, la_stream_t stream
   if (s != LA_OK) return s;
   if (p.n_seqs == 0 || p.n_q_tokens == 0) return LA_OK;
   if ((int64_t)p.n_seqs * p.n_kv > 65535) return LA_ERR_UNSUPPORTED;
-  const bool tc = a->io_dtype == LA_BF16 && p.value_path == LA_VALUE_REORDERED && bf16_prefill_supported(p);
+  const bool tc = a->io_dtype == LA_BF16 &&
+                  ((p.value_path == LA_VALUE_REORDERED && bf16_prefill_supported(p)) ||
+                   (p.value_path == LA_VALUE_PER_TILE && bf16_prefill_per_tile_supported(p)));
   if (!tc && simt_smem_bytes(p) > 227 * 1024) return LA_ERR_UNSUPPORTED;
   p.err = error_word_ptr();
   if (!p.err) return LA_ERR_CUDA;

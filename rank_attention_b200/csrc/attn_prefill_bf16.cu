@@ -24,6 +24,11 @@
 // refills.  The compute warps build tile n+1
 // before the softmax of tile n, so the S MMA of tile n+1 runs during that
 // softmax and the P V MMA of tile n during the next build.
+// The per-tile value arm (VT, the ablation of the reordering) instead builds
+// V^a = V_base + s LRv B_v^a per tile (dV on the tensor cores, the sum over
+// V_base in shared memory, like K^a), keeps P in shared memory (TMEM holds dV
+// where the reordered arm keeps P and O_lr) and accumulates O += P V^a: the
+// head-dimension rebuild per tile that the reordering removes.
 // Where whole CTAs would leave SMs idle, the launch runs each block as a
 // cluster of two CTAs over the two halves of its key tiles (template KS = 2),
 // merged over distributed shared memory.  With one LR cache per agent the LR
@@ -53,12 +58,13 @@ constexpr int PKT = 128;                 // keys per tile
 constexpr int PM = 128;                  // query rows per CTA
 constexpr int PNC = 8;                   // compute warps
 constexpr int PNTHR = 32 * (PNC + 2);  // + the MMA warp + the TMA refill warp
-// TMEM columns
+// TMEM columns (the per-tile value arm: dV at 256, O at 384, P in shared memory)
 constexpr int T_DK = 0, T_S = 128, T_P = 256, T_O = 320, T_OL = 448, T_COLS = 512;
+constexpr int T_DV = 256, T_OV = 384;
 // named barriers (0 is __syncthreads)
 constexpr int PBAR_CW = 1, PBAR_PAIR = 2;  // PBAR_PAIR + sub-partition: the two warps of a row block
 
-template <int R>
+template <int R, bool VT = false>
 struct PCfg {
   // a K stage holds the K_base tile and the tile's LRk columns, a V stage the
   // V_base tile and its LRv columns: r columns of the LR rows, one TMA box
@@ -75,23 +81,26 @@ struct PCfg {
   static constexpr int OFF_V = OFF_K + 2 * STAGE;               // [NV] V stages
   static constexpr int OFF_BK = OFF_V + NV * STAGE;
   static constexpr int OFF_BV = OFF_BK + align1k(B_BYTES);
-  static constexpr int OFF_MISC = OFF_BV + align1k(B_BYTES);
+  static constexpr int OFF_P = OFF_BV + align1k(B_BYTES);       // per-tile value arm: P [128][128] bf16
+  static constexpr int OFF_MISC = OFF_P + (VT ? PM * PKT * 2 : 0);
   // misc: anchors [2][64] float2, exchange [2][8][32] float, theta [64] double,
-  // 16 mbarriers, the TMEM slot
-  static constexpr int MISC = 1024 + 2048 + 512 + 128 + 16;
+  // 18 mbarriers, the TMEM slot
+  static constexpr int MISC = 1024 + 2048 + 512 + 144 + 16;
   static constexpr size_t SMEM = 1024 + OFF_MISC + MISC;
 };
 
-template <int R, int KS>
+template <int R, int KS, bool VT>
 __global__ void __launch_bounds__(PNTHR, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV,
                       const __grid_constant__ CUtensorMap tmL,
-                      const __grid_constant__ CUtensorMap tmB, const AttnParams p,
+                      const __grid_constant__ CUtensorMap tmB,
+                      const __grid_constant__ CUtensorMap tmBv, const AttnParams p,
                       const __grid_constant__ RopeTheta rt) {
   constexpr int ksplit = KS;   // 1, or 2: the keys of a block split over a cluster of two CTAs
-  using C = PCfg<R>;
+  using C = PCfg<R, VT>;
+  constexpr int TO = VT ? T_OV : T_O;   // O^T's TMEM columns
   constexpr int D = PD;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
@@ -103,8 +112,9 @@ __global__ void __launch_bounds__(PNTHR, 1)
   float2* anc = reinterpret_cast<float2*>(misc);               // [2][64] s (cos, sin)(k0 theta_i)
   float* xch = reinterpret_cast<float*>(misc + 1024);          // [2][8][32]
   double* theta = reinterpret_cast<double*>(misc + 3072);      // [64]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(misc + 3584);   // [16]
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(misc + 3584 + 128);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(misc + 3584);   // [18]
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(misc + 3584 + 144);
+  const uint32_t p_u = sb + C::OFF_P;   // the per-tile value arm's P
   const __nv_bfloat16* bvs = reinterpret_cast<const __nv_bfloat16*>(smem + C::OFF_BV);
   __shared__ int s_fail;
 
@@ -115,6 +125,7 @@ __global__ void __launch_bounds__(PNTHR, 1)
   auto vempty = [&](int s) { return b0 + 48 + 8 * s; };
   const uint32_t qbar = b0 + 64, bvbar = b0 + 72, dkfull = b0 + 80, kaready = b0 + 88;
   const uint32_t sfull = b0 + 96, staken = b0 + 104, pfull = b0 + 112, pvdone = b0 + 120;
+  const uint32_t dvfull = b0 + 128, varready = b0 + 136;   // the per-tile value arm
 
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int gq = lane >> 2, t4 = lane & 3;
@@ -164,6 +175,8 @@ __global__ void __launch_bounds__(PNTHR, 1)
     mbar_init(staken, PNC);
     mbar_init(pfull, PNC);
     mbar_init(pvdone, 1);
+    mbar_init(dvfull, 1);
+    mbar_init(varready, PNC);
     fence_mbar_init();
     tma_prefetch(&tmQ);
     tma_prefetch(&tmB);
@@ -186,7 +199,13 @@ __global__ void __launch_bounds__(PNTHR, 1)
         if (C::NV > 1) load_v(1);
       }
     }
-    if (half == 0) {  // B_v^a: only the CTA that writes the output
+    if constexpr (VT) {  // B_v^a, the B operand of dV (every CTA)
+      tma_prefetch(&tmBv);
+      mbar_expect_tx(bvbar, (uint32_t)C::B_BYTES);
+#pragma unroll
+      for (int b = 0; b < D / 64; ++b)
+        tma_load_3d(bv_u + b * R * 128, &tmBv, bvbar, kvh * D + 64 * b, 0, agent);
+    } else if (half == 0) {  // B_v^a: only the CTA that writes the output
       const __nv_bfloat16* Bv = reinterpret_cast<const __nv_bfloat16*>(p.B_v);
       mbar_expect_tx(bvbar, (uint32_t)C::B_BYTES);
       for (int j = 0; j < R; ++j)
@@ -244,6 +263,10 @@ __global__ void __launch_bounds__(PNTHR, 1)
       const uint64_t dBk = umma_desc(bk_u, R * 128, 1024, 2);
       const uint64_t dV = umma_desc(v_u, PKT * 128, 1024, 2);
       const uint64_t dLRv = umma_desc(v_u + C::KV, PKT * C::LR_ROWB, 8 * C::LR_ROWB, C::LR_LAYOUT);
+      // the per-tile value arm: LRv as the K-major A operand of dV, B_v^a, P
+      const uint64_t dLRvA = umma_desc(v_u + C::KV, 16, 8 * C::LR_ROWB, C::LR_LAYOUT);
+      const uint64_t dBv = umma_desc(bv_u, R * 128, 1024, 2);
+      const uint64_t dPs = umma_desc(p_u, 16, 1024, 2);
       auto mma_dk = [&](int n) {  // dK = LRk B_k^a
         if (!mbar_wait(kfull(n & 1), (n >> 1) & 1)) fail = 1;
         tc_fence_after();
@@ -253,13 +276,32 @@ __global__ void __launch_bounds__(PNTHR, 1)
           umma_bf16(tmem + T_DK, umma_desc_add(lr, ks * 32), umma_desc_add(dBk, ks * 16 * 128), ID_DK, ks > 0);
         umma_commit(dkfull);
       };
-      auto mma_pv = [&](int n) {  // O += P V_base, O_lr += P LR
+      auto mma_dv = [&](int n) {  // dV = LRv B_v^a (the per-tile value arm)
+        if (!mbar_wait(vfull(n % C::NV), (n / C::NV) & 1)) fail = 1;
+        tc_fence_after();
+        const uint64_t lr = umma_desc_add(dLRvA, (n % C::NV) * C::STAGE);
+#pragma unroll
+        for (int ks = 0; ks < R / 16; ++ks)
+          umma_bf16(tmem + T_DV, umma_desc_add(lr, ks * 32), umma_desc_add(dBv, ks * 16 * 128), ID_DK, ks > 0);
+        umma_commit(dvfull);
+      };
+      auto mma_pv = [&](int n) {  // O += P V_base, O_lr += P LR (the per-tile arm: O += P V^a)
         if (!mbar_wait(pfull, n & 1)) fail = 1;
         if (!mbar_wait(vfull(n % C::NV), (n / C::NV) & 1)) fail = 1;
+        if (VT && !mbar_wait(varready, n & 1)) fail = 1;
         tc_fence_after();
         const uint64_t vd = umma_desc_add(dV, (n % C::NV) * C::STAGE);
         const uint64_t ld = umma_desc_add(dLRv, (n % C::NV) * C::STAGE);
         const uint32_t acc = n > 0 ? 1u : 0u;
+        if constexpr (VT) {
+#pragma unroll
+          for (int ks = 0; ks < PKT / 16; ++ks)
+            umma_bf16(tmem + TO, umma_desc_add(dPs, (ks >> 2) * (PM * 128) + (ks & 3) * 32),
+                      umma_desc_add(vd, ks * 16 * 128), ID_PV, ks > 0 ? 1u : acc);
+          umma_commit(pvdone);
+          umma_commit(vempty(n % C::NV));
+          return;
+        }
 #pragma unroll
         for (int ks = 0; ks < PKT / 16; ++ks)
           umma_bf16_ts(tmem + T_O, tmem + T_P + ks * 8, umma_desc_add(vd, ks * 16 * 128), ID_PV,
@@ -272,6 +314,7 @@ __global__ void __launch_bounds__(PNTHR, 1)
         umma_commit(vempty(n % C::NV));
       };
       if (!mbar_wait(qbar, 0)) fail = 1;
+      if (VT && !mbar_wait(bvbar, 0)) fail = 1;
       mma_dk(0);
       for (int n = 0; n < NT; ++n) {
         if (!mbar_wait(kaready, n & 1)) fail = 1;
@@ -286,6 +329,7 @@ __global__ void __launch_bounds__(PNTHR, 1)
         umma_commit(kempty(n & 1));
         if (n + 1 < NT) mma_dk(n + 1);
         if (n > 0) mma_pv(n - 1);
+        if constexpr (VT) mma_dv(n);   // dV(n-1) has been read: P V(n-1) waited for V^a(n-1)
       }
       mma_pv(NT - 1);
       // loads in flight when the loop ends are all consumed: every issued tile is used
@@ -413,7 +457,7 @@ __global__ void __launch_bounds__(PNTHR, 1)
         if (n > 0 && __any_sync(0xffffffffu, m_ref != -INFINITY)) {
           if (!mbar_wait(pvdone, (n - 1) & 1)) fail = 1;  // O holds every tile before this one
           tc_fence_after();
-          const uint32_t to = tmem + T_O + 64 * ch + ((uint32_t)(32 * sp) << 16);
+          const uint32_t to = tmem + TO + 64 * ch + ((uint32_t)(32 * sp) << 16);
 #pragma unroll 1
           for (int h = 0; h < 4; ++h) {
             uint32_t ov[16];
@@ -423,7 +467,7 @@ __global__ void __launch_bounds__(PNTHR, 1)
             for (int c = 0; c < 16; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * corr);
             tmem_st32x32b_x16(to + 16 * h, ov);
           }
-          if (ch == 0) {
+          if (!VT && ch == 0) {
             const uint32_t tol = tmem + T_OL + ((uint32_t)(32 * sp) << 16);
 #pragma unroll 1
             for (int h = 0; h < R / 16; ++h) {
@@ -459,11 +503,49 @@ __global__ void __launch_bounds__(PNTHR, 1)
       lsum += ls;
       if (n > 0 && !mbar_wait(pvdone, (n - 1) & 1)) fail = 1;  // the P V MMA of tile n-1 is done
       tc_fence_after();
-      tmem_st32x32b_x32(tmem + T_P + 32 * ch + ((uint32_t)(32 * sp) << 16), pk);
-      tmem_wait_st();
+      if constexpr (VT) {   // P into shared memory: row `row`, keys 64 ch .. +63 (one 128-byte-swizzled box row)
+        const uint32_t prow = p_u + (uint32_t)ch * (PM * 128) + (uint32_t)row * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c)
+          sts128(prow + (uint32_t)((c ^ (row & 7)) << 4), pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        fence_proxy_async_smem();
+      } else {
+        tmem_st32x32b_x32(tmem + T_P + 32 * ch + ((uint32_t)(32 * sp) << 16), pk);
+        tmem_wait_st();
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(pfull);
+    };
+
+    // the per-tile value arm: V^a = V_base + s dV over V_base in shared memory;
+    // this thread: key 32 sp + lane, the 64 columns of box ch
+    auto vbuild = [&](int n) {
+      if (!mbar_wait(dvfull, n & 1)) fail = 1;
+      tc_fence_after();
+      const int key = 32 * sp + lane;
+      uint32_t dv[2][32];
+      const uint32_t td = tmem + T_DV + 64 * ch + ((uint32_t)(32 * sp) << 16);
+      tmem_ld32x32b_x32(dv[0], td);
+      tmem_ld32x32b_x32(dv[1], td + 32);
+      tmem_wait_ld_r32(dv[0]);
+      tmem_wait_ld_r32(dv[1]);
+      const uint32_t vrow = v_u + (uint32_t)(n % C::NV) * C::STAGE + (uint32_t)ch * (PKT * 128) + (uint32_t)key * 128;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {   // 8 columns a 16-byte chunk
+        const uint32_t a = vrow + (uint32_t)((c ^ (key & 7)) << 4);
+        const uint4 v = lds128(a);
+        const uint32_t* d8 = dv[c >> 2] + 8 * (c & 3);
+        const float2 b0 = unpack_bf16(v.x), b1 = unpack_bf16(v.y), b2 = unpack_bf16(v.z), b3 = unpack_bf16(v.w);
+        sts128(a, pack_bf16(fmaf(p.s, __uint_as_float(d8[0]), b0.x), fmaf(p.s, __uint_as_float(d8[1]), b0.y)),
+               pack_bf16(fmaf(p.s, __uint_as_float(d8[2]), b1.x), fmaf(p.s, __uint_as_float(d8[3]), b1.y)),
+               pack_bf16(fmaf(p.s, __uint_as_float(d8[4]), b2.x), fmaf(p.s, __uint_as_float(d8[5]), b2.y)),
+               pack_bf16(fmaf(p.s, __uint_as_float(d8[6]), b3.x), fmaf(p.s, __uint_as_float(d8[7]), b3.y)));
+      }
+      fence_proxy_async_smem();   // the P V MMA reads V^a through the async proxy
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(varready);
     };
 
     if (work) {
@@ -486,6 +568,7 @@ __global__ void __launch_bounds__(PNTHR, 1)
       bar_sync(PBAR_CW, 32 * PNC);  // anchors of tile i+1 are in place
       if (i + 1 < NT) build(i + 1);
       softmax(i);
+      if constexpr (VT) vbuild(i);
       if (tid < D / 2 && i + 2 < NT) {
         const float2 cs = rope_cs_exact((int64_t)(nb + i + 2) * PKT, theta[tid]);
         anc[(i & 1) * 64 + tid] = make_float2(cs.x * p.s, cs.y * p.s);
@@ -507,7 +590,7 @@ __global__ void __launch_bounds__(PNTHR, 1)
 #pragma unroll 1
           for (int h = 0; h < 4; ++h) {
             uint32_t ov[16];
-            tmem_ld32x32b_x16(ov, tmem + T_O + 64 * ch + 16 * h + ((uint32_t)(32 * sp) << 16));
+            tmem_ld32x32b_x16(ov, tmem + TO + 64 * ch + 16 * h + ((uint32_t)(32 * sp) << 16));
             tmem_wait_ld_r16(ov);
 #pragma unroll
             for (int c = 0; c < 16; c += 4)
@@ -516,7 +599,7 @@ __global__ void __launch_bounds__(PNTHR, 1)
           }
           if (ch == 0) {
 #pragma unroll 1
-            for (int h = 0; h < R / 16; ++h) {
+            for (int h = 0; h < (VT ? 0 : R / 16); ++h) {
               uint32_t t16[16];
               tmem_ld32x32b_x16(t16, tmem + T_OL + 16 * h + ((uint32_t)(32 * sp) << 16));
               tmem_wait_ld_r16(t16);
@@ -535,6 +618,7 @@ __global__ void __launch_bounds__(PNTHR, 1)
     }
     if (half == 0) {
     // ---- epilogue: out = (O + s O_lr B_v^a) / l for this warp's 64 columns
+    // (the per-tile value arm: out = O / l)
     if (!mbar_wait(pvdone, (NT - 1) & 1)) fail = 1;
     if (!mbar_wait(bvbar, 0)) fail = 1;
     tc_fence_after();
@@ -542,9 +626,9 @@ __global__ void __launch_bounds__(PNTHR, 1)
     lx[w * 32 + lane] = lsum;
     bar_sync(PBAR_PAIR + sp, 64);
     float l = lsum + lx[(w ^ 4) * 32 + lane];
-    uint32_t olr[R];   // P LRv, this thread's row
+    uint32_t olr[R];   // P LRv, this thread's row (the reordered arm)
 #pragma unroll
-    for (int h = 0; h < R / 16; ++h) {
+    for (int h = 0; h < (VT ? 0 : R / 16); ++h) {
       uint32_t t16[16];
       tmem_ld32x32b_x16(t16, tmem + T_OL + 16 * h + ((uint32_t)(32 * sp) << 16));
       tmem_wait_ld_r16(t16);
@@ -566,7 +650,7 @@ __global__ void __launch_bounds__(PNTHR, 1)
         a1 = m1 == -INFINITY ? 0.f : fast_exp2(m1 - M);
         l = a0 * l + a1 * l1;
 #pragma unroll
-        for (int j = 0; j < R; j += 4) {
+        for (int j = 0; j < (VT ? 0 : R); j += 4) {
           const float4 r4 = dsmem_ld4(dsmem_addr(xl + (uint32_t)((j / 4) * PM + row) * 16, 1));
           olr[j] = __float_as_uint(fmaf(a0, __uint_as_float(olr[j]), a1 * r4.x));
           olr[j + 1] = __float_as_uint(fmaf(a0, __uint_as_float(olr[j + 1]), a1 * r4.y));
@@ -581,7 +665,7 @@ __global__ void __launch_bounds__(PNTHR, 1)
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       uint32_t ov[32];
-      tmem_ld32x32b_x32(ov, tmem + T_O + 64 * ch + 32 * h + ((uint32_t)(32 * sp) << 16));
+      tmem_ld32x32b_x32(ov, tmem + TO + 64 * ch + 32 * h + ((uint32_t)(32 * sp) << 16));
       tmem_wait_ld_r32(ov);
       if constexpr (KS > 1) {
         if (merge) {
@@ -600,7 +684,7 @@ __global__ void __launch_bounds__(PNTHR, 1)
 #pragma unroll
       for (int c = 0; c < 32; ++c) z[c] = 0.f;
 #pragma unroll
-      for (int j = 0; j < R; ++j) {
+      for (int j = 0; j < (VT ? 0 : R); ++j) {   // the per-tile arm has V^a in O already
         const float o = __uint_as_float(olr[j]);
         const __nv_bfloat16* brow = bvs + j * D + 64 * ch + 32 * h;
 #pragma unroll
@@ -644,7 +728,7 @@ __global__ void __launch_bounds__(PNTHR, 1)
 
 // ------------------------------------------------------------------ host
 bool prefill_maps(const AttnParams& p, CUtensorMap* mq, CUtensorMap* mk, CUtensorMap* mv,
-                  CUtensorMap* ml, CUtensorMap* mb) {
+                  CUtensorMap* ml, CUtensorMap* mb, CUtensorMap* mbv) {
   auto enc = encode_fn();
   if (!enc) return false;
   const int D = PD, R = p.r, g = p.g;
@@ -689,6 +773,11 @@ bool prefill_maps(const AttnParams& p, CUtensorMap* mq, CUtensorMap* mk, CUtenso
           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return false;
+  // B_v the same way (the per-tile value arm's dV operand)
+  if (enc(mbv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(p.B_v), bd, bs, bb, one,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
   return true;
 }
 
@@ -701,9 +790,9 @@ bool prefill_maps(const AttnParams& p, CUtensorMap* mq, CUtensorMap* mk, CUtenso
 // a last wave that is mostly empty (768 CTAs on 148 SMs: 720 whole in 5 waves,
 // the last two blocks' 48 as 96 halves in one half-length wave, instead of
 // 6 waves).  Returns nA in [0, nblk].
-template <int R>
+template <int R, bool VT>
 int prefill_whole_blocks(const AttnParams& p, int nblk) {
-  using C = PCfg<R>;
+  using C = PCfg<R, VT>;
   const int64_t tiles = (p.q_pos0 + p.n_q_tokens + PKT - 1) / PKT;
   if (tiles < 4) return nblk;
   int dev = 0, sms = 0;
@@ -712,8 +801,8 @@ int prefill_whole_blocks(const AttnParams& p, int nblk) {
     cudaGetLastError();
     return nblk;
   }
-  static int pairs[64] = {};   // resident CTA pairs per device (0: not queried yet)
-  int& np = pairs[dev & 63];
+  static int pairs[2][64] = {};   // resident CTA pairs per device (0: not queried yet)
+  int& np = pairs[VT ? 1 : 0][dev & 63];
   if (np == 0) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * (unsigned)sms, 1, 1);
@@ -727,9 +816,9 @@ int prefill_whole_blocks(const AttnParams& p, int nblk) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaFuncSetAttribute(prefill_tc_kernel<R, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(prefill_tc_kernel<R, 2, VT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)C::SMEM) != cudaSuccess ||
-        cudaOccupancyMaxActiveClusters(&n, prefill_tc_kernel<R, 2>, &cfg) != cudaSuccess || n < 1) {
+        cudaOccupancyMaxActiveClusters(&n, prefill_tc_kernel<R, 2, VT>, &cfg) != cudaSuccess || n < 1) {
       cudaGetLastError();
       n = -1;
     }
@@ -749,24 +838,24 @@ int prefill_whole_blocks(const AttnParams& p, int nblk) {
   return best;
 }
 
-template <int R>
+template <int R, bool VT>
 cudaError_t launch_prefill_tc(const AttnParams& p, cudaStream_t st) {
-  using C = PCfg<R>;
+  using C = PCfg<R, VT>;
   RopeTheta rt;
   for (int i = 0; i < 64; ++i) {
     rt.theta[i] = std::pow(p.rope_base, -2.0 * i / PD);
     rt.thetaf[i] = (float)rt.theta[i];
   }
-  CUtensorMap mq, mk, mv, ml, mb;
-  if (!prefill_maps(p, &mq, &mk, &mv, &ml, &mb)) return cudaErrorInvalidValue;
+  CUtensorMap mq, mk, mv, ml, mb, mbv;
+  if (!prefill_maps(p, &mq, &mk, &mv, &ml, &mb, &mbv)) return cudaErrorInvalidValue;
   const int QB = PM / p.g;
   const int nblk = (p.n_q_tokens + QB - 1) / QB;
-  const int nA = prefill_whole_blocks<R>(p, nblk);
+  const int nA = prefill_whole_blocks<R, VT>(p, nblk);
   // blocks [0, nA) as whole CTAs, blocks [nA, nblk) as key halves on CTA pairs
   for (int ks = 1; ks <= 2; ++ks) {
     const int nb = ks == 1 ? nA : nblk - nA;
     if (nb == 0) continue;
-    auto kern = ks > 1 ? prefill_tc_kernel<R, 2> : prefill_tc_kernel<R, 1>;
+    auto kern = ks > 1 ? prefill_tc_kernel<R, 2, VT> : prefill_tc_kernel<R, 1, VT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
     if (e != cudaSuccess) return e;
     AttnParams pk = p;
@@ -783,7 +872,7 @@ cudaError_t launch_prefill_tc(const AttnParams& p, cudaStream_t st) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = ks > 1 ? 1 : 0;
-    e = cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, ml, mb, pk, rt);
+    e = cudaLaunchKernelEx(&cfg, kern, mq, mk, mv, ml, mb, mbv, pk, rt);
     if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
@@ -800,13 +889,23 @@ bool bf16_prefill_supported(const AttnParams& p) {
   return PCfg<16>::SMEM <= 227 * 1024 && PCfg<32>::SMEM <= 227 * 1024 && PCfg<64>::SMEM <= 227 * 1024;
 }
 
+// The per-tile value arm (V^a rebuilt per tile): r = 16, where its P buffer
+// fits beside the stages
+bool bf16_prefill_per_tile_supported(const AttnParams& p) {
+  return bf16_prefill_supported(p) && p.r == 16 && PCfg<16, true>::SMEM <= 227 * 1024;
+}
+
 cudaError_t launch_prefill_bf16(const AttnParams& pin, la_dtype out, cudaStream_t st) {
   AttnParams p = pin;
   p.out_bf16 = out == LA_BF16;
+  if (p.value_path == LA_VALUE_PER_TILE) {
+    if (!bf16_prefill_per_tile_supported(p)) return cudaErrorInvalidValue;
+    return launch_prefill_tc<16, true>(p, st);
+  }
   switch (p.r) {
-    case 16: return launch_prefill_tc<16>(p, st);
-    case 32: return launch_prefill_tc<32>(p, st);
-    default: return launch_prefill_tc<64>(p, st);
+    case 16: return launch_prefill_tc<16, false>(p, st);
+    case 32: return launch_prefill_tc<32, false>(p, st);
+    default: return launch_prefill_tc<64, false>(p, st);
   }
 }
 

@@ -379,7 +379,8 @@ cudaError_t launch_io(const AttnParams& p, la_dtype io, la_dtype out, cudaStream
 }
 
 cudaError_t launch_attn_simt(const AttnParams& p, la_dtype io, la_dtype out, cudaStream_t st) {
-  return p.value_path == LA_VALUE_PER_TILE ? launch_io<true>(p, io, out, st)
+  const bool per_tile = p.value_path == LA_VALUE_PER_TILE || p.value_path == LA_VALUE_PER_TILE_GENERIC;
+  return per_tile ? launch_io<true>(p, io, out, st)
                                            : launch_io<false>(p, io, out, st);
 }
 

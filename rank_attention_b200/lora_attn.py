@@ -22,7 +22,7 @@ LA_OK, LA_ERR_INVALID_ARG, LA_ERR_UNSUPPORTED, LA_ERR_CAPACITY = 0, 1, 2, 3
 LA_ERR_WORKSPACE, LA_ERR_CUDA, LA_ERR_DEVICE_CHECK, LA_ERR_SCRATCH_LIMIT = 4, 5, 6, 7
 LA_STATIC_SCRATCH_BYTES = 4 << 20
 LA_F32, LA_BF16 = 0, 1
-LA_VALUE_REORDERED, LA_VALUE_REORDERED_GENERIC, LA_VALUE_PER_TILE = 0, 1, 2
+LA_VALUE_REORDERED, LA_VALUE_REORDERED_GENERIC, LA_VALUE_PER_TILE, LA_VALUE_PER_TILE_GENERIC = 0, 1, 2, 3
 LA_DEV_KV_LEN, LA_DEV_PIPE_WAIT, LA_DEV_MERGE_WAIT = 1, 2, 4
 
 EXPORTED = ("la_status_string", "lr_cache_append", "lora_attn_prefill", "lora_attn_decode",

@@ -120,7 +120,7 @@ BAD_ATTN = [
     (dict(lr_agent_stride=-4096), la.LA_ERR_INVALID_ARG),
     (dict(lr_agent_stride=4097), la.LA_ERR_INVALID_ARG),   # not a multiple of 16 bytes
     (dict(lr_agent_stride=2048), la.LA_ERR_INVALID_ARG),   # overlaps the next agent's cache
-    (dict(value_path=3), la.LA_ERR_INVALID_ARG),
+    (dict(value_path=4), la.LA_ERR_INVALID_ARG),
     (dict(value_path=-1), la.LA_ERR_INVALID_ARG),
 ]
 

@@ -837,11 +837,14 @@ def _run_path(la, s, dd, value_path):
     W.LLAMA8B_PREFILL_16K.replace(kv_len=300, n_q_tokens=45, seed=82),
     W.LLAMA8B_DECODE_8K.replace(kv_len=500, seed=83, lr_per_agent=True),
     W.TINY_FP32.replace(kv_len=150, seed=84),
+    W.LLAMA8B_PREFILL_16K.replace(kv_len=2000, n_q_tokens=300, seed=85),
 ])
-@pytest.mark.parametrize("value_path", [1, 2])
+@pytest.mark.parametrize("value_path", [1, 2, 3])
 def test_value_paths_match_the_oracle(la, shape, value_path):
-    """The generic kernel with the reordered value side (1) and with V^a rebuilt
-    per tile (2): both equal the oracle (which materialises V^a)."""
+    """The reordered value side on the generic kernel (1) and V^a rebuilt per
+    tile (2: on the tensor-core prefill for the bf16 r = 16 prefills, several
+    query blocks, key tiles and a ragged tail in the larger one; 3: on the
+    generic kernel) all equal the oracle, which materialises V^a."""
     inp = W.direct_cache_inputs(shape)
     got = _run_path(la, shape, to_device(inp), value_path)
     ref = oracle.lora_attention(inp["k_base"], inp["v_base"], inp["lr"], inp["B_k"], inp["B_v"],
