@@ -52,6 +52,16 @@ __device__ __forceinline__ uint32_t add_to_f16x2(uint32_t base_bf16x2, float2 d)
   __half2 h = __floats2half2_rn(b.x + d.x, b.y + d.y);
   return *reinterpret_cast<uint32_t*>(&h);
 }
+// a bf16 pair as a packed fp32 pair (exact), and a packed fp32 pair rounded
+// once to an fp16 pair
+__device__ __forceinline__ uint64_t bf16x2_f2(uint32_t v) {
+  return f2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
+}
+__device__ __forceinline__ uint32_t f2_f16x2(uint64_t v) {
+  const float2 f = f2_unpack(v);
+  __half2 h = __floats2half2_rn(f.x, f.y);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
 
 constexpr int PD = 128;                  // head_dim
 constexpr int PKT = 128;                 // keys per tile
@@ -389,7 +399,7 @@ __global__ void __launch_bounds__(PNTHR, 1)
         for (int q = 0; q < 2; ++q) {
           const int i0 = 16 * grp + 8 * q + 2 * t4;
           const float2 a0 = an[i0], a1 = an[i0 + 1];
-          const uint64_t ac = f2(a0.x, a1.x), as = f2(a0.y, a1.y);
+          const uint64_t ac = f2(a0.x, a1.x), as = f2(a0.y, a1.y), nas = f2(-a0.y, -a1.y);
           const uint32_t cx = (uint32_t)(((2 * grp + q) ^ gq) << 4);
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
@@ -398,11 +408,12 @@ __global__ void __launch_bounds__(PNTHR, 1)
             const uint64_t c = RC[grp][hh][q], sn = RS[grp][hh][q];
             const uint64_t y1 = sub_f2(mul_f2(x1, c), mul_f2(x2, sn));   // R(j) dK
             const uint64_t y2 = fma_f2(x2, c, mul_f2(x1, sn));
-            const float2 z1 = f2_unpack(sub_f2(mul_f2(ac, y1), mul_f2(as, y2)));   // s R(k0) y
-            const float2 z2 = f2_unpack(fma_f2(ac, y2, mul_f2(as, y1)));
+            // K_base + s R(k0) y, the base added inside the rotation's FMAs
             const uint32_t o1 = rowb + hh * 1024 + cx, o2 = o1 + PKT * 128;
-            sts32(o1, add_to_f16x2(lds32(o1), z1));
-            sts32(o2, add_to_f16x2(lds32(o2), z2));
+            const uint64_t z1 = fma_f2(ac, y1, fma_f2(nas, y2, bf16x2_f2(lds32(o1))));
+            const uint64_t z2 = fma_f2(ac, y2, fma_f2(as, y1, bf16x2_f2(lds32(o2))));
+            sts32(o1, f2_f16x2(z1));
+            sts32(o2, f2_f16x2(z2));
           }
         }
       }

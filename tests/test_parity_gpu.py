@@ -358,10 +358,10 @@ def test_decode_step_from_host_equals_device_step(la, kv_lens, per_agent, packed
 @pytest.mark.parametrize("r,n_agents,per_agent", [(16, 3, False), (32, 5, False), (16, 3, True),
                                                   (64, 4, False)])
 def test_decode_step_equals_append_then_decode(la, r, n_agents, per_agent):
-    """The one-launch step (the decode forms the new token's LR row itself; r =
-    16, 32) and its two-launch form (r = 64: a row-append kernel, then the
-    decode) against lr_cache_append followed by lora_attn_decode: the rows
-    agree within one bf16 ulp, the outputs within the parity bar."""
+    """The step (a row-append kernel at the device's kv_len, then the decode)
+    against lr_cache_append at host positions followed by lora_attn_decode:
+    the rows agree within one bf16 ulp (different summation orders), the
+    outputs within the parity bar."""
     kv_lens = (1000, 777)
     s = W.LLAMA8B_DECODE_8K.replace(kv_len=1000, n_seqs=2, r=r, alpha=2.0 * r, n_agents=n_agents,
                                     seed=48 + r, lr_per_agent=per_agent)
