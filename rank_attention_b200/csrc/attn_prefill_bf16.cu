@@ -389,12 +389,19 @@ __global__ void __launch_bounds__(PNTHR, 1)
       // this lane's pair of K elements in a 128-byte-swizzled row: key kb + gq
       // (+8), 16-byte chunk (2 grp + q) ^ gq, word t4; columns + d/2 are one box on
       const uint32_t rowb = kst + (uint32_t)(kb + gq) * 128 + 4 * t4;
+      // every group's delta columns requested before one wait: [grp][0..7] the
+      // columns i, [grp][8..15] the columns i + d/2
+      uint32_t xx[4][16];
 #pragma unroll
       for (int grp = 0; grp < 4; ++grp) {
-        uint32_t xl[8], xh[8];
-        tmem_ld16x256_x2(xl, tl + 16 * grp);
-        tmem_ld16x256_x2(xh, tl + 16 * grp + D / 2);
-        tmem_wait_ld_regs(xl, xh);
+        tmem_ld16x256_x2(*reinterpret_cast<uint32_t(*)[8]>(&xx[grp][0]), tl + 16 * grp);
+        tmem_ld16x256_x2(*reinterpret_cast<uint32_t(*)[8]>(&xx[grp][8]), tl + 16 * grp + D / 2);
+      }
+      tmem_wait_ld_all(xx);
+#pragma unroll
+      for (int grp = 0; grp < 4; ++grp) {
+        const uint32_t* xl = xx[grp];
+        const uint32_t* xh = xx[grp] + 8;
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
           const int i0 = 16 * grp + 8 * q + 2 * t4;
