@@ -8,6 +8,7 @@
 // This generic kernel accumulates in fp32 and serves fp32 inputs and every
 // rank; the bf16 tensor-core kernel covers the large bf16 chunks.
 #include "la_internal.cuh"
+#include "ptx.cuh"
 
 namespace la {
 namespace {
@@ -84,14 +85,16 @@ cudaError_t launch_r(const void* X, int64_t ldx, int64_t n, int64_t H, const voi
 
 // The one new row of a decode step for every sequence q, at row kv_len[q] - 1
 // of every LR cache l (one shared, or one per agent with its own A):
-// lr[l][q][kv_len[q] - 1] = x[q] A[l].  One CTA per (q, l) streams A[l] in
-// 16-byte vectors, every load of a pass issued before the first is used (the
-// row is a few hundred kilobytes of A against one SM's memory pipe): a thread
-// keeps one vector column of A and every RP-th row; lanes of one column meet by
-// shuffles, warps in shared memory.  A kv_len[q] outside [1, max_kv_len] is
+// lr[l][q][kv_len[q] - 1] = x[q] A[l].  A cluster of RA_CL CTAs per (q, l)
+// splits the hidden rows (one SM alone cannot keep enough of A in flight);
+// in a CTA a thread keeps one 16-byte column vector of A and every RP-th row,
+// all loads of a pass issued before the first is used; lanes of one column
+// meet by shuffles, warps in shared memory, the CTAs over distributed shared
+// memory, where rank 0 writes the row.  A kv_len[q] outside [1, max_kv_len] is
 // reported, nothing written.
-constexpr int RA_NT = 512;   // threads of the row append
-constexpr int RA_U = 16;     // vectors in flight per thread
+constexpr int RA_NT = 256;   // threads of a row-append CTA
+constexpr int RA_U = 8;      // vectors in flight per thread
+constexpr int RA_CL = 8;     // CTAs of a cluster (hidden split)
 
 template <typename T>
 __global__ void __launch_bounds__(RA_NT) append_row_at_len_kernel(
@@ -103,35 +106,36 @@ __global__ void __launch_bounds__(RA_NT) append_row_at_len_kernel(
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   constexpr int VE = 16 / (int)sizeof(T);   // elements of a 16-byte vector
   __shared__ float red[RA_NT / 32][128];
-  const int q = blockIdx.x, l = blockIdx.y;
+  __shared__ float part[128];               // this CTA's sums, read by rank 0
+  const int rank = blockIdx.x, q = blockIdx.y, l = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int64_t len = kv_len[q];
-  if (len < 1 || len > max_kv_len) {
-    if (tid == 0) atomicOr(err, 1);
-    return;
-  }
+  const bool bad = len < 1 || len > max_kv_len;   // uniform over the cluster
   const int VR = C / VE;            // vectors of an A row (divides 32)
   const int RP = RA_NT / VR;        // rows of one pass over the CTA
   const int cv = tid % VR;
-  const T* xq = x + (int64_t)q * H;
-  const uint4* Av = reinterpret_cast<const uint4*>(A + (int64_t)l * a_stride);
+  const int64_t hb = rank * H / RA_CL, he = (rank + 1) * H / RA_CL;
   float acc[VE];
 #pragma unroll
   for (int e = 0; e < VE; ++e) acc[e] = 0.f;
-  for (int64_t h0 = tid / VR; h0 < H; h0 += (int64_t)RP * RA_U) {
-    uint4 av[RA_U];
-    float xv[RA_U];
+  if (!bad) {
+    const T* xq = x + (int64_t)q * H;
+    const uint4* Av = reinterpret_cast<const uint4*>(A + (int64_t)l * a_stride);
+    for (int64_t h0 = hb + tid / VR; h0 < he; h0 += (int64_t)RP * RA_U) {
+      uint4 av[RA_U];
+      float xv[RA_U];
 #pragma unroll
-    for (int u = 0; u < RA_U; ++u) {
-      const int64_t h = h0 + (int64_t)u * RP;
-      av[u] = h < H ? __ldg(Av + h * VR + cv) : make_uint4(0, 0, 0, 0);
-      xv[u] = h < H ? to_f32(xq[h]) : 0.f;
-    }
+      for (int u = 0; u < RA_U; ++u) {
+        const int64_t h = h0 + (int64_t)u * RP;
+        av[u] = h < he ? __ldg(Av + h * VR + cv) : make_uint4(0, 0, 0, 0);
+        xv[u] = h < he ? to_f32(xq[h]) : 0.f;
+      }
 #pragma unroll
-    for (int u = 0; u < RA_U; ++u) {
-      const T* e8 = reinterpret_cast<const T*>(&av[u]);
+      for (int u = 0; u < RA_U; ++u) {
+        const T* e8 = reinterpret_cast<const T*>(&av[u]);
 #pragma unroll
-      for (int e = 0; e < VE; ++e) acc[e] = fmaf(xv[u], to_f32(e8[e]), acc[e]);
+        for (int e = 0; e < VE; ++e) acc[e] = fmaf(xv[u], to_f32(e8[e]), acc[e]);
+      }
     }
   }
   // lanes lane, lane ^ VR, ... hold the same column vector
@@ -146,8 +150,18 @@ __global__ void __launch_bounds__(RA_NT) append_row_at_len_kernel(
     float v = 0.f;
 #pragma unroll
     for (int ww = 0; ww < RA_NT / 32; ++ww) v += red[ww][tid];
+    part[tid] = v;
+  }
+  ptx::cluster_sync_all();   // every CTA's sums are in place
+  if (rank == 0 && tid < C && !bad) {
+    float v = 0.f;
+    const uint32_t pa = ptx::smem_u32(part + tid);
+#pragma unroll
+    for (int k = 0; k < RA_CL; ++k) v += ptx::dsmem_ld(ptx::dsmem_addr(pa, k));
     lr[(int64_t)l * lr_agent + (int64_t)q * lr_seq + (len - 1) * C + tid] = from_f32<T>(v);
   }
+  if (rank == 0 && tid == 0 && bad) atomicOr(err, 1);
+  ptx::cluster_sync_all();   // no CTA leaves while rank 0 reads its sums
 }
 
 }  // namespace
@@ -159,15 +173,28 @@ cudaError_t launch_append_row_at_len(const void* x, const void* A, int64_t a_str
   const int ve = dt == LA_F32 ? 4 : 8;
   if (2 * r > 128 || (2 * r) % ve != 0 || 32 % ((2 * r) / ve) != 0 || n_seqs < 1 || n_lr < 1)
     return cudaErrorInvalidValue;
-  dim3 grid(n_seqs, n_lr);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(RA_CL, (unsigned)n_seqs, (unsigned)n_lr);
+  cfg.blockDim = dim3(RA_NT);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = RA_CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e;
   if (dt == LA_F32)
-    append_row_at_len_kernel<float><<<grid, RA_NT, 0, st>>>(
-        static_cast<const float*>(x), static_cast<const float*>(A), a_stride, static_cast<float*>(lr),
-        lr_seq, lr_agent, kv_len, max_kv_len, H, 2 * r, err);
+    e = cudaLaunchKernelEx(&cfg, append_row_at_len_kernel<float>, static_cast<const float*>(x),
+                           static_cast<const float*>(A), a_stride, static_cast<float*>(lr), lr_seq,
+                           lr_agent, kv_len, max_kv_len, H, 2 * r, err);
   else
-    append_row_at_len_kernel<__nv_bfloat16><<<grid, RA_NT, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(A), a_stride,
-        static_cast<__nv_bfloat16*>(lr), lr_seq, lr_agent, kv_len, max_kv_len, H, 2 * r, err);
+    e = cudaLaunchKernelEx(&cfg, append_row_at_len_kernel<__nv_bfloat16>,
+                           static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(A),
+                           a_stride, static_cast<__nv_bfloat16*>(lr), lr_seq, lr_agent, kv_len,
+                           max_kv_len, H, 2 * r, err);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
