@@ -85,7 +85,7 @@ cudaError_t launch_r(const void* X, int64_t ldx, int64_t n, int64_t H, const voi
 
 // The one new row of a decode step for every sequence q, at row kv_len[q] - 1
 // of every LR cache l (one shared, or one per agent with its own A):
-// lr[l][q][kv_len[q] - 1] = x[q] A[l].  A cluster of RA_CL CTAs per (q, l)
+// lr[l][q][kv_len[q] - 1] = x[q] A[l].  A cluster of 16 (else 8) CTAs per (q, l)
 // splits the hidden rows (one SM alone cannot keep enough of A in flight);
 // in a CTA a thread keeps one 16-byte column vector of A and every RP-th row,
 // all loads of a pass issued before the first is used; lanes of one column
@@ -94,7 +94,6 @@ cudaError_t launch_r(const void* X, int64_t ldx, int64_t n, int64_t H, const voi
 // reported, nothing written.
 constexpr int RA_NT = 256;   // threads of a row-append CTA
 constexpr int RA_U = 8;      // vectors in flight per thread
-constexpr int RA_CL = 8;     // CTAs of a cluster (hidden split)
 
 template <typename T>
 __global__ void __launch_bounds__(RA_NT) append_row_at_len_kernel(
@@ -107,14 +106,14 @@ __global__ void __launch_bounds__(RA_NT) append_row_at_len_kernel(
   constexpr int VE = 16 / (int)sizeof(T);   // elements of a 16-byte vector
   __shared__ float red[RA_NT / 32][128];
   __shared__ float part[128];               // this CTA's sums, read by rank 0
-  const int rank = blockIdx.x, q = blockIdx.y, l = blockIdx.z;
+  const int rank = blockIdx.x, ncl = gridDim.x, q = blockIdx.y, l = blockIdx.z;   // one cluster in x
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int64_t len = kv_len[q];
   const bool bad = len < 1 || len > max_kv_len;   // uniform over the cluster
   const int VR = C / VE;            // vectors of an A row (divides 32)
   const int RP = RA_NT / VR;        // rows of one pass over the CTA
   const int cv = tid % VR;
-  const int64_t hb = rank * H / RA_CL, he = (rank + 1) * H / RA_CL;
+  const int64_t hb = rank * H / ncl, he = (rank + 1) * H / ncl;
   float acc[VE];
 #pragma unroll
   for (int e = 0; e < VE; ++e) acc[e] = 0.f;
@@ -156,8 +155,7 @@ __global__ void __launch_bounds__(RA_NT) append_row_at_len_kernel(
   if (rank == 0 && tid < C && !bad) {
     float v = 0.f;
     const uint32_t pa = ptx::smem_u32(part + tid);
-#pragma unroll
-    for (int k = 0; k < RA_CL; ++k) v += ptx::dsmem_ld(ptx::dsmem_addr(pa, k));
+    for (int k = 0; k < ncl; ++k) v += ptx::dsmem_ld(ptx::dsmem_addr(pa, k));
     lr[(int64_t)l * lr_agent + (int64_t)q * lr_seq + (len - 1) * C + tid] = from_f32<T>(v);
   }
   if (rank == 0 && tid == 0 && bad) atomicOr(err, 1);
@@ -173,17 +171,33 @@ cudaError_t launch_append_row_at_len(const void* x, const void* A, int64_t a_str
   const int ve = dt == LA_F32 ? 4 : 8;
   if (2 * r > 128 || (2 * r) % ve != 0 || 32 % ((2 * r) / ve) != 0 || n_seqs < 1 || n_lr < 1)
     return cudaErrorInvalidValue;
+  // 16 CTAs a cluster (a non-portable size) where the device takes it, else 8;
+  // decided once by an occupancy query, so that no launch is tried and refused
+  // (a refused launch would break a stream capture)
+  static int ncl_of[2] = {0, 0};
+  int& ncl = ncl_of[dt == LA_F32 ? 0 : 1];
+  const void* kfn = dt == LA_F32 ? reinterpret_cast<const void*>(append_row_at_len_kernel<float>)
+                                 : reinterpret_cast<const void*>(append_row_at_len_kernel<__nv_bfloat16>);
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(RA_CL, (unsigned)n_seqs, (unsigned)n_lr);
   cfg.blockDim = dim3(RA_NT);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = RA_CL;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if (ncl == 0) {
+    int n = 0;
+    cfg.gridDim = dim3(16, 1, 1);
+    attr[0].val.clusterDim.x = 16;
+    const bool ok16 = cudaFuncSetAttribute(kfn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess &&
+                      cudaOccupancyMaxActiveClusters(&n, kfn, &cfg) == cudaSuccess && n >= 1;
+    cudaGetLastError();
+    ncl = ok16 ? 16 : 8;
+  }
+  cfg.gridDim = dim3((unsigned)ncl, (unsigned)n_seqs, (unsigned)n_lr);
+  attr[0].val.clusterDim.x = (unsigned)ncl;
   cudaError_t e;
   if (dt == LA_F32)
     e = cudaLaunchKernelEx(&cfg, append_row_at_len_kernel<float>, static_cast<const float*>(x),

@@ -63,6 +63,29 @@ __device__ __forceinline__ uint32_t f2_f16x2(uint64_t v) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// 2^x for a pair on the FMA pipe, beside the SFU's ex2 (the softmax's
+// exponentials would otherwise queue on the SFU alone): x = n + f with n the
+// nearest integer (the 1.5 * 2^23 rounding constant), f in [-1/2, 1/2]; 2^f by
+// a degree-3 polynomial fitted here for least maximum relative error on that
+// interval (Remez exchange: 7.5e-5, below the bf16 rounding P gets), and 2^n
+// added to the exponent field.  x is clamped at -126, so a masked score gives
+// about 1e-38 instead of 0 and the sum never leaves the normal range.
+__device__ __forceinline__ uint64_t exp2_poly_f2(uint64_t x2) {
+  constexpr float kRound = 12582912.f;   // 1.5 * 2^23
+  const float2 xv = f2_unpack(x2);
+  const uint64_t x = f2(fmaxf(xv.x, -126.f), fmaxf(xv.y, -126.f));
+  const uint64_t t = add_f2(x, f2(kRound, kRound));
+  const uint64_t fr = sub_f2(x, sub_f2(t, f2(kRound, kRound)));
+  uint64_t p = fma_f2(f2(0.05517166853f, 0.05517166853f), fr, f2(0.24261112511f, 0.24261112511f));
+  p = fma_f2(p, fr, f2(0.69326096773f, 0.69326096773f));
+  p = fma_f2(p, fr, f2(0.99992805719f, 0.99992805719f));
+  const float2 pv = f2_unpack(p), tv = f2_unpack(t);
+  return f2(__uint_as_float(__float_as_uint(pv.x) + (__float_as_uint(tv.x) << 23)),
+            __uint_as_float(__float_as_uint(pv.y) + (__float_as_uint(tv.y) << 23)));
+}
+// every kPolyExpEvery-th pair of a softmax row goes through exp2_poly_f2 (0: none)
+constexpr int kPolyExpEvery = 4;
+
 constexpr int PD = 128;                  // head_dim
 constexpr int PKT = 128;                 // keys per tile
 constexpr int PM = 128;                  // query rows per CTA
@@ -389,19 +412,12 @@ __global__ void __launch_bounds__(PNTHR, 1)
       // this lane's pair of K elements in a 128-byte-swizzled row: key kb + gq
       // (+8), 16-byte chunk (2 grp + q) ^ gq, word t4; columns + d/2 are one box on
       const uint32_t rowb = kst + (uint32_t)(kb + gq) * 128 + 4 * t4;
-      // every group's delta columns requested before one wait: [grp][0..7] the
-      // columns i, [grp][8..15] the columns i + d/2
-      uint32_t xx[4][16];
 #pragma unroll
       for (int grp = 0; grp < 4; ++grp) {
-        tmem_ld16x256_x2(*reinterpret_cast<uint32_t(*)[8]>(&xx[grp][0]), tl + 16 * grp);
-        tmem_ld16x256_x2(*reinterpret_cast<uint32_t(*)[8]>(&xx[grp][8]), tl + 16 * grp + D / 2);
-      }
-      tmem_wait_ld_all(xx);
-#pragma unroll
-      for (int grp = 0; grp < 4; ++grp) {
-        const uint32_t* xl = xx[grp];
-        const uint32_t* xh = xx[grp] + 8;
+        uint32_t xl[8], xh[8];
+        tmem_ld16x256_x2(xl, tl + 16 * grp);
+        tmem_ld16x256_x2(xh, tl + 16 * grp + D / 2);
+        tmem_wait_ld_regs(xl, xh);
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
           const int i0 = 16 * grp + 8 * q + 2 * t4;
@@ -511,8 +527,17 @@ __global__ void __launch_bounds__(PNTHR, 1)
       for (int h = 0; h < 2; ++h)
 #pragma unroll
         for (int c = 0; c < 32; c += 2) {
-          const float2 xa = f2_unpack(fma_f2(f2(__uint_as_float(sv[h][c]), __uint_as_float(sv[h][c + 1])), scl, nmu));
-          const float p0 = fast_exp2(xa.x), p1 = fast_exp2(xa.y);
+          const uint64_t xa2 = fma_f2(f2(__uint_as_float(sv[h][c]), __uint_as_float(sv[h][c + 1])), scl, nmu);
+          float p0, p1;
+          if (kPolyExpEvery > 0 && (c / 2) % (kPolyExpEvery > 0 ? kPolyExpEvery : 1) == 0) {
+            const float2 pp = f2_unpack(exp2_poly_f2(xa2));
+            p0 = pp.x;
+            p1 = pp.y;
+          } else {
+            const float2 xa = f2_unpack(xa2);
+            p0 = fast_exp2(xa.x);
+            p1 = fast_exp2(xa.y);
+          }
           acc = add_f2(acc, f2(p0, p1));
           pk[16 * h + c / 2] = pack_bf16(p0, p1);
         }

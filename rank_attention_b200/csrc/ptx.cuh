@@ -268,16 +268,6 @@ __device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&a)[8], uint32_t (&b
                :
                : "memory");
 }
-// One tcgen05.wait::ld for several loads: the registers of every load are
-// named after the wait, so that no use moves above it
-template <int A, int B>
-__device__ __forceinline__ void tmem_wait_ld_all(uint32_t (&r)[A][B]) {
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-  for (int i = 0; i < A; ++i)
-#pragma unroll
-    for (int j = 0; j < B; ++j) asm volatile("" : "+r"(r[i][j]));
-}
 // 32 TMEM lanes x 32 columns: thread t gets lane t, 32 consecutive columns
 __device__ __forceinline__ void tmem_ld32x32b_x32(uint32_t (&r)[32], uint32_t taddr) {
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
