@@ -108,8 +108,6 @@ __global__ void __launch_bounds__(RA_NT) append_row_at_len_kernel(
   __shared__ float part[128];               // this CTA's sums, read by rank 0
   const int rank = blockIdx.x, ncl = gridDim.x, q = blockIdx.y, l = blockIdx.z;   // one cluster in x
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-  const int64_t len = kv_len[q];
-  const bool bad = len < 1 || len > max_kv_len;   // uniform over the cluster
   const int VR = C / VE;            // vectors of an A row (divides 32)
   const int RP = RA_NT / VR;        // rows of one pass over the CTA
   const int cv = tid % VR;
@@ -117,7 +115,7 @@ __global__ void __launch_bounds__(RA_NT) append_row_at_len_kernel(
   float acc[VE];
 #pragma unroll
   for (int e = 0; e < VE; ++e) acc[e] = 0.f;
-  if (!bad) {
+  {   // A's rows do not depend on the sequence's length: read before it arrives
     const T* xq = x + (int64_t)q * H;
     const uint4* Av = reinterpret_cast<const uint4*>(A + (int64_t)l * a_stride);
     for (int64_t h0 = hb + tid / VR; h0 < he; h0 += (int64_t)RP * RA_U) {
@@ -152,6 +150,8 @@ __global__ void __launch_bounds__(RA_NT) append_row_at_len_kernel(
     part[tid] = v;
   }
   ptx::cluster_sync_all();   // every CTA's sums are in place
+  const int64_t len = kv_len[q];
+  const bool bad = len < 1 || len > max_kv_len;
   if (rank == 0 && tid < C && !bad) {
     float v = 0.f;
     const uint32_t pa = ptx::smem_u32(part + tid);

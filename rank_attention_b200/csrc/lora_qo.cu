@@ -271,6 +271,184 @@ __global__ void __launch_bounds__(kOThreads) output_delta_kernel(
   }
 }
 
+// bf16 query side, 16 tokens a CTA: a thread owns 8 adjacent frequencies of
+// one head (16-byte vectors at columns i and i + d/2, the RoPE pairs) and
+// forms their deltas for 4 tokens at a time from one 16-byte read of each
+// B_q^a row; the base projections are read and the rotated queries written in
+// 16-byte vectors.  (cos, sin) of the CTA's positions are formed once (angle
+// reduced in fp64) in shared memory, with the tokens' LR rows.
+constexpr int kQ2Threads = 256;
+constexpr int kQ2Tok = 16;
+
+template <int R>
+__global__ void __launch_bounds__(kQ2Threads, 2) query_expand_v_kernel(
+    const __nv_bfloat16* __restrict__ q_base, const __nv_bfloat16* __restrict__ lr_q,
+    const __nv_bfloat16* __restrict__ B_q, __nv_bfloat16* q_out, int n_agents, int n_tok, int n_q,
+    int d, float s, RopeTheta rt, const int32_t* __restrict__ pos_end) {
+  __shared__ float lr[kQ2Tok][R];
+  __shared__ float2 cs[kQ2Tok][64];
+  const int h2 = d / 2, ld = n_q * d;
+  const int tb = blockIdx.x * kQ2Tok, agent = blockIdx.y, seq = blockIdx.z;
+  const int nt = min(kQ2Tok, n_tok - tb);
+  const int64_t row0 = ((int64_t)seq * n_agents + agent) * n_tok + tb;
+  const int64_t pos0 = (int64_t)pos_end[seq] - n_tok + tb;
+  for (int u = threadIdx.x; u < nt * R; u += kQ2Threads)
+    lr[u / R][u % R] = __bfloat162float(lr_q[(row0 + u / R) * R + u % R]);
+  for (int u = threadIdx.x; u < nt * h2; u += kQ2Threads)
+    cs[u / h2][u % h2] = rope_cs_exact(pos0 + u / h2, rt.theta[u % h2]);
+  __syncthreads();
+  const __nv_bfloat16* B = B_q + (int64_t)agent * R * ld;
+  const int cph = h2 / 8;                       // 8-frequency chunks of a head
+  for (int item = threadIdx.x; item < n_q * cph; item += kQ2Threads) {
+    const int h = item / cph, i0 = (item % cph) * 8;
+    const int c1 = h * d + i0, c2 = c1 + h2;
+#pragma unroll 1
+    for (int g0 = 0; g0 < nt; g0 += 4) {
+      float x1[4][8], x2[4][8];
+#pragma unroll
+      for (int tt = 0; tt < 4; ++tt)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) x1[tt][j] = x2[tt][j] = 0.f;
+#pragma unroll 2
+      for (int m = 0; m < R; ++m) {
+        const Vec8<__nv_bfloat16> b1 = ld8<__nv_bfloat16>(B + (int64_t)m * ld + c1);
+        const Vec8<__nv_bfloat16> b2 = ld8<__nv_bfloat16>(B + (int64_t)m * ld + c2);
+#pragma unroll
+        for (int tt = 0; tt < 4; ++tt) {
+          const float l = lr[(g0 + tt) & (kQ2Tok - 1)][m];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            x1[tt][j] = fmaf(l, b1.v[j], x1[tt][j]);
+            x2[tt][j] = fmaf(l, b2.v[j], x2[tt][j]);
+          }
+        }
+      }
+#pragma unroll
+      for (int tt = 0; tt < 4; ++tt) {
+        const int tok = g0 + tt;
+        if (tok < nt) {
+          const __nv_bfloat16* qb = q_base + (row0 + tok) * ld;
+          const Vec8<__nv_bfloat16> a1 = ld8<__nv_bfloat16>(qb + c1), a2 = ld8<__nv_bfloat16>(qb + c2);
+          uint32_t o1[4], o2[4];
+#pragma unroll
+          for (int j = 0; j < 8; j += 2) {
+            const float2 ca = cs[tok][i0 + j], cb = cs[tok][i0 + j + 1];
+            const float y1a = fmaf(s, x1[tt][j], a1.v[j]), y2a = fmaf(s, x2[tt][j], a2.v[j]);
+            const float y1b = fmaf(s, x1[tt][j + 1], a1.v[j + 1]), y2b = fmaf(s, x2[tt][j + 1], a2.v[j + 1]);
+            o1[j / 2] = pack_bf16(y1a * ca.x - y2a * ca.y, y1b * cb.x - y2b * cb.y);
+            o2[j / 2] = pack_bf16(y2a * ca.x + y1a * ca.y, y2b * cb.x + y1b * cb.y);
+          }
+          __nv_bfloat16* qo = q_out + (row0 + tok) * ld;
+          *reinterpret_cast<uint4*>(qo + c1) = make_uint4(o1[0], o1[1], o1[2], o1[3]);
+          *reinterpret_cast<uint4*>(qo + c2) = make_uint4(o2[0], o2[1], o2[2], o2[3]);
+        }
+      }
+    }
+  }
+}
+
+// bf16 output side on the tensor cores: one CTA per (16 tokens, agent,
+// sequence).  The shrink t = O A_o (16 tokens x r) runs as warp MMAs
+// (m16n8k16, fp32 accumulation): warp w takes every 8th 16-wide slice of d_in,
+// its A operand is the tokens' o rows read straight from memory, its B operand
+// A_o's 8 x 8 blocks read as rows and transposed in registers (movmatrix); the
+// warps' partial sums meet in shared memory.  The expand y += s t B_o^a stays
+// on the CUDA cores in fp32: a thread owns 8 consecutive output columns, reads
+// each row of B_o^a once as a 16-byte vector for 8 tokens, and updates y in
+// 16-byte vectors.  A_o and B_o^a are read once per 16 tokens.
+constexpr int kO2Threads = 256;
+constexpr int kO2Tok = 16;
+
+template <int R>
+__global__ void __launch_bounds__(kO2Threads, 2) output_delta_tc_kernel(
+    const __nv_bfloat16* __restrict__ o, const __nv_bfloat16* __restrict__ A_o, int64_t a_agent_stride,
+    const __nv_bfloat16* __restrict__ B_o, __nv_bfloat16* y, int n_agents, int n_tok, int d_in,
+    int d_out, float s) {
+  constexpr int NTN = R / 8;   // 8-column tiles of t
+  __shared__ float part[kO2Threads / 32][kO2Tok][R + 1];
+  __shared__ float t[kO2Tok][R];
+  const int tb = blockIdx.x * kO2Tok, agent = blockIdx.y, seq = blockIdx.z;
+  const int nt = min(kO2Tok, n_tok - tb);
+  const int64_t row0 = ((int64_t)seq * n_agents + agent) * n_tok + tb;
+  const __nv_bfloat16* A = A_o + agent * a_agent_stride;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, gq = lane >> 2, t4 = lane & 3;
+
+  // ---- shrink: t = O A_o on the tensor cores
+  float D[NTN][4];
+#pragma unroll
+  for (int n = 0; n < NTN; ++n) D[n][0] = D[n][1] = D[n][2] = D[n][3] = 0.f;
+  const uint32_t* olo = reinterpret_cast<const uint32_t*>(o + (row0 + gq) * d_in);
+  const uint32_t* ohi = reinterpret_cast<const uint32_t*>(o + (row0 + gq + 8) * d_in);
+  const bool vlo = gq < nt, vhi = gq + 8 < nt;
+  for (int k0 = 16 * w; k0 < d_in; k0 += 16 * (kO2Threads / 32)) {
+    uint32_t a[4];
+    a[0] = vlo ? __ldg(olo + (k0 >> 1) + t4) : 0u;
+    a[1] = vhi ? __ldg(ohi + (k0 >> 1) + t4) : 0u;
+    a[2] = vlo ? __ldg(olo + (k0 >> 1) + 4 + t4) : 0u;
+    a[3] = vhi ? __ldg(ohi + (k0 >> 1) + 4 + t4) : 0u;
+#pragma unroll
+    for (int n = 0; n < NTN; ++n) {
+      const uint32_t m0 = __ldg(reinterpret_cast<const uint32_t*>(A + (int64_t)(k0 + gq) * R + 8 * n + 2 * t4));
+      const uint32_t m1 = __ldg(reinterpret_cast<const uint32_t*>(A + (int64_t)(k0 + 8 + gq) * R + 8 * n + 2 * t4));
+      ptx::mma16816(D[n], a, ptx::movmatrix_t(m0), ptx::movmatrix_t(m1));
+    }
+  }
+#pragma unroll
+  for (int n = 0; n < NTN; ++n) {
+    part[w][gq][8 * n + 2 * t4] = D[n][0];
+    part[w][gq][8 * n + 2 * t4 + 1] = D[n][1];
+    part[w][gq + 8][8 * n + 2 * t4] = D[n][2];
+    part[w][gq + 8][8 * n + 2 * t4 + 1] = D[n][3];
+  }
+  __syncthreads();
+  for (int i = tid; i < kO2Tok * R; i += kO2Threads) {
+    const int tt = i / R, m = i % R;
+    float v = 0.f;
+#pragma unroll
+    for (int ww = 0; ww < kO2Threads / 32; ++ww) v += part[ww][tt][m];
+    t[tt][m] = v;
+  }
+  __syncthreads();
+
+  // ---- expand: y += s t B_o^a, 8 columns a thread, 8 tokens at a time
+  const __nv_bfloat16* B = B_o + (int64_t)agent * R * d_out;
+  for (int c = tid * 8; c < d_out; c += kO2Threads * 8) {
+#pragma unroll 1
+    for (int h = 0; h < kO2Tok / 8; ++h) {
+      if (8 * h >= nt) break;
+      float z[8][8];
+#pragma unroll
+      for (int tt = 0; tt < 8; ++tt)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) z[tt][j] = 0.f;
+#pragma unroll 2
+      for (int m = 0; m < R; ++m) {
+        const Vec8<__nv_bfloat16> b = ld8<__nv_bfloat16>(B + (int64_t)m * d_out + c);
+#pragma unroll
+        for (int tt = 0; tt < 8; ++tt) {
+          const float tv = t[8 * h + tt][m];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) z[tt][j] = fmaf(tv, b.v[j], z[tt][j]);
+        }
+      }
+#pragma unroll
+      for (int tt = 0; tt < 8; ++tt) {
+        if (8 * h + tt < nt) {
+          const uint4 yv = *reinterpret_cast<const uint4*>(y + (row0 + 8 * h + tt) * d_out + c);
+          const uint32_t yw[4] = {yv.x, yv.y, yv.z, yv.w};
+          uint32_t ow[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float y0 = __uint_as_float(yw[j] << 16), y1 = __uint_as_float(yw[j] & 0xffff0000u);
+            ow[j] = pack_bf16(fmaf(s, z[tt][2 * j], y0), fmaf(s, z[tt][2 * j + 1], y1));
+          }
+          *reinterpret_cast<uint4*>(y + (row0 + 8 * h + tt) * d_out + c) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+        }
+      }
+    }
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_query_expand(const void* q_base, const void* lr_q, const void* B_q, void* q_out,
@@ -281,6 +459,22 @@ cudaError_t launch_query_expand(const void* q_base, const void* lr_q, const void
   for (int i = 0; i < 64; ++i) {
     rt.theta[i] = i < d / 2 ? std::pow(rope_base, -2.0 * i / d) : 0.0;
     rt.thetaf[i] = (float)rt.theta[i];
+  }
+  // bf16 with 16-byte aligned rows: 16 tokens a CTA, 16-byte vectors
+  if (dt == LA_BF16 && ((int64_t)n_q * d) % 8 == 0 && (reinterpret_cast<uintptr_t>(q_base) & 15) == 0 &&
+      (reinterpret_cast<uintptr_t>(q_out) & 15) == 0 && (reinterpret_cast<uintptr_t>(B_q) & 15) == 0) {
+    const dim3 g2((unsigned)((n_tok + kQ2Tok - 1) / kQ2Tok), (unsigned)n_agents, (unsigned)n_seqs);
+    auto qb = static_cast<const __nv_bfloat16*>(q_base);
+    auto lq = static_cast<const __nv_bfloat16*>(lr_q);
+    auto bq = static_cast<const __nv_bfloat16*>(B_q);
+    auto qo = static_cast<__nv_bfloat16*>(q_out);
+    switch (r) {
+      case 8: query_expand_v_kernel<8><<<g2, kQ2Threads, 0, st>>>(qb, lq, bq, qo, n_agents, n_tok, n_q, d, s, rt, pos_end); break;
+      case 16: query_expand_v_kernel<16><<<g2, kQ2Threads, 0, st>>>(qb, lq, bq, qo, n_agents, n_tok, n_q, d, s, rt, pos_end); break;
+      case 32: query_expand_v_kernel<32><<<g2, kQ2Threads, 0, st>>>(qb, lq, bq, qo, n_agents, n_tok, n_q, d, s, rt, pos_end); break;
+      default: query_expand_v_kernel<64><<<g2, kQ2Threads, 0, st>>>(qb, lq, bq, qo, n_agents, n_tok, n_q, d, s, rt, pos_end); break;
+    }
+    return cudaGetLastError();
   }
   const int hpb = kQThreads / (d / 2 / kQF);
   const int hblocks = (n_q + hpb - 1) / hpb;
@@ -302,6 +496,26 @@ cudaError_t launch_query_expand(const void* q_base, const void* lr_q, const void
 cudaError_t launch_output_delta(const void* o, const void* A_o, int64_t a_agent_stride,
                                 const void* B_o, void* y, int n_seqs, int n_agents, int n_tok,
                                 int d_in, int d_out, int r, float s, la_dtype dt, cudaStream_t st) {
+  // bf16 with d_in a multiple of 16 (the MMA's k) and 16-byte aligned rows: the
+  // tensor-core shrink
+  const bool tc = dt == LA_BF16 && d_in % 16 == 0 && d_out % 8 == 0 &&
+                  (reinterpret_cast<uintptr_t>(o) & 15) == 0 && (reinterpret_cast<uintptr_t>(y) & 15) == 0 &&
+                  (reinterpret_cast<uintptr_t>(B_o) & 15) == 0 && (reinterpret_cast<uintptr_t>(A_o) & 3) == 0 &&
+                  (a_agent_stride & 1) == 0;
+  if (tc) {
+    const dim3 g2((unsigned)((n_tok + kO2Tok - 1) / kO2Tok), (unsigned)n_agents, (unsigned)n_seqs);
+    auto o2 = static_cast<const __nv_bfloat16*>(o);
+    auto a2 = static_cast<const __nv_bfloat16*>(A_o);
+    auto b2 = static_cast<const __nv_bfloat16*>(B_o);
+    auto y2 = static_cast<__nv_bfloat16*>(y);
+    switch (r) {
+      case 8: output_delta_tc_kernel<8><<<g2, kO2Threads, 0, st>>>(o2, a2, a_agent_stride, b2, y2, n_agents, n_tok, d_in, d_out, s); break;
+      case 16: output_delta_tc_kernel<16><<<g2, kO2Threads, 0, st>>>(o2, a2, a_agent_stride, b2, y2, n_agents, n_tok, d_in, d_out, s); break;
+      case 32: output_delta_tc_kernel<32><<<g2, kO2Threads, 0, st>>>(o2, a2, a_agent_stride, b2, y2, n_agents, n_tok, d_in, d_out, s); break;
+      default: output_delta_tc_kernel<64><<<g2, kO2Threads, 0, st>>>(o2, a2, a_agent_stride, b2, y2, n_agents, n_tok, d_in, d_out, s); break;
+    }
+    return cudaGetLastError();
+  }
   const int cblocks = (d_out + kOColBlock - 1) / kOColBlock;
   const dim3 grid((unsigned)((int64_t)(n_tok + kOTok - 1) / kOTok * cblocks), (unsigned)n_agents,
                   (unsigned)n_seqs);

@@ -751,6 +751,9 @@ def _qo_inputs(n_seqs, n_agents, n_tok, n_q, d, r, dtype, seed):
     (torch.bfloat16, 1, 3, 1, 32, 128, 16, False),    # one decode step of the 3-agent layer
     (torch.bfloat16, 2, 2, 37, 32, 128, 64, True),    # a ragged prefill chunk, in place
     (torch.float32, 2, 3, 5, 4, 64, 8, False),        # the tiny fp32 shape
+    (torch.bfloat16, 1, 3, 1024, 32, 128, 16, False), # the 1024-token chunk of the 3-agent layer
+    (torch.bfloat16, 1, 2, 20, 8, 64, 32, True),      # head_dim 64, r = 32, ragged, in place
+    (torch.bfloat16, 2, 1, 17, 4, 128, 8, False),     # r = 8, fewer heads than threads
 ])
 def test_query_expand_against_oracle(la, dtype, n_seqs, n_agents, n_tok, n_q, d, r, in_place):
     q_base, lr_q, B_q = _qo_inputs(n_seqs, n_agents, n_tok, n_q, d, r, dtype, 300 + r)
@@ -769,12 +772,17 @@ def test_query_expand_against_oracle(la, dtype, n_seqs, n_agents, n_tok, n_q, d,
     assert_parity(to_np(out), ref, dtype)
 
 
-@pytest.mark.parametrize("dtype,n_seqs,n_agents,n_tok,r,per_agent_A", [
-    (torch.bfloat16, 1, 3, 1, 16, False),     # a decode step, shared A_o
-    (torch.bfloat16, 2, 2, 19, 64, True),     # ragged token blocks, per-agent A_o
-    (torch.float32, 1, 2, 9, 8, False),
+@pytest.mark.parametrize("dtype,n_seqs,n_agents,n_tok,r,per_agent_A,zero_base", [
+    (torch.bfloat16, 1, 3, 1, 16, False, False),     # a decode step, shared A_o
+    (torch.bfloat16, 2, 2, 19, 64, True, False),     # ragged token blocks, per-agent A_o
+    (torch.float32, 1, 2, 9, 8, False, False),
+    # y = 0 on entry: the bf16 delta alone against the oracle (tensor-core shrink)
+    (torch.bfloat16, 1, 3, 1024, 16, False, True),   # the 1024-token chunk of the 3-agent layer
+    (torch.bfloat16, 2, 2, 19, 64, True, True),
+    (torch.bfloat16, 1, 2, 33, 8, False, True),
+    (torch.bfloat16, 1, 1, 16, 32, True, True),
 ])
-def test_output_delta_against_oracle(la, dtype, n_seqs, n_agents, n_tok, r, per_agent_A):
+def test_output_delta_against_oracle(la, dtype, n_seqs, n_agents, n_tok, r, per_agent_A, zero_base):
     d_in, d_out = 4096, 4096
     g = torch.Generator().manual_seed(400 + r)
     o = torch.randn(n_seqs, n_agents, n_tok, d_in, generator=g).to(dtype)
@@ -782,6 +790,8 @@ def test_output_delta_against_oracle(la, dtype, n_seqs, n_agents, n_tok, r, per_
     A_o = (0.02 * torch.randn(*A_shape, generator=g)).to(dtype)
     B_o = (0.02 * torch.randn(n_agents, r, d_out, generator=g)).to(dtype)
     y0 = torch.randn(n_seqs, n_agents, n_tok, d_out, generator=g).to(dtype)
+    if zero_base:
+        y0.zero_()
     y = y0.to(DEV)
     s = 2.0
     la.lora_output_delta(o.to(DEV), A_o.to(DEV), B_o.to(DEV), y, lora_scale=s)
