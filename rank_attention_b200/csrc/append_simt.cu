@@ -107,6 +107,7 @@ __global__ void __launch_bounds__(RA_NT) append_row_at_len_kernel(
   __shared__ float red[RA_NT / 32][128];
   __shared__ float part[128];               // this CTA's sums, read by rank 0
   const int rank = blockIdx.x, ncl = gridDim.x, q = blockIdx.y, l = blockIdx.z;   // one cluster in x
+  const int64_t len = kv_len[q];   // requested now, first used at the end
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   const int VR = C / VE;            // vectors of an A row (divides 32)
   const int RP = RA_NT / VR;        // rows of one pass over the CTA
@@ -150,12 +151,16 @@ __global__ void __launch_bounds__(RA_NT) append_row_at_len_kernel(
     part[tid] = v;
   }
   ptx::cluster_sync_all();   // every CTA's sums are in place
-  const int64_t len = kv_len[q];
   const bool bad = len < 1 || len > max_kv_len;
   if (rank == 0 && tid < C && !bad) {
-    float v = 0.f;
+    // every CTA's sum requested before the first is added
+    float pv[16];
     const uint32_t pa = ptx::smem_u32(part + tid);
-    for (int k = 0; k < ncl; ++k) v += ptx::dsmem_ld(ptx::dsmem_addr(pa, k));
+#pragma unroll
+    for (int k = 0; k < 16; ++k) pv[k] = k < ncl ? ptx::dsmem_ld(ptx::dsmem_addr(pa, k)) : 0.f;
+    float v = 0.f;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) v += pv[k];
     lr[(int64_t)l * lr_agent + (int64_t)q * lr_seq + (len - 1) * C + tid] = from_f32<T>(v);
   }
   if (rank == 0 && tid == 0 && bad) atomicOr(err, 1);

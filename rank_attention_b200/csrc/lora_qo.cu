@@ -304,6 +304,14 @@ __global__ void __launch_bounds__(kQ2Threads, 2) query_expand_v_kernel(
     const int c1 = h * d + i0, c2 = c1 + h2;
 #pragma unroll 1
     for (int g0 = 0; g0 < nt; g0 += 4) {
+      // the group's base projections requested before the deltas are formed
+      uint4 qa[4][2];
+#pragma unroll
+      for (int tt = 0; tt < 4; ++tt) {
+        const __nv_bfloat16* qb = q_base + (row0 + g0 + tt) * ld;
+        qa[tt][0] = g0 + tt < nt ? *reinterpret_cast<const uint4*>(qb + c1) : make_uint4(0, 0, 0, 0);
+        qa[tt][1] = g0 + tt < nt ? *reinterpret_cast<const uint4*>(qb + c2) : make_uint4(0, 0, 0, 0);
+      }
       float x1[4][8], x2[4][8];
 #pragma unroll
       for (int tt = 0; tt < 4; ++tt)
@@ -327,8 +335,8 @@ __global__ void __launch_bounds__(kQ2Threads, 2) query_expand_v_kernel(
       for (int tt = 0; tt < 4; ++tt) {
         const int tok = g0 + tt;
         if (tok < nt) {
-          const __nv_bfloat16* qb = q_base + (row0 + tok) * ld;
-          const Vec8<__nv_bfloat16> a1 = ld8<__nv_bfloat16>(qb + c1), a2 = ld8<__nv_bfloat16>(qb + c2);
+          const Vec8<__nv_bfloat16> a1 = ld8<__nv_bfloat16>(reinterpret_cast<const __nv_bfloat16*>(&qa[tt][0]));
+          const Vec8<__nv_bfloat16> a2 = ld8<__nv_bfloat16>(reinterpret_cast<const __nv_bfloat16*>(&qa[tt][1]));
           uint32_t o1[4], o2[4];
 #pragma unroll
           for (int j = 0; j < 8; j += 2) {
@@ -397,8 +405,10 @@ __global__ void __launch_bounds__(kO2Threads, 2) output_delta_tc_kernel(
   for (int n = 0; n < NTN; ++n) {
     part[w][gq][8 * n + 2 * t4] = D[n][0];
     part[w][gq][8 * n + 2 * t4 + 1] = D[n][1];
-    part[w][gq + 8][8 * n + 2 * t4] = D[n][2];
-    part[w][gq + 8][8 * n + 2 * t4 + 1] = D[n][3];
+    if (gq + 8 < kO2Tok) {   // the MMA's rows 8 .. 15 exist only with 16 tokens a CTA
+      part[w][gq + 8][8 * n + 2 * t4] = D[n][2];
+      part[w][gq + 8][8 * n + 2 * t4 + 1] = D[n][3];
+    }
   }
   __syncthreads();
   for (int i = tid; i < kO2Tok * R; i += kO2Threads) {
