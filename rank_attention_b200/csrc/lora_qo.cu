@@ -355,6 +355,84 @@ __global__ void __launch_bounds__(kQ2Threads, 2) query_expand_v_kernel(
   }
 }
 
+// bf16 query side on the tensor cores (r >= 16): one CTA per (16 tokens,
+// agent, sequence).  The deltas D = lr_q B_q^a (16 tokens x 8 columns a tile)
+// are warp MMAs (m16n8k16, fp32 accumulation; bf16 x bf16 products are exact
+// in fp32, as on the CUDA cores): the A operand is the tokens' LR rows, the B
+// operand B_q^a's 8 x 8 blocks read as rows and transposed in registers
+// (movmatrix), so that B_q^a is read once per 16 tokens.  A warp takes the
+// column tiles c and c + d/2 of a head together, so each thread holds both
+// elements of its RoPE pairs, adds them to the base projection and rotates.
+template <int R>
+__global__ void __launch_bounds__(kQ2Threads) query_expand_tc_kernel(
+    const __nv_bfloat16* q_base, const __nv_bfloat16* __restrict__ lr_q,
+    const __nv_bfloat16* __restrict__ B_q, __nv_bfloat16* q_out, int n_agents, int n_tok, int n_q,
+    int d, float s, RopeTheta rt, const int32_t* __restrict__ pos_end) {
+  constexpr int KS = R / 16;                   // k-steps of the MMA
+  __shared__ __align__(16) uint32_t lrs[kQ2Tok][R / 2 + 4];   // bf16 pairs, padded rows
+  __shared__ float2 cs[kQ2Tok][64];
+  const int h2 = d / 2, ld = n_q * d;
+  const int tb = blockIdx.x * kQ2Tok, agent = blockIdx.y, seq = blockIdx.z;
+  const int nt = min(kQ2Tok, n_tok - tb);
+  const int64_t row0 = ((int64_t)seq * n_agents + agent) * n_tok + tb;
+  const int64_t pos0 = (int64_t)pos_end[seq] - n_tok + tb;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, gq = lane >> 2, t4 = lane & 3;
+  for (int u = tid; u < kQ2Tok * (R / 2); u += kQ2Threads) {
+    const int tt = u / (R / 2), c = u % (R / 2);
+    lrs[tt][c] = tt < nt ? *reinterpret_cast<const uint32_t*>(lr_q + (row0 + tt) * R + 2 * c) : 0u;
+  }
+  for (int u = tid; u < nt * h2; u += kQ2Threads)
+    cs[u / h2][u % h2] = rope_cs_exact(pos0 + u / h2, rt.theta[u % h2]);
+  __syncthreads();
+  // A fragments (tokens x r), the same for every column tile
+  uint32_t a[KS][4];
+#pragma unroll
+  for (int k = 0; k < KS; ++k) {
+    a[k][0] = lrs[gq][8 * k + t4];
+    a[k][1] = lrs[gq + 8][8 * k + t4];
+    a[k][2] = lrs[gq][8 * k + 4 + t4];
+    a[k][3] = lrs[gq + 8][8 * k + 4 + t4];
+  }
+  const __nv_bfloat16* B = B_q + (int64_t)agent * R * ld;
+  const bool v0 = gq < nt, v1 = gq + 8 < nt;
+  const int tph = h2 / 8;                       // column-tile pairs of a head
+  for (int pr = w; pr < n_q * tph; pr += kQ2Threads / 32) {
+    const int h = pr / tph, c = 8 * (pr % tph) + 2 * t4;   // this thread's columns c, c + 1 (and + d/2)
+    const int64_t col1 = (int64_t)h * d + c, col2 = col1 + h2;
+    // the base projections, requested before the MMAs
+    const uint32_t* qb0 = reinterpret_cast<const uint32_t*>(q_base + (row0 + gq) * ld);
+    const uint32_t* qb1 = reinterpret_cast<const uint32_t*>(q_base + (row0 + gq + 8) * ld);
+    const uint32_t b00 = v0 ? qb0[col1 >> 1] : 0u, b01 = v0 ? qb0[col2 >> 1] : 0u;
+    const uint32_t b10 = v1 ? qb1[col1 >> 1] : 0u, b11 = v1 ? qb1[col2 >> 1] : 0u;
+    float d1[4] = {0.f, 0.f, 0.f, 0.f}, d2[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int k = 0; k < KS; ++k) {
+      const __nv_bfloat16* Bk = B + (int64_t)(16 * k + gq) * ld + (int64_t)h * d + 8 * (pr % tph) + 2 * t4;
+      const uint32_t m10 = __ldg(reinterpret_cast<const uint32_t*>(Bk));
+      const uint32_t m11 = __ldg(reinterpret_cast<const uint32_t*>(Bk + 8 * (int64_t)ld));
+      const uint32_t m20 = __ldg(reinterpret_cast<const uint32_t*>(Bk + h2));
+      const uint32_t m21 = __ldg(reinterpret_cast<const uint32_t*>(Bk + 8 * (int64_t)ld + h2));
+      ptx::mma16816(d1, a[k], ptx::movmatrix_t(m10), ptx::movmatrix_t(m11));
+      ptx::mma16816(d2, a[k], ptx::movmatrix_t(m20), ptx::movmatrix_t(m21));
+    }
+    // rows gq (d[0], d[1]) and gq + 8 (d[2], d[3]); columns c, c + 1
+#pragma unroll
+    for (int hr = 0; hr < 2; ++hr) {
+      const int tok = gq + 8 * hr;
+      if (tok >= nt) continue;
+      const uint32_t u1 = hr ? b10 : b00, u2 = hr ? b11 : b01;
+      const float2 ca = cs[tok][c], cb = cs[tok][c + 1];
+      const float y1a = fmaf(s, d1[2 * hr], __uint_as_float(u1 << 16));
+      const float y1b = fmaf(s, d1[2 * hr + 1], __uint_as_float(u1 & 0xffff0000u));
+      const float y2a = fmaf(s, d2[2 * hr], __uint_as_float(u2 << 16));
+      const float y2b = fmaf(s, d2[2 * hr + 1], __uint_as_float(u2 & 0xffff0000u));
+      uint32_t* qo = reinterpret_cast<uint32_t*>(q_out + (row0 + tok) * ld);
+      qo[col1 >> 1] = pack_bf16(y1a * ca.x - y2a * ca.y, y1b * cb.x - y2b * cb.y);
+      qo[col2 >> 1] = pack_bf16(y2a * ca.x + y1a * ca.y, y2b * cb.x + y1b * cb.y);
+    }
+  }
+}
+
 // bf16 output side on the tensor cores: one CTA per (16 tokens, agent,
 // sequence).  The shrink t = O A_o (16 tokens x r) runs as warp MMAs
 // (m16n8k16, fp32 accumulation): warp w takes every 8th 16-wide slice of d_in,
@@ -478,11 +556,11 @@ cudaError_t launch_query_expand(const void* q_base, const void* lr_q, const void
     auto lq = static_cast<const __nv_bfloat16*>(lr_q);
     auto bq = static_cast<const __nv_bfloat16*>(B_q);
     auto qo = static_cast<__nv_bfloat16*>(q_out);
-    switch (r) {
+    switch (r) {   // r = 8: the CUDA-core kernel (the MMA's k is 16)
       case 8: query_expand_v_kernel<8><<<g2, kQ2Threads, 0, st>>>(qb, lq, bq, qo, n_agents, n_tok, n_q, d, s, rt, pos_end); break;
-      case 16: query_expand_v_kernel<16><<<g2, kQ2Threads, 0, st>>>(qb, lq, bq, qo, n_agents, n_tok, n_q, d, s, rt, pos_end); break;
-      case 32: query_expand_v_kernel<32><<<g2, kQ2Threads, 0, st>>>(qb, lq, bq, qo, n_agents, n_tok, n_q, d, s, rt, pos_end); break;
-      default: query_expand_v_kernel<64><<<g2, kQ2Threads, 0, st>>>(qb, lq, bq, qo, n_agents, n_tok, n_q, d, s, rt, pos_end); break;
+      case 16: query_expand_tc_kernel<16><<<g2, kQ2Threads, 0, st>>>(qb, lq, bq, qo, n_agents, n_tok, n_q, d, s, rt, pos_end); break;
+      case 32: query_expand_tc_kernel<32><<<g2, kQ2Threads, 0, st>>>(qb, lq, bq, qo, n_agents, n_tok, n_q, d, s, rt, pos_end); break;
+      default: query_expand_tc_kernel<64><<<g2, kQ2Threads, 0, st>>>(qb, lq, bq, qo, n_agents, n_tok, n_q, d, s, rt, pos_end); break;
     }
     return cudaGetLastError();
   }
