@@ -271,7 +271,9 @@ la_status lora_attn_prefill(const la_attn_args* args, la_stream_t stream);
 /*
  * lora_attn_decode -- one query token per (sequence, agent), split over the
  * sequence (split-K).  On the tensor-core path (bf16, head_dim 128, r in
- * {16, 32, 64}, at most three agents) the partial results are merged inside
+ * {16, 32, 64}, at most three agents) the rotated key delta and the scaled
+ * queries s q are scored in fp16: they must stay below 65504 in magnitude
+ * there.  On that path the partial results are merged inside
  * the same launch: that launch is cooperative (every CTA resident at once,
  * at most one per SM), so it fails with LA_ERR_CUDA on a device whose SMs
  * are partly taken by a context limit.  Other shapes merge in the same

@@ -22,7 +22,8 @@
 //      q . K^a_t = q . K_base,t + (s R(-k0) q) . R(j) (LRk_t B_k^a):
 //    dK^a comes out of TMEM in the mma.sync fragment layout, is turned by
 //    R(j) -- whose cos / sin are per-thread constants, j being fixed per
-//    thread -- and scored (mma.sync) against the tile's rotated queries
+//    thread; the turn runs on f16 pairs -- and scored (f16 mma.sync) against
+//    the tile's rotated queries
 //    Q' = s R(-k0) Q.  The tile's row maxima meet in shared memory; the warps
 //    write P (bf16) and rescale O_base^T in TMEM when a row's maximum moved.
 //  * 2 value warps: the value side reordered (LRAgent explainer, Metodologia
@@ -729,7 +730,7 @@ struct TCfg {
 };
 
 // Q' = R(-k0) Q scaled by s for one frequency i of every row, from the
-// scaled (cos, sin)(k0 theta_i) (bf16 in, bf16 out; swizzled 64-column boxes).
+// scaled (cos, sin)(k0 theta_i) (bf16 in, f16 out; swizzled 64-column boxes).
 template <int D, int SRC_ROWS, int DST_ROWS>
 __device__ __forceinline__ void rotate_queries_cs(uint32_t qs_u, uint32_t qp_u, float c, float sn, int i) {
 #pragma unroll 4
@@ -738,8 +739,8 @@ __device__ __forceinline__ void rotate_queries_cs(uint32_t qs_u, uint32_t qp_u, 
     asm volatile("ld.shared.b16 %0, [%1];" : "=h"(a) : "r"(qs_u + tile_off<D, SRC_ROWS>(row, i)));
     asm volatile("ld.shared.b16 %0, [%1];" : "=h"(b) : "r"(qs_u + tile_off<D, SRC_ROWS>(row, i + D / 2)));
     const float x1 = __uint_as_float((uint32_t)a << 16), x2 = __uint_as_float((uint32_t)b << 16);
-    const __nv_bfloat16 y1 = __float2bfloat16_rn(fmaf(x1, c, x2 * sn));
-    const __nv_bfloat16 y2 = __float2bfloat16_rn(fmaf(x2, c, -x1 * sn));
+    const __half y1 = __float2half_rn(fmaf(x1, c, x2 * sn));
+    const __half y2 = __float2half_rn(fmaf(x2, c, -x1 * sn));
     sts16(qp_u + tile_off<D, DST_ROWS>(row, i), *reinterpret_cast<const uint16_t*>(&y1));
     sts16(qp_u + tile_off<D, DST_ROWS>(row, i + D / 2), *reinterpret_cast<const uint16_t*>(&y2));
   }
@@ -880,9 +881,9 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
   const int64_t kvl = p.kv_len[seq];  // in flight while the constants are computed
   const int sp = w & 3, kb = 32 * sp + 16 * (w >> 2);  // score warp: TMEM sub-partition, first key
   // R(j) for this thread's keys j = kb + gq + 8 hh and its frequencies
-  // i = 16 grp + 8 q + 2 t4 (+1), as (cos, cos) and (sin, sin) pairs over the
-  // two adjacent frequencies: the operands of the packed f32x2 rotation
-  uint64_t RC[C::NG][2][2], RS[C::NG][2][2];
+  // i = 16 grp + 8 q + 2 t4 (+1), as (cos, cos) and (sin, sin) f16 pairs over
+  // the two adjacent frequencies: the operands of the packed f16x2 rotation
+  uint32_t RC[C::NG][2][2], RS[C::NG][2][2];
   if (w < TC_NES) {
 #pragma unroll
     for (int grp = 0; grp < C::NG; ++grp)
@@ -894,8 +895,8 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
         for (int hh = 0; hh < 2; ++hh) {
           const float j = (float)(kb + gq + 8 * hh);
           const float2 a = sincos_small(j * th0), b = sincos_small(j * th1);
-          RC[grp][hh][q] = f2(a.x, b.x);
-          RS[grp][hh][q] = f2(a.y, b.y);
+          RC[grp][hh][q] = pack_half2(make_float2(a.x, b.x));
+          RS[grp][hh][q] = pack_half2(make_float2(a.y, b.y));
         }
       }
   }
@@ -943,8 +944,8 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
       for (int e = 0; e < 4; ++e) {
         const float2 a = unpack_bf16(x1[e]), b = unpack_bf16(x2[e]);
         const float2 c0 = cs0[8 * c + 2 * e], c1 = cs0[8 * c + 2 * e + 1];
-        o1[e] = pack_bf16(fmaf(a.x, c0.x, b.x * c0.y), fmaf(a.y, c1.x, b.y * c1.y));
-        o2[e] = pack_bf16(fmaf(b.x, c0.x, -a.x * c0.y), fmaf(b.y, c1.x, -a.y * c1.y));
+        o1[e] = pack_half2(make_float2(fmaf(a.x, c0.x, b.x * c0.y), fmaf(a.y, c1.x, b.y * c1.y)));
+        o2[e] = pack_half2(make_float2(fmaf(b.x, c0.x, -a.x * c0.y), fmaf(b.y, c1.x, -a.y * c1.y)));
       }
       *reinterpret_cast<uint4*>(qpb0 + tile_off<D, ROWS>(row, c * 8)) = y1;
       *reinterpret_cast<uint4*>(qpb0 + tile_off<D, ROWS>(row, c * 8 + D / 2)) = y2;
@@ -1023,20 +1024,23 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
             for (int q = 0; q < 2; ++q)
 #pragma unroll
               for (int hh = 0; hh < 2; ++hh) {
-                // (x1, x2) = delta columns (i, i + d/2) at two adjacent i; R(j) x
-                const uint64_t x1 = f2(__uint_as_float(xl[cb][4 * q + 2 * hh]), __uint_as_float(xl[cb][4 * q + 2 * hh + 1]));
-                const uint64_t x2 = f2(__uint_as_float(xh[cb][4 * q + 2 * hh]), __uint_as_float(xh[cb][4 * q + 2 * hh + 1]));
-                const uint64_t c = RC[grp][hh][q], sn = RS[grp][hh][q];
-                const float2 l2 = f2_unpack(sub_f2(mul_f2(x1, c), mul_f2(x2, sn)));
-                const float2 h2 = f2_unpack(fma_f2(x2, c, mul_f2(x1, sn)));
-                A_lo[2 * q + hh] = pack_bf16(l2.x, l2.y);
-                A_hi[2 * q + hh] = pack_bf16(h2.x, h2.y);
+                // (x1, x2) = delta columns (i, i + d/2) at two adjacent i, as
+                // f16 pairs; R(j) x in f16x2 arithmetic: the rotated delta is the
+                // f16 A operand of the scoring MMA
+                const __half2 x1 = __floats2half2_rn(__uint_as_float(xl[cb][4 * q + 2 * hh]), __uint_as_float(xl[cb][4 * q + 2 * hh + 1]));
+                const __half2 x2 = __floats2half2_rn(__uint_as_float(xh[cb][4 * q + 2 * hh]), __uint_as_float(xh[cb][4 * q + 2 * hh + 1]));
+                const __half2 c = *reinterpret_cast<const __half2*>(&RC[grp][hh][q]);
+                const __half2 sn = *reinterpret_cast<const __half2*>(&RS[grp][hh][q]);
+                const __half2 l2 = __hfma2(x1, c, __hneg2(__hmul2(x2, sn)));
+                const __half2 h2 = __hfma2(x2, c, __hmul2(x1, sn));
+                A_lo[2 * q + hh] = *reinterpret_cast<const uint32_t*>(&l2);
+                A_hi[2 * q + hh] = *reinterpret_cast<const uint32_t*>(&h2);
               }
             uint32_t bq[4];
             ldsm_x4(bq, qpb + tile_off<D, ROWS>(8 * pa + rr, 16 * grp + (mi & 1) * 8 + (mi >> 1) * (D / 2)));
             if (!mn) bq[0] = bq[1] = bq[2] = bq[3] = 0u;
-            mma16816(Sd, A_lo, bq[0], bq[1]);
-            mma16816(Sd, A_hi, bq[2], bq[3]);
+            mma16816_f16(Sd, A_lo, bq[0], bq[1]);
+            mma16816_f16(Sd, A_hi, bq[2], bq[3]);
           }
 #pragma unroll
           for (int pt = 0; pt < NT; ++pt)
