@@ -29,6 +29,10 @@ What it computes, and from which passage:
   BaseShared.  PreLRShared fills every agent's cache when a chunk first passes
   through the model -- PReCache blog (rit.work), how PReCache precomputes each
   role's cache.
+* A decode split over devices by key slices (no passage on the pages: the
+  decode's split-K merge of partial softmax results, taken across devices):
+  ``decode_slice`` and ``combine_slices``, pinned by the merge reproducing
+  the whole decode.
 
 The oracle MATERIALISES every agent's full K^a and V^a and runs a naive
 two-pass softmax (max, then exp / sum).  It does not use the reordered value
@@ -259,3 +263,49 @@ def lora_attention(k_base, v_base, lr, B_k, B_v, q, kv_len, *, lora_scale: float
                     kv_len=kv_len[s_], q_positions=qpos, lora_scale=lora_scale,
                     softmax_scale=softmax_scale, rope_base=rope_base)
     return out
+
+
+# ----------------------------------------------------------------------------
+# Sequence-sharded decode: one slice of the keys, and the merge of slices
+# ----------------------------------------------------------------------------
+# The pages show no multi-device step.  A device holding keys [lo, hi) of a
+# sequence decodes over those keys alone; the attention over all keys is the
+# merge of the slices' results by the online-softmax rescale (the same merge
+# that combines the splits of one device's decode).
+def decode_slice(k_base, v_base, lr, B_k, B_v, q, *, seq: int, agent: int, kv_head: int,
+                 lo: int, hi: int, lora_scale: float, softmax_scale: float, rope_base: float):
+    """Decode of one (sequence, agent, KV head) over keys [lo, hi) only, at
+    their own positions lo .. hi - 1.  Returns (out [g, d], M [g], L [g]):
+    out = softmax over the slice's keys times V^a, M = max_t (q . K^a_t) *
+    softmax_scale * log2(e), L = sum_t 2^((q . K^a_t) * softmax_scale *
+    log2(e) - M); an empty slice gives out 0, M = -inf, L = 0."""
+    d = k_base.shape[-1]
+    r = lr.shape[-1] // 2
+    g = q.shape[3] // k_base.shape[1]
+    heads = range(kv_head * g, (kv_head + 1) * g)
+    if hi <= lo:
+        return np.zeros((g, d)), np.full(g, -np.inf), np.zeros(g)
+    kpos = np.arange(lo, hi)
+    lr_s = _np64(lr[agent, seq, lo:hi] if lr.ndim == 4 else lr[seq, lo:hi])
+    cols = slice(kv_head * d, (kv_head + 1) * d)
+    Ka = agent_keys(k_base[seq, kv_head, lo:hi], lr_s[:, :r], _np64(B_k[agent])[:, cols],
+                    lora_scale, kpos, rope_base)
+    Va = agent_values(v_base[seq, kv_head, lo:hi], lr_s[:, r:], _np64(B_v[agent])[:, cols],
+                      lora_scale)
+    qh = _np64(q[seq, agent, 0])[list(heads)]             # [g, d]
+    z = (qh @ Ka.T) * softmax_scale * np.log2(np.e)        # scores in log2 units
+    M = z.max(axis=1)
+    e = np.exp2(z - M[:, None])
+    L = e.sum(axis=1)
+    return (e / L[:, None]) @ Va, M, L
+
+
+def combine_slices(outs, Ms, Ls) -> np.ndarray:
+    """Merge of slice results of the same rows: outs [n, rows, d], Ms, Ls
+    [n, rows].  w_p = 2^(M_p - M*) L_p with M* = max_p M_p;
+    out = sum_p w_p out_p / sum_p w_p (0 where no slice has keys)."""
+    outs, Ms, Ls = _np64(outs), _np64(Ms), _np64(Ls)
+    Mx = Ms.max(axis=0)
+    w = np.where(Ls > 0, np.exp2(Ms - np.where(np.isfinite(Mx), Mx, 0.0)[None]) * Ls, 0.0)
+    tot = w.sum(axis=0)
+    return np.where(tot[..., None] > 0, (w[..., None] * outs).sum(axis=0) / np.where(tot > 0, tot, 1.0)[..., None], 0.0)
