@@ -189,6 +189,19 @@ typedef struct {
    * role's cache.  The base cache stays shared in both cases. */
   int64_t lr_agent_stride;
   int32_t value_path;   /* la_value_path; 0 (zeroed struct) = LA_VALUE_REORDERED */
+  /* Sequence-sharded decode: several devices each hold a slice of every
+   * sequence's keys (both fields 0 / NULL in a zeroed struct: the unsharded
+   * decode).  key_pos0: position of the caches' key row 0, so local key t is
+   * RoPE'd as position key_pos0 + t.  row_stats: device float
+   * [n_seqs][n_agents][n_q_heads][2] that the decode fills, per output row,
+   * with M = max_t (q . K^a_t) * softmax_scale * log2(e) over its keys and
+   * L = sum_t 2^(q . K^a_t * softmax_scale * log2(e) - M); with row_stats a
+   * kv_len[q] of 0 is allowed (no keys: output 0, M = -inf, L = 0).  Either
+   * needs the tensor-core decode (bf16, head_dim 128, r in {16, 32, 64});
+   * elsewhere it returns LA_ERR_UNSUPPORTED.  lora_attn_decode_combine merges
+   * the slices' outputs. */
+  int64_t key_pos0;
+  float* row_stats;
 } la_attn_args;
 
 /*
@@ -294,6 +307,28 @@ la_status lora_attn_decode(const la_attn_args* args, void* workspace, size_t wor
 
 /* Workspace bytes lora_attn_decode needs for these arguments (0 if invalid). */
 size_t lora_attn_decode_workspace_bytes(const la_attn_args* args);
+
+/*
+ * lora_attn_decode_combine -- merge the decodes of n_parts key slices of the
+ * same queries (the sequence-sharded decode: each slice decoded with
+ * row_stats, on its own device, and the slices' outputs and stats gathered,
+ * e.g. by an all-gather over NCCL).  The combine step of the split-K decode,
+ * across devices: with M* = max_p M_p and w_p = 2^(M_p - M*) L_p,
+ *   out[row] = sum_p w_p outs[p][row] / sum_p w_p
+ * (0 where every L_p is 0).  Each slice's output already holds its own
+ * B_v^a term, which is linear, so the merge needs nothing else.  The pages
+ * show no multi-device step: this is the decode's split-K combine (the
+ * online-softmax merge of partial results) taken across devices.
+ *   outs   device, [n_parts][rows][d] of out_dtype (fp32 or bf16)
+ *   stats  device fp32, [n_parts][rows][2]: (M, L) as row_stats writes them
+ *   out    device, [rows][d] of out_dtype; may not overlap outs
+ * rows = n_seqs * n_agents * n_q_heads.  Asynchronous on `stream`.
+ * Errors: LA_ERR_INVALID_ARG (null or unaligned pointers, n_parts < 1,
+ * rows < 0, d not a positive multiple of 4, bad dtype), LA_ERR_CUDA.
+ */
+la_status lora_attn_decode_combine(const void* outs, const float* stats, int32_t n_parts,
+                                   int64_t rows, int32_t d, la_dtype out_dtype, void* out,
+                                   la_stream_t stream);
 
 /*
  * lora_attn_decode_static_scratch -- lora_attn_decode for callers that cannot

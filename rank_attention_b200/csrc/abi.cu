@@ -70,6 +70,8 @@ la_status check_attn(const la_attn_args* a, int decode, AttnParams* p) {
        a->lr_agent_stride < (int64_t)(a->n_seqs > 0 ? a->n_seqs - 1 : 0) * a->lr_seq_stride + a->L_max * 2 * a->r))
     return LA_ERR_INVALID_ARG;
   if (a->value_path < LA_VALUE_REORDERED || a->value_path > LA_VALUE_PER_TILE_GENERIC) return LA_ERR_INVALID_ARG;
+  if (a->key_pos0 < 0 || (reinterpret_cast<uintptr_t>(a->row_stats) & 7u) != 0) return LA_ERR_INVALID_ARG;
+  if (!decode && (a->key_pos0 != 0 || a->row_stats)) return LA_ERR_UNSUPPORTED;   // decode only
   const int g = a->n_q_heads / a->n_kv_heads;
   if ((int64_t)a->n_agents * g > kMaxRowsSimt) return LA_ERR_UNSUPPORTED;
   if (decode) {
@@ -112,6 +114,8 @@ la_status check_attn(const la_attn_args* a, int decode, AttnParams* p) {
   p->q_pos0 = a->q_pos0;
   p->n_q_tokens = decode ? 1 : a->n_q_tokens;
   p->decode = decode;
+  p->key_pos0 = a->key_pos0;
+  p->row_stats = a->row_stats;
   return LA_OK;
 }
 
@@ -330,6 +334,9 @@ la_status decode_prepare(const la_attn_args* a, void* workspace, size_t workspac
     return LA_OK;
   }
   DecodePlan d = plan_decode(*p, a->io_dtype);
+  // the sequence-sharded decode's inputs: the tensor-core decode only
+  if ((p->key_pos0 != 0 || p->row_stats) && !(d.kind == 1 && bf16_decode_uses_tc(*p)))
+    return LA_ERR_UNSUPPORTED;
   const size_t need = d.partial_bytes + d.counter_bytes;   // 0: no workspace, NULL allowed
   if (need > 0 && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
                    workspace_bytes < need))
@@ -474,6 +481,7 @@ extern "C" la_status lora_materialize_agent_kv(const la_attn_args* a, void* k_ou
   AttnParams p;
   la_status s = check_attn(a, 1, &p);
   if (s != LA_OK) return s;
+  if (a->key_pos0 != 0 || a->row_stats) return LA_ERR_UNSUPPORTED;   // the whole cache, unsharded
   if (!k_out || !v_out || !aligned16(k_out) || !aligned16(v_out)) return LA_ERR_INVALID_ARG;
   if (p.n_seqs == 0) return LA_OK;
   if (p.n_seqs > 65535 || (p.max_kv_len + 3) / 4 > 0x7fffffff) return LA_ERR_UNSUPPORTED;

@@ -904,11 +904,12 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
   if (w >= TC_NES && w < TC_NES + NPV) {
     // the first tile's query rotation R(-k_lo), scaled by s (exact in fp64)
     for (int i = tid - 32 * TC_NES; i < D / 2; i += 32 * NPV) {
-      const float2 cs = rope_cs_exact(k_lo, rt.theta[i]);
+      const float2 cs = rope_cs_exact(k_lo + p.key_pos0, rt.theta[i]);
       cs0[i] = make_float2(cs.x * p.s, cs.y * p.s);
     }
   }
-  if (kvl < 1 || kvl > p.max_kv_len) {
+  // a sharded decode's slice may hold none of a sequence's keys (kv_len 0)
+  if (kvl < (p.row_stats ? 0 : 1) || kvl > p.max_kv_len) {
     if (tid == 0 && split == 0) atomicOr(p.err, 1);
     if (w == TC_NES + NPV && lane == 0) {  // the copies in flight land before the CTA leaves
       mbar_wait(qbar, 0);
@@ -1203,7 +1204,7 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
       if (n + 1 < n_tiles) {
         if (qi < D / 2) {
           if (((n + 1) & 15) == 0) {
-            const float2 cs = rope_cs_exact(k0 + KT, theta[qi]);
+            const float2 cs = rope_cs_exact(p.key_pos0 + k0 + KT, theta[qi]);
             qcs = make_float2(cs.x * p.s, cs.y * p.s);
           } else {
             qcs = make_float2(fmaf(qcs.x, qstep.x, -qcs.y * qstep.y), fmaf(qcs.y, qstep.x, qcs.x * qstep.y));
@@ -1415,6 +1416,11 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
   if (s_fail && tid == 0) atomicOr(p.err, 2);
   if (ns == 1) {
     if (s_fail) return;
+    if (p.row_stats)   // (M, L) of every row, for the combine of a sequence-sharded decode
+      for (int row = tid; row < n_rows; row += TC_NTHR) {
+        const int64_t ri = ((int64_t)seq * na_tot + agent0 + row / g) * p.n_q + kvh * g + row % g;
+        reinterpret_cast<float2*>(p.row_stats)[ri] = make_float2(Mo[row * W + D + R], Mo[row * W + D + R + 1]);
+      }
     for (int i = tid; i < n_rows * D; i += TC_NTHR) {
       const int row = i / D, c = i % D;
       const int a = row / g, gi = row % g;
@@ -1501,6 +1507,10 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) lt += __shfl_xor_sync(0xffffffffu, lt, o);
     const float wk = lt > 0.f ? e / lt : 0.f;
+    if (p.row_stats && lane == 0) {   // (M, L) of the row over all its splits
+      const int64_t ri = ((int64_t)seq * na_tot + agent0 + row / g) * p.n_q + kvh * g + row % g;
+      reinterpret_cast<float2*>(p.row_stats)[ri] = make_float2(mx, lt);
+    }
     if (lane < ns) {
       Wf[r * kMaxSplits + lane] = wk;
       float4* tr = reinterpret_cast<float4*>(T + ((size_t)r * ns + lane) * R);
@@ -1799,6 +1809,8 @@ cudaError_t launch_tc(const AttnParams& p, cudaStream_t st) {
 }
 
 }  // namespace
+
+bool bf16_decode_uses_tc(const AttnParams& p) { return tc_supported(p); }
 
 bool bf16_decode_supported(const AttnParams& p) {
   if (tc_supported(p)) return true;

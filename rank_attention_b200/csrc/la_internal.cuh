@@ -45,6 +45,8 @@ struct AttnParams {
   int agent_group;         // tensor-core decode: agents per CTA (grid z runs over the groups)
   int value_path;          // la_value_path: 0 fastest reordered, 1 generic reordered, 2 per tile
   int blk0;                // tensor-core prefill, split launch: the first block of rows it covers
+  int64_t key_pos0;        // decode: position of key row 0 (sequence-sharded decode)
+  float* row_stats;        // decode: (M, L) per output row, or null
 };
 
 // Device error word of the library (address on the current device).
@@ -58,6 +60,8 @@ cudaError_t launch_append_bf16_mma(const void* X, int64_t ldx, int64_t n, int64_
                                    const void* A, int r, void* lr, int64_t pos0, int n_seqs,
                                    int64_t sx, int64_t slr, cudaStream_t st);
 cudaError_t launch_attn_simt(const AttnParams& p, la_dtype io, la_dtype out, cudaStream_t st);
+// the bf16 decode of these parameters runs on the tensor-core kernel
+bool bf16_decode_uses_tc(const AttnParams& p);
 cudaError_t launch_append_row_at_len(const void* x, const void* A, int64_t a_stride, void* lr,
                                      int64_t lr_seq, int64_t lr_agent, int n_lr,
                                      const int32_t* kv_len, int64_t max_kv_len, int n_seqs,

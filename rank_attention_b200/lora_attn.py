@@ -29,7 +29,8 @@ EXPORTED = ("la_status_string", "lr_cache_append", "lora_attn_prefill", "lora_at
             "lora_attn_decode_workspace_bytes", "la_device_check",
             "lora_attn_decode_static_scratch", "lora_materialize_agent_kv",
             "lr_cache_append_agents", "lora_query_expand", "lora_output_delta",
-            "la_device_check_word", "lora_decode_step_host", "lora_attn_decode_step")
+            "la_device_check_word", "lora_decode_step_host", "lora_attn_decode_step",
+            "lora_attn_decode_combine")
 
 
 class LoraAttnError(RuntimeError):
@@ -61,6 +62,8 @@ class AttnArgs(ctypes.Structure):
         ("io_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int),
         ("lr_agent_stride", ctypes.c_int64),
         ("value_path", ctypes.c_int32),
+        ("key_pos0", ctypes.c_int64),
+        ("row_stats", ctypes.c_void_p),
     ]
 
 
@@ -116,6 +119,10 @@ def _load() -> ctypes.CDLL:
     lib.lora_materialize_agent_kv.restype = ctypes.c_int
     lib.lora_materialize_agent_kv.argtypes = [ctypes.POINTER(AttnArgs), ctypes.c_void_p,
                                               ctypes.c_void_p, ctypes.c_void_p]
+    lib.lora_attn_decode_combine.restype = ctypes.c_int
+    lib.lora_attn_decode_combine.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
+                                             ctypes.c_int64, ctypes.c_int32, ctypes.c_int,
+                                             ctypes.c_void_p, ctypes.c_void_p]
     return lib
 
 
@@ -214,13 +221,17 @@ def lora_output_delta(o: torch.Tensor, A_o: torch.Tensor, B_o: torch.Tensor, y: 
 
 def make_args(k_base, v_base, lr, B_k, B_v, q, out, *, lora_scale: float, rope_base: float,
               softmax_scale: Optional[float] = None, kv_len: Optional[torch.Tensor] = None,
-              max_kv_len: int = 0, q_pos0: int = 0, value_path: int = LA_VALUE_REORDERED) -> AttnArgs:
+              max_kv_len: int = 0, q_pos0: int = 0, value_path: int = LA_VALUE_REORDERED,
+              key_pos0: int = 0, row_stats: Optional[torch.Tensor] = None) -> AttnArgs:
     """Fill la_attn_args from tensors.
 
     k_base, v_base [n_seqs, n_kv, L_max, d] (any strides with a unit last
     stride); lr [n_seqs, L_max, 2r], one LR cache shared by every agent, or
     [n_agents, n_seqs, L_max, 2r], one per agent; B_k, B_v [n_agents, r, n_kv*d];
-    q, out [n_seqs, n_agents, n_tok, n_q, d] contiguous; kv_len int32 [n_seqs]."""
+    q, out [n_seqs, n_agents, n_tok, n_q, d] contiguous; kv_len int32 [n_seqs].
+    Sequence-sharded decode: key_pos0 is the position of the caches' key row 0;
+    row_stats a float32 [n_seqs, n_agents, n_q, 2] tensor the decode fills
+    with each row's (M, L) for lora_attn_decode_combine."""
     n_seqs, n_kv, L_max, d = k_base.shape
     n_agents, n_tok, n_q = q.shape[1], q.shape[2], q.shape[3]
     per_agent = lr.dim() == 4
@@ -252,6 +263,11 @@ def make_args(k_base, v_base, lr, B_k, B_v, q, out, *, lora_scale: float, rope_b
     a.io_dtype, a.out_dtype = _dt(k_base), _dt(out)
     a.lr_agent_stride = lr_agent_stride
     a.value_path = value_path
+    a.key_pos0 = key_pos0
+    if row_stats is not None:
+        assert row_stats.dtype == torch.float32 and row_stats.is_contiguous()
+        assert row_stats.numel() == 2 * n_seqs * n_agents * n_q
+    a.row_stats = row_stats.data_ptr() if row_stats is not None else None
     return a
 
 
@@ -271,6 +287,21 @@ def lora_attn_decode(args: AttnArgs, workspace: torch.Tensor, stream=None) -> No
     st = lib.lora_attn_decode(ctypes.byref(args), workspace.data_ptr(), workspace.numel(),
                               _stream(stream))
     _check(st, "lora_attn_decode")
+
+
+def lora_attn_decode_combine(outs: torch.Tensor, stats: torch.Tensor, out: torch.Tensor,
+                             stream=None) -> None:
+    """Merge the decodes of n_parts key slices of the same queries: outs
+    [n_parts, *rows, d] (fp32 or bf16), stats float32 [n_parts, *rows, 2] as
+    row_stats holds them, out [*rows, d] of outs' dtype; all contiguous."""
+    assert outs.is_contiguous() and stats.is_contiguous() and out.is_contiguous()
+    assert stats.dtype == torch.float32 and out.dtype == outs.dtype
+    n_parts, d = outs.shape[0], outs.shape[-1]
+    rows = out.numel() // d
+    assert outs.numel() == n_parts * rows * d and stats.numel() == 2 * n_parts * rows
+    st = lib.lora_attn_decode_combine(outs.data_ptr(), stats.data_ptr(), n_parts, rows, d, _dt(out),
+                                      out.data_ptr(), _stream(stream))
+    _check(st, "lora_attn_decode_combine")
 
 
 def lora_attn_decode_step(args: AttnArgs, A_kv: torch.Tensor, x_new: torch.Tensor,

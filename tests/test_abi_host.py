@@ -290,3 +290,41 @@ def test_packed_step_inputs_back_to_back():
     assert kv.data_ptr() == q.data_ptr() + q.numel() * 2
     assert kv.dtype == torch.int32 and kv.numel() == 2
     assert buf.numel() == (x.numel() + q.numel()) * 2 + 8
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(key_pos0=-1), la.LA_ERR_INVALID_ARG),
+    (dict(row_stats=FAKE + 4), la.LA_ERR_INVALID_ARG),
+    # the generic fp32 decode does not take the sharded decode's inputs
+    (dict(key_pos0=128), la.LA_ERR_UNSUPPORTED),
+    (dict(row_stats=FAKE), la.LA_ERR_UNSUPPORTED),
+])
+def test_sharded_decode_inputs_checked(kw, status):
+    a = _args(**kw)
+    assert la.lib.lora_attn_decode(ctypes.byref(a), FAKE, 1 << 20, None) == status
+
+
+@pytest.mark.parametrize("kw", [dict(key_pos0=128), dict(row_stats=FAKE)])
+def test_sharded_inputs_refused_outside_the_decode(kw):
+    a = _args(**kw)
+    assert la.lib.lora_attn_prefill(ctypes.byref(a), None) == la.LA_ERR_UNSUPPORTED
+    assert la.lib.lora_materialize_agent_kv(ctypes.byref(a), FAKE, FAKE, None) == la.LA_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(outs=0), la.LA_ERR_INVALID_ARG),
+    (dict(stats=0), la.LA_ERR_INVALID_ARG),
+    (dict(out=0), la.LA_ERR_INVALID_ARG),
+    (dict(n_parts=0), la.LA_ERR_INVALID_ARG),
+    (dict(rows=-1), la.LA_ERR_INVALID_ARG),
+    (dict(d=6), la.LA_ERR_INVALID_ARG),
+    (dict(dt=3), la.LA_ERR_INVALID_ARG),
+    (dict(outs=FAKE + 8), la.LA_ERR_INVALID_ARG),         # fp32 rows read four at a time
+    (dict(stats=FAKE + 4), la.LA_ERR_INVALID_ARG),
+    (dict(rows=0), la.LA_OK),                             # nothing to merge, nothing launched
+])
+def test_combine_checks(kw, status):
+    a = dict(outs=FAKE, stats=FAKE, n_parts=2, rows=8, d=128, dt=la.LA_F32, out=FAKE)
+    a.update(kw)
+    assert la.lib.lora_attn_decode_combine(a["outs"], a["stats"], a["n_parts"], a["rows"], a["d"],
+                                           a["dt"], a["out"], None) == status
