@@ -18,7 +18,7 @@
 // The running max is rescaled lazily: O and l are corrected only when a row's
 // maximum grows by more than 2^8, so P <= 256 and the correction is rare.
 //
-// Warps: 8 compute warps build K^a (16 keys each, the mma fragment layout of
+// Warps: 8 compute warps build K^a in f16x2 arithmetic (16 keys each, the mma fragment layout of
 // the delta) and run the softmax (two warps per TMEM sub-partition, 64 keys
 // each); warp 8 issues the MMAs (and the first loads), warp 9 the TMA
 // refills.  The compute warps build tile n+1
@@ -51,6 +51,13 @@ __device__ __forceinline__ uint32_t add_to_f16x2(uint32_t base_bf16x2, float2 d)
   const float2 b = unpack_bf16(base_bf16x2);
   __half2 h = __floats2half2_rn(b.x + d.x, b.y + d.y);
   return *reinterpret_cast<uint32_t*>(&h);
+}
+// f16 pairs as 32-bit words and back, and a bf16 pair as an f16 pair (exact
+// within f16's range)
+__device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
+__device__ __forceinline__ __half2 bits_h2(uint32_t v) { return *reinterpret_cast<__half2*>(&v); }
+__device__ __forceinline__ __half2 bf16x2_h2(uint32_t v) {
+  return __floats2half2_rn(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
 }
 // a bf16 pair as a packed fp32 pair (exact), and a packed fp32 pair rounded
 // once to an fp16 pair
@@ -251,9 +258,9 @@ __global__ void __launch_bounds__(PNTHR, 1)
   // frequencies, and the first two tiles' anchors s R(k0)
   const int sp = w & 3, ch = w >> 2;
   const int kb = 32 * sp + 16 * ch;   // build: this warp's 16 keys (its TMEM lanes)
-  // (cos, cos) and (sin, sin) over two adjacent frequencies: the operands of
-  // the packed f32x2 rotation
-  uint64_t RC[4][2][2], RS[4][2][2];
+  // (cos, cos) and (sin, sin) f16 pairs over two adjacent frequencies: the
+  // operands of the packed f16x2 rotation
+  uint32_t RC[4][2][2], RS[4][2][2];
   if (w < PNC) {
 #pragma unroll
     for (int grp = 0; grp < 4; ++grp)
@@ -265,8 +272,8 @@ __global__ void __launch_bounds__(PNTHR, 1)
         for (int hh = 0; hh < 2; ++hh) {
           const float j = (float)(kb + gq + 8 * hh);
           const float2 a = sincos_small(j * th0), b = sincos_small(j * th1);
-          RC[grp][hh][q] = f2(a.x, b.x);
-          RS[grp][hh][q] = f2(a.y, b.y);
+          RC[grp][hh][q] = h2_bits(__floats2half2_rn(a.x, b.x));
+          RS[grp][hh][q] = h2_bits(__floats2half2_rn(a.y, b.y));
         }
       }
   }
@@ -422,21 +429,23 @@ __global__ void __launch_bounds__(PNTHR, 1)
         for (int q = 0; q < 2; ++q) {
           const int i0 = 16 * grp + 8 * q + 2 * t4;
           const float2 a0 = an[i0], a1 = an[i0 + 1];
-          const uint64_t ac = f2(a0.x, a1.x), as = f2(a0.y, a1.y), nas = f2(-a0.y, -a1.y);
+          const __half2 ac = __floats2half2_rn(a0.x, a1.x), as = __floats2half2_rn(a0.y, a1.y);
+          const __half2 nas = __hneg2(as);
           const uint32_t cx = (uint32_t)(((2 * grp + q) ^ gq) << 4);
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
-            const uint64_t x1 = f2(__uint_as_float(xl[4 * q + 2 * hh]), __uint_as_float(xl[4 * q + 2 * hh + 1]));
-            const uint64_t x2 = f2(__uint_as_float(xh[4 * q + 2 * hh]), __uint_as_float(xh[4 * q + 2 * hh + 1]));
-            const uint64_t c = RC[grp][hh][q], sn = RS[grp][hh][q];
-            const uint64_t y1 = sub_f2(mul_f2(x1, c), mul_f2(x2, sn));   // R(j) dK
-            const uint64_t y2 = fma_f2(x2, c, mul_f2(x1, sn));
-            // K_base + s R(k0) y, the base added inside the rotation's FMAs
+            // in f16x2 arithmetic: the delta pairs, R(j) dK, then K_base + s R(k0) y
+            // with the base added inside the rotation's FMAs
+            const __half2 x1 = __floats2half2_rn(__uint_as_float(xl[4 * q + 2 * hh]), __uint_as_float(xl[4 * q + 2 * hh + 1]));
+            const __half2 x2 = __floats2half2_rn(__uint_as_float(xh[4 * q + 2 * hh]), __uint_as_float(xh[4 * q + 2 * hh + 1]));
+            const __half2 c = bits_h2(RC[grp][hh][q]), sn = bits_h2(RS[grp][hh][q]);
+            const __half2 y1 = __hfma2(x1, c, __hneg2(__hmul2(x2, sn)));   // R(j) dK
+            const __half2 y2 = __hfma2(x2, c, __hmul2(x1, sn));
             const uint32_t o1 = rowb + hh * 1024 + cx, o2 = o1 + PKT * 128;
-            const uint64_t z1 = fma_f2(ac, y1, fma_f2(nas, y2, bf16x2_f2(lds32(o1))));
-            const uint64_t z2 = fma_f2(ac, y2, fma_f2(as, y1, bf16x2_f2(lds32(o2))));
-            sts32(o1, f2_f16x2(z1));
-            sts32(o2, f2_f16x2(z2));
+            const __half2 z1 = __hfma2(ac, y1, __hfma2(nas, y2, bf16x2_h2(lds32(o1))));
+            const __half2 z2 = __hfma2(ac, y2, __hfma2(as, y1, bf16x2_h2(lds32(o2))));
+            sts32(o1, h2_bits(z1));
+            sts32(o2, h2_bits(z2));
           }
         }
       }
