@@ -238,7 +238,11 @@ la_status lora_attn_decode_step(const la_attn_args* args, const void* A_kv, cons
  *      new token's LR row of every sequence q at position kv_len_host[q] - 1
  *      (with args->lr_agent_stride > 0, one row per agent into that agent's
  *      own cache, X A_a), then the decode;
- *   3. copies args->out -> out_host.
+ *   3. copies args->out -> out_host; or, when out_host is pinned host memory
+ *      mapped into the device's address space (as memory from cudaHostAlloc
+ *      is under unified addressing; cudaPointerGetAttributes reports a device
+ *      alias), no copy: the decode writes its outputs straight into out_host
+ *      and args->out is left as it was.
  * out_host holds the step's outputs once the stream has been synchronised.
  * Pinned (page-locked) host buffers make the copies asynchronous; pageable
  * ones are still correct, with the copies staged by the CUDA runtime.  When
@@ -249,7 +253,8 @@ la_status lora_attn_decode_step(const la_attn_args* args, const void* A_kv, cons
  *
  *   args        as lora_attn_decode; args->q, args->kv_len and args->lr_cache
  *               are device buffers this call writes (the copies and the
- *               append), args->out the device buffer it copies back.
+ *               append), args->out the device buffer it copies back (not
+ *               used when out_host is mapped pinned memory, step 3).
  *   A_kv        device, [hidden][2r] (shared A) or [n_agents][hidden][2r]
  *               (args->lr_agent_stride > 0), io dtype.
  *   x_dev       device staging of n_seqs * hidden elements (io dtype), 16-byte
