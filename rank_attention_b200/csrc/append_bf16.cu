@@ -31,7 +31,17 @@ constexpr int KC = 64;     // hidden columns per stage
 constexpr int NTHR = 256;     // 4 row groups x 2 column groups
 constexpr int NSTAGE = 3;
 constexpr int kMaxHS = 16;
-constexpr int kSMs = 148;
+// SMs of the current device, for splitting the hidden dimension over about
+// one wave of CTAs (148 on B200, also the answer when the query fails)
+int current_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) {
+    cudaGetLastError();
+    return 148;
+  }
+  return n;
+}
 
 
 template <int R>
@@ -341,7 +351,7 @@ cudaError_t launch_r(const void* X, int64_t ldx, int64_t n, int64_t H, const voi
       return cudaErrorInvalidValue;
     using Tf = TCfgA<R>;
     const int64_t mt2 = (n + TM2 - 1) / TM2;
-    int hs2 = (int)(kSMs / (mt2 * n_seqs));
+    int hs2 = (int)(current_sms() / (mt2 * n_seqs));
     if (hs2 > kMaxHS) hs2 = kMaxHS;
     if (hs2 > kchunks) hs2 = kchunks;
     if (hs2 < 1) hs2 = 1;
@@ -370,7 +380,7 @@ cudaError_t launch_r(const void* X, int64_t ldx, int64_t n, int64_t H, const voi
     return cudaGetLastError();
   }
   const int64_t mtiles = (n + TM - 1) / TM;
-  int hs = (int)(kSMs / (mtiles * n_seqs));
+  int hs = (int)(current_sms() / (mtiles * n_seqs));
   if (hs > kMaxHS) hs = kMaxHS;
   if (hs > kchunks) hs = kchunks;
   if (hs < 1) hs = 1;

@@ -15,7 +15,7 @@ import pytest
 import torch
 
 from rank_attention_b200 import workloads as W
-from tests.helpers import assert_parity, to_np
+from tests.helpers import assert_parity, oracle_decode, to_np
 
 DEV = "cuda"
 FAKE = 0x10000  # 16-byte aligned, never dereferenced
@@ -49,6 +49,7 @@ def _compare(la, s, inp):
         torch.cuda.synchronize()
         assert la.la_device_check() == la.LA_OK
         assert_parity(to_np(out), to_np(ref), s.dtype)
+    assert_parity(to_np(out), oracle_decode(inp, s), s.dtype)   # and the oracle itself
 
 
 @pytest.mark.gpu
