@@ -755,6 +755,58 @@ def oracle_step(inp, new, s):
                                  mode="decode")
 
 
+def time_oracle_samples(budget_s: float = 10.0) -> dict:
+    """The oracle on bounded samples of the prefill and the 32k sweep: one
+    (agent, KV head) unit each, scaled by the units of a whole launch."""
+    import numpy as np
+    from oracle import impl as oracle
+    from rank_attention_b200 import workloads as W
+    res = {}
+    # prefill, 16384 + 1024: the last 64 chunk tokens of one unit (its K^a and V^a
+    # over all 17408 keys materialised, then their attention)
+    s = W.LLAMA8B_PREFILL_16K
+    inp = W.direct_cache_inputs(s)
+    g = s.n_q_heads // s.n_kv_heads
+    toks = list(range(s.n_q_tokens - 64, s.n_q_tokens))
+    qpos = s.q_pos0 + np.arange(s.n_q_tokens)
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        oracle.lora_attention_unit(inp["k_base"], inp["v_base"], inp["lr"], inp["B_k"], inp["B_v"],
+                                   inp["q"], seq=0, agent=0, kv_head=0, kv_len=s.kv_len,
+                                   q_positions=qpos, lora_scale=s.lora_scale,
+                                   softmax_scale=s.softmax_scale, rope_base=s.rope_base,
+                                   q_tokens=toks)
+        n += 1
+        if time.perf_counter() - t0 > budget_s / 2:
+            break
+    per = (time.perf_counter() - t0) / n
+    pairs = g * sum(int(qpos[j]) + 1 for j in toks)
+    res["prefill"] = {"workload": s.name, "TFLOP/s": 4 * s.head_dim * pairs / per / 1e12,
+                      "sample": f"one (agent, KV head) unit, the last {len(toks)} chunk tokens x "
+                                f"{g} heads over all {s.kv_len} keys, {n} runs"}
+    # decode sweep at 32k: one (sequence, agent, KV head) unit of the 16 x 5 x 8
+    s = W.llama8b_sweep(32768).replace(n_seqs=1)
+    inp = W.direct_cache_inputs(s)
+    t0 = time.perf_counter()
+    n = 0
+    while True:
+        oracle.lora_attention_unit(inp["k_base"], inp["v_base"], inp["lr"], inp["B_k"], inp["B_v"],
+                                   inp["q"], seq=0, agent=0, kv_head=0, kv_len=s.kv_len,
+                                   q_positions=[s.kv_len - 1], lora_scale=s.lora_scale,
+                                   softmax_scale=s.softmax_scale, rope_base=s.rope_base)
+        n += 1
+        if time.perf_counter() - t0 > budget_s / 2:
+            break
+    per = (time.perf_counter() - t0) / n
+    units = 16 * s.n_agents * s.n_kv_heads
+    res["sweep_32k"] = {"workload": W.llama8b_sweep(32768).name,
+                        "agent_tokens_per_s": 16 * s.n_agents / (per * units),
+                        "sample": f"one (sequence, agent, KV head) unit of {units}, {n} runs, "
+                                  "scaled by the units of a step"}
+    return res
+
+
 def blas_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
@@ -1008,7 +1060,8 @@ def run_ours(args):
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": blas_threads(),
                                 "kind": "oracle",
                                 "sample": f"{n} full decode steps of {s.name} on the host",
-                                "tiny_fp32": time_oracle_tiny()}
+                                "tiny_fp32": time_oracle_tiny(),
+                                "other_configs": time_oracle_samples()}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
