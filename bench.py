@@ -575,7 +575,7 @@ class ClockSampler:
 # DRAM bytes per decode launch from an ncu capture of the workload, keyed by the
 # sha256 prefix of the decode kernel's source: reported only while the kernel is
 # unchanged since the counters were taken.
-DECODE_TRAFFIC = {"1b967558da805ce6": 34417408}
+DECODE_TRAFFIC = {"e792fb7ef9ab6297": 34422272}
 
 
 def decode_source_sha() -> str:

@@ -380,6 +380,7 @@ la_status step_launch(AttnParams& p, int kind, const la_attn_args* a, const void
                                                  a->lr_agent_stride, n_lr, a->kv_len, a->max_kv_len,
                                                  a->n_seqs, hidden, a->r, a->io_dtype, p.err, st);
   if (e != cudaSuccess) return LA_ERR_CUDA;
+  p.early = 1;   // the append writes LR rows only: the decode may read its other inputs at once
   return decode_launch(p, kind, a, st);
 }
 }  // namespace

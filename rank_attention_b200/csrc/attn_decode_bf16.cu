@@ -818,7 +818,9 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
   const uint32_t pvdone = tfull + 48;             // the P V_base MMA of a tile has completed
   const int64_t ldB = (int64_t)p.n_kv * D;
 
-  auto issue = [&](int n) {  // TMA of tile n into stage n % ST (one thread)
+  // TMA of tile n into stage n % ST (one thread): the base tiles (and the
+  // stage's whole byte count), then the LR rows
+  auto issue_kv = [&](int n) {
     const int s = n % ST;
     const uint32_t sb = area_u + s * C::STAGE;
     const uint32_t bar = full_u + 8 * s;
@@ -830,12 +832,23 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
       tma_load_4d(sb + b * KT * 128, &tmK, bar, 64 * b, key0, kvh, seq);
       tma_load_4d(sb + C::KV_TILE + b * KT * 128, &tmV, bar, 64 * b, key0, kvh, seq);
     }
+  };
+  auto issue_lr = [&](int n) {
+    const int s = n % ST;
+    const uint32_t sb = area_u + s * C::STAGE;
+    const uint32_t bar = full_u + 8 * s;
+    const int key0 = (int)(k_lo + (int64_t)n * KT);
+    const int nlr = PA ? na : 1;
     constexpr int LB = (2 * R) < 64 ? 2 * R : 64;
     for (int al = 0; al < nlr; ++al)
 #pragma unroll
       for (int b = 0; b < (2 * R) / LB; ++b)
         tma_load_4d(sb + 2 * C::KV_TILE + al * C::LR_TILE + b * KT * LB * 2, &tmL, bar, LB * b, key0, seq,
                     PA ? agent0 + al : lra);
+  };
+  auto issue = [&](int n) {
+    issue_kv(n);
+    issue_lr(n);
   };
 
   // ---- first loads (independent of kv_len): queries, B_k^a, the first tiles, B_v^a
@@ -857,10 +870,13 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
     tma_prefetch(&tmK);
     tma_prefetch(&tmV);
     tma_prefetch(&tmL);
-    // launched as a programmatic dependent of the preceding kernel (the LR
-    // append of the step): everything above overlaps its tail; every read of
-    // an input comes after the wait (a no-op without a preceding kernel)
-    pdl_wait();
+    // launched as a programmatic dependent of the preceding kernel: everything
+    // above overlaps its tail, and every read of an input comes after the wait
+    // (a no-op without a preceding kernel) -- except in a decode step, whose
+    // preceding kernel (the row append) writes only LR rows: there the
+    // queries, B_k and the first base tiles are requested at once, and only
+    // the LR rows wait
+    if (!p.early) pdl_wait();
     // each agent's g query rows of this KV head are contiguous
     const __nv_bfloat16* Q = reinterpret_cast<const __nv_bfloat16*>(p.q);
     mbar_expect_tx(qbar, (uint32_t)(n_rows * D * 2));
@@ -875,9 +891,17 @@ __global__ void __launch_bounds__(TC_NTHR, 1)
         tma_load_3d(bks_u + a * align1k(C::BK_BYTES) + b * R * 128, &tmB, bkbar, kvh * D + 64 * b, 0, agent0 + a);
     // the first stages before kv_len is known: tiles of this split's range
     // (by max_kv_len) past the sequence's length are loaded but never used
-    for (int n = 0; n < n_spec; ++n) issue(n);
+    if (p.early) {
+      for (int n = 0; n < n_spec; ++n) issue_kv(n);
+      pdl_wait();   // the append's LR rows are complete and visible
+      for (int n = 0; n < n_spec; ++n) issue_lr(n);
+    } else {
+      for (int n = 0; n < n_spec; ++n) issue(n);
+    }
   }
-  pdl_wait();
+  // kv_len is written before the step's append, so a step reads it at once;
+  // the LR rows (the append's output) are read only by the TMA thread's loads
+  if (!p.early) pdl_wait();
   const int64_t kvl = p.kv_len[seq];  // in flight while the constants are computed
   const int sp = w & 3, kb = 32 * sp + 16 * (w >> 2);  // score warp: TMEM sub-partition, first key
   // R(j) for this thread's keys j = kb + gq + 8 hh and its frequencies

@@ -45,6 +45,7 @@ struct AttnParams {
   int agent_group;         // tensor-core decode: agents per CTA (grid z runs over the groups)
   int value_path;          // la_value_path: 0 fastest reordered, 1 generic reordered, 2 per tile
   int blk0;                // tensor-core prefill, split launch: the first block of rows it covers
+  int early;               // decode step: the kernel before it writes only LR rows
   int64_t key_pos0;        // decode: position of key row 0 (sequence-sharded decode)
   float* row_stats;        // decode: (M, L) per output row, or null
 };
