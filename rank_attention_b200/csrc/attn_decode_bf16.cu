@@ -36,7 +36,9 @@
 //  row: out = (sum_k w_k O_base,k + s (sum_k w_k O_lr,k) B_v^a) with
 //  w_k = 2^(m_k - M) / sum_k 2^(m_k - M) l_k.  The launch is a programmatic
 //  dependent of the kernel before it (the step's LR append): the set-up runs
-//  while that kernel finishes, every input is read after griddepcontrol.wait.
+//  while that kernel finishes, every input is read after griddepcontrol.wait
+//  -- in a decode step every input but the LR rows (the append's output) is
+//  read at once, and only the LR loads wait.
 //
 // decode_bf16_kernel + decode_merge_kernel (shapes the first kernel does not
 // take: d = 64, r = 8).  The same tiling with mma.sync for every product and a
